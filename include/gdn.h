@@ -1,0 +1,153 @@
+/*
+ * gdn.h -- C ABI of the B200 (sm_100a) Gated DeltaNet forward library.
+ *
+ * The operation.  The LinMorph project page (Abstract; "Why learn the
+ * initialization?") converts softmax self-attention blocks of a video DiT into
+ * Gated DeltaNet (GDN) modules built from update gates, decay terms, short
+ * convolutions and normalization parameters.  The recurrence is the gated
+ * delta rule of "Gated Delta Networks: Improving Mamba2 with Delta Rule"
+ * (reference [57] on the VMonarch page, References).  gdn_forward computes,
+ * for every batch item b and head h over the frame-major flattened video
+ * token sequence t = 0..T-1 (token = f*H_lat*W_lat + y*W_lat + x):
+ *
+ *   q' = SiLU(conv4(q)), k' = SiLU(conv4(k)), v^ = SiLU(conv4(v))
+ *        conv4: causal depthwise kernel-4 convolution over t, tap 3 on the
+ *        current token, zero history before t = 0 of each batch item, no bias
+ *   q^ = q'/sqrt(|q'|^2 + l2_eps),  k^ = k'/sqrt(|k'|^2 + l2_eps)
+ *   alpha_t = exp(-exp(A_log[h]) * softplus(g_t + dt_bias[h])),  beta_t = sigmoid(b_t)
+ *   S_t = alpha_t S_{t-1} (I - beta_t k^_t k^_t^T) + beta_t v^_t k^_t^T,  S_{-1} = 0
+ *   o_t = S_t q^_t / sqrt(d_k)
+ *   y_t = o_t / sqrt(mean(o_t^2) + norm_eps) * norm_w * SiLU(z_t)
+ *
+ * S is d_v x d_k per (b, h) and is carried in fp32.  The result y is the
+ * layer output before the output projection.
+ *
+ * Layouts (row-major, element strides):
+ *   q, k   [B][T][H][d_k]   token stride tok_stride (elements; 0 = H*d_k)
+ *   v, z   [B][T][H][d_v]   token stride tok_stride (0 = H*d_v)
+ *   g, b   [B][T][H] fp32
+ *   conv_q, conv_k [H*d_k][4] fp32; conv_v [H*d_v][4] fp32 (tap 3 = current token)
+ *   A_log, dt_bias [H] fp32;  norm_w [d_v] fp32 (shared by all heads)
+ *   y      [B][T][H][d_v], dense, type out_dtype
+ * q, k, v, z have type in_dtype.
+ *
+ * Ownership.  The caller owns every buffer: inputs, output, workspace and
+ * staging.  The library allocates no device memory; a plan holds host state
+ * only (plus nothing on the device).  All device pointers must be 16-byte
+ * aligned and tok_stride * element size must be a multiple of 16 bytes.
+ *
+ * Errors.  Every call returns a gdn_status; no C++ exception crosses the ABI.
+ * gdn_forward validates its arguments on the host and returns
+ * GDN_ERR_INVALID_ARG / GDN_ERR_UNSUPPORTED without launching anything.  The
+ * launches are asynchronous on the caller's stream: errors the kernels detect
+ * on the device (a bounded wait that ran out, a failed debug check) are
+ * written to a status word inside the workspace and read back by
+ * gdn_get_device_status, which synchronises the stream.
+ *
+ * Concurrency.  A plan is immutable after gdn_plan and may be shared by
+ * threads.  Forwards that may overlap on the GPU need distinct workspaces.
+ */
+#ifndef GDN_B200_H_
+#define GDN_B200_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *gdn_stream_t; /* same type as cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size or stride, T = 0 with B*H > 0 ... */
+    GDN_ERR_UNSUPPORTED = 2,  /* a configuration this build does not implement */
+    GDN_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed (launch, copy, tensor map) */
+    GDN_ERR_TIMEOUT = 4,      /* a device-side bounded wait ran out (status word) */
+    GDN_ERR_DEVICE_CHECK = 5, /* a device-side debug check failed (status word) */
+    GDN_ERR_NO_DEVICE = 6     /* no sm_100 device is current */
+} gdn_status;
+
+typedef enum {
+    GDN_DTYPE_BF16 = 0,
+    GDN_DTYPE_F32 = 1,
+    GDN_DTYPE_F16 = 2
+} gdn_dtype;
+
+/* Plan flags. */
+#define GDN_FLAG_DEBUG_CHECKS 0x1u       /* device-side index/alignment checks into the status word */
+#define GDN_FLAG_FORCE_SIMT 0x2u         /* use the fp32 CUDA-core path even where the tensor path applies */
+#define GDN_FLAG_TEST_WAIT_TIMEOUT 0x100u /* test hook: the scan kernel waits on a barrier nothing
+                                            arrives on, gives up after ~50 ms and reports
+                                            GDN_ERR_TIMEOUT in the status word */
+
+typedef struct {
+    int B, T, H, d_k, d_v;   /* d_k == d_v, 64 or 128; B, H >= 1; T >= 1 */
+    gdn_dtype in_dtype;      /* q, k, v, z */
+    gdn_dtype out_dtype;     /* y */
+    int conv_size;           /* must be 4 */
+    int chunk;               /* UT-transform chunk; must be 64 */
+    float l2_eps;            /* inside the sqrt of the q/k L2 norm (1e-6 typical) */
+    float norm_eps;          /* inside the sqrt of the output RMSNorm (1e-6 typical) */
+    long long tok_stride;    /* elements between consecutive tokens of q,k,v,z; 0 = H*d */
+    unsigned flags;          /* GDN_FLAG_* */
+} gdn_config;
+
+typedef struct {
+    const void *q, *k, *v, *z;                 /* [B][T][H][d] in_dtype, device */
+    const float *g, *b;                        /* [B][T][H] fp32, device */
+    const float *conv_q, *conv_k, *conv_v;     /* [H*d][4] fp32, device */
+    const float *A_log, *dt_bias;              /* [H] fp32, device */
+    const float *norm_w;                       /* [d_v] fp32, device */
+} gdn_inputs;
+
+typedef struct gdn_plan_s *gdn_plan_t;
+
+/* Validate cfg and build a plan for the current CUDA device.  On success
+ * *out receives the plan and *workspace_bytes the size of the device
+ * workspace gdn_forward needs (256-byte alignment required).  Host only: no
+ * allocation or launch on the device.  Errors: INVALID_ARG (null pointers or
+ * invalid sizes), UNSUPPORTED (d not in {64, 128}, d_k != d_v, conv_size != 4,
+ * chunk != 64, an output type not in {bf16, f16, f32}), NO_DEVICE. */
+gdn_status gdn_plan(const gdn_config *cfg, gdn_plan_t *out, size_t *workspace_bytes);
+
+/* Enqueue the forward on `stream`: y <- GDN(inputs).  Every pointer is a
+ * device pointer; workspace has at least *workspace_bytes from gdn_plan.
+ * Returns after enqueueing; host-side argument errors return before any
+ * launch. */
+gdn_status gdn_forward(gdn_plan_t plan, const gdn_inputs *in, void *y, void *workspace,
+                       gdn_stream_t stream);
+
+/* Bytes of device staging memory gdn_forward_host needs (inputs + output). */
+size_t gdn_staging_bytes(gdn_plan_t plan);
+
+/* End-to-end call with HOST buffers: copies every input from host memory
+ * (pinned memory recommended) into `staging` (device, gdn_staging_bytes),
+ * runs gdn_forward, and copies y back into the host buffer y_host, all
+ * enqueued on `stream` (one cudaMemcpyAsync per buffer).  The call returns
+ * after enqueueing; synchronise the stream before reading y_host. */
+gdn_status gdn_forward_host(gdn_plan_t plan, const gdn_inputs *in_host, void *y_host,
+                            void *staging, void *workspace, gdn_stream_t stream);
+
+/* Synchronise `stream`, then read and clear the device status word in the
+ * workspace.  Returns GDN_OK, GDN_ERR_TIMEOUT or GDN_ERR_DEVICE_CHECK (or
+ * GDN_ERR_CUDA if the synchronisation itself failed). */
+gdn_status gdn_get_device_status(gdn_plan_t plan, void *workspace, gdn_stream_t stream);
+
+/* Number of kernel launches one gdn_forward enqueues for this plan. */
+int gdn_launches_per_forward(gdn_plan_t plan);
+
+/* 1 if the plan runs the tensor-core (tcgen05) path, 0 for the fp32 CUDA-core path. */
+int gdn_plan_uses_tensor_path(gdn_plan_t plan);
+
+/* Free a plan (host memory only).  NULL is accepted. */
+gdn_status gdn_destroy(gdn_plan_t plan);
+
+/* Static description of a status code. */
+const char *gdn_status_string(gdn_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_B200_H_ */
