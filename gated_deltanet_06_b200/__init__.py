@@ -1,0 +1,187 @@
+"""Python binding of libgdn_b200.so, the sm_100a Gated DeltaNet forward.
+
+Argument marshalling only: every step of the forward runs in the library's
+CUDA kernels.  The binding fails loudly (ImportError) when the library has
+not been built; there is no fallback.  PyTorch is used for device memory and
+streams only.
+
+    import gated_deltanet_06_b200 as gdn
+    y = gdn.forward(q, k, v, z, g, b, conv_q, conv_k, conv_v, A_log, dt_bias, norm_w)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdn_b200.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "gdn.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python gated_deltanet_06_b200/build.py` "
+                      "(the GDN forward has no CPU fallback)")
+_lib = ctypes.CDLL(LIB_PATH)
+
+# gdn_status
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE_CHECK, ERR_NO_DEVICE = range(7)
+# gdn_dtype
+DTYPE_BF16, DTYPE_F32, DTYPE_F16 = 0, 1, 2
+FLAG_DEBUG_CHECKS = 0x1
+FLAG_FORCE_SIMT = 0x2
+FLAG_TEST_WAIT_TIMEOUT = 0x100
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("d_k", ctypes.c_int),
+                ("d_v", ctypes.c_int), ("in_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
+                ("conv_size", ctypes.c_int), ("chunk", ctypes.c_int), ("l2_eps", ctypes.c_float),
+                ("norm_eps", ctypes.c_float), ("tok_stride", ctypes.c_longlong), ("flags", ctypes.c_uint)]
+
+
+class Inputs(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("q", "k", "v", "z", "g", "b", "conv_q", "conv_k", "conv_v",
+                                                 "A_log", "dt_bias", "norm_w")]
+
+
+_vp = ctypes.c_void_p
+_lib.gdn_plan.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(_vp), ctypes.POINTER(ctypes.c_size_t)]
+_lib.gdn_plan.restype = ctypes.c_int
+_lib.gdn_forward.argtypes = [_vp, ctypes.POINTER(Inputs), _vp, _vp, _vp]
+_lib.gdn_forward.restype = ctypes.c_int
+_lib.gdn_forward_host.argtypes = [_vp, ctypes.POINTER(Inputs), _vp, _vp, _vp, _vp]
+_lib.gdn_forward_host.restype = ctypes.c_int
+_lib.gdn_staging_bytes.argtypes = [_vp]
+_lib.gdn_staging_bytes.restype = ctypes.c_size_t
+_lib.gdn_get_device_status.argtypes = [_vp, _vp, _vp]
+_lib.gdn_get_device_status.restype = ctypes.c_int
+_lib.gdn_launches_per_forward.argtypes = [_vp]
+_lib.gdn_launches_per_forward.restype = ctypes.c_int
+_lib.gdn_plan_uses_tensor_path.argtypes = [_vp]
+_lib.gdn_plan_uses_tensor_path.restype = ctypes.c_int
+_lib.gdn_workspace_offsets.argtypes = [_vp, ctypes.POINTER(ctypes.c_size_t), ctypes.c_int]
+_lib.gdn_workspace_offsets.restype = ctypes.c_int
+_lib.gdn_destroy.argtypes = [_vp]
+_lib.gdn_destroy.restype = ctypes.c_int
+_lib.gdn_status_string.argtypes = [ctypes.c_int]
+_lib.gdn_status_string.restype = ctypes.c_char_p
+
+
+class GDNError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+def status_string(s: int) -> str:
+    return _lib.gdn_status_string(int(s)).decode()
+
+
+def declared_symbols() -> list[str]:
+    """Function names include/gdn.h declares."""
+    text = open(HEADER_PATH).read()
+    return sorted(set(re.findall(r"^[A-Za-z_][\w \*]*?\b(gdn_\w+)\s*\(", text, flags=re.M)))
+
+
+def library():
+    return _lib
+
+
+def _check(rc: int, where: str):
+    if rc != OK:
+        raise GDNError(rc, where)
+
+
+class Plan:
+    """A gdn_plan_t: validated shapes and the workspace layout (host state only)."""
+
+    def __init__(self, B, T, H, d, in_dtype=DTYPE_BF16, out_dtype=None, l2_eps=1e-6, norm_eps=1e-6,
+                 tok_stride=0, flags=0):
+        self.cfg = Config(B, T, H, d, d, in_dtype, in_dtype if out_dtype is None else out_dtype, 4, 64,
+                          l2_eps, norm_eps, tok_stride, flags)
+        self._h = _vp()
+        ws = ctypes.c_size_t()
+        _check(_lib.gdn_plan(ctypes.byref(self.cfg), ctypes.byref(self._h), ctypes.byref(ws)), "gdn_plan")
+        self.workspace_bytes = ws.value
+
+    @property
+    def handle(self):
+        return self._h
+
+    @property
+    def staging_bytes(self) -> int:
+        return _lib.gdn_staging_bytes(self._h)
+
+    @property
+    def launches(self) -> int:
+        return _lib.gdn_launches_per_forward(self._h)
+
+    @property
+    def uses_tensor_path(self) -> bool:
+        return bool(_lib.gdn_plan_uses_tensor_path(self._h))
+
+    def forward_raw(self, ptrs: dict, y: int, workspace: int, stream: int) -> None:
+        """gdn_forward with raw device addresses (ints)."""
+        ins = Inputs(*[ptrs[n] for n, _ in Inputs._fields_])
+        _check(_lib.gdn_forward(self._h, ctypes.byref(ins), y, workspace, stream), "gdn_forward")
+
+    def forward_host_raw(self, ptrs: dict, y_host: int, staging: int, workspace: int, stream: int) -> None:
+        """gdn_forward_host with raw host input addresses and device staging/workspace."""
+        ins = Inputs(*[ptrs[n] for n, _ in Inputs._fields_])
+        _check(_lib.gdn_forward_host(self._h, ctypes.byref(ins), y_host, staging, workspace, stream),
+               "gdn_forward_host")
+
+    WS_FIELDS = ("status", "qh", "kh", "vh", "G", "beta", "log_alpha", "W", "U", "Qt", "Kt", "Aqk", "o")
+
+    def workspace_offsets(self) -> dict:
+        arr = (ctypes.c_size_t * 13)()
+        n = _lib.gdn_workspace_offsets(self._h, arr, 13)
+        return {self.WS_FIELDS[i]: arr[i] for i in range(n)}
+
+    def device_status(self, workspace: int, stream: int) -> int:
+        return _lib.gdn_get_device_status(self._h, workspace, stream)
+
+    def close(self):
+        if self._h:
+            _lib.gdn_destroy(self._h)
+            self._h = _vp()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+# ------------------------------------------------------------- torch helpers
+def _torch_dtype_code(t):
+    import torch
+    return {torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_F16, torch.float32: DTYPE_F32}[t]
+
+
+_NAMES = ("q", "k", "v", "z", "g", "b", "conv_q", "conv_k", "conv_v", "A_log", "dt_bias", "norm_w")
+
+
+def tensor_ptrs(tensors: dict) -> dict:
+    return {n: tensors[n].data_ptr() for n in _NAMES}
+
+
+def forward(q, k, v, z, g, b, conv_q, conv_k, conv_v, A_log, dt_bias, norm_w, out_dtype=None,
+            l2_eps=1e-6, norm_eps=1e-6, plan: Plan | None = None, workspace=None, y=None, stream=None):
+    """GDN forward on CUDA tensors (q, k, v, z [B,T,H,d]; g, b [B,T,H] fp32; conv_* [H*d,4];
+    A_log, dt_bias [H]; norm_w [d]).  Returns y [B,T,H,d]."""
+    import torch
+    B, T, H, d = q.shape
+    in_code = _torch_dtype_code(q.dtype)
+    odt = q.dtype if out_dtype is None else out_dtype
+    if plan is None:
+        plan = Plan(B, T, H, d, in_code, _torch_dtype_code(odt), l2_eps, norm_eps, q.stride(1))
+    if workspace is None:
+        workspace = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=q.device)
+    if y is None:
+        y = torch.empty((B, T, H, d), dtype=odt, device=q.device)
+    s = torch.cuda.current_stream(q.device).cuda_stream if stream is None else stream
+    t = dict(q=q, k=k, v=v, z=z, g=g, b=b, conv_q=conv_q, conv_k=conv_k, conv_v=conv_v, A_log=A_log,
+             dt_bias=dt_bias, norm_w=norm_w)
+    plan.forward_raw(tensor_ptrs(t), y.data_ptr(), workspace.data_ptr(), s)
+    return y

@@ -1,0 +1,338 @@
+// gdn_api.cu -- the C ABI declared in include/gdn.h: plan validation and
+// workspace layout, tensor-map construction, and the launch sequence of the
+// GDN forward.  No device memory is allocated here; every buffer is the
+// caller's.
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+
+#include "gdn.h"
+#include "gdn_common.cuh"
+#include "gdn_internal.h"
+
+using namespace gdn;
+
+struct gdn_plan_s {
+    gdn_config cfg;
+    int device;
+    bool tensor;
+    int Tp, NB;
+    long long tok_stride;
+    size_t in_esize, out_esize, inter_esize;
+    // workspace layout
+    size_t off_status, off_qh, off_kh, off_vh, off_G, off_beta, off_la;
+    size_t off_W, off_U, off_Qt, off_Kt, off_Aqk, off_o, ws_bytes;
+    // staging layout (gdn_forward_host)
+    size_t st_q, st_k, st_v, st_z, st_g, st_b, st_cq, st_ck, st_cv, st_A, st_dt, st_nw, st_y, staging_bytes;
+};
+
+namespace {
+
+constexpr unsigned long long kWaitLimitNs = 2000ull * 1000 * 1000;  // 2 s per device-side wait
+
+size_t esize(gdn_dtype t) { return t == GDN_DTYPE_F32 ? 4 : 2; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+InType in_type(gdn_dtype t) {
+    return t == GDN_DTYPE_BF16 ? InType::BF16 : (t == GDN_DTYPE_F16 ? InType::F16 : InType::F32);
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// [rows][128] fp16 row-major, loaded as {64, 128} boxes with the 128-byte swizzle.
+bool make_tile_map(CUtensorMap *m, void *base, unsigned long long rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {128, rows};
+    const cuuint64_t strides[1] = {128 * 2};
+    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *gdn_status_string(gdn_status s) {
+    switch (s) {
+        case GDN_OK: return "ok";
+        case GDN_ERR_INVALID_ARG: return "invalid argument";
+        case GDN_ERR_UNSUPPORTED: return "unsupported configuration";
+        case GDN_ERR_CUDA: return "CUDA error";
+        case GDN_ERR_TIMEOUT: return "device-side wait timed out";
+        case GDN_ERR_DEVICE_CHECK: return "device-side check failed";
+        case GDN_ERR_NO_DEVICE: return "no sm_100 CUDA device";
+    }
+    return "unknown status";
+}
+
+gdn_status gdn_plan(const gdn_config *cfg, gdn_plan_t *out, size_t *workspace_bytes) {
+    if (!cfg || !out || !workspace_bytes) return GDN_ERR_INVALID_ARG;
+    *out = nullptr;
+    const gdn_config c = *cfg;
+    if (c.B < 1 || c.H < 1 || c.T < 1 || c.d_k < 1 || c.d_v < 1) return GDN_ERR_INVALID_ARG;
+    if (!(c.l2_eps >= 0.0f) || !(c.norm_eps >= 0.0f) || !isfinite(c.l2_eps) || !isfinite(c.norm_eps))
+        return GDN_ERR_INVALID_ARG;
+    if (c.in_dtype != GDN_DTYPE_BF16 && c.in_dtype != GDN_DTYPE_F16 && c.in_dtype != GDN_DTYPE_F32)
+        return GDN_ERR_UNSUPPORTED;
+    if (c.out_dtype != GDN_DTYPE_BF16 && c.out_dtype != GDN_DTYPE_F16 && c.out_dtype != GDN_DTYPE_F32)
+        return GDN_ERR_UNSUPPORTED;
+    if (c.d_k != c.d_v || (c.d_k != 64 && c.d_k != 128)) return GDN_ERR_UNSUPPORTED;
+    if (c.conv_size != 4 || c.chunk != 64) return GDN_ERR_UNSUPPORTED;
+    const int d = c.d_k;
+    const long long dense = static_cast<long long>(c.H) * d;
+    const long long ts = c.tok_stride == 0 ? dense : c.tok_stride;
+    if (ts < dense) return GDN_ERR_INVALID_ARG;
+    if ((ts * static_cast<long long>(esize(c.in_dtype))) % 16 != 0) return GDN_ERR_INVALID_ARG;
+    const long long Tp = (static_cast<long long>(c.T) + kBlk - 1) / kBlk * kBlk;
+    const long long BH = static_cast<long long>(c.B) * c.H;
+    if (BH * Tp >= (1ll << 31)) return GDN_ERR_UNSUPPORTED;  // TMA row coordinates are int32
+
+    int dev = -1, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return GDN_ERR_NO_DEVICE; }
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess || major != 10) {
+        cudaGetLastError();
+        return GDN_ERR_NO_DEVICE;
+    }
+
+    gdn_plan_s *p = new (std::nothrow) gdn_plan_s;
+    if (!p) return GDN_ERR_INVALID_ARG;
+    memset(p, 0, sizeof(*p));
+    p->cfg = c;
+    p->device = dev;
+    p->tensor = (c.in_dtype != GDN_DTYPE_F32) && d == 128 && !(c.flags & GDN_FLAG_FORCE_SIMT);
+    p->Tp = static_cast<int>(Tp);
+    p->NB = static_cast<int>(Tp / kBlk);
+    p->tok_stride = ts;
+    p->in_esize = esize(c.in_dtype);
+    p->out_esize = esize(c.out_dtype);
+    p->inter_esize = p->tensor ? 2 : 4;
+
+    const size_t A = 1024;
+    const size_t nTok = static_cast<size_t>(BH) * Tp;
+    const size_t act = nTok * d;
+    size_t off = 0;
+    p->off_status = off; off = align_up(off + 256, A);
+    p->off_qh = off; off = align_up(off + act * p->inter_esize, A);
+    p->off_kh = off; off = align_up(off + act * p->inter_esize, A);
+    p->off_vh = off; off = align_up(off + act * p->inter_esize, A);
+    p->off_G = off; off = align_up(off + nTok * 4, A);
+    p->off_beta = off; off = align_up(off + nTok * 4, A);
+    p->off_la = off; off = align_up(off + nTok * 4, A);
+    if (p->tensor) {
+        p->off_W = off; off = align_up(off + act * 2, A);
+        p->off_U = off; off = align_up(off + act * 2, A);
+        p->off_Qt = off; off = align_up(off + act * 2, A);
+        p->off_Kt = off; off = align_up(off + act * 2, A);
+        p->off_Aqk = off; off = align_up(off + act * 2, A);
+    }
+    p->off_o = off; off = align_up(off + static_cast<size_t>(c.B) * c.T * c.H * d * 4, A);
+    p->ws_bytes = off;
+
+    const size_t ntok_in = static_cast<size_t>(c.B) * c.T;
+    const size_t a_in = ntok_in * c.H * d * p->in_esize;
+    off = 0;
+    p->st_q = off; off = align_up(off + a_in, 256);
+    p->st_k = off; off = align_up(off + a_in, 256);
+    p->st_v = off; off = align_up(off + a_in, 256);
+    p->st_z = off; off = align_up(off + a_in, 256);
+    p->st_g = off; off = align_up(off + ntok_in * c.H * 4, 256);
+    p->st_b = off; off = align_up(off + ntok_in * c.H * 4, 256);
+    p->st_cq = off; off = align_up(off + static_cast<size_t>(c.H) * d * 16, 256);
+    p->st_ck = off; off = align_up(off + static_cast<size_t>(c.H) * d * 16, 256);
+    p->st_cv = off; off = align_up(off + static_cast<size_t>(c.H) * d * 16, 256);
+    p->st_A = off; off = align_up(off + static_cast<size_t>(c.H) * 4, 256);
+    p->st_dt = off; off = align_up(off + static_cast<size_t>(c.H) * 4, 256);
+    p->st_nw = off; off = align_up(off + static_cast<size_t>(d) * 4, 256);
+    p->st_y = off; off = align_up(off + ntok_in * c.H * d * p->out_esize, 256);
+    p->staging_bytes = off;
+
+    *out = p;
+    *workspace_bytes = p->ws_bytes;
+    return GDN_OK;
+}
+
+gdn_status gdn_destroy(gdn_plan_t plan) {
+    delete plan;
+    return GDN_OK;
+}
+
+int gdn_launches_per_forward(gdn_plan_t plan) { return plan ? (plan->tensor ? 4 : 3) : 0; }
+
+int gdn_plan_uses_tensor_path(gdn_plan_t plan) { return plan && plan->tensor ? 1 : 0; }
+
+size_t gdn_staging_bytes(gdn_plan_t plan) { return plan ? plan->staging_bytes : 0; }
+
+int gdn_workspace_offsets(gdn_plan_t plan, size_t *offsets, int n) {
+    if (!plan || !offsets || n <= 0) return 0;
+    const size_t all[13] = {plan->off_status, plan->off_qh, plan->off_kh, plan->off_vh, plan->off_G,
+                            plan->off_beta, plan->off_la, plan->off_W, plan->off_U, plan->off_Qt,
+                            plan->off_Kt, plan->off_Aqk, plan->off_o};
+    const int m = n < 13 ? n : 13;
+    for (int i = 0; i < m; ++i) offsets[i] = all[i];
+    return m;
+}
+
+gdn_status gdn_forward(gdn_plan_t plan, const gdn_inputs *in, void *y, void *workspace, gdn_stream_t stream) {
+    if (!plan || !in || !y || !workspace) return GDN_ERR_INVALID_ARG;
+    const gdn_config &c = plan->cfg;
+    const void *ptrs16[] = {in->q, in->k, in->v, in->z, y};
+    for (const void *q : ptrs16)
+        if (!q || !aligned16(q)) return GDN_ERR_INVALID_ARG;
+    const void *ptrs4[] = {in->g, in->b, in->conv_q, in->conv_k, in->conv_v, in->A_log, in->dt_bias, in->norm_w};
+    for (const void *q : ptrs4)
+        if (!q || (reinterpret_cast<uintptr_t>(q) & 3u)) return GDN_ERR_INVALID_ARG;
+    const void *ptrsw[] = {in->conv_q, in->conv_k, in->conv_v};
+    for (const void *q : ptrsw)
+        if (!aligned16(q)) return GDN_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return GDN_ERR_INVALID_ARG;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != plan->device) return GDN_ERR_INVALID_ARG;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    int *status = reinterpret_cast<int *>(ws + plan->off_status);
+    float *G = reinterpret_cast<float *>(ws + plan->off_G);
+    float *beta = reinterpret_cast<float *>(ws + plan->off_beta);
+    float *la = reinterpret_cast<float *>(ws + plan->off_la);
+    float *o = reinterpret_cast<float *>(ws + plan->off_o);
+    const int d = c.d_k;
+
+    if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return GDN_ERR_CUDA;
+
+    PrepParams pp;
+    pp.q = in->q; pp.k = in->k; pp.v = in->v;
+    pp.tok_stride = plan->tok_stride;
+    pp.g = in->g; pp.b = in->b;
+    pp.conv_q = in->conv_q; pp.conv_k = in->conv_k; pp.conv_v = in->conv_v;
+    pp.A_log = in->A_log; pp.dt_bias = in->dt_bias;
+    pp.qh = ws + plan->off_qh; pp.kh = ws + plan->off_kh; pp.vh = ws + plan->off_vh;
+    pp.G = G; pp.beta = beta; pp.log_alpha = la;
+    pp.B = c.B; pp.T = c.T; pp.H = c.H; pp.d = d; pp.Tp = plan->Tp;
+    pp.l2_eps = c.l2_eps;
+    pp.q_scale = 1.0f / sqrtf(static_cast<float>(d));
+    if (launch_prep(pp, in_type(c.in_dtype), plan->tensor, s) != cudaSuccess) return GDN_ERR_CUDA;
+
+    if (plan->tensor) {
+        const unsigned long long rows = static_cast<unsigned long long>(c.B) * c.H * plan->Tp;
+        CUtensorMap tmQ, tmK, tmV, tmW, tmU, tmQt, tmKt, tmAqk;
+        if (!make_tile_map(&tmQ, ws + plan->off_qh, rows) || !make_tile_map(&tmK, ws + plan->off_kh, rows) ||
+            !make_tile_map(&tmV, ws + plan->off_vh, rows) || !make_tile_map(&tmW, ws + plan->off_W, rows) ||
+            !make_tile_map(&tmU, ws + plan->off_U, rows) || !make_tile_map(&tmQt, ws + plan->off_Qt, rows) ||
+            !make_tile_map(&tmKt, ws + plan->off_Kt, rows) || !make_tile_map(&tmAqk, ws + plan->off_Aqk, rows))
+            return GDN_ERR_CUDA;
+        ChunkParams cp;
+        cp.G = G; cp.beta = beta;
+        cp.W = reinterpret_cast<__half *>(ws + plan->off_W);
+        cp.U = reinterpret_cast<__half *>(ws + plan->off_U);
+        cp.Qt = reinterpret_cast<__half *>(ws + plan->off_Qt);
+        cp.Kt = reinterpret_cast<__half *>(ws + plan->off_Kt);
+        cp.Aqk = reinterpret_cast<__half *>(ws + plan->off_Aqk);
+        cp.BH = c.B * c.H; cp.Tp = plan->Tp; cp.NB = plan->NB;
+        cp.status = status;
+        cp.wait_limit_ns = kWaitLimitNs;
+        if (launch_chunk(cp, tmK, tmV, tmQ, s) != cudaSuccess) return GDN_ERR_CUDA;
+        ScanParams sp;
+        sp.G = G; sp.o = o;
+        sp.B = c.B; sp.T = c.T; sp.H = c.H; sp.Tp = plan->Tp; sp.NB = plan->NB;
+        sp.status = status;
+        sp.wait_limit_ns = kWaitLimitNs;
+        sp.test_wait_timeout = (c.flags & GDN_FLAG_TEST_WAIT_TIMEOUT) ? 1 : 0;
+        if (launch_scan(sp, tmW, tmQt, tmKt, tmAqk, tmU, s) != cudaSuccess) return GDN_ERR_CUDA;
+    } else {
+        RecurParams rp;
+        rp.qh = reinterpret_cast<const float *>(ws + plan->off_qh);
+        rp.kh = reinterpret_cast<const float *>(ws + plan->off_kh);
+        rp.vh = reinterpret_cast<const float *>(ws + plan->off_vh);
+        rp.log_alpha = la; rp.beta = beta; rp.o = o;
+        rp.B = c.B; rp.T = c.T; rp.H = c.H; rp.d = d; rp.Tp = plan->Tp;
+        if (launch_recurrence(rp, s) != cudaSuccess) return GDN_ERR_CUDA;
+    }
+
+    OutParams op;
+    op.o = o; op.z = in->z; op.tok_stride = plan->tok_stride; op.norm_w = in->norm_w; op.y = y;
+    op.B = c.B; op.T = c.T; op.H = c.H; op.dv = c.d_v; op.eps = c.norm_eps;
+    if (launch_output(op, in_type(c.in_dtype), in_type(c.out_dtype), s) != cudaSuccess) return GDN_ERR_CUDA;
+    return GDN_OK;
+}
+
+gdn_status gdn_forward_host(gdn_plan_t plan, const gdn_inputs *in_host, void *y_host, void *staging,
+                            void *workspace, gdn_stream_t stream) {
+    if (!plan || !in_host || !y_host || !staging || !workspace) return GDN_ERR_INVALID_ARG;
+    const gdn_config &c = plan->cfg;
+    const int d = c.d_k;
+    if (plan->tok_stride != static_cast<long long>(c.H) * d) return GDN_ERR_UNSUPPORTED;  // host buffers are dense
+    if (reinterpret_cast<uintptr_t>(staging) & 255u) return GDN_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *st = static_cast<uint8_t *>(staging);
+    const size_t ntok = static_cast<size_t>(c.B) * c.T;
+    const size_t a_in = ntok * c.H * d * plan->in_esize;
+    const size_t gb = ntok * c.H * 4;
+    const size_t cw = static_cast<size_t>(c.H) * d * 16;
+    struct Copy { size_t off; const void *src; size_t bytes; } copies[] = {
+        {plan->st_q, in_host->q, a_in}, {plan->st_k, in_host->k, a_in}, {plan->st_v, in_host->v, a_in},
+        {plan->st_z, in_host->z, a_in}, {plan->st_g, in_host->g, gb}, {plan->st_b, in_host->b, gb},
+        {plan->st_cq, in_host->conv_q, cw}, {plan->st_ck, in_host->conv_k, cw}, {plan->st_cv, in_host->conv_v, cw},
+        {plan->st_A, in_host->A_log, static_cast<size_t>(c.H) * 4},
+        {plan->st_dt, in_host->dt_bias, static_cast<size_t>(c.H) * 4},
+        {plan->st_nw, in_host->norm_w, static_cast<size_t>(d) * 4}};
+    for (const Copy &cp : copies) {
+        if (!cp.src) return GDN_ERR_INVALID_ARG;
+        if (cudaMemcpyAsync(st + cp.off, cp.src, cp.bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return GDN_ERR_CUDA;
+    }
+    gdn_inputs dev;
+    dev.q = st + plan->st_q; dev.k = st + plan->st_k; dev.v = st + plan->st_v; dev.z = st + plan->st_z;
+    dev.g = reinterpret_cast<const float *>(st + plan->st_g);
+    dev.b = reinterpret_cast<const float *>(st + plan->st_b);
+    dev.conv_q = reinterpret_cast<const float *>(st + plan->st_cq);
+    dev.conv_k = reinterpret_cast<const float *>(st + plan->st_ck);
+    dev.conv_v = reinterpret_cast<const float *>(st + plan->st_cv);
+    dev.A_log = reinterpret_cast<const float *>(st + plan->st_A);
+    dev.dt_bias = reinterpret_cast<const float *>(st + plan->st_dt);
+    dev.norm_w = reinterpret_cast<const float *>(st + plan->st_nw);
+    const gdn_status rc = gdn_forward(plan, &dev, st + plan->st_y, workspace, stream);
+    if (rc != GDN_OK) return rc;
+    if (cudaMemcpyAsync(y_host, st + plan->st_y, ntok * c.H * d * plan->out_esize, cudaMemcpyDeviceToHost, s) !=
+        cudaSuccess)
+        return GDN_ERR_CUDA;
+    return GDN_OK;
+}
+
+gdn_status gdn_get_device_status(gdn_plan_t plan, void *workspace, gdn_stream_t stream) {
+    if (!plan || !workspace) return GDN_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int *status = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + plan->off_status);
+    int host = 0;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return GDN_ERR_CUDA;
+    if (cudaMemcpy(&host, status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return GDN_ERR_CUDA;
+    if (cudaMemset(status, 0, sizeof(int)) != cudaSuccess) return GDN_ERR_CUDA;
+    if (host == kStatusTimeout) return GDN_ERR_TIMEOUT;
+    if (host != kStatusOk) return GDN_ERR_DEVICE_CHECK;
+    return GDN_OK;
+}
+
+}  // extern "C"

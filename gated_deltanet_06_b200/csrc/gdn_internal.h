@@ -1,0 +1,76 @@
+// gdn_internal.h -- host-side launchers of the GDN forward kernels and the
+// parameter blocks they take.  Internal to the library (not installed).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace gdn {
+
+enum class InType { BF16 = 0, F32 = 1, F16 = 2 };
+
+// Prep: conv4 + SiLU on q, k, v; L2 norm (and the 1/sqrt(d_k) output scale
+// folded into q^); log-decay, in-block cumulative log-decay, update gate.
+struct PrepParams {
+    const void *q, *k, *v;
+    long long tok_stride;          // elements between tokens of q, k, v
+    const float *g, *b;            // [B][T][H]
+    const float *conv_q, *conv_k, *conv_v;  // [H*d][4]
+    const float *A_log, *dt_bias;  // [H]
+    void *qh, *kh, *vh;            // [B][H][Tp][d]  (fp16 or fp32)
+    float *G;                      // [B][H][Tp] in-block (128) inclusive cumsum of log alpha
+    float *beta;                   // [B][H][Tp]
+    float *log_alpha;              // [B][H][Tp]
+    int B, T, H, d, Tp;
+    float l2_eps, q_scale;
+};
+cudaError_t launch_prep(const PrepParams &p, InType in, bool out_f16, cudaStream_t s);
+
+// Intra-block UT transform on tensor cores (d = 128, fp16 operands).
+struct ChunkParams {
+    const float *G, *beta;          // [BH][Tp]
+    __half *W, *U, *Qt, *Kt, *Aqk;  // [BH][Tp][128]
+    int BH, Tp, NB;
+    int *status;
+    unsigned long long wait_limit_ns;
+};
+cudaError_t launch_chunk(const ChunkParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                         const CUtensorMap &tmQ, cudaStream_t s);
+
+// Inter-block state scan + block outputs on tensor cores (d = 128).
+struct ScanParams {
+    const float *G;  // [BH][Tp]
+    float *o;        // [B][T][H][128] fp32
+    int B, T, H, Tp, NB;
+    int *status;
+    unsigned long long wait_limit_ns;
+    int test_wait_timeout;
+};
+cudaError_t launch_scan(const ScanParams &p, const CUtensorMap &tmW, const CUtensorMap &tmQt,
+                        const CUtensorMap &tmKt, const CUtensorMap &tmAqk, const CUtensorMap &tmU,
+                        cudaStream_t s);
+
+// Sequential fp32 recurrence on CUDA cores (fp32 inputs or d = 64).
+struct RecurParams {
+    const float *qh, *kh, *vh;  // [B][H][Tp][d]
+    const float *log_alpha, *beta;
+    float *o;  // [B][T][H][d]
+    int B, T, H, d, Tp;
+};
+cudaError_t launch_recurrence(const RecurParams &p, cudaStream_t s);
+
+// y = o / sqrt(mean(o^2) + eps) * w * SiLU(z)
+struct OutParams {
+    const float *o;  // [B][T][H][dv]
+    const void *z;
+    long long tok_stride;  // of z
+    const float *norm_w;
+    void *y;  // [B][T][H][dv]
+    int B, T, H, dv;
+    float eps;
+};
+cudaError_t launch_output(const OutParams &p, InType zt, InType yt, cudaStream_t s);
+
+}  // namespace gdn

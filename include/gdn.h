@@ -140,6 +140,17 @@ int gdn_launches_per_forward(gdn_plan_t plan);
 /* 1 if the plan runs the tensor-core (tcgen05) path, 0 for the fp32 CUDA-core path. */
 int gdn_plan_uses_tensor_path(gdn_plan_t plan);
 
+/* Introspection for per-stage tests: writes up to n byte offsets, inside the
+ * workspace, of the intermediates of the last forward, in this order:
+ *   0 status word (int), 1 q^ (scaled by 1/sqrt(d_k)), 2 k^, 3 v^
+ *     ([B][H][Tp][d], fp16 on the tensor path, fp32 otherwise; Tp = T rounded
+ *     up to 128),
+ *   4 G (in-block cumulative log decay), 5 beta, 6 log alpha ([B][H][Tp] fp32),
+ *   7 W, 8 U, 9 Qt, 10 Kt, 11 Aqk ([B][H][Tp][128] fp16; tensor path only,
+ *     else 0), 12 o ([B][T][H][d_v] fp32, before the output norm).
+ * Returns the number of offsets written (13 at most). */
+int gdn_workspace_offsets(gdn_plan_t plan, size_t *offsets, int n);
+
 /* Free a plan (host memory only).  NULL is accepted. */
 gdn_status gdn_destroy(gdn_plan_t plan);
 
