@@ -1,0 +1,404 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 GDN forward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--T T] [--no-cpu-baseline] [--no-e2e]
+
+A step is one whole GDN forward (prep, UT transform, scan, output) over the
+workload with its inputs resident in HBM; the L2 cache is flushed (256 MiB
+write) before every step, outside the timed interval.  Each step is timed
+with CUDA events on the launching stream; per-kernel times come from events
+the library records between its launches (gdn_forward_timed).  With N > 1
+(torchrun) every rank runs its own replica of the workload (the forward has
+no cross-GPU exchange) and the time is the max over ranks.  Rank 0 prints one
+JSON line.
+
+--impl reference times the oracle (the plain fp64 CPU statement of the
+method) on this host's cores, on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import gdn_inputs  # noqa: E402
+
+METRIC = "GDN fwd Mtokens/s at T=32760,H=12,d=128 bf16; % of tensor/HBM roofline"
+UNIT = "Mtokens/s"
+FLUSH_BYTES = 256 << 20
+KERNELS_TENSOR_SEG = ("prep", "chunk", "transfer", "combine", "scan")
+KERNELS_TENSOR_ONE = ("prep", "chunk", "scan")
+KERNELS_SIMT = ("prep", "recurrence", "output")
+KERNEL_SOURCES = {"prep": "gdn_prep.cu", "chunk": "gdn_chunk.cu", "transfer": "gdn_scan.cu",
+                  "combine": "gdn_scan.cu", "scan": "gdn_scan.cu", "recurrence": "gdn_simt.cu",
+                  "output": "gdn_simt.cu"}
+
+
+def path_bytes_per_token_head(d, s_in, s_out):
+    # q, k, v, z in; g, b fp32 in; y out (parameters negligible)
+    return 4 * d * s_in + 8 + d * s_out
+
+
+def path_flops_per_token_head(d, C=64):
+    # five C x C x d block products counted as full tiles + three C x d x d products per chunk
+    return 10 * C * d + 6 * d * d
+
+
+def kernel_work_per_token_head(name, d, s_in, s_out):
+    """Algorithmic bytes and flops each kernel must move / do per (token, head)
+    on the tensor path (fp16 intermediates, fp32 o)."""
+    if name == "prep":      # q k v in, g b in; q^ k^ v^ fp16 out; G beta log-alpha out
+        return 3 * d * s_in + 8 + 3 * d * 2 + 12, 0
+    if name == "chunk":     # q^ k^ v^ + G beta in; W U Qt Kt Aqk out; K K^T, Q K^T, W, U products
+        return 3 * d * 2 + 8 + 5 * 128 * 2, 4 * 2 * 128 * d
+    if name == "transfer":  # W U Kt in; W [S|P]^T and Kt^T Delta with N = 2d
+        return 3 * 128 * 2, 2 * 2 * 128 * 2 * d
+    if name == "combine":   # per-segment states only (negligible per token)
+        return 0, 0
+    if name == "scan":      # W U Qt Kt Aqk + z in, y out; W S^T, Qt S^T, Kt^T Delta, Aqk Delta
+        return 5 * 128 * 2 + d * s_in + d * s_out, 4 * 2 * 128 * d
+    if name == "output":    # o fp32 + z in; y out
+        return d * 4 + d * s_in + d * s_out, 0
+    if name == "recurrence":
+        return 3 * d * 4 + 8 + d * 4, 6 * d * d
+    raise KeyError(name)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return dict(hbm_gbs=float(j["hbm_gbs"]), bf16_tflops=float(j["bf16_tflops"]),
+                    bf16_tflops_sustained=float(j.get("bf16_tflops_sustained", j["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def kernel_source_sha(name):
+    with open(os.path.join(ROOT, "gated_deltanet_06_b200", "csrc", KERNEL_SOURCES[name]), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def ncu_traffic(name, workload):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's
+    source is unchanged since the capture; else None."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    e = j.get(name, {}).get(workload)
+    if not e or e.get("source_sha") != kernel_source_sha(name):
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.dev = device_index
+
+    def start(self):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        idx = self.dev
+        if vis:
+            try:
+                idx = int(vis.split(",")[self.dev])
+            except (ValueError, IndexError):
+                idx = None
+        sel = ["-i", str(idx)] if idx is not None else []
+        self.err = os.path.join(ROOT, "gpurun_out", "clock_sampler.err") if os.path.isdir(
+            os.path.join(ROOT, "gpurun_out")) else os.devnull
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                                          "-lms", "100"] + sel, stdout=subprocess.PIPE,
+                                         stderr=open(self.err, "w"), text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [[x.strip() for x in line.split(",")] for line in out.strip().splitlines() if line.strip()]
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                s = float(r[1]); mx = float(r[2])
+            except (ValueError, IndexError):
+                continue
+            sm.append(s)
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        loaded = [s for s in sm if mx and s >= 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def oracle_rate(w, T_sample, threads):
+    import oracle
+    inp = gdn_inputs.workload_inputs(w, T=T_sample)
+    t0 = time.perf_counter()
+    oracle.forward(inp, nthreads=threads)
+    return time.perf_counter() - t0
+
+
+def cpu_threads(w):
+    return max(1, min(w.B * w.H, os.cpu_count() or 1))
+
+
+def calibrate_oracle_T(w, seconds, threads):
+    t_small = 256
+    dt = oracle_rate(w, t_small, threads)
+    per_tok = dt / t_small
+    return int(max(256, min(w.T, seconds / max(per_tok, 1e-9))))
+
+
+def run_cpu_baseline(w, budget_s=12.0):
+    threads = cpu_threads(w)
+    T_s = calibrate_oracle_T(w, budget_s, threads)
+    dt = oracle_rate(w, T_s, threads)
+    return {"value": w.B * T_s / dt / 1e6, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{w.name} at T={T_s} instead of {w.T} (same seed, distributions, B and H; "
+                      f"cost is linear in T): fp64 sequential recurrence, {threads} threads, {dt:.1f} s"}
+
+
+def reference_arm(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    threads = cpu_threads(w)
+    per_step = max(0.2, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    T_s = calibrate_oracle_T(w, per_step, threads)
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt = oracle_rate(w, T_s, threads)
+        if i >= args.warmup:
+            times.append(dt)
+    total = sum(times)
+    value = w.B * T_s * len(times) / total / 1e6
+    sample = (f"{w.name} at T={T_s} instead of {w.T} per step (same seed, distributions, B and H; "
+              f"cost is linear in T): fp64 sequential recurrence, {threads} threads")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "d": w.d, "sample_T": T_s},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=gdn_inputs.HEADLINE.name)
+    ap.add_argument("--T", type=int, default=None, help="override the sequence length (profiling runs)")
+    ap.add_argument("--out-dtype", default=None, choices=[None, "bf16", "f16", "f32"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--load-seconds", type=float, default=1.5)
+    args = ap.parse_args()
+    w = gdn_inputs.by_name(args.workload)
+    if args.T:
+        w = gdn_inputs.Workload(w.name + f"_T{args.T}", w.B, w.H, args.T, w.d, w.dtype, w.g_mean, w.seed, w.note)
+    if args.impl == "reference":
+        return reference_arm(args, w)
+
+    import torch
+    import torch.distributed as dist
+
+    import gated_deltanet_06_b200 as gdn
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+
+    inp = gdn_inputs.workload_inputs(w, T=args.T)
+    tens = {}
+    for n in ("q", "k", "v", "z"):
+        if w.dtype == "bf16":
+            tens[n] = torch.from_numpy(inp[n + "_bits"].view(np.int16)).view(torch.bfloat16).to(dev)
+        else:
+            tens[n] = torch.from_numpy(inp[n]).to(dev)
+    for n in ("g", "b", "conv_q", "conv_k", "conv_v", "A_log", "dt_bias", "norm_w"):
+        tens[n] = torch.from_numpy(np.ascontiguousarray(inp[n], dtype=np.float32)).to(dev)
+    in_code = gdn.DTYPE_BF16 if w.dtype == "bf16" else gdn.DTYPE_F32
+    out_name = args.out_dtype or ("bf16" if w.dtype == "bf16" else "f32")
+    out_code = {"bf16": gdn.DTYPE_BF16, "f16": gdn.DTYPE_F16, "f32": gdn.DTYPE_F32}[out_name]
+    out_t = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[out_name]
+    plan = gdn.Plan(w.B, w.T, w.H, w.d, in_code, out_code)
+    ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=dev)
+    y = torch.empty((w.B, w.T, w.H, w.d), dtype=out_t, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    s = stream.cuda_stream
+    ptrs = gdn.tensor_ptrs(tens)
+    L = plan.launches
+    if plan.uses_tensor_path:
+        names = KERNELS_TENSOR_SEG if plan.segments > 1 else KERNELS_TENSOR_ONE
+    else:
+        names = KERNELS_SIMT
+    assert len(names) == L
+
+    for _ in range(args.warmup):
+        plan.forward_raw(ptrs, y.data_ptr(), ws.data_ptr(), s)
+    torch.cuda.synchronize()
+    # untimed load phase so that the clock samples see the GPU busy with this work
+    sampler = ClockSampler(local)
+    sampler.start()
+    t_end = time.perf_counter() + args.load_seconds
+    while time.perf_counter() < t_end:
+        for _ in range(20):
+            plan.forward_raw(ptrs, y.data_ptr(), ws.data_ptr(), s)
+        torch.cuda.synchronize()
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(L + 1)] for _ in range(args.steps)]
+    for row in events:  # torch creates the underlying cudaEvent_t on first record
+        for e in row:
+            e.record(stream)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        flush.zero_()
+        plan.forward_timed_raw(ptrs, y.data_ptr(), ws.data_ptr(), s, [e.cuda_event for e in events[k]])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    st = plan.device_status(ws.data_ptr(), s)
+    if st != gdn.OK:
+        raise SystemExit(f"device status after timing: {gdn.status_string(st)}")
+
+    step_ms = [events[k][0].elapsed_time(events[k][L]) for k in range(args.steps)]
+    kern_ms = {names[i]: statistics.mean(events[k][i].elapsed_time(events[k][i + 1]) for k in range(args.steps))
+               for i in range(L)}
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    tokens = w.B * w.T
+    value = world * tokens / (ms_per_step / 1e3) / 1e6
+
+    # end to end through the public host-buffer entry point
+    e2e = None
+    if not args.no_e2e:
+        host = {n: tens[n].cpu().pin_memory() for n in tens}
+        y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+        staging = torch.empty(plan.staging_bytes, dtype=torch.uint8, device=dev)
+        hptrs = gdn.tensor_ptrs(host)
+        n_e2e = max(3, min(args.steps, 10))
+        plan.forward_host_raw(hptrs, y_host.data_ptr(), staging.data_ptr(), ws.data_ptr(), s)
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        ev0.record(stream)
+        for _ in range(n_e2e):
+            plan.forward_host_raw(hptrs, y_host.data_ptr(), staging.data_ptr(), ws.data_ptr(), s)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([ev0.elapsed_time(ev1) / n_e2e], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        h2d = sum(host[n].numel() * host[n].element_size() for n in host)
+        d2h = y_host.numel() * y_host.element_size()
+        e2e = {"value": world * tokens / (float(te.item()) / 1e3) / 1e6, "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n_e2e}
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
+    peaks = load_peaks()
+    s_in = 2 if w.dtype == "bf16" else 4
+    s_out = {"bf16": 2, "f16": 2, "f32": 4}[out_name]
+    units = w.B * w.T * w.H
+    top = max(kern_ms, key=kern_ms.get)
+    kb, kf = kernel_work_per_token_head(top, w.d, s_in, s_out)
+    if top == "transfer":  # pass A covers every segment but the last
+        ns = plan.segments
+        ls = -(-(-(-w.T // 128)) // ns)
+        units = w.B * w.H * min((ns - 1) * ls * 128, w.T)
+    t_top = kern_ms[top] / 1e3
+    ach_gbs = kb * units / t_top / 1e9
+    ach_tfs = kf * units / t_top / 1e12
+    # a kernel is reported against the roof it is closer to
+    if kf and ach_tfs / peaks["bf16_tflops"] > ach_gbs / peaks["hbm_gbs"]:
+        roof = {"bound": "tensor", "achieved": ach_tfs, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": ach_tfs / peaks["bf16_tflops"]}
+    else:
+        roof = {"bound": "hbm", "achieved": ach_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach_gbs / peaks["hbm_gbs"]}
+    traffic = ncu_traffic(top, w.name)
+    roof.update(kernel=top, traffic=traffic, peak_source=peaks["source"] + " (MEASURED_PEAKS.json)"
+                if peaks["source"] == "measured" else "fallback",
+                algorithmic_bytes_per_launch=kb * units, algorithmic_flops_per_launch=kf * units,
+                avg_launch_ms=kern_ms[top], units_per_launch=units)
+    units = w.B * w.T * w.H
+    pb = path_bytes_per_token_head(w.d, s_in, s_out)
+    pf = path_flops_per_token_head(w.d)
+    t_roof = max(pb * units / (peaks["hbm_gbs"] * 1e9), pf * units / (peaks["bf16_tflops"] * 1e12))
+    path_roof = {"bytes_per_token_head": pb, "flops_per_token_head": pf, "roofline_ms": t_roof * 1e3,
+                 "roofline_Mtokens_s": tokens / t_roof / 1e6, "frac": (t_roof * 1e3) / ms_per_step}
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = run_cpu_baseline(w)
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f16-mma/f32", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "d": w.d, "in_dtype": w.dtype,
+                       "out_dtype": out_name, "g_mean": w.g_mean, "seed": w.seed,
+                       "l2": "flushed before every step (256 MiB write, outside the timed interval)",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "roofline": roof, "path_roofline": path_roof, "kernels_ms": kern_ms,
+            "segments": plan.segments, "cpu_baseline": cpu, "e2e": e2e,
+            "clocks": clocks, "gpu_launches": L * args.steps,
+            "gpu": torch.cuda.get_device_name(dev)}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

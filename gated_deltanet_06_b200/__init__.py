@@ -49,6 +49,8 @@ _lib.gdn_plan.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(_vp), ctypes.PO
 _lib.gdn_plan.restype = ctypes.c_int
 _lib.gdn_forward.argtypes = [_vp, ctypes.POINTER(Inputs), _vp, _vp, _vp]
 _lib.gdn_forward.restype = ctypes.c_int
+_lib.gdn_forward_timed.argtypes = [_vp, ctypes.POINTER(Inputs), _vp, _vp, _vp, ctypes.POINTER(_vp), ctypes.c_int]
+_lib.gdn_forward_timed.restype = ctypes.c_int
 _lib.gdn_forward_host.argtypes = [_vp, ctypes.POINTER(Inputs), _vp, _vp, _vp, _vp]
 _lib.gdn_forward_host.restype = ctypes.c_int
 _lib.gdn_staging_bytes.argtypes = [_vp]
@@ -59,6 +61,8 @@ _lib.gdn_launches_per_forward.argtypes = [_vp]
 _lib.gdn_launches_per_forward.restype = ctypes.c_int
 _lib.gdn_plan_uses_tensor_path.argtypes = [_vp]
 _lib.gdn_plan_uses_tensor_path.restype = ctypes.c_int
+_lib.gdn_plan_segments.argtypes = [_vp]
+_lib.gdn_plan_segments.restype = ctypes.c_int
 _lib.gdn_workspace_offsets.argtypes = [_vp, ctypes.POINTER(ctypes.c_size_t), ctypes.c_int]
 _lib.gdn_workspace_offsets.restype = ctypes.c_int
 _lib.gdn_destroy.argtypes = [_vp]
@@ -120,10 +124,21 @@ class Plan:
     def uses_tensor_path(self) -> bool:
         return bool(_lib.gdn_plan_uses_tensor_path(self._h))
 
+    @property
+    def segments(self) -> int:
+        return _lib.gdn_plan_segments(self._h)
+
     def forward_raw(self, ptrs: dict, y: int, workspace: int, stream: int) -> None:
         """gdn_forward with raw device addresses (ints)."""
         ins = Inputs(*[ptrs[n] for n, _ in Inputs._fields_])
         _check(_lib.gdn_forward(self._h, ctypes.byref(ins), y, workspace, stream), "gdn_forward")
+
+    def forward_timed_raw(self, ptrs: dict, y: int, workspace: int, stream: int, events: list) -> None:
+        """gdn_forward_timed: `events` are cudaEvent_t handles (ints), launches + 1 of them."""
+        ins = Inputs(*[ptrs[n] for n, _ in Inputs._fields_])
+        arr = (_vp * len(events))(*events)
+        _check(_lib.gdn_forward_timed(self._h, ctypes.byref(ins), y, workspace, stream, arr, len(events)),
+               "gdn_forward_timed")
 
     def forward_host_raw(self, ptrs: dict, y_host: int, staging: int, workspace: int, stream: int) -> None:
         """gdn_forward_host with raw host input addresses and device staging/workspace."""
@@ -131,11 +146,12 @@ class Plan:
         _check(_lib.gdn_forward_host(self._h, ctypes.byref(ins), y_host, staging, workspace, stream),
                "gdn_forward_host")
 
-    WS_FIELDS = ("status", "qh", "kh", "vh", "G", "beta", "log_alpha", "W", "U", "Qt", "Kt", "Aqk", "o")
+    WS_FIELDS = ("status", "qh", "kh", "vh", "G", "beta", "log_alpha", "W", "U", "Qt", "Kt", "Aqk", "o", "Zloc",
+                 "Sstart")
 
     def workspace_offsets(self) -> dict:
-        arr = (ctypes.c_size_t * 13)()
-        n = _lib.gdn_workspace_offsets(self._h, arr, 13)
+        arr = (ctypes.c_size_t * len(self.WS_FIELDS))()
+        n = _lib.gdn_workspace_offsets(self._h, arr, len(self.WS_FIELDS))
         return {self.WS_FIELDS[i]: arr[i] for i in range(n)}
 
     def device_status(self, workspace: int, stream: int) -> int:

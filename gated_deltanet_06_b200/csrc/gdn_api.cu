@@ -18,12 +18,12 @@ struct gdn_plan_s {
     gdn_config cfg;
     int device;
     bool tensor;
-    int Tp, NB;
+    int Tp, NB, NS, Ls;
     long long tok_stride;
     size_t in_esize, out_esize, inter_esize;
     // workspace layout
     size_t off_status, off_qh, off_kh, off_vh, off_G, off_beta, off_la;
-    size_t off_W, off_U, off_Qt, off_Kt, off_Aqk, off_o, ws_bytes;
+    size_t off_W, off_U, off_Qt, off_Kt, off_Aqk, off_Zloc, off_Sstart, off_o, ws_bytes;
     // staging layout (gdn_forward_host)
     size_t st_q, st_k, st_v, st_z, st_g, st_b, st_cq, st_ck, st_cv, st_A, st_dt, st_nw, st_y, staging_bytes;
 };
@@ -111,9 +111,10 @@ gdn_status gdn_plan(const gdn_config *cfg, gdn_plan_t *out, size_t *workspace_by
     const long long BH = static_cast<long long>(c.B) * c.H;
     if (BH * Tp >= (1ll << 31)) return GDN_ERR_UNSUPPORTED;  // TMA row coordinates are int32
 
-    int dev = -1, major = 0;
+    int dev = -1, major = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return GDN_ERR_NO_DEVICE; }
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess || major != 10) {
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess || major != 10 ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
         cudaGetLastError();
         return GDN_ERR_NO_DEVICE;
     }
@@ -126,6 +127,14 @@ gdn_status gdn_plan(const gdn_config *cfg, gdn_plan_t *out, size_t *workspace_by
     p->tensor = (c.in_dtype != GDN_DTYPE_F32) && d == 128 && !(c.flags & GDN_FLAG_FORCE_SIMT);
     p->Tp = static_cast<int>(Tp);
     p->NB = static_cast<int>(Tp / kBlk);
+    // segments: about one scan CTA per SM over all (b, h)
+    {
+        long long ns = sms / BH;
+        if (ns < 1) ns = 1;
+        if (ns > p->NB) ns = p->NB;
+        p->Ls = static_cast<int>((p->NB + ns - 1) / ns);
+        p->NS = (p->NB + p->Ls - 1) / p->Ls;
+    }
     p->tok_stride = ts;
     p->in_esize = esize(c.in_dtype);
     p->out_esize = esize(c.out_dtype);
@@ -148,8 +157,11 @@ gdn_status gdn_plan(const gdn_config *cfg, gdn_plan_t *out, size_t *workspace_by
         p->off_Qt = off; off = align_up(off + act * 2, A);
         p->off_Kt = off; off = align_up(off + act * 2, A);
         p->off_Aqk = off; off = align_up(off + act * 2, A);
+        p->off_Zloc = off; off = align_up(off + static_cast<size_t>(BH) * p->NS * 128 * 256 * 4, A);
+        p->off_Sstart = off; off = align_up(off + static_cast<size_t>(BH) * p->NS * 128 * 128 * 4, A);
+    } else {
+        p->off_o = off; off = align_up(off + static_cast<size_t>(c.B) * c.T * c.H * d * 4, A);
     }
-    p->off_o = off; off = align_up(off + static_cast<size_t>(c.B) * c.T * c.H * d * 4, A);
     p->ws_bytes = off;
 
     const size_t ntok_in = static_cast<size_t>(c.B) * c.T;
@@ -180,23 +192,30 @@ gdn_status gdn_destroy(gdn_plan_t plan) {
     return GDN_OK;
 }
 
-int gdn_launches_per_forward(gdn_plan_t plan) { return plan ? (plan->tensor ? 4 : 3) : 0; }
+int gdn_launches_per_forward(gdn_plan_t plan) {
+    if (!plan) return 0;
+    if (!plan->tensor) return 3;          // prep, recurrence, output
+    return plan->NS > 1 ? 5 : 3;          // prep, chunk, [transfer, combine,] scan+output
+}
 
 int gdn_plan_uses_tensor_path(gdn_plan_t plan) { return plan && plan->tensor ? 1 : 0; }
+
+int gdn_plan_segments(gdn_plan_t plan) { return plan && plan->tensor ? plan->NS : 0; }
 
 size_t gdn_staging_bytes(gdn_plan_t plan) { return plan ? plan->staging_bytes : 0; }
 
 int gdn_workspace_offsets(gdn_plan_t plan, size_t *offsets, int n) {
     if (!plan || !offsets || n <= 0) return 0;
-    const size_t all[13] = {plan->off_status, plan->off_qh, plan->off_kh, plan->off_vh, plan->off_G,
+    const size_t all[15] = {plan->off_status, plan->off_qh, plan->off_kh, plan->off_vh, plan->off_G,
                             plan->off_beta, plan->off_la, plan->off_W, plan->off_U, plan->off_Qt,
-                            plan->off_Kt, plan->off_Aqk, plan->off_o};
-    const int m = n < 13 ? n : 13;
+                            plan->off_Kt, plan->off_Aqk, plan->off_o, plan->off_Zloc, plan->off_Sstart};
+    const int m = n < 15 ? n : 15;
     for (int i = 0; i < m; ++i) offsets[i] = all[i];
     return m;
 }
 
-gdn_status gdn_forward(gdn_plan_t plan, const gdn_inputs *in, void *y, void *workspace, gdn_stream_t stream) {
+static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, void *workspace,
+                               gdn_stream_t stream, void *const *events) {
     if (!plan || !in || !y || !workspace) return GDN_ERR_INVALID_ARG;
     const gdn_config &c = plan->cfg;
     const void *ptrs16[] = {in->q, in->k, in->v, in->z, y};
@@ -222,6 +241,11 @@ gdn_status gdn_forward(gdn_plan_t plan, const gdn_inputs *in, void *y, void *wor
     const int d = c.d_k;
 
     if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return GDN_ERR_CUDA;
+    int ev = 0;
+    auto mark = [&]() -> bool {
+        if (!events) return true;
+        return cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[ev++]), s) == cudaSuccess;
+    };
 
     PrepParams pp;
     pp.q = in->q; pp.k = in->k; pp.v = in->v;
@@ -234,7 +258,7 @@ gdn_status gdn_forward(gdn_plan_t plan, const gdn_inputs *in, void *y, void *wor
     pp.B = c.B; pp.T = c.T; pp.H = c.H; pp.d = d; pp.Tp = plan->Tp;
     pp.l2_eps = c.l2_eps;
     pp.q_scale = 1.0f / sqrtf(static_cast<float>(d));
-    if (launch_prep(pp, in_type(c.in_dtype), plan->tensor, s) != cudaSuccess) return GDN_ERR_CUDA;
+    if (!mark() || launch_prep(pp, in_type(c.in_dtype), plan->tensor, s) != cudaSuccess) return GDN_ERR_CUDA;
 
     if (plan->tensor) {
         const unsigned long long rows = static_cast<unsigned long long>(c.B) * c.H * plan->Tp;
@@ -254,14 +278,26 @@ gdn_status gdn_forward(gdn_plan_t plan, const gdn_inputs *in, void *y, void *wor
         cp.BH = c.B * c.H; cp.Tp = plan->Tp; cp.NB = plan->NB;
         cp.status = status;
         cp.wait_limit_ns = kWaitLimitNs;
-        if (launch_chunk(cp, tmK, tmV, tmQ, s) != cudaSuccess) return GDN_ERR_CUDA;
+        if (!mark() || launch_chunk(cp, tmK, tmV, tmQ, s) != cudaSuccess) return GDN_ERR_CUDA;
         ScanParams sp;
-        sp.G = G; sp.o = o;
-        sp.B = c.B; sp.T = c.T; sp.H = c.H; sp.Tp = plan->Tp; sp.NB = plan->NB;
+        sp.G = G;
+        sp.Zloc = reinterpret_cast<float *>(ws + plan->off_Zloc);
+        sp.Sstart = reinterpret_cast<float *>(ws + plan->off_Sstart);
+        sp.z = in->z; sp.tok_stride = plan->tok_stride; sp.norm_w = in->norm_w; sp.y = y;
+        sp.out_kind = c.out_dtype == GDN_DTYPE_BF16 ? 0 : (c.out_dtype == GDN_DTYPE_F32 ? 1 : 2);
+        sp.eps = c.norm_eps;
+        sp.B = c.B; sp.T = c.T; sp.H = c.H; sp.Tp = plan->Tp; sp.NB = plan->NB; sp.NS = plan->NS; sp.Ls = plan->Ls;
         sp.status = status;
         sp.wait_limit_ns = kWaitLimitNs;
         sp.test_wait_timeout = (c.flags & GDN_FLAG_TEST_WAIT_TIMEOUT) ? 1 : 0;
-        if (launch_scan(sp, tmW, tmQt, tmKt, tmAqk, tmU, s) != cudaSuccess) return GDN_ERR_CUDA;
+        if (plan->NS > 1) {
+            if (!mark() || launch_transfer(sp, tmW, tmKt, tmU, s) != cudaSuccess) return GDN_ERR_CUDA;
+            if (!mark() || launch_combine(sp, s) != cudaSuccess) return GDN_ERR_CUDA;
+        }
+        if (!mark() || launch_scan_out(sp, in_type(c.in_dtype), tmW, tmQt, tmKt, tmAqk, tmU, s) != cudaSuccess)
+            return GDN_ERR_CUDA;
+        if (!mark()) return GDN_ERR_CUDA;
+        return GDN_OK;
     } else {
         RecurParams rp;
         rp.qh = reinterpret_cast<const float *>(ws + plan->off_qh);
@@ -269,14 +305,28 @@ gdn_status gdn_forward(gdn_plan_t plan, const gdn_inputs *in, void *y, void *wor
         rp.vh = reinterpret_cast<const float *>(ws + plan->off_vh);
         rp.log_alpha = la; rp.beta = beta; rp.o = o;
         rp.B = c.B; rp.T = c.T; rp.H = c.H; rp.d = d; rp.Tp = plan->Tp;
-        if (launch_recurrence(rp, s) != cudaSuccess) return GDN_ERR_CUDA;
+        if (!mark() || launch_recurrence(rp, s) != cudaSuccess) return GDN_ERR_CUDA;
     }
 
     OutParams op;
     op.o = o; op.z = in->z; op.tok_stride = plan->tok_stride; op.norm_w = in->norm_w; op.y = y;
     op.B = c.B; op.T = c.T; op.H = c.H; op.dv = c.d_v; op.eps = c.norm_eps;
-    if (launch_output(op, in_type(c.in_dtype), in_type(c.out_dtype), s) != cudaSuccess) return GDN_ERR_CUDA;
+    if (!mark() || launch_output(op, in_type(c.in_dtype), in_type(c.out_dtype), s) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (!mark()) return GDN_ERR_CUDA;
     return GDN_OK;
+}
+
+gdn_status gdn_forward(gdn_plan_t plan, const gdn_inputs *in, void *y, void *workspace, gdn_stream_t stream) {
+    return forward_impl(plan, in, y, workspace, stream, nullptr);
+}
+
+gdn_status gdn_forward_timed(gdn_plan_t plan, const gdn_inputs *in, void *y, void *workspace,
+                             gdn_stream_t stream, void *const *events, int n_events) {
+    if (!plan || !events || n_events != gdn_launches_per_forward(plan) + 1) return GDN_ERR_INVALID_ARG;
+    for (int i = 0; i < n_events; ++i)
+        if (!events[i]) return GDN_ERR_INVALID_ARG;
+    return forward_impl(plan, in, y, workspace, stream, events);
 }
 
 gdn_status gdn_forward_host(gdn_plan_t plan, const gdn_inputs *in_host, void *y_host, void *staging,

@@ -39,18 +39,29 @@ struct ChunkParams {
 cudaError_t launch_chunk(const ChunkParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
                          const CUtensorMap &tmQ, cudaStream_t s);
 
-// Inter-block state scan + block outputs on tensor cores (d = 128).
+// Inter-block state scan on tensor cores (d = 128), parallel over segments of
+// Ls blocks: pass A (transfer), combine, pass C (outputs + fused output step).
 struct ScanParams {
-    const float *G;  // [BH][Tp]
-    float *o;        // [B][T][H][128] fp32
-    int B, T, H, Tp, NB;
+    const float *G;          // [BH][Tp]
+    float *Zloc;             // [BH][NS][128][256]: S_loc^T | P^T per segment (pass A)
+    float *Sstart;           // [BH][NS][128][128]: S^T at each segment start (combine)
+    const void *z;           // [B][T][H][128], token stride tok_stride
+    long long tok_stride;
+    const float *norm_w;     // [128]
+    void *y;                 // [B][T][H][128]
+    int out_kind;            // 0 bf16, 1 f32, 2 f16
+    float eps;
+    int B, T, H, Tp, NB, NS, Ls;
     int *status;
     unsigned long long wait_limit_ns;
     int test_wait_timeout;
 };
-cudaError_t launch_scan(const ScanParams &p, const CUtensorMap &tmW, const CUtensorMap &tmQt,
-                        const CUtensorMap &tmKt, const CUtensorMap &tmAqk, const CUtensorMap &tmU,
-                        cudaStream_t s);
+cudaError_t launch_transfer(const ScanParams &p, const CUtensorMap &tmW, const CUtensorMap &tmKt,
+                            const CUtensorMap &tmU, cudaStream_t s);
+cudaError_t launch_combine(const ScanParams &p, cudaStream_t s);
+cudaError_t launch_scan_out(const ScanParams &p, InType zt, const CUtensorMap &tmW, const CUtensorMap &tmQt,
+                            const CUtensorMap &tmKt, const CUtensorMap &tmAqk, const CUtensorMap &tmU,
+                            cudaStream_t s);
 
 // Sequential fp32 recurrence on CUDA cores (fp32 inputs or d = 64).
 struct RecurParams {

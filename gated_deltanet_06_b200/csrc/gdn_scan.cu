@@ -1,20 +1,26 @@
-// gdn_scan.cu -- K3 of the GDN forward: the inter-block state scan of the
-// gated delta rule (reference [57] on the VMonarch page) and the block
-// outputs, on 5th-generation tensor cores.  One CTA carries the fp32 state
-// S (d_v x d_k = 128 x 128) of one (b, h) through its 128-token blocks:
+// gdn_scan.cu -- the inter-block part of the gated delta rule (reference [57]
+// on the VMonarch page) on 5th-generation tensor cores, parallel over
+// segments of the sequence, and the output step.
 //
-//   X     = W S^T                     (tcgen05, TMEM)
-//   Delta = U - X                     (consumer warps, fp32 -> fp16 operand)
-//   S^T  <- e^(G_last) S^T + Kt^T Delta   (tcgen05 for Kt^T Delta; the fp32
-//                                        state lives in the consumer threads'
-//                                        registers, one d_k row per thread)
-//   O     = Qt S^T + Aqk Delta        (tcgen05, accumulated in TMEM)
-//
-// with Kt = diag(e^(G_last - G)) K, Qt = diag(e^G) Q and Aqk the decay-masked
-// Q K^T from the chunk kernel.  Warp 4 is the producer: one lane issues the
-// TMA loads of the next block as soon as each tile's last reader has
-// finished, and issues every MMA.  Warps 0-3 are the consumers: thread r owns
-// TMEM lane r.  All hand-offs are mbarriers with bounded waits, so a lost
+// Per 128-token block c, with W, U, Kt = diag(e^(G_last - G)) K, Qt =
+// diag(e^G) Q and the decay-masked Aqk from the chunk kernel, the state moves
+//   Delta = U - W S^T,  S^T <- e^(G_last) S^T + Kt^T Delta,
+// and the block output is O = Qt S^T + Aqk Delta.  Substituting, S_end =
+// S_start P + S_loc for a run of blocks, with P = prod_c (e^(G_last) I - W^T Kt)
+// and S_loc the end state from S_start = 0.  So the sequence is cut into
+// segments processed in parallel:
+//   pass A  (gdn_transfer_kernel): per segment, run the state and the
+//           transfer together as one 256-column state [S^T | P^T] from
+//           [0 | I]; write both (fp32).
+//   combine (gdn_combine_kernel): S_start(j+1)^T = P_j^T S_start(j)^T + S_loc(j)^T,
+//           sequential over segments, fp32 on CUDA cores.
+//   pass C  (gdn_scan_out_kernel): per segment, run the state from S_start and
+//           emit the block outputs, with the output step fused into the
+//           epilogue:  y = o / sqrt(mean(o^2) + eps) * w * SiLU(z).
+// In both tensor-core kernels a producer warp issues the TMA loads of the next
+// block as soon as each tile's last reader has finished, and all MMAs;
+// consumer warps own TMEM lanes (one row each) and keep the fp32 state in
+// registers.  Every hand-off is an mbarrier with a bounded wait, so a lost
 // arrival ends the kernel with a timeout status instead of a hang.
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
@@ -22,25 +28,37 @@
 namespace gdn {
 namespace {
 
-constexpr uint32_t OFF_W = 0;
-constexpr uint32_t OFF_QT = 32768;
-constexpr uint32_t OFF_KT = 65536;
-constexpr uint32_t OFF_AQK = 98304;
-constexpr uint32_t OFF_U = 131072;
-constexpr uint32_t OFF_S = 163840;   // S^T as fp16 MN-major B operand (rows d_k, cols d_v)
-constexpr uint32_t OFF_D = 196608;   // Delta as fp16 MN-major B operand (rows token, cols d_v)
+__device__ __forceinline__ void store_f16_chunk(uint8_t *tile, int rows, int r, int chunk16, const float *v) {
+    uint4 u;
+    u.x = pack_half2(v[0], v[1]);
+    u.y = pack_half2(v[2], v[3]);
+    u.z = pack_half2(v[4], v[5]);
+    u.w = pack_half2(v[6], v[7]);
+    *reinterpret_cast<uint4 *>(tile + tile_off(rows, r, chunk16)) = u;
+}
+
+// Warp-uniform bounded wait (every lane waits; the warp proceeds only if all did).
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t ph, volatile AbortState *ab, int *status,
+                                          uint64_t lim) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, ph, ab, status, lim));
+}
+
+// ============================================================ pass A
+namespace ta {
+constexpr uint32_t OFF_W = 0, OFF_KT = 32768, OFF_U = 65536;
+constexpr uint32_t OFF_Z = 98304;    // [S^T | P^T] fp16, 128 rows (d_k) x 256, MN-major B (4 panels)
+constexpr uint32_t OFF_D = 163840;   // Delta fp16, 128 rows (token) x 256, MN-major B
 constexpr uint32_t OFF_BAR = 229376;
-constexpr int NBAR = 11;
-constexpr uint32_t SMEM_USED = OFF_BAR + NBAR * 8 + 16;
-constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
+constexpr int NBAR = 7;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
+enum { FULL_W = 0, FULL_U, FULL_K, MMA_X, MMA_P, CONS_D, CONS_S };
+constexpr uint32_t TM_X = 0, TM_P = 256;
+}  // namespace ta
 
-enum { B_FULL_WQ = 0, B_FULL_U, B_FULL_KA, B_MMA_X, B_MMA_P, B_MMA_O, B_CONS_D, B_CONS_S, B_CONS_O0, B_CONS_O1, B_TEST };
-constexpr uint32_t TM_X = 0, TM_P = 128, TM_O = 256;  // O double-buffered: 256 and 384
-
-__global__ void __launch_bounds__(160, 1)
-    gdn_scan_kernel(const ScanParams p, const __grid_constant__ CUtensorMap tmW,
-                    const __grid_constant__ CUtensorMap tmQt, const __grid_constant__ CUtensorMap tmKt,
-                    const __grid_constant__ CUtensorMap tmAqk, const __grid_constant__ CUtensorMap tmU) {
+__global__ void __launch_bounds__(288, 1)
+    gdn_transfer_kernel(const ScanParams p, const __grid_constant__ CUtensorMap tmW,
+                        const __grid_constant__ CUtensorMap tmKt, const __grid_constant__ CUtensorMap tmU) {
+    using namespace ta;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
@@ -48,14 +66,264 @@ __global__ void __launch_bounds__(160, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NBAR);
     AbortState *ab = reinterpret_cast<AbortState *>(tmem_slot + 1);
 
-    const int h = blockIdx.x, b = blockIdx.y;
+    const int seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int bh = b * p.H + h;
+    const int c0 = seg * p.Ls, c1 = min(c0 + p.Ls, p.NB);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int NB = p.NB;
     const uint64_t lim = p.wait_limit_ns;
 
     if (tid == 0) {
-        for (int i = 0; i < NBAR; ++i) mbar_init(&bars[i], (i >= B_CONS_D && i <= B_CONS_O1) ? 4 : 1);
+        for (int i = 0; i < NBAR; ++i) mbar_init(&bars[i], (i == CONS_D || i == CONS_S) ? 8 : 1);
+        ab->flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 8) {
+        if (lane == 0) {
+            const int rowbase = bh * p.Tp;
+            auto load2 = [&](uint32_t off, const CUtensorMap *m, uint64_t *bar, int c) {
+                mbar_arrive_expect_tx(bar, 32768);
+                tma_load_2d(sm + off, m, bar, 0, rowbase + c * kBlk);
+                tma_load_2d(sm + off + 16384, m, bar, 64, rowbase + c * kBlk);
+            };
+            load2(OFF_W, &tmW, &bars[FULL_W], c0);
+            load2(OFF_U, &tmU, &bars[FULL_U], c0);
+            load2(OFF_KT, &tmKt, &bars[FULL_K], c0);
+            const uint32_t id_x = idesc_f16_f32(128, 256, false, true);
+            const uint32_t id_p = idesc_f16_f32(128, 256, true, true);
+            bool ok = true;
+            for (int c = c0; ok && c < c1; ++c) {
+                const uint32_t ph = (c - c0) & 1;
+                ok = mbar_wait(&bars[FULL_W], ph, ab, p.status, lim) && mbar_wait(&bars[CONS_S], ph, ab, p.status, lim);
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_f16(tmem + TM_X, sdesc_sw128(sbase + OFF_W + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                             sdesc_sw128(sbase + OFF_Z + kk * 2048, 16384, 1024), id_x, kk > 0);
+                umma_commit(&bars[MMA_X]);
+                ok = mbar_wait(&bars[MMA_X], ph, ab, p.status, lim);
+                if (!ok) break;
+                if (c + 1 < c1) load2(OFF_W, &tmW, &bars[FULL_W], c + 1);
+                ok = mbar_wait(&bars[FULL_K], ph, ab, p.status, lim) && mbar_wait(&bars[CONS_D], ph, ab, p.status, lim);
+                if (!ok) break;
+                if (c + 1 < c1) load2(OFF_U, &tmU, &bars[FULL_U], c + 1);
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_f16(tmem + TM_P, sdesc_sw128(sbase + OFF_KT + kk * 2048, 16384, 1024),
+                             sdesc_sw128(sbase + OFF_D + kk * 2048, 16384, 1024), id_p, kk > 0);
+                umma_commit(&bars[MMA_P]);
+                ok = mbar_wait(&bars[MMA_P], ph, ab, p.status, lim);
+                if (!ok) break;
+                if (c + 1 < c1) load2(OFF_KT, &tmKt, &bars[FULL_K], c + 1);
+            }
+        }
+    } else {
+        const int q = warp & 3, half = warp >> 2;  // half 0: S^T columns, half 1: P^T columns
+        const int r = q * 32 + lane;
+        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+        float Z[128];
+#pragma unroll
+        for (int i = 0; i < 128; ++i) Z[i] = (half == 1 && i == r) ? 1.0f : 0.0f;
+#pragma unroll
+        for (int c8 = 0; c8 < 16; ++c8) store_f16_chunk(sm + OFF_Z, 128, r, half * 16 + c8, &Z[c8 * 8]);
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[CONS_S]);
+        const float *Gbh = p.G + static_cast<size_t>(bh) * p.Tp;
+        bool ok = true;
+        for (int c = c0; c < c1; ++c) {
+            const uint32_t ph = (c - c0) & 1;
+            const float gC = __expf(fminf(Gbh[c * kBlk + kBlk - 1], 0.0f));
+            ok = warp_wait(&bars[MMA_X], ph, ab, p.status, lim) && warp_wait(&bars[FULL_U], ph, ab, p.status, lim);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                float x[32];
+                tmem_ld32(tmem + lane_base + TM_X + half * 128 + ch * 32, x);
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    float dlt[8];
+                    if (half == 0) {
+                        const uint4 uu = *reinterpret_cast<const uint4 *>(sm + OFF_U + tile_off(128, r, ch * 4 + qq));
+                        const uint32_t w4[4] = {uu.x, uu.y, uu.z, uu.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 u2 = unpack_half2(w4[e]);
+                            dlt[2 * e] = u2.x - x[qq * 8 + 2 * e];
+                            dlt[2 * e + 1] = u2.y - x[qq * 8 + 2 * e + 1];
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) dlt[e] = -x[qq * 8 + e];
+                    }
+                    store_f16_chunk(sm + OFF_D, 128, r, half * 16 + ch * 4 + qq, dlt);
+                }
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[CONS_D]);
+            ok = warp_wait(&bars[MMA_P], ph, ab, p.status, lim);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                float pv[32];
+                tmem_ld32(tmem + lane_base + TM_P + half * 128 + ch * 32, pv);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) Z[ch * 32 + i] = fmaf(gC, Z[ch * 32 + i], pv[i]);
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq)
+                    store_f16_chunk(sm + OFF_Z, 128, r, half * 16 + ch * 4 + qq, &Z[ch * 32 + qq * 8]);
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[CONS_S]);
+        }
+        if (ok) {
+            float *dst = p.Zloc + ((static_cast<size_t>(bh) * p.NS + seg) * 128 + r) * 256 + half * 128;
+#pragma unroll
+            for (int i = 0; i < 128; i += 4) *reinterpret_cast<float4 *>(dst + i) = make_float4(Z[i], Z[i + 1], Z[i + 2], Z[i + 3]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// ============================================================ combine
+// S_start(j+1)^T = P_j^T S_start(j)^T + S_loc(j)^T, sequential over j; one CTA
+// per (8-column slice of S^T, head); thread t owns row t of the slice.
+__global__ void __launch_bounds__(128) gdn_combine_kernel(const ScanParams p) {
+    __shared__ float cur[128][8];
+    const int slice = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int bh = b * p.H + h;
+    const int t = threadIdx.x;
+    const int c0 = slice * 8;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) cur[t][c] = 0.0f;
+    __syncthreads();
+    for (int j = 0; j + 1 < p.NS; ++j) {
+        const float *zrow = p.Zloc + ((static_cast<size_t>(bh) * p.NS + j) * 128 + t) * 256;
+        float acc[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[c] = zrow[c0 + c];  // S_loc^T
+        const float *prow = zrow + 128;                       // P^T row t
+#pragma unroll 4
+        for (int i = 0; i < 128; i += 4) {
+            const float4 pv = *reinterpret_cast<const float4 *>(prow + i);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                acc[c] = fmaf(pv.x, cur[i][c], acc[c]);
+                acc[c] = fmaf(pv.y, cur[i + 1][c], acc[c]);
+                acc[c] = fmaf(pv.z, cur[i + 2][c], acc[c]);
+                acc[c] = fmaf(pv.w, cur[i + 3][c], acc[c]);
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int c = 0; c < 8; ++c) cur[t][c] = acc[c];
+        float *dst = p.Sstart + ((static_cast<size_t>(bh) * p.NS + j + 1) * 128 + t) * 128 + c0;
+        *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4 *>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        __syncthreads();
+    }
+}
+
+// ============================================================ pass C
+namespace tc {
+constexpr uint32_t OFF_W = 0, OFF_QT = 32768, OFF_KT = 65536, OFF_AQK = 98304, OFF_U = 131072;
+constexpr uint32_t OFF_S = 163840;  // S^T fp16 MN-major B operand (rows d_k, cols d_v)
+constexpr uint32_t OFF_D = 196608;  // Delta fp16 MN-major B operand (rows token, cols d_v)
+constexpr uint32_t OFF_BAR = 229376;
+constexpr int NBAR = 11;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
+enum { FULL_WQ = 0, FULL_U, FULL_KA, MMA_X, MMA_P, MMA_O, CONS_D, CONS_S, CONS_O0, CONS_O1, TEST };
+constexpr uint32_t TM_X = 0, TM_P = 128, TM_O = 256;  // O double-buffered: 256 and 384
+}  // namespace tc
+
+template <typename ZT, typename YT>
+__device__ __forceinline__ void load8(const ZT *p, float (&f)[8]);
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16, float>(const __nv_bfloat16 *p, float (&f)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i]));
+        f[2 * i] = x.x;
+        f[2 * i + 1] = x.y;
+    }
+}
+template <>
+__device__ __forceinline__ void load8<__half, float>(const __half *p, float (&f)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 x = unpack_half2(w[i]);
+        f[2 * i] = x.x;
+        f[2 * i + 1] = x.y;
+    }
+}
+
+__device__ __forceinline__ void store_y8(void *y, int out_kind, size_t idx, const float *v) {
+    if (out_kind == 0) {  // bf16
+        uint4 u;
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+            w[i] = *reinterpret_cast<uint32_t *>(&b2);
+        }
+        u.x = w[0]; u.y = w[1]; u.z = w[2]; u.w = w[3];
+        *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(y) + idx) = u;
+    } else if (out_kind == 2) {  // f16
+        uint4 u;
+        u.x = pack_half2(v[0], v[1]); u.y = pack_half2(v[2], v[3]);
+        u.z = pack_half2(v[4], v[5]); u.w = pack_half2(v[6], v[7]);
+        *reinterpret_cast<uint4 *>(static_cast<__half *>(y) + idx) = u;
+    } else {
+        float *d = static_cast<float *>(y) + idx;
+        *reinterpret_cast<float4 *>(d) = make_float4(v[0], v[1], v[2], v[3]);
+        *reinterpret_cast<float4 *>(d + 4) = make_float4(v[4], v[5], v[6], v[7]);
+    }
+}
+
+template <typename ZT>
+__global__ void __launch_bounds__(160, 1)
+    gdn_scan_out_kernel(const ScanParams p, const __grid_constant__ CUtensorMap tmW,
+                        const __grid_constant__ CUtensorMap tmQt, const __grid_constant__ CUtensorMap tmKt,
+                        const __grid_constant__ CUtensorMap tmAqk, const __grid_constant__ CUtensorMap tmU) {
+    using namespace tc;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NBAR);
+    AbortState *ab = reinterpret_cast<AbortState *>(tmem_slot + 1);
+
+    const int seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int bh = b * p.H + h;
+    const int c0 = seg * p.Ls, c1 = min(c0 + p.Ls, p.NB);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint64_t lim = p.wait_limit_ns;
+
+    if (tid == 0) {
+        for (int i = 0; i < NBAR; ++i) mbar_init(&bars[i], (i >= CONS_D && i <= CONS_O1) ? 4 : 1);
         ab->flag = 0;
         fence_mbar_init();
     }
@@ -72,43 +340,45 @@ __global__ void __launch_bounds__(160, 1)
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             bool ok = true;
-            if (p.test_wait_timeout) ok = mbar_wait(&bars[B_TEST], 0, ab, p.status, 50ull * 1000 * 1000);
+            if (p.test_wait_timeout) {
+                // test hook: wait on a barrier nothing arrives on (bounded, ~50 ms), before anything is in
+                // flight; the wait sets the timeout status and the abort flag, and every thread exits
+                mbar_wait(&bars[TEST], 0, ab, p.status, 50ull * 1000 * 1000);
+                ok = false;
+            }
             const int rowbase = bh * p.Tp;
+            auto load2 = [&](uint32_t off, const CUtensorMap *m, uint64_t *bar, int c) {
+                tma_load_2d(sm + off, m, bar, 0, rowbase + c * kBlk);
+                tma_load_2d(sm + off + 16384, m, bar, 64, rowbase + c * kBlk);
+            };
             auto load_wq = [&](int c) {
-                mbar_arrive_expect_tx(&bars[B_FULL_WQ], 65536);
-                const int y = rowbase + c * kBlk;
-                tma_load_2d(sm + OFF_W, &tmW, &bars[B_FULL_WQ], 0, y);
-                tma_load_2d(sm + OFF_W + 16384, &tmW, &bars[B_FULL_WQ], 64, y);
-                tma_load_2d(sm + OFF_QT, &tmQt, &bars[B_FULL_WQ], 0, y);
-                tma_load_2d(sm + OFF_QT + 16384, &tmQt, &bars[B_FULL_WQ], 64, y);
+                mbar_arrive_expect_tx(&bars[FULL_WQ], 65536);
+                load2(OFF_W, &tmW, &bars[FULL_WQ], c);
+                load2(OFF_QT, &tmQt, &bars[FULL_WQ], c);
             };
             auto load_u = [&](int c) {
-                mbar_arrive_expect_tx(&bars[B_FULL_U], 32768);
-                const int y = rowbase + c * kBlk;
-                tma_load_2d(sm + OFF_U, &tmU, &bars[B_FULL_U], 0, y);
-                tma_load_2d(sm + OFF_U + 16384, &tmU, &bars[B_FULL_U], 64, y);
+                mbar_arrive_expect_tx(&bars[FULL_U], 32768);
+                load2(OFF_U, &tmU, &bars[FULL_U], c);
             };
             auto load_ka = [&](int c) {
-                mbar_arrive_expect_tx(&bars[B_FULL_KA], 65536);
-                const int y = rowbase + c * kBlk;
-                tma_load_2d(sm + OFF_KT, &tmKt, &bars[B_FULL_KA], 0, y);
-                tma_load_2d(sm + OFF_KT + 16384, &tmKt, &bars[B_FULL_KA], 64, y);
-                tma_load_2d(sm + OFF_AQK, &tmAqk, &bars[B_FULL_KA], 0, y);
-                tma_load_2d(sm + OFF_AQK + 16384, &tmAqk, &bars[B_FULL_KA], 64, y);
+                mbar_arrive_expect_tx(&bars[FULL_KA], 65536);
+                load2(OFF_KT, &tmKt, &bars[FULL_KA], c);
+                load2(OFF_AQK, &tmAqk, &bars[FULL_KA], c);
             };
             if (ok) {
-                load_wq(0);
-                load_u(0);
-                load_ka(0);
+                load_wq(c0);
+                load_u(c0);
+                load_ka(c0);
             }
             const uint32_t id_kmn = idesc_f16_f32(128, 128, false, true);
             const uint32_t id_mnmn = idesc_f16_f32(128, 128, true, true);
-            for (int c = 0; ok && c < NB; ++c) {
-                const uint32_t ph = c & 1;
-                const uint32_t tO = tmem + TM_O + (c & 1) * 128;
-                ok = mbar_wait(&bars[B_FULL_WQ], ph, ab, p.status, lim) &&
-                     mbar_wait(&bars[B_CONS_S], ph, ab, p.status, lim) &&
-                     (c < 2 || mbar_wait(&bars[B_CONS_O0 + (c & 1)], ((c >> 1) - 1) & 1, ab, p.status, lim));
+            for (int c = c0; ok && c < c1; ++c) {
+                const int i = c - c0;
+                const uint32_t ph = i & 1;
+                const uint32_t tO = tmem + TM_O + (i & 1) * 128;
+                ok = mbar_wait(&bars[FULL_WQ], ph, ab, p.status, lim) &&
+                     mbar_wait(&bars[CONS_S], ph, ab, p.status, lim) &&
+                     (i < 2 || mbar_wait(&bars[CONS_O0 + (i & 1)], ((i >> 1) - 1) & 1, ab, p.status, lim));
                 if (!ok) break;
                 tc_fence_after();
                 // X = W S^T ; O = Qt S^T   (A K-major, B = S^T MN-major)
@@ -119,21 +389,21 @@ __global__ void __launch_bounds__(160, 1)
                     umma_f16(tmem + TM_X, sdesc_sw128(sbase + OFF_W + aoff, 16, 1024), bd, id_kmn, kk > 0);
                     umma_f16(tO, sdesc_sw128(sbase + OFF_QT + aoff, 16, 1024), bd, id_kmn, kk > 0);
                 }
-                umma_commit(&bars[B_MMA_X]);
-                ok = mbar_wait(&bars[B_MMA_X], ph, ab, p.status, lim);
+                umma_commit(&bars[MMA_X]);
+                ok = mbar_wait(&bars[MMA_X], ph, ab, p.status, lim);
                 if (!ok) break;
-                if (c + 1 < NB) load_wq(c + 1);
-                ok = mbar_wait(&bars[B_FULL_KA], ph, ab, p.status, lim) &&
-                     mbar_wait(&bars[B_CONS_D], ph, ab, p.status, lim);
+                if (c + 1 < c1) load_wq(c + 1);
+                ok = mbar_wait(&bars[FULL_KA], ph, ab, p.status, lim) &&
+                     mbar_wait(&bars[CONS_D], ph, ab, p.status, lim);
                 if (!ok) break;
-                if (c + 1 < NB) load_u(c + 1);
+                if (c + 1 < c1) load_u(c + 1);
                 tc_fence_after();
                 // P = Kt^T Delta  (A = Kt read MN-major: M = d_k, K = token; B = Delta MN-major)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     umma_f16(tmem + TM_P, sdesc_sw128(sbase + OFF_KT + kk * 2048, 16384, 1024),
                              sdesc_sw128(sbase + OFF_D + kk * 2048, 16384, 1024), id_mnmn, kk > 0);
-                umma_commit(&bars[B_MMA_P]);
+                umma_commit(&bars[MMA_P]);
                 // O += Aqk Delta  (A K-major: M = token r, K = token i)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -141,10 +411,10 @@ __global__ void __launch_bounds__(160, 1)
                     umma_f16(tO, sdesc_sw128(sbase + OFF_AQK + aoff, 16, 1024),
                              sdesc_sw128(sbase + OFF_D + kk * 2048, 16384, 1024), id_kmn, 1);
                 }
-                umma_commit(&bars[B_MMA_O]);
-                ok = mbar_wait(&bars[B_MMA_O], ph, ab, p.status, lim);
+                umma_commit(&bars[MMA_O]);
+                ok = mbar_wait(&bars[MMA_O], ph, ab, p.status, lim);
                 if (!ok) break;
-                if (c + 1 < NB) load_ka(c + 1);
+                if (c + 1 < c1) load_ka(c + 1);
             }
         }
     } else {
@@ -152,22 +422,30 @@ __global__ void __launch_bounds__(160, 1)
         const int r = tid;  // TMEM lane: token row (X, O) or d_k row (P)
         const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
         float S[128];  // row r of S^T (= column r of S), fp32
+        if (seg == 0) {
 #pragma unroll
-        for (int i = 0; i < 128; ++i) S[i] = 0.0f;
+            for (int i = 0; i < 128; ++i) S[i] = 0.0f;
+        } else {
+            const float *src = p.Sstart + ((static_cast<size_t>(bh) * p.NS + seg) * 128 + r) * 128;
 #pragma unroll
-        for (int c16 = 0; c16 < 16; ++c16)
-            *reinterpret_cast<uint4 *>(sm + OFF_S + tile_off(128, r, c16)) = make_uint4(0, 0, 0, 0);
+            for (int i = 0; i < 128; i += 4) {
+                const float4 v = *reinterpret_cast<const float4 *>(src + i);
+                S[i] = v.x; S[i + 1] = v.y; S[i + 2] = v.z; S[i + 3] = v.w;
+            }
+        }
+#pragma unroll
+        for (int c8 = 0; c8 < 16; ++c8) store_f16_chunk(sm + OFF_S, 128, r, c8, &S[c8 * 8]);
         fence_proxy_async();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[B_CONS_S]);
+        if (lane == 0) mbar_arrive(&bars[CONS_S]);
 
         const float *Gbh = p.G + static_cast<size_t>(bh) * p.Tp;
-        for (int c = 0; c < NB; ++c) {
-            const uint32_t ph = c & 1;
+        const ZT *z = static_cast<const ZT *>(p.z);
+        for (int c = c0; c < c1; ++c) {
+            const int i = c - c0;
+            const uint32_t ph = i & 1;
             const float gC = __expf(fminf(Gbh[c * kBlk + kBlk - 1], 0.0f));
-            // every wait below is made warp-uniform before the .sync.aligned TMEM loads
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_MMA_X], ph, ab, p.status, lim) &&
-                                             mbar_wait(&bars[B_FULL_U], ph, ab, p.status, lim)))
+            if (!(warp_wait(&bars[MMA_X], ph, ab, p.status, lim) && warp_wait(&bars[FULL_U], ph, ab, p.status, lim)))
                 break;
             tc_fence_after();
             // Delta = U - X, row r
@@ -176,67 +454,77 @@ __global__ void __launch_bounds__(160, 1)
                 float x[32];
                 tmem_ld32(tmem + lane_base + TM_X + ch * 32, x);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t off = tile_off(128, r, ch * 4 + q);
-                    const uint4 uu = *reinterpret_cast<const uint4 *>(sm + OFF_U + off);
-                    const uint32_t w[4] = {uu.x, uu.y, uu.z, uu.w};
-                    uint32_t o[4];
+                for (int qq = 0; qq < 4; ++qq) {
+                    const uint4 uu = *reinterpret_cast<const uint4 *>(sm + OFF_U + tile_off(128, r, ch * 4 + qq));
+                    const uint32_t w4[4] = {uu.x, uu.y, uu.z, uu.w};
+                    float dlt[8];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float2 u2 = unpack_half2(w[e]);
-                        o[e] = pack_half2(u2.x - x[q * 8 + 2 * e], u2.y - x[q * 8 + 2 * e + 1]);
+                        const float2 u2 = unpack_half2(w4[e]);
+                        dlt[2 * e] = u2.x - x[qq * 8 + 2 * e];
+                        dlt[2 * e + 1] = u2.y - x[qq * 8 + 2 * e + 1];
                     }
-                    *reinterpret_cast<uint4 *>(sm + OFF_D + off) = make_uint4(o[0], o[1], o[2], o[3]);
+                    store_f16_chunk(sm + OFF_D, 128, r, ch * 4 + qq, dlt);
                 }
             }
             fence_proxy_async();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[B_CONS_D]);
+            if (lane == 0) mbar_arrive(&bars[CONS_D]);
 
             // S^T row r <- gC * S^T row r + P row r
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_MMA_P], ph, ab, p.status, lim))) break;
+            if (!warp_wait(&bars[MMA_P], ph, ab, p.status, lim)) break;
             tc_fence_after();
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
                 float pv[32];
                 tmem_ld32(tmem + lane_base + TM_P + ch * 32, pv);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) S[ch * 32 + i] = fmaf(gC, S[ch * 32 + i], pv[i]);
+                for (int e = 0; e < 32; ++e) S[ch * 32 + e] = fmaf(gC, S[ch * 32 + e], pv[e]);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int e0 = ch * 32 + q * 8;
-                    uint4 u;
-                    u.x = pack_half2(S[e0 + 0], S[e0 + 1]);
-                    u.y = pack_half2(S[e0 + 2], S[e0 + 3]);
-                    u.z = pack_half2(S[e0 + 4], S[e0 + 5]);
-                    u.w = pack_half2(S[e0 + 6], S[e0 + 7]);
-                    *reinterpret_cast<uint4 *>(sm + OFF_S + tile_off(128, r, ch * 4 + q)) = u;
-                }
+                for (int qq = 0; qq < 4; ++qq) store_f16_chunk(sm + OFF_S, 128, r, ch * 4 + qq, &S[ch * 32 + qq * 8]);
             }
             fence_proxy_async();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[B_CONS_S]);
+            if (lane == 0) mbar_arrive(&bars[CONS_S]);
 
-            // block output rows
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_MMA_O], ph, ab, p.status, lim))) break;
+            // output step: y = o / sqrt(mean(o^2) + eps) * w * SiLU(z)
+            if (!warp_wait(&bars[MMA_O], ph, ab, p.status, lim)) break;
             tc_fence_after();
-            const int t = c * kBlk + r;
-            float *orow = p.o + ((static_cast<size_t>(b) * p.T + t) * p.H + h) * kD;
+            const uint32_t tO = tmem + lane_base + TM_O + (i & 1) * 128;
+            float ss = 0.0f;
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
                 float ov[32];
-                tmem_ld32(tmem + lane_base + TM_O + (c & 1) * 128 + ch * 32, ov);
-                if (t < p.T) {
+                tmem_ld32(tO + ch * 32, ov);
 #pragma unroll
-                    for (int i = 0; i < 32; i += 4)
-                        *reinterpret_cast<float4 *>(orow + ch * 32 + i) = make_float4(ov[i], ov[i + 1], ov[i + 2], ov[i + 3]);
+                for (int e = 0; e < 32; ++e) ss = fmaf(ov[e], ov[e], ss);
+            }
+            const float rn = 1.0f / sqrtf(ss * (1.0f / 128.0f) + p.eps);
+            const int t = c * kBlk + r;
+            const bool live = t < p.T;
+            const size_t zrow = (static_cast<size_t>(b) * p.T + (live ? t : 0)) * p.tok_stride + static_cast<size_t>(h) * kD;
+            const size_t yrow = ((static_cast<size_t>(b) * p.T + (live ? t : 0)) * p.H + h) * kD;
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                float ov[32];
+                tmem_ld32(tO + ch * 32, ov);
+                if (live) {
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq) {
+                        const int col = ch * 32 + qq * 8;
+                        float zf[8], yv[8];
+                        load8<ZT, float>(z + zrow + col, zf);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) yv[e] = ov[qq * 8 + e] * rn * p.norm_w[col + e] * silu_f(zf[e]);
+                        store_y8(p.y, p.out_kind, yrow + col, yv);
+                    }
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[B_CONS_O0 + (c & 1)]);
+            if (lane == 0) mbar_arrive(&bars[CONS_O0 + (i & 1)]);
         }
     }
 
@@ -246,20 +534,47 @@ __global__ void __launch_bounds__(160, 1)
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
+template <typename K>
+cudaError_t set_smem(K kernel, uint32_t bytes, bool &done) {
+    if (done) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+    if (e == cudaSuccess) done = true;
+    return e;
+}
+
 }  // namespace
 
-cudaError_t launch_scan(const ScanParams &p, const CUtensorMap &tmW, const CUtensorMap &tmQt,
-                        const CUtensorMap &tmKt, const CUtensorMap &tmAqk, const CUtensorMap &tmU,
-                        cudaStream_t s) {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gdn_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(SMEM_BYTES));
+cudaError_t launch_transfer(const ScanParams &p, const CUtensorMap &tmW, const CUtensorMap &tmKt,
+                            const CUtensorMap &tmU, cudaStream_t s) {
+    static bool attr = false;
+    cudaError_t e = set_smem(gdn_transfer_kernel, ta::SMEM_BYTES, attr);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.NS - 1, p.H, p.B);
+    gdn_transfer_kernel<<<grid, 288, ta::SMEM_BYTES, s>>>(p, tmW, tmKt, tmU);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const ScanParams &p, cudaStream_t s) {
+    dim3 grid(16, p.H, p.B);
+    gdn_combine_kernel<<<grid, 128, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scan_out(const ScanParams &p, InType zt, const CUtensorMap &tmW, const CUtensorMap &tmQt,
+                            const CUtensorMap &tmKt, const CUtensorMap &tmAqk, const CUtensorMap &tmU,
+                            cudaStream_t s) {
+    dim3 grid(p.NS, p.H, p.B);
+    if (zt == InType::F16) {
+        static bool attr = false;
+        cudaError_t e = set_smem(gdn_scan_out_kernel<__half>, tc::SMEM_BYTES, attr);
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        gdn_scan_out_kernel<__half><<<grid, 160, tc::SMEM_BYTES, s>>>(p, tmW, tmQt, tmKt, tmAqk, tmU);
+    } else {
+        static bool attr = false;
+        cudaError_t e = set_smem(gdn_scan_out_kernel<__nv_bfloat16>, tc::SMEM_BYTES, attr);
+        if (e != cudaSuccess) return e;
+        gdn_scan_out_kernel<__nv_bfloat16><<<grid, 160, tc::SMEM_BYTES, s>>>(p, tmW, tmQt, tmKt, tmAqk, tmU);
     }
-    dim3 grid(p.H, p.B);
-    gdn_scan_kernel<<<grid, 160, SMEM_BYTES, s>>>(p, tmW, tmQt, tmKt, tmAqk, tmU);
     return cudaGetLastError();
 }
 

@@ -118,6 +118,13 @@ gdn_status gdn_plan(const gdn_config *cfg, gdn_plan_t *out, size_t *workspace_by
 gdn_status gdn_forward(gdn_plan_t plan, const gdn_inputs *in, void *y, void *workspace,
                        gdn_stream_t stream);
 
+/* gdn_forward with per-kernel timing: events[i] (a cudaEvent_t the caller
+ * created) is recorded on `stream` just before the i-th kernel launch and
+ * events[L] after the last one, L = gdn_launches_per_forward(plan);
+ * n_events must be L + 1.  Same arguments, errors and result as gdn_forward. */
+gdn_status gdn_forward_timed(gdn_plan_t plan, const gdn_inputs *in, void *y, void *workspace,
+                             gdn_stream_t stream, void *const *events, int n_events);
+
 /* Bytes of device staging memory gdn_forward_host needs (inputs + output). */
 size_t gdn_staging_bytes(gdn_plan_t plan);
 
@@ -134,11 +141,17 @@ gdn_status gdn_forward_host(gdn_plan_t plan, const gdn_inputs *in_host, void *y_
  * GDN_ERR_CUDA if the synchronisation itself failed). */
 gdn_status gdn_get_device_status(gdn_plan_t plan, void *workspace, gdn_stream_t stream);
 
-/* Number of kernel launches one gdn_forward enqueues for this plan. */
+/* Number of kernel launches one gdn_forward enqueues for this plan: 3 or 5 on
+ * the tensor path (prep, UT transform, [segment transfer, combine,] scan with
+ * the output step), 3 on the CUDA-core path (prep, recurrence, output). */
 int gdn_launches_per_forward(gdn_plan_t plan);
 
 /* 1 if the plan runs the tensor-core (tcgen05) path, 0 for the fp32 CUDA-core path. */
 int gdn_plan_uses_tensor_path(gdn_plan_t plan);
+
+/* Number of sequence segments the tensor path scans in parallel for each
+ * (b, h) (about one scan CTA per SM over all heads); 0 on the CUDA-core path. */
+int gdn_plan_segments(gdn_plan_t plan);
 
 /* Introspection for per-stage tests: writes up to n byte offsets, inside the
  * workspace, of the intermediates of the last forward, in this order:
@@ -147,8 +160,11 @@ int gdn_plan_uses_tensor_path(gdn_plan_t plan);
  *     up to 128),
  *   4 G (in-block cumulative log decay), 5 beta, 6 log alpha ([B][H][Tp] fp32),
  *   7 W, 8 U, 9 Qt, 10 Kt, 11 Aqk ([B][H][Tp][128] fp16; tensor path only,
- *     else 0), 12 o ([B][T][H][d_v] fp32, before the output norm).
- * Returns the number of offsets written (13 at most). */
+ *     else 0), 12 o ([B][T][H][d_v] fp32 before the output norm; CUDA-core
+ *     path only, else 0), 13 per-segment [S_loc^T | P^T] ([B][H][NS][128][256]
+ *     fp32) and 14 segment start states S^T ([B][H][NS][128][128] fp32)
+ *     (tensor path only, else 0).
+ * Returns the number of offsets written (15 at most). */
 int gdn_workspace_offsets(gdn_plan_t plan, size_t *offsets, int n);
 
 /* Free a plan (host memory only).  NULL is accepted. */

@@ -90,3 +90,43 @@ def chunk_core(qh, kh, vh, log_alpha, beta, C=64, operand=None, store=None):
                 rows = min(C, T - c * C)
                 o[b, c * C:c * C + rows, h] = O[:rows]
     return o
+
+
+def segment_start_states(kh, vh, log_alpha, beta, C=128, Ls=2):
+    """Segment-parallel form of the inter-block state (one (b, h), inputs
+    [T, d]): each segment of Ls blocks runs the combined state [S^T | P^T]
+    from [0 | I] block by block (P is the segment's transfer matrix, S_loc its
+    end state from zero), then S_start(j+1)^T = P_j^T S_start(j)^T + S_loc(j)^T.
+    Returns the list of S^T at every segment start (d_k x d_v)."""
+    T, d = kh.shape
+    nb = -(-T // C)
+    Tp = nb * C
+
+    def pad(x):
+        out = np.zeros((Tp,) + x.shape[1:])
+        out[:T] = x
+        return out
+    K, V, la, be = pad(kh), pad(vh), pad(log_alpha), pad(beta)
+    ns = -(-nb // Ls)
+    zloc = []
+    for j in range(ns - 1):
+        Zt = np.zeros((d, 2 * d))
+        Zt[:, d:] = np.eye(d)
+        for c in range(j * Ls, min((j + 1) * Ls, nb)):
+            sl = slice(c * C, (c + 1) * C)
+            Kc, Vc, G, bc = K[sl], V[sl], np.cumsum(la[sl]), be[sl]
+            D = np.minimum(G[:, None] - G[None, :], 0.0)
+            L = np.tril(np.ones((C, C)), -1) * bc[:, None] * np.exp(D) * (Kc @ Kc.T)
+            Tm = np.linalg.inv(np.eye(C) + L)
+            W = Tm @ ((bc * np.exp(G))[:, None] * Kc)
+            U = Tm @ (bc[:, None] * Vc)
+            Kt = np.exp(G[-1] - G)[:, None] * Kc
+            Delta = np.concatenate([U, np.zeros((C, d))], 1) - W @ Zt
+            Zt = np.exp(G[-1]) * Zt + Kt.T @ Delta
+        zloc.append(Zt)
+    St = np.zeros((d, d))
+    starts = [St]
+    for j in range(ns - 1):
+        St = zloc[j][:, d:] @ St + zloc[j][:, :d]
+        starts.append(St)
+    return starts

@@ -153,6 +153,30 @@ def test_forward_host_matches_device_forward():
     assert torch.equal(y_host, y_dev.cpu())
 
 
+def test_forward_timed_records_every_launch_and_matches_forward():
+    import torch
+    import gated_deltanet_06_b200 as gdn
+    inp = gdn_inputs.make_inputs(1, 400, 2, 128, "bf16", 0.0, seed=28)
+    t = torch_inputs(inp)
+    plan = gdn.Plan(1, 400, 2, 128, gdn.DTYPE_BF16)
+    ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device="cuda")
+    y1 = gdn.forward(**t, plan=plan, workspace=ws)
+    y2 = torch.empty_like(y1)
+    stream = torch.cuda.current_stream()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(plan.launches + 1)]
+    for e in ev:
+        e.record(stream)
+    plan.forward_timed_raw(gdn.tensor_ptrs(t), y2.data_ptr(), ws.data_ptr(), stream.cuda_stream,
+                           [e.cuda_event for e in ev])
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    times = [ev[i].elapsed_time(ev[i + 1]) for i in range(plan.launches)]
+    assert all(x >= 0 for x in times) and sum(times) > 0
+    with pytest.raises(gdn.GDNError):
+        plan.forward_timed_raw(gdn.tensor_ptrs(t), y2.data_ptr(), ws.data_ptr(), stream.cuda_stream,
+                               [e.cuda_event for e in ev[:-1]])
+
+
 # ---------------------------------------------------------------- error paths
 def test_invalid_arguments_are_rejected_before_launch():
     import torch

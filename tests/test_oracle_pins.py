@@ -313,3 +313,21 @@ def test_workload_shapes_match_video_geometry():
     # the T3-Video page's Table 1 attention MACs for Wan2.1-1.3B at 480x832 (98.9T)
     # equal 2 * T^2 * d_model * layers at T = 32760, d_model = 1536, 30 layers
     assert abs(2 * 32760 ** 2 * 1536 * 30 / 1e12 - 98.9) < 0.05
+
+
+@pytest.mark.parametrize("Ls", [1, 2, 3])
+def test_segment_parallel_states_equal_sequential_states(Ls):
+    # the segment form (per-segment transfer matrices combined afterwards) gives
+    # the same state at every segment start as the token-by-token recurrence
+    from chunk_model import segment_start_states
+    T, d, C = 700, 16, 64
+    inp = gdn_inputs.make_inputs(1, T, 1, d, "f32", -3.0, seed=Ls)
+    _, it = oracle.forward(inp, intermediates=True)
+    starts = segment_start_states(it["kh"][0, :, 0], it["vh"][0, :, 0], np.log(it["alpha"][0, :, 0]),
+                                  it["beta"][0, :, 0], C=C, Ls=Ls)
+    assert len(starts) == -(-(-(-T // C)) // Ls)
+    for j, St in enumerate(starts[1:], start=1):
+        t_end = j * Ls * C
+        _, S = oracle.core(it["qh"][:, :t_end], it["kh"][:, :t_end], it["vh"][:, :t_end], it["alpha"][:, :t_end],
+                           it["beta"][:, :t_end], return_state=True)
+        np.testing.assert_allclose(St, S[0, 0].T, rtol=0, atol=1e-12 * max(1.0, np.abs(S).max()))
