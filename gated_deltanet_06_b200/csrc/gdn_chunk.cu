@@ -34,6 +34,8 @@ constexpr uint32_t OFF_LH = OFF_UNION + 32768;    //   fp16 128 rows x 64 (L[:, 
 constexpr uint32_t OFF_T1 = OFF_UNION + 49152;    //   fp16 64 x 64 (T_1^T), K-major B
 constexpr uint32_t OFF_T2 = OFF_UNION + 57344;    //   fp16 64 rows x 128 ([0; T_2]), MN-major A
 constexpr uint32_t OFF_P = OFF_UNION + 73728;     //   fp16 64 x 64 (L_21 T_1), MN-major B
+constexpr uint32_t OFF_AQK = OFF_UNION + 49152;   //   fp16 128x128 Aqk staging for the bulk store
+                                                  //   (done reading before T_1/T_2/P are written)
 constexpr uint32_t OFF_A1 = OFF_UNION + 0;        //   fp16 128x128 T diag(beta e^G), K-major A
 constexpr uint32_t OFF_A2 = OFF_UNION + 32768;    //   fp16 128x128 T diag(beta), K-major A
 constexpr uint32_t OFF_G = OFF_UNION + 81920;     // fp32 [128]
@@ -44,21 +46,12 @@ constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 
 constexpr uint32_t TM_AKK = 0, TM_QK = 128, TM_Y = 256, TM_T2P = 320, TM_W = 0, TM_U = 128;
 
-__device__ __forceinline__ void store_row_f16(__half *dst, const float *v, int n) {
-    // n multiple of 8; dst 16-byte aligned
-    for (int c = 0; c < n; c += 8) {
-        uint4 u;
-        u.x = pack_half2(v[c + 0], v[c + 1]);
-        u.y = pack_half2(v[c + 2], v[c + 3]);
-        u.z = pack_half2(v[c + 4], v[c + 5]);
-        u.w = pack_half2(v[c + 6], v[c + 7]);
-        *reinterpret_cast<uint4 *>(dst + c) = u;
-    }
-}
-
 __global__ void __launch_bounds__(128, 1)
     gdn_chunk_kernel(const ChunkParams p, const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ) {
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ,
+                     const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmU,
+                     const __grid_constant__ CUtensorMap tmQt, const __grid_constant__ CUtensorMap tmKt,
+                     const __grid_constant__ CUtensorMap tmAqk) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
@@ -103,7 +96,9 @@ __global__ void __launch_bounds__(128, 1)
         tma_load_2d(sm + OFF_Q, &tmQ, bar_load, 0, y);
         tma_load_2d(sm + OFF_Q + 16384, &tmQ, bar_load, 64, y);
     }
+    if (tid == 0) GDN_TRACE_AT(0);
     mbar_wait(bar_load, 0, ab, p.status, p.wait_limit_ns);
+    if (tid == 0) GDN_TRACE_AT(1);
     __syncthreads();
     if (ab->flag) goto teardown;
 
@@ -164,9 +159,7 @@ __global__ void __launch_bounds__(128, 1)
                         make_float4(l[i], l[i + 1], l[i + 2], l[i + 3]);
             }
         }
-        // Aqk row r, and the decayed copies of K and Q
-        const float Glast = sG[kBlk - 1];
-        __half *aqk_row = p.Aqk + (row0 + r) * kD;
+        // Aqk row r (staged for a bulk store); Qt = e^G Q written over the Q tile in place
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
             float a[32];
@@ -176,51 +169,69 @@ __global__ void __launch_bounds__(128, 1)
                 const int j = c * 32 + i;
                 a[i] = (j <= r) ? __expf(fminf(Gr - sG[j], 0.0f)) * a[i] : 0.0f;
             }
-            store_row_f16(aqk_row + c * 32, a, 32);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                uint4 u;
+                u.x = pack_half2(a[q4 * 8 + 0], a[q4 * 8 + 1]);
+                u.y = pack_half2(a[q4 * 8 + 2], a[q4 * 8 + 3]);
+                u.z = pack_half2(a[q4 * 8 + 4], a[q4 * 8 + 5]);
+                u.w = pack_half2(a[q4 * 8 + 6], a[q4 * 8 + 7]);
+                *reinterpret_cast<uint4 *>(sm + OFF_AQK + tile_off(128, r, c * 4 + q4)) = u;
+            }
         }
         const float fq = __expf(fminf(Gr, 0.0f));
-        const float fk = __expf(fminf(Glast - Gr, 0.0f));
-        __half *qt_row = p.Qt + (row0 + r) * kD;
-        __half *kt_row = p.Kt + (row0 + r) * kD;
 #pragma unroll 4
         for (int c = 0; c < 16; ++c) {
-            const uint4 uq = *reinterpret_cast<const uint4 *>(sm + OFF_Q + tile_off(128, r, c));
-            const uint4 uk = *reinterpret_cast<const uint4 *>(sm + OFF_K + tile_off(128, r, c));
-            const uint32_t wq[4] = {uq.x, uq.y, uq.z, uq.w}, wk[4] = {uk.x, uk.y, uk.z, uk.w};
-            uint32_t oq[4], ok[4];
+            uint4 *pq = reinterpret_cast<uint4 *>(sm + OFF_Q + tile_off(128, r, c));
+            const uint4 uq = *pq;
+            const uint32_t wq[4] = {uq.x, uq.y, uq.z, uq.w};
+            uint32_t oq[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const float2 xq = unpack_half2(wq[i]), xk = unpack_half2(wk[i]);
+                const float2 xq = unpack_half2(wq[i]);
                 oq[i] = pack_half2(xq.x * fq, xq.y * fq);
-                ok[i] = pack_half2(xk.x * fk, xk.y * fk);
             }
-            *reinterpret_cast<uint4 *>(qt_row + c * 8) = make_uint4(oq[0], oq[1], oq[2], oq[3]);
-            *reinterpret_cast<uint4 *>(kt_row + c * 8) = make_uint4(ok[0], ok[1], ok[2], ok[3]);
+            *pq = make_uint4(oq[0], oq[1], oq[2], oq[3]);
         }
     }
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
+    if (tid == 0) {
+        const int y = static_cast<int>(row0);
+        tma_store_2d(&tmAqk, sm + OFF_AQK, 0, y);
+        tma_store_2d(&tmAqk, sm + OFF_AQK + 16384, 64, y);
+        tma_store_2d(&tmQt, sm + OFF_Q, 0, y);
+        tma_store_2d(&tmQt, sm + OFF_Q + 16384, 64, y);
+        bulk_commit();
+    }
 
+    if (tid == 0) GDN_TRACE_AT(2);
     // ---- two 64x64 unit lower-triangular inverses, one column per thread
     float col[64];
     {
         const int i = r & 63;
         const float *Ld = reinterpret_cast<const float *>(sm + (r < 64 ? OFF_LD1 : OFF_LD2));
+        // four independent partial sums per row keep the FMA pipe busy
 #pragma unroll
         for (int rr = 0; rr < 64; ++rr) {
-            float acc = (rr == i) ? 1.0f : 0.0f;
+            float a0 = (rr == i) ? 1.0f : 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
 #pragma unroll
             for (int j4 = 0; j4 < rr; j4 += 4) {
                 const float4 l = *reinterpret_cast<const float4 *>(Ld + rr * 64 + j4);
-                acc = fmaf(-l.x, col[j4], acc);
-                if (j4 + 1 < rr) acc = fmaf(-l.y, col[j4 + 1], acc);
-                if (j4 + 2 < rr) acc = fmaf(-l.z, col[j4 + 2], acc);
-                if (j4 + 3 < rr) acc = fmaf(-l.w, col[j4 + 3], acc);
+                a0 = fmaf(-l.x, col[j4], a0);
+                if (j4 + 1 < rr) a1 = fmaf(-l.y, col[j4 + 1], a1);
+                if (j4 + 2 < rr) a2 = fmaf(-l.z, col[j4 + 2], a2);
+                if (j4 + 3 < rr) a3 = fmaf(-l.w, col[j4 + 3], a3);
             }
-            col[rr] = acc;
+            col[rr] = (a0 + a1) + (a2 + a3);
         }
     }
+    if (tid == 0) GDN_TRACE_AT(3);
+    // T_1, T_2, P below overwrite the Aqk staging area: the bulk store must have read it
+    if (tid == 0) bulk_wait_read_all();
+    if (tid == 0) GDN_TRACE_AT(4);
+    __syncthreads();
     // T_1^T as the K-major B operand (row i = column i of T_1)
     if (r < 64) {
 #pragma unroll
@@ -303,6 +314,7 @@ __global__ void __launch_bounds__(128, 1)
     if (ab->flag) goto teardown;
     tc_fence_after();
 
+    if (tid == 0) GDN_TRACE_AT(5);
     // ---- A1 = T diag(beta e^G), A2 = T diag(beta): K-major A operands (row r, column j)
     {
         uint8_t *A1 = sm + OFF_A1;
@@ -361,6 +373,7 @@ __global__ void __launch_bounds__(128, 1)
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
+    if (tid == 0) GDN_TRACE_AT(6);
     // ---- W = A1 K, U = A2 V  (A K-major; B = the TMA tiles read MN-major: K = token, N = channel)
     if (tid == 0) {
         tc_fence_after();
@@ -380,20 +393,65 @@ __global__ void __launch_bounds__(128, 1)
     __syncthreads();
     if (ab->flag) goto teardown;
     tc_fence_after();
+    if (tid == 0) GDN_TRACE_AT(7);
     {
-        __half *w_row = p.W + (row0 + r) * kD;
-        __half *u_row = p.U + (row0 + r) * kD;
+        // W -> A1 area, U -> A2 area (both free now), Kt = e^(G_last - G) K over the K tile in place
+        const float fk = __expf(fminf(sG[kBlk - 1] - sG[r], 0.0f));
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
             float a[32];
             tmem_ld32(tmem + lane_base + TM_W + c * 32, a);
-            store_row_f16(w_row + c * 32, a, 32);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                uint4 u;
+                u.x = pack_half2(a[q4 * 8 + 0], a[q4 * 8 + 1]);
+                u.y = pack_half2(a[q4 * 8 + 2], a[q4 * 8 + 3]);
+                u.z = pack_half2(a[q4 * 8 + 4], a[q4 * 8 + 5]);
+                u.w = pack_half2(a[q4 * 8 + 6], a[q4 * 8 + 7]);
+                *reinterpret_cast<uint4 *>(sm + OFF_A1 + tile_off(128, r, c * 4 + q4)) = u;
+            }
             tmem_ld32(tmem + lane_base + TM_U + c * 32, a);
-            store_row_f16(u_row + c * 32, a, 32);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                uint4 u;
+                u.x = pack_half2(a[q4 * 8 + 0], a[q4 * 8 + 1]);
+                u.y = pack_half2(a[q4 * 8 + 2], a[q4 * 8 + 3]);
+                u.z = pack_half2(a[q4 * 8 + 4], a[q4 * 8 + 5]);
+                u.w = pack_half2(a[q4 * 8 + 6], a[q4 * 8 + 7]);
+                *reinterpret_cast<uint4 *>(sm + OFF_A2 + tile_off(128, r, c * 4 + q4)) = u;
+            }
+        }
+#pragma unroll 4
+        for (int c = 0; c < 16; ++c) {
+            uint4 *pk = reinterpret_cast<uint4 *>(sm + OFF_K + tile_off(128, r, c));
+            const uint4 uk = *pk;
+            const uint32_t wk[4] = {uk.x, uk.y, uk.z, uk.w};
+            uint32_t ok4[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 xk = unpack_half2(wk[i]);
+                ok4[i] = pack_half2(xk.x * fk, xk.y * fk);
+            }
+            *pk = make_uint4(ok4[0], ok4[1], ok4[2], ok4[3]);
         }
     }
+    fence_proxy_async();
+    __syncthreads();
+    if (tid == 0) {
+        const int y = static_cast<int>(row0);
+        tma_store_2d(&tmW, sm + OFF_A1, 0, y);
+        tma_store_2d(&tmW, sm + OFF_A1 + 16384, 64, y);
+        tma_store_2d(&tmU, sm + OFF_A2, 0, y);
+        tma_store_2d(&tmU, sm + OFF_A2 + 16384, 64, y);
+        tma_store_2d(&tmKt, sm + OFF_K, 0, y);
+        tma_store_2d(&tmKt, sm + OFF_K + 16384, 64, y);
+        bulk_commit();
+    }
 
+    if (tid == 0) GDN_TRACE_AT(8);
 teardown:
+    if (tid == 0) bulk_wait_all();  // every bulk store issued by this CTA has completed
+    if (tid == 0) GDN_TRACE_AT(9);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -403,7 +461,9 @@ teardown:
 }  // namespace
 
 cudaError_t launch_chunk(const ChunkParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
-                         const CUtensorMap &tmQ, cudaStream_t s) {
+                         const CUtensorMap &tmQ, const CUtensorMap &tmW, const CUtensorMap &tmU,
+                         const CUtensorMap &tmQt, const CUtensorMap &tmKt, const CUtensorMap &tmAqk,
+                         cudaStream_t s) {
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(gdn_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -412,8 +472,10 @@ cudaError_t launch_chunk(const ChunkParams &p, const CUtensorMap &tmK, const CUt
         attr_set = true;
     }
     dim3 grid(p.NB, p.BH);
-    gdn_chunk_kernel<<<grid, 128, SMEM_BYTES, s>>>(p, tmK, tmV, tmQ);
+    gdn_chunk_kernel<<<grid, 128, SMEM_BYTES, s>>>(p, tmK, tmV, tmQ, tmW, tmU, tmQt, tmKt, tmAqk);
     return cudaGetLastError();
 }
 
 }  // namespace gdn
+
+GDN_TRACE_EXPORT(chunk)

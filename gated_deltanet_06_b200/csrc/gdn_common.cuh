@@ -31,6 +31,34 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
+// Optional phase timeline for kernel tuning: compiled in only with -DGDN_TRACE
+// (never in the shipped build).  GDN_TRACE_AT(slot) records the global timer
+// of the calling thread into this translation unit's device-side array when
+// the CTA is the first one; GDN_TRACE_EXPORT(name) defines the host reader
+// gdn_trace_read_<name> for that array.
+#ifdef GDN_TRACE
+static __device__ unsigned long long g_gdn_trace[8192];
+#define GDN_TRACE_AT(slot)                                                                   \
+    do {                                                                                     \
+        if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && (slot) >= 0 && (slot) < 8192) \
+            ::gdn::g_gdn_trace[(slot)] = ::gdn::globaltimer_ns();                            \
+    } while (0)
+#define GDN_TRACE_EXPORT(name)                                                                        \
+    extern "C" int gdn_trace_read_##name(unsigned long long *host, int n) {                           \
+        static unsigned long long zeros[8192];                                                         \
+        if (n > 8192) n = 8192;                                                                        \
+        if (cudaMemcpyFromSymbol(host, ::gdn::g_gdn_trace, n * sizeof(unsigned long long)) != cudaSuccess) \
+            return -1;                                                                                 \
+        cudaMemcpyToSymbol(::gdn::g_gdn_trace, zeros, sizeof(zeros));                                  \
+        return n;                                                                                      \
+    }
+#else
+#define GDN_TRACE_AT(slot) \
+    do {                   \
+    } while (0)
+#define GDN_TRACE_EXPORT(name)
+#endif
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
@@ -94,6 +122,28 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
+// 2-D tiled bulk tensor store shared -> global (bulk async-group completion).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+                 "r"(smem_u32(src)), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until every committed bulk store has finished reading its shared-memory source
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// wait until every committed bulk store has completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Prefetch a 2-D tile of a tensor map into L2 (no shared memory involved).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *map, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int x, int y, int z) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(map), "r"(x), "r"(y),
+                 "r"(z)
+                 : "memory");
+}
+
 // Make generic-proxy writes to shared memory visible to the async proxy
 // (tensor core / TMA) before they are consumed there.
 __device__ __forceinline__ void fence_proxy_async() {
@@ -153,6 +203,27 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Each thread of the warp writes 32 consecutive 32-bit columns of its own TMEM lane.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+        "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+        "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+        "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+        "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // ---------------------------------------------------------- UMMA descriptors
 // Shared-memory matrix descriptor, SWIZZLE_128B canonical layout (sm100
 // version field = 1).  lbo/sbo in bytes.
@@ -205,7 +276,9 @@ __device__ __forceinline__ float2 unpack_half2(uint32_t u) {
     return __half22float2(h);
 }
 
-__device__ __forceinline__ float silu_f(float u) { return u / (1.0f + __expf(-u)); }
+// SiLU with the fast reciprocal divide (2 ulp); for u -> -inf the denominator
+// overflows and the result is 0, the limit of u e^u.
+__device__ __forceinline__ float silu_f(float u) { return __fdividef(u, 1.0f + __expf(-u)); }
 
 __device__ __forceinline__ float softplus_f(float x) { return x > 20.0f ? x : log1pf(expf(x)); }
 

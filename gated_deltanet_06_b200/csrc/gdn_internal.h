@@ -25,8 +25,14 @@ struct PrepParams {
     float *log_alpha;              // [B][H][Tp]
     int B, T, H, d, Tp;
     float l2_eps, q_scale;
+    int *status;
+    unsigned long long wait_limit_ns;
 };
 cudaError_t launch_prep(const PrepParams &p, InType in, bool out_f16, cudaStream_t s);
+// Tensor path (16-bit inputs, d = 128): raw tiles staged by TMA through the
+// 3-D maps tmq/tmk/tmv over [B][T][H*d] (box {64, 131, 1}).
+cudaError_t launch_prep_tma(const PrepParams &p, InType in, const CUtensorMap &tmq, const CUtensorMap &tmk,
+                            const CUtensorMap &tmv, cudaStream_t s);
 
 // Intra-block UT transform on tensor cores (d = 128, fp16 operands).
 struct ChunkParams {
@@ -37,7 +43,9 @@ struct ChunkParams {
     unsigned long long wait_limit_ns;
 };
 cudaError_t launch_chunk(const ChunkParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
-                         const CUtensorMap &tmQ, cudaStream_t s);
+                         const CUtensorMap &tmQ, const CUtensorMap &tmW, const CUtensorMap &tmU,
+                         const CUtensorMap &tmQt, const CUtensorMap &tmKt, const CUtensorMap &tmAqk,
+                         cudaStream_t s);
 
 // Inter-block state scan on tensor cores (d = 128), parallel over segments of
 // Ls blocks: pass A (transfer), combine, pass C (outputs + fused output step).
@@ -61,7 +69,7 @@ cudaError_t launch_transfer(const ScanParams &p, const CUtensorMap &tmW, const C
 cudaError_t launch_combine(const ScanParams &p, cudaStream_t s);
 cudaError_t launch_scan_out(const ScanParams &p, InType zt, const CUtensorMap &tmW, const CUtensorMap &tmQt,
                             const CUtensorMap &tmKt, const CUtensorMap &tmAqk, const CUtensorMap &tmU,
-                            cudaStream_t s);
+                            const CUtensorMap &tmZ, cudaStream_t s);
 
 // Sequential fp32 recurrence on CUDA cores (fp32 inputs or d = 64).
 struct RecurParams {

@@ -170,6 +170,129 @@ __global__ void __launch_bounds__(256) gdn_prep_kernel(const PrepParams p) {
     }
 }
 
+// Tensor-path variant (16-bit inputs, d = 128): one thread issues TMA loads of
+// the three raw 131-token x 128-channel tiles (3 tokens of conv history; rows
+// before t = 0 of the batch item and past T come back as zeros from the
+// tensor map's out-of-bounds fill), and all 256 threads then work out of
+// shared memory.  About 100 KB of shared memory per CTA keeps two CTAs, i.e.
+// two whole tiles of loads, in flight per SM.
+constexpr int kRawRows = kBlk + 3;
+constexpr uint32_t kRawHalf = kRawRows * 128;  // bytes of one {64 ch, 131 tok} box
+constexpr uint32_t kPrepSmem = 6 * kRawHalf + 64 + 128;
+
+template <typename InT>
+__global__ void __launch_bounds__(256, 2)
+    gdn_prep_tma_kernel(const PrepParams p, const __grid_constant__ CUtensorMap tmq,
+                        const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
+    constexpr int D = 128, CPR = 16, RPT = 8;
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + 6 * kRawHalf);
+    float *warp_tot = reinterpret_cast<float *>(bar + 1);
+    __shared__ AbortState ab;
+
+    const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int t0 = blk * kBlk;
+    const int tid = threadIdx.x;
+    const size_t bh = static_cast<size_t>(b) * p.H + h;
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        ab.flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        mbar_arrive_expect_tx(bar, 6 * kRawHalf);
+        const CUtensorMap *maps[3] = {&tmq, &tmk, &tmv};
+        for (int w = 0; w < 3; ++w)
+            for (int hf = 0; hf < 2; ++hf)
+                asm volatile(
+                    "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
+                        smem_u32(sm + (w * 2 + hf) * kRawHalf)),
+                    "l"(maps[w]), "r"(smem_u32(bar)), "r"(h * D + hf * 64), "r"(t0 - 3), "r"(b)
+                    : "memory");
+    }
+    // gates and the in-block cumulative log decay while the tiles land
+    float la = 0.0f, be = 0.0f;
+    {
+        const int t = t0 + tid;
+        if (tid < kBlk && t < p.T) {
+            const size_t gi = (static_cast<size_t>(b) * p.T + t) * p.H + h;
+            const float xg = p.g[gi] + p.dt_bias[h];
+            la = -expf(p.A_log[h]) * softplus_f(xg);
+            be = 1.0f / (1.0f + expf(-p.b[gi]));
+        }
+        float cs = la;
+        const int lane = tid & 31, wid = tid >> 5;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float n = __shfl_up_sync(0xffffffffu, cs, off);
+            if (lane >= off) cs += n;
+        }
+        if (lane == 31) warp_tot[wid] = cs;
+        __syncthreads();
+        if (tid < kBlk) {
+            float pre = 0.0f;
+            for (int i = 0; i < wid; ++i) pre += warp_tot[i];
+            const size_t o = bh * p.Tp + t;
+            p.G[o] = cs + pre;
+            p.beta[o] = be;
+            p.log_alpha[o] = la;
+        }
+    }
+    const bool ok = mbar_wait(bar, 0, &ab, p.status, p.wait_limit_ns);
+    if (!__syncthreads_and(ok)) return;
+
+    const int cg = tid % CPR, rg = tid / CPR;
+    const int c0 = cg * 8;
+    const int rbeg = rg * RPT;
+    const uint32_t coff = (cg >> 3) * kRawHalf + (cg & 7) * 16;
+#pragma unroll 1
+    for (int which = 0; which < 3; ++which) {
+        const float *w = which == 0 ? p.conv_q : (which == 1 ? p.conv_k : p.conv_v);
+        __half *out = static_cast<__half *>(which == 0 ? p.qh : (which == 1 ? p.kh : p.vh));
+        const uint8_t *tile = sm + which * 2 * kRawHalf + coff;
+        float wt[8][4];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const float4 t4 = reinterpret_cast<const float4 *>(w)[static_cast<size_t>(h) * D + c0 + c];
+            wt[c][0] = t4.x; wt[c][1] = t4.y; wt[c][2] = t4.z; wt[c][3] = t4.w;
+        }
+        float win[4][8];
+#pragma unroll
+        for (int i = 0; i < 3; ++i) In8<InT>::load(reinterpret_cast<const InT *>(tile + (rbeg + i) * 128), win[i]);
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) {
+            In8<InT>::load(reinterpret_cast<const InT *>(tile + (rbeg + r + 3) * 128), win[(r + 3) & 3]);
+            float u[8];
+            float ss = 0.0f;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                float a = wt[c][0] * win[r & 3][c];
+                a = fmaf(wt[c][1], win[(r + 1) & 3][c], a);
+                a = fmaf(wt[c][2], win[(r + 2) & 3][c], a);
+                a = fmaf(wt[c][3], win[(r + 3) & 3][c], a);
+                u[c] = silu_f(a);
+                ss = fmaf(u[c], u[c], ss);
+            }
+            if (which < 2) {
+#pragma unroll
+                for (int off = CPR / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                float sc = 1.0f / sqrtf(ss + p.l2_eps);
+                if (which == 0) sc *= p.q_scale;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) u[c] *= sc;
+            }
+            const int t = t0 + rbeg + r;
+            if (t >= p.T) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) u[c] = 0.0f;
+            }
+            store8<__half>(out + (bh * p.Tp + t) * D + c0, u);
+        }
+    }
+}
+
 template <typename InT, typename OutT>
 cudaError_t launch_typed(const PrepParams &p, cudaStream_t s) {
     dim3 grid(p.Tp / kBlk, p.H, p.B);
@@ -181,6 +304,30 @@ cudaError_t launch_typed(const PrepParams &p, cudaStream_t s) {
 }
 
 }  // namespace
+
+cudaError_t launch_prep_tma(const PrepParams &p, InType in, const CUtensorMap &tmq, const CUtensorMap &tmk,
+                            const CUtensorMap &tmv, cudaStream_t s) {
+    static bool attr_bf = false, attr_h = false;
+    dim3 grid(p.Tp / kBlk, p.H, p.B);
+    if (in == InType::BF16) {
+        if (!attr_bf) {
+            cudaError_t e = cudaFuncSetAttribute(gdn_prep_tma_kernel<__nv_bfloat16>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kPrepSmem);
+            if (e != cudaSuccess) return e;
+            attr_bf = true;
+        }
+        gdn_prep_tma_kernel<__nv_bfloat16><<<grid, 256, kPrepSmem, s>>>(p, tmq, tmk, tmv);
+    } else {
+        if (!attr_h) {
+            cudaError_t e = cudaFuncSetAttribute(gdn_prep_tma_kernel<__half>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kPrepSmem);
+            if (e != cudaSuccess) return e;
+            attr_h = true;
+        }
+        gdn_prep_tma_kernel<__half><<<grid, 256, kPrepSmem, s>>>(p, tmq, tmk, tmv);
+    }
+    return cudaGetLastError();
+}
 
 cudaError_t launch_prep(const PrepParams &p, InType in, bool out_f16, cudaStream_t s) {
     if (out_f16) {

@@ -52,7 +52,9 @@ constexpr uint32_t OFF_BAR = 229376;
 constexpr int NBAR = 7;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
 enum { FULL_W = 0, FULL_U, FULL_K, MMA_X, MMA_P, CONS_D, CONS_S };
-constexpr uint32_t TM_X = 0, TM_P = 256;
+// X and P share 256 columns (X is read out before P is written); the fp32
+// state [S^T | P^T] lives in the other 256.
+constexpr uint32_t TM_X = 0, TM_P = 0, TM_Z = 256;
 }  // namespace ta
 
 __global__ void __launch_bounds__(288, 1)
@@ -102,6 +104,14 @@ __global__ void __launch_bounds__(288, 1)
             bool ok = true;
             for (int c = c0; ok && c < c1; ++c) {
                 const uint32_t ph = (c - c0) & 1;
+                if (c + 2 < c1) {  // pull the tiles of block c+2 into L2 ahead of their TMA loads
+                    const int y2 = rowbase + (c + 2) * kBlk;
+                    for (int hf = 0; hf < 2; ++hf) {
+                        tma_prefetch_2d(&tmW, hf * 64, y2);
+                        tma_prefetch_2d(&tmU, hf * 64, y2);
+                        tma_prefetch_2d(&tmKt, hf * 64, y2);
+                    }
+                }
                 ok = mbar_wait(&bars[FULL_W], ph, ab, p.status, lim) && mbar_wait(&bars[CONS_S], ph, ab, p.status, lim);
                 if (!ok) break;
                 tc_fence_after();
@@ -131,12 +141,19 @@ __global__ void __launch_bounds__(288, 1)
         const int q = warp & 3, half = warp >> 2;  // half 0: S^T columns, half 1: P^T columns
         const int r = q * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-        float Z[128];
+        const uint32_t tz = tmem + lane_base + TM_Z + half * 128;
 #pragma unroll
-        for (int i = 0; i < 128; ++i) Z[i] = (half == 1 && i == r) ? 1.0f : 0.0f;
+        for (int ch = 0; ch < 4; ++ch) {
+            float v[32];
 #pragma unroll
-        for (int c8 = 0; c8 < 16; ++c8) store_f16_chunk(sm + OFF_Z, 128, r, half * 16 + c8, &Z[c8 * 8]);
+            for (int e = 0; e < 32; ++e) v[e] = (half == 1 && ch * 32 + e == r) ? 1.0f : 0.0f;
+            tmem_st32(tz + ch * 32, v);
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) store_f16_chunk(sm + OFF_Z, 128, r, half * 16 + ch * 4 + qq, &v[qq * 8]);
+        }
+        tmem_st_wait();
         fence_proxy_async();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[CONS_S]);
         const float *Gbh = p.G + static_cast<size_t>(bh) * p.Tp;
@@ -179,23 +196,33 @@ __global__ void __launch_bounds__(288, 1)
             tc_fence_after();
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
-                float pv[32];
+                float pv[32], zv[32];
                 tmem_ld32(tmem + lane_base + TM_P + half * 128 + ch * 32, pv);
+                tmem_ld32(tz + ch * 32, zv);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) Z[ch * 32 + i] = fmaf(gC, Z[ch * 32 + i], pv[i]);
+                for (int e = 0; e < 32; ++e) zv[e] = fmaf(gC, zv[e], pv[e]);
+                tmem_st32(tz + ch * 32, zv);
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq)
-                    store_f16_chunk(sm + OFF_Z, 128, r, half * 16 + ch * 4 + qq, &Z[ch * 32 + qq * 8]);
+                    store_f16_chunk(sm + OFF_Z, 128, r, half * 16 + ch * 4 + qq, &zv[qq * 8]);
             }
+            tmem_st_wait();
             fence_proxy_async();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[CONS_S]);
         }
         if (ok) {
+            tc_fence_after();
             float *dst = p.Zloc + ((static_cast<size_t>(bh) * p.NS + seg) * 128 + r) * 256 + half * 128;
 #pragma unroll
-            for (int i = 0; i < 128; i += 4) *reinterpret_cast<float4 *>(dst + i) = make_float4(Z[i], Z[i + 1], Z[i + 2], Z[i + 3]);
+            for (int ch = 0; ch < 4; ++ch) {
+                float zv[32];
+                tmem_ld32(tz + ch * 32, zv);
+#pragma unroll
+                for (int e = 0; e < 32; e += 4)
+                    *reinterpret_cast<float4 *>(dst + ch * 32 + e) = make_float4(zv[e], zv[e + 1], zv[e + 2], zv[e + 3]);
+            }
         }
     }
     tc_fence_before();
@@ -206,39 +233,44 @@ __global__ void __launch_bounds__(288, 1)
 
 // ============================================================ combine
 // S_start(j+1)^T = P_j^T S_start(j)^T + S_loc(j)^T, sequential over j; one CTA
-// per (8-column slice of S^T, head); thread t owns row t of the slice.
-__global__ void __launch_bounds__(128) gdn_combine_kernel(const ScanParams p) {
-    __shared__ float cur[128][8];
+// per (8-column slice of S^T, head), 256 threads: thread (t, half) owns row t
+// and 4 of the 8 columns; the P^T row is brought into registers in one round
+// trip per segment.
+__global__ void __launch_bounds__(256) gdn_combine_kernel(const ScanParams p) {
+    __shared__ __align__(16) float cur[128][8];
     const int slice = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int bh = b * p.H + h;
-    const int t = threadIdx.x;
-    const int c0 = slice * 8;
+    const int t = threadIdx.x >> 1, half = threadIdx.x & 1;
+    const int c0 = slice * 8 + half * 4;
+    if (threadIdx.x < 128) {
 #pragma unroll
-    for (int c = 0; c < 8; ++c) cur[t][c] = 0.0f;
+        for (int c = 0; c < 8; ++c) cur[threadIdx.x][c] = 0.0f;
+    }
     __syncthreads();
     for (int j = 0; j + 1 < p.NS; ++j) {
         const float *zrow = p.Zloc + ((static_cast<size_t>(bh) * p.NS + j) * 128 + t) * 256;
-        float acc[8];
+        const float4 sl = *reinterpret_cast<const float4 *>(zrow + c0);  // S_loc^T
+        float acc[4] = {sl.x, sl.y, sl.z, sl.w};
+        const float4 *prow = reinterpret_cast<const float4 *>(zrow + 128);  // P^T row t
+        float4 pr[32];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) acc[c] = zrow[c0 + c];  // S_loc^T
-        const float *prow = zrow + 128;                       // P^T row t
-#pragma unroll 4
-        for (int i = 0; i < 128; i += 4) {
-            const float4 pv = *reinterpret_cast<const float4 *>(prow + i);
+        for (int i = 0; i < 32; ++i) pr[i] = __ldg(prow + i);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                acc[c] = fmaf(pv.x, cur[i][c], acc[c]);
-                acc[c] = fmaf(pv.y, cur[i + 1][c], acc[c]);
-                acc[c] = fmaf(pv.z, cur[i + 2][c], acc[c]);
-                acc[c] = fmaf(pv.w, cur[i + 3][c], acc[c]);
+        for (int i4 = 0; i4 < 32; ++i4) {
+            const float pv[4] = {pr[i4].x, pr[i4].y, pr[i4].z, pr[i4].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float4 cv = *reinterpret_cast<const float4 *>(&cur[i4 * 4 + e][half * 4]);
+                acc[0] = fmaf(pv[e], cv.x, acc[0]);
+                acc[1] = fmaf(pv[e], cv.y, acc[1]);
+                acc[2] = fmaf(pv[e], cv.z, acc[2]);
+                acc[3] = fmaf(pv[e], cv.w, acc[3]);
             }
         }
         __syncthreads();
-#pragma unroll
-        for (int c = 0; c < 8; ++c) cur[t][c] = acc[c];
+        *reinterpret_cast<float4 *>(&cur[t][half * 4]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
         float *dst = p.Sstart + ((static_cast<size_t>(bh) * p.NS + j + 1) * 128 + t) * 128 + c0;
         *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        *reinterpret_cast<float4 *>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
         __syncthreads();
     }
 }
@@ -250,9 +282,13 @@ constexpr uint32_t OFF_S = 163840;  // S^T fp16 MN-major B operand (rows d_k, co
 constexpr uint32_t OFF_D = 196608;  // Delta fp16 MN-major B operand (rows token, cols d_v)
 constexpr uint32_t OFF_BAR = 229376;
 constexpr int NBAR = 11;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
+constexpr uint32_t OFF_NW = OFF_BAR + NBAR * 8 + 16;  // norm weight, fp32 [128]
+constexpr uint32_t SMEM_BYTES = OFF_NW + 512 + 1024;
 enum { FULL_WQ = 0, FULL_U, FULL_KA, MMA_X, MMA_P, MMA_O, CONS_D, CONS_S, CONS_O0, CONS_O1, TEST };
-constexpr uint32_t TM_X = 0, TM_P = 128, TM_O = 256;  // O double-buffered: 256 and 384
+constexpr int kScanThreads = 288;  // warps 0-3 state, warp 4 producer, warps 5-8 output step
+// X and P share columns (X is read out before P is written, P before the next X);
+// the fp32 state S^T lives in TMEM; O is double-buffered (256 and 384).
+constexpr uint32_t TM_X = 0, TM_P = 0, TM_S = 128, TM_O = 256;
 }  // namespace tc
 
 template <typename ZT, typename YT>
@@ -304,10 +340,11 @@ __device__ __forceinline__ void store_y8(void *y, int out_kind, size_t idx, cons
 }
 
 template <typename ZT>
-__global__ void __launch_bounds__(160, 1)
+__global__ void __launch_bounds__(tc::kScanThreads, 1)
     gdn_scan_out_kernel(const ScanParams p, const __grid_constant__ CUtensorMap tmW,
                         const __grid_constant__ CUtensorMap tmQt, const __grid_constant__ CUtensorMap tmKt,
-                        const __grid_constant__ CUtensorMap tmAqk, const __grid_constant__ CUtensorMap tmU) {
+                        const __grid_constant__ CUtensorMap tmAqk, const __grid_constant__ CUtensorMap tmU,
+                        const __grid_constant__ CUtensorMap tmZ) {
     using namespace tc;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -322,11 +359,13 @@ __global__ void __launch_bounds__(160, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint64_t lim = p.wait_limit_ns;
 
+    float *sNW = reinterpret_cast<float *>(sm + OFF_NW);
     if (tid == 0) {
         for (int i = 0; i < NBAR; ++i) mbar_init(&bars[i], (i >= CONS_D && i <= CONS_O1) ? 4 : 1);
         ab->flag = 0;
         fence_mbar_init();
     }
+    if (tid < kD) sNW[tid] = p.norm_w[tid];
     if (warp == 0) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
@@ -336,7 +375,57 @@ __global__ void __launch_bounds__(160, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
+    if (warp >= 5) {
+        // ------------------------------------------- output step (warps 5-8)
+        // y = o / sqrt(mean(o^2) + eps) * w * SiLU(z) for the block rows this
+        // warp's TMEM lane quarter holds; the z row is fetched before the
+        // accumulator is read so its latency overlaps the TMEM traffic.
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+        const ZT *z = static_cast<const ZT *>(p.z);
+        for (int c = c0; c < c1; ++c) {
+            const int i = c - c0;
+            const int t = c * kBlk + r;
+            const bool live = t < p.T;
+            const size_t zrow = (static_cast<size_t>(b) * p.T + (live ? t : 0)) * p.tok_stride + static_cast<size_t>(h) * kD;
+            const size_t yrow = ((static_cast<size_t>(b) * p.T + (live ? t : 0)) * p.H + h) * kD;
+            uint4 zr[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) zr[k] = live ? *reinterpret_cast<const uint4 *>(z + zrow + k * 8) : make_uint4(0, 0, 0, 0);
+            if (!warp_wait(&bars[MMA_O], i & 1, ab, p.status, lim)) break;
+            tc_fence_after();
+            const uint32_t tO = tmem + lane_base + TM_O + (i & 1) * 128;
+            float ss = 0.0f;
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                float ov[32];
+                tmem_ld32(tO + ch * 32, ov);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) ss = fmaf(ov[e], ov[e], ss);
+            }
+            const float rn = 1.0f / sqrtf(ss * (1.0f / 128.0f) + p.eps);
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                float ov[32];
+                tmem_ld32(tO + ch * 32, ov);
+                if (live) {
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq) {
+                        const int col = ch * 32 + qq * 8;
+                        float zf[8], yv[8];
+                        load8<ZT, float>(reinterpret_cast<const ZT *>(&zr[ch * 4 + qq]), zf);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) yv[e] = ov[qq * 8 + e] * rn * sNW[col + e] * silu_f(zf[e]);
+                        store_y8(p.y, p.out_kind, yrow + col, yv);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[CONS_O0 + (i & 1)]);
+        }
+    } else if (warp == 4) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             bool ok = true;
@@ -369,6 +458,8 @@ __global__ void __launch_bounds__(160, 1)
                 load_wq(c0);
                 load_u(c0);
                 load_ka(c0);
+                if (c0 * kBlk < p.T)
+                    for (int hf = 0; hf < 2; ++hf) tma_prefetch_3d(&tmZ, h * kD + hf * 64, c0 * kBlk, b);
             }
             const uint32_t id_kmn = idesc_f16_f32(128, 128, false, true);
             const uint32_t id_mnmn = idesc_f16_f32(128, 128, true, true);
@@ -376,9 +467,26 @@ __global__ void __launch_bounds__(160, 1)
                 const int i = c - c0;
                 const uint32_t ph = i & 1;
                 const uint32_t tO = tmem + TM_O + (i & 1) * 128;
-                ok = mbar_wait(&bars[FULL_WQ], ph, ab, p.status, lim) &&
-                     mbar_wait(&bars[CONS_S], ph, ab, p.status, lim) &&
-                     (i < 2 || mbar_wait(&bars[CONS_O0 + (i & 1)], ((i >> 1) - 1) & 1, ab, p.status, lim));
+                if (c + 2 < c1) {  // pull the tiles of block c+2 into L2 ahead of their TMA loads
+                    const int y2 = rowbase + (c + 2) * kBlk;
+                    for (int hf = 0; hf < 2; ++hf) {
+                        tma_prefetch_2d(&tmW, hf * 64, y2);
+                        tma_prefetch_2d(&tmQt, hf * 64, y2);
+                        tma_prefetch_2d(&tmU, hf * 64, y2);
+                        tma_prefetch_2d(&tmKt, hf * 64, y2);
+                        tma_prefetch_2d(&tmAqk, hf * 64, y2);
+                    }
+                }
+                if (c + 1 < c1 && (c + 1) * kBlk < p.T) {  // z rows the epilogue of block c+1 reads
+                    for (int hf = 0; hf < 2; ++hf) tma_prefetch_3d(&tmZ, h * kD + hf * 64, (c + 1) * kBlk, b);
+                }
+                GDN_TRACE_AT(4096 + 64 * i + 0);
+                ok = mbar_wait(&bars[FULL_WQ], ph, ab, p.status, lim);
+                GDN_TRACE_AT(4096 + 64 * i + 1);
+                ok = ok && mbar_wait(&bars[CONS_S], ph, ab, p.status, lim);
+                GDN_TRACE_AT(4096 + 64 * i + 2);
+                ok = ok && (i < 2 || mbar_wait(&bars[CONS_O0 + (i & 1)], ((i >> 1) - 1) & 1, ab, p.status, lim));
+                GDN_TRACE_AT(4096 + 64 * i + 3);
                 if (!ok) break;
                 tc_fence_after();
                 // X = W S^T ; O = Qt S^T   (A K-major, B = S^T MN-major)
@@ -390,11 +498,15 @@ __global__ void __launch_bounds__(160, 1)
                     umma_f16(tO, sdesc_sw128(sbase + OFF_QT + aoff, 16, 1024), bd, id_kmn, kk > 0);
                 }
                 umma_commit(&bars[MMA_X]);
+                GDN_TRACE_AT(4096 + 64 * i + 4);
                 ok = mbar_wait(&bars[MMA_X], ph, ab, p.status, lim);
+                GDN_TRACE_AT(4096 + 64 * i + 5);
                 if (!ok) break;
                 if (c + 1 < c1) load_wq(c + 1);
-                ok = mbar_wait(&bars[FULL_KA], ph, ab, p.status, lim) &&
-                     mbar_wait(&bars[CONS_D], ph, ab, p.status, lim);
+                ok = mbar_wait(&bars[FULL_KA], ph, ab, p.status, lim);
+                GDN_TRACE_AT(4096 + 64 * i + 6);
+                ok = ok && mbar_wait(&bars[CONS_D], ph, ab, p.status, lim);
+                GDN_TRACE_AT(4096 + 64 * i + 7);
                 if (!ok) break;
                 if (c + 1 < c1) load_u(c + 1);
                 tc_fence_after();
@@ -412,41 +524,53 @@ __global__ void __launch_bounds__(160, 1)
                              sdesc_sw128(sbase + OFF_D + kk * 2048, 16384, 1024), id_kmn, 1);
                 }
                 umma_commit(&bars[MMA_O]);
+                GDN_TRACE_AT(4096 + 64 * i + 8);
                 ok = mbar_wait(&bars[MMA_O], ph, ab, p.status, lim);
+                GDN_TRACE_AT(4096 + 64 * i + 9);
                 if (!ok) break;
                 if (c + 1 < c1) load_ka(c + 1);
             }
         }
     } else {
         // ----------------------------------------------------------- consumers
-        const int r = tid;  // TMEM lane: token row (X, O) or d_k row (P)
+        const int r = tid;  // TMEM lane: token row (X) or d_k row (P, S^T)
         const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-        float S[128];  // row r of S^T (= column r of S), fp32
-        if (seg == 0) {
+        // initial state: S^T row r (= column r of S) into TMEM (fp32) and the fp16 operand tile
 #pragma unroll
-            for (int i = 0; i < 128; ++i) S[i] = 0.0f;
-        } else {
-            const float *src = p.Sstart + ((static_cast<size_t>(bh) * p.NS + seg) * 128 + r) * 128;
+        for (int ch = 0; ch < 4; ++ch) {
+            float v[32];
+            if (seg == 0) {
 #pragma unroll
-            for (int i = 0; i < 128; i += 4) {
-                const float4 v = *reinterpret_cast<const float4 *>(src + i);
-                S[i] = v.x; S[i + 1] = v.y; S[i + 2] = v.z; S[i + 3] = v.w;
+                for (int e = 0; e < 32; ++e) v[e] = 0.0f;
+            } else {
+                const float *src = p.Sstart + ((static_cast<size_t>(bh) * p.NS + seg) * 128 + r) * 128 + ch * 32;
+#pragma unroll
+                for (int e = 0; e < 32; e += 4) {
+                    const float4 x = *reinterpret_cast<const float4 *>(src + e);
+                    v[e] = x.x; v[e + 1] = x.y; v[e + 2] = x.z; v[e + 3] = x.w;
+                }
             }
-        }
+            tmem_st32(tmem + lane_base + TM_S + ch * 32, v);
 #pragma unroll
-        for (int c8 = 0; c8 < 16; ++c8) store_f16_chunk(sm + OFF_S, 128, r, c8, &S[c8 * 8]);
+            for (int qq = 0; qq < 4; ++qq) store_f16_chunk(sm + OFF_S, 128, r, ch * 4 + qq, &v[qq * 8]);
+        }
+        tmem_st_wait();
         fence_proxy_async();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[CONS_S]);
 
         const float *Gbh = p.G + static_cast<size_t>(bh) * p.Tp;
-        const ZT *z = static_cast<const ZT *>(p.z);
         for (int c = c0; c < c1; ++c) {
             const int i = c - c0;
             const uint32_t ph = i & 1;
             const float gC = __expf(fminf(Gbh[c * kBlk + kBlk - 1], 0.0f));
-            if (!(warp_wait(&bars[MMA_X], ph, ab, p.status, lim) && warp_wait(&bars[FULL_U], ph, ab, p.status, lim)))
-                break;
+            const bool tr = (tid == 0);
+            if (tr) GDN_TRACE_AT(4096 + 64 * i + 16);
+            if (!warp_wait(&bars[MMA_X], ph, ab, p.status, lim)) break;
+            if (tr) GDN_TRACE_AT(4096 + 64 * i + 17);
+            if (!warp_wait(&bars[FULL_U], ph, ab, p.status, lim)) break;
+            if (tr) GDN_TRACE_AT(4096 + 64 * i + 18);
             tc_fence_after();
             // Delta = U - X, row r
 #pragma unroll
@@ -471,60 +595,29 @@ __global__ void __launch_bounds__(160, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[CONS_D]);
+            if (tr) GDN_TRACE_AT(4096 + 64 * i + 19);
 
-            // S^T row r <- gC * S^T row r + P row r
+            // S^T row r <- gC * S^T row r + P row r  (state in TMEM, fp16 copy for the next MMAs)
             if (!warp_wait(&bars[MMA_P], ph, ab, p.status, lim)) break;
+            if (tr) GDN_TRACE_AT(4096 + 64 * i + 20);
             tc_fence_after();
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
-                float pv[32];
+                float pv[32], sv[32];
                 tmem_ld32(tmem + lane_base + TM_P + ch * 32, pv);
+                tmem_ld32(tmem + lane_base + TM_S + ch * 32, sv);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) S[ch * 32 + e] = fmaf(gC, S[ch * 32 + e], pv[e]);
+                for (int e = 0; e < 32; ++e) sv[e] = fmaf(gC, sv[e], pv[e]);
+                tmem_st32(tmem + lane_base + TM_S + ch * 32, sv);
 #pragma unroll
-                for (int qq = 0; qq < 4; ++qq) store_f16_chunk(sm + OFF_S, 128, r, ch * 4 + qq, &S[ch * 32 + qq * 8]);
+                for (int qq = 0; qq < 4; ++qq) store_f16_chunk(sm + OFF_S, 128, r, ch * 4 + qq, &sv[qq * 8]);
             }
+            tmem_st_wait();
             fence_proxy_async();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[CONS_S]);
-
-            // output step: y = o / sqrt(mean(o^2) + eps) * w * SiLU(z)
-            if (!warp_wait(&bars[MMA_O], ph, ab, p.status, lim)) break;
-            tc_fence_after();
-            const uint32_t tO = tmem + lane_base + TM_O + (i & 1) * 128;
-            float ss = 0.0f;
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                float ov[32];
-                tmem_ld32(tO + ch * 32, ov);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) ss = fmaf(ov[e], ov[e], ss);
-            }
-            const float rn = 1.0f / sqrtf(ss * (1.0f / 128.0f) + p.eps);
-            const int t = c * kBlk + r;
-            const bool live = t < p.T;
-            const size_t zrow = (static_cast<size_t>(b) * p.T + (live ? t : 0)) * p.tok_stride + static_cast<size_t>(h) * kD;
-            const size_t yrow = ((static_cast<size_t>(b) * p.T + (live ? t : 0)) * p.H + h) * kD;
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                float ov[32];
-                tmem_ld32(tO + ch * 32, ov);
-                if (live) {
-#pragma unroll
-                    for (int qq = 0; qq < 4; ++qq) {
-                        const int col = ch * 32 + qq * 8;
-                        float zf[8], yv[8];
-                        load8<ZT, float>(z + zrow + col, zf);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) yv[e] = ov[qq * 8 + e] * rn * p.norm_w[col + e] * silu_f(zf[e]);
-                        store_y8(p.y, p.out_kind, yrow + col, yv);
-                    }
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[CONS_O0 + (i & 1)]);
+            if (tr) GDN_TRACE_AT(4096 + 64 * i + 21);
         }
     }
 
@@ -556,26 +649,28 @@ cudaError_t launch_transfer(const ScanParams &p, const CUtensorMap &tmW, const C
 
 cudaError_t launch_combine(const ScanParams &p, cudaStream_t s) {
     dim3 grid(16, p.H, p.B);
-    gdn_combine_kernel<<<grid, 128, 0, s>>>(p);
+    gdn_combine_kernel<<<grid, 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_scan_out(const ScanParams &p, InType zt, const CUtensorMap &tmW, const CUtensorMap &tmQt,
                             const CUtensorMap &tmKt, const CUtensorMap &tmAqk, const CUtensorMap &tmU,
-                            cudaStream_t s) {
+                            const CUtensorMap &tmZ, cudaStream_t s) {
     dim3 grid(p.NS, p.H, p.B);
     if (zt == InType::F16) {
         static bool attr = false;
         cudaError_t e = set_smem(gdn_scan_out_kernel<__half>, tc::SMEM_BYTES, attr);
         if (e != cudaSuccess) return e;
-        gdn_scan_out_kernel<__half><<<grid, 160, tc::SMEM_BYTES, s>>>(p, tmW, tmQt, tmKt, tmAqk, tmU);
+        gdn_scan_out_kernel<__half><<<grid, tc::kScanThreads, tc::SMEM_BYTES, s>>>(p, tmW, tmQt, tmKt, tmAqk, tmU, tmZ);
     } else {
         static bool attr = false;
         cudaError_t e = set_smem(gdn_scan_out_kernel<__nv_bfloat16>, tc::SMEM_BYTES, attr);
         if (e != cudaSuccess) return e;
-        gdn_scan_out_kernel<__nv_bfloat16><<<grid, 160, tc::SMEM_BYTES, s>>>(p, tmW, tmQt, tmKt, tmAqk, tmU);
+        gdn_scan_out_kernel<__nv_bfloat16><<<grid, tc::kScanThreads, tc::SMEM_BYTES, s>>>(p, tmW, tmQt, tmKt, tmAqk, tmU, tmZ);
     }
     return cudaGetLastError();
 }
 
 }  // namespace gdn
+
+GDN_TRACE_EXPORT(scan)
