@@ -53,6 +53,9 @@ _lib.gdn_forward_timed.argtypes = [_vp, ctypes.POINTER(Inputs), _vp, _vp, _vp, c
 _lib.gdn_forward_timed.restype = ctypes.c_int
 _lib.gdn_forward_host.argtypes = [_vp, ctypes.POINTER(Inputs), _vp, _vp, _vp, _vp]
 _lib.gdn_forward_host.restype = ctypes.c_int
+_lib.gdn_forward_noalloc.argtypes = [_vp, ctypes.POINTER(Inputs), _vp, _vp]
+_lib.gdn_forward_noalloc.restype = ctypes.c_int
+NOALLOC_SCRATCH_BYTES = 64 << 20
 _lib.gdn_staging_bytes.argtypes = [_vp]
 _lib.gdn_staging_bytes.restype = ctypes.c_size_t
 _lib.gdn_get_device_status.argtypes = [_vp, _vp, _vp]
@@ -139,6 +142,12 @@ class Plan:
         arr = (_vp * len(events))(*events)
         _check(_lib.gdn_forward_timed(self._h, ctypes.byref(ins), y, workspace, stream, arr, len(events)),
                "gdn_forward_timed")
+
+    def forward_noalloc_raw(self, ptrs: dict, y: int, stream: int) -> None:
+        """gdn_forward_noalloc: the workspace comes from the library's fixed
+        device array instead of the caller (for callers that cannot allocate)."""
+        ins = Inputs(*[ptrs[n] for n, _ in Inputs._fields_])
+        _check(_lib.gdn_forward_noalloc(self._h, ctypes.byref(ins), y, stream), "gdn_forward_noalloc")
 
     def forward_host_raw(self, ptrs: dict, y_host: int, staging: int, workspace: int, stream: int) -> None:
         """gdn_forward_host with raw host input addresses and device staging/workspace."""

@@ -90,6 +90,8 @@ bool make_raw_map(CUtensorMap *m, const void *base, int B, int T, int Hd, long l
 }  // namespace
 
 
+size_t gdn::plan_workspace_bytes(const gdn_plan_s *plan) { return plan ? plan->ws_bytes : 0; }
+
 extern "C" {
 
 const char *gdn_status_string(gdn_status s) {

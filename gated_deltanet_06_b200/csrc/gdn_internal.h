@@ -93,3 +93,9 @@ struct OutParams {
 cudaError_t launch_output(const OutParams &p, InType zt, InType yt, cudaStream_t s);
 
 }  // namespace gdn
+
+struct gdn_plan_s;
+namespace gdn {
+// Workspace bytes a plan's forward needs (the value gdn_plan reported).
+size_t plan_workspace_bytes(const gdn_plan_s *plan);
+}  // namespace gdn

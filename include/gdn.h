@@ -136,6 +136,29 @@ size_t gdn_staging_bytes(gdn_plan_t plan);
 gdn_status gdn_forward_host(gdn_plan_t plan, const gdn_inputs *in_host, void *y_host,
                             void *staging, void *workspace, gdn_stream_t stream);
 
+/* No counterpart in the method's pages: an allocation-free variant of
+ * gdn_forward for callers that cannot allocate device memory (code running
+ * where cudaMalloc is off limits, or a caller whose device memory is all
+ * reserved by a framework and which can hand over only input and output
+ * pointers).  The workspace comes from one fixed array of
+ * GDN_NOALLOC_SCRATCH_BYTES inside the library's device image, held by every
+ * GPU that loads the library until the process exits; no cudaMalloc, cudaFree
+ * or allocating library routine is called.  Same inputs, output and result as
+ * gdn_forward.  Errors: INVALID_ARG (null plan, inputs or y, or the checks of
+ * gdn_forward), UNSUPPORTED when the plan's workspace is larger than
+ * GDN_NOALLOC_SCRATCH_BYTES (nothing is enqueued), CUDA if the array's device
+ * address cannot be looked up.  The first call on a device looks that address
+ * up (cudaGetSymbolAddress, with the device current) and caches it, so make
+ * that first call before any stream capture.  All calls on a device share the
+ * array: calls that may overlap on the GPU (unordered streams, several host
+ * threads) race on it; calls on one stream are safe.  The array keeps the last
+ * call's contents; the only value that must start at zero, the device status
+ * word, is cleared at the start of every call.  Device-side status is not
+ * readable through this entry point (it has no workspace pointer to pass to
+ * gdn_get_device_status). */
+#define GDN_NOALLOC_SCRATCH_BYTES (64ull << 20)
+gdn_status gdn_forward_noalloc(gdn_plan_t plan, const gdn_inputs *in, void *y, gdn_stream_t stream);
+
 /* Synchronise `stream`, then read and clear the device status word in the
  * workspace.  Returns GDN_OK, GDN_ERR_TIMEOUT or GDN_ERR_DEVICE_CHECK (or
  * GDN_ERR_CUDA if the synchronisation itself failed). */
