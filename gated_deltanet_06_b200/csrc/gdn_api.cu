@@ -73,14 +73,15 @@ bool make_tile_map(CUtensorMap *m, void *base, unsigned long long rows) {
 }
 
 // Raw activations [B][T][H*d] (token stride tok_stride elements), 16-bit,
-// loaded as {64 channels, 131 tokens, 1} boxes without swizzle.
-bool make_raw_map(CUtensorMap *m, const void *base, int B, int T, int Hd, long long tok_stride, int box_rows) {
+// loaded as {box_cols channels, box_rows tokens, 1} boxes without swizzle.
+bool make_raw_map(CUtensorMap *m, const void *base, int B, int T, int Hd, long long tok_stride, int box_rows,
+                  int box_cols) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(Hd), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(B)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(tok_stride) * 2,
                                    static_cast<cuuint64_t>(tok_stride) * 2 * static_cast<cuuint64_t>(T)};
-    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1};
     const cuuint32_t es[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void *>(base), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -280,9 +281,9 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
     pp.wait_limit_ns = kWaitLimitNs;
     if (plan->tensor) {
         CUtensorMap rq, rk, rv;
-        if (!make_raw_map(&rq, in->q, c.B, c.T, c.H * d, plan->tok_stride, kBlk + 3) ||
-            !make_raw_map(&rk, in->k, c.B, c.T, c.H * d, plan->tok_stride, kBlk + 3) ||
-            !make_raw_map(&rv, in->v, c.B, c.T, c.H * d, plan->tok_stride, kBlk + 3))
+        if (!make_raw_map(&rq, in->q, c.B, c.T, c.H * d, plan->tok_stride, 64 + 3, 128) ||
+            !make_raw_map(&rk, in->k, c.B, c.T, c.H * d, plan->tok_stride, 64 + 3, 128) ||
+            !make_raw_map(&rv, in->v, c.B, c.T, c.H * d, plan->tok_stride, 64 + 3, 128))
             return GDN_ERR_CUDA;
         if (!mark() || launch_prep_tma(pp, in_type(c.in_dtype), rq, rk, rv, s) != cudaSuccess) return GDN_ERR_CUDA;
     } else if (!mark() || launch_prep(pp, in_type(c.in_dtype), false, s) != cudaSuccess) {
@@ -325,7 +326,7 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
             if (!mark() || launch_combine(sp, s) != cudaSuccess) return GDN_ERR_CUDA;
         }
         CUtensorMap tmZ;
-        if (!make_raw_map(&tmZ, in->z, c.B, c.T, c.H * d, plan->tok_stride, kBlk)) return GDN_ERR_CUDA;
+        if (!make_raw_map(&tmZ, in->z, c.B, c.T, c.H * d, plan->tok_stride, kBlk, 128)) return GDN_ERR_CUDA;
         if (!mark() || launch_scan_out(sp, in_type(c.in_dtype), tmW, tmQt, tmKt, tmAqk, tmU, tmZ, s) != cudaSuccess)
             return GDN_ERR_CUDA;
         if (!mark()) return GDN_ERR_CUDA;

@@ -15,38 +15,46 @@
 // and stores W, U, Kt, Qt, Aqk (fp16) for the inter-block scan with TMA bulk
 // stores.  Only exponentials of non-positive differences of the cumulative
 // log decay G are taken.  Two warp groups work side by side: warps 0-3 build
-// L and solve for T (thread j owns column j of T), warps 4-7 build Aqk and Qt
-// meanwhile.  Every operand the threads build is written in the 128B-swizzled
-// layout the UMMA descriptors and the TMA read directly, one contiguous row
-// per thread: T enters the W/U products transposed (MN-major), which is why
-// the off-diagonal block is formed as T_21^T.
+// L and solve for T (thread j owns column j of T), warps 4-7 build Qt and
+// Aqk meanwhile.  Every operand the threads build is written in the
+// 128B-swizzled layout the UMMA descriptors and the TMA read directly, one
+// contiguous row per thread: T enters the W/U products transposed (MN-major),
+// which is why the off-diagonal block is formed as T_21^T.
+//
+// Footprint: about 108 KB of shared memory and 256 TMEM columns, so that two
+// CTAs share an SM and one's tensor and memory phases hide the other's
+// thread phases.  Shared memory is reused through the block's life: the Q tile
+// becomes Qt, then the staging area of Aqk, then the V tile, then the staging
+// area of U; the L blocks become the merge operands, then the transposed T.
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 
 namespace gdn {
 namespace {
 
+constexpr int LD_STRIDE = 68;  // fp32 row stride of the L blocks (padded: rows written by different threads
+                               // land in different banks)
 // Shared-memory map (offsets from a 1024-byte aligned base).
-constexpr uint32_t OFF_K = 0;              // 128x128 fp16 panel tile (TMA): K, later Kt
-constexpr uint32_t OFF_V = 32768;          // 128x128 fp16 panel tile (TMA): V
-constexpr uint32_t OFF_Q = 65536;          // 128x128 fp16 panel tile (TMA): Q, later Qt
-constexpr uint32_t OFF_UNION = 98304;      // 80 KB, reused between phases:
-constexpr uint32_t OFF_LD1 = OFF_UNION + 0;       //   fp32 64x64, L diagonal block 1
-constexpr uint32_t OFF_LD2 = OFF_UNION + 16384;   //   fp32 64x64, L diagonal block 2
-constexpr uint32_t OFF_LH = OFF_UNION + 32768;    //   fp16 128 rows x 64: L[:, 0:64], K-major A
-constexpr uint32_t OFF_AQK = OFF_UNION + 49152;   //   fp16 128x128 Aqk staging for its bulk store
-constexpr uint32_t OFF_T1 = OFF_UNION + 49152;    //   fp16 64 x 64: T_1^T, K-major B   (after the Aqk store read)
-constexpr uint32_t OFF_T2T = OFF_UNION + 57344;   //   fp16 64 x 64: T_2^T, MN-major B
-constexpr uint32_t OFF_PA = OFF_UNION + 65536;    //   fp16 64 rows x 128: [P | 0], MN-major A (M padded to 128)
-constexpr uint32_t OFF_A1 = OFF_UNION + 0;        //   fp16 128x128 (T diag(beta e^G))^T, MN-major A; then W staging
-constexpr uint32_t OFF_A2 = OFF_UNION + 32768;    //   fp16 128x128 (T diag(beta))^T, MN-major A; then U staging
-constexpr uint32_t OFF_G = OFF_UNION + 81920;     // fp32 [128]
-constexpr uint32_t OFF_BETA = OFF_G + 512;        // fp32 [128]
-constexpr uint32_t OFF_BAR = OFF_BETA + 512;      // 2 mbarriers, tmem slot, abort flag
+constexpr uint32_t OFF_K = 0;              // 128x128 fp16 panel tile (TMA): K; later Kt
+constexpr uint32_t OFF_QV = 32768;         // 128x128 fp16: Q -> Qt -> Aqk staging -> V (TMA) -> U staging
+constexpr uint32_t OFF_LD = 65536;         // fp32 64 x 68 L_11 then 64 x 68 L_22 (34816 B); later:
+constexpr uint32_t OFF_T1 = OFF_LD + 0;            //   fp16 64 x 64: T_1^T, K-major B
+constexpr uint32_t OFF_T2T = OFF_LD + 8192;        //   fp16 64 x 64: T_2^T, MN-major B
+constexpr uint32_t OFF_PA = OFF_LD + 16384;        //   fp16 64 rows x 128: [P | 0], MN-major A
+constexpr uint32_t OFF_A = OFF_LD + 0;             //   fp16 128x128 transposed T (scaled), MN-major A; then W staging
+constexpr uint32_t OFF_L21 = OFF_LD + 34816;       // fp16 64 x 64: L_21 rows, K-major
+// The P = L_21 T_1 product reads a 128-row A operand starting 64 rows before L_21: its upper half
+// is whatever the bytes there are, and the rows of the product it feeds are never read.
+constexpr uint32_t OFF_LHA = OFF_L21 - 8192;
+constexpr uint32_t OFF_G = OFF_L21 + 8192;         // fp32 [128]
+constexpr uint32_t OFF_BETA = OFF_G + 512;         // fp32 [128]
+constexpr uint32_t OFF_BAR = OFF_BETA + 512;       // 2 mbarriers, tmem slot, abort flag
 constexpr uint32_t SMEM_USED = OFF_BAR + 32;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
+static_assert(OFF_LHA % 1024 == 0 && OFF_L21 % 1024 == 0 && OFF_PA % 1024 == 0, "swizzle atoms need 1 KB alignment");
+static_assert(SMEM_BYTES * 2 <= 227 * 1024, "two CTAs per SM");
 
-constexpr uint32_t TM_AKK = 0, TM_QK = 128, TM_Y = 256, TM_D2 = 320, TM_W = 0, TM_U = 128;
+constexpr uint32_t TM_AKK = 0, TM_QK = 128, TM_Y = 0, TM_D2 = 64, TM_U = 128, TM_W = 0;  // 256 columns
 
 __device__ __forceinline__ void put8(uint8_t *tile, int rows, int r, int chunk16, const float *v) {
     uint4 u;
@@ -60,7 +68,34 @@ __device__ __forceinline__ void put8(uint8_t *tile, int rows, int r, int chunk16
 // named barrier for one warp group (128 threads); id 1 or 2
 __device__ __forceinline__ void group_sync(int id) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
 
-__global__ void __launch_bounds__(256, 1)
+// Transposed, column-scaled T as an MN-major A operand: row j holds T[0..127][j] * s_j.
+// Thread j (warps 0-3) owns column j: T_1 / T_2 entries are in col[], the T_21 entries
+// (j < 64) in TMEM lane j as -D2.
+__device__ __forceinline__ void build_tT(uint8_t *dst, int j, const float (&col)[64], float s, uint32_t tD2) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        float lo[8], hi[8];
+        if (j < 64) {
+            float d[8];
+            tmem_ld8(tD2 + c * 8, d);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                lo[e] = col[c * 8 + e] * s;
+                hi[e] = -d[e] * s;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                lo[e] = 0.0f;
+                hi[e] = col[c * 8 + e] * s;
+            }
+        }
+        put8(dst, 128, j, c, lo);
+        put8(dst, 128, j, 8 + c, hi);
+    }
+}
+
+__global__ void __launch_bounds__(256, 2)
     gdn_chunk_kernel(const ChunkParams p, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmU,
@@ -78,7 +113,7 @@ __global__ void __launch_bounds__(256, 1)
 
     const int blk = blockIdx.x, bh = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5;
-    const bool groupL = tid < 128;  // warps 0-3: L and T;  warps 4-7: Aqk, Qt
+    const bool groupL = tid < 128;  // warps 0-3: L and T;  warps 4-7: Qt, Aqk
     const int r = tid & 127;        // TMEM lane / row (or T column) owned by this thread
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const size_t row0 = static_cast<size_t>(bh) * p.Tp + static_cast<size_t>(blk) * kBlk;
@@ -91,7 +126,7 @@ __global__ void __launch_bounds__(256, 1)
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(tmem_slot, 512);
+        tmem_alloc(tmem_slot, 256);
         tmem_relinquish();
     }
     if (groupL) {
@@ -106,13 +141,11 @@ __global__ void __launch_bounds__(256, 1)
     float col[64];
 
     if (tid == 0) {
-        mbar_arrive_expect_tx(bar_load, 3u * 32768u);
+        mbar_arrive_expect_tx(bar_load, 2u * 32768u);
         tma_load_2d(sm + OFF_K, &tmK, bar_load, 0, y0);
         tma_load_2d(sm + OFF_K + 16384, &tmK, bar_load, 64, y0);
-        tma_load_2d(sm + OFF_V, &tmV, bar_load, 0, y0);
-        tma_load_2d(sm + OFF_V + 16384, &tmV, bar_load, 64, y0);
-        tma_load_2d(sm + OFF_Q, &tmQ, bar_load, 0, y0);
-        tma_load_2d(sm + OFF_Q + 16384, &tmQ, bar_load, 64, y0);
+        tma_load_2d(sm + OFF_QV, &tmQ, bar_load, 0, y0);
+        tma_load_2d(sm + OFF_QV + 16384, &tmQ, bar_load, 64, y0);
     }
     if (tid == 0) GDN_TRACE_AT(0);
     mbar_wait(bar_load, 0, ab, p.status, p.wait_limit_ns);
@@ -129,7 +162,7 @@ __global__ void __launch_bounds__(256, 1)
             const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
             const uint64_t dk = sdesc_sw128(sbase + OFF_K + koff, 16, 1024);
             umma_f16(tmem + TM_AKK, dk, dk, idesc, kk > 0);
-            umma_f16(tmem + TM_QK, sdesc_sw128(sbase + OFF_Q + koff, 16, 1024), dk, idesc, kk > 0);
+            umma_f16(tmem + TM_QK, sdesc_sw128(sbase + OFF_QV + koff, 16, 1024), dk, idesc, kk > 0);
         }
         umma_commit(bar_mma);
     }
@@ -140,10 +173,10 @@ __global__ void __launch_bounds__(256, 1)
     tc_fence_after();
 
     if (groupL) {
-        // ---- L row r: fp32 diagonal blocks for the solves, fp16 left half for P = L_21 T_1
+        // ---- L row r: fp32 diagonal blocks for the solves; fp16 L_21 rows for P = L_21 T_1
         const float Gr = sG[r], br = sBeta[r];
-        float *Ld1 = reinterpret_cast<float *>(sm + OFF_LD1);
-        float *Ld2 = reinterpret_cast<float *>(sm + OFF_LD2);
+        float *Ld1 = reinterpret_cast<float *>(sm + OFF_LD);
+        float *Ld2 = Ld1 + 64 * LD_STRIDE;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
             float a[32];
@@ -158,15 +191,16 @@ __global__ void __launch_bounds__(256, 1)
                 if (r < 64) {
 #pragma unroll
                     for (int i = 0; i < 32; i += 4)
-                        *reinterpret_cast<float4 *>(Ld1 + r * 64 + c * 32 + i) =
+                        *reinterpret_cast<float4 *>(Ld1 + r * LD_STRIDE + c * 32 + i) =
                             make_float4(l[i], l[i + 1], l[i + 2], l[i + 3]);
-                }
+                } else {
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) put8(sm + OFF_LH, 128, r, c * 4 + q4, &l[q4 * 8]);
+                    for (int q4 = 0; q4 < 4; ++q4) put8(sm + OFF_LHA, 128, r, c * 4 + q4, &l[q4 * 8]);
+                }
             } else if (r >= 64) {
 #pragma unroll
                 for (int i = 0; i < 32; i += 4)
-                    *reinterpret_cast<float4 *>(Ld2 + (r - 64) * 64 + (c - 2) * 32 + i) =
+                    *reinterpret_cast<float4 *>(Ld2 + (r - 64) * LD_STRIDE + (c - 2) * 32 + i) =
                         make_float4(l[i], l[i + 1], l[i + 2], l[i + 3]);
             }
         }
@@ -177,13 +211,13 @@ __global__ void __launch_bounds__(256, 1)
         //      four independent partial sums per row keep the FMA pipe busy
         {
             const int i = r & 63;
-            const float *Ld = reinterpret_cast<const float *>(sm + (r < 64 ? OFF_LD1 : OFF_LD2));
+            const float *Ld = r < 64 ? Ld1 : Ld2;
 #pragma unroll
             for (int rr = 0; rr < 64; ++rr) {
                 float a0 = (rr == i) ? 1.0f : 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
 #pragma unroll
                 for (int j4 = 0; j4 < rr; j4 += 4) {
-                    const float4 l = *reinterpret_cast<const float4 *>(Ld + rr * 64 + j4);
+                    const float4 l = *reinterpret_cast<const float4 *>(Ld + rr * LD_STRIDE + j4);
                     a0 = fmaf(-l.x, col[j4], a0);
                     if (j4 + 1 < rr) a1 = fmaf(-l.y, col[j4 + 1], a1);
                     if (j4 + 2 < rr) a2 = fmaf(-l.z, col[j4 + 2], a2);
@@ -194,24 +228,13 @@ __global__ void __launch_bounds__(256, 1)
         }
         if (tid == 0) GDN_TRACE_AT(3);
     } else {
-        // ---- Aqk row r (staged for a bulk store); Qt = e^G Q over the Q tile in place
+        // ---- Qt = e^G Q over the Q tile in place -> bulk store; then Aqk rows staged in the
+        //      same area -> bulk store; then the V tile is loaded into it
         const float Gr = sG[r];
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-            float a[32];
-            tmem_ld32(tmem + lane_base + TM_QK + c * 32, a);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int j = c * 32 + i;
-                a[i] = (j <= r) ? __expf(fminf(Gr - sG[j], 0.0f)) * a[i] : 0.0f;
-            }
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) put8(sm + OFF_AQK, 128, r, c * 4 + q4, &a[q4 * 8]);
-        }
         const float fq = __expf(fminf(Gr, 0.0f));
 #pragma unroll 4
         for (int c = 0; c < 16; ++c) {
-            uint4 *pq = reinterpret_cast<uint4 *>(sm + OFF_Q + tile_off(128, r, c));
+            uint4 *pq = reinterpret_cast<uint4 *>(sm + OFF_QV + tile_off(128, r, c));
             const uint4 uq = *pq;
             const uint32_t wq[4] = {uq.x, uq.y, uq.z, uq.w};
             uint32_t oq[4];
@@ -225,19 +248,41 @@ __global__ void __launch_bounds__(256, 1)
         fence_proxy_async();
         group_sync(2);
         if (tid == 128) {
-            tma_store_2d(&tmAqk, sm + OFF_AQK, 0, y0);
-            tma_store_2d(&tmAqk, sm + OFF_AQK + 16384, 64, y0);
-            tma_store_2d(&tmQt, sm + OFF_Q, 0, y0);
-            tma_store_2d(&tmQt, sm + OFF_Q + 16384, 64, y0);
+            tma_store_2d(&tmQt, sm + OFF_QV, 0, y0);
+            tma_store_2d(&tmQt, sm + OFF_QV + 16384, 64, y0);
             bulk_commit();
-            bulk_wait_read_all();  // the Aqk staging area is reused below
+            bulk_wait_read_all();
+        }
+        group_sync(2);
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+            float a[32];
+            tmem_ld32(tmem + lane_base + TM_QK + c * 32, a);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int j = c * 32 + i;
+                a[i] = (j <= r) ? __expf(fminf(Gr - sG[j], 0.0f)) * a[i] : 0.0f;
+            }
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) put8(sm + OFF_QV, 128, r, c * 4 + q4, &a[q4 * 8]);
+        }
+        fence_proxy_async();
+        group_sync(2);
+        if (tid == 128) {
+            tma_store_2d(&tmAqk, sm + OFF_QV, 0, y0);
+            tma_store_2d(&tmAqk, sm + OFF_QV + 16384, 64, y0);
+            bulk_commit();
+            bulk_wait_read_all();
+            mbar_arrive_expect_tx(bar_load, 32768u);
+            tma_load_2d(sm + OFF_QV, &tmV, bar_load, 0, y0);
+            tma_load_2d(sm + OFF_QV + 16384, &tmV, bar_load, 64, y0);
         }
     }
     tc_fence_before();
     __syncthreads();
     if (tid == 0) GDN_TRACE_AT(4);
 
-    // ---- merge: Y = L[:, 0:64] T_1 (rows 64..127 are P = L_21 T_1), then T_21^T = -P^T T_2^T
+    // ---- merge: Y = [. ; L_21] T_1 (rows 64..127 are P = L_21 T_1), then T_21^T = -P^T T_2^T
     if (groupL && r < 64) {  // T_1^T as the K-major B operand: row i = column i of T_1
 #pragma unroll
         for (int c = 0; c < 8; ++c) put8(sm + OFF_T1, 64, r, c, &col[c * 8]);
@@ -249,7 +294,7 @@ __global__ void __launch_bounds__(256, 1)
         const uint32_t idesc = idesc_f16_f32(128, 64, false, false);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-            umma_f16(tmem + TM_Y, sdesc_sw128(sbase + OFF_LH + kk * 32, 16, 1024),
+            umma_f16(tmem + TM_Y, sdesc_sw128(sbase + OFF_LHA + kk * 32, 16, 1024),
                      sdesc_sw128(sbase + OFF_T1 + kk * 32, 16, 1024), idesc, kk > 0);
         umma_commit(bar_mma);
     }
@@ -295,61 +340,56 @@ __global__ void __launch_bounds__(256, 1)
     tc_fence_after();
     if (tid == 0) GDN_TRACE_AT(5);
 
-    // ---- A1 = (T diag(beta e^G))^T and A2 = (T diag(beta))^T as MN-major A operands:
-    //      row j holds column j of T (rows r = 0..127 along M), scaled by s_j
+    // ---- U = T diag(beta) V: A = (T diag(beta))^T (MN-major), B = the V tile (MN-major)
+    if (groupL) build_tT(sm + OFF_A, r, col, sBeta[r], tmem + lane_base + TM_D2);
+    fence_proxy_async();
+    tc_fence_before();
+    mbar_wait(bar_load, 1, ab, p.status, p.wait_limit_ns);  // the V tile
+    __syncthreads();
+    if (ab->flag) goto teardown;
+    if (tid == 0) GDN_TRACE_AT(6);
+    if (tid == 0) {
+        tc_fence_after();
+        const uint32_t idesc = idesc_f16_f32(128, 128, true, true);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+            umma_f16(tmem + TM_U, sdesc_sw128(sbase + OFF_A + kk * 2048, 16384, 1024),
+                     sdesc_sw128(sbase + OFF_QV + kk * 2048, 16384, 1024), idesc, kk > 0);
+        umma_commit(bar_mma);
+    }
+    mbar_wait(bar_mma, mma_phase, ab, p.status, p.wait_limit_ns);
+    mma_phase ^= 1;
+    __syncthreads();
+    if (ab->flag) goto teardown;
+    tc_fence_after();
+    // ---- W = T diag(beta e^G) K: rebuild the A tile with the other scaling; U rows -> staging
     if (groupL) {
-        const int j = r;
-        const float s2 = sBeta[j];
-        const float s1 = s2 * __expf(fminf(sG[j], 0.0f));
-        float hi[64];  // T[64..127][j]
-        if (j < 64) {
+        build_tT(sm + OFF_A, r, col, sBeta[r] * __expf(fminf(sG[r], 0.0f)), tmem + lane_base + TM_D2);
+    } else {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+            float a[32];
+            tmem_ld32(tmem + lane_base + TM_U + c * 32, a);
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                float a[32];
-                tmem_ld32(tmem + lane_base + TM_D2 + c * 32, a);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) hi[c * 32 + e] = -a[e];
-            }
-        } else {
-#pragma unroll
-            for (int e = 0; e < 64; ++e) {
-                hi[e] = col[e];
-                col[e] = 0.0f;  // T[0..63][j] = 0 for j >= 64
-            }
-        }
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            float v1[8], v2[8], w1[8], w2[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                v1[e] = col[c * 8 + e] * s1;
-                v2[e] = col[c * 8 + e] * s2;
-                w1[e] = hi[c * 8 + e] * s1;
-                w2[e] = hi[c * 8 + e] * s2;
-            }
-            put8(sm + OFF_A1, 128, j, c, v1);
-            put8(sm + OFF_A2, 128, j, c, v2);
-            put8(sm + OFF_A1, 128, j, 8 + c, w1);
-            put8(sm + OFF_A2, 128, j, 8 + c, w2);
+            for (int q4 = 0; q4 < 4; ++q4) put8(sm + OFF_QV, 128, r, c * 4 + q4, &a[q4 * 8]);
         }
     }
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) GDN_TRACE_AT(6);
-    // ---- W = T diag(beta e^G) K, U = T diag(beta) V  (A = the transposed tiles above, B = the
-    //      K and V tiles; both read MN-major: K index = token j)
     if (tid == 0) {
         tc_fence_after();
         const uint32_t idesc = idesc_f16_f32(128, 128, true, true);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            umma_f16(tmem + TM_W, sdesc_sw128(sbase + OFF_A1 + kk * 2048, 16384, 1024),
+        for (int kk = 0; kk < 8; ++kk)
+            umma_f16(tmem + TM_W, sdesc_sw128(sbase + OFF_A + kk * 2048, 16384, 1024),
                      sdesc_sw128(sbase + OFF_K + kk * 2048, 16384, 1024), idesc, kk > 0);
-            umma_f16(tmem + TM_U, sdesc_sw128(sbase + OFF_A2 + kk * 2048, 16384, 1024),
-                     sdesc_sw128(sbase + OFF_V + kk * 2048, 16384, 1024), idesc, kk > 0);
-        }
         umma_commit(bar_mma);
+    }
+    if (tid == 128) {
+        tma_store_2d(&tmU, sm + OFF_QV, 0, y0);
+        tma_store_2d(&tmU, sm + OFF_QV + 16384, 64, y0);
+        bulk_commit();
     }
     mbar_wait(bar_mma, mma_phase, ab, p.status, p.wait_limit_ns);
     mma_phase ^= 1;
@@ -358,14 +398,16 @@ __global__ void __launch_bounds__(256, 1)
     tc_fence_after();
     if (tid == 0) GDN_TRACE_AT(7);
     if (groupL) {
-        // W row r -> A1 area (free now); Kt = e^(G_last - G) K over the K tile in place
+        // W row r -> the A area (free now)
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
             float a[32];
             tmem_ld32(tmem + lane_base + TM_W + c * 32, a);
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) put8(sm + OFF_A1, 128, r, c * 4 + q4, &a[q4 * 8]);
+            for (int q4 = 0; q4 < 4; ++q4) put8(sm + OFF_A, 128, r, c * 4 + q4, &a[q4 * 8]);
         }
+    } else {
+        // Kt = e^(G_last - G) K over the K tile in place
         const float fk = __expf(fminf(sG[kBlk - 1] - sG[r], 0.0f));
 #pragma unroll 4
         for (int c = 0; c < 16; ++c) {
@@ -380,23 +422,12 @@ __global__ void __launch_bounds__(256, 1)
             }
             *pk = make_uint4(o4[0], o4[1], o4[2], o4[3]);
         }
-    } else {
-        // U row r -> A2 area
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-            float a[32];
-            tmem_ld32(tmem + lane_base + TM_U + c * 32, a);
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) put8(sm + OFF_A2, 128, r, c * 4 + q4, &a[q4 * 8]);
-        }
     }
     fence_proxy_async();
     __syncthreads();
     if (tid == 0) {
-        tma_store_2d(&tmW, sm + OFF_A1, 0, y0);
-        tma_store_2d(&tmW, sm + OFF_A1 + 16384, 64, y0);
-        tma_store_2d(&tmU, sm + OFF_A2, 0, y0);
-        tma_store_2d(&tmU, sm + OFF_A2 + 16384, 64, y0);
+        tma_store_2d(&tmW, sm + OFF_A, 0, y0);
+        tma_store_2d(&tmW, sm + OFF_A + 16384, 64, y0);
         tma_store_2d(&tmKt, sm + OFF_K, 0, y0);
         tma_store_2d(&tmKt, sm + OFF_K + 16384, 64, y0);
         bulk_commit();
@@ -409,7 +440,7 @@ teardown:
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem, 512);
+    if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
 }  // namespace

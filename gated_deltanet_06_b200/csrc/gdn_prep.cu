@@ -170,29 +170,36 @@ __global__ void __launch_bounds__(256) gdn_prep_kernel(const PrepParams p) {
     }
 }
 
-// Tensor-path variant (16-bit inputs, d = 128): one thread issues TMA loads of
-// the three raw 131-token x 128-channel tiles (3 tokens of conv history; rows
-// before t = 0 of the batch item and past T come back as zeros from the
-// tensor map's out-of-bounds fill), and all 256 threads then work out of
-// shared memory.  About 100 KB of shared memory per CTA keeps two CTAs, i.e.
-// two whole tiles of loads, in flight per SM.
-constexpr int kRawRows = kBlk + 3;
-constexpr uint32_t kRawHalf = kRawRows * 128;  // bytes of one {64 ch, 131 tok} box
-constexpr uint32_t kPrepSmem = 6 * kRawHalf + 64 + 128;
+// Tensor-path variant (16-bit inputs, d = 128).  One CTA prepares 64 tokens
+// of one (b, h): one thread issues TMA loads of the three raw 67-token x
+// 128-channel tiles (3 tokens of conv history; rows before t = 0 of the batch
+// item and past T come back as zeros from the tensor map's out-of-bounds
+// fill), the conv weights are staged in shared memory meanwhile, and all 256
+// threads then work out of shared memory.  About 58 KB of shared memory and
+// at most 85 registers per thread keep three CTAs in flight per SM.  The gates
+// of the whole 128-token block are evaluated by both of its halves (the
+// in-block cumulative sum needs the first half), each storing its own half.
+constexpr int kPrepTok = 64;
+constexpr int kRawRows = kPrepTok + 3;
+constexpr uint32_t kRawTile = kRawRows * 256;          // bytes of one {128 ch, 67 tok} box (256-byte rows)
+constexpr uint32_t kPrepW = 3 * 128 * 16;              // conv weights of q, k, v for one head (fp32)
+constexpr uint32_t kPrepSmem = 3 * kRawTile + kPrepW + 64 + 128;
 
 template <typename InT>
-__global__ void __launch_bounds__(256, 2)
+__global__ void __launch_bounds__(256, 3)
     gdn_prep_tma_kernel(const PrepParams p, const __grid_constant__ CUtensorMap tmq,
                         const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
-    constexpr int D = 128, CPR = 16, RPT = 8;
+    constexpr int D = 128, CPR = 16, RPT = 4;
     extern __shared__ __align__(128) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + 6 * kRawHalf);
+    float4 *sW = reinterpret_cast<float4 *>(sm + 3 * kRawTile);  // [3][128] taps
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + 3 * kRawTile + kPrepW);
     float *warp_tot = reinterpret_cast<float *>(bar + 1);
     __shared__ AbortState ab;
 
-    const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int t0 = blk * kBlk;
+    const int part = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int t0 = part * kPrepTok;          // first token of this CTA
+    const int tb = t0 & ~(kBlk - 1);         // first token of its 128-token block
     const int tid = threadIdx.x;
     const size_t bh = static_cast<size_t>(b) * p.H + h;
     if (tid == 0) {
@@ -201,26 +208,36 @@ __global__ void __launch_bounds__(256, 2)
         fence_mbar_init();
     }
     __syncthreads();
+    if (tid == 0) GDN_TRACE_AT(0);
     if (tid == 0) {
-        mbar_arrive_expect_tx(bar, 6 * kRawHalf);
+        mbar_arrive_expect_tx(bar, 3 * kRawTile);
         const CUtensorMap *maps[3] = {&tmq, &tmk, &tmv};
         for (int w = 0; w < 3; ++w)
-            for (int hf = 0; hf < 2; ++hf)
-                asm volatile(
-                    "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
-                        smem_u32(sm + (w * 2 + hf) * kRawHalf)),
-                    "l"(maps[w]), "r"(smem_u32(bar)), "r"(h * D + hf * 64), "r"(t0 - 3), "r"(b)
-                    : "memory");
+            asm volatile(
+                "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
+                    smem_u32(sm + w * kRawTile)),
+                "l"(maps[w]), "r"(smem_u32(bar)), "r"(h * D), "r"(t0 - 3), "r"(b)
+                : "memory");
     }
-    // gates and the in-block cumulative log decay while the tiles land
-    float la = 0.0f, be = 0.0f;
+    // conv taps of this head into shared memory, laid out [tensor][channel-in-group][group] so
+    // that the 16 threads of a token row read 16 consecutive float4
+    for (int i = tid; i < 3 * 128; i += 256) {
+        const int which = i >> 7, ch = i & 127;
+        const float *w = which == 0 ? p.conv_q : (which == 1 ? p.conv_k : p.conv_v);
+        sW[which * 128 + (ch & 7) * 16 + (ch >> 3)] = reinterpret_cast<const float4 *>(w)[static_cast<size_t>(h) * D + ch];
+    }
+    // gates of the whole 128-token block and its in-block cumulative log decay
     {
-        const int t = t0 + tid;
+        const float eA = __expf(p.A_log[h]);
+        const float dtb = p.dt_bias[h];
+        float la = 0.0f, be = 0.0f;
+        const int t = tb + tid;
         if (tid < kBlk && t < p.T) {
             const size_t gi = (static_cast<size_t>(b) * p.T + t) * p.H + h;
-            const float xg = p.g[gi] + p.dt_bias[h];
-            la = -expf(p.A_log[h]) * softplus_f(xg);
-            be = 1.0f / (1.0f + expf(-p.b[gi]));
+            const float xg = p.g[gi] + dtb;
+            const float sp = xg > 20.0f ? xg : __logf(1.0f + __expf(xg));
+            la = -eA * sp;
+            be = __fdividef(1.0f, 1.0f + __expf(-p.b[gi]));
         }
         float cs = la;
         const int lane = tid & 31, wid = tid >> 5;
@@ -231,7 +248,7 @@ __global__ void __launch_bounds__(256, 2)
         }
         if (lane == 31) warp_tot[wid] = cs;
         __syncthreads();
-        if (tid < kBlk) {
+        if (tid >= t0 - tb && tid < t0 - tb + kPrepTok) {
             float pre = 0.0f;
             for (int i = 0; i < wid; ++i) pre += warp_tot[i];
             const size_t o = bh * p.Tp + t;
@@ -240,45 +257,43 @@ __global__ void __launch_bounds__(256, 2)
             p.log_alpha[o] = la;
         }
     }
+    if (tid == 0) GDN_TRACE_AT(1);
     const bool ok = mbar_wait(bar, 0, &ab, p.status, p.wait_limit_ns);
+    if (tid == 0) GDN_TRACE_AT(2);
     if (!__syncthreads_and(ok)) return;
 
     const int cg = tid % CPR, rg = tid / CPR;
     const int c0 = cg * 8;
     const int rbeg = rg * RPT;
-    const uint32_t coff = (cg >> 3) * kRawHalf + (cg & 7) * 16;
+    const uint32_t coff = cg * 16;
 #pragma unroll 1
     for (int which = 0; which < 3; ++which) {
-        const float *w = which == 0 ? p.conv_q : (which == 1 ? p.conv_k : p.conv_v);
         __half *out = static_cast<__half *>(which == 0 ? p.qh : (which == 1 ? p.kh : p.vh));
-        const uint8_t *tile = sm + which * 2 * kRawHalf + coff;
-        float wt[8][4];
+        const uint8_t *tile = sm + which * kRawTile + coff;
+        float4 wt[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const float4 t4 = reinterpret_cast<const float4 *>(w)[static_cast<size_t>(h) * D + c0 + c];
-            wt[c][0] = t4.x; wt[c][1] = t4.y; wt[c][2] = t4.z; wt[c][3] = t4.w;
-        }
+        for (int c = 0; c < 8; ++c) wt[c] = sW[which * 128 + c * 16 + cg];
         float win[4][8];
 #pragma unroll
-        for (int i = 0; i < 3; ++i) In8<InT>::load(reinterpret_cast<const InT *>(tile + (rbeg + i) * 128), win[i]);
+        for (int i = 0; i < 3; ++i) In8<InT>::load(reinterpret_cast<const InT *>(tile + (rbeg + i) * 256), win[i]);
 #pragma unroll
         for (int r = 0; r < RPT; ++r) {
-            In8<InT>::load(reinterpret_cast<const InT *>(tile + (rbeg + r + 3) * 128), win[(r + 3) & 3]);
+            In8<InT>::load(reinterpret_cast<const InT *>(tile + (rbeg + r + 3) * 256), win[(r + 3) & 3]);
             float u[8];
             float ss = 0.0f;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
-                float a = wt[c][0] * win[r & 3][c];
-                a = fmaf(wt[c][1], win[(r + 1) & 3][c], a);
-                a = fmaf(wt[c][2], win[(r + 2) & 3][c], a);
-                a = fmaf(wt[c][3], win[(r + 3) & 3][c], a);
+                float a = wt[c].x * win[r & 3][c];
+                a = fmaf(wt[c].y, win[(r + 1) & 3][c], a);
+                a = fmaf(wt[c].z, win[(r + 2) & 3][c], a);
+                a = fmaf(wt[c].w, win[(r + 3) & 3][c], a);
                 u[c] = silu_f(a);
                 ss = fmaf(u[c], u[c], ss);
             }
             if (which < 2) {
 #pragma unroll
                 for (int off = CPR / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-                float sc = 1.0f / sqrtf(ss + p.l2_eps);
+                float sc = rsqrtf(ss + p.l2_eps);
                 if (which == 0) sc *= p.q_scale;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) u[c] *= sc;
@@ -290,6 +305,7 @@ __global__ void __launch_bounds__(256, 2)
             }
             store8<__half>(out + (bh * p.Tp + t) * D + c0, u);
         }
+        if (tid == 0) GDN_TRACE_AT(3 + which);
     }
 }
 
@@ -308,7 +324,7 @@ cudaError_t launch_typed(const PrepParams &p, cudaStream_t s) {
 cudaError_t launch_prep_tma(const PrepParams &p, InType in, const CUtensorMap &tmq, const CUtensorMap &tmk,
                             const CUtensorMap &tmv, cudaStream_t s) {
     static bool attr_bf = false, attr_h = false;
-    dim3 grid(p.Tp / kBlk, p.H, p.B);
+    dim3 grid(p.Tp / kPrepTok, p.H, p.B);
     if (in == InType::BF16) {
         if (!attr_bf) {
             cudaError_t e = cudaFuncSetAttribute(gdn_prep_tma_kernel<__nv_bfloat16>,
@@ -341,3 +357,5 @@ cudaError_t launch_prep(const PrepParams &p, InType in, bool out_f16, cudaStream
 }
 
 }  // namespace gdn
+
+GDN_TRACE_EXPORT(prep)

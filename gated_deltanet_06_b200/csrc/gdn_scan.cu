@@ -233,24 +233,37 @@ __global__ void __launch_bounds__(288, 1)
 
 // ============================================================ combine
 // S_start(j+1)^T = P_j^T S_start(j)^T + S_loc(j)^T, sequential over j; one CTA
-// per (8-column slice of S^T, head), 256 threads: thread (t, half) owns row t
-// and 4 of the 8 columns; the P^T row is brought into registers in one round
-// trip per segment.
+// per (16-column slice of S^T, head), 256 threads: thread (t, half) owns row
+// t and 8 of the 16 columns; the two threads of a row load the P^T row in the
+// same instruction (one set of transactions), and the rows of the next
+// segment are pulled into L2 while this one is computed.
 __global__ void __launch_bounds__(256) gdn_combine_kernel(const ScanParams p) {
-    __shared__ __align__(16) float cur[128][8];
+    __shared__ __align__(16) float cur[128][16];
     const int slice = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int bh = b * p.H + h;
     const int t = threadIdx.x >> 1, half = threadIdx.x & 1;
-    const int c0 = slice * 8 + half * 4;
+    const int c0 = slice * 16 + half * 8;
     if (threadIdx.x < 128) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) cur[threadIdx.x][c] = 0.0f;
+        for (int c = 0; c < 16; ++c) cur[threadIdx.x][c] = 0.0f;
     }
     __syncthreads();
     for (int j = 0; j + 1 < p.NS; ++j) {
         const float *zrow = p.Zloc + ((static_cast<size_t>(bh) * p.NS + j) * 128 + t) * 256;
-        const float4 sl = *reinterpret_cast<const float4 *>(zrow + c0);  // S_loc^T
-        float acc[4] = {sl.x, sl.y, sl.z, sl.w};
+        if (j + 2 < p.NS) {
+            const char *nxt = reinterpret_cast<const char *>(zrow + 128 * 256) + half * 512;
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(nxt));
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(nxt + 128));
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(nxt + 256));
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(nxt + 384));
+        }
+        float acc[8];
+        {
+            const float4 s0 = *reinterpret_cast<const float4 *>(zrow + c0);  // S_loc^T
+            const float4 s1 = *reinterpret_cast<const float4 *>(zrow + c0 + 4);
+            acc[0] = s0.x; acc[1] = s0.y; acc[2] = s0.z; acc[3] = s0.w;
+            acc[4] = s1.x; acc[5] = s1.y; acc[6] = s1.z; acc[7] = s1.w;
+        }
         const float4 *prow = reinterpret_cast<const float4 *>(zrow + 128);  // P^T row t
         float4 pr[32];
 #pragma unroll
@@ -260,17 +273,24 @@ __global__ void __launch_bounds__(256) gdn_combine_kernel(const ScanParams p) {
             const float pv[4] = {pr[i4].x, pr[i4].y, pr[i4].z, pr[i4].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const float4 cv = *reinterpret_cast<const float4 *>(&cur[i4 * 4 + e][half * 4]);
-                acc[0] = fmaf(pv[e], cv.x, acc[0]);
-                acc[1] = fmaf(pv[e], cv.y, acc[1]);
-                acc[2] = fmaf(pv[e], cv.z, acc[2]);
-                acc[3] = fmaf(pv[e], cv.w, acc[3]);
+                const float4 ca = *reinterpret_cast<const float4 *>(&cur[i4 * 4 + e][half * 8]);
+                const float4 cb = *reinterpret_cast<const float4 *>(&cur[i4 * 4 + e][half * 8 + 4]);
+                acc[0] = fmaf(pv[e], ca.x, acc[0]);
+                acc[1] = fmaf(pv[e], ca.y, acc[1]);
+                acc[2] = fmaf(pv[e], ca.z, acc[2]);
+                acc[3] = fmaf(pv[e], ca.w, acc[3]);
+                acc[4] = fmaf(pv[e], cb.x, acc[4]);
+                acc[5] = fmaf(pv[e], cb.y, acc[5]);
+                acc[6] = fmaf(pv[e], cb.z, acc[6]);
+                acc[7] = fmaf(pv[e], cb.w, acc[7]);
             }
         }
         __syncthreads();
-        *reinterpret_cast<float4 *>(&cur[t][half * 4]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4 *>(&cur[t][half * 8]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4 *>(&cur[t][half * 8 + 4]) = make_float4(acc[4], acc[5], acc[6], acc[7]);
         float *dst = p.Sstart + ((static_cast<size_t>(bh) * p.NS + j + 1) * 128 + t) * 128 + c0;
         *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4 *>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
         __syncthreads();
     }
 }
@@ -285,7 +305,7 @@ constexpr int NBAR = 11;
 constexpr uint32_t OFF_NW = OFF_BAR + NBAR * 8 + 16;  // norm weight, fp32 [128]
 constexpr uint32_t SMEM_BYTES = OFF_NW + 512 + 1024;
 enum { FULL_WQ = 0, FULL_U, FULL_KA, MMA_X, MMA_P, MMA_O, CONS_D, CONS_S, CONS_O0, CONS_O1, TEST };
-constexpr int kScanThreads = 288;  // warps 0-3 state, warp 4 producer, warps 5-8 output step
+constexpr int kScanThreads = 416;  // warps 0-3 state, warp 4 producer, warps 5-12 output step
 // X and P share columns (X is read out before P is written, P before the next X);
 // the fp32 state S^T lives in TMEM; O is double-buffered (256 and 384).
 constexpr uint32_t TM_X = 0, TM_P = 0, TM_S = 128, TM_O = 256;
@@ -361,7 +381,8 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
 
     float *sNW = reinterpret_cast<float *>(sm + OFF_NW);
     if (tid == 0) {
-        for (int i = 0; i < NBAR; ++i) mbar_init(&bars[i], (i >= CONS_D && i <= CONS_O1) ? 4 : 1);
+        for (int i = 0; i < NBAR; ++i)
+            mbar_init(&bars[i], (i == CONS_D || i == CONS_S) ? 4 : ((i == CONS_O0 || i == CONS_O1) ? 8 : 1));
         ab->flag = 0;
         fence_mbar_init();
     }
@@ -376,11 +397,12 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp >= 5) {
-        // ------------------------------------------- output step (warps 5-8)
-        // y = o / sqrt(mean(o^2) + eps) * w * SiLU(z) for the block rows this
-        // warp's TMEM lane quarter holds; the z row is fetched before the
-        // accumulator is read so its latency overlaps the TMEM traffic.
-        const int q = warp & 3;
+        // ------------------------------------------ output step (warps 5-12)
+        // y = o / sqrt(mean(o^2) + eps) * w * SiLU(z): two warps per TMEM lane
+        // quarter, each for 64 of the 128 columns of its rows; the z half-row
+        // is fetched before the accumulator is read so its latency overlaps
+        // the TMEM traffic.
+        const int q = warp & 3, part = (warp - 5) >> 2;  // a warp reads only its own TMEM lane quarter
         const int r = q * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         const ZT *z = static_cast<const ZT *>(p.z);
@@ -388,11 +410,12 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
             const int i = c - c0;
             const int t = c * kBlk + r;
             const bool live = t < p.T;
-            const size_t zrow = (static_cast<size_t>(b) * p.T + (live ? t : 0)) * p.tok_stride + static_cast<size_t>(h) * kD;
-            const size_t yrow = ((static_cast<size_t>(b) * p.T + (live ? t : 0)) * p.H + h) * kD;
-            uint4 zr[16];
+            const size_t zrow = (static_cast<size_t>(b) * p.T + (live ? t : 0)) * p.tok_stride +
+                                static_cast<size_t>(h) * kD + part * 64;
+            const size_t yrow = ((static_cast<size_t>(b) * p.T + (live ? t : 0)) * p.H + h) * kD + part * 64;
+            uint4 zr[8];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) zr[k] = live ? *reinterpret_cast<const uint4 *>(z + zrow + k * 8) : make_uint4(0, 0, 0, 0);
+            for (int k = 0; k < 8; ++k) zr[k] = live ? *reinterpret_cast<const uint4 *>(z + zrow + k * 8) : make_uint4(0, 0, 0, 0);
             if (!warp_wait(&bars[MMA_O], i & 1, ab, p.status, lim)) break;
             tc_fence_after();
             const uint32_t tO = tmem + lane_base + TM_O + (i & 1) * 128;
@@ -406,17 +429,18 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
             }
             const float rn = 1.0f / sqrtf(ss * (1.0f / 128.0f) + p.eps);
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
+            for (int ch = 0; ch < 2; ++ch) {
                 float ov[32];
-                tmem_ld32(tO + ch * 32, ov);
+                tmem_ld32(tO + part * 64 + ch * 32, ov);
                 if (live) {
 #pragma unroll
                     for (int qq = 0; qq < 4; ++qq) {
-                        const int col = ch * 32 + qq * 8;
+                        const int col = ch * 32 + qq * 8;  // within this warp's 64 columns
                         float zf[8], yv[8];
                         load8<ZT, float>(reinterpret_cast<const ZT *>(&zr[ch * 4 + qq]), zf);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) yv[e] = ov[qq * 8 + e] * rn * sNW[col + e] * silu_f(zf[e]);
+                        for (int e = 0; e < 8; ++e)
+                            yv[e] = ov[qq * 8 + e] * rn * sNW[part * 64 + col + e] * silu_f(zf[e]);
                         store_y8(p.y, p.out_kind, yrow + col, yv);
                     }
                 }
@@ -458,8 +482,7 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
                 load_wq(c0);
                 load_u(c0);
                 load_ka(c0);
-                if (c0 * kBlk < p.T)
-                    for (int hf = 0; hf < 2; ++hf) tma_prefetch_3d(&tmZ, h * kD + hf * 64, c0 * kBlk, b);
+                if (c0 * kBlk < p.T) tma_prefetch_3d(&tmZ, h * kD, c0 * kBlk, b);
             }
             const uint32_t id_kmn = idesc_f16_f32(128, 128, false, true);
             const uint32_t id_mnmn = idesc_f16_f32(128, 128, true, true);
@@ -477,9 +500,8 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
                         tma_prefetch_2d(&tmAqk, hf * 64, y2);
                     }
                 }
-                if (c + 1 < c1 && (c + 1) * kBlk < p.T) {  // z rows the epilogue of block c+1 reads
-                    for (int hf = 0; hf < 2; ++hf) tma_prefetch_3d(&tmZ, h * kD + hf * 64, (c + 1) * kBlk, b);
-                }
+                if (c + 1 < c1 && (c + 1) * kBlk < p.T)  // z rows the epilogue of block c+1 reads
+                    tma_prefetch_3d(&tmZ, h * kD, (c + 1) * kBlk, b);
                 GDN_TRACE_AT(4096 + 64 * i + 0);
                 ok = mbar_wait(&bars[FULL_WQ], ph, ab, p.status, lim);
                 GDN_TRACE_AT(4096 + 64 * i + 1);
@@ -648,7 +670,7 @@ cudaError_t launch_transfer(const ScanParams &p, const CUtensorMap &tmW, const C
 }
 
 cudaError_t launch_combine(const ScanParams &p, cudaStream_t s) {
-    dim3 grid(16, p.H, p.B);
+    dim3 grid(8, p.H, p.B);
     gdn_combine_kernel<<<grid, 256, 0, s>>>(p);
     return cudaGetLastError();
 }
