@@ -299,7 +299,9 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
             !make_tile_map(&tmKt, ws + plan->off_Kt, rows) || !make_tile_map(&tmAqk, ws + plan->off_Aqk, rows))
             return GDN_ERR_CUDA;
         ChunkParams cp;
-        cp.G = G; cp.beta = beta;
+        cp.g = in->g; cp.bg = in->b; cp.A_log = in->A_log; cp.dt_bias = in->dt_bias;
+        cp.G = G; cp.beta = beta; cp.log_alpha = la;
+        cp.T = c.T; cp.H = c.H;
         cp.W = reinterpret_cast<__half *>(ws + plan->off_W);
         cp.U = reinterpret_cast<__half *>(ws + plan->off_U);
         cp.Qt = reinterpret_cast<__half *>(ws + plan->off_Qt);

@@ -48,7 +48,8 @@ constexpr uint32_t OFF_L21 = OFF_LD + 34816;       // fp16 64 x 64: L_21 rows, K
 constexpr uint32_t OFF_LHA = OFF_L21 - 8192;
 constexpr uint32_t OFF_G = OFF_L21 + 8192;         // fp32 [128]
 constexpr uint32_t OFF_BETA = OFF_G + 512;         // fp32 [128]
-constexpr uint32_t OFF_BAR = OFF_BETA + 512;       // 2 mbarriers, tmem slot, abort flag
+constexpr uint32_t OFF_WT = OFF_BETA + 512;        // fp32 [4]: per-warp totals of the gate scan
+constexpr uint32_t OFF_BAR = OFF_WT + 16;          // 2 mbarriers, tmem slot, abort flag
 constexpr uint32_t SMEM_USED = OFF_BAR + 32;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(OFF_LHA % 1024 == 0 && OFF_L21 % 1024 == 0 && OFF_PA % 1024 == 0, "swizzle atoms need 1 KB alignment");
@@ -129,17 +130,7 @@ __global__ void __launch_bounds__(256, 2)
         tmem_alloc(tmem_slot, 256);
         tmem_relinquish();
     }
-    if (groupL) {
-        sG[r] = p.G[row0 + r];
-        sBeta[r] = p.beta[row0 + r];
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    uint32_t mma_phase = 0;
-    float col[64];
-
+    __syncthreads();  // barrier init visible before the TMA below uses it
     if (tid == 0) {
         mbar_arrive_expect_tx(bar_load, 2u * 32768u);
         tma_load_2d(sm + OFF_K, &tmK, bar_load, 0, y0);
@@ -147,6 +138,42 @@ __global__ void __launch_bounds__(256, 2)
         tma_load_2d(sm + OFF_QV, &tmQ, bar_load, 0, y0);
         tma_load_2d(sm + OFF_QV + 16384, &tmQ, bar_load, 64, y0);
     }
+    if (groupL) {
+        // gates of the block while the tiles land: log alpha = -exp(A_log) softplus(g + dt_bias),
+        // beta = sigmoid(b), G = inclusive cumulative sum of log alpha over the block
+        float *warp_tot = reinterpret_cast<float *>(sm + OFF_WT);
+        const int bb = bh / p.H, hh = bh - bb * p.H;
+        const int t = blk * kBlk + r;
+        float la = 0.0f, be = 0.0f;
+        if (t < p.T) {
+            const size_t gi = (static_cast<size_t>(bb) * p.T + t) * p.H + hh;
+            const float xg = p.g[gi] + p.dt_bias[hh];
+            const float sp = xg > 20.0f ? xg : __logf(1.0f + __expf(xg));
+            la = -__expf(p.A_log[hh]) * sp;
+            be = __fdividef(1.0f, 1.0f + __expf(-p.bg[gi]));
+        }
+        float cs = la;
+        const int lane = tid & 31;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float n = __shfl_up_sync(0xffffffffu, cs, off);
+            if (lane >= off) cs += n;
+        }
+        if (lane == 31) warp_tot[warp] = cs;
+        group_sync(1);
+        for (int w = 0; w < warp; ++w) cs += warp_tot[w];
+        sG[r] = cs;
+        sBeta[r] = be;
+        p.G[row0 + r] = cs;
+        p.beta[row0 + r] = be;
+        p.log_alpha[row0 + r] = la;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    uint32_t mma_phase = 0;
+    float col[64];
     if (tid == 0) GDN_TRACE_AT(0);
     mbar_wait(bar_load, 0, ab, p.status, p.wait_limit_ns);
     if (tid == 0) GDN_TRACE_AT(1);

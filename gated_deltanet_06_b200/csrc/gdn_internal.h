@@ -34,9 +34,14 @@ cudaError_t launch_prep(const PrepParams &p, InType in, bool out_f16, cudaStream
 cudaError_t launch_prep_tma(const PrepParams &p, InType in, const CUtensorMap &tmq, const CUtensorMap &tmk,
                             const CUtensorMap &tmv, cudaStream_t s);
 
-// Intra-block UT transform on tensor cores (d = 128, fp16 operands).
+// Intra-block UT transform on tensor cores (d = 128, fp16 operands).  It
+// also evaluates the gates of its block from g, b (and writes G, beta, log
+// alpha for the scan and the stage tests).
 struct ChunkParams {
-    const float *G, *beta;          // [BH][Tp]
+    const float *g, *bg;            // [B][T][H]
+    const float *A_log, *dt_bias;   // [H]
+    float *G, *beta, *log_alpha;    // [BH][Tp]
+    int T, H;
     __half *W, *U, *Qt, *Kt, *Aqk;  // [BH][Tp][128]
     int BH, Tp, NB;
     int *status;

@@ -176,9 +176,8 @@ __global__ void __launch_bounds__(256) gdn_prep_kernel(const PrepParams p) {
 // item and past T come back as zeros from the tensor map's out-of-bounds
 // fill), the conv weights are staged in shared memory meanwhile, and all 256
 // threads then work out of shared memory.  About 58 KB of shared memory and
-// at most 85 registers per thread keep three CTAs in flight per SM.  The gates
-// of the whole 128-token block are evaluated by both of its halves (the
-// in-block cumulative sum needs the first half), each storing its own half.
+// at most 85 registers per thread keep three CTAs in flight per SM.  On this
+// path the gates are evaluated by the chunk kernel, which needs them first.
 constexpr int kPrepTok = 64;
 constexpr int kRawRows = kPrepTok + 3;
 constexpr uint32_t kRawTile = kRawRows * 256;          // bytes of one {128 ch, 67 tok} box (256-byte rows)
@@ -194,12 +193,10 @@ __global__ void __launch_bounds__(256, 3)
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     float4 *sW = reinterpret_cast<float4 *>(sm + 3 * kRawTile);  // [3][128] taps
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + 3 * kRawTile + kPrepW);
-    float *warp_tot = reinterpret_cast<float *>(bar + 1);
     __shared__ AbortState ab;
 
     const int part = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int t0 = part * kPrepTok;          // first token of this CTA
-    const int tb = t0 & ~(kBlk - 1);         // first token of its 128-token block
     const int tid = threadIdx.x;
     const size_t bh = static_cast<size_t>(b) * p.H + h;
     if (tid == 0) {
@@ -226,37 +223,7 @@ __global__ void __launch_bounds__(256, 3)
         const float *w = which == 0 ? p.conv_q : (which == 1 ? p.conv_k : p.conv_v);
         sW[which * 128 + (ch & 7) * 16 + (ch >> 3)] = reinterpret_cast<const float4 *>(w)[static_cast<size_t>(h) * D + ch];
     }
-    // gates of the whole 128-token block and its in-block cumulative log decay
-    {
-        const float eA = __expf(p.A_log[h]);
-        const float dtb = p.dt_bias[h];
-        float la = 0.0f, be = 0.0f;
-        const int t = tb + tid;
-        if (tid < kBlk && t < p.T) {
-            const size_t gi = (static_cast<size_t>(b) * p.T + t) * p.H + h;
-            const float xg = p.g[gi] + dtb;
-            const float sp = xg > 20.0f ? xg : __logf(1.0f + __expf(xg));
-            la = -eA * sp;
-            be = __fdividef(1.0f, 1.0f + __expf(-p.b[gi]));
-        }
-        float cs = la;
-        const int lane = tid & 31, wid = tid >> 5;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const float n = __shfl_up_sync(0xffffffffu, cs, off);
-            if (lane >= off) cs += n;
-        }
-        if (lane == 31) warp_tot[wid] = cs;
-        __syncthreads();
-        if (tid >= t0 - tb && tid < t0 - tb + kPrepTok) {
-            float pre = 0.0f;
-            for (int i = 0; i < wid; ++i) pre += warp_tot[i];
-            const size_t o = bh * p.Tp + t;
-            p.G[o] = cs + pre;
-            p.beta[o] = be;
-            p.log_alpha[o] = la;
-        }
-    }
+    __syncthreads();  // conv taps in shared memory
     if (tid == 0) GDN_TRACE_AT(1);
     const bool ok = mbar_wait(bar, 0, &ab, p.status, p.wait_limit_ns);
     if (tid == 0) GDN_TRACE_AT(2);

@@ -22,6 +22,8 @@
 // consumer warps own TMEM lanes (one row each) and keep the fp32 state in
 // registers.  Every hand-off is an mbarrier with a bounded wait, so a lost
 // arrival ends the kernel with a timeout status instead of a hang.
+#include <type_traits>
+
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 
@@ -398,56 +400,122 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
 
     if (warp >= 5) {
         // ------------------------------------------ output step (warps 5-12)
-        // y = o / sqrt(mean(o^2) + eps) * w * SiLU(z): two warps per TMEM lane
-        // quarter, each for 64 of the 128 columns of its rows; the z half-row
-        // is fetched before the accumulator is read so its latency overlaps
-        // the TMEM traffic.
+        // y = o / sqrt(mean(o^2) + eps) * w * SiLU(z).  Two warps per TMEM lane quarter,
+        // each for 16 rows: the accumulator is read in the 16-lane layout (a row spread
+        // over a quad of lanes), and z and y move as 16-byte pieces of a row, turned into
+        // and out of that layout by 4x4 transposes inside each quad, so that every warp
+        // access touches 8 rows x 64 contiguous bytes instead of 32 scattered rows.
         const int q = warp & 3, part = (warp - 5) >> 2;  // a warp reads only its own TMEM lane quarter
-        const int r = q * 32 + lane;
-        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+        const int quad = lane >> 2, t0 = lane & 3;
+        const int rA = q * 32 + part * 16 + quad, rB = rA + 8;  // block rows of this thread
+        const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32 + part * 16) << 16);
         const ZT *z = static_cast<const ZT *>(p.z);
         for (int c = c0; c < c1; ++c) {
             const int i = c - c0;
-            const int t = c * kBlk + r;
-            const bool live = t < p.T;
-            const size_t zrow = (static_cast<size_t>(b) * p.T + (live ? t : 0)) * p.tok_stride +
-                                static_cast<size_t>(h) * kD + part * 64;
-            const size_t yrow = ((static_cast<size_t>(b) * p.T + (live ? t : 0)) * p.H + h) * kD + part * 64;
-            uint4 zr[8];
+            const int tA = c * kBlk + rA, tB = c * kBlk + rB;
+            const bool liveA = tA < p.T, liveB = tB < p.T;
+            const size_t zA = (static_cast<size_t>(b) * p.T + (liveA ? tA : 0)) * p.tok_stride + static_cast<size_t>(h) * kD;
+            const size_t zB = (static_cast<size_t>(b) * p.T + (liveB ? tB : 0)) * p.tok_stride + static_cast<size_t>(h) * kD;
+            const size_t yA = ((static_cast<size_t>(b) * p.T + (liveA ? tA : 0)) * p.H + h) * kD;
+            const size_t yB = ((static_cast<size_t>(b) * p.T + (liveB ? tB : 0)) * p.H + h) * kD;
+            const bool tre = (warp == 5 && lane == 0);
+            if (tre) GDN_TRACE_AT(4096 + 64 * i + 32);
+            // z: lane t0 of the quad fetches columns 8(4k + t0) .. +7 of its two rows
+            uint4 za[4], zb[4];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) zr[k] = live ? *reinterpret_cast<const uint4 *>(z + zrow + k * 8) : make_uint4(0, 0, 0, 0);
-            if (!warp_wait(&bars[MMA_O], i & 1, ab, p.status, lim)) break;
-            tc_fence_after();
-            const uint32_t tO = tmem + lane_base + TM_O + (i & 1) * 128;
-            float ss = 0.0f;
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                float ov[32];
-                tmem_ld32(tO + ch * 32, ov);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) ss = fmaf(ov[e], ov[e], ss);
+            for (int k = 0; k < 4; ++k) {
+                const int col = 8 * (4 * k + t0);
+                za[k] = liveA ? *reinterpret_cast<const uint4 *>(z + zA + col) : make_uint4(0, 0, 0, 0);
+                zb[k] = liveB ? *reinterpret_cast<const uint4 *>(z + zB + col) : make_uint4(0, 0, 0, 0);
             }
-            const float rn = 1.0f / sqrtf(ss * (1.0f / 128.0f) + p.eps);
+            if (!warp_wait(&bars[MMA_O], i & 1, ab, p.status, lim)) break;
+            if (tre) GDN_TRACE_AT(4096 + 64 * i + 33);
+            tc_fence_after();
+            const uint32_t tO = tbase + TM_O + (i & 1) * 128;
+            float ssA = 0.0f, ssB = 0.0f;
+            {
+                uint32_t v[64];
+                tmem_ld16x256b_x16(tO, v);
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-                float ov[32];
-                tmem_ld32(tO + part * 64 + ch * 32, ov);
-                if (live) {
+                for (int g = 0; g < 16; ++g) {
+                    const float a0 = __uint_as_float(v[4 * g]), a1 = __uint_as_float(v[4 * g + 1]);
+                    const float b0 = __uint_as_float(v[4 * g + 2]), b1 = __uint_as_float(v[4 * g + 3]);
+                    ssA = fmaf(a0, a0, fmaf(a1, a1, ssA));
+                    ssB = fmaf(b0, b0, fmaf(b1, b1, ssB));
+                }
+            }
+            ssA += __shfl_xor_sync(0xffffffffu, ssA, 1);
+            ssA += __shfl_xor_sync(0xffffffffu, ssA, 2);
+            ssB += __shfl_xor_sync(0xffffffffu, ssB, 1);
+            ssB += __shfl_xor_sync(0xffffffffu, ssB, 2);
+            const float rnA = 1.0f / sqrtf(ssA * (1.0f / 128.0f) + p.eps);
+            const float rnB = 1.0f / sqrtf(ssB * (1.0f / 128.0f) + p.eps);
+            if (tre) GDN_TRACE_AT(4096 + 64 * i + 34);
 #pragma unroll
-                    for (int qq = 0; qq < 4; ++qq) {
-                        const int col = ch * 32 + qq * 8;  // within this warp's 64 columns
-                        float zf[8], yv[8];
-                        load8<ZT, float>(reinterpret_cast<const ZT *>(&zr[ch * 4 + qq]), zf);
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t v[32];
+                tmem_ld16x256b_x8(tO + hf * 64, v);  // groups g = 8hf .. 8hf+7
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            yv[e] = ov[qq * 8 + e] * rn * sNW[part * 64 + col + e] * silu_f(zf[e]);
-                        store_y8(p.y, p.out_kind, yrow + col, yv);
+                for (int kk = 0; kk < 2; ++kk) {
+                    const int k = 2 * hf + kk;  // groups 4k .. 4k+3
+                    uint32_t wa[4] = {za[k].x, za[k].y, za[k].z, za[k].w};
+                    uint32_t wb[4] = {zb[k].x, zb[k].y, zb[k].z, zb[k].w};
+                    quad_transpose(wa, t0);  // wa[j] = z pair (col 8(4k+j) + 2t0, +1) of row A
+                    quad_transpose(wb, t0);
+                    float yf[2][4][2];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int gl = 4 * kk + j;  // group within this half
+                        const int col = 8 * (4 * k + j) + 2 * t0;
+                        const float w0 = sNW[col], w1 = sNW[col + 1];
+                        float2 fa, fb;
+                        if constexpr (sizeof(ZT) == 2 && std::is_same<ZT, __half>::value) {
+                            fa = unpack_half2(wa[j]);
+                            fb = unpack_half2(wb[j]);
+                        } else {
+                            fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wa[j]));
+                            fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wb[j]));
+                        }
+                        yf[0][j][0] = __uint_as_float(v[4 * gl]) * rnA * w0 * silu_f(fa.x);
+                        yf[0][j][1] = __uint_as_float(v[4 * gl + 1]) * rnA * w1 * silu_f(fa.y);
+                        yf[1][j][0] = __uint_as_float(v[4 * gl + 2]) * rnB * w0 * silu_f(fb.x);
+                        yf[1][j][1] = __uint_as_float(v[4 * gl + 3]) * rnB * w1 * silu_f(fb.y);
+                    }
+                    if (p.out_kind == 1) {  // fp32: each lane stores its 8-byte pairs (a quad covers 32 bytes)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int col = 8 * (4 * k + j) + 2 * t0;
+                            if (liveA) *reinterpret_cast<float2 *>(static_cast<float *>(p.y) + yA + col) = make_float2(yf[0][j][0], yf[0][j][1]);
+                            if (liveB) *reinterpret_cast<float2 *>(static_cast<float *>(p.y) + yB + col) = make_float2(yf[1][j][0], yf[1][j][1]);
+                        }
+                    } else {  // 16-bit: back to 16-byte pieces of a row, then one 16-byte store per row
+                        uint32_t ya[4], yb[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            if (p.out_kind == 0) {
+                                __nv_bfloat162 pa = __floats2bfloat162_rn(yf[0][j][0], yf[0][j][1]);
+                                __nv_bfloat162 pb = __floats2bfloat162_rn(yf[1][j][0], yf[1][j][1]);
+                                ya[j] = *reinterpret_cast<uint32_t *>(&pa);
+                                yb[j] = *reinterpret_cast<uint32_t *>(&pb);
+                            } else {
+                                ya[j] = pack_half2(yf[0][j][0], yf[0][j][1]);
+                                yb[j] = pack_half2(yf[1][j][0], yf[1][j][1]);
+                            }
+                        }
+                        quad_transpose(ya, t0);  // ya = the 4 pairs of group 4k + t0 of row A
+                        quad_transpose(yb, t0);
+                        const int col = 8 * (4 * k + t0);
+                        uint16_t *y16 = static_cast<uint16_t *>(p.y);
+                        if (liveA) *reinterpret_cast<uint4 *>(y16 + yA + col) = make_uint4(ya[0], ya[1], ya[2], ya[3]);
+                        if (liveB) *reinterpret_cast<uint4 *>(y16 + yB + col) = make_uint4(yb[0], yb[1], yb[2], yb[3]);
                     }
                 }
             }
+            if (tre) GDN_TRACE_AT(4096 + 64 * i + 35);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[CONS_O0 + (i & 1)]);
+            if (tre) GDN_TRACE_AT(4096 + 64 * i + 36);
         }
     } else if (warp == 4) {
         // ------------------------------------------------------------ producer
