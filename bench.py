@@ -58,10 +58,10 @@ def path_flops_per_token_head(d, C=64):
 def kernel_work_per_token_head(name, d, s_in, s_out):
     """Algorithmic bytes and flops each kernel must move / do per (token, head)
     on the tensor path (fp16 intermediates, fp32 o)."""
-    if name == "prep":      # q k v in, g b in; q^ k^ v^ fp16 out; G beta log-alpha out
-        return 3 * d * s_in + 8 + 3 * d * 2 + 12, 0
-    if name == "chunk":     # q^ k^ v^ + G beta in; W U Qt Kt Aqk out; K K^T, Q K^T, W, U products
-        return 3 * d * 2 + 8 + 5 * 128 * 2, 4 * 2 * 128 * d
+    if name == "prep":      # q k v in; q^ k^ v^ fp16 out
+        return 3 * d * s_in + 3 * d * 2, 0
+    if name == "chunk":     # q^ k^ v^ + g b in; W U Qt Kt Aqk + G beta log-alpha out; K K^T, Q K^T, W, U
+        return 3 * d * 2 + 8 + 5 * 128 * 2 + 12, 4 * 2 * 128 * d
     if name == "transfer":  # W U Kt in; W [S|P]^T and Kt^T Delta with N = 2d
         return 3 * 128 * 2, 2 * 2 * 128 * 2 * d
     if name == "combine":   # per-segment states only (negligible per token)
