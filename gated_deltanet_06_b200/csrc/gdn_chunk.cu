@@ -16,16 +16,23 @@
 // stores.  Only exponentials of non-positive differences of the cumulative
 // log decay G are taken.  Two warp groups work side by side: warps 0-3 build
 // L and solve for T (thread j owns column j of T), warps 4-7 build Qt and
-// Aqk meanwhile.  Every operand the threads build is written in the
-// 128B-swizzled layout the UMMA descriptors and the TMA read directly, one
-// contiguous row per thread: T enters the W/U products transposed (MN-major),
-// which is why the off-diagonal block is formed as T_21^T.
+// Aqk and Kt meanwhile, then scale the V tile and a fresh copy of the K tile
+// into V~ = diag(beta) V and K~ = diag(beta e^G) K, so that T enters both
+// U = T V~ and W = T K~ unscaled and its operand is built once.  Every
+// operand the threads build is written in the 128B-swizzled layout the UMMA
+// descriptors and the TMA read directly, one contiguous row per thread: T
+// enters the W/U products transposed (MN-major), which is why the
+// off-diagonal block is formed as T_21^T.  The decay factors of L and Aqk
+// below the diagonal 32x32 blocks are split as e^(G_r - G_m) e^(G_m - G_j)
+// (m the last row of j's group, both exponents <= 0), one exponential per
+// row and per column instead of one per entry.
 //
 // Footprint: about 108 KB of shared memory and 256 TMEM columns, so that two
 // CTAs share an SM and one's tensor and memory phases hide the other's
 // thread phases.  Shared memory is reused through the block's life: the Q tile
-// becomes Qt, then the staging area of Aqk, then the V tile, then the staging
-// area of U; the L blocks become the merge operands, then the transposed T.
+// becomes Qt, then the staging area of Aqk, then V~, then the staging area of
+// U; the K tile becomes Kt, then K~; the L blocks become the merge operands,
+// then the transposed T, then the staging area of W.
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 
@@ -49,8 +56,9 @@ constexpr uint32_t OFF_LHA = OFF_L21 - 8192;
 constexpr uint32_t OFF_G = OFF_L21 + 8192;         // fp32 [128]
 constexpr uint32_t OFF_BETA = OFF_G + 512;         // fp32 [128]
 constexpr uint32_t OFF_WT = OFF_BETA + 512;        // fp32 [4]: per-warp totals of the gate scan
-constexpr uint32_t OFF_BAR = OFF_WT + 16;          // 2 mbarriers, tmem slot, abort flag
-constexpr uint32_t SMEM_USED = OFF_BAR + 32;
+constexpr uint32_t OFF_EC = OFF_WT + 16;           // fp32 [128]: e^(G_m - G_j), m = last row of j's 32-row group
+constexpr uint32_t OFF_BAR = OFF_EC + 512;         // 4 mbarriers, tmem slot, abort flag
+constexpr uint32_t SMEM_USED = OFF_BAR + 48;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(OFF_LHA % 1024 == 0 && OFF_L21 % 1024 == 0 && OFF_PA % 1024 == 0, "swizzle atoms need 1 KB alignment");
 static_assert(SMEM_BYTES * 2 <= 227 * 1024, "two CTAs per SM");
@@ -107,9 +115,12 @@ __global__ void __launch_bounds__(256, 2)
     const uint32_t sbase = smem_u32(sm);
     float *sG = reinterpret_cast<float *>(sm + OFF_G);
     float *sBeta = reinterpret_cast<float *>(sm + OFF_BETA);
-    uint64_t *bar_load = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
+    float *sEc = reinterpret_cast<float *>(sm + OFF_EC);
+    uint64_t *bar_load = reinterpret_cast<uint64_t *>(sm + OFF_BAR);  // K and Q tiles
     uint64_t *bar_mma = bar_load + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_load + 2);
+    uint64_t *bar_v = bar_load + 2;   // V tile
+    uint64_t *bar_kr = bar_load + 3;  // K tile again, after Kt has been stored from it
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_load + 4);
     AbortState *ab = reinterpret_cast<AbortState *>(tmem_slot + 1);
 
     const int blk = blockIdx.x, bh = blockIdx.y;
@@ -123,6 +134,8 @@ __global__ void __launch_bounds__(256, 2)
     if (tid == 0) {
         mbar_init(bar_load, 1);
         mbar_init(bar_mma, 1);
+        mbar_init(bar_v, 1);
+        mbar_init(bar_kr, 1);
         ab->flag = 0;
         fence_mbar_init();
     }
@@ -167,6 +180,10 @@ __global__ void __launch_bounds__(256, 2)
         p.G[row0 + r] = cs;
         p.beta[row0 + r] = be;
         p.log_alpha[row0 + r] = la;
+        group_sync(1);
+        // column factors of the split decay: for j in 32-row group c and r past that group,
+        // e^(G_r - G_j) = e^(G_r - G_m) e^(G_m - G_j) with m = 32c + 31, both exponents <= 0
+        sEc[r] = __expf(fminf(sG[r | 31] - cs, 0.0f));
     }
     tc_fence_before();
     __syncthreads();
@@ -200,19 +217,28 @@ __global__ void __launch_bounds__(256, 2)
     tc_fence_after();
 
     if (groupL) {
-        // ---- L row r: fp32 diagonal blocks for the solves; fp16 L_21 rows for P = L_21 T_1
+        // ---- L row r: fp32 diagonal blocks for the solves; fp16 L_21 rows for P = L_21 T_1.
+        //      Warp w owns rows 32w .. 32w+31: column group c < w lies wholly below the diagonal
+        //      (split decay, no exponential per entry), c == w holds the diagonal, c > w is zero
+        //      and never read.
         const float Gr = sG[r], br = sBeta[r];
         float *Ld1 = reinterpret_cast<float *>(sm + OFF_LD);
         float *Ld2 = Ld1 + 64 * LD_STRIDE;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c <= warp; ++c) {
             float a[32];
             tmem_ld32(tmem + lane_base + TM_AKK + c * 32, a);
             float l[32];
+            if (c < warp) {
+                const float fr = br * __expf(fminf(Gr - sG[c * 32 + 31], 0.0f));
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int j = c * 32 + i;
-                l[i] = (j < r) ? br * __expf(fminf(Gr - sG[j], 0.0f)) * a[i] : 0.0f;
+                for (int i = 0; i < 32; ++i) l[i] = fr * sEc[c * 32 + i] * a[i];
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int j = c * 32 + i;
+                    l[i] = (j < r) ? br * __expf(fminf(Gr - sG[j], 0.0f)) * a[i] : 0.0f;
+                }
             }
             if (c < 2) {
                 if (r < 64) {
@@ -224,7 +250,7 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) put8(sm + OFF_LHA, 128, r, c * 4 + q4, &l[q4 * 8]);
                 }
-            } else if (r >= 64) {
+            } else {  // c >= 2 implies r >= 64
 #pragma unroll
                 for (int i = 0; i < 32; i += 4)
                     *reinterpret_cast<float4 *>(Ld2 + (r - 64) * LD_STRIDE + (c - 2) * 32 + i) =
@@ -255,8 +281,11 @@ __global__ void __launch_bounds__(256, 2)
         }
         if (tid == 0) GDN_TRACE_AT(3);
     } else {
-        // ---- Qt = e^G Q over the Q tile in place -> bulk store; then Aqk rows staged in the
-        //      same area -> bulk store; then the V tile is loaded into it
+        // ---- Qt = e^G Q over the Q tile in place -> bulk store; Aqk rows staged in the same
+        //      area -> bulk store, then the V tile is loaded into it; Kt = e^(G_last - G) K over
+        //      the K tile in place -> bulk store, then the K tile is loaded again; finally
+        //      V~ = diag(beta) V and K~ = diag(beta e^G) K in place, the B operands of U = T V~
+        //      and W = T K~
         const float Gr = sG[r];
         const float fq = __expf(fminf(Gr, 0.0f));
 #pragma unroll 4
@@ -281,14 +310,26 @@ __global__ void __launch_bounds__(256, 2)
             bulk_wait_read_all();
         }
         group_sync(2);
+        const int w = warp & 3;  // rows 32w .. 32w+31: same split of the decay as the L rows
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
             float a[32];
-            tmem_ld32(tmem + lane_base + TM_QK + c * 32, a);
+            if (c > w) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int j = c * 32 + i;
-                a[i] = (j <= r) ? __expf(fminf(Gr - sG[j], 0.0f)) * a[i] : 0.0f;
+                for (int i = 0; i < 32; ++i) a[i] = 0.0f;
+            } else {
+                tmem_ld32(tmem + lane_base + TM_QK + c * 32, a);
+                if (c < w) {
+                    const float fr = __expf(fminf(Gr - sG[c * 32 + 31], 0.0f));
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) a[i] *= fr * sEc[c * 32 + i];
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int j = c * 32 + i;
+                        a[i] = (j <= r) ? __expf(fminf(Gr - sG[j], 0.0f)) * a[i] : 0.0f;
+                    }
+                }
             }
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) put8(sm + OFF_QV, 128, r, c * 4 + q4, &a[q4 * 8]);
@@ -300,10 +341,69 @@ __global__ void __launch_bounds__(256, 2)
             tma_store_2d(&tmAqk, sm + OFF_QV + 16384, 64, y0);
             bulk_commit();
             bulk_wait_read_all();
-            mbar_arrive_expect_tx(bar_load, 32768u);
-            tma_load_2d(sm + OFF_QV, &tmV, bar_load, 0, y0);
-            tma_load_2d(sm + OFF_QV + 16384, &tmV, bar_load, 64, y0);
+            mbar_arrive_expect_tx(bar_v, 32768u);
+            tma_load_2d(sm + OFF_QV, &tmV, bar_v, 0, y0);
+            tma_load_2d(sm + OFF_QV + 16384, &tmV, bar_v, 64, y0);
         }
+        // Kt (the K tile's last use as plain K was the A_kk product, complete before this branch)
+        const float fk = __expf(fminf(sG[kBlk - 1] - Gr, 0.0f));
+#pragma unroll 4
+        for (int c = 0; c < 16; ++c) {
+            uint4 *pk = reinterpret_cast<uint4 *>(sm + OFF_K + tile_off(128, r, c));
+            const uint4 uk = *pk;
+            const uint32_t wk[4] = {uk.x, uk.y, uk.z, uk.w};
+            uint32_t o4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 xk = unpack_half2(wk[e]);
+                o4[e] = pack_half2(xk.x * fk, xk.y * fk);
+            }
+            *pk = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        }
+        fence_proxy_async();
+        group_sync(2);
+        if (tid == 128) {
+            tma_store_2d(&tmKt, sm + OFF_K, 0, y0);
+            tma_store_2d(&tmKt, sm + OFF_K + 16384, 64, y0);
+            bulk_commit();
+            bulk_wait_read_all();
+            mbar_arrive_expect_tx(bar_kr, 32768u);
+            tma_load_2d(sm + OFF_K, &tmK, bar_kr, 0, y0);
+            tma_load_2d(sm + OFF_K + 16384, &tmK, bar_kr, 64, y0);
+        }
+        // V~ and K~, row r each
+        const float sv = sBeta[r], sk = sBeta[r] * fq;
+        if (mbar_wait(bar_v, 0, ab, p.status, p.wait_limit_ns)) {
+#pragma unroll 4
+            for (int c = 0; c < 16; ++c) {
+                uint4 *pv = reinterpret_cast<uint4 *>(sm + OFF_QV + tile_off(128, r, c));
+                const uint4 uv = *pv;
+                const uint32_t wv[4] = {uv.x, uv.y, uv.z, uv.w};
+                uint32_t o4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 xv = unpack_half2(wv[e]);
+                    o4[e] = pack_half2(xv.x * sv, xv.y * sv);
+                }
+                *pv = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+            }
+        }
+        if (mbar_wait(bar_kr, 0, ab, p.status, p.wait_limit_ns)) {
+#pragma unroll 4
+            for (int c = 0; c < 16; ++c) {
+                uint4 *pk = reinterpret_cast<uint4 *>(sm + OFF_K + tile_off(128, r, c));
+                const uint4 uk = *pk;
+                const uint32_t wk[4] = {uk.x, uk.y, uk.z, uk.w};
+                uint32_t o4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 xk = unpack_half2(wk[e]);
+                    o4[e] = pack_half2(xk.x * sk, xk.y * sk);
+                }
+                *pk = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+            }
+        }
+        fence_proxy_async();
     }
     tc_fence_before();
     __syncthreads();
@@ -367,11 +467,11 @@ __global__ void __launch_bounds__(256, 2)
     tc_fence_after();
     if (tid == 0) GDN_TRACE_AT(5);
 
-    // ---- U = T diag(beta) V: A = (T diag(beta))^T (MN-major), B = the V tile (MN-major)
-    if (groupL) build_tT(sm + OFF_A, r, col, sBeta[r], tmem + lane_base + TM_D2);
+    // ---- U = T V~ and W = T K~, one commit: A = T^T (MN-major, shared), B = the V~ / K~ tiles
+    //      (MN-major)
+    if (groupL) build_tT(sm + OFF_A, r, col, 1.0f, tmem + lane_base + TM_D2);
     fence_proxy_async();
     tc_fence_before();
-    mbar_wait(bar_load, 1, ab, p.status, p.wait_limit_ns);  // the V tile
     __syncthreads();
     if (ab->flag) goto teardown;
     if (tid == 0) GDN_TRACE_AT(6);
@@ -382,41 +482,11 @@ __global__ void __launch_bounds__(256, 2)
         for (int kk = 0; kk < 8; ++kk)
             umma_f16(tmem + TM_U, sdesc_sw128(sbase + OFF_A + kk * 2048, 16384, 1024),
                      sdesc_sw128(sbase + OFF_QV + kk * 2048, 16384, 1024), idesc, kk > 0);
-        umma_commit(bar_mma);
-    }
-    mbar_wait(bar_mma, mma_phase, ab, p.status, p.wait_limit_ns);
-    mma_phase ^= 1;
-    __syncthreads();
-    if (ab->flag) goto teardown;
-    tc_fence_after();
-    // ---- W = T diag(beta e^G) K: rebuild the A tile with the other scaling; U rows -> staging
-    if (groupL) {
-        build_tT(sm + OFF_A, r, col, sBeta[r] * __expf(fminf(sG[r], 0.0f)), tmem + lane_base + TM_D2);
-    } else {
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-            float a[32];
-            tmem_ld32(tmem + lane_base + TM_U + c * 32, a);
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) put8(sm + OFF_QV, 128, r, c * 4 + q4, &a[q4 * 8]);
-        }
-    }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-        tc_fence_after();
-        const uint32_t idesc = idesc_f16_f32(128, 128, true, true);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
             umma_f16(tmem + TM_W, sdesc_sw128(sbase + OFF_A + kk * 2048, 16384, 1024),
                      sdesc_sw128(sbase + OFF_K + kk * 2048, 16384, 1024), idesc, kk > 0);
         umma_commit(bar_mma);
-    }
-    if (tid == 128) {
-        tma_store_2d(&tmU, sm + OFF_QV, 0, y0);
-        tma_store_2d(&tmU, sm + OFF_QV + 16384, 64, y0);
-        bulk_commit();
     }
     mbar_wait(bar_mma, mma_phase, ab, p.status, p.wait_limit_ns);
     mma_phase ^= 1;
@@ -424,30 +494,16 @@ __global__ void __launch_bounds__(256, 2)
     if (ab->flag) goto teardown;
     tc_fence_after();
     if (tid == 0) GDN_TRACE_AT(7);
-    if (groupL) {
-        // W row r -> the A area (free now)
+    // ---- W rows (group L) into the A area, U rows (group Q) into the V~ area; bulk stores
+    {
+        uint8_t *dst = sm + (groupL ? OFF_A : OFF_QV);
+        const uint32_t tcol = groupL ? TM_W : TM_U;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
             float a[32];
-            tmem_ld32(tmem + lane_base + TM_W + c * 32, a);
+            tmem_ld32(tmem + lane_base + tcol + c * 32, a);
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) put8(sm + OFF_A, 128, r, c * 4 + q4, &a[q4 * 8]);
-        }
-    } else {
-        // Kt = e^(G_last - G) K over the K tile in place
-        const float fk = __expf(fminf(sG[kBlk - 1] - sG[r], 0.0f));
-#pragma unroll 4
-        for (int c = 0; c < 16; ++c) {
-            uint4 *pk = reinterpret_cast<uint4 *>(sm + OFF_K + tile_off(128, r, c));
-            const uint4 uk = *pk;
-            const uint32_t wk[4] = {uk.x, uk.y, uk.z, uk.w};
-            uint32_t o4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 xk = unpack_half2(wk[e]);
-                o4[e] = pack_half2(xk.x * fk, xk.y * fk);
-            }
-            *pk = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+            for (int q4 = 0; q4 < 4; ++q4) put8(dst, 128, r, c * 4 + q4, &a[q4 * 8]);
         }
     }
     fence_proxy_async();
@@ -455,8 +511,11 @@ __global__ void __launch_bounds__(256, 2)
     if (tid == 0) {
         tma_store_2d(&tmW, sm + OFF_A, 0, y0);
         tma_store_2d(&tmW, sm + OFF_A + 16384, 64, y0);
-        tma_store_2d(&tmKt, sm + OFF_K, 0, y0);
-        tma_store_2d(&tmKt, sm + OFF_K + 16384, 64, y0);
+        bulk_commit();
+    }
+    if (tid == 128) {
+        tma_store_2d(&tmU, sm + OFF_QV, 0, y0);
+        tma_store_2d(&tmU, sm + OFF_QV + 16384, 64, y0);
         bulk_commit();
     }
     if (tid == 0) GDN_TRACE_AT(8);

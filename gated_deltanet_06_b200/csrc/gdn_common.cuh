@@ -340,7 +340,23 @@ __device__ __forceinline__ float2 unpack_half2(uint32_t u) {
 
 // SiLU with the fast reciprocal divide (2 ulp); for u -> -inf the denominator
 // overflows and the result is 0, the limit of u e^u.
+// SiLU for the fp32 CUDA-core path (held to 1e-5 relative).
 __device__ __forceinline__ float silu_f(float u) { return __fdividef(u, 1.0f + __expf(-u)); }
+
+// SiLU for the tensor-core path: u * sigmoid(u) = h + h * tanh(h) with h = u / 2 (from
+// sigmoid(u) = (1 + tanh(u/2)) / 2), one hardware tanh (tanh.approx.f32) instead of an
+// exponential and a reciprocal.  This halves the special-function work of the prep kernel and
+// the output epilogue; its error stays below the fp16 rounding the prepared values get next
+// (measured: no change in the output's error against the oracle at 3 digits).
+__device__ __forceinline__ float tanh_approx(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float silu_tc(float u) {
+    const float h = 0.5f * u;
+    return fmaf(h, tanh_approx(h), h);
+}
 
 __device__ __forceinline__ float softplus_f(float x) { return x > 20.0f ? x : log1pf(expf(x)); }
 

@@ -195,7 +195,9 @@ __global__ void __launch_bounds__(256, 3)
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + 3 * kRawTile + kPrepW);
     __shared__ AbortState ab;
 
-    const int part = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    // heads vary fastest over the grid, so the CTAs in flight together read whole token rows of
+    // the [B][T][H*d] inputs (sequential DRAM pages) rather than one head's 256-byte slice of each
+    const int h = blockIdx.x % p.H, part = blockIdx.x / p.H, b = blockIdx.y;
     const int t0 = part * kPrepTok;          // first token of this CTA
     const int tid = threadIdx.x;
     const size_t bh = static_cast<size_t>(b) * p.H + h;
@@ -254,7 +256,7 @@ __global__ void __launch_bounds__(256, 3)
                 a = fmaf(wt[c].y, win[(r + 1) & 3][c], a);
                 a = fmaf(wt[c].z, win[(r + 2) & 3][c], a);
                 a = fmaf(wt[c].w, win[(r + 3) & 3][c], a);
-                u[c] = silu_f(a);
+                u[c] = silu_tc(a);
                 ss = fmaf(u[c], u[c], ss);
             }
             if (which < 2) {
@@ -291,7 +293,7 @@ cudaError_t launch_typed(const PrepParams &p, cudaStream_t s) {
 cudaError_t launch_prep_tma(const PrepParams &p, InType in, const CUtensorMap &tmq, const CUtensorMap &tmk,
                             const CUtensorMap &tmv, cudaStream_t s) {
     static bool attr_bf = false, attr_h = false;
-    dim3 grid(p.Tp / kPrepTok, p.H, p.B);
+    dim3 grid((p.Tp / kPrepTok) * p.H, p.B);
     if (in == InType::BF16) {
         if (!attr_bf) {
             cudaError_t e = cudaFuncSetAttribute(gdn_prep_tma_kernel<__nv_bfloat16>,

@@ -13,7 +13,8 @@
 //           transfer together as one 256-column state [S^T | P^T] from
 //           [0 | I]; write both (fp32).
 //   combine (gdn_combine_kernel): S_start(j+1)^T = P_j^T S_start(j)^T + S_loc(j)^T,
-//           sequential over segments, fp32 on CUDA cores.
+//           sequential over segments, fp32 on CUDA cores, P_j^T staged in
+//           shared memory one segment ahead.
 //   pass C  (gdn_scan_out_kernel): per segment, run the state from S_start and
 //           emit the block outputs, with the output step fused into the
 //           epilogue:  y = o / sqrt(mean(o^2) + eps) * w * SiLU(z).
@@ -234,66 +235,112 @@ __global__ void __launch_bounds__(288, 1)
 }
 
 // ============================================================ combine
-// S_start(j+1)^T = P_j^T S_start(j)^T + S_loc(j)^T, sequential over j; one CTA
-// per (16-column slice of S^T, head), 256 threads: thread (t, half) owns row
-// t and 8 of the 16 columns; the two threads of a row load the P^T row in the
-// same instruction (one set of transactions), and the rows of the next
-// segment are pulled into L2 while this one is computed.
-__global__ void __launch_bounds__(256) gdn_combine_kernel(const ScanParams p) {
-    __shared__ __align__(16) float cur[128][16];
+// S_start(j+1)^T = P_j^T S_start(j)^T + S_loc(j)^T, sequential over j, in
+// fp32 on CUDA cores.  One CTA per (16-column slice of S^T, head), 256
+// threads; S_start(0) = 0, so S_start(1) = S_loc(0) needs no product.  P_j^T
+// (128 x 128 fp32) is double-buffered in shared memory with cp.async, the
+// copy of P_(j+1)^T in flight while step j is computed, and this thread's
+// entries of S_loc(j+1) are loaded one step ahead too.  Rows are padded to
+// 132 floats so that the 8 rows a warp reads in one instruction fall in
+// different banks.  Thread (warp w, lane l) owns rows (w%4)*8 + l%8 + 32k,
+// k = 0..3, and the two columns (w/4)*8 + (l/8)*2 + {0,1} of the slice; the
+// current state is kept transposed (column-major) so that its reads are
+// 16-byte broadcasts.  The product is bound by shared-memory wavefronts: a
+// 4 x 2 register tile per thread feeds 32 FMAs from 6 16-byte loads.
+namespace cb {
+constexpr int RS = 132;  // padded row stride (floats)
+constexpr uint32_t SMEM_BYTES = (2 * 128 * RS + 16 * RS) * 4;
+}  // namespace cb
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__global__ void __launch_bounds__(256, 1) gdn_combine_kernel(const ScanParams p) {
+    using cb::RS;
+    extern __shared__ __align__(16) float csm[];
+    float *PT = csm;                   // [2][128][RS]: P_j^T, row t = column t of P_j
+    float *curT = csm + 2 * 128 * RS;  // [16][RS]: column c of the slice of S_start(j)^T
     const int slice = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int bh = b * p.H + h;
-    const int t = threadIdx.x >> 1, half = threadIdx.x & 1;
-    const int c0 = slice * 16 + half * 8;
-    if (threadIdx.x < 128) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int rbase = (warp & 3) * 8 + (lane & 7);
+    const int cl = (warp >> 2) * 8 + (lane >> 3) * 2;  // local column pair cl, cl + 1
+    const int col = slice * 16 + cl;
+    constexpr size_t kZ = 128 * 256;                    // floats per (bh, segment) of Zloc
+    const float *Z = p.Zloc + static_cast<size_t>(bh) * p.NS * kZ;
+    float *Sst = p.Sstart + static_cast<size_t>(bh) * p.NS * 128 * 128;
+    if (p.NS < 2) return;
+
+    auto load_pt = [&](int j) {  // rows of P_j^T: 32 16-byte pieces each, a warp per row at a time
+        const float *src = Z + j * kZ + 128;
+        float *dst = PT + (j & 1) * 128 * RS;
+#pragma unroll 4
+        for (int e = tid; e < 128 * 32; e += 256) {
+            const int t = e >> 5, q = e & 31;
+            cp_async16(dst + t * RS + q * 4, src + static_cast<size_t>(t) * 256 + q * 4);
+        }
+        cp_async_commit();
+    };
+    auto load_sl = [&](int j, float2 (&v)[4]) {  // this thread's entries of S_loc(j)^T
 #pragma unroll
-        for (int c = 0; c < 16; ++c) cur[threadIdx.x][c] = 0.0f;
+        for (int k = 0; k < 4; ++k)
+            v[k] = *reinterpret_cast<const float2 *>(Z + j * kZ + static_cast<size_t>(rbase + 32 * k) * 256 + col);
+    };
+    if (tid == 0) GDN_TRACE_AT(2048);
+    if (p.NS > 2) load_pt(1);
+
+    // S_start(1) = S_loc(0)
+    for (int e = tid; e < 128 * 16; e += 256) {
+        const int t = e >> 4, c = e & 15;
+        const float v = Z[static_cast<size_t>(t) * 256 + slice * 16 + c];
+        curT[c * RS + t] = v;
+        Sst[(static_cast<size_t>(1) * 128 + t) * 128 + slice * 16 + c] = v;
     }
-    __syncthreads();
-    for (int j = 0; j + 1 < p.NS; ++j) {
-        const float *zrow = p.Zloc + ((static_cast<size_t>(bh) * p.NS + j) * 128 + t) * 256;
+    float2 sl[4];
+    if (p.NS > 2) load_sl(1, sl);
+    for (int j = 1; j + 1 < p.NS; ++j) {
+        float2 sn[4];
         if (j + 2 < p.NS) {
-            const char *nxt = reinterpret_cast<const char *>(zrow + 128 * 256) + half * 512;
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(nxt));
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(nxt + 128));
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(nxt + 256));
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(nxt + 384));
+            load_sl(j + 1, sn);
+            load_pt(j + 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
         }
-        float acc[8];
-        {
-            const float4 s0 = *reinterpret_cast<const float4 *>(zrow + c0);  // S_loc^T
-            const float4 s1 = *reinterpret_cast<const float4 *>(zrow + c0 + 4);
-            acc[0] = s0.x; acc[1] = s0.y; acc[2] = s0.z; acc[3] = s0.w;
-            acc[4] = s1.x; acc[5] = s1.y; acc[6] = s1.z; acc[7] = s1.w;
-        }
-        const float4 *prow = reinterpret_cast<const float4 *>(zrow + 128);  // P^T row t
-        float4 pr[32];
+        if (tid == 0) GDN_TRACE_AT(2048 + 8 * j);
+        __syncthreads();  // P_j^T and the current state visible to all
+        if (tid == 0) GDN_TRACE_AT(2048 + 8 * j + 1);
+        const float *P = PT + (j & 1) * 128 * RS;
+        float acc[4][2];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) pr[i] = __ldg(prow + i);
+        for (int k = 0; k < 4; ++k) acc[k][0] = acc[k][1] = 0.0f;
+#pragma unroll 4
+        for (int i = 0; i < 128; i += 4) {
+            const float4 c0 = *reinterpret_cast<const float4 *>(curT + cl * RS + i);
+            const float4 c1 = *reinterpret_cast<const float4 *>(curT + (cl + 1) * RS + i);
 #pragma unroll
-        for (int i4 = 0; i4 < 32; ++i4) {
-            const float pv[4] = {pr[i4].x, pr[i4].y, pr[i4].z, pr[i4].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float4 ca = *reinterpret_cast<const float4 *>(&cur[i4 * 4 + e][half * 8]);
-                const float4 cb = *reinterpret_cast<const float4 *>(&cur[i4 * 4 + e][half * 8 + 4]);
-                acc[0] = fmaf(pv[e], ca.x, acc[0]);
-                acc[1] = fmaf(pv[e], ca.y, acc[1]);
-                acc[2] = fmaf(pv[e], ca.z, acc[2]);
-                acc[3] = fmaf(pv[e], ca.w, acc[3]);
-                acc[4] = fmaf(pv[e], cb.x, acc[4]);
-                acc[5] = fmaf(pv[e], cb.y, acc[5]);
-                acc[6] = fmaf(pv[e], cb.z, acc[6]);
-                acc[7] = fmaf(pv[e], cb.w, acc[7]);
+            for (int k = 0; k < 4; ++k) {
+                const float4 a = *reinterpret_cast<const float4 *>(P + (rbase + 32 * k) * RS + i);
+                acc[k][0] = fmaf(a.x, c0.x, fmaf(a.y, c0.y, fmaf(a.z, c0.z, fmaf(a.w, c0.w, acc[k][0]))));
+                acc[k][1] = fmaf(a.x, c1.x, fmaf(a.y, c1.y, fmaf(a.z, c1.z, fmaf(a.w, c1.w, acc[k][1]))));
             }
         }
-        __syncthreads();
-        *reinterpret_cast<float4 *>(&cur[t][half * 8]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        *reinterpret_cast<float4 *>(&cur[t][half * 8 + 4]) = make_float4(acc[4], acc[5], acc[6], acc[7]);
-        float *dst = p.Sstart + ((static_cast<size_t>(bh) * p.NS + j + 1) * 128 + t) * 128 + c0;
-        *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        *reinterpret_cast<float4 *>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
-        __syncthreads();
+        if (tid == 0) GDN_TRACE_AT(2048 + 8 * j + 2);
+        __syncthreads();  // every read of this step's state and P_j^T buffer is done
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int t = rbase + 32 * k;
+            const float v0 = acc[k][0] + sl[k].x, v1 = acc[k][1] + sl[k].y;
+            curT[cl * RS + t] = v0;
+            curT[(cl + 1) * RS + t] = v1;
+            *reinterpret_cast<float2 *>(Sst + (static_cast<size_t>(j + 1) * 128 + t) * 128 + col) = make_float2(v0, v1);
+            if (j + 2 < p.NS) sl[k] = sn[k];
+        }
+        if (tid == 0) GDN_TRACE_AT(2048 + 8 * j + 3);
     }
 }
 
@@ -312,54 +359,6 @@ constexpr int kScanThreads = 416;  // warps 0-3 state, warp 4 producer, warps 5-
 // the fp32 state S^T lives in TMEM; O is double-buffered (256 and 384).
 constexpr uint32_t TM_X = 0, TM_P = 0, TM_S = 128, TM_O = 256;
 }  // namespace tc
-
-template <typename ZT, typename YT>
-__device__ __forceinline__ void load8(const ZT *p, float (&f)[8]);
-template <>
-__device__ __forceinline__ void load8<__nv_bfloat16, float>(const __nv_bfloat16 *p, float (&f)[8]) {
-    const uint4 u = *reinterpret_cast<const uint4 *>(p);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i]));
-        f[2 * i] = x.x;
-        f[2 * i + 1] = x.y;
-    }
-}
-template <>
-__device__ __forceinline__ void load8<__half, float>(const __half *p, float (&f)[8]) {
-    const uint4 u = *reinterpret_cast<const uint4 *>(p);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 x = unpack_half2(w[i]);
-        f[2 * i] = x.x;
-        f[2 * i + 1] = x.y;
-    }
-}
-
-__device__ __forceinline__ void store_y8(void *y, int out_kind, size_t idx, const float *v) {
-    if (out_kind == 0) {  // bf16
-        uint4 u;
-        uint32_t w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-            w[i] = *reinterpret_cast<uint32_t *>(&b2);
-        }
-        u.x = w[0]; u.y = w[1]; u.z = w[2]; u.w = w[3];
-        *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(y) + idx) = u;
-    } else if (out_kind == 2) {  // f16
-        uint4 u;
-        u.x = pack_half2(v[0], v[1]); u.y = pack_half2(v[2], v[3]);
-        u.z = pack_half2(v[4], v[5]); u.w = pack_half2(v[6], v[7]);
-        *reinterpret_cast<uint4 *>(static_cast<__half *>(y) + idx) = u;
-    } else {
-        float *d = static_cast<float *>(y) + idx;
-        *reinterpret_cast<float4 *>(d) = make_float4(v[0], v[1], v[2], v[3]);
-        *reinterpret_cast<float4 *>(d + 4) = make_float4(v[4], v[5], v[6], v[7]);
-    }
-}
 
 template <typename ZT>
 __global__ void __launch_bounds__(tc::kScanThreads, 1)
@@ -476,10 +475,10 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
                             fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wa[j]));
                             fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wb[j]));
                         }
-                        yf[0][j][0] = __uint_as_float(v[4 * gl]) * rnA * w0 * silu_f(fa.x);
-                        yf[0][j][1] = __uint_as_float(v[4 * gl + 1]) * rnA * w1 * silu_f(fa.y);
-                        yf[1][j][0] = __uint_as_float(v[4 * gl + 2]) * rnB * w0 * silu_f(fb.x);
-                        yf[1][j][1] = __uint_as_float(v[4 * gl + 3]) * rnB * w1 * silu_f(fb.y);
+                        yf[0][j][0] = __uint_as_float(v[4 * gl]) * rnA * w0 * silu_tc(fa.x);
+                        yf[0][j][1] = __uint_as_float(v[4 * gl + 1]) * rnA * w1 * silu_tc(fa.y);
+                        yf[1][j][0] = __uint_as_float(v[4 * gl + 2]) * rnB * w0 * silu_tc(fb.x);
+                        yf[1][j][1] = __uint_as_float(v[4 * gl + 3]) * rnB * w1 * silu_tc(fb.y);
                     }
                     if (p.out_kind == 1) {  // fp32: each lane stores its 8-byte pairs (a quad covers 32 bytes)
 #pragma unroll
@@ -738,8 +737,11 @@ cudaError_t launch_transfer(const ScanParams &p, const CUtensorMap &tmW, const C
 }
 
 cudaError_t launch_combine(const ScanParams &p, cudaStream_t s) {
+    static bool attr = false;
+    cudaError_t e = set_smem(gdn_combine_kernel, cb::SMEM_BYTES, attr);
+    if (e != cudaSuccess) return e;
     dim3 grid(8, p.H, p.B);
-    gdn_combine_kernel<<<grid, 256, 0, s>>>(p);
+    gdn_combine_kernel<<<grid, 256, cb::SMEM_BYTES, s>>>(p);
     return cudaGetLastError();
 }
 
