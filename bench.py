@@ -7,8 +7,9 @@
 A step is one whole GDN forward (prep, UT transform, scan, output) over the
 workload with its inputs resident in HBM; the L2 cache is flushed (256 MiB
 write) before every step, outside the timed interval.  Each step is timed
-with CUDA events on the launching stream; per-kernel times come from events
-the library records between its launches (gdn_forward_timed).  With N > 1
+with CUDA events on the launching stream around the plain forward; per-kernel
+times come from separate runs in which the library records events between its
+launches (gdn_forward_timed), which serialises them.  With N > 1
 (torchrun) every rank runs its own replica of the workload (the forward has
 no cross-GPU exchange) and the time is the max over ranks.  Rank 0 prints one
 JSON line.
@@ -287,16 +288,17 @@ def main():
             plan.forward_raw(ptrs, y.data_ptr(), ws.data_ptr(), s)
         torch.cuda.synchronize()
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(L + 1)] for _ in range(args.steps)]
-    for row in events:  # torch creates the underlying cudaEvent_t on first record
-        for e in row:
-            e.record(stream)
+    # timed steps: the plain forward (consecutive kernels overlap their launch and prologue with
+    # the previous kernel's tail), one event pair per step around it
+    ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     for k in range(args.steps):
         flush.zero_()
-        plan.forward_timed_raw(ptrs, y.data_ptr(), ws.data_ptr(), s, [e.cuda_event for e in events[k]])
+        ev_step[k][0].record(stream)
+        plan.forward_raw(ptrs, y.data_ptr(), ws.data_ptr(), s)
+        ev_step[k][1].record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -304,9 +306,21 @@ def main():
     st = plan.device_status(ws.data_ptr(), s)
     if st != gdn.OK:
         raise SystemExit(f"device status after timing: {gdn.status_string(st)}")
+    step_ms = [a.elapsed_time(b) for a, b in ev_step]
 
-    step_ms = [events[k][0].elapsed_time(events[k][L]) for k in range(args.steps)]
-    kern_ms = {names[i]: statistics.mean(events[k][i].elapsed_time(events[k][i + 1]) for k in range(args.steps))
+    # per-kernel breakdown (not part of the timed steps): the library records an event before each
+    # launch and after the last one (gdn_forward_timed), which also serialises the launches
+    n_kt = max(3, min(args.steps, 10))
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(L + 1)] for _ in range(n_kt)]
+    for row in events:  # torch creates the underlying cudaEvent_t on first record
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+    for k in range(n_kt):
+        flush.zero_()
+        plan.forward_timed_raw(ptrs, y.data_ptr(), ws.data_ptr(), s, [e.cuda_event for e in events[k]])
+    torch.cuda.synchronize()
+    kern_ms = {names[i]: statistics.mean(events[k][i].elapsed_time(events[k][i + 1]) for k in range(n_kt))
                for i in range(L)}
     total_ms = sum(step_ms)
     t = torch.tensor([total_ms], dtype=torch.float64, device=dev)

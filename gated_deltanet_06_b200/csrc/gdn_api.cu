@@ -310,7 +310,10 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
         cp.BH = c.B * c.H; cp.Tp = plan->Tp; cp.NB = plan->NB;
         cp.status = status;
         cp.wait_limit_ns = kWaitLimitNs;
-        if (!mark() || launch_chunk(cp, tmK, tmV, tmQ, tmW, tmU, tmQt, tmKt, tmAqk, s) != cudaSuccess)
+        // Kernels after the first start with programmatic dependent launch (prologue overlapped with
+        // the previous kernel's tail), except when per-kernel events are recorded between them.
+        const bool pdl = events == nullptr;
+        if (!mark() || launch_chunk(cp, tmK, tmV, tmQ, tmW, tmU, tmQt, tmKt, tmAqk, s, pdl) != cudaSuccess)
             return GDN_ERR_CUDA;
         ScanParams sp;
         sp.G = G;
@@ -324,12 +327,12 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
         sp.wait_limit_ns = kWaitLimitNs;
         sp.test_wait_timeout = (c.flags & GDN_FLAG_TEST_WAIT_TIMEOUT) ? 1 : 0;
         if (plan->NS > 1) {
-            if (!mark() || launch_transfer(sp, tmW, tmKt, tmU, s) != cudaSuccess) return GDN_ERR_CUDA;
-            if (!mark() || launch_combine(sp, s) != cudaSuccess) return GDN_ERR_CUDA;
+            if (!mark() || launch_transfer(sp, tmW, tmKt, tmU, s, pdl) != cudaSuccess) return GDN_ERR_CUDA;
+            if (!mark() || launch_combine(sp, s, pdl) != cudaSuccess) return GDN_ERR_CUDA;
         }
         CUtensorMap tmZ;
         if (!make_raw_map(&tmZ, in->z, c.B, c.T, c.H * d, plan->tok_stride, kBlk, 128)) return GDN_ERR_CUDA;
-        if (!mark() || launch_scan_out(sp, in_type(c.in_dtype), tmW, tmQt, tmKt, tmAqk, tmU, tmZ, s) != cudaSuccess)
+        if (!mark() || launch_scan_out(sp, in_type(c.in_dtype), tmW, tmQt, tmKt, tmAqk, tmU, tmZ, s, pdl) != cudaSuccess)
             return GDN_ERR_CUDA;
         if (!mark()) return GDN_ERR_CUDA;
         return GDN_OK;

@@ -151,7 +151,9 @@ __global__ void __launch_bounds__(256, 2)
         tmem_alloc(tmem_slot, 256);
         tmem_relinquish();
     }
+    pdl_launch_dependents();
     __syncthreads();  // barrier init visible before the TMA below uses it
+    pdl_wait();       // the prep kernel's q^, k^, v^ are complete
     if (tid == 0) {
         mbar_arrive_expect_tx(bar_load, 2u * 32768u);
         tma_load_2d(sm + OFF_K, &tmK, bar_load, 0, y0);
@@ -496,7 +498,7 @@ teardown:
 cudaError_t launch_chunk(const ChunkParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
                          const CUtensorMap &tmQ, const CUtensorMap &tmW, const CUtensorMap &tmU,
                          const CUtensorMap &tmQt, const CUtensorMap &tmKt, const CUtensorMap &tmAqk,
-                         cudaStream_t s) {
+                         cudaStream_t s, bool pdl) {
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(gdn_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -505,8 +507,8 @@ cudaError_t launch_chunk(const ChunkParams &p, const CUtensorMap &tmK, const CUt
         attr_set = true;
     }
     dim3 grid(p.NB, p.BH);
-    gdn_chunk_kernel<<<grid, 256, SMEM_BYTES, s>>>(p, tmK, tmV, tmQ, tmW, tmU, tmQt, tmKt, tmAqk);
-    return cudaGetLastError();
+    return launch_k(gdn_chunk_kernel, grid, dim3(256), SMEM_BYTES, s, pdl, p, tmK, tmV, tmQ, tmW, tmU, tmQt, tmKt,
+                    tmAqk);
 }
 
 }  // namespace gdn

@@ -59,6 +59,15 @@ static __device__ unsigned long long g_gdn_trace[8192];
 #define GDN_TRACE_EXPORT(name)
 #endif
 
+// ------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while the
+// previous kernel in the stream is still finishing: it runs its prologue, then
+// waits here until that kernel has completed and its writes are visible (a
+// no-op when launched normally).  launch_dependents lets the next kernel in
+// the stream start early the same way.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));

@@ -11,6 +11,25 @@ namespace gdn {
 
 enum class InType { BF16 = 0, F32 = 1, F16 = 2 };
 
+// Kernel launch, optionally with programmatic stream serialization: the kernel
+// may then be scheduled while the previous kernel in the stream finishes; it
+// must call pdl_wait() before touching that kernel's outputs.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                            const Args &...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Prep: conv4 + SiLU on q, k, v; L2 norm (and the 1/sqrt(d_k) output scale
 // folded into q^); log-decay, in-block cumulative log-decay, update gate.
 struct PrepParams {
@@ -50,7 +69,7 @@ struct ChunkParams {
 cudaError_t launch_chunk(const ChunkParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
                          const CUtensorMap &tmQ, const CUtensorMap &tmW, const CUtensorMap &tmU,
                          const CUtensorMap &tmQt, const CUtensorMap &tmKt, const CUtensorMap &tmAqk,
-                         cudaStream_t s);
+                         cudaStream_t s, bool pdl);
 
 // Inter-block state scan on tensor cores (d = 128), parallel over segments of
 // Ls blocks: pass A (transfer), combine, pass C (outputs + fused output step).
@@ -69,12 +88,13 @@ struct ScanParams {
     unsigned long long wait_limit_ns;
     int test_wait_timeout;
 };
+// pdl: launch with programmatic stream serialization (see launch_k).
 cudaError_t launch_transfer(const ScanParams &p, const CUtensorMap &tmW, const CUtensorMap &tmKt,
-                            const CUtensorMap &tmU, cudaStream_t s);
-cudaError_t launch_combine(const ScanParams &p, cudaStream_t s);
+                            const CUtensorMap &tmU, cudaStream_t s, bool pdl);
+cudaError_t launch_combine(const ScanParams &p, cudaStream_t s, bool pdl);
 cudaError_t launch_scan_out(const ScanParams &p, InType zt, const CUtensorMap &tmW, const CUtensorMap &tmQt,
                             const CUtensorMap &tmKt, const CUtensorMap &tmAqk, const CUtensorMap &tmU,
-                            const CUtensorMap &tmZ, cudaStream_t s);
+                            const CUtensorMap &tmZ, cudaStream_t s, bool pdl);
 
 // Sequential fp32 recurrence on CUDA cores (fp32 inputs or d = 64).
 struct RecurParams {

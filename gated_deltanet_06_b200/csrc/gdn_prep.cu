@@ -210,6 +210,7 @@ __global__ void __launch_bounds__(256, 2)
         ab.flag = 0;
         fence_mbar_init();
     }
+    pdl_launch_dependents();
     __syncthreads();
     auto issue = [&](int n, int L) {  // thread 0: the raw boxes of tile L into stage n & 1
         const int part = L % nparts, bh = L / nparts;

@@ -86,10 +86,12 @@ __global__ void __launch_bounds__(288, 1)
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
+    pdl_launch_dependents();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();  // the UT kernel's tiles are complete
 
     if (warp == 8) {
         if (lane == 0) {
@@ -273,6 +275,8 @@ __global__ void __launch_bounds__(256, 1) gdn_combine_kernel(const ScanParams p)
     constexpr size_t kZ = 128 * 256;                    // floats per (bh, segment) of Zloc
     const float *Z = p.Zloc + static_cast<size_t>(bh) * p.NS * kZ;
     float *Sst = p.Sstart + static_cast<size_t>(bh) * p.NS * 128 * 128;
+    pdl_launch_dependents();
+    pdl_wait();  // the transfer pass's [S_loc^T | P^T] are complete
     if (p.NS < 2) return;
 
     auto load_pt = [&](int j) {  // rows of P_j^T: 32 16-byte pieces each, a warp per row at a time
@@ -396,6 +400,7 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();  // the segment start states (and the UT kernel's tiles) are complete
 
     if (warp >= 5) {
         // ------------------------------------------ output step (warps 5-12)
@@ -727,40 +732,38 @@ cudaError_t set_smem(K kernel, uint32_t bytes, bool &done) {
 }  // namespace
 
 cudaError_t launch_transfer(const ScanParams &p, const CUtensorMap &tmW, const CUtensorMap &tmKt,
-                            const CUtensorMap &tmU, cudaStream_t s) {
+                            const CUtensorMap &tmU, cudaStream_t s, bool pdl) {
     static bool attr = false;
     cudaError_t e = set_smem(gdn_transfer_kernel, ta::SMEM_BYTES, attr);
     if (e != cudaSuccess) return e;
     dim3 grid(p.NS - 1, p.H, p.B);
-    gdn_transfer_kernel<<<grid, 288, ta::SMEM_BYTES, s>>>(p, tmW, tmKt, tmU);
-    return cudaGetLastError();
+    return launch_k(gdn_transfer_kernel, grid, dim3(288), ta::SMEM_BYTES, s, pdl, p, tmW, tmKt, tmU);
 }
 
-cudaError_t launch_combine(const ScanParams &p, cudaStream_t s) {
+cudaError_t launch_combine(const ScanParams &p, cudaStream_t s, bool pdl) {
     static bool attr = false;
     cudaError_t e = set_smem(gdn_combine_kernel, cb::SMEM_BYTES, attr);
     if (e != cudaSuccess) return e;
     dim3 grid(8, p.H, p.B);
-    gdn_combine_kernel<<<grid, 256, cb::SMEM_BYTES, s>>>(p);
-    return cudaGetLastError();
+    return launch_k(gdn_combine_kernel, grid, dim3(256), cb::SMEM_BYTES, s, pdl, p);
 }
 
 cudaError_t launch_scan_out(const ScanParams &p, InType zt, const CUtensorMap &tmW, const CUtensorMap &tmQt,
                             const CUtensorMap &tmKt, const CUtensorMap &tmAqk, const CUtensorMap &tmU,
-                            const CUtensorMap &tmZ, cudaStream_t s) {
+                            const CUtensorMap &tmZ, cudaStream_t s, bool pdl) {
     dim3 grid(p.NS, p.H, p.B);
     if (zt == InType::F16) {
         static bool attr = false;
         cudaError_t e = set_smem(gdn_scan_out_kernel<__half>, tc::SMEM_BYTES, attr);
         if (e != cudaSuccess) return e;
-        gdn_scan_out_kernel<__half><<<grid, tc::kScanThreads, tc::SMEM_BYTES, s>>>(p, tmW, tmQt, tmKt, tmAqk, tmU, tmZ);
-    } else {
-        static bool attr = false;
-        cudaError_t e = set_smem(gdn_scan_out_kernel<__nv_bfloat16>, tc::SMEM_BYTES, attr);
-        if (e != cudaSuccess) return e;
-        gdn_scan_out_kernel<__nv_bfloat16><<<grid, tc::kScanThreads, tc::SMEM_BYTES, s>>>(p, tmW, tmQt, tmKt, tmAqk, tmU, tmZ);
+        return launch_k(gdn_scan_out_kernel<__half>, grid, dim3(tc::kScanThreads), tc::SMEM_BYTES, s, pdl, p, tmW,
+                        tmQt, tmKt, tmAqk, tmU, tmZ);
     }
-    return cudaGetLastError();
+    static bool attr = false;
+    cudaError_t e = set_smem(gdn_scan_out_kernel<__nv_bfloat16>, tc::SMEM_BYTES, attr);
+    if (e != cudaSuccess) return e;
+    return launch_k(gdn_scan_out_kernel<__nv_bfloat16>, grid, dim3(tc::kScanThreads), tc::SMEM_BYTES, s, pdl, p, tmW,
+                    tmQt, tmKt, tmAqk, tmU, tmZ);
 }
 
 }  // namespace gdn
