@@ -60,12 +60,12 @@ EncodeTiledFn encode_fn() {
 }
 
 // [rows][128] fp16 row-major, loaded as {64, 128} boxes with the 128-byte swizzle.
-bool make_tile_map(CUtensorMap *m, void *base, unsigned long long rows) {
+bool make_tile_map(CUtensorMap *m, void *base, unsigned long long rows, unsigned box_rows = 128) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[2] = {128, rows};
     const cuuint64_t strides[1] = {128 * 2};
-    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t box[2] = {64, box_rows};
     const cuuint32_t es[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -292,11 +292,12 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
 
     if (plan->tensor) {
         const unsigned long long rows = static_cast<unsigned long long>(c.B) * c.H * plan->Tp;
-        CUtensorMap tmQ, tmK, tmV, tmW, tmU, tmQt, tmKt, tmAqk;
+        CUtensorMap tmQ, tmK, tmV, tmW, tmU, tmQt, tmKt, tmAqk, tmAqkH;
         if (!make_tile_map(&tmQ, ws + plan->off_qh, rows) || !make_tile_map(&tmK, ws + plan->off_kh, rows) ||
             !make_tile_map(&tmV, ws + plan->off_vh, rows) || !make_tile_map(&tmW, ws + plan->off_W, rows) ||
             !make_tile_map(&tmU, ws + plan->off_U, rows) || !make_tile_map(&tmQt, ws + plan->off_Qt, rows) ||
-            !make_tile_map(&tmKt, ws + plan->off_Kt, rows) || !make_tile_map(&tmAqk, ws + plan->off_Aqk, rows))
+            !make_tile_map(&tmKt, ws + plan->off_Kt, rows) || !make_tile_map(&tmAqk, ws + plan->off_Aqk, rows) ||
+            !make_tile_map(&tmAqkH, ws + plan->off_Aqk, rows, 64))  // Aqk's lower-right quadrant
             return GDN_ERR_CUDA;
         ChunkParams cp;
         cp.g = in->g; cp.bg = in->b; cp.A_log = in->A_log; cp.dt_bias = in->dt_bias;
@@ -313,7 +314,7 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
         // Kernels after the first start with programmatic dependent launch (prologue overlapped with
         // the previous kernel's tail), except when per-kernel events are recorded between them.
         const bool pdl = events == nullptr;
-        if (!mark() || launch_chunk(cp, tmK, tmV, tmQ, tmW, tmU, tmQt, tmKt, tmAqk, s, pdl) != cudaSuccess)
+        if (!mark() || launch_chunk(cp, tmK, tmV, tmQ, tmW, tmU, tmQt, tmKt, tmAqk, tmAqkH, s, pdl) != cudaSuccess)
             return GDN_ERR_CUDA;
         ScanParams sp;
         sp.G = G;
@@ -332,7 +333,7 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
         }
         CUtensorMap tmZ;
         if (!make_raw_map(&tmZ, in->z, c.B, c.T, c.H * d, plan->tok_stride, kBlk, 128)) return GDN_ERR_CUDA;
-        if (!mark() || launch_scan_out(sp, in_type(c.in_dtype), tmW, tmQt, tmKt, tmAqk, tmU, tmZ, s, pdl) != cudaSuccess)
+        if (!mark() || launch_scan_out(sp, in_type(c.in_dtype), tmW, tmQt, tmKt, tmAqk, tmAqkH, tmU, tmZ, s, pdl) != cudaSuccess)
             return GDN_ERR_CUDA;
         if (!mark()) return GDN_ERR_CUDA;
         return GDN_OK;

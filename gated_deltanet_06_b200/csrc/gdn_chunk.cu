@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(256, 2)
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmU,
                      const __grid_constant__ CUtensorMap tmQt, const __grid_constant__ CUtensorMap tmKt,
-                     const __grid_constant__ CUtensorMap tmAqk) {
+                     const __grid_constant__ CUtensorMap tmAqk, const __grid_constant__ CUtensorMap tmAqkH) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
@@ -424,8 +424,9 @@ __global__ void __launch_bounds__(256, 2)
         fence_proxy_async();
         group_sync(2);
         if (tid == 128) {
+            // Aqk is block lower triangular: its upper-right 64x64 quadrant (zero) is not stored
             tma_store_2d(&tmAqk, sm + OFF_QV, 0, y0);
-            tma_store_2d(&tmAqk, sm + OFF_QV + 16384, 64, y0);
+            tma_store_2d(&tmAqkH, sm + OFF_QV + 16384 + 64 * 128, 64, y0 + 64);
             bulk_commit();
             bulk_wait_read_all();
             mbar_arrive_expect_tx(bar_v, 32768u);
@@ -498,7 +499,7 @@ teardown:
 cudaError_t launch_chunk(const ChunkParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
                          const CUtensorMap &tmQ, const CUtensorMap &tmW, const CUtensorMap &tmU,
                          const CUtensorMap &tmQt, const CUtensorMap &tmKt, const CUtensorMap &tmAqk,
-                         cudaStream_t s, bool pdl) {
+                         const CUtensorMap &tmAqkH, cudaStream_t s, bool pdl) {
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(gdn_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -508,7 +509,7 @@ cudaError_t launch_chunk(const ChunkParams &p, const CUtensorMap &tmK, const CUt
     }
     dim3 grid(p.NB, p.BH);
     return launch_k(gdn_chunk_kernel, grid, dim3(256), SMEM_BYTES, s, pdl, p, tmK, tmV, tmQ, tmW, tmU, tmQt, tmKt,
-                    tmAqk);
+                    tmAqk, tmAqkH);
 }
 
 }  // namespace gdn

@@ -69,7 +69,7 @@ struct ChunkParams {
 cudaError_t launch_chunk(const ChunkParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
                          const CUtensorMap &tmQ, const CUtensorMap &tmW, const CUtensorMap &tmU,
                          const CUtensorMap &tmQt, const CUtensorMap &tmKt, const CUtensorMap &tmAqk,
-                         cudaStream_t s, bool pdl);
+                         const CUtensorMap &tmAqkH, cudaStream_t s, bool pdl);
 
 // Inter-block state scan on tensor cores (d = 128), parallel over segments of
 // Ls blocks: pass A (transfer), combine, pass C (outputs + fused output step).
@@ -93,8 +93,8 @@ cudaError_t launch_transfer(const ScanParams &p, const CUtensorMap &tmW, const C
                             const CUtensorMap &tmU, cudaStream_t s, bool pdl);
 cudaError_t launch_combine(const ScanParams &p, cudaStream_t s, bool pdl);
 cudaError_t launch_scan_out(const ScanParams &p, InType zt, const CUtensorMap &tmW, const CUtensorMap &tmQt,
-                            const CUtensorMap &tmKt, const CUtensorMap &tmAqk, const CUtensorMap &tmU,
-                            const CUtensorMap &tmZ, cudaStream_t s, bool pdl);
+                            const CUtensorMap &tmKt, const CUtensorMap &tmAqk, const CUtensorMap &tmAqkH,
+                            const CUtensorMap &tmU, const CUtensorMap &tmZ, cudaStream_t s, bool pdl);
 
 // Sequential fp32 recurrence on CUDA cores (fp32 inputs or d = 64).
 struct RecurParams {

@@ -13,8 +13,8 @@
 //           transfer together as one 256-column state [S^T | P^T] from
 //           [0 | I]; write both (fp32).
 //   combine (gdn_combine_kernel): S_start(j+1)^T = P_j^T S_start(j)^T + S_loc(j)^T,
-//           sequential over segments, fp32 on CUDA cores, P_j^T staged in
-//           shared memory one segment ahead.
+//           sequential over segments, split-precision tf32 tensor-core products
+//           (close to fp32), P_j^T staged in shared memory one segment ahead.
 //   pass C  (gdn_scan_out_kernel): per segment, run the state from S_start and
 //           emit the block outputs, with the output step fused into the
 //           epilogue:  y = o / sqrt(mean(o^2) + eps) * w * SiLU(z).
@@ -237,18 +237,18 @@ __global__ void __launch_bounds__(288, 1)
 }
 
 // ============================================================ combine
-// S_start(j+1)^T = P_j^T S_start(j)^T + S_loc(j)^T, sequential over j, in
-// fp32 on CUDA cores.  One CTA per (16-column slice of S^T, head), 256
-// threads; S_start(0) = 0, so S_start(1) = S_loc(0) needs no product.  P_j^T
-// (128 x 128 fp32) is double-buffered in shared memory with cp.async, the
-// copy of P_(j+1)^T in flight while step j is computed, and this thread's
-// entries of S_loc(j+1) are loaded one step ahead too.  Rows are padded to
-// 132 floats so that the 8 rows a warp reads in one instruction fall in
-// different banks.  Thread (warp w, lane l) owns rows (w%4)*8 + l%8 + 32k,
-// k = 0..3, and the two columns (w/4)*8 + (l/8)*2 + {0,1} of the slice; the
-// current state is kept transposed (column-major) so that its reads are
-// 16-byte broadcasts.  The product is bound by shared-memory wavefronts: a
-// 4 x 2 register tile per thread feeds 32 FMAs from 6 16-byte loads.
+// S_start(j+1)^T = P_j^T S_start(j)^T + S_loc(j)^T, sequential over j.  One
+// CTA per (16-column slice of S^T, head), 256 threads; S_start(0) = 0, so
+// S_start(1) = S_loc(0) needs no product.  P_j^T (128 x 128 fp32) is
+// double-buffered in shared memory with cp.async, the copy of P_(j+1)^T in
+// flight while step j is computed, and this thread's entries of S_loc(j+1)
+// are loaded one step ahead too.  The product runs on warp-level tensor cores
+// (mma.sync m16n8k8, tf32) in split precision: each fp32 operand x is split
+// into tf32 parts hi + lo and the product accumulates hi*hi + hi*lo + lo*hi
+// in fp32, close to fp32 accuracy.  Warp w owns rows 16w .. 16w+15 of the
+// slice; rows are padded to 132 floats, so that the scalar fragment loads
+// (8 rows x 4 columns per instruction) fall in 32 different banks, and the
+// current state is kept transposed (column-major) for the B fragments.
 namespace cb {
 constexpr int RS = 132;  // padded row stride (floats)
 constexpr uint32_t SMEM_BYTES = (2 * 128 * RS + 16 * RS) * 4;
@@ -261,6 +261,21 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
+// x = hi + lo, both tf32 (round to nearest, ties away)
+__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo) {
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
+    const float r = x - __uint_as_float(hi);
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(r));
+}
+// d += a (16x8 tf32, row fragment) * b (8x8 tf32, column fragment)
+__device__ __forceinline__ void mma1688_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
 __global__ void __launch_bounds__(256, 1) gdn_combine_kernel(const ScanParams p) {
     using cb::RS;
     extern __shared__ __align__(16) float csm[];
@@ -269,10 +284,9 @@ __global__ void __launch_bounds__(256, 1) gdn_combine_kernel(const ScanParams p)
     const int slice = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int bh = b * p.H + h;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int rbase = (warp & 3) * 8 + (lane & 7);
-    const int cl = (warp >> 2) * 8 + (lane >> 3) * 2;  // local column pair cl, cl + 1
-    const int col = slice * 16 + cl;
-    constexpr size_t kZ = 128 * 256;                    // floats per (bh, segment) of Zloc
+    const int g = lane >> 2, t4 = lane & 3;
+    const int r0 = warp * 16;  // this warp's rows r0 + g and r0 + g + 8
+    constexpr size_t kZ = 128 * 256;  // floats per (bh, segment) of Zloc
     const float *Z = p.Zloc + static_cast<size_t>(bh) * p.NS * kZ;
     float *Sst = p.Sstart + static_cast<size_t>(bh) * p.NS * 128 * 128;
     pdl_launch_dependents();
@@ -289,10 +303,14 @@ __global__ void __launch_bounds__(256, 1) gdn_combine_kernel(const ScanParams p)
         }
         cp_async_commit();
     };
-    auto load_sl = [&](int j, float2 (&v)[4]) {  // this thread's entries of S_loc(j)^T
+    // this thread's accumulator entries of S_loc(j)^T: rows r0+g (+8), columns 8n + 2t4 (+1), n = 0, 1
+    auto load_sl = [&](int j, float2 (&v)[2][2]) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-            v[k] = *reinterpret_cast<const float2 *>(Z + j * kZ + static_cast<size_t>(rbase + 32 * k) * 256 + col);
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+                v[n][hh] = *reinterpret_cast<const float2 *>(Z + j * kZ + static_cast<size_t>(r0 + g + 8 * hh) * 256 +
+                                                            slice * 16 + 8 * n + 2 * t4);
     };
     if (tid == 0) GDN_TRACE_AT(2048);
     if (p.NS > 2) load_pt(1);
@@ -304,10 +322,10 @@ __global__ void __launch_bounds__(256, 1) gdn_combine_kernel(const ScanParams p)
         curT[c * RS + t] = v;
         Sst[(static_cast<size_t>(1) * 128 + t) * 128 + slice * 16 + c] = v;
     }
-    float2 sl[4];
+    float2 sl[2][2];
     if (p.NS > 2) load_sl(1, sl);
     for (int j = 1; j + 1 < p.NS; ++j) {
-        float2 sn[4];
+        float2 sn[2][2];
         if (j + 2 < p.NS) {
             load_sl(j + 1, sn);
             load_pt(j + 1);
@@ -319,30 +337,59 @@ __global__ void __launch_bounds__(256, 1) gdn_combine_kernel(const ScanParams p)
         __syncthreads();  // P_j^T and the current state visible to all
         if (tid == 0) GDN_TRACE_AT(2048 + 8 * j + 1);
         const float *P = PT + (j & 1) * 128 * RS;
-        float acc[4][2];
+        // three accumulators per output tile (hi*hi, hi*lo, lo*hi): independent mma chains
+        float acc[2][4], ahl[2][4], alh[2][4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) acc[k][0] = acc[k][1] = 0.0f;
+        for (int n = 0; n < 2; ++n) {
+            acc[n][0] = sl[n][0].x;
+            acc[n][1] = sl[n][0].y;
+            acc[n][2] = sl[n][1].x;
+            acc[n][3] = sl[n][1].y;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) ahl[n][e] = alh[n][e] = 0.0f;
+        }
 #pragma unroll 4
-        for (int i = 0; i < 128; i += 4) {
-            const float4 c0 = *reinterpret_cast<const float4 *>(curT + cl * RS + i);
-            const float4 c1 = *reinterpret_cast<const float4 *>(curT + (cl + 1) * RS + i);
+        for (int k0 = 0; k0 < 128; k0 += 8) {
+            uint32_t ah[4], al[4];
+            split_tf32(P[(r0 + g) * RS + k0 + t4], ah[0], al[0]);
+            split_tf32(P[(r0 + g + 8) * RS + k0 + t4], ah[1], al[1]);
+            split_tf32(P[(r0 + g) * RS + k0 + t4 + 4], ah[2], al[2]);
+            split_tf32(P[(r0 + g + 8) * RS + k0 + t4 + 4], ah[3], al[3]);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float4 a = *reinterpret_cast<const float4 *>(P + (rbase + 32 * k) * RS + i);
-                acc[k][0] = fmaf(a.x, c0.x, fmaf(a.y, c0.y, fmaf(a.z, c0.z, fmaf(a.w, c0.w, acc[k][0]))));
-                acc[k][1] = fmaf(a.x, c1.x, fmaf(a.y, c1.y, fmaf(a.z, c1.z, fmaf(a.w, c1.w, acc[k][1]))));
+            for (int n = 0; n < 2; ++n) {
+                uint32_t bh2[2], bl2[2];
+                split_tf32(curT[(8 * n + g) * RS + k0 + t4], bh2[0], bl2[0]);
+                split_tf32(curT[(8 * n + g) * RS + k0 + t4 + 4], bh2[1], bl2[1]);
+                mma1688_tf32(alh[n], al, bh2);
+                mma1688_tf32(ahl[n], ah, bl2);
+                mma1688_tf32(acc[n], ah, bh2);
             }
         }
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[n][e] += ahl[n][e] + alh[n][e];
         if (tid == 0) GDN_TRACE_AT(2048 + 8 * j + 2);
         __syncthreads();  // every read of this step's state and P_j^T buffer is done
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int t = rbase + 32 * k;
-            const float v0 = acc[k][0] + sl[k].x, v1 = acc[k][1] + sl[k].y;
-            curT[cl * RS + t] = v0;
-            curT[(cl + 1) * RS + t] = v1;
-            *reinterpret_cast<float2 *>(Sst + (static_cast<size_t>(j + 1) * 128 + t) * 128 + col) = make_float2(v0, v1);
-            if (j + 2 < p.NS) sl[k] = sn[k];
+        for (int n = 0; n < 2; ++n) {
+            const int c = 8 * n + 2 * t4;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int t = r0 + g + 8 * hh;
+                const float v0 = acc[n][2 * hh], v1 = acc[n][2 * hh + 1];
+                curT[c * RS + t] = v0;
+                curT[(c + 1) * RS + t] = v1;
+                *reinterpret_cast<float2 *>(Sst + (static_cast<size_t>(j + 1) * 128 + t) * 128 + slice * 16 + c) =
+                    make_float2(v0, v1);
+            }
+        }
+        if (j + 2 < p.NS) {
+#pragma unroll
+            for (int n = 0; n < 2; ++n) {
+                sl[n][0] = sn[n][0];
+                sl[n][1] = sn[n][1];
+            }
         }
         if (tid == 0) GDN_TRACE_AT(2048 + 8 * j + 3);
     }
@@ -368,8 +415,8 @@ template <typename ZT>
 __global__ void __launch_bounds__(tc::kScanThreads, 1)
     gdn_scan_out_kernel(const ScanParams p, const __grid_constant__ CUtensorMap tmW,
                         const __grid_constant__ CUtensorMap tmQt, const __grid_constant__ CUtensorMap tmKt,
-                        const __grid_constant__ CUtensorMap tmAqk, const __grid_constant__ CUtensorMap tmU,
-                        const __grid_constant__ CUtensorMap tmZ) {
+                        const __grid_constant__ CUtensorMap tmAqk, const __grid_constant__ CUtensorMap tmAqkH,
+                        const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmZ) {
     using namespace tc;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -392,6 +439,10 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
         fence_mbar_init();
     }
     if (tid < kD) sNW[tid] = p.norm_w[tid];
+    // Aqk's upper-right 64x64 quadrant is zero and never loaded: clear it once
+    for (int e = tid; e < 64 * 128 / 16; e += kScanThreads)
+        reinterpret_cast<uint4 *>(sm + OFF_AQK + 16384)[e] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async();
     if (warp == 0) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
@@ -545,10 +596,11 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
                 mbar_arrive_expect_tx(&bars[FULL_U], 32768);
                 load2(OFF_U, &tmU, &bars[FULL_U], c);
             };
-            auto load_ka = [&](int c) {
-                mbar_arrive_expect_tx(&bars[FULL_KA], 65536);
+            auto load_ka = [&](int c) {  // Kt, and Aqk but for its zero upper-right quadrant
+                mbar_arrive_expect_tx(&bars[FULL_KA], 32768 + 16384 + 8192);
                 load2(OFF_KT, &tmKt, &bars[FULL_KA], c);
-                load2(OFF_AQK, &tmAqk, &bars[FULL_KA], c);
+                tma_load_2d(sm + OFF_AQK, &tmAqk, &bars[FULL_KA], 0, rowbase + c * kBlk);
+                tma_load_2d(sm + OFF_AQK + 16384 + 64 * 128, &tmAqkH, &bars[FULL_KA], 64, rowbase + c * kBlk + 64);
             };
             if (ok) {
                 load_wq(c0);
@@ -569,7 +621,8 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
                         tma_prefetch_2d(&tmQt, hf * 64, y2);
                         tma_prefetch_2d(&tmU, hf * 64, y2);
                         tma_prefetch_2d(&tmKt, hf * 64, y2);
-                        tma_prefetch_2d(&tmAqk, hf * 64, y2);
+                        if (hf == 0) tma_prefetch_2d(&tmAqk, 0, y2);
+                        else tma_prefetch_2d(&tmAqkH, 64, y2 + 64);
                     }
                 }
                 if (c + 1 < c1 && (c + 1) * kBlk < p.T)  // z rows the epilogue of block c+1 reads
@@ -749,21 +802,21 @@ cudaError_t launch_combine(const ScanParams &p, cudaStream_t s, bool pdl) {
 }
 
 cudaError_t launch_scan_out(const ScanParams &p, InType zt, const CUtensorMap &tmW, const CUtensorMap &tmQt,
-                            const CUtensorMap &tmKt, const CUtensorMap &tmAqk, const CUtensorMap &tmU,
-                            const CUtensorMap &tmZ, cudaStream_t s, bool pdl) {
+                            const CUtensorMap &tmKt, const CUtensorMap &tmAqk, const CUtensorMap &tmAqkH,
+                            const CUtensorMap &tmU, const CUtensorMap &tmZ, cudaStream_t s, bool pdl) {
     dim3 grid(p.NS, p.H, p.B);
     if (zt == InType::F16) {
         static bool attr = false;
         cudaError_t e = set_smem(gdn_scan_out_kernel<__half>, tc::SMEM_BYTES, attr);
         if (e != cudaSuccess) return e;
         return launch_k(gdn_scan_out_kernel<__half>, grid, dim3(tc::kScanThreads), tc::SMEM_BYTES, s, pdl, p, tmW,
-                        tmQt, tmKt, tmAqk, tmU, tmZ);
+                        tmQt, tmKt, tmAqk, tmAqkH, tmU, tmZ);
     }
     static bool attr = false;
     cudaError_t e = set_smem(gdn_scan_out_kernel<__nv_bfloat16>, tc::SMEM_BYTES, attr);
     if (e != cudaSuccess) return e;
     return launch_k(gdn_scan_out_kernel<__nv_bfloat16>, grid, dim3(tc::kScanThreads), tc::SMEM_BYTES, s, pdl, p, tmW,
-                    tmQt, tmKt, tmAqk, tmU, tmZ);
+                    tmQt, tmKt, tmAqk, tmAqkH, tmU, tmZ);
 }
 
 }  // namespace gdn

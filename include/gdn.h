@@ -183,7 +183,8 @@ int gdn_plan_segments(gdn_plan_t plan);
  *     up to 128),
  *   4 G (in-block cumulative log decay), 5 beta, 6 log alpha ([B][H][Tp] fp32),
  *   7 W, 8 U, 9 Qt, 10 Kt, 11 Aqk ([B][H][Tp][128] fp16; tensor path only,
- *     else 0), 12 o ([B][T][H][d_v] fp32 before the output norm; CUDA-core
+ *     else 0; Aqk is block lower triangular and its upper-right 64x64
+ *     quadrant in each 128-row block is never written), 12 o ([B][T][H][d_v] fp32 before the output norm; CUDA-core
  *     path only, else 0), 13 per-segment [S_loc^T | P^T] ([B][H][NS][128][256]
  *     fp32) and 14 segment start states S^T ([B][H][NS][128][128] fp32)
  *     (tensor path only, else 0).

@@ -84,7 +84,13 @@ def test_stage_outputs_of_tensor_path(T, g_mean):
     # K2: UT transform and decayed operands
     for name in ("Kt", "Qt", "Aqk", "W", "U"):
         got = _ws_array(ws, off[name], n_act, torch.float16).reshape(ref[name].shape)
-        r = _rel(got, ref[name])
+        want = ref[name]
+        if name == "Aqk":  # block lower triangular: the zero upper-right 64x64 quadrant is not stored
+            keep = np.ones((BLK, BLK), bool)
+            keep[:64, 64:] = False
+            keep = np.tile(keep, (Tp // BLK, 1))
+            got, want = got[..., keep], want[..., keep]
+        r = _rel(got, want)
         assert r < 5e-3, f"{name}: rel-L2 {r:.3e}"
     # segment transfer + combine: S^T at every segment start vs the oracle's state there
     NB = Tp // BLK
