@@ -52,10 +52,13 @@ constexpr uint32_t OFF_W = 0, OFF_KT = 32768, OFF_U = 65536;
 constexpr uint32_t OFF_Z = 98304;    // [S^T | P^T] fp16, 128 rows (d_k) x 256, MN-major B (4 panels)
 constexpr uint32_t OFF_D = 163840;   // Delta fp16, 128 rows (token) x 256, MN-major B
 constexpr uint32_t OFF_BAR = 229376;
-constexpr int NBAR = 7;
+constexpr int NBAR = 11;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
-enum { FULL_W = 0, FULL_U, FULL_K, MMA_X, MMA_P, CONS_D, CONS_S };
-// X and P share 256 columns (X is read out before P is written); the fp32
+// The two halves of the state (S^T: columns 0-127, P^T: 128-255) evolve independently, so each
+// has its own products and hand-offs (index + half): the tensor core works on one half while the
+// other half's warps process theirs.
+enum { FULL_W = 0, FULL_U, FULL_K, MMA_X, MMA_P = MMA_X + 2, CONS_D = MMA_P + 2, CONS_S = CONS_D + 2 };
+// Per half, X and P share 128 columns (X is read out before P is written); the fp32
 // state [S^T | P^T] lives in the other 256.
 constexpr uint32_t TM_X = 0, TM_P = 0, TM_Z = 256;
 }  // namespace ta
@@ -78,7 +81,7 @@ __global__ void __launch_bounds__(288, 1)
     const uint64_t lim = p.wait_limit_ns;
 
     if (tid == 0) {
-        for (int i = 0; i < NBAR; ++i) mbar_init(&bars[i], (i == CONS_D || i == CONS_S) ? 8 : 1);
+        for (int i = 0; i < NBAR; ++i) mbar_init(&bars[i], i >= CONS_D ? 4 : 1);
         ab->flag = 0;
         fence_mbar_init();
     }
@@ -104,8 +107,8 @@ __global__ void __launch_bounds__(288, 1)
             load2(OFF_W, &tmW, &bars[FULL_W], c0);
             load2(OFF_U, &tmU, &bars[FULL_U], c0);
             load2(OFF_KT, &tmKt, &bars[FULL_K], c0);
-            const uint32_t id_x = idesc_f16_f32(128, 256, false, true);
-            const uint32_t id_p = idesc_f16_f32(128, 256, true, true);
+            const uint32_t id_x = idesc_f16_f32(128, 128, false, true);
+            const uint32_t id_p = idesc_f16_f32(128, 128, true, true);
             bool ok = true;
             for (int c = c0; ok && c < c1; ++c) {
                 const uint32_t ph = (c - c0) & 1;
@@ -117,27 +120,38 @@ __global__ void __launch_bounds__(288, 1)
                         tma_prefetch_2d(&tmKt, hf * 64, y2);
                     }
                 }
-                ok = mbar_wait(&bars[FULL_W], ph, ab, p.status, lim) && mbar_wait(&bars[CONS_S], ph, ab, p.status, lim);
-                if (!ok) break;
-                tc_fence_after();
+                ok = mbar_wait(&bars[FULL_W], ph, ab, p.status, lim);
+                // X_h = W [S^T | P^T]_h  (A = W K-major, B = the half's two panels of Z, MN-major)
+                for (int hf = 0; ok && hf < 2; ++hf) {
+                    ok = mbar_wait(&bars[CONS_S + hf], ph, ab, p.status, lim);
+                    if (!ok) break;
+                    tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_f16(tmem + TM_X, sdesc_sw128(sbase + OFF_W + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                             sdesc_sw128(sbase + OFF_Z + kk * 2048, 16384, 1024), id_x, kk > 0);
-                umma_commit(&bars[MMA_X]);
-                ok = mbar_wait(&bars[MMA_X], ph, ab, p.status, lim);
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_f16(tmem + TM_X + hf * 128,
+                                 sdesc_sw128(sbase + OFF_W + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                                 sdesc_sw128(sbase + OFF_Z + hf * 32768 + kk * 2048, 16384, 1024), id_x, kk > 0);
+                    umma_commit(&bars[MMA_X + hf]);
+                }
+                ok = ok && mbar_wait(&bars[MMA_X], ph, ab, p.status, lim) &&
+                     mbar_wait(&bars[MMA_X + 1], ph, ab, p.status, lim);
                 if (!ok) break;
                 if (c + 1 < c1) load2(OFF_W, &tmW, &bars[FULL_W], c + 1);
-                ok = mbar_wait(&bars[FULL_K], ph, ab, p.status, lim) && mbar_wait(&bars[CONS_D], ph, ab, p.status, lim);
-                if (!ok) break;
-                if (c + 1 < c1) load2(OFF_U, &tmU, &bars[FULL_U], c + 1);
-                tc_fence_after();
+                ok = mbar_wait(&bars[FULL_K], ph, ab, p.status, lim);
+                // P_h = Kt^T Delta_h  (A = Kt MN-major: M = d_k, K = token; B = the half's panels of Delta)
+                for (int hf = 0; ok && hf < 2; ++hf) {
+                    ok = mbar_wait(&bars[CONS_D + hf], ph, ab, p.status, lim);
+                    if (!ok) break;
+                    if (hf == 0 && c + 1 < c1) load2(OFF_U, &tmU, &bars[FULL_U], c + 1);  // U's only readers are done
+                    tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_f16(tmem + TM_P, sdesc_sw128(sbase + OFF_KT + kk * 2048, 16384, 1024),
-                             sdesc_sw128(sbase + OFF_D + kk * 2048, 16384, 1024), id_p, kk > 0);
-                umma_commit(&bars[MMA_P]);
-                ok = mbar_wait(&bars[MMA_P], ph, ab, p.status, lim);
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_f16(tmem + TM_P + hf * 128, sdesc_sw128(sbase + OFF_KT + kk * 2048, 16384, 1024),
+                                 sdesc_sw128(sbase + OFF_D + hf * 32768 + kk * 2048, 16384, 1024), id_p, kk > 0);
+                    umma_commit(&bars[MMA_P + hf]);
+                }
+                ok = ok && mbar_wait(&bars[MMA_P], ph, ab, p.status, lim) &&
+                     mbar_wait(&bars[MMA_P + 1], ph, ab, p.status, lim);
                 if (!ok) break;
                 if (c + 1 < c1) load2(OFF_KT, &tmKt, &bars[FULL_K], c + 1);
             }
@@ -160,13 +174,14 @@ __global__ void __launch_bounds__(288, 1)
         fence_proxy_async();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[CONS_S]);
+        if (lane == 0) mbar_arrive(&bars[CONS_S + half]);
         const float *Gbh = p.G + static_cast<size_t>(bh) * p.Tp;
         bool ok = true;
         for (int c = c0; c < c1; ++c) {
             const uint32_t ph = (c - c0) & 1;
             const float gC = __expf(fminf(Gbh[c * kBlk + kBlk - 1], 0.0f));
-            ok = warp_wait(&bars[MMA_X], ph, ab, p.status, lim) && warp_wait(&bars[FULL_U], ph, ab, p.status, lim);
+            ok = warp_wait(&bars[MMA_X + half], ph, ab, p.status, lim) &&
+                 (half == 1 || warp_wait(&bars[FULL_U], ph, ab, p.status, lim));
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
@@ -195,8 +210,8 @@ __global__ void __launch_bounds__(288, 1)
             fence_proxy_async();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[CONS_D]);
-            ok = warp_wait(&bars[MMA_P], ph, ab, p.status, lim);
+            if (lane == 0) mbar_arrive(&bars[CONS_D + half]);
+            ok = warp_wait(&bars[MMA_P + half], ph, ab, p.status, lim);
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
@@ -215,7 +230,7 @@ __global__ void __launch_bounds__(288, 1)
             fence_proxy_async();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[CONS_S]);
+            if (lane == 0) mbar_arrive(&bars[CONS_S + half]);
         }
         if (ok) {
             tc_fence_after();
