@@ -315,6 +315,7 @@ __global__ void __launch_bounds__(256, 2)
             *reinterpret_cast<uint32_t *>(Tt + tile_elem_off(128, 16 * i + g + 8, col + 8)) = pack_half2(o1[2], o1[3]);
         }
         group_sync(1);
+        if (tid == 0) GDN_TRACE_AT(20);
         // ---- block rows i = 1..7: T_ij = -sum_{k=j}^{i-1} M_ik T_kj, as two 16x8 halves each; the
         //      2i halves of a level are spread over the four warps, computed, then (after a barrier,
         //      since M_ij is still read by the level's other halves) written over M_ij
@@ -352,6 +353,7 @@ __global__ void __launch_bounds__(256, 2)
                 }
             }
             group_sync(1);
+            if (tid == 0) GDN_TRACE_AT(20 + i);
         }
         fence_proxy_async();  // T is read by the tensor cores next
         if (tid == 0) GDN_TRACE_AT(4);
@@ -384,6 +386,7 @@ __global__ void __launch_bounds__(256, 2)
                 *pu = make_uint4(os[0], os[1], os[2], os[3]);
             }
         }
+        if (tid == 128) GDN_TRACE_AT(10);
         // ---- Qt = e^G Q over the Q tile in place -> bulk store
         scale_row(sm + OFF_QV, r, fq);
         fence_proxy_async();
@@ -395,6 +398,7 @@ __global__ void __launch_bounds__(256, 2)
             bulk_wait_read_all();
         }
         group_sync(2);
+        if (tid == 128) GDN_TRACE_AT(11);
         // ---- Aqk rows (same split of the decay as the L rows) staged in the same area -> bulk
         //      store; then the V tile is loaded into it
         const int w = warp & 3;
@@ -433,9 +437,11 @@ __global__ void __launch_bounds__(256, 2)
             tma_load_2d(sm + OFF_QV, &tmV, bar_v, 0, y0);
             tma_load_2d(sm + OFF_QV + 16384, &tmV, bar_v, 64, y0);
         }
+        if (tid == 128) GDN_TRACE_AT(12);
         // ---- V~ = diag(beta) V, row r
         if (mbar_wait(bar_v, 0, ab, p.status, p.wait_limit_ns)) scale_row(sm + OFF_QV, r, sBeta[r]);
         fence_proxy_async();
+        if (tid == 128) GDN_TRACE_AT(13);
     }
     tc_fence_before();
     __syncthreads();  // T, V~ and K~ complete

@@ -1,0 +1,39 @@
+"""Back-to-back forwards on one stream and one workspace.
+
+Consecutive kernels of a forward start early (programmatic dependent launch:
+each runs its prologue while the previous kernel finishes and waits before
+touching its outputs), and consecutive forwards reuse the workspace.  Two
+input sets alternate ten times with no synchronisation in between; every
+output must equal, bit for bit, the output of a single forward on a fresh
+workspace.  The shape (48 heads, 12 blocks) gives segments of several blocks,
+so that every kernel of the tensor path runs with more than one block per CTA.
+"""
+import pytest
+
+import gdn_inputs
+from gpu_util import torch_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def test_alternating_forwards_on_one_workspace_match_fresh_runs():
+    import torch
+    import gated_deltanet_06_b200 as gdn
+    B, T, H, d = 2, 1500, 24, 128
+    sets = [torch_inputs(gdn_inputs.make_inputs(B, T, H, d, "bf16", g, seed=s)) for g, s in ((-1.0, 41), (-6.0, 42))]
+    plan = gdn.Plan(B, T, H, d, gdn.DTYPE_BF16)
+    assert plan.uses_tensor_path and plan.segments > 1 and plan.segments < -(-T // 128)
+    fresh = []
+    for t in sets:
+        ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device="cuda")
+        fresh.append(gdn.forward(**t, plan=plan, workspace=ws))
+    torch.cuda.synchronize()
+    ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device="cuda")
+    outs = []
+    for k in range(10):
+        outs.append(gdn.forward(**sets[k % 2], plan=plan, workspace=ws))
+    torch.cuda.synchronize()
+    assert plan.device_status(ws.data_ptr(), torch.cuda.current_stream().cuda_stream) == gdn.OK
+    for k, y in enumerate(outs):
+        assert torch.equal(y, fresh[k % 2]), f"forward {k} differs from a fresh run"
+    assert not torch.equal(fresh[0], fresh[1])
