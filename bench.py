@@ -220,6 +220,21 @@ def reference_arm(args, w):
     return 0
 
 
+def ranks_max(x, world, dist=None, device=None):
+    """The max of x over the ranks (every rank gets it); x itself with one rank."""
+    if world <= 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, tokens_per_rank, ms_per_step):
+    """Whole-job Mtokens/s: every rank processes its own replica of the workload per step."""
+    return world * tokens_per_rank / (ms_per_step / 1e3) / 1e6
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -327,14 +342,10 @@ def main():
     torch.cuda.synchronize()
     kern_ms = {names[i]: statistics.mean(events[k][i].elapsed_time(events[k][i + 1]) for k in range(n_kt))
                for i in range(L)}
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = ranks_max(sum(step_ms), world, dist, dev)
     ms_per_step = total_ms / args.steps
     tokens = w.B * w.T
-    value = world * tokens / (ms_per_step / 1e3) / 1e6
+    value = job_throughput(world, tokens, ms_per_step)
 
     # end to end through the public host-buffer entry point
     e2e = None
@@ -354,12 +365,10 @@ def main():
             plan.forward_host_raw(hptrs, y_host.data_ptr(), staging.data_ptr(), ws.data_ptr(), s)
         ev1.record(stream)
         torch.cuda.synchronize()
-        te = torch.tensor([ev0.elapsed_time(ev1) / n_e2e], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        te_ms = ranks_max(ev0.elapsed_time(ev1) / n_e2e, world, dist, dev)
         h2d = sum(host[n].numel() * host[n].element_size() for n in host)
         d2h = y_host.numel() * y_host.element_size()
-        e2e = {"value": world * tokens / (float(te.item()) / 1e3) / 1e6, "unit": UNIT,
+        e2e = {"value": job_throughput(world, tokens, te_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n_e2e}
 
     if rank != 0:
