@@ -314,7 +314,7 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
         // Kernels after the first start with programmatic dependent launch (prologue overlapped with
         // the previous kernel's tail), except when per-kernel events are recorded between them.
         const bool pdl = events == nullptr;
-        if (!mark() || launch_chunk(cp, tmK, tmV, tmQ, tmW, tmU, tmQt, tmKt, tmAqk, tmAqkH, s, pdl) != cudaSuccess)
+        if (!mark() || launch_chunk(cp, tmK, tmV, tmQ, tmW, tmU, tmQt, tmAqk, tmAqkH, s, pdl) != cudaSuccess)
             return GDN_ERR_CUDA;
         ScanParams sp;
         sp.G = G;

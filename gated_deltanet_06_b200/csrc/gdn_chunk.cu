@@ -118,8 +118,8 @@ __global__ void __launch_bounds__(256, 2)
     gdn_chunk_kernel(const ChunkParams p, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmU,
-                     const __grid_constant__ CUtensorMap tmQt, const __grid_constant__ CUtensorMap tmKt,
-                     const __grid_constant__ CUtensorMap tmAqk, const __grid_constant__ CUtensorMap tmAqkH) {
+                     const __grid_constant__ CUtensorMap tmQt, const __grid_constant__ CUtensorMap tmAqk,
+                     const __grid_constant__ CUtensorMap tmAqkH) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
@@ -504,8 +504,8 @@ teardown:
 
 cudaError_t launch_chunk(const ChunkParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
                          const CUtensorMap &tmQ, const CUtensorMap &tmW, const CUtensorMap &tmU,
-                         const CUtensorMap &tmQt, const CUtensorMap &tmKt, const CUtensorMap &tmAqk,
-                         const CUtensorMap &tmAqkH, cudaStream_t s, bool pdl) {
+                         const CUtensorMap &tmQt, const CUtensorMap &tmAqk, const CUtensorMap &tmAqkH,
+                         cudaStream_t s, bool pdl) {
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(gdn_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -514,8 +514,8 @@ cudaError_t launch_chunk(const ChunkParams &p, const CUtensorMap &tmK, const CUt
         attr_set = true;
     }
     dim3 grid(p.NB, p.BH);
-    return launch_k(gdn_chunk_kernel, grid, dim3(256), SMEM_BYTES, s, pdl, p, tmK, tmV, tmQ, tmW, tmU, tmQt, tmKt,
-                    tmAqk, tmAqkH);
+    return launch_k(gdn_chunk_kernel, grid, dim3(256), SMEM_BYTES, s, pdl, p, tmK, tmV, tmQ, tmW, tmU, tmQt, tmAqk,
+                    tmAqkH);
 }
 
 }  // namespace gdn

@@ -68,8 +68,8 @@ struct ChunkParams {
 };
 cudaError_t launch_chunk(const ChunkParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
                          const CUtensorMap &tmQ, const CUtensorMap &tmW, const CUtensorMap &tmU,
-                         const CUtensorMap &tmQt, const CUtensorMap &tmKt, const CUtensorMap &tmAqk,
-                         const CUtensorMap &tmAqkH, cudaStream_t s, bool pdl);
+                         const CUtensorMap &tmQt, const CUtensorMap &tmAqk, const CUtensorMap &tmAqkH,
+                         cudaStream_t s, bool pdl);  // Kt is written with plain coalesced stores
 
 // Inter-block state scan on tensor cores (d = 128), parallel over segments of
 // Ls blocks: pass A (transfer), combine, pass C (outputs + fused output step).

@@ -11,18 +11,21 @@
 // segments processed in parallel:
 //   pass A  (gdn_transfer_kernel): per segment, run the state and the
 //           transfer together as one 256-column state [S^T | P^T] from
-//           [0 | I]; write both (fp32).
+//           [0 | I], its two halves as independent, interleaved chains;
+//           write both (fp32).
 //   combine (gdn_combine_kernel): S_start(j+1)^T = P_j^T S_start(j)^T + S_loc(j)^T,
 //           sequential over segments, split-precision tf32 tensor-core products
 //           (close to fp32), P_j^T staged in shared memory one segment ahead.
 //   pass C  (gdn_scan_out_kernel): per segment, run the state from S_start and
 //           emit the block outputs, with the output step fused into the
 //           epilogue:  y = o / sqrt(mean(o^2) + eps) * w * SiLU(z).
-// In both tensor-core kernels a producer warp issues the TMA loads of the next
-// block as soon as each tile's last reader has finished, and all MMAs;
-// consumer warps own TMEM lanes (one row each) and keep the fp32 state in
-// registers.  Every hand-off is an mbarrier with a bounded wait, so a lost
-// arrival ends the kernel with a timeout status instead of a hang.
+// In both passes a producer warp issues the TMA loads of the next block as
+// soon as each tile's last reader has finished, and all MMAs; consumer warps
+// own TMEM lanes (one row each) and keep the fp32 state in TMEM.  Every
+// hand-off is an mbarrier with a bounded wait, so a lost arrival ends the
+// kernel with a timeout status instead of a hang.  All three kernels are
+// launched behind the previous kernel with programmatic dependent launch and
+// wait for it (griddepcontrol.wait) before reading its outputs.
 #include <type_traits>
 
 #include "gdn_common.cuh"
