@@ -148,6 +148,19 @@ def forward(inp: dict, l2_eps=DEFAULT_L2_EPS, norm_eps=DEFAULT_NORM_EPS, nthread
     return (y, inter) if intermediates else y
 
 
+def forward_with_state(inp: dict, s0=None, l2_eps=DEFAULT_L2_EPS, norm_eps=DEFAULT_NORM_EPS, nthreads=None):
+    """Steps 1-5 with the recurrent state carried in and out: s0
+    [B,H,d_v,d_k] (None = zero) is the state S before token 0; returns y and
+    the state after token T-1.  Composed of the step functions above; the
+    short convolutions still see zero history before token 0."""
+    qh = l2norm(conv_silu(inp["q"], inp["conv_q"]), l2_eps)
+    kh = l2norm(conv_silu(inp["k"], inp["conv_k"]), l2_eps)
+    vh = conv_silu(inp["v"], inp["conv_v"])
+    alpha, beta = gates(inp["g"], inp["b"], inp["A_log"], inp["dt_bias"])
+    o, s_end = core(qh, kh, vh, alpha, beta, s0=s0, return_state=True, nthreads=nthreads)
+    return output(o, inp["z"], inp["norm_w"], norm_eps), s_end
+
+
 class _swapped_library:
     """Context manager used by the oracle's own mutation tests: temporarily
     route every call above to another build of gdn_oracle.c (a copy with a

@@ -331,3 +331,27 @@ def test_segment_parallel_states_equal_sequential_states(Ls):
         _, S = oracle.core(it["qh"][:, :t_end], it["kh"][:, :t_end], it["vh"][:, :t_end], it["alpha"][:, :t_end],
                            it["beta"][:, :t_end], return_state=True)
         np.testing.assert_allclose(St, S[0, 0].T, rtol=0, atol=1e-12 * max(1.0, np.abs(S).max()))
+
+
+# ------------------------------------------------ carried state (streaming)
+def test_forward_with_zero_initial_state_is_the_plain_forward():
+    inp = gdn_inputs.make_inputs(1, 130, 2, 16, "f32", -1.0, seed=61)
+    y, s = oracle.forward_with_state(inp)
+    np.testing.assert_allclose(y, oracle.forward(inp), rtol=1e-12, atol=1e-14)
+    assert s.shape == (1, 2, 16, 16)
+
+
+def test_streaming_in_two_pieces_equals_one_pass():
+    # g ~ N(-6, 1): alpha ~ 0.95-0.99, so the carried state dominates the second piece
+    from state_util import split_stream
+    inp = gdn_inputs.make_inputs(1, 300, 2, 32, "f32", -6.0, seed=62)
+    y, s = oracle.forward_with_state(inp)
+    p1, p2 = split_stream(inp, 170)
+    y1, s1 = oracle.forward_with_state(p1)
+    y2, s2 = oracle.forward_with_state(p2, s0=s1)
+    np.testing.assert_allclose(y1, y[:, :170], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(y2[:, 3:], y[:, 170:], rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(s2, s, rtol=1e-9, atol=1e-12)
+    # without the carried state the second piece differs
+    y2z, _ = oracle.forward_with_state(p2)
+    assert np.abs(y2z[:, 3:] - y[:, 170:]).max() > 1e-3
