@@ -246,6 +246,7 @@ def main():
     ap.add_argument("--out-dtype", default=None, choices=[None, "bf16", "f16", "f32"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-state", action="store_true", help="skip the carried-state timing")
     ap.add_argument("--load-seconds", type=float, default=1.5)
     args = ap.parse_args()
     w = gdn_inputs.by_name(args.workload)
@@ -347,6 +348,27 @@ def main():
     tokens = w.B * w.T
     value = job_throughput(world, tokens, ms_per_step)
 
+    # the same forward with the recurrent state carried in and out (gdn_forward_state): an initial
+    # state read and the final state written, [B][H][d][d] fp32 each
+    state_io = None
+    if not args.no_state:
+        s0 = torch.randn((w.B, w.H, w.d, w.d), dtype=torch.float32, device=dev).mul_(0.5)
+        s_end = torch.empty_like(s0)
+        n_st = max(3, min(args.steps, 10))
+        for _ in range(2):
+            plan.forward_state_raw(ptrs, s0.data_ptr(), y.data_ptr(), s_end.data_ptr(), ws.data_ptr(), s)
+        ev_st = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_st)]
+        torch.cuda.synchronize()
+        for k in range(n_st):
+            flush.zero_()
+            ev_st[k][0].record(stream)
+            plan.forward_state_raw(ptrs, s0.data_ptr(), y.data_ptr(), s_end.data_ptr(), ws.data_ptr(), s)
+            ev_st[k][1].record(stream)
+        torch.cuda.synchronize()
+        st_ms = ranks_max(sum(a.elapsed_time(b) for a, b in ev_st), world, dist, dev) / n_st
+        state_io = {"ms_per_step": st_ms, "value": job_throughput(world, w.B * w.T, st_ms), "unit": UNIT,
+                    "state_bytes_per_step": 2 * w.B * w.H * w.d * w.d * 4, "steps": n_st}
+
     # end to end through the public host-buffer entry point
     e2e = None
     if not args.no_e2e:
@@ -419,7 +441,7 @@ def main():
                        "l2": "flushed before every step (256 MiB write, outside the timed interval)",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "roofline": roof, "path_roofline": path_roof, "kernels_ms": kern_ms,
-            "segments": plan.segments, "cpu_baseline": cpu, "e2e": e2e,
+            "segments": plan.segments, "cpu_baseline": cpu, "e2e": e2e, "state_io": state_io,
             "clocks": clocks, "gpu_launches": L * args.steps,
             "gpu": torch.cuda.get_device_name(dev)}
     print(json.dumps(line), flush=True)

@@ -49,6 +49,8 @@ _lib.gdn_plan.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(_vp), ctypes.PO
 _lib.gdn_plan.restype = ctypes.c_int
 _lib.gdn_forward.argtypes = [_vp, ctypes.POINTER(Inputs), _vp, _vp, _vp]
 _lib.gdn_forward.restype = ctypes.c_int
+_lib.gdn_forward_state.argtypes = [_vp, ctypes.POINTER(Inputs), _vp, _vp, _vp, _vp, _vp]
+_lib.gdn_forward_state.restype = ctypes.c_int
 _lib.gdn_forward_timed.argtypes = [_vp, ctypes.POINTER(Inputs), _vp, _vp, _vp, ctypes.POINTER(_vp), ctypes.c_int]
 _lib.gdn_forward_timed.restype = ctypes.c_int
 _lib.gdn_forward_host.argtypes = [_vp, ctypes.POINTER(Inputs), _vp, _vp, _vp, _vp]
@@ -136,6 +138,12 @@ class Plan:
         ins = Inputs(*[ptrs[n] for n, _ in Inputs._fields_])
         _check(_lib.gdn_forward(self._h, ctypes.byref(ins), y, workspace, stream), "gdn_forward")
 
+    def forward_state_raw(self, ptrs: dict, s0: int, y: int, s_end: int, workspace: int, stream: int) -> None:
+        """gdn_forward_state: s0 / s_end are device addresses of [B][H][d][d] fp32 states (0 = none)."""
+        ins = Inputs(*[ptrs[n] for n, _ in Inputs._fields_])
+        _check(_lib.gdn_forward_state(self._h, ctypes.byref(ins), s0 or None, y, s_end or None, workspace, stream),
+               "gdn_forward_state")
+
     def forward_timed_raw(self, ptrs: dict, y: int, workspace: int, stream: int, events: list) -> None:
         """gdn_forward_timed: `events` are cudaEvent_t handles (ints), launches + 1 of them."""
         ins = Inputs(*[ptrs[n] for n, _ in Inputs._fields_])
@@ -192,9 +200,12 @@ def tensor_ptrs(tensors: dict) -> dict:
 
 
 def forward(q, k, v, z, g, b, conv_q, conv_k, conv_v, A_log, dt_bias, norm_w, out_dtype=None,
-            l2_eps=1e-6, norm_eps=1e-6, plan: Plan | None = None, workspace=None, y=None, stream=None):
+            l2_eps=1e-6, norm_eps=1e-6, plan: Plan | None = None, workspace=None, y=None, stream=None,
+            s0=None, return_state=False):
     """GDN forward on CUDA tensors (q, k, v, z [B,T,H,d]; g, b [B,T,H] fp32; conv_* [H*d,4];
-    A_log, dt_bias [H]; norm_w [d]).  Returns y [B,T,H,d]."""
+    A_log, dt_bias [H]; norm_w [d]).  Returns y [B,T,H,d].  With s0 (a [B,H,d,d] fp32 state S[i][j],
+    i over d_v, j over d_k) the recurrence starts from it; with return_state=True the call returns
+    (y, s_end), s_end the [B,H,d,d] fp32 state after the last token."""
     import torch
     B, T, H, d = q.shape
     in_code = _torch_dtype_code(q.dtype)
@@ -208,5 +219,12 @@ def forward(q, k, v, z, g, b, conv_q, conv_k, conv_v, A_log, dt_bias, norm_w, ou
     s = torch.cuda.current_stream(q.device).cuda_stream if stream is None else stream
     t = dict(q=q, k=k, v=v, z=z, g=g, b=b, conv_q=conv_q, conv_k=conv_k, conv_v=conv_v, A_log=A_log,
              dt_bias=dt_bias, norm_w=norm_w)
-    plan.forward_raw(tensor_ptrs(t), y.data_ptr(), workspace.data_ptr(), s)
-    return y
+    if s0 is None and not return_state:
+        plan.forward_raw(tensor_ptrs(t), y.data_ptr(), workspace.data_ptr(), s)
+        return y
+    if s0 is not None and (s0.dtype != torch.float32 or tuple(s0.shape) != (B, H, d, d) or not s0.is_contiguous()):
+        raise ValueError("s0 must be a contiguous [B, H, d, d] float32 tensor")
+    s_end = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device) if return_state else None
+    plan.forward_state_raw(tensor_ptrs(t), 0 if s0 is None else s0.data_ptr(), y.data_ptr(),
+                           0 if s_end is None else s_end.data_ptr(), workspace.data_ptr(), s)
+    return (y, s_end) if return_state else y

@@ -234,9 +234,16 @@ int gdn_workspace_offsets(gdn_plan_t plan, size_t *offsets, int n) {
 }
 
 static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, void *workspace,
-                               gdn_stream_t stream, void *const *events) {
+                               gdn_stream_t stream, void *const *events, const float *s0 = nullptr,
+                               float *s_end = nullptr) {
     if (!plan || !in || !y || !workspace) return GDN_ERR_INVALID_ARG;
     const gdn_config &c = plan->cfg;
+    if ((s0 && !aligned16(s0)) || (s_end && !aligned16(s_end))) return GDN_ERR_INVALID_ARG;
+    if (s0 && s_end) {  // the end state is written while other CTAs may still read the initial one
+        const size_t bytes = static_cast<size_t>(c.B) * c.H * c.d_v * c.d_k * sizeof(float);
+        const uintptr_t a = reinterpret_cast<uintptr_t>(s0), e = reinterpret_cast<uintptr_t>(s_end);
+        if (a < e + bytes && e < a + bytes) return GDN_ERR_INVALID_ARG;
+    }
     const void *ptrs16[] = {in->q, in->k, in->v, in->z, y};
     for (const void *q : ptrs16)
         if (!q || !aligned16(q)) return GDN_ERR_INVALID_ARG;
@@ -327,6 +334,8 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
         sp.status = status;
         sp.wait_limit_ns = kWaitLimitNs;
         sp.test_wait_timeout = (c.flags & GDN_FLAG_TEST_WAIT_TIMEOUT) ? 1 : 0;
+        sp.s0 = s0;
+        sp.s_end = s_end;
         if (plan->NS > 1) {
             if (!mark() || launch_transfer(sp, tmW, tmKt, tmU, s, pdl) != cudaSuccess) return GDN_ERR_CUDA;
             if (!mark() || launch_combine(sp, s, pdl) != cudaSuccess) return GDN_ERR_CUDA;
@@ -344,6 +353,7 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
         rp.vh = reinterpret_cast<const float *>(ws + plan->off_vh);
         rp.log_alpha = la; rp.beta = beta; rp.o = o;
         rp.B = c.B; rp.T = c.T; rp.H = c.H; rp.d = d; rp.Tp = plan->Tp;
+        rp.s0 = s0; rp.s_end = s_end;
         if (!mark() || launch_recurrence(rp, s) != cudaSuccess) return GDN_ERR_CUDA;
     }
 
@@ -358,6 +368,11 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
 
 gdn_status gdn_forward(gdn_plan_t plan, const gdn_inputs *in, void *y, void *workspace, gdn_stream_t stream) {
     return forward_impl(plan, in, y, workspace, stream, nullptr);
+}
+
+gdn_status gdn_forward_state(gdn_plan_t plan, const gdn_inputs *in, const float *s0, void *y, float *s_end,
+                             void *workspace, gdn_stream_t stream) {
+    return forward_impl(plan, in, y, workspace, stream, nullptr, s0, s_end);
 }
 
 gdn_status gdn_forward_timed(gdn_plan_t plan, const gdn_inputs *in, void *y, void *workspace,

@@ -87,6 +87,8 @@ struct ScanParams {
     int *status;
     unsigned long long wait_limit_ns;
     int test_wait_timeout;
+    const float *s0;         // [BH][128 (d_v)][128 (d_k)] state before token 0, or null (zero)
+    float *s_end;            // [BH][128][128] state after token T-1, or null (not wanted)
 };
 // pdl: launch with programmatic stream serialization (see launch_k).
 cudaError_t launch_transfer(const ScanParams &p, const CUtensorMap &tmW, const CUtensorMap &tmKt,
@@ -102,6 +104,8 @@ struct RecurParams {
     const float *log_alpha, *beta;
     float *o;  // [B][T][H][d]
     int B, T, H, d, Tp;
+    const float *s0;  // [B*H][d][d] (S[i][j], i over d_v) before token 0, or null (zero)
+    float *s_end;     // [B*H][d][d] after token T-1, or null
 };
 cudaError_t launch_recurrence(const RecurParams &p, cudaStream_t s);
 

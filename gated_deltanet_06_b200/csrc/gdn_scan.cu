@@ -12,13 +12,16 @@
 //   pass A  (gdn_transfer_kernel): per segment, run the state and the
 //           transfer together as one 256-column state [S^T | P^T] from
 //           [0 | I], its two halves as independent, interleaved chains;
-//           write both (fp32).
+//           write both (fp32).  With a given initial state S_0, segment 0
+//           starts from [S_0^T | I] and so ends at S_start(1) itself.
 //   combine (gdn_combine_kernel): S_start(j+1)^T = P_j^T S_start(j)^T + S_loc(j)^T,
 //           sequential over segments, split-precision tf32 tensor-core products
 //           (close to fp32), P_j^T staged in shared memory one segment ahead.
-//   pass C  (gdn_scan_out_kernel): per segment, run the state from S_start and
-//           emit the block outputs, with the output step fused into the
-//           epilogue:  y = o / sqrt(mean(o^2) + eps) * w * SiLU(z).
+//   pass C  (gdn_scan_out_kernel): per segment, run the state from S_start
+//           (S_0 or zero for segment 0) and emit the block outputs, with the
+//           output step fused into the epilogue:
+//           y = o / sqrt(mean(o^2) + eps) * w * SiLU(z);
+//           the last segment writes the final state when it is wanted.
 // In both passes a producer warp issues the TMA loads of the next block as
 // soon as each tile's last reader has finished, and all MMAs; consumer warps
 // own TMEM lanes (one row each) and keep the fp32 state in TMEM.  Every
@@ -169,6 +172,12 @@ __global__ void __launch_bounds__(288, 1)
             float v[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] = (half == 1 && ch * 32 + e == r) ? 1.0f : 0.0f;
+            if (half == 0 && seg == 0 && p.s0) {
+                // a given initial state: segment 0 then ends at S_start(1) itself (S_loc(0) = s0 P_0 + S_loc)
+                const float *src = p.s0 + (static_cast<size_t>(bh) * 128 + ch * 32) * 128 + r;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] = src[static_cast<size_t>(e) * 128];
+            }
             tmem_st32(tz + ch * 32, v);
 #pragma unroll
             for (int qq = 0; qq < 4; ++qq) store_f16_chunk(sm + OFF_Z, 128, r, half * 16 + ch * 4 + qq, &v[qq * 8]);
@@ -705,8 +714,10 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
         for (int ch = 0; ch < 4; ++ch) {
             float v[32];
             if (seg == 0) {
+                // S^T row r = column r of the initial state (zero unless one is given)
+                const float *src = p.s0 ? p.s0 + (static_cast<size_t>(bh) * 128 + ch * 32) * 128 + r : nullptr;
 #pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] = 0.0f;
+                for (int e = 0; e < 32; ++e) v[e] = src ? src[static_cast<size_t>(e) * 128] : 0.0f;
             } else {
                 const float *src = p.Sstart + ((static_cast<size_t>(bh) * p.NS + seg) * 128 + r) * 128 + ch * 32;
 #pragma unroll
@@ -726,7 +737,9 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
         if (lane == 0) mbar_arrive(&bars[CONS_S]);
 
         const float *Gbh = p.G + static_cast<size_t>(bh) * p.Tp;
+        bool done = true;
         for (int c = c0; c < c1; ++c) {
+            done = false;
             const int i = c - c0;
             const uint32_t ph = i & 1;
             const float gC = __expf(fminf(Gbh[c * kBlk + kBlk - 1], 0.0f));
@@ -783,6 +796,19 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[CONS_S]);
             if (tr) GDN_TRACE_AT(4096 + 64 * i + 21);
+            done = true;
+        }
+        if (done && p.s_end && seg == p.NS - 1) {
+            // the state after the last block (padding tokens leave it unchanged): S^T row r is
+            // column r of S; a warp's 32 lanes write 32 consecutive floats of each row of S
+            float *dst = p.s_end + (static_cast<size_t>(bh) * 128) * 128 + r;
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                float sv[32];
+                tmem_ld32(tmem + lane_base + TM_S + ch * 32, sv);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) dst[static_cast<size_t>(ch * 32 + e) * 128] = sv[e];
+            }
         }
     }
 

@@ -21,9 +21,10 @@ __global__ void __launch_bounds__(D) gdn_recurrence_kernel(const RecurParams p) 
     __shared__ float sk[TT][D], sq[TT][D], sv[TT][D], sa[TT], sb[TT];
     const int h = blockIdx.x, b = blockIdx.y, i = threadIdx.x;
     const size_t bh = static_cast<size_t>(b) * p.H + h;
-    float S[D];
+    float S[D];  // row i of the state (d_v index i, d_k index j)
+    const float *s0 = p.s0 ? p.s0 + (bh * D + i) * D : nullptr;
 #pragma unroll
-    for (int j = 0; j < D; ++j) S[j] = 0.0f;
+    for (int j = 0; j < D; ++j) S[j] = s0 ? s0[j] : 0.0f;
     for (int t0 = 0; t0 < p.T; t0 += TT) {
         __syncthreads();
 #pragma unroll 4
@@ -54,6 +55,11 @@ __global__ void __launch_bounds__(D) gdn_recurrence_kernel(const RecurParams p) 
             }
             p.o[((static_cast<size_t>(b) * p.T + t0 + tok) * p.H + h) * D + i] = o;
         }
+    }
+    if (p.s_end) {
+        float *se = p.s_end + (bh * D + i) * D;
+#pragma unroll
+        for (int j = 0; j < D; ++j) se[j] = S[j];
     }
 }
 

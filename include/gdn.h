@@ -118,6 +118,27 @@ gdn_status gdn_plan(const gdn_config *cfg, gdn_plan_t *out, size_t *workspace_by
 gdn_status gdn_forward(gdn_plan_t plan, const gdn_inputs *in, void *y, void *workspace,
                        gdn_stream_t stream);
 
+/* gdn_forward with the recurrent state carried in and out, for processing a
+ * sequence in pieces (streaming, or a sequence longer than one call).  The
+ * recurrence of the gated delta rule (reference [57] on the VMonarch page,
+ * References) starts from S_{-1} = s0 instead of zero, and the state after
+ * token T-1 is written to s_end:
+ *   s0, s_end  [B][H][d_v][d_k] fp32 row-major, S[i][j] with i over d_v and j
+ *              over d_k (so that o_t = S_t q^_t); device pointers, 16-byte
+ *              aligned, owned by the caller.  s0 = NULL starts from zero (the
+ *              result is then bit for bit that of gdn_forward); s_end = NULL
+ *              skips the write.  The two must not overlap (ping-pong two
+ *              buffers between pieces): INVALID_ARG otherwise.
+ * Only the recurrent state is carried.  The short convolutions of each call
+ * see zero history before its token 0; a caller that needs the exact
+ * continuation of a longer sequence prepends the previous piece's last 3
+ * tokens with neutral gates (b = -200, so beta = 0 in fp32 and the state
+ * only decays; g = -200 too, so alpha = 1 in fp32 and it does not decay) and
+ * drops their 3 outputs.  Same inputs, output, errors and asynchrony as
+ * gdn_forward; s_end is complete when the stream reaches the call's end. */
+gdn_status gdn_forward_state(gdn_plan_t plan, const gdn_inputs *in, const float *s0, void *y, float *s_end,
+                             void *workspace, gdn_stream_t stream);
+
 /* gdn_forward with per-kernel timing: events[i] (a cudaEvent_t the caller
  * created) is recorded on `stream` just before the i-th kernel launch and
  * events[L] after the last one, L = gdn_launches_per_forward(plan);

@@ -28,3 +28,9 @@ def split_stream(inp: dict, t1: int, hist: int = 3):
         second[n] = second[n].copy()
         second[n][:, :hist] = -200.0
     return first, second
+
+
+def random_state(B: int, H: int, d: int, seed: int, scale: float = 0.5) -> np.ndarray:
+    """A seeded [B, H, d, d] fp32 state S (S[i][j]: i over d_v, j over d_k)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    return (np.float32(scale) * rng.standard_normal((B, H, d, d), dtype=np.float32)).astype(np.float32)
