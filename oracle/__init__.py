@@ -161,6 +161,30 @@ def forward_with_state(inp: dict, s0=None, l2_eps=DEFAULT_L2_EPS, norm_eps=DEFAU
     return output(o, inp["z"], inp["norm_w"], norm_eps), s_end
 
 
+_T_AXIS = ("q", "k", "v", "z", "g", "b")
+
+
+def _flip_time(inp: dict) -> dict:
+    out = dict(inp)
+    for n in _T_AXIS:
+        out[n] = np.ascontiguousarray(inp[n][:, ::-1])
+    return out
+
+
+def reverse(inp: dict, s0=None, l2_eps=DEFAULT_L2_EPS, norm_eps=DEFAULT_NORM_EPS, nthreads=None):
+    """The anti-causal (reverse-direction) scan: steps 1-5 over the token order
+    T-1, ..., 0, i.e. the forward of the time-reversed sequence, with its
+    outputs put back in the original order.  Its short convolutions see the
+    current and the three FOLLOWING tokens (zero past T-1), and the state runs
+    from token T-1 down to token 0.  The pages leave the scan direction open
+    (the LinGen page's linear branch is a bidirectional Mamba2 block); this is
+    the one direction-reversal reading: the same operator on the reversed
+    sequence.  Returns (y, state after token 0); s0 is the state before token
+    T-1."""
+    y, s_end = forward_with_state(_flip_time(inp), s0=s0, l2_eps=l2_eps, norm_eps=norm_eps, nthreads=nthreads)
+    return np.ascontiguousarray(y[:, ::-1]), s_end
+
+
 class _swapped_library:
     """Context manager used by the oracle's own mutation tests: temporarily
     route every call above to another build of gdn_oracle.c (a copy with a

@@ -355,3 +355,42 @@ def test_streaming_in_two_pieces_equals_one_pass():
     # without the carried state the second piece differs
     y2z, _ = oracle.forward_with_state(p2)
     assert np.abs(y2z[:, 3:] - y[:, 170:]).max() > 1e-3
+
+
+# ------------------------------------------------ reverse-direction scan
+def test_reverse_scan_is_anti_causal():
+    # outputs at t > t0 never see token t0; the output at t0 does
+    inp = gdn_inputs.make_inputs(1, 90, 2, 16, "f32", -1.0, seed=71)
+    y, _ = oracle.reverse(inp)
+    t0 = 40
+    p = {n: (a.copy() if isinstance(a, np.ndarray) else a) for n, a in inp.items()}
+    p["k"][:, t0] += 0.5
+    p["g"][:, t0] -= 2.0
+    y2, _ = oracle.reverse(p)
+    np.testing.assert_array_equal(y2[:, t0 + 1:], y[:, t0 + 1:])
+    assert np.abs(y2[:, t0] - y[:, t0]).max() > 1e-6
+
+
+def test_reverse_scan_last_token_is_a_one_token_forward():
+    # the last token is the first of the reversed sequence: zero conv history and zero state,
+    # so its output is the forward of that token alone
+    from state_util import slice_tokens
+    inp = gdn_inputs.make_inputs(1, 50, 3, 16, "f32", 0.0, seed=72)
+    y, _ = oracle.reverse(inp)
+    one = oracle.forward(slice_tokens(inp, 49, 50))
+    np.testing.assert_allclose(y[:, 49], one[:, 0], rtol=1e-13, atol=1e-15)
+    # and the first token's output differs from the causal forward's (the direction matters)
+    assert np.abs(y[:, 0] - oracle.forward(inp)[:, 0]).max() > 1e-3
+
+
+def test_reverse_scan_conv_looks_ahead():
+    # with the decay at full strength for every token after the first (alpha ~ 0: the state keeps
+    # only the current token), token t's output depends on tokens t..t+3 only, through the conv
+    inp = gdn_inputs.make_inputs(1, 40, 1, 16, "f32", 0.0, seed=73)
+    inp["g"][:] = 60.0
+    inp["A_log"][:] = np.log(16.0)
+    y, _ = oracle.reverse(inp)
+    from state_util import slice_tokens
+    for t in (5, 20, 36):
+        window = oracle.reverse(slice_tokens(inp, t, min(t + 4, 40)))[0]
+        np.testing.assert_allclose(y[:, t], window[:, 0], rtol=1e-9, atol=1e-12)
