@@ -5,9 +5,14 @@ tolerances of the method's parity bar.
 Tolerances (fixed here, used by every parity test):
   * fp32 inputs:              rel-L2 <= 1e-5
   * bf16 inputs, fp32 output: rel-L2 <= 2e-3 and max |y - y_ref| <= 2e-2
-  * bf16 inputs, bf16 output: rel-L2 <= 2e-3 and |y - y_ref| <= 2e-2 + 1 bf16 ulp(|y_ref|)
-    elementwise (the output rounding alone is half an ulp, which exceeds 2e-2
-    for |y| >= 8).
+  * bf16 inputs, bf16 output: rel-L2 <= 2e-3 + rel-L2(bf16(y_ref), y_ref) and
+    |y - y_ref| <= 2e-2 + 1 bf16 ulp(|y_ref|) elementwise.  The 2e-3 bar is on
+    the computed value; rounding the output to bf16 adds an error that does
+    not depend on the implementation.  By the triangle inequality a value
+    within the bar, rounded to bf16, is within the bar plus the rounding error
+    of the exact result (about 1.7e-3 on large outputs, up to 3e-3 on a few
+    hundred elements).  Half an ulp also exceeds 2e-2 for |y| >= 8, hence the
+    elementwise ulp.
 rel-L2 = ||y - y_ref||_2 / ||y_ref||_2 over the whole tensor.
 """
 from __future__ import annotations
@@ -66,7 +71,12 @@ def check_parity(y, ref, in_dtype: str, out_dtype: str, what=""):
     if in_dtype == "f32":
         assert r <= REL_L2_F32, f"{what}: rel-L2 {r:.3e} > {REL_L2_F32}"
         return r, float(err.max())
-    assert r <= REL_L2_BF16, f"{what}: rel-L2 {r:.3e} > {REL_L2_BF16}"
+    bar = REL_L2_BF16
+    if out_dtype == "bf16":
+        import gdn_inputs
+        rounded = gdn_inputs.bf16_bits_to_f32(gdn_inputs.f32_to_bf16_bits(ref.astype(np.float32)))
+        bar += rel_l2(rounded.astype(np.float64), ref)
+    assert r <= bar, f"{what}: rel-L2 {r:.3e} > {bar:.3e}"
     if out_dtype == "bf16":
         bound = MAX_ABS_BF16 + bf16_ulp(ref)
         bad = err > bound
