@@ -247,6 +247,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-state", action="store_true", help="skip the carried-state timing")
+    ap.add_argument("--no-reverse", action="store_true", help="skip the reverse-scan timing")
     ap.add_argument("--load-seconds", type=float, default=1.5)
     args = ap.parse_args()
     w = gdn_inputs.by_name(args.workload)
@@ -369,6 +370,30 @@ def main():
         state_io = {"ms_per_step": st_ms, "value": job_throughput(world, w.B * w.T, st_ms), "unit": UNIT,
                     "state_bytes_per_step": 2 * w.B * w.H * w.d * w.d * 4, "steps": n_st}
 
+    # the reverse (anti-causal) scan of the same workload, its own plan and workspace
+    reverse = None
+    if not args.no_reverse:
+        plan_r = gdn.Plan(w.B, w.T, w.H, w.d, in_code, out_code, flags=gdn.FLAG_REVERSE)
+        ws_r = torch.empty(plan_r.workspace_bytes, dtype=torch.uint8, device=dev)
+        n_r = max(3, min(args.steps, 10))
+        for _ in range(2):
+            plan_r.forward_raw(ptrs, y.data_ptr(), ws_r.data_ptr(), s)
+        ev_r = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_r)]
+        torch.cuda.synchronize()
+        for k in range(n_r):
+            flush.zero_()
+            ev_r[k][0].record(stream)
+            plan_r.forward_raw(ptrs, y.data_ptr(), ws_r.data_ptr(), s)
+            ev_r[k][1].record(stream)
+        torch.cuda.synchronize()
+        st = plan_r.device_status(ws_r.data_ptr(), s)
+        if st != gdn.OK:
+            raise SystemExit(f"device status after the reverse scan: {gdn.status_string(st)}")
+        r_ms = ranks_max(sum(a.elapsed_time(b) for a, b in ev_r), world, dist, dev) / n_r
+        reverse = {"ms_per_step": r_ms, "value": job_throughput(world, w.B * w.T, r_ms), "unit": UNIT,
+                   "steps": n_r}
+        del ws_r
+
     # end to end through the public host-buffer entry point
     e2e = None
     if not args.no_e2e:
@@ -442,6 +467,7 @@ def main():
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "roofline": roof, "path_roofline": path_roof, "kernels_ms": kern_ms,
             "segments": plan.segments, "cpu_baseline": cpu, "e2e": e2e, "state_io": state_io,
+            "reverse": reverse,
             "clocks": clocks, "gpu_launches": L * args.steps,
             "gpu": torch.cuda.get_device_name(dev)}
     print(json.dumps(line), flush=True)

@@ -29,6 +29,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE_CHECK, E
 DTYPE_BF16, DTYPE_F32, DTYPE_F16 = 0, 1, 2
 FLAG_DEBUG_CHECKS = 0x1
 FLAG_FORCE_SIMT = 0x2
+FLAG_REVERSE = 0x4
 FLAG_TEST_WAIT_TIMEOUT = 0x100
 
 
@@ -201,17 +202,22 @@ def tensor_ptrs(tensors: dict) -> dict:
 
 def forward(q, k, v, z, g, b, conv_q, conv_k, conv_v, A_log, dt_bias, norm_w, out_dtype=None,
             l2_eps=1e-6, norm_eps=1e-6, plan: Plan | None = None, workspace=None, y=None, stream=None,
-            s0=None, return_state=False):
+            s0=None, return_state=False, reverse=False):
     """GDN forward on CUDA tensors (q, k, v, z [B,T,H,d]; g, b [B,T,H] fp32; conv_* [H*d,4];
     A_log, dt_bias [H]; norm_w [d]).  Returns y [B,T,H,d].  With s0 (a [B,H,d,d] fp32 state S[i][j],
     i over d_v, j over d_k) the recurrence starts from it; with return_state=True the call returns
-    (y, s_end), s_end the [B,H,d,d] fp32 state after the last token."""
+    (y, s_end), s_end the [B,H,d,d] fp32 state after the last token.  reverse=True runs the
+    anti-causal scan (token T-1 first; s0 / s_end are then the states before token T-1 and after
+    token 0); a given plan must carry FLAG_REVERSE exactly when reverse=True."""
     import torch
     B, T, H, d = q.shape
     in_code = _torch_dtype_code(q.dtype)
     odt = q.dtype if out_dtype is None else out_dtype
     if plan is None:
-        plan = Plan(B, T, H, d, in_code, _torch_dtype_code(odt), l2_eps, norm_eps, q.stride(1))
+        plan = Plan(B, T, H, d, in_code, _torch_dtype_code(odt), l2_eps, norm_eps, q.stride(1),
+                    flags=FLAG_REVERSE if reverse else 0)
+    elif bool(plan.cfg.flags & FLAG_REVERSE) != bool(reverse):
+        raise ValueError("the plan's scan direction differs from reverse=")
     if workspace is None:
         workspace = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=q.device)
     if y is None:

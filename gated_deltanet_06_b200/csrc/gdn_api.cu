@@ -286,6 +286,8 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
     pp.q_scale = 1.0f / sqrtf(static_cast<float>(d));
     pp.status = status;
     pp.wait_limit_ns = kWaitLimitNs;
+    const int rev = (c.flags & GDN_FLAG_REVERSE) ? 1 : 0;
+    pp.rev = rev;
     if (plan->tensor) {
         CUtensorMap rq, rk, rv;
         if (!make_raw_map(&rq, in->q, c.B, c.T, c.H * d, plan->tok_stride, 64 + 3, 128) ||
@@ -318,6 +320,7 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
         cp.BH = c.B * c.H; cp.Tp = plan->Tp; cp.NB = plan->NB;
         cp.status = status;
         cp.wait_limit_ns = kWaitLimitNs;
+        cp.rev = rev;
         // Kernels after the first start with programmatic dependent launch (prologue overlapped with
         // the previous kernel's tail), except when per-kernel events are recorded between them.
         const bool pdl = events == nullptr;
@@ -336,6 +339,7 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
         sp.test_wait_timeout = (c.flags & GDN_FLAG_TEST_WAIT_TIMEOUT) ? 1 : 0;
         sp.s0 = s0;
         sp.s_end = s_end;
+        sp.rev = rev;
         if (plan->NS > 1) {
             if (!mark() || launch_transfer(sp, tmW, tmKt, tmU, s, pdl) != cudaSuccess) return GDN_ERR_CUDA;
             if (!mark() || launch_combine(sp, s, pdl) != cudaSuccess) return GDN_ERR_CUDA;
@@ -353,7 +357,7 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
         rp.vh = reinterpret_cast<const float *>(ws + plan->off_vh);
         rp.log_alpha = la; rp.beta = beta; rp.o = o;
         rp.B = c.B; rp.T = c.T; rp.H = c.H; rp.d = d; rp.Tp = plan->Tp;
-        rp.s0 = s0; rp.s_end = s_end;
+        rp.s0 = s0; rp.s_end = s_end; rp.rev = rev;
         if (!mark() || launch_recurrence(rp, s) != cudaSuccess) return GDN_ERR_CUDA;
     }
 

@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(256, 2)
         const int t = blk * kBlk + r;
         float la = 0.0f, be = 0.0f;
         if (t < p.T) {
-            const size_t gi = (static_cast<size_t>(bb) * p.T + t) * p.H + hh;
+            const size_t gi = (static_cast<size_t>(bb) * p.T + (p.rev ? p.T - 1 - t : t)) * p.H + hh;
             const float xg = p.g[gi] + p.dt_bias[hh];
             const float sp = xg > 20.0f ? xg : __logf(1.0f + __expf(xg));
             la = -__expf(p.A_log[hh]) * sp;

@@ -46,6 +46,7 @@ struct PrepParams {
     float l2_eps, q_scale;
     int *status;
     unsigned long long wait_limit_ns;
+    int rev;                       // reverse scan: internal token t is input token T-1-t
 };
 cudaError_t launch_prep(const PrepParams &p, InType in, bool out_f16, cudaStream_t s);
 // Tensor path (16-bit inputs, d = 128): raw tiles staged by TMA through the
@@ -65,6 +66,7 @@ struct ChunkParams {
     int BH, Tp, NB;
     int *status;
     unsigned long long wait_limit_ns;
+    int rev;                        // reverse scan: block row t holds the gates of input token T-1-t
 };
 cudaError_t launch_chunk(const ChunkParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
                          const CUtensorMap &tmQ, const CUtensorMap &tmW, const CUtensorMap &tmU,
@@ -89,6 +91,7 @@ struct ScanParams {
     int test_wait_timeout;
     const float *s0;         // [BH][128 (d_v)][128 (d_k)] state before token 0, or null (zero)
     float *s_end;            // [BH][128][128] state after token T-1, or null (not wanted)
+    int rev;                 // reverse scan: block row t is z / y token T-1-t
 };
 // pdl: launch with programmatic stream serialization (see launch_k).
 cudaError_t launch_transfer(const ScanParams &p, const CUtensorMap &tmW, const CUtensorMap &tmKt,
@@ -106,6 +109,7 @@ struct RecurParams {
     int B, T, H, d, Tp;
     const float *s0;  // [B*H][d][d] (S[i][j], i over d_v) before token 0, or null (zero)
     float *s_end;     // [B*H][d][d] after token T-1, or null
+    int rev;          // reverse scan: internal token t is written to o row T-1-t
 };
 cudaError_t launch_recurrence(const RecurParams &p, cudaStream_t s);
 

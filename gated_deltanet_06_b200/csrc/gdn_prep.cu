@@ -11,6 +11,9 @@
 // and every global access is a 16-byte vector.  Outputs are written head-major
 // [B][H][Tp][d] (Tp = T rounded up to 128, padded rows zero, beta = 0,
 // log alpha = 0) so that every 128-token block is one contiguous tile.
+// For the reverse (anti-causal) scan the internal order is the reversed one:
+// internal token t is input token T-1-t, so everything after this kernel
+// runs unchanged, and the conv's history is the following input tokens.
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 
@@ -105,7 +108,8 @@ __global__ void __launch_bounds__(256) gdn_prep_kernel(const PrepParams p) {
         for (int i = 0; i < RPT + 3; ++i) {
             const int t = t0 + rbeg - 3 + i;
             if (t >= 0 && t < p.T) {
-                In8<InT>::load(x + (static_cast<size_t>(b) * p.T + t) * p.tok_stride + static_cast<size_t>(h) * D + c0,
+                const int ti = p.rev ? p.T - 1 - t : t;  // input token
+                In8<InT>::load(x + (static_cast<size_t>(b) * p.T + ti) * p.tok_stride + static_cast<size_t>(h) * D + c0,
                                xin[i]);
             } else {
 #pragma unroll
@@ -146,7 +150,7 @@ __global__ void __launch_bounds__(256) gdn_prep_kernel(const PrepParams p) {
     float la = 0.0f, be = 0.0f;
     const int t = t0 + tid;
     if (tid < kBlk && t < p.T) {
-        const size_t gi = (static_cast<size_t>(b) * p.T + t) * p.H + h;
+        const size_t gi = (static_cast<size_t>(b) * p.T + (p.rev ? p.T - 1 - t : t)) * p.H + h;
         const float xg = p.g[gi] + p.dt_bias[h];
         la = -expf(p.A_log[h]) * softplus_f(xg);
         be = 1.0f / (1.0f + expf(-p.b[gi]));
@@ -179,7 +183,10 @@ __global__ void __launch_bounds__(256) gdn_prep_kernel(const PrepParams p) {
 // the current one out of shared memory.  The conv weights of a head are
 // staged once per change of head, which a contiguous range of tiles makes
 // rare.  About 107 KB of shared memory: two CTAs per SM.  On this path the
-// gates are evaluated by the chunk kernel, which needs them first.
+// gates are evaluated by the chunk kernel, which needs them first.  For the
+// reverse scan the box of internal tokens t0..t0+63 starts at input token
+// T-64-t0 (its 3 extra rows are the following tokens, zero past T-1) and is
+// read bottom-up: box row 66-k in place of row k.
 constexpr int kPrepTok = 64;
 constexpr int kRawRows = kPrepTok + 3;
 constexpr uint32_t kRawTile = kRawRows * 256;          // bytes of one {128 ch, 67 tok} box (256-byte rows)
@@ -222,7 +229,8 @@ __global__ void __launch_bounds__(256, 2)
             asm volatile(
                 "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
                     smem_u32(dst + w * kRawTile)),
-                "l"(maps[w]), "r"(smem_u32(&bar[n & 1])), "r"(h * D), "r"(part * kPrepTok - 3), "r"(b)
+                "l"(maps[w]), "r"(smem_u32(&bar[n & 1])), "r"(h * D),
+                "r"(p.rev ? p.T - kPrepTok - part * kPrepTok : part * kPrepTok - 3), "r"(b)
                 : "memory");
     };
     if (tid == 0 && first < last) issue(0, first);
@@ -231,6 +239,8 @@ __global__ void __launch_bounds__(256, 2)
     const int c0 = cg * 8;
     const int rbeg = rg * RPT;
     const uint32_t coff = cg * 16;
+    // box row of window row k (k = 0..66; k = r + 3 is internal token t0 + r)
+    const int rsign = p.rev ? -256 : 256, rzero = p.rev ? 66 * 256 : 0;
     int cur_h = -1;
     for (int L = first, n = 0; L < last; ++L, ++n) {
         if (tid == 0 && L + 1 < last) issue(n + 1, L + 1);  // stage (n+1)&1 was released at the end of tile n-1
@@ -265,10 +275,11 @@ __global__ void __launch_bounds__(256, 2)
             for (int c = 0; c < 8; ++c) wt[c] = sW[which * 128 + c * 16 + cg];
             float win[4][8];
 #pragma unroll
-            for (int i = 0; i < 3; ++i) In8<InT>::load(reinterpret_cast<const InT *>(tile + (rbeg + i) * 256), win[i]);
+            for (int i = 0; i < 3; ++i)
+                In8<InT>::load(reinterpret_cast<const InT *>(tile + rzero + (rbeg + i) * rsign), win[i]);
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
-                In8<InT>::load(reinterpret_cast<const InT *>(tile + (rbeg + r + 3) * 256), win[(r + 3) & 3]);
+                In8<InT>::load(reinterpret_cast<const InT *>(tile + rzero + (rbeg + r + 3) * rsign), win[(r + 3) & 3]);
                 float u[8];
                 float ss = 0.0f;
 #pragma unroll

@@ -496,10 +496,12 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
             const int i = c - c0;
             const int tA = c * kBlk + rA, tB = c * kBlk + rB;
             const bool liveA = tA < p.T, liveB = tB < p.T;
-            const size_t zA = (static_cast<size_t>(b) * p.T + (liveA ? tA : 0)) * p.tok_stride + static_cast<size_t>(h) * kD;
-            const size_t zB = (static_cast<size_t>(b) * p.T + (liveB ? tB : 0)) * p.tok_stride + static_cast<size_t>(h) * kD;
-            const size_t yA = ((static_cast<size_t>(b) * p.T + (liveA ? tA : 0)) * p.H + h) * kD;
-            const size_t yB = ((static_cast<size_t>(b) * p.T + (liveB ? tB : 0)) * p.H + h) * kD;
+            // input / output token of each row (the reverse scan's rows run backwards)
+            const int xA = liveA ? (p.rev ? p.T - 1 - tA : tA) : 0, xB = liveB ? (p.rev ? p.T - 1 - tB : tB) : 0;
+            const size_t zA = (static_cast<size_t>(b) * p.T + xA) * p.tok_stride + static_cast<size_t>(h) * kD;
+            const size_t zB = (static_cast<size_t>(b) * p.T + xB) * p.tok_stride + static_cast<size_t>(h) * kD;
+            const size_t yA = ((static_cast<size_t>(b) * p.T + xA) * p.H + h) * kD;
+            const size_t yB = ((static_cast<size_t>(b) * p.T + xB) * p.H + h) * kD;
             const bool tre = (warp == 5 && lane == 0);
             if (tre) GDN_TRACE_AT(4096 + 64 * i + 32);
             // z: lane t0 of the quad fetches columns 8(4k + t0) .. +7 of its two rows
@@ -629,11 +631,13 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
                 tma_load_2d(sm + OFF_AQK, &tmAqk, &bars[FULL_KA], 0, rowbase + c * kBlk);
                 tma_load_2d(sm + OFF_AQK + 16384 + 64 * 128, &tmAqkH, &bars[FULL_KA], 64, rowbase + c * kBlk + 64);
             };
+            // first z row of block c in input order (clamped at 0; the box covers the block's rows)
+            auto zrow = [&](int c) { return p.rev ? max(p.T - (c + 1) * kBlk, 0) : c * kBlk; };
             if (ok) {
                 load_wq(c0);
                 load_u(c0);
                 load_ka(c0);
-                if (c0 * kBlk < p.T) tma_prefetch_3d(&tmZ, h * kD, c0 * kBlk, b);
+                if (c0 * kBlk < p.T) tma_prefetch_3d(&tmZ, h * kD, zrow(c0), b);
             }
             const uint32_t id_kmn = idesc_f16_f32(128, 128, false, true);
             const uint32_t id_mnmn = idesc_f16_f32(128, 128, true, true);
@@ -653,7 +657,7 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
                     }
                 }
                 if (c + 1 < c1 && (c + 1) * kBlk < p.T)  // z rows the epilogue of block c+1 reads
-                    tma_prefetch_3d(&tmZ, h * kD, (c + 1) * kBlk, b);
+                    tma_prefetch_3d(&tmZ, h * kD, zrow(c + 1), b);
                 GDN_TRACE_AT(4096 + 64 * i + 0);
                 ok = mbar_wait(&bars[FULL_WQ], ph, ab, p.status, lim);
                 GDN_TRACE_AT(4096 + 64 * i + 1);

@@ -53,7 +53,8 @@ __global__ void __launch_bounds__(D) gdn_recurrence_kernel(const RecurParams p) 
                 S[j] = fmaf(a, fmaf(-c1, kj, S[j]), c2 * kj);
                 o = fmaf(S[j], sq[tok][j], o);
             }
-            p.o[((static_cast<size_t>(b) * p.T + t0 + tok) * p.H + h) * D + i] = o;
+            const int to = p.rev ? p.T - 1 - (t0 + tok) : t0 + tok;  // input token order
+            p.o[((static_cast<size_t>(b) * p.T + to) * p.H + h) * D + i] = o;
         }
     }
     if (p.s_end) {

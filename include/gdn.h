@@ -77,6 +77,16 @@ typedef enum {
 /* Plan flags. */
 #define GDN_FLAG_DEBUG_CHECKS 0x1u       /* device-side index/alignment checks into the status word */
 #define GDN_FLAG_FORCE_SIMT 0x2u         /* use the fp32 CUDA-core path even where the tensor path applies */
+#define GDN_FLAG_REVERSE 0x4u            /* reverse (anti-causal) scan: the operation above on the
+                                            time-reversed sequence, outputs in the original order.
+                                            The state runs from token T-1 down to token 0 (S_{-1} of
+                                            gdn_forward_state is the state before token T-1, s_end the
+                                            state after token 0), and each conv4 sees the current and
+                                            the 3 FOLLOWING tokens, zero past T-1.  The pages leave
+                                            the scan direction open (the LinGen page's linear branch
+                                            is a bidirectional Mamba2 block); a bidirectional layer is
+                                            a forward and a reverse call on the same or separate
+                                            parameters, combined by the caller. */
 #define GDN_FLAG_TEST_WAIT_TIMEOUT 0x100u /* test hook: the scan kernel waits on a barrier nothing
                                             arrives on, gives up after ~50 ms and reports
                                             GDN_ERR_TIMEOUT in the status word */
@@ -198,7 +208,8 @@ int gdn_plan_uses_tensor_path(gdn_plan_t plan);
 int gdn_plan_segments(gdn_plan_t plan);
 
 /* Introspection for per-stage tests: writes up to n byte offsets, inside the
- * workspace, of the intermediates of the last forward, in this order:
+ * workspace, of the intermediates of the last forward (token rows in scan
+ * order: reversed for GDN_FLAG_REVERSE, except o), in this order:
  *   0 status word (int), 1 q^ (scaled by 1/sqrt(d_k)), 2 k^, 3 v^
  *     ([B][H][Tp][d], fp16 on the tensor path, fp32 otherwise; Tp = T rounded
  *     up to 128),
