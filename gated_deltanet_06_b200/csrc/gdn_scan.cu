@@ -428,10 +428,12 @@ constexpr uint32_t OFF_W = 0, OFF_QT = 32768, OFF_KT = 65536, OFF_AQK = 98304, O
 constexpr uint32_t OFF_S = 163840;  // S^T fp16 MN-major B operand (rows d_k, cols d_v)
 constexpr uint32_t OFF_D = 196608;  // Delta fp16 MN-major B operand (rows token, cols d_v)
 constexpr uint32_t OFF_BAR = 229376;
-constexpr int NBAR = 11;
+constexpr int NBAR = 12;
 constexpr uint32_t OFF_NW = OFF_BAR + NBAR * 8 + 16;  // norm weight, fp32 [128]
 constexpr uint32_t SMEM_BYTES = OFF_NW + 512 + 1024;
-enum { FULL_WQ = 0, FULL_U, FULL_KA, MMA_X, MMA_P, MMA_O, CONS_D, CONS_S, CONS_O0, CONS_O1, TEST };
+// One O-complete barrier per O buffer: with a single one, the producer could complete blocks i and
+// i + 1 before the output warps wait for block i, whose parity wait would then alias block i + 2.
+enum { FULL_WQ = 0, FULL_U, FULL_KA, MMA_X, MMA_P, MMA_O0, MMA_O1, CONS_D, CONS_S, CONS_O0, CONS_O1, TEST };
 constexpr int kScanThreads = 416;  // warps 0-3 state, warp 4 producer, warps 5-12 output step
 // X and P share columns (X is read out before P is written, P before the next X);
 // the fp32 state S^T lives in TMEM; O is double-buffered (256 and 384).
@@ -512,7 +514,7 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
                 za[k] = liveA ? *reinterpret_cast<const uint4 *>(z + zA + col) : make_uint4(0, 0, 0, 0);
                 zb[k] = liveB ? *reinterpret_cast<const uint4 *>(z + zB + col) : make_uint4(0, 0, 0, 0);
             }
-            if (!warp_wait(&bars[MMA_O], i & 1, ab, p.status, lim)) break;
+            if (!warp_wait(&bars[MMA_O0 + (i & 1)], (i >> 1) & 1, ab, p.status, lim)) break;
             if (tre) GDN_TRACE_AT(4096 + 64 * i + 33);
             tc_fence_after();
             const uint32_t tO = tbase + TM_O + (i & 1) * 128;
@@ -701,9 +703,9 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
                     umma_f16(tO, sdesc_sw128(sbase + OFF_AQK + aoff, 16, 1024),
                              sdesc_sw128(sbase + OFF_D + kk * 2048, 16384, 1024), id_kmn, 1);
                 }
-                umma_commit(&bars[MMA_O]);
+                umma_commit(&bars[MMA_O0 + (i & 1)]);
                 GDN_TRACE_AT(4096 + 64 * i + 8);
-                ok = mbar_wait(&bars[MMA_O], ph, ab, p.status, lim);
+                ok = mbar_wait(&bars[MMA_O0 + (i & 1)], (i >> 1) & 1, ab, p.status, lim);
                 GDN_TRACE_AT(4096 + 64 * i + 9);
                 if (!ok) break;
                 if (c + 1 < c1) load_ka(c + 1);
