@@ -161,6 +161,21 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def other_gpu_processes(device_index):
+    """Compute processes other than this one on the GPU (another tenant time-slicing it would
+    distort every timing), or None where NVML cannot tell."""
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        idx = int(vis.split(",")[device_index]) if vis else device_index
+        h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+        procs = pynvml.nvmlDeviceGetComputeRunningProcesses(h)
+        return sorted({p.pid for p in procs if p.pid != os.getpid()})
+    except Exception:
+        return None
+
+
 def oracle_rate(w, T_sample, threads):
     import oracle
     inp = gdn_inputs.workload_inputs(w, T=T_sample)
@@ -248,6 +263,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-state", action="store_true", help="skip the carried-state timing")
     ap.add_argument("--no-reverse", action="store_true", help="skip the reverse-scan timing")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward timing")
     ap.add_argument("--load-seconds", type=float, default=1.5)
     args = ap.parse_args()
     w = gdn_inputs.by_name(args.workload)
@@ -302,6 +318,7 @@ def main():
         plan.forward_raw(ptrs, y.data_ptr(), ws.data_ptr(), s)
     torch.cuda.synchronize()
     # untimed load phase so that the clock samples see the GPU busy with this work
+    others_before = other_gpu_processes(local)
     sampler = ClockSampler(local)
     sampler.start()
     t_end = time.perf_counter() + args.load_seconds
@@ -325,10 +342,20 @@ def main():
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
+    others_after = other_gpu_processes(local)
     st = plan.device_status(ws.data_ptr(), s)
     if st != gdn.OK:
         raise SystemExit(f"device status after timing: {gdn.status_string(st)}")
     step_ms = [a.elapsed_time(b) for a, b in ev_step]
+    # each forward clears the device status word, so the check above sees only the last step:
+    # repeat the steps untimed, reading the status after every one (a bounded device wait that ran
+    # out in any of them would show here)
+    for _ in range(args.steps):
+        flush.zero_()
+        plan.forward_raw(ptrs, y.data_ptr(), ws.data_ptr(), s)
+        st = plan.device_status(ws.data_ptr(), s)
+        if st != gdn.OK:
+            raise SystemExit(f"device status in the per-step check: {gdn.status_string(st)}")
 
     # per-kernel breakdown (not part of the timed steps): the library records an event before each
     # launch and after the last one (gdn_forward_timed), which also serialises the launches
@@ -393,6 +420,36 @@ def main():
         reverse = {"ms_per_step": r_ms, "value": job_throughput(world, w.B * w.T, r_ms), "unit": UNIT,
                    "steps": n_r}
         del ws_r
+
+    # the backward (gradient of sum(y * dy) w.r.t. every input and parameter) of the same workload
+    bwd = None
+    if not args.no_backward:
+        ws_b = torch.empty(plan.backward_workspace_bytes, dtype=torch.uint8, device=dev)
+        dy = torch.randn((w.B, w.T, w.H, w.d), device=dev).to(out_t)
+        f32 = dict(dtype=torch.float32, device=dev)
+        gr = {n: torch.empty((w.B, w.T, w.H, w.d), **f32) for n in ("dq", "dk", "dv", "dz")}
+        gr.update(dg=torch.empty((w.B, w.T, w.H), **f32), db=torch.empty((w.B, w.T, w.H), **f32),
+                  dA_log=torch.empty(w.H, **f32), ddt_bias=torch.empty(w.H, **f32), dnorm_w=torch.empty(w.d, **f32))
+        for n in ("dconv_q", "dconv_k", "dconv_v"):
+            gr[n] = torch.empty((w.H * w.d, 4), **f32)
+        gp = {n: gr[n].data_ptr() for n in gdn.GRAD_NAMES}
+        n_b = 3
+        plan.backward_raw(ptrs, dy.data_ptr(), gp, ws_b.data_ptr(), s)
+        ev_b = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_b)]
+        torch.cuda.synchronize()
+        for k in range(n_b):
+            flush.zero_()
+            ev_b[k][0].record(stream)
+            plan.backward_raw(ptrs, dy.data_ptr(), gp, ws_b.data_ptr(), s)
+            ev_b[k][1].record(stream)
+        torch.cuda.synchronize()
+        st = plan.device_status(ws_b.data_ptr(), s)
+        if st != gdn.OK:
+            raise SystemExit(f"device status after the backward: {gdn.status_string(st)}")
+        b_ms = ranks_max(sum(a.elapsed_time(b) for a, b in ev_b), world, dist, dev) / n_b
+        bwd = {"ms_per_step": b_ms, "value": job_throughput(world, w.B * w.T, b_ms), "unit": UNIT,
+               "steps": n_b, "launches_per_step": plan.backward_launches, "precision": "fp32 CUDA cores"}
+        del ws_b, gr, dy
 
     # end to end through the public host-buffer entry point
     e2e = None
@@ -467,8 +524,11 @@ def main():
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "roofline": roof, "path_roofline": path_roof, "kernels_ms": kern_ms,
             "segments": plan.segments, "cpu_baseline": cpu, "e2e": e2e, "state_io": state_io,
-            "reverse": reverse,
+            "reverse": reverse, "backward": bwd,
             "clocks": clocks, "gpu_launches": L * args.steps,
+            "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms), "max": max(step_ms)},
+            "other_gpu_processes": None if others_before is None or others_after is None
+            else sorted(set(others_before) | set(others_after)),
             "gpu": torch.cuda.get_device_name(dev)}
     print(json.dumps(line), flush=True)
     if world > 1:

@@ -45,6 +45,13 @@ class Inputs(ctypes.Structure):
                                                  "A_log", "dt_bias", "norm_w")]
 
 
+GRAD_NAMES = ("dq", "dk", "dv", "dz", "dg", "db", "dconv_q", "dconv_k", "dconv_v", "dA_log", "ddt_bias", "dnorm_w")
+
+
+class Grads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in GRAD_NAMES]
+
+
 _vp = ctypes.c_void_p
 _lib.gdn_plan.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(_vp), ctypes.POINTER(ctypes.c_size_t)]
 _lib.gdn_plan.restype = ctypes.c_int
@@ -52,6 +59,12 @@ _lib.gdn_forward.argtypes = [_vp, ctypes.POINTER(Inputs), _vp, _vp, _vp]
 _lib.gdn_forward.restype = ctypes.c_int
 _lib.gdn_forward_state.argtypes = [_vp, ctypes.POINTER(Inputs), _vp, _vp, _vp, _vp, _vp]
 _lib.gdn_forward_state.restype = ctypes.c_int
+_lib.gdn_backward.argtypes = [_vp, ctypes.POINTER(Inputs), _vp, ctypes.POINTER(Grads), _vp, _vp]
+_lib.gdn_backward.restype = ctypes.c_int
+_lib.gdn_backward_workspace_bytes.argtypes = [_vp]
+_lib.gdn_backward_workspace_bytes.restype = ctypes.c_size_t
+_lib.gdn_backward_launches.argtypes = [_vp]
+_lib.gdn_backward_launches.restype = ctypes.c_int
 _lib.gdn_forward_timed.argtypes = [_vp, ctypes.POINTER(Inputs), _vp, _vp, _vp, ctypes.POINTER(_vp), ctypes.c_int]
 _lib.gdn_forward_timed.restype = ctypes.c_int
 _lib.gdn_forward_host.argtypes = [_vp, ctypes.POINTER(Inputs), _vp, _vp, _vp, _vp]
@@ -145,6 +158,20 @@ class Plan:
         _check(_lib.gdn_forward_state(self._h, ctypes.byref(ins), s0 or None, y, s_end or None, workspace, stream),
                "gdn_forward_state")
 
+    @property
+    def backward_workspace_bytes(self) -> int:
+        return _lib.gdn_backward_workspace_bytes(self._h)
+
+    @property
+    def backward_launches(self) -> int:
+        return _lib.gdn_backward_launches(self._h)
+
+    def backward_raw(self, ptrs: dict, dy: int, grads: dict, workspace: int, stream: int) -> None:
+        """gdn_backward with raw device addresses: grads maps GRAD_NAMES to fp32 buffers."""
+        ins = Inputs(*[ptrs[n] for n, _ in Inputs._fields_])
+        gr = Grads(*[grads[n] for n in GRAD_NAMES])
+        _check(_lib.gdn_backward(self._h, ctypes.byref(ins), dy, ctypes.byref(gr), workspace, stream), "gdn_backward")
+
     def forward_timed_raw(self, ptrs: dict, y: int, workspace: int, stream: int, events: list) -> None:
         """gdn_forward_timed: `events` are cudaEvent_t handles (ints), launches + 1 of them."""
         ins = Inputs(*[ptrs[n] for n, _ in Inputs._fields_])
@@ -234,3 +261,29 @@ def forward(q, k, v, z, g, b, conv_q, conv_k, conv_v, A_log, dt_bias, norm_w, ou
     plan.forward_state_raw(tensor_ptrs(t), 0 if s0 is None else s0.data_ptr(), y.data_ptr(),
                            0 if s_end is None else s_end.data_ptr(), workspace.data_ptr(), s)
     return (y, s_end) if return_state else y
+
+
+def backward(q, k, v, z, g, b, conv_q, conv_k, conv_v, A_log, dt_bias, norm_w, dy, l2_eps=1e-6, norm_eps=1e-6,
+             plan: Plan | None = None, workspace=None, stream=None) -> dict:
+    """Gradients of sum(y * dy) for the forward of the same arguments (dy [B,T,H,d], the output's
+    dtype).  Returns a dict of fp32 CUDA tensors keyed by GRAD_NAMES (dq .. dnorm_w)."""
+    import torch
+    B, T, H, d = q.shape
+    if plan is None:
+        plan = Plan(B, T, H, d, _torch_dtype_code(q.dtype), _torch_dtype_code(dy.dtype), l2_eps, norm_eps,
+                    q.stride(1))
+    if workspace is None:
+        workspace = torch.empty(plan.backward_workspace_bytes, dtype=torch.uint8, device=q.device)
+    dev = q.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = {n: torch.empty((B, T, H, d), **f32) for n in ("dq", "dk", "dv", "dz")}
+    out.update(dg=torch.empty((B, T, H), **f32), db=torch.empty((B, T, H), **f32),
+               dA_log=torch.empty(H, **f32), ddt_bias=torch.empty(H, **f32), dnorm_w=torch.empty(d, **f32))
+    for n in ("dconv_q", "dconv_k", "dconv_v"):
+        out[n] = torch.empty((H * d, 4), **f32)
+    s = torch.cuda.current_stream(dev).cuda_stream if stream is None else stream
+    t = dict(q=q, k=k, v=v, z=z, g=g, b=b, conv_q=conv_q, conv_k=conv_k, conv_v=conv_v, A_log=A_log,
+             dt_bias=dt_bias, norm_w=norm_w)
+    plan.backward_raw(tensor_ptrs(t), dy.contiguous().data_ptr(), {n: out[n].data_ptr() for n in GRAD_NAMES},
+                      workspace.data_ptr(), s)
+    return out

@@ -24,6 +24,9 @@ struct gdn_plan_s {
     // workspace layout
     size_t off_status, off_qh, off_kh, off_vh, off_G, off_beta, off_la;
     size_t off_W, off_U, off_Qt, off_Kt, off_Aqk, off_Zloc, off_Sstart, off_o, ws_bytes;
+    // backward workspace layout (gdn_backward)
+    size_t b_status, b_qh, b_kh, b_vh, b_G, b_beta, b_la, b_o, b_ckpt, b_dO, b_dvh, b_dqp, b_dkp, b_dap, b_dbp,
+        b_dnw, b_dconv, b_dA, b_ddt, bws_bytes;
     // staging layout (gdn_forward_host)
     size_t st_q, st_k, st_v, st_z, st_g, st_b, st_cq, st_ck, st_cv, st_A, st_dt, st_nw, st_y, staging_bytes;
 };
@@ -182,6 +185,35 @@ gdn_status gdn_plan(const gdn_config *cfg, gdn_plan_t *out, size_t *workspace_by
         p->off_o = off; off = align_up(off + static_cast<size_t>(c.B) * c.T * c.H * d * 4, A);
     }
     p->ws_bytes = off;
+
+    {  // backward: the forward recomputed in fp32, checkpoints, gradient intermediates and partial sums
+        const size_t act4 = nTok * d * 4, tok4 = nTok * 4;
+        const size_t G = static_cast<size_t>(d) / 8;
+        const size_t NC = (static_cast<size_t>(c.T) + 7) / 8;
+        const size_t ntile = static_cast<size_t>(Tp) / 64;
+        const size_t nout = static_cast<size_t>(bwd_out_blocks(static_cast<long long>(c.B) * c.T * c.H));
+        size_t o2 = 0;
+        p->b_status = o2; o2 = align_up(o2 + 256, A);
+        p->b_qh = o2; o2 = align_up(o2 + act4, A);
+        p->b_kh = o2; o2 = align_up(o2 + act4, A);
+        p->b_vh = o2; o2 = align_up(o2 + act4, A);
+        p->b_G = o2; o2 = align_up(o2 + tok4, A);
+        p->b_beta = o2; o2 = align_up(o2 + tok4, A);
+        p->b_la = o2; o2 = align_up(o2 + tok4, A);
+        p->b_o = o2; o2 = align_up(o2 + static_cast<size_t>(c.B) * c.T * c.H * d * 4, A);
+        p->b_ckpt = o2; o2 = align_up(o2 + static_cast<size_t>(BH) * NC * d * d * 4, A);
+        p->b_dO = o2; o2 = align_up(o2 + act4, A);
+        p->b_dvh = o2; o2 = align_up(o2 + act4, A);
+        p->b_dqp = o2; o2 = align_up(o2 + G * act4, A);
+        p->b_dkp = o2; o2 = align_up(o2 + G * act4, A);
+        p->b_dap = o2; o2 = align_up(o2 + G * tok4, A);
+        p->b_dbp = o2; o2 = align_up(o2 + G * tok4, A);
+        p->b_dnw = o2; o2 = align_up(o2 + nout * d * 4, A);
+        p->b_dconv = o2; o2 = align_up(o2 + static_cast<size_t>(c.B) * ntile * 3 * c.H * d * 4 * 4, A);
+        p->b_dA = o2; o2 = align_up(o2 + static_cast<size_t>(BH) * ntile * 4, A);
+        p->b_ddt = o2; o2 = align_up(o2 + static_cast<size_t>(BH) * ntile * 4, A);
+        p->bws_bytes = o2;
+    }
 
     const size_t ntok_in = static_cast<size_t>(c.B) * c.T;
     const size_t a_in = ntok_in * c.H * d * p->in_esize;
@@ -427,6 +459,74 @@ gdn_status gdn_forward_host(gdn_plan_t plan, const gdn_inputs *in_host, void *y_
     if (cudaMemcpyAsync(y_host, st + plan->st_y, ntok * c.H * d * plan->out_esize, cudaMemcpyDeviceToHost, s) !=
         cudaSuccess)
         return GDN_ERR_CUDA;
+    return GDN_OK;
+}
+
+size_t gdn_backward_workspace_bytes(gdn_plan_t plan) { return plan ? plan->bws_bytes : 0; }
+
+int gdn_backward_launches(gdn_plan_t plan) { return plan ? 6 : 0; }  // prep + the five backward kernels
+
+gdn_status gdn_backward(gdn_plan_t plan, const gdn_inputs *in, const void *dy, const gdn_grads *gr, void *workspace,
+                        gdn_stream_t stream) {
+    if (!plan || !in || !dy || !gr || !workspace) return GDN_ERR_INVALID_ARG;
+    const gdn_config &c = plan->cfg;
+    if (c.flags & GDN_FLAG_REVERSE) return GDN_ERR_UNSUPPORTED;
+    const void *ptrs16[] = {in->q, in->k, in->v, in->z, dy, gr->dq, gr->dk, gr->dv, gr->dz};
+    for (const void *q : ptrs16)
+        if (!q || !aligned16(q)) return GDN_ERR_INVALID_ARG;
+    const void *ptrs4[] = {in->g, in->b, in->conv_q, in->conv_k, in->conv_v, in->A_log, in->dt_bias, in->norm_w,
+                           gr->dg, gr->db, gr->dconv_q, gr->dconv_k, gr->dconv_v, gr->dA_log, gr->ddt_bias,
+                           gr->dnorm_w};
+    for (const void *q : ptrs4)
+        if (!q || (reinterpret_cast<uintptr_t>(q) & 3u)) return GDN_ERR_INVALID_ARG;
+    const void *ptrsw[] = {in->conv_q, in->conv_k, in->conv_v};
+    for (const void *q : ptrsw)
+        if (!aligned16(q)) return GDN_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return GDN_ERR_INVALID_ARG;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != plan->device) return GDN_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const int d = c.d_k;
+    int *status = reinterpret_cast<int *>(ws + plan->b_status);
+    if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return GDN_ERR_CUDA;
+    auto F = [&](size_t off) { return reinterpret_cast<float *>(ws + off); };
+
+    PrepParams pp;
+    memset(&pp, 0, sizeof(pp));
+    pp.q = in->q; pp.k = in->k; pp.v = in->v;
+    pp.tok_stride = plan->tok_stride;
+    pp.g = in->g; pp.b = in->b;
+    pp.conv_q = in->conv_q; pp.conv_k = in->conv_k; pp.conv_v = in->conv_v;
+    pp.A_log = in->A_log; pp.dt_bias = in->dt_bias;
+    pp.qh = F(plan->b_qh); pp.kh = F(plan->b_kh); pp.vh = F(plan->b_vh);
+    pp.G = F(plan->b_G); pp.beta = F(plan->b_beta); pp.log_alpha = F(plan->b_la);
+    pp.B = c.B; pp.T = c.T; pp.H = c.H; pp.d = d; pp.Tp = plan->Tp;
+    pp.l2_eps = c.l2_eps;
+    pp.q_scale = 1.0f / sqrtf(static_cast<float>(d));
+    pp.status = status;
+    pp.wait_limit_ns = kWaitLimitNs;
+    pp.rev = 0;
+    if (launch_prep(pp, in_type(c.in_dtype), false, s) != cudaSuccess) return GDN_ERR_CUDA;
+
+    BwdParams bp;
+    bp.q = in->q; bp.k = in->k; bp.v = in->v; bp.z = in->z; bp.dy = dy;
+    bp.tok_stride = plan->tok_stride;
+    bp.g = in->g; bp.bg = in->b; bp.conv_q = in->conv_q; bp.conv_k = in->conv_k; bp.conv_v = in->conv_v;
+    bp.A_log = in->A_log; bp.dt_bias = in->dt_bias; bp.norm_w = in->norm_w;
+    bp.qh = F(plan->b_qh); bp.kh = F(plan->b_kh); bp.vh = F(plan->b_vh);
+    bp.log_alpha = F(plan->b_la); bp.beta = F(plan->b_beta);
+    bp.o = F(plan->b_o); bp.ckpt = F(plan->b_ckpt); bp.dO = F(plan->b_dO); bp.dvh = F(plan->b_dvh);
+    bp.dq_part = F(plan->b_dqp); bp.dk_part = F(plan->b_dkp); bp.da_part = F(plan->b_dap); bp.db_part = F(plan->b_dbp);
+    bp.dnw_part = F(plan->b_dnw); bp.dconv_part = F(plan->b_dconv); bp.dA_part = F(plan->b_dA);
+    bp.ddt_part = F(plan->b_ddt);
+    bp.dq = gr->dq; bp.dk = gr->dk; bp.dv = gr->dv; bp.dz = gr->dz; bp.dg = gr->dg; bp.db = gr->db;
+    bp.dconv_q = gr->dconv_q; bp.dconv_k = gr->dconv_k; bp.dconv_v = gr->dconv_v;
+    bp.dA_log = gr->dA_log; bp.ddt_bias = gr->ddt_bias; bp.dnorm_w = gr->dnorm_w;
+    bp.B = c.B; bp.T = c.T; bp.H = c.H; bp.d = d; bp.Tp = plan->Tp;
+    bp.l2_eps = c.l2_eps; bp.norm_eps = c.norm_eps; bp.q_scale = pp.q_scale;
+    int n = 0;
+    if (launch_backward(bp, in_type(c.in_dtype), in_type(c.out_dtype), s, &n) != cudaSuccess) return GDN_ERR_CUDA;
     return GDN_OK;
 }
 

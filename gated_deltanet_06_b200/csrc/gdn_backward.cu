@@ -1,0 +1,570 @@
+// gdn_backward.cu -- the gradient of the GDN forward (the gated delta rule of
+// reference [57] on the VMonarch page, with the LinMorph page's short
+// convolutions, normalizations, decay terms and update gates) with respect to
+// every input and parameter, in fp32 on CUDA cores.
+//
+// The recurrence, rearranged: u_t = S_{t-1} k^_t, delta_t = beta_t (v^_t -
+// alpha_t u_t), S_t = alpha_t S_{t-1} + delta_t k^_t^T, o_t = S_t q^_t.  Row i
+// of S (a d_v index) only ever meets row i of S, forwards and backwards: with
+// D_t = dL/dS_t,
+//   D_t += do_t q^_t^T;  ddelta = D_t k^_t;  du = -alpha beta ddelta;
+//   D_{t-1} = alpha D_t + du k^_t^T,
+// so the state and its gradient split into groups of R = 8 rows, one CTA per
+// (group, head).  What does couple the rows are the outputs
+//   dq^_t = S_t^T do_t,  dk^_t = D_t^T delta_t + S_{t-1}^T du,
+//   dalpha_t = <D_t, S_{t-1}> - beta u.ddelta,  dbeta_t = ddelta.(v^ - alpha u),
+// sums over rows that feed nothing back: each CTA writes its group's partial
+// sums, and the token kernel adds the groups.  Kernels, in order:
+//   prep (the forward's fp32 prep, recomputed) -> gdn_bwd_fwd_rows (o and a
+//   checkpoint of S every C = 8 tokens) -> gdn_bwd_out (RMSNorm and SiLU(z)
+//   gate backwards: do, dz, norm-weight partials) -> gdn_bwd_core (per chunk
+//   of C tokens, last to first: states recomputed from the checkpoint into
+//   shared memory, the gradient run backwards, the row sums taken from shared
+//   memory) -> gdn_bwd_tokens (group sums, L2-norm, SiLU and conv backwards,
+//   gates) -> gdn_bwd_params (sums over tokens of the parameter gradients).
+#include "gdn_common.cuh"
+#include "gdn_internal.h"
+
+namespace gdn {
+namespace {
+
+constexpr int kR = 8;     // rows of S per CTA
+constexpr int kC = 8;     // tokens per checkpoint chunk
+constexpr int kTile = 64; // tokens per CTA of the token kernel
+
+template <typename T>
+__device__ __forceinline__ float ldf(const T *p);
+template <>
+__device__ __forceinline__ float ldf<float>(const float *p) { return *p; }
+template <>
+__device__ __forceinline__ float ldf<__nv_bfloat16>(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+template <>
+__device__ __forceinline__ float ldf<__half>(const __half *p) { return __half2float(*p); }
+
+__device__ __forceinline__ float sigm(float x) { return 1.0f / (1.0f + expf(-x)); }
+// d SiLU(a) / da
+__device__ __forceinline__ float dsilu(float a) {
+    const float s = sigm(a);
+    return s * (1.0f + a * (1.0f - s));
+}
+// sum over the 16 lanes of a row (lanes 16k .. 16k+15)
+__device__ __forceinline__ float sum16(float x) {
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    return x;
+}
+
+// ------------------------------------------------------------ forward rows
+// One CTA per (group of kR rows, h, b), 128 threads: thread (r, cb) holds
+// columns cb*CW .. +CW-1 of row g*kR + r of S.  Writes o [B][T][H][D] and the
+// state before every chunk of kC tokens.
+template <int D>
+__global__ void __launch_bounds__(128) gdn_bwd_fwd_rows(const BwdParams p) {
+    constexpr int CW = D / 16;
+    __shared__ float sq[kC][D], sk[kC][D], sv[kC][kR], sa[kC], sb[kC];
+    const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const size_t bh = static_cast<size_t>(b) * p.H + h;
+    const int tid = threadIdx.x, r = tid >> 4, cb = tid & 15;
+    const int i = g * kR + r, j0 = cb * CW;
+    const int NC = (p.T + kC - 1) / kC;
+    float S[CW];
+#pragma unroll
+    for (int e = 0; e < CW; ++e) S[e] = 0.0f;
+    for (int c = 0; c < NC; ++c) {
+        const int c0 = c * kC, n = min(kC, p.T - c0);
+        __syncthreads();
+        for (int e = tid; e < kC * D; e += 128) {
+            const size_t src = (bh * p.Tp + c0 + e / D) * D + e % D;
+            sq[e / D][e % D] = p.qh[src];
+            sk[e / D][e % D] = p.kh[src];
+        }
+        if (tid < kC * kR) sv[tid / kR][tid % kR] = p.vh[(bh * p.Tp + c0 + tid / kR) * D + g * kR + tid % kR];
+        if (tid < kC) {
+            sa[tid] = expf(p.log_alpha[bh * p.Tp + c0 + tid]);
+            sb[tid] = p.beta[bh * p.Tp + c0 + tid];
+        }
+        __syncthreads();
+        float *ck = p.ckpt + ((bh * NC + c) * D + i) * D + j0;
+#pragma unroll
+        for (int e = 0; e < CW; ++e) ck[e] = S[e];
+        for (int tt = 0; tt < n; ++tt) {
+            float u = 0.0f;
+#pragma unroll
+            for (int e = 0; e < CW; ++e) u = fmaf(S[e], sk[tt][j0 + e], u);
+            u = sum16(u);
+            const float dl = sb[tt] * (sv[tt][r] - sa[tt] * u);
+            float ov = 0.0f;
+#pragma unroll
+            for (int e = 0; e < CW; ++e) {
+                S[e] = fmaf(sa[tt], S[e], dl * sk[tt][j0 + e]);
+                ov = fmaf(S[e], sq[tt][j0 + e], ov);
+            }
+            ov = sum16(ov);
+            if (cb == 0) p.o[((static_cast<size_t>(b) * p.T + c0 + tt) * p.H + h) * D + i] = ov;
+        }
+    }
+}
+
+// ------------------------------------------------------------ output step backwards
+// One warp per (b, t, h) row.  y = o rn w SiLU(z), rn = 1/sqrt(mean(o^2) + eps):
+//   gz = dy w SiLU(z);  do = rn gz - o rn^3 (o . gz) / D;  dz = dy o rn w SiLU'(z);
+//   dw += dy o rn SiLU(z)  (per-CTA partial sums, in a fixed order).
+template <typename ZT, typename YT, int D>
+__global__ void __launch_bounds__(256) gdn_bwd_out(const BwdParams p) {
+    constexpr int PER = D / 32;
+    __shared__ float sw[8][D];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const long long nrows = static_cast<long long>(p.B) * p.T * p.H;
+    float w[PER], dw[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+        w[e] = p.norm_w[lane * PER + e];
+        dw[e] = 0.0f;
+    }
+    const ZT *z = static_cast<const ZT *>(p.z);
+    const YT *dy = static_cast<const YT *>(p.dy);
+    for (long long row = blockIdx.x * 8ll + warp; row < nrows; row += gridDim.x * 8ll) {
+        const long long tok = row / p.H;  // b * T + t
+        const int hh = static_cast<int>(row % p.H);
+        const int bb = static_cast<int>(tok / p.T), t = static_cast<int>(tok % p.T);
+        float ov[PER], zv[PER], gv[PER], sz[PER];
+        float ss = 0.0f;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+            const int c = lane * PER + e;
+            ov[e] = p.o[row * D + c];
+            zv[e] = ldf<ZT>(z + tok * p.tok_stride + static_cast<long long>(hh) * D + c);
+            gv[e] = ldf<YT>(dy + row * D + c);
+            ss = fmaf(ov[e], ov[e], ss);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        const float rn = 1.0f / sqrtf(ss / D + p.norm_eps);
+        float og = 0.0f;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+            sz[e] = zv[e] * sigm(zv[e]);
+            og = fmaf(ov[e], gv[e] * w[e] * sz[e], og);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) og += __shfl_xor_sync(0xffffffffu, og, off);
+        const float k3 = rn * rn * rn * og / D;
+        const size_t bhr = static_cast<size_t>(bb) * p.H + hh;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+            const int c = lane * PER + e;
+            const float gz = gv[e] * w[e] * sz[e];
+            p.dO[(bhr * p.Tp + t) * D + c] = rn * gz - ov[e] * k3;
+            p.dz[row * D + c] = gv[e] * ov[e] * rn * w[e] * dsilu(zv[e]);
+            dw[e] = fmaf(gv[e] * ov[e] * rn, sz[e], dw[e]);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < PER; ++e) sw[warp][lane * PER + e] = dw[e];
+    __syncthreads();
+    for (int c = threadIdx.x; c < D; c += 256) {
+        float s = 0.0f;
+        for (int k = 0; k < 8; ++k) s += sw[k][c];
+        p.dnw_part[static_cast<size_t>(blockIdx.x) * D + c] = s;
+    }
+}
+
+// ------------------------------------------------------------ the recurrence backwards
+// Same CTA layout as gdn_bwd_fwd_rows.  Per chunk of kC tokens, last chunk
+// first: the states before each token (and after the last) are recomputed
+// from the checkpoint into sS, the gradient D runs backwards through the
+// chunk (kept in registers across chunks, each D_t also stored in sD), and
+// the row sums of the chunk are then taken from shared memory.
+template <int D>
+struct CoreSmem {
+    float S[kC + 1][kR][D];  // slot s: state before token c0 + s
+    float Dg[kC][kR][D];     // D_t after do_t q^_t^T is added
+    float q[kC][D], k[kC][D];
+    float v[kC][kR], dO[kC][kR], u[kC][kR], dl[kC][kR], ddl[kC][kR], du[kC][kR];
+    float a[kC], be[kC];
+    float part[kC][128];     // per-thread pieces of <D_t, S_{t-1}>
+};
+
+template <int D>
+__global__ void __launch_bounds__(128) gdn_bwd_core(const BwdParams p) {
+    constexpr int CW = D / 16;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    CoreSmem<D> &sm = *reinterpret_cast<CoreSmem<D> *>(smem_raw);
+    const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const size_t bh = static_cast<size_t>(b) * p.H + h;
+    const size_t BH = static_cast<size_t>(p.B) * p.H;
+    const int tid = threadIdx.x, r = tid >> 4, cb = tid & 15;
+    const int i = g * kR + r, j0 = cb * CW;
+    const int NC = (p.T + kC - 1) / kC;
+    float Dr[CW];
+#pragma unroll
+    for (int e = 0; e < CW; ++e) Dr[e] = 0.0f;
+    for (int c = NC - 1; c >= 0; --c) {
+        const int c0 = c * kC, n = min(kC, p.T - c0);
+        __syncthreads();  // the previous chunk's row sums are done with the buffers
+        for (int e = tid; e < kC * D; e += 128) {
+            const size_t src = (bh * p.Tp + c0 + e / D) * D + e % D;
+            sm.q[e / D][e % D] = p.qh[src];
+            sm.k[e / D][e % D] = p.kh[src];
+        }
+        if (tid < kC * kR) {
+            const size_t src = (bh * p.Tp + c0 + tid / kR) * D + g * kR + tid % kR;
+            sm.v[tid / kR][tid % kR] = p.vh[src];
+            sm.dO[tid / kR][tid % kR] = p.dO[src];
+        }
+        if (tid < kC) {
+            sm.a[tid] = expf(p.log_alpha[bh * p.Tp + c0 + tid]);
+            sm.be[tid] = p.beta[bh * p.Tp + c0 + tid];
+        }
+        float S[CW];
+        const float *ck = p.ckpt + ((bh * NC + c) * D + i) * D + j0;
+#pragma unroll
+        for (int e = 0; e < CW; ++e) S[e] = ck[e];
+        __syncthreads();
+        // states of the chunk
+        for (int tt = 0; tt < n; ++tt) {
+            float u = 0.0f;
+#pragma unroll
+            for (int e = 0; e < CW; ++e) {
+                sm.S[tt][r][j0 + e] = S[e];
+                u = fmaf(S[e], sm.k[tt][j0 + e], u);
+            }
+            u = sum16(u);
+            const float dl = sm.be[tt] * (sm.v[tt][r] - sm.a[tt] * u);
+#pragma unroll
+            for (int e = 0; e < CW; ++e) S[e] = fmaf(sm.a[tt], S[e], dl * sm.k[tt][j0 + e]);
+            if (cb == 0) {
+                sm.u[tt][r] = u;
+                sm.dl[tt][r] = dl;
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < CW; ++e) sm.S[n][r][j0 + e] = S[e];
+        // the gradient, backwards through the chunk
+        for (int tt = n - 1; tt >= 0; --tt) {
+            const float dov = sm.dO[tt][r];
+            float ddl = 0.0f, pr = 0.0f;
+#pragma unroll
+            for (int e = 0; e < CW; ++e) {
+                Dr[e] = fmaf(dov, sm.q[tt][j0 + e], Dr[e]);
+                sm.Dg[tt][r][j0 + e] = Dr[e];
+                ddl = fmaf(Dr[e], sm.k[tt][j0 + e], ddl);
+                pr = fmaf(Dr[e], sm.S[tt][r][j0 + e], pr);
+            }
+            ddl = sum16(ddl);
+            sm.part[tt][tid] = pr;
+            const float du = -sm.a[tt] * sm.be[tt] * ddl;
+            if (cb == 0) {
+                sm.ddl[tt][r] = ddl;
+                sm.du[tt][r] = du;
+                p.dvh[(bh * p.Tp + c0 + tt) * D + i] = sm.be[tt] * ddl;
+            }
+#pragma unroll
+            for (int e = 0; e < CW; ++e) Dr[e] = fmaf(sm.a[tt], Dr[e], du * sm.k[tt][j0 + e]);
+        }
+        __syncthreads();
+        // row sums of the chunk (this group's part)
+        for (int e = tid; e < n * D; e += 128) {
+            const int tt = e / D, j = e % D;
+            float dq = 0.0f, dk = 0.0f;
+#pragma unroll
+            for (int rr = 0; rr < kR; ++rr) {
+                dq = fmaf(sm.S[tt + 1][rr][j], sm.dO[tt][rr], dq);
+                dk = fmaf(sm.Dg[tt][rr][j], sm.dl[tt][rr], dk);
+                dk = fmaf(sm.S[tt][rr][j], sm.du[tt][rr], dk);
+            }
+            const size_t dst = ((g * BH + bh) * p.Tp + c0 + tt) * D + j;
+            p.dq_part[dst] = dq;
+            p.dk_part[dst] = dk;
+        }
+        const int warp = tid >> 5, lane = tid & 31;
+        for (int tt = warp; tt < n; tt += 4) {
+            float s = sm.part[tt][lane] + sm.part[tt][lane + 32] + sm.part[tt][lane + 64] + sm.part[tt][lane + 96];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+            if (lane == 0) {
+                float ud = 0.0f, db = 0.0f;
+                for (int rr = 0; rr < kR; ++rr) {
+                    ud = fmaf(sm.u[tt][rr], sm.ddl[tt][rr], ud);
+                    db = fmaf(sm.ddl[tt][rr], sm.v[tt][rr] - sm.a[tt] * sm.u[tt][rr], db);
+                }
+                const size_t dst = (g * BH + bh) * p.Tp + c0 + tt;
+                p.da_part[dst] = s - sm.be[tt] * ud;
+                p.db_part[dst] = db;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------ per-token backwards
+// One CTA per (64-token tile, h, b), 256 threads = CPR channel groups of 8 x
+// runs of tokens.  For q, k, v in turn: dq^ / dk^ = the sum of the groups'
+// parts (dv^ is whole); back through the L2 norm (q^ carries 1/sqrt(d_k)) and
+// SiLU into da for the tile's tokens and the 3 after it (conv recomputed from
+// the inputs); then dx[t] = sum_k w_k da[t+3-k] and the conv-weight sums of the
+// tile.  Threads 0..63 also take the gates of the tile's tokens.
+template <typename InT, int D>
+__global__ void __launch_bounds__(256) gdn_bwd_tokens(const BwdParams p) {
+    constexpr int CPR = D / 8, RG = 256 / CPR;
+    __shared__ float sda[kTile + 3][D];
+    __shared__ float sred[RG][32];  // conv-weight partials of one channel group, reduced over runs
+    __shared__ float sg[2][2];
+    const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const size_t bh = static_cast<size_t>(b) * p.H + h;
+    const size_t BH = static_cast<size_t>(p.B) * p.H;
+    const int t0 = tile * kTile;
+    const int tid = threadIdx.x, cg = tid % CPR, rg = tid / CPR, c0 = cg * 8;
+    const int G = D / kR;
+    const int ntile = p.Tp / kTile;
+
+    for (int which = 0; which < 3; ++which) {
+        const InT *x = static_cast<const InT *>(which == 0 ? p.q : (which == 1 ? p.k : p.v));
+        const float *w = which == 0 ? p.conv_q : (which == 1 ? p.conv_k : p.conv_v);
+        float *dx = which == 0 ? p.dq : (which == 1 ? p.dk : p.dv);
+        float wt[8][4];
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+            const float4 t4 = reinterpret_cast<const float4 *>(w)[static_cast<size_t>(h) * D + c0 + cc];
+            wt[cc][0] = t4.x; wt[cc][1] = t4.y; wt[cc][2] = t4.z; wt[cc][3] = t4.w;
+        }
+        auto xat = [&](int t, int cc) -> float {
+            return (t >= 0 && t < p.T)
+                       ? ldf<InT>(x + (static_cast<size_t>(b) * p.T + t) * p.tok_stride + static_cast<size_t>(h) * D + c0 + cc)
+                       : 0.0f;
+        };
+        __syncthreads();  // the previous tensor's reads of sda are done
+        // every thread runs the same number of steps (the row sums below shuffle across lanes)
+        for (int m = 0; m < (kTile + 3 + RG - 1) / RG; ++m) {
+            const int tt = rg + m * RG;
+            const bool inside = tt < kTile + 3;
+            const int t = t0 + tt;
+            float a[8], s[8], dh[8];
+            float ss = 0.0f;
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) {
+                float acc = 0.0f;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) acc = fmaf(wt[cc][k], xat(t - 3 + k, cc), acc);
+                a[cc] = acc;
+                s[cc] = acc * sigm(acc);
+                ss = fmaf(s[cc], s[cc], ss);
+                dh[cc] = 0.0f;
+            }
+            const bool live = inside && t < p.T;
+            if (live) {
+                if (which < 2) {
+                    const float *part = which == 0 ? p.dq_part : p.dk_part;
+                    for (int gg = 0; gg < G; ++gg) {
+                        const float *src = part + ((gg * BH + bh) * p.Tp + t) * D + c0;
+                        const float4 x0 = reinterpret_cast<const float4 *>(src)[0];
+                        const float4 x1 = reinterpret_cast<const float4 *>(src)[1];
+                        dh[0] += x0.x; dh[1] += x0.y; dh[2] += x0.z; dh[3] += x0.w;
+                        dh[4] += x1.x; dh[5] += x1.y; dh[6] += x1.z; dh[7] += x1.w;
+                    }
+                } else {
+                    const float *src = p.dvh + (bh * p.Tp + t) * D + c0;
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) dh[cc] = src[cc];
+                }
+            }
+            if (which < 2) {
+#pragma unroll
+                for (int off = CPR / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                const float nrm = sqrtf(ss + p.l2_eps);
+                const float sc = which == 0 ? p.q_scale : 1.0f;
+                float proj = 0.0f;
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) proj = fmaf(s[cc] / nrm, dh[cc], proj);
+#pragma unroll
+                for (int off = CPR / 2; off > 0; off >>= 1) proj += __shfl_xor_sync(0xffffffffu, proj, off);
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) dh[cc] = sc * (dh[cc] - (s[cc] / nrm) * proj) / nrm;
+            }
+            if (inside) {
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) sda[tt][c0 + cc] = live ? dh[cc] * dsilu(a[cc]) : 0.0f;
+            }
+        }
+        __syncthreads();
+        float dw[8][4];
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) dw[cc][k] = 0.0f;
+        for (int tt = rg; tt < kTile; tt += RG) {
+            const int t = t0 + tt;
+            if (t >= p.T) break;
+            float o8[8];
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) {
+                float acc = 0.0f;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    acc = fmaf(wt[cc][k], sda[tt + 3 - k][c0 + cc], acc);
+                    dw[cc][k] = fmaf(sda[tt][c0 + cc], xat(t - 3 + k, cc), dw[cc][k]);
+                }
+                o8[cc] = acc;
+            }
+            float *dst = dx + (static_cast<size_t>(b) * p.T + t) * p.H * D + static_cast<size_t>(h) * D + c0;
+            reinterpret_cast<float4 *>(dst)[0] = make_float4(o8[0], o8[1], o8[2], o8[3]);
+            reinterpret_cast<float4 *>(dst)[1] = make_float4(o8[4], o8[5], o8[6], o8[7]);
+        }
+        // conv-weight sums over the tile: reduce the RG runs, one channel group at a time
+        float *out = p.dconv_part + ((static_cast<size_t>(b) * ntile + tile) * 3 + which) * static_cast<size_t>(p.H) * D * 4;
+        for (int q = 0; q < CPR; ++q) {
+            __syncthreads();
+            if (cg == q) {
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) sred[rg][cc * 4 + k] = dw[cc][k];
+            }
+            __syncthreads();
+            if (tid < 32) {
+                float s = 0.0f;
+                for (int rr = 0; rr < RG; ++rr) s += sred[rr][tid];
+                out[(static_cast<size_t>(h) * D + q * 8) * 4 + tid] = s;
+            }
+        }
+    }
+
+    // gates: log alpha = -exp(A_log) softplus(g + dt_bias), beta = sigmoid(b)
+    float dla_la = 0.0f, dgv = 0.0f;
+    if (tid < kTile) {
+        const int t = t0 + tid;
+        if (t < p.T) {
+            float da = 0.0f, db = 0.0f;
+            for (int gg = 0; gg < G; ++gg) {
+                da += p.da_part[(gg * BH + bh) * p.Tp + t];
+                db += p.db_part[(gg * BH + bh) * p.Tp + t];
+            }
+            const size_t gi = (static_cast<size_t>(b) * p.T + t) * p.H + h;
+            const float xg = p.g[gi] + p.dt_bias[h];
+            const float eA = expf(p.A_log[h]);
+            const float la = -eA * softplus_f(xg);
+            const float dla = da * expf(la);
+            dgv = dla * (-eA * sigm(xg));
+            dla_la = dla * la;
+            const float be = sigm(p.bg[gi]);
+            p.dg[gi] = dgv;
+            p.db[gi] = db * be * (1.0f - be);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            dla_la += __shfl_xor_sync(0xffffffffu, dla_la, off);
+            dgv += __shfl_xor_sync(0xffffffffu, dgv, off);
+        }
+        if ((tid & 31) == 0) {
+            sg[tid >> 5][0] = dla_la;
+            sg[tid >> 5][1] = dgv;
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        const size_t k = (static_cast<size_t>(b) * p.H + h) * ntile + tile;
+        p.dA_part[k] = sg[0][0] + sg[1][0];
+        p.ddt_part[k] = sg[0][1] + sg[1][1];
+    }
+}
+
+// ------------------------------------------------------------ parameter sums
+// One thread per parameter gradient element, summing its partials in a fixed order.
+__global__ void __launch_bounds__(256) gdn_bwd_params(const BwdParams p, int D, int nout_part) {
+    const int HD4 = p.H * D * 4;
+    const int ntile = p.Tp / kTile;
+    const int total = 3 * HD4 + 2 * p.H + D;
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
+        if (e < 3 * HD4) {
+            const int which = e / HD4, k = e % HD4;
+            float s = 0.0f;
+            for (int bt = 0; bt < p.B * ntile; ++bt) s += p.dconv_part[(static_cast<size_t>(bt) * 3 + which) * HD4 + k];
+            (which == 0 ? p.dconv_q : (which == 1 ? p.dconv_k : p.dconv_v))[k] = s;
+        } else if (e < 3 * HD4 + 2 * p.H) {
+            const int k = e - 3 * HD4, h = k % p.H;
+            const float *part = k < p.H ? p.dA_part : p.ddt_part;
+            float s = 0.0f;
+            for (int b = 0; b < p.B; ++b)
+                for (int t = 0; t < ntile; ++t) s += part[(static_cast<size_t>(b) * p.H + h) * ntile + t];
+            (k < p.H ? p.dA_log : p.ddt_bias)[h] = s;
+        } else {
+            const int c = e - 3 * HD4 - 2 * p.H;
+            float s = 0.0f;
+            for (int q = 0; q < nout_part; ++q) s += p.dnw_part[static_cast<size_t>(q) * D + c];
+            p.dnorm_w[c] = s;
+        }
+    }
+}
+
+template <typename ZT, typename YT>
+cudaError_t launch_out_bwd(const BwdParams &p, int blocks, cudaStream_t s) {
+    if (p.d == 128) gdn_bwd_out<ZT, YT, 128><<<blocks, 256, 0, s>>>(p);
+    else gdn_bwd_out<ZT, YT, 64><<<blocks, 256, 0, s>>>(p);
+    return cudaGetLastError();
+}
+template <typename ZT>
+cudaError_t launch_out_bwd_z(const BwdParams &p, InType yt, int blocks, cudaStream_t s) {
+    if (yt == InType::BF16) return launch_out_bwd<ZT, __nv_bfloat16>(p, blocks, s);
+    if (yt == InType::F16) return launch_out_bwd<ZT, __half>(p, blocks, s);
+    return launch_out_bwd<ZT, float>(p, blocks, s);
+}
+
+template <int D>
+cudaError_t launch_core_bwd(const BwdParams &p, cudaStream_t s) {
+    static bool attr = false;
+    const int bytes = static_cast<int>(sizeof(CoreSmem<D>));
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(gdn_bwd_core<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    gdn_bwd_core<D><<<dim3(D / kR, p.H, p.B), 128, bytes, s>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename InT>
+cudaError_t launch_tokens_bwd(const BwdParams &p, cudaStream_t s) {
+    const dim3 grid(p.Tp / kTile, p.H, p.B);
+    if (p.d == 128) gdn_bwd_tokens<InT, 128><<<grid, 256, 0, s>>>(p);
+    else gdn_bwd_tokens<InT, 64><<<grid, 256, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int bwd_out_blocks(long long rows) {
+    long long blocks = (rows + 7) / 8;
+    return static_cast<int>(blocks < 1024 ? blocks : 1024);
+}
+
+cudaError_t launch_backward(const BwdParams &p, InType in, InType out, cudaStream_t s, int *launches) {
+    cudaError_t e;
+    int n = 0;
+    const dim3 grid_rows(p.d / kR, p.H, p.B);
+    if (p.d == 128) gdn_bwd_fwd_rows<128><<<grid_rows, 128, 0, s>>>(p);
+    else gdn_bwd_fwd_rows<64><<<grid_rows, 128, 0, s>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    ++n;
+    const int nb = bwd_out_blocks(static_cast<long long>(p.B) * p.T * p.H);
+    if (in == InType::BF16) e = launch_out_bwd_z<__nv_bfloat16>(p, out, nb, s);
+    else if (in == InType::F16) e = launch_out_bwd_z<__half>(p, out, nb, s);
+    else e = launch_out_bwd_z<float>(p, out, nb, s);
+    if (e != cudaSuccess) return e;
+    ++n;
+    e = p.d == 128 ? launch_core_bwd<128>(p, s) : launch_core_bwd<64>(p, s);
+    if (e != cudaSuccess) return e;
+    ++n;
+    if (in == InType::BF16) e = launch_tokens_bwd<__nv_bfloat16>(p, s);
+    else if (in == InType::F16) e = launch_tokens_bwd<__half>(p, s);
+    else e = launch_tokens_bwd<float>(p, s);
+    if (e != cudaSuccess) return e;
+    ++n;
+    gdn_bwd_params<<<64, 256, 0, s>>>(p, p.d, nb);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    ++n;
+    if (launches) *launches = n;
+    return cudaSuccess;
+}
+
+}  // namespace gdn
+
+GDN_TRACE_EXPORT(backward)

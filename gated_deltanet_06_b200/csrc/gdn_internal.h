@@ -125,6 +125,36 @@ struct OutParams {
 };
 cudaError_t launch_output(const OutParams &p, InType zt, InType yt, cudaStream_t s);
 
+// Backward (fp32, CUDA cores): the gradient of the forward with respect to
+// every input and parameter, for L = sum(y * dy).
+struct BwdParams {
+    const void *q, *k, *v, *z;      // inputs as in PrepParams / OutParams (token stride tok_stride)
+    const void *dy;                 // [B][T][H][d], out dtype, dense
+    long long tok_stride;
+    const float *g, *bg, *conv_q, *conv_k, *conv_v, *A_log, *dt_bias, *norm_w;
+    // the forward, recomputed (prep with fp32 outputs) and kept for the backward
+    const float *qh, *kh, *vh, *log_alpha, *beta;  // [BH][Tp][d] / [BH][Tp]
+    float *o;                       // [B][T][H][d]
+    float *ckpt;                    // [BH][ceil(T/8)][d][d]: the state before every 8th token
+    float *dO, *dvh;                // [BH][Tp][d]
+    float *dq_part, *dk_part;       // [d/8][BH][Tp][d]: per row-group sums
+    float *da_part, *db_part;       // [d/8][BH][Tp]
+    float *dnw_part;                // [bwd_out_blocks][d]
+    float *dconv_part;              // [B][Tp/64][3][H*d][4]
+    float *dA_part, *ddt_part;      // [B][H][Tp/64]
+    // results (fp32, dense)
+    float *dq, *dk, *dv, *dz;       // [B][T][H][d]
+    float *dg, *db;                 // [B][T][H]
+    float *dconv_q, *dconv_k, *dconv_v;  // [H*d][4]
+    float *dA_log, *ddt_bias;       // [H]
+    float *dnorm_w;                 // [d]
+    int B, T, H, d, Tp;
+    float l2_eps, norm_eps, q_scale;
+};
+int bwd_out_blocks(long long rows);
+// Enqueues the five backward kernels after the prep; *launches receives their count.
+cudaError_t launch_backward(const BwdParams &p, InType in, InType out, cudaStream_t s, int *launches);
+
 }  // namespace gdn
 
 struct gdn_plan_s;

@@ -190,6 +190,39 @@ gdn_status gdn_forward_host(gdn_plan_t plan, const gdn_inputs *in_host, void *y_
 #define GDN_NOALLOC_SCRATCH_BYTES (64ull << 20)
 gdn_status gdn_forward_noalloc(gdn_plan_t plan, const gdn_inputs *in, void *y, gdn_stream_t stream);
 
+/* Gradients of L = sum(y * dy) (fp32, dense, device, written not
+ * accumulated; caller-owned). */
+typedef struct {
+    float *dq, *dk, *dv, *dz;            /* [B][T][H][d], 16-byte aligned */
+    float *dg, *db;                      /* [B][T][H] */
+    float *dconv_q, *dconv_k, *dconv_v;  /* [H*d][4] */
+    float *dA_log, *ddt_bias;            /* [H] */
+    float *dnorm_w;                      /* [d_v] */
+} gdn_grads;
+
+/* Bytes of device workspace gdn_backward needs for this plan (256-byte
+ * aligned; a separate size from gdn_forward's): the forward recomputed in
+ * fp32, the state every 8 tokens, and per-group partial sums. */
+size_t gdn_backward_workspace_bytes(gdn_plan_t plan);
+
+/* Kernel launches one gdn_backward enqueues (6). */
+int gdn_backward_launches(gdn_plan_t plan);
+
+/* No counterpart written out in the pages, which train the GDN modules
+ * (the LinMorph page: distillation and joint recovery after the weight
+ * mapping) without giving the gradient: the gradient of the forward of
+ * gdn_forward with respect to every input and parameter, for the loss
+ * L = sum(y * dy).  dy is [B][T][H][d_v] of the plan's out_dtype, dense.
+ * Computed in fp32 on CUDA cores for every plan (bf16/f16 inputs are widened
+ * exactly): the forward is recomputed from the inputs, the recurrence's state
+ * is checkpointed every 8 tokens and rebuilt chunk by chunk while its
+ * gradient runs backwards.  Deterministic: every sum has a fixed order.
+ * Errors: INVALID_ARG (null or misaligned pointers, the workspace checks of
+ * gdn_forward), UNSUPPORTED for GDN_FLAG_REVERSE plans; asynchronous on
+ * `stream` like gdn_forward. */
+gdn_status gdn_backward(gdn_plan_t plan, const gdn_inputs *in, const void *dy, const gdn_grads *grads,
+                        void *workspace, gdn_stream_t stream);
+
 /* Synchronise `stream`, then read and clear the device status word in the
  * workspace.  Returns GDN_OK, GDN_ERR_TIMEOUT or GDN_ERR_DEVICE_CHECK (or
  * GDN_ERR_CUDA if the synchronisation itself failed). */
