@@ -447,8 +447,19 @@ def main():
         if st != gdn.OK:
             raise SystemExit(f"device status after the backward: {gdn.status_string(st)}")
         b_ms = ranks_max(sum(a.elapsed_time(b) for a, b in ev_b), world, dist, dev) / n_b
+        # per-kernel breakdown (events between the launches, one more run)
+        LB = plan.backward_launches
+        evk = [torch.cuda.Event(enable_timing=True) for _ in range(LB + 1)]
+        for e in evk:
+            e.record(stream)
+        torch.cuda.synchronize()
+        flush.zero_()
+        plan.backward_timed_raw(ptrs, dy.data_ptr(), gp, ws_b.data_ptr(), s, [e.cuda_event for e in evk])
+        torch.cuda.synchronize()
+        bnames = ("prep_f32", "fwd_rows", "out_bwd", "core_bwd", "tokens_bwd", "params")
         bwd = {"ms_per_step": b_ms, "value": job_throughput(world, w.B * w.T, b_ms), "unit": UNIT,
-               "steps": n_b, "launches_per_step": plan.backward_launches, "precision": "fp32 CUDA cores"}
+               "steps": n_b, "launches_per_step": LB, "precision": "fp32 CUDA cores",
+               "kernels_ms": {bnames[i]: evk[i].elapsed_time(evk[i + 1]) for i in range(LB)}}
         del ws_b, gr, dy
 
     # end to end through the public host-buffer entry point

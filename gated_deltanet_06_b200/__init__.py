@@ -61,6 +61,9 @@ _lib.gdn_forward_state.argtypes = [_vp, ctypes.POINTER(Inputs), _vp, _vp, _vp, _
 _lib.gdn_forward_state.restype = ctypes.c_int
 _lib.gdn_backward.argtypes = [_vp, ctypes.POINTER(Inputs), _vp, ctypes.POINTER(Grads), _vp, _vp]
 _lib.gdn_backward.restype = ctypes.c_int
+_lib.gdn_backward_timed.argtypes = [_vp, ctypes.POINTER(Inputs), _vp, ctypes.POINTER(Grads), _vp, _vp,
+                                    ctypes.POINTER(_vp), ctypes.c_int]
+_lib.gdn_backward_timed.restype = ctypes.c_int
 _lib.gdn_backward_workspace_bytes.argtypes = [_vp]
 _lib.gdn_backward_workspace_bytes.restype = ctypes.c_size_t
 _lib.gdn_backward_launches.argtypes = [_vp]
@@ -171,6 +174,14 @@ class Plan:
         ins = Inputs(*[ptrs[n] for n, _ in Inputs._fields_])
         gr = Grads(*[grads[n] for n in GRAD_NAMES])
         _check(_lib.gdn_backward(self._h, ctypes.byref(ins), dy, ctypes.byref(gr), workspace, stream), "gdn_backward")
+
+    def backward_timed_raw(self, ptrs: dict, dy: int, grads: dict, workspace: int, stream: int, events: list) -> None:
+        """gdn_backward_timed: `events` are cudaEvent_t handles (ints), backward_launches + 1 of them."""
+        ins = Inputs(*[ptrs[n] for n, _ in Inputs._fields_])
+        gr = Grads(*[grads[n] for n in GRAD_NAMES])
+        arr = (_vp * len(events))(*events)
+        _check(_lib.gdn_backward_timed(self._h, ctypes.byref(ins), dy, ctypes.byref(gr), workspace, stream, arr,
+                                       len(events)), "gdn_backward_timed")
 
     def forward_timed_raw(self, ptrs: dict, y: int, workspace: int, stream: int, events: list) -> None:
         """gdn_forward_timed: `events` are cudaEvent_t handles (ints), launches + 1 of them."""

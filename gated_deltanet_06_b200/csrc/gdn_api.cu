@@ -466,8 +466,8 @@ size_t gdn_backward_workspace_bytes(gdn_plan_t plan) { return plan ? plan->bws_b
 
 int gdn_backward_launches(gdn_plan_t plan) { return plan ? 6 : 0; }  // prep + the five backward kernels
 
-gdn_status gdn_backward(gdn_plan_t plan, const gdn_inputs *in, const void *dy, const gdn_grads *gr, void *workspace,
-                        gdn_stream_t stream) {
+static gdn_status backward_impl(gdn_plan_t plan, const gdn_inputs *in, const void *dy, const gdn_grads *gr,
+                                void *workspace, gdn_stream_t stream, void *const *events) {
     if (!plan || !in || !dy || !gr || !workspace) return GDN_ERR_INVALID_ARG;
     const gdn_config &c = plan->cfg;
     if (c.flags & GDN_FLAG_REVERSE) return GDN_ERR_UNSUPPORTED;
@@ -507,6 +507,7 @@ gdn_status gdn_backward(gdn_plan_t plan, const gdn_inputs *in, const void *dy, c
     pp.status = status;
     pp.wait_limit_ns = kWaitLimitNs;
     pp.rev = 0;
+    if (events && cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[0]), s) != cudaSuccess) return GDN_ERR_CUDA;
     if (launch_prep(pp, in_type(c.in_dtype), false, s) != cudaSuccess) return GDN_ERR_CUDA;
 
     BwdParams bp;
@@ -526,8 +527,23 @@ gdn_status gdn_backward(gdn_plan_t plan, const gdn_inputs *in, const void *dy, c
     bp.B = c.B; bp.T = c.T; bp.H = c.H; bp.d = d; bp.Tp = plan->Tp;
     bp.l2_eps = c.l2_eps; bp.norm_eps = c.norm_eps; bp.q_scale = pp.q_scale;
     int n = 0;
-    if (launch_backward(bp, in_type(c.in_dtype), in_type(c.out_dtype), s, &n) != cudaSuccess) return GDN_ERR_CUDA;
+    if (launch_backward(bp, in_type(c.in_dtype), in_type(c.out_dtype), s, &n, events ? events + 1 : nullptr) !=
+        cudaSuccess)
+        return GDN_ERR_CUDA;
     return GDN_OK;
+}
+
+gdn_status gdn_backward(gdn_plan_t plan, const gdn_inputs *in, const void *dy, const gdn_grads *gr, void *workspace,
+                        gdn_stream_t stream) {
+    return backward_impl(plan, in, dy, gr, workspace, stream, nullptr);
+}
+
+gdn_status gdn_backward_timed(gdn_plan_t plan, const gdn_inputs *in, const void *dy, const gdn_grads *gr,
+                              void *workspace, gdn_stream_t stream, void *const *events, int n_events) {
+    if (!plan || !events || n_events != gdn_backward_launches(plan) + 1) return GDN_ERR_INVALID_ARG;
+    for (int i = 0; i < n_events; ++i)
+        if (!events[i]) return GDN_ERR_INVALID_ARG;
+    return backward_impl(plan, in, dy, gr, workspace, stream, events);
 }
 
 gdn_status gdn_get_device_status(gdn_plan_t plan, void *workspace, gdn_stream_t stream) {

@@ -56,52 +56,80 @@ __device__ __forceinline__ float sum16(float x) {
 
 // ------------------------------------------------------------ forward rows
 // One CTA per (group of kR rows, h, b), 128 threads: thread (r, cb) holds
-// columns cb*CW .. +CW-1 of row g*kR + r of S.  Writes o [B][T][H][D] and the
-// state before every chunk of kC tokens.
+// columns cb, cb + 16, cb + 32, ... of row g*kR + r of S (so that the 16
+// lanes of a row touch 16 consecutive words of shared memory).  Writes o [B][T][H][D] and the
+// state before every chunk of kC tokens.  The next chunk's q^, k^, v^ rows and
+// gates are copied into the other shared buffer while this one is computed.
+template <int D>
+struct Stage {
+    float q[2][kC][D], k[2][kC][D], v[2][kC][kR], la[2][kC], be[2][kC];
+};
+
+// thread tid's share of the copies of chunk c into buffer buf (v: rows g*kR ..; dO likewise if given)
+template <int D>
+__device__ __forceinline__ void stage_chunk(Stage<D> &st, float (*dO)[kC][kR], const BwdParams &p, size_t bh,
+                                            int g, int c, int buf, int tid) {
+    const int c0 = c * kC;
+    for (int e = tid; e < kC * D / 4; e += 128) {
+        const int tt = e / (D / 4), j = (e % (D / 4)) * 4;
+        const size_t src = (bh * p.Tp + c0 + tt) * D + j;
+        cp_async16(&st.q[buf][tt][j], p.qh + src);
+        cp_async16(&st.k[buf][tt][j], p.kh + src);
+    }
+    if (tid < kC * kR) {
+        const size_t src = (bh * p.Tp + c0 + tid / kR) * D + g * kR + tid % kR;
+        cp_async4(&st.v[buf][tid / kR][tid % kR], p.vh + src);
+        if (dO) cp_async4(&dO[buf][tid / kR][tid % kR], p.dO + src);
+    }
+    if (tid < kC) {
+        cp_async4(&st.la[buf][tid], p.log_alpha + bh * p.Tp + c0 + tid);
+        cp_async4(&st.be[buf][tid], p.beta + bh * p.Tp + c0 + tid);
+    }
+    cp_async_commit();
+}
+
 template <int D>
 __global__ void __launch_bounds__(128) gdn_bwd_fwd_rows(const BwdParams p) {
     constexpr int CW = D / 16;
-    __shared__ float sq[kC][D], sk[kC][D], sv[kC][kR], sa[kC], sb[kC];
+    __shared__ __align__(16) Stage<D> st;
     const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const size_t bh = static_cast<size_t>(b) * p.H + h;
     const int tid = threadIdx.x, r = tid >> 4, cb = tid & 15;
-    const int i = g * kR + r, j0 = cb * CW;
+    const int i = g * kR + r;
     const int NC = (p.T + kC - 1) / kC;
     float S[CW];
 #pragma unroll
     for (int e = 0; e < CW; ++e) S[e] = 0.0f;
+    stage_chunk<D>(st, nullptr, p, bh, g, 0, 0, tid);
     for (int c = 0; c < NC; ++c) {
-        const int c0 = c * kC, n = min(kC, p.T - c0);
-        __syncthreads();
-        for (int e = tid; e < kC * D; e += 128) {
-            const size_t src = (bh * p.Tp + c0 + e / D) * D + e % D;
-            sq[e / D][e % D] = p.qh[src];
-            sk[e / D][e % D] = p.kh[src];
+        const int c0 = c * kC, n = min(kC, p.T - c0), buf = c & 1;
+        if (c + 1 < NC) {
+            stage_chunk<D>(st, nullptr, p, bh, g, c + 1, buf ^ 1, tid);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
         }
-        if (tid < kC * kR) sv[tid / kR][tid % kR] = p.vh[(bh * p.Tp + c0 + tid / kR) * D + g * kR + tid % kR];
-        if (tid < kC) {
-            sa[tid] = expf(p.log_alpha[bh * p.Tp + c0 + tid]);
-            sb[tid] = p.beta[bh * p.Tp + c0 + tid];
-        }
-        __syncthreads();
-        float *ck = p.ckpt + ((bh * NC + c) * D + i) * D + j0;
+        __syncthreads();  // chunk c's rows are visible
+        float *ck = p.ckpt + ((bh * NC + c) * D + i) * D + cb;
 #pragma unroll
-        for (int e = 0; e < CW; ++e) ck[e] = S[e];
+        for (int e = 0; e < CW; ++e) ck[16 * e] = S[e];
         for (int tt = 0; tt < n; ++tt) {
+            const float a = expf(st.la[buf][tt]), be = st.be[buf][tt];
             float u = 0.0f;
 #pragma unroll
-            for (int e = 0; e < CW; ++e) u = fmaf(S[e], sk[tt][j0 + e], u);
+            for (int e = 0; e < CW; ++e) u = fmaf(S[e], st.k[buf][tt][cb + 16 * e], u);
             u = sum16(u);
-            const float dl = sb[tt] * (sv[tt][r] - sa[tt] * u);
+            const float dl = be * (st.v[buf][tt][r] - a * u);
             float ov = 0.0f;
 #pragma unroll
             for (int e = 0; e < CW; ++e) {
-                S[e] = fmaf(sa[tt], S[e], dl * sk[tt][j0 + e]);
-                ov = fmaf(S[e], sq[tt][j0 + e], ov);
+                S[e] = fmaf(a, S[e], dl * st.k[buf][tt][cb + 16 * e]);
+                ov = fmaf(S[e], st.q[buf][tt][cb + 16 * e], ov);
             }
             ov = sum16(ov);
             if (cb == 0) p.o[((static_cast<size_t>(b) * p.T + c0 + tt) * p.H + h) * D + i] = ov;
         }
+        __syncthreads();  // buffer buf is read out before chunk c + 2 is copied into it
     }
 }
 
@@ -172,16 +200,18 @@ __global__ void __launch_bounds__(256) gdn_bwd_out(const BwdParams p) {
 // ------------------------------------------------------------ the recurrence backwards
 // Same CTA layout as gdn_bwd_fwd_rows.  Per chunk of kC tokens, last chunk
 // first: the states before each token (and after the last) are recomputed
-// from the checkpoint into sS, the gradient D runs backwards through the
-// chunk (kept in registers across chunks, each D_t also stored in sD), and
-// the row sums of the chunk are then taken from shared memory.
+// from the checkpoint into S, the gradient D runs backwards through the chunk
+// (kept in registers across chunks, each D_t also stored in Dg), and the row
+// sums of the chunk are then taken from shared memory.  The next chunk's
+// inputs (and, in registers, its checkpoint) are fetched during this one.
 template <int D>
 struct CoreSmem {
-    float S[kC + 1][kR][D];  // slot s: state before token c0 + s
-    float Dg[kC][kR][D];     // D_t after do_t q^_t^T is added
-    float q[kC][D], k[kC][D];
-    float v[kC][kR], dO[kC][kR], u[kC][kR], dl[kC][kR], ddl[kC][kR], du[kC][kR];
-    float a[kC], be[kC];
+    // rows padded by 16 floats: the two rows a warp touches fall in different banks
+    float S[kC + 1][kR][D + 16];  // slot s: state before token c0 + s
+    float Dg[kC][kR][D + 16];     // D_t after do_t q^_t^T is added
+    Stage<D> st;
+    float dO[2][kC][kR];
+    float u[kC][kR], dl[kC][kR], ddl[kC][kR], du[kC][kR];
     float part[kC][128];     // per-thread pieces of <D_t, S_{t-1}>
 };
 
@@ -194,73 +224,74 @@ __global__ void __launch_bounds__(128) gdn_bwd_core(const BwdParams p) {
     const size_t bh = static_cast<size_t>(b) * p.H + h;
     const size_t BH = static_cast<size_t>(p.B) * p.H;
     const int tid = threadIdx.x, r = tid >> 4, cb = tid & 15;
-    const int i = g * kR + r, j0 = cb * CW;
+    const int i = g * kR + r;
     const int NC = (p.T + kC - 1) / kC;
-    float Dr[CW];
+    float Dr[CW], ckn[CW];
 #pragma unroll
     for (int e = 0; e < CW; ++e) Dr[e] = 0.0f;
-    for (int c = NC - 1; c >= 0; --c) {
-        const int c0 = c * kC, n = min(kC, p.T - c0);
-        __syncthreads();  // the previous chunk's row sums are done with the buffers
-        for (int e = tid; e < kC * D; e += 128) {
-            const size_t src = (bh * p.Tp + c0 + e / D) * D + e % D;
-            sm.q[e / D][e % D] = p.qh[src];
-            sm.k[e / D][e % D] = p.kh[src];
-        }
-        if (tid < kC * kR) {
-            const size_t src = (bh * p.Tp + c0 + tid / kR) * D + g * kR + tid % kR;
-            sm.v[tid / kR][tid % kR] = p.vh[src];
-            sm.dO[tid / kR][tid % kR] = p.dO[src];
-        }
-        if (tid < kC) {
-            sm.a[tid] = expf(p.log_alpha[bh * p.Tp + c0 + tid]);
-            sm.be[tid] = p.beta[bh * p.Tp + c0 + tid];
-        }
-        float S[CW];
-        const float *ck = p.ckpt + ((bh * NC + c) * D + i) * D + j0;
+    auto load_ck = [&](int c) {
+        const float *ck = p.ckpt + ((bh * NC + c) * D + i) * D + cb;
 #pragma unroll
-        for (int e = 0; e < CW; ++e) S[e] = ck[e];
-        __syncthreads();
+        for (int e = 0; e < CW; ++e) ckn[e] = ck[16 * e];
+    };
+    stage_chunk<D>(sm.st, sm.dO, p, bh, g, NC - 1, (NC - 1) & 1, tid);
+    load_ck(NC - 1);
+    for (int c = NC - 1; c >= 0; --c) {
+        const int c0 = c * kC, n = min(kC, p.T - c0), buf = c & 1;
+        float S[CW];
+#pragma unroll
+        for (int e = 0; e < CW; ++e) S[e] = ckn[e];
+        if (c > 0) {
+            stage_chunk<D>(sm.st, sm.dO, p, bh, g, c - 1, buf ^ 1, tid);
+            load_ck(c - 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();  // chunk c's inputs are visible; the previous chunk's row sums are done
+        const Stage<D> &st = sm.st;
         // states of the chunk
         for (int tt = 0; tt < n; ++tt) {
+            const float a = expf(st.la[buf][tt]), be = st.be[buf][tt];
             float u = 0.0f;
 #pragma unroll
             for (int e = 0; e < CW; ++e) {
-                sm.S[tt][r][j0 + e] = S[e];
-                u = fmaf(S[e], sm.k[tt][j0 + e], u);
+                sm.S[tt][r][cb + 16 * e] = S[e];
+                u = fmaf(S[e], st.k[buf][tt][cb + 16 * e], u);
             }
             u = sum16(u);
-            const float dl = sm.be[tt] * (sm.v[tt][r] - sm.a[tt] * u);
+            const float dl = be * (st.v[buf][tt][r] - a * u);
 #pragma unroll
-            for (int e = 0; e < CW; ++e) S[e] = fmaf(sm.a[tt], S[e], dl * sm.k[tt][j0 + e]);
+            for (int e = 0; e < CW; ++e) S[e] = fmaf(a, S[e], dl * st.k[buf][tt][cb + 16 * e]);
             if (cb == 0) {
                 sm.u[tt][r] = u;
                 sm.dl[tt][r] = dl;
             }
         }
 #pragma unroll
-        for (int e = 0; e < CW; ++e) sm.S[n][r][j0 + e] = S[e];
+        for (int e = 0; e < CW; ++e) sm.S[n][r][cb + 16 * e] = S[e];
         // the gradient, backwards through the chunk
         for (int tt = n - 1; tt >= 0; --tt) {
-            const float dov = sm.dO[tt][r];
+            const float a = expf(st.la[buf][tt]), be = st.be[buf][tt];
+            const float dov = sm.dO[buf][tt][r];
             float ddl = 0.0f, pr = 0.0f;
 #pragma unroll
             for (int e = 0; e < CW; ++e) {
-                Dr[e] = fmaf(dov, sm.q[tt][j0 + e], Dr[e]);
-                sm.Dg[tt][r][j0 + e] = Dr[e];
-                ddl = fmaf(Dr[e], sm.k[tt][j0 + e], ddl);
-                pr = fmaf(Dr[e], sm.S[tt][r][j0 + e], pr);
+                Dr[e] = fmaf(dov, st.q[buf][tt][cb + 16 * e], Dr[e]);
+                sm.Dg[tt][r][cb + 16 * e] = Dr[e];
+                ddl = fmaf(Dr[e], st.k[buf][tt][cb + 16 * e], ddl);
+                pr = fmaf(Dr[e], sm.S[tt][r][cb + 16 * e], pr);
             }
             ddl = sum16(ddl);
             sm.part[tt][tid] = pr;
-            const float du = -sm.a[tt] * sm.be[tt] * ddl;
+            const float du = -a * be * ddl;
             if (cb == 0) {
                 sm.ddl[tt][r] = ddl;
                 sm.du[tt][r] = du;
-                p.dvh[(bh * p.Tp + c0 + tt) * D + i] = sm.be[tt] * ddl;
+                p.dvh[(bh * p.Tp + c0 + tt) * D + i] = be * ddl;
             }
 #pragma unroll
-            for (int e = 0; e < CW; ++e) Dr[e] = fmaf(sm.a[tt], Dr[e], du * sm.k[tt][j0 + e]);
+            for (int e = 0; e < CW; ++e) Dr[e] = fmaf(a, Dr[e], du * st.k[buf][tt][cb + 16 * e]);
         }
         __syncthreads();
         // row sums of the chunk (this group's part)
@@ -269,7 +300,7 @@ __global__ void __launch_bounds__(128) gdn_bwd_core(const BwdParams p) {
             float dq = 0.0f, dk = 0.0f;
 #pragma unroll
             for (int rr = 0; rr < kR; ++rr) {
-                dq = fmaf(sm.S[tt + 1][rr][j], sm.dO[tt][rr], dq);
+                dq = fmaf(sm.S[tt + 1][rr][j], sm.dO[buf][tt][rr], dq);
                 dk = fmaf(sm.Dg[tt][rr][j], sm.dl[tt][rr], dk);
                 dk = fmaf(sm.S[tt][rr][j], sm.du[tt][rr], dk);
             }
@@ -283,16 +314,18 @@ __global__ void __launch_bounds__(128) gdn_bwd_core(const BwdParams p) {
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
             if (lane == 0) {
+                const float a = expf(st.la[buf][tt]), be = st.be[buf][tt];
                 float ud = 0.0f, db = 0.0f;
                 for (int rr = 0; rr < kR; ++rr) {
                     ud = fmaf(sm.u[tt][rr], sm.ddl[tt][rr], ud);
-                    db = fmaf(sm.ddl[tt][rr], sm.v[tt][rr] - sm.a[tt] * sm.u[tt][rr], db);
+                    db = fmaf(sm.ddl[tt][rr], st.v[buf][tt][rr] - a * sm.u[tt][rr], db);
                 }
                 const size_t dst = (g * BH + bh) * p.Tp + c0 + tt;
-                p.da_part[dst] = s - sm.be[tt] * ud;
+                p.da_part[dst] = s - be * ud;
                 p.db_part[dst] = db;
             }
         }
+        __syncthreads();  // buffer buf and the chunk arrays are read out before they are refilled
     }
 }
 
@@ -536,31 +569,42 @@ int bwd_out_blocks(long long rows) {
     return static_cast<int>(blocks < 1024 ? blocks : 1024);
 }
 
-cudaError_t launch_backward(const BwdParams &p, InType in, InType out, cudaStream_t s, int *launches) {
+cudaError_t launch_backward(const BwdParams &p, InType in, InType out, cudaStream_t s, int *launches,
+                            void *const *events) {
     cudaError_t e;
     int n = 0;
+    // events[i] (optional) is recorded before the i-th launch, events[5] after the last
+    auto mark = [&](int i) -> cudaError_t {
+        return events ? cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[i]), s) : cudaSuccess;
+    };
+    if ((e = mark(0)) != cudaSuccess) return e;
     const dim3 grid_rows(p.d / kR, p.H, p.B);
     if (p.d == 128) gdn_bwd_fwd_rows<128><<<grid_rows, 128, 0, s>>>(p);
     else gdn_bwd_fwd_rows<64><<<grid_rows, 128, 0, s>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     ++n;
+    if ((e = mark(1)) != cudaSuccess) return e;
     const int nb = bwd_out_blocks(static_cast<long long>(p.B) * p.T * p.H);
     if (in == InType::BF16) e = launch_out_bwd_z<__nv_bfloat16>(p, out, nb, s);
     else if (in == InType::F16) e = launch_out_bwd_z<__half>(p, out, nb, s);
     else e = launch_out_bwd_z<float>(p, out, nb, s);
     if (e != cudaSuccess) return e;
     ++n;
+    if ((e = mark(2)) != cudaSuccess) return e;
     e = p.d == 128 ? launch_core_bwd<128>(p, s) : launch_core_bwd<64>(p, s);
     if (e != cudaSuccess) return e;
     ++n;
+    if ((e = mark(3)) != cudaSuccess) return e;
     if (in == InType::BF16) e = launch_tokens_bwd<__nv_bfloat16>(p, s);
     else if (in == InType::F16) e = launch_tokens_bwd<__half>(p, s);
     else e = launch_tokens_bwd<float>(p, s);
     if (e != cudaSuccess) return e;
     ++n;
+    if ((e = mark(4)) != cudaSuccess) return e;
     gdn_bwd_params<<<64, 256, 0, s>>>(p, p.d, nb);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     ++n;
+    if ((e = mark(5)) != cudaSuccess) return e;
     if (launches) *launches = n;
     return cudaSuccess;
 }

@@ -350,6 +350,17 @@ __device__ __forceinline__ float2 unpack_half2(uint32_t u) {
 // SiLU with the fast reciprocal divide (2 ulp); for u -> -inf the denominator
 // overflows and the result is 0, the limit of u e^u.
 // SiLU for the fp32 CUDA-core path (held to 1e-5 relative).
+// Asynchronous global -> shared copies (16 bytes, L2 only; 4 bytes), committed and waited in groups.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 __device__ __forceinline__ float silu_f(float u) { return __fdividef(u, 1.0f + __expf(-u)); }
 
 // SiLU for the tensor-core path: u * sigmoid(u) = h + h * tanh(h) with h = u / 2 (from

@@ -152,8 +152,10 @@ struct BwdParams {
     float l2_eps, norm_eps, q_scale;
 };
 int bwd_out_blocks(long long rows);
-// Enqueues the five backward kernels after the prep; *launches receives their count.
-cudaError_t launch_backward(const BwdParams &p, InType in, InType out, cudaStream_t s, int *launches);
+// Enqueues the five backward kernels after the prep; *launches receives their count.  events
+// (optional, 6 cudaEvent_t) are recorded before each launch and after the last.
+cudaError_t launch_backward(const BwdParams &p, InType in, InType out, cudaStream_t s, int *launches,
+                            void *const *events = nullptr);
 
 }  // namespace gdn
 

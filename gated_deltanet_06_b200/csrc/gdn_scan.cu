@@ -281,12 +281,6 @@ constexpr int RS = 132;  // padded row stride (floats)
 constexpr uint32_t SMEM_BYTES = (2 * 128 * RS + 16 * RS) * 4;
 }  // namespace cb
 
-__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // x = hi + lo, both tf32 (round to nearest, ties away)
 __device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo) {

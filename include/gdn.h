@@ -223,6 +223,12 @@ int gdn_backward_launches(gdn_plan_t plan);
 gdn_status gdn_backward(gdn_plan_t plan, const gdn_inputs *in, const void *dy, const gdn_grads *grads,
                         void *workspace, gdn_stream_t stream);
 
+/* gdn_backward with per-kernel timing, as gdn_forward_timed: events[i] is
+ * recorded before the i-th of the gdn_backward_launches(plan) launches and
+ * events[L] after the last; n_events must be L + 1. */
+gdn_status gdn_backward_timed(gdn_plan_t plan, const gdn_inputs *in, const void *dy, const gdn_grads *grads,
+                              void *workspace, gdn_stream_t stream, void *const *events, int n_events);
+
 /* Synchronise `stream`, then read and clear the device status word in the
  * workspace.  Returns GDN_OK, GDN_ERR_TIMEOUT or GDN_ERR_DEVICE_CHECK (or
  * GDN_ERR_CUDA if the synchronisation itself failed). */
