@@ -31,6 +31,7 @@ namespace {
 constexpr int kR = 8;     // rows of S per CTA
 constexpr int kC = 8;     // tokens per checkpoint chunk
 constexpr int kTile = 64; // tokens per CTA of the token kernel
+constexpr int kBT = 256;  // threads per CTA of the row kernels: one warp per row of S
 
 template <typename T>
 __device__ __forceinline__ float ldf(const T *p);
@@ -47,18 +48,18 @@ __device__ __forceinline__ float dsilu(float a) {
     const float s = sigm(a);
     return s * (1.0f + a * (1.0f - s));
 }
-// sum over the 16 lanes of a row (lanes 16k .. 16k+15)
-__device__ __forceinline__ float sum16(float x) {
+// sum over the 32 lanes of a warp (one row of S)
+__device__ __forceinline__ float rowsum(float x) {
 #pragma unroll
-    for (int off = 8; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
     return x;
 }
 
 // ------------------------------------------------------------ forward rows
-// One CTA per (group of kR rows, h, b), 128 threads: thread (r, cb) holds
-// columns cb, cb + 16, cb + 32, ... of row g*kR + r of S (so that the 16
-// lanes of a row touch 16 consecutive words of shared memory).  Writes o [B][T][H][D] and the
-// state before every chunk of kC tokens.  The next chunk's q^, k^, v^ rows and
+// One CTA per (group of kR rows, h, b), kBT threads, one warp per row: lane cb
+// holds columns cb, cb + 32, ... of row g*kR + r of S, so that a warp touches
+// 32 consecutive words of shared memory.  Writes o [B][T][H][D] and the state
+// before every chunk of kC tokens.  The next chunk's q^, k^, v^ rows and
 // gates are copied into the other shared buffer while this one is computed.
 template <int D>
 struct Stage {
@@ -70,7 +71,7 @@ template <int D>
 __device__ __forceinline__ void stage_chunk(Stage<D> &st, float (*dO)[kC][kR], const BwdParams &p, size_t bh,
                                             int g, int c, int buf, int tid) {
     const int c0 = c * kC;
-    for (int e = tid; e < kC * D / 4; e += 128) {
+    for (int e = tid; e < kC * D / 4; e += kBT) {
         const int tt = e / (D / 4), j = (e % (D / 4)) * 4;
         const size_t src = (bh * p.Tp + c0 + tt) * D + j;
         cp_async16(&st.q[buf][tt][j], p.qh + src);
@@ -89,12 +90,12 @@ __device__ __forceinline__ void stage_chunk(Stage<D> &st, float (*dO)[kC][kR], c
 }
 
 template <int D>
-__global__ void __launch_bounds__(128) gdn_bwd_fwd_rows(const BwdParams p) {
-    constexpr int CW = D / 16;
+__global__ void __launch_bounds__(kBT) gdn_bwd_fwd_rows(const BwdParams p) {
+    constexpr int CW = D / 32;
     __shared__ __align__(16) Stage<D> st;
     const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const size_t bh = static_cast<size_t>(b) * p.H + h;
-    const int tid = threadIdx.x, r = tid >> 4, cb = tid & 15;
+    const int tid = threadIdx.x, r = tid >> 5, cb = tid & 31;
     const int i = g * kR + r;
     const int NC = (p.T + kC - 1) / kC;
     float S[CW];
@@ -112,21 +113,21 @@ __global__ void __launch_bounds__(128) gdn_bwd_fwd_rows(const BwdParams p) {
         __syncthreads();  // chunk c's rows are visible
         float *ck = p.ckpt + ((bh * NC + c) * D + i) * D + cb;
 #pragma unroll
-        for (int e = 0; e < CW; ++e) ck[16 * e] = S[e];
+        for (int e = 0; e < CW; ++e) ck[32 * e] = S[e];
         for (int tt = 0; tt < n; ++tt) {
             const float a = expf(st.la[buf][tt]), be = st.be[buf][tt];
             float u = 0.0f;
 #pragma unroll
-            for (int e = 0; e < CW; ++e) u = fmaf(S[e], st.k[buf][tt][cb + 16 * e], u);
-            u = sum16(u);
+            for (int e = 0; e < CW; ++e) u = fmaf(S[e], st.k[buf][tt][cb + 32 * e], u);
+            u = rowsum(u);
             const float dl = be * (st.v[buf][tt][r] - a * u);
             float ov = 0.0f;
 #pragma unroll
             for (int e = 0; e < CW; ++e) {
-                S[e] = fmaf(a, S[e], dl * st.k[buf][tt][cb + 16 * e]);
-                ov = fmaf(S[e], st.q[buf][tt][cb + 16 * e], ov);
+                S[e] = fmaf(a, S[e], dl * st.k[buf][tt][cb + 32 * e]);
+                ov = fmaf(S[e], st.q[buf][tt][cb + 32 * e], ov);
             }
-            ov = sum16(ov);
+            ov = rowsum(ov);
             if (cb == 0) p.o[((static_cast<size_t>(b) * p.T + c0 + tt) * p.H + h) * D + i] = ov;
         }
         __syncthreads();  // buffer buf is read out before chunk c + 2 is copied into it
@@ -206,24 +207,23 @@ __global__ void __launch_bounds__(256) gdn_bwd_out(const BwdParams p) {
 // inputs (and, in registers, its checkpoint) are fetched during this one.
 template <int D>
 struct CoreSmem {
-    // rows padded by 16 floats: the two rows a warp touches fall in different banks
-    float S[kC + 1][kR][D + 16];  // slot s: state before token c0 + s
-    float Dg[kC][kR][D + 16];     // D_t after do_t q^_t^T is added
+    float S[kC + 1][kR][D];  // slot s: state before token c0 + s
+    float Dg[kC][kR][D];     // D_t after do_t q^_t^T is added
     Stage<D> st;
     float dO[2][kC][kR];
     float u[kC][kR], dl[kC][kR], ddl[kC][kR], du[kC][kR];
-    float part[kC][128];     // per-thread pieces of <D_t, S_{t-1}>
+    float part[kC][kBT];     // per-thread pieces of <D_t, S_{t-1}>
 };
 
 template <int D>
-__global__ void __launch_bounds__(128) gdn_bwd_core(const BwdParams p) {
-    constexpr int CW = D / 16;
+__global__ void __launch_bounds__(kBT) gdn_bwd_core(const BwdParams p) {
+    constexpr int CW = D / 32;
     extern __shared__ __align__(16) uint8_t smem_raw[];
     CoreSmem<D> &sm = *reinterpret_cast<CoreSmem<D> *>(smem_raw);
     const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const size_t bh = static_cast<size_t>(b) * p.H + h;
     const size_t BH = static_cast<size_t>(p.B) * p.H;
-    const int tid = threadIdx.x, r = tid >> 4, cb = tid & 15;
+    const int tid = threadIdx.x, r = tid >> 5, cb = tid & 31;
     const int i = g * kR + r;
     const int NC = (p.T + kC - 1) / kC;
     float Dr[CW], ckn[CW];
@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(128) gdn_bwd_core(const BwdParams p) {
     auto load_ck = [&](int c) {
         const float *ck = p.ckpt + ((bh * NC + c) * D + i) * D + cb;
 #pragma unroll
-        for (int e = 0; e < CW; ++e) ckn[e] = ck[16 * e];
+        for (int e = 0; e < CW; ++e) ckn[e] = ck[32 * e];
     };
     stage_chunk<D>(sm.st, sm.dO, p, bh, g, NC - 1, (NC - 1) & 1, tid);
     load_ck(NC - 1);
@@ -256,20 +256,20 @@ __global__ void __launch_bounds__(128) gdn_bwd_core(const BwdParams p) {
             float u = 0.0f;
 #pragma unroll
             for (int e = 0; e < CW; ++e) {
-                sm.S[tt][r][cb + 16 * e] = S[e];
-                u = fmaf(S[e], st.k[buf][tt][cb + 16 * e], u);
+                sm.S[tt][r][cb + 32 * e] = S[e];
+                u = fmaf(S[e], st.k[buf][tt][cb + 32 * e], u);
             }
-            u = sum16(u);
+            u = rowsum(u);
             const float dl = be * (st.v[buf][tt][r] - a * u);
 #pragma unroll
-            for (int e = 0; e < CW; ++e) S[e] = fmaf(a, S[e], dl * st.k[buf][tt][cb + 16 * e]);
+            for (int e = 0; e < CW; ++e) S[e] = fmaf(a, S[e], dl * st.k[buf][tt][cb + 32 * e]);
             if (cb == 0) {
                 sm.u[tt][r] = u;
                 sm.dl[tt][r] = dl;
             }
         }
 #pragma unroll
-        for (int e = 0; e < CW; ++e) sm.S[n][r][cb + 16 * e] = S[e];
+        for (int e = 0; e < CW; ++e) sm.S[n][r][cb + 32 * e] = S[e];
         // the gradient, backwards through the chunk
         for (int tt = n - 1; tt >= 0; --tt) {
             const float a = expf(st.la[buf][tt]), be = st.be[buf][tt];
@@ -277,12 +277,12 @@ __global__ void __launch_bounds__(128) gdn_bwd_core(const BwdParams p) {
             float ddl = 0.0f, pr = 0.0f;
 #pragma unroll
             for (int e = 0; e < CW; ++e) {
-                Dr[e] = fmaf(dov, st.q[buf][tt][cb + 16 * e], Dr[e]);
-                sm.Dg[tt][r][cb + 16 * e] = Dr[e];
-                ddl = fmaf(Dr[e], st.k[buf][tt][cb + 16 * e], ddl);
-                pr = fmaf(Dr[e], sm.S[tt][r][cb + 16 * e], pr);
+                Dr[e] = fmaf(dov, st.q[buf][tt][cb + 32 * e], Dr[e]);
+                sm.Dg[tt][r][cb + 32 * e] = Dr[e];
+                ddl = fmaf(Dr[e], st.k[buf][tt][cb + 32 * e], ddl);
+                pr = fmaf(Dr[e], sm.S[tt][r][cb + 32 * e], pr);
             }
-            ddl = sum16(ddl);
+            ddl = rowsum(ddl);
             sm.part[tt][tid] = pr;
             const float du = -a * be * ddl;
             if (cb == 0) {
@@ -291,11 +291,11 @@ __global__ void __launch_bounds__(128) gdn_bwd_core(const BwdParams p) {
                 p.dvh[(bh * p.Tp + c0 + tt) * D + i] = be * ddl;
             }
 #pragma unroll
-            for (int e = 0; e < CW; ++e) Dr[e] = fmaf(a, Dr[e], du * st.k[buf][tt][cb + 16 * e]);
+            for (int e = 0; e < CW; ++e) Dr[e] = fmaf(a, Dr[e], du * st.k[buf][tt][cb + 32 * e]);
         }
         __syncthreads();
         // row sums of the chunk (this group's part)
-        for (int e = tid; e < n * D; e += 128) {
+        for (int e = tid; e < n * D; e += kBT) {
             const int tt = e / D, j = e % D;
             float dq = 0.0f, dk = 0.0f;
 #pragma unroll
@@ -309,8 +309,10 @@ __global__ void __launch_bounds__(128) gdn_bwd_core(const BwdParams p) {
             p.dk_part[dst] = dk;
         }
         const int warp = tid >> 5, lane = tid & 31;
-        for (int tt = warp; tt < n; tt += 4) {
-            float s = sm.part[tt][lane] + sm.part[tt][lane + 32] + sm.part[tt][lane + 64] + sm.part[tt][lane + 96];
+        for (int tt = warp; tt < n; tt += kBT / 32) {
+            float s = 0.0f;
+#pragma unroll
+            for (int q = 0; q < kBT / 32; ++q) s += sm.part[tt][lane + 32 * q];
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
             if (lane == 0) {
@@ -550,7 +552,7 @@ cudaError_t launch_core_bwd(const BwdParams &p, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    gdn_bwd_core<D><<<dim3(D / kR, p.H, p.B), 128, bytes, s>>>(p);
+    gdn_bwd_core<D><<<dim3(D / kR, p.H, p.B), kBT, bytes, s>>>(p);
     return cudaGetLastError();
 }
 
@@ -579,8 +581,8 @@ cudaError_t launch_backward(const BwdParams &p, InType in, InType out, cudaStrea
     };
     if ((e = mark(0)) != cudaSuccess) return e;
     const dim3 grid_rows(p.d / kR, p.H, p.B);
-    if (p.d == 128) gdn_bwd_fwd_rows<128><<<grid_rows, 128, 0, s>>>(p);
-    else gdn_bwd_fwd_rows<64><<<grid_rows, 128, 0, s>>>(p);
+    if (p.d == 128) gdn_bwd_fwd_rows<128><<<grid_rows, kBT, 0, s>>>(p);
+    else gdn_bwd_fwd_rows<64><<<grid_rows, kBT, 0, s>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     ++n;
     if ((e = mark(1)) != cudaSuccess) return e;

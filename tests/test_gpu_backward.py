@@ -1,11 +1,11 @@
 """gdn_backward on a B200 against the oracle's backward (fp64, written out
 per step and pinned by finite differences).
 
-The bar: the backward runs in fp32 on CUDA cores for every plan, like the
-fp32 forward whose bar is rel-L2 <= 1e-5; its outputs are longer chains of
-fp32 operations (the gradient runs back through the whole recurrence, and the
-parameter gradients are sums over every token), so each gradient tensor is
-held to rel-L2 <= 1e-4 against the oracle on the same inputs and dy.
+The bar: the backward runs in fp32 on CUDA cores for every plan, so each
+gradient tensor takes the fp32 forward's bar, rel-L2 <= 1e-5 against the
+oracle on the same inputs and dy.  Measured: about 2e-7 for the per-token
+gradients and up to 1.2e-6 for dA_log and ddt_bias, whose H entries are each
+a sum over every token with cancellation.
 """
 import numpy as np
 import pytest
@@ -16,7 +16,7 @@ from oracle import backward as ob
 
 pytestmark = pytest.mark.gpu
 
-REL_L2_GRAD = 1e-4
+REL_L2_GRAD = 1e-5
 KEY = {"dq": "q", "dk": "k", "dv": "v", "dz": "z", "dg": "g", "db": "b", "dconv_q": "conv_q",
        "dconv_k": "conv_k", "dconv_v": "conv_v", "dA_log": "A_log", "ddt_bias": "dt_bias", "dnorm_w": "norm_w"}
 
