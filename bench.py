@@ -462,29 +462,58 @@ def main():
                "kernels_ms": {bnames[i]: evk[i].elapsed_time(evk[i + 1]) for i in range(LB)}}
         del ws_b, gr, dy
 
-    # end to end through the public host-buffer entry point
+    # end to end through the public host-buffer entry point (gdn_forward_host: every input copied from
+    # pinned host memory, the forward, y copied back), first on one stream, then on two streams that
+    # take alternate steps with their own staging, workspace and host output, so that one step's
+    # host-to-device copies overlap the previous step's compute and device-to-host copy
     e2e = None
     if not args.no_e2e:
         host = {n: tens[n].cpu().pin_memory() for n in tens}
-        y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-        staging = torch.empty(plan.staging_bytes, dtype=torch.uint8, device=dev)
         hptrs = gdn.tensor_ptrs(host)
-        n_e2e = max(3, min(args.steps, 10))
-        plan.forward_host_raw(hptrs, y_host.data_ptr(), staging.data_ptr(), ws.data_ptr(), s)
-        torch.cuda.synchronize()
-        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if world > 1:
-            dist.barrier()
-        ev0.record(stream)
-        for _ in range(n_e2e):
-            plan.forward_host_raw(hptrs, y_host.data_ptr(), staging.data_ptr(), ws.data_ptr(), s)
-        ev1.record(stream)
-        torch.cuda.synchronize()
-        te_ms = ranks_max(ev0.elapsed_time(ev1) / n_e2e, world, dist, dev)
+        n_e2e = max(4, min(args.steps, 10))
+        y_hosts = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for _ in range(2)]
+        stagings = [torch.empty(plan.staging_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
+        wss = [ws, torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=dev)]
+        streams = [torch.cuda.Stream(dev), torch.cuda.Stream(dev)]
+
+        def run_e2e(nstreams):
+            for i in range(nstreams):  # warm-up
+                plan.forward_host_raw(hptrs, y_hosts[i].data_ptr(), stagings[i].data_ptr(), wss[i].data_ptr(),
+                                      streams[i].cuda_stream)
+            torch.cuda.synchronize()
+            if world > 1:
+                dist.barrier()
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ev0.record(stream)
+            for i in range(nstreams):
+                streams[i].wait_event(ev0)
+            for k in range(n_e2e):
+                i = k % nstreams
+                plan.forward_host_raw(hptrs, y_hosts[i].data_ptr(), stagings[i].data_ptr(), wss[i].data_ptr(),
+                                      streams[i].cuda_stream)
+            for i in range(nstreams):
+                ev = torch.cuda.Event()
+                ev.record(streams[i])
+                stream.wait_event(ev)
+            ev1.record(stream)
+            torch.cuda.synchronize()
+            for i in range(nstreams):
+                st = plan.device_status(wss[i].data_ptr(), streams[i].cuda_stream)
+                if st != gdn.OK:
+                    raise SystemExit(f"device status after the end-to-end steps: {gdn.status_string(st)}")
+            return ranks_max(ev0.elapsed_time(ev1) / n_e2e, world, dist, dev)
+
+        serial_ms = run_e2e(1)
+        te_ms = run_e2e(2)
+        if not torch.equal(y_hosts[0], y_hosts[1]):
+            raise SystemExit("the two streams' end-to-end outputs differ")
         h2d = sum(host[n].numel() * host[n].element_size() for n in host)
-        d2h = y_host.numel() * y_host.element_size()
+        d2h = y_hosts[0].numel() * y_hosts[0].element_size()
         e2e = {"value": job_throughput(world, tokens, te_ms), "unit": UNIT,
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n_e2e}
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n_e2e,
+               "streams": 2, "ms_per_step": te_ms,
+               "one_stream": {"value": job_throughput(world, tokens, serial_ms), "ms_per_step": serial_ms}}
+        del wss[1], stagings
 
     if rank != 0:
         if world > 1:

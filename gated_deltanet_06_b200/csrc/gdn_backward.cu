@@ -114,7 +114,10 @@ __global__ void __launch_bounds__(kBT) gdn_bwd_fwd_rows(const BwdParams p) {
         float *ck = p.ckpt + ((bh * NC + c) * D + i) * D + cb;
 #pragma unroll
         for (int e = 0; e < CW; ++e) ck[32 * e] = S[e];
-        for (int tt = 0; tt < n; ++tt) {
+        // unrolled over the chunk (n is uniform): token t's output sum overlaps token t + 1's update
+#pragma unroll
+        for (int tt = 0; tt < kC; ++tt) {
+            if (tt >= n) break;
             const float a = expf(st.la[buf][tt]), be = st.be[buf][tt];
             float u = 0.0f;
 #pragma unroll
@@ -251,7 +254,9 @@ __global__ void __launch_bounds__(kBT) gdn_bwd_core(const BwdParams p) {
         __syncthreads();  // chunk c's inputs are visible; the previous chunk's row sums are done
         const Stage<D> &st = sm.st;
         // states of the chunk
-        for (int tt = 0; tt < n; ++tt) {
+#pragma unroll
+        for (int tt = 0; tt < kC; ++tt) {
+            if (tt >= n) break;
             const float a = expf(st.la[buf][tt]), be = st.be[buf][tt];
             float u = 0.0f;
 #pragma unroll
@@ -271,7 +276,10 @@ __global__ void __launch_bounds__(kBT) gdn_bwd_core(const BwdParams p) {
 #pragma unroll
         for (int e = 0; e < CW; ++e) sm.S[n][r][cb + 32 * e] = S[e];
         // the gradient, backwards through the chunk
-        for (int tt = n - 1; tt >= 0; --tt) {
+#pragma unroll
+        for (int t2 = kC - 1; t2 >= 0; --t2) {
+            const int tt = t2 - (kC - n);  // tokens n-1 .. 0
+            if (tt < 0) break;
             const float a = expf(st.la[buf][tt]), be = st.be[buf][tt];
             const float dov = sm.dO[buf][tt][r];
             float ddl = 0.0f, pr = 0.0f;
