@@ -124,8 +124,7 @@ class ClockSampler:
             except (ValueError, IndexError):
                 idx = None
         sel = ["-i", str(idx)] if idx is not None else []
-        self.err = os.path.join(ROOT, "gpurun_out", "clock_sampler.err") if os.path.isdir(
-            os.path.join(ROOT, "gpurun_out")) else os.devnull
+        self.err = os.devnull
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
                                           "-lms", "100"] + sel, stdout=subprocess.PIPE,
