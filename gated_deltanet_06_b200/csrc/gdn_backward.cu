@@ -553,13 +553,10 @@ cudaError_t launch_out_bwd_z(const BwdParams &p, InType yt, int blocks, cudaStre
 
 template <int D>
 cudaError_t launch_core_bwd(const BwdParams &p, cudaStream_t s) {
-    static bool attr = false;
+    static SmemOnce once;
     const int bytes = static_cast<int>(sizeof(CoreSmem<D>));
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(gdn_bwd_core<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    cudaError_t e = raise_smem_once(once, gdn_bwd_core<D>, bytes);
+    if (e != cudaSuccess) return e;
     gdn_bwd_core<D><<<dim3(D / kR, p.H, p.B), kBT, bytes, s>>>(p);
     return cudaGetLastError();
 }

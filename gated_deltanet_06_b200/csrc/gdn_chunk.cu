@@ -506,13 +506,9 @@ cudaError_t launch_chunk(const ChunkParams &p, const CUtensorMap &tmK, const CUt
                          const CUtensorMap &tmQ, const CUtensorMap &tmW, const CUtensorMap &tmU,
                          const CUtensorMap &tmQt, const CUtensorMap &tmAqk, const CUtensorMap &tmAqkH,
                          cudaStream_t s, bool pdl) {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gdn_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(SMEM_BYTES));
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static SmemOnce once;
+    cudaError_t e = raise_smem_once(once, gdn_chunk_kernel, static_cast<int>(SMEM_BYTES));
+    if (e != cudaSuccess) return e;
     dim3 grid(p.NB, p.BH);
     return launch_k(gdn_chunk_kernel, grid, dim3(256), SMEM_BYTES, s, pdl, p, tmK, tmV, tmQ, tmW, tmU, tmQt, tmAqk,
                     tmAqkH);

@@ -7,7 +7,26 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace gdn {
+
+// Raise a kernel's dynamic shared-memory limit once per device.  Safe to call from
+// several host threads (a repeated call only repeats the same attribute set).
+constexpr int kMaxDevices = 64;
+struct SmemOnce {
+    std::atomic<int> done[kMaxDevices];  // zero-initialised: objects of this type are static
+};
+template <typename K>
+inline cudaError_t raise_smem_once(SmemOnce &once, K kernel, int bytes) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < kMaxDevices && once.done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) once.done[dev].store(1, std::memory_order_release);
+    return e;
+}
 
 enum class InType { BF16 = 0, F32 = 1, F16 = 2 };
 

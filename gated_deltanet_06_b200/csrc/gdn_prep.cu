@@ -325,27 +325,19 @@ cudaError_t launch_typed(const PrepParams &p, cudaStream_t s) {
 
 cudaError_t launch_prep_tma(const PrepParams &p, InType in, const CUtensorMap &tmq, const CUtensorMap &tmk,
                             const CUtensorMap &tmv, cudaStream_t s) {
-    static bool attr_bf = false, attr_h = false;
+    static SmemOnce once_bf, once_h;
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return cudaErrorInvalidDevice;
     const long long ntiles = static_cast<long long>(p.Tp / kPrepTok) * p.H * p.B;
     dim3 grid(static_cast<unsigned>(ntiles < 2LL * sms ? ntiles : 2LL * sms));
     if (in == InType::BF16) {
-        if (!attr_bf) {
-            cudaError_t e = cudaFuncSetAttribute(gdn_prep_tma_kernel<__nv_bfloat16>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kPrepSmem);
-            if (e != cudaSuccess) return e;
-            attr_bf = true;
-        }
+        cudaError_t e = raise_smem_once(once_bf, gdn_prep_tma_kernel<__nv_bfloat16>, static_cast<int>(kPrepSmem));
+        if (e != cudaSuccess) return e;
         gdn_prep_tma_kernel<__nv_bfloat16><<<grid, 256, kPrepSmem, s>>>(p, tmq, tmk, tmv);
     } else {
-        if (!attr_h) {
-            cudaError_t e = cudaFuncSetAttribute(gdn_prep_tma_kernel<__half>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kPrepSmem);
-            if (e != cudaSuccess) return e;
-            attr_h = true;
-        }
+        cudaError_t e = raise_smem_once(once_h, gdn_prep_tma_kernel<__half>, static_cast<int>(kPrepSmem));
+        if (e != cudaSuccess) return e;
         gdn_prep_tma_kernel<__half><<<grid, 256, kPrepSmem, s>>>(p, tmq, tmk, tmv);
     }
     return cudaGetLastError();

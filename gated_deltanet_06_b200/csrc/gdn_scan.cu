@@ -818,28 +818,21 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-template <typename K>
-cudaError_t set_smem(K kernel, uint32_t bytes, bool &done) {
-    if (done) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
-    if (e == cudaSuccess) done = true;
-    return e;
-}
 
 }  // namespace
 
 cudaError_t launch_transfer(const ScanParams &p, const CUtensorMap &tmW, const CUtensorMap &tmKt,
                             const CUtensorMap &tmU, cudaStream_t s, bool pdl) {
-    static bool attr = false;
-    cudaError_t e = set_smem(gdn_transfer_kernel, ta::SMEM_BYTES, attr);
+    static SmemOnce once;
+    cudaError_t e = raise_smem_once(once, gdn_transfer_kernel, static_cast<int>(ta::SMEM_BYTES));
     if (e != cudaSuccess) return e;
     dim3 grid(p.NS - 1, p.H, p.B);
     return launch_k(gdn_transfer_kernel, grid, dim3(288), ta::SMEM_BYTES, s, pdl, p, tmW, tmKt, tmU);
 }
 
 cudaError_t launch_combine(const ScanParams &p, cudaStream_t s, bool pdl) {
-    static bool attr = false;
-    cudaError_t e = set_smem(gdn_combine_kernel, cb::SMEM_BYTES, attr);
+    static SmemOnce once;
+    cudaError_t e = raise_smem_once(once, gdn_combine_kernel, static_cast<int>(cb::SMEM_BYTES));
     if (e != cudaSuccess) return e;
     dim3 grid(8, p.H, p.B);
     return launch_k(gdn_combine_kernel, grid, dim3(256), cb::SMEM_BYTES, s, pdl, p);
@@ -850,14 +843,14 @@ cudaError_t launch_scan_out(const ScanParams &p, InType zt, const CUtensorMap &t
                             const CUtensorMap &tmU, const CUtensorMap &tmZ, cudaStream_t s, bool pdl) {
     dim3 grid(p.NS, p.H, p.B);
     if (zt == InType::F16) {
-        static bool attr = false;
-        cudaError_t e = set_smem(gdn_scan_out_kernel<__half>, tc::SMEM_BYTES, attr);
+        static SmemOnce once;
+        cudaError_t e = raise_smem_once(once, gdn_scan_out_kernel<__half>, static_cast<int>(tc::SMEM_BYTES));
         if (e != cudaSuccess) return e;
         return launch_k(gdn_scan_out_kernel<__half>, grid, dim3(tc::kScanThreads), tc::SMEM_BYTES, s, pdl, p, tmW,
                         tmQt, tmKt, tmAqk, tmAqkH, tmU, tmZ);
     }
-    static bool attr = false;
-    cudaError_t e = set_smem(gdn_scan_out_kernel<__nv_bfloat16>, tc::SMEM_BYTES, attr);
+    static SmemOnce once;
+    cudaError_t e = raise_smem_once(once, gdn_scan_out_kernel<__nv_bfloat16>, static_cast<int>(tc::SMEM_BYTES));
     if (e != cudaSuccess) return e;
     return launch_k(gdn_scan_out_kernel<__nv_bfloat16>, grid, dim3(tc::kScanThreads), tc::SMEM_BYTES, s, pdl, p, tmW,
                     tmQt, tmKt, tmAqk, tmAqkH, tmU, tmZ);
