@@ -130,3 +130,123 @@ def segment_start_states(kh, vh, log_alpha, beta, C=128, Ls=2):
         St = zloc[j][:, d:] @ St + zloc[j][:, :d]
         starts.append(St)
     return starts
+
+
+def chunk_core_backward(qh, kh, vh, log_alpha, beta, do, C=64):
+    """Gradients of the recurrence (step 4) by the block algebra above, for
+    L with dL/do = do: returns dq^ (unscaled q^), dk^, dv^, d log alpha and
+    dbeta, all [B,T,H,...] fp64.  The design of a blocked backward: per
+    block, last block first, carrying dS = dL/dS at the block's end:
+
+      O   = diag(e^G) Q S0^T + P Delta,  P = (M o e^(G_r-G_i) o Q K^T)
+      S_C = e^(G_C) S0 + Delta^T Kd,     Kd = diag(e^(G_C-G)) K
+      Delta = U - W S0^T,  W = T diag(beta e^G) K,  U = T diag(beta) V,
+      T = (I + L)^-1,      L = tril_strict(beta_r e^(G_r-G_j) K K^T)
+
+    taken back in reverse order (dT to dL through dL = -T^T dT T^T), with
+    every e^G factor's gradient collected into dG and d log alpha the
+    reverse cumulative sum of dG."""
+    B, T, H, dk = qh.shape
+    dv = vh.shape[-1]
+    nc = -(-T // C)
+    Tp = nc * C
+    scale = 1.0 / np.sqrt(dk)
+    out = {n: np.zeros(s) for n, s in (("dq", qh.shape), ("dk", kh.shape), ("dv", vh.shape),
+                                       ("dla", log_alpha.shape), ("dbeta", beta.shape))}
+    strict = np.tril(np.ones((C, C)), -1)
+    incl = np.tril(np.ones((C, C)))
+    I = np.eye(C)
+    for b in range(B):
+        for h in range(H):
+            def pad(x):
+                o_ = np.zeros((Tp,) + x.shape[1:])
+                o_[:T] = x
+                return o_
+            Q = pad(qh[b, :, h]) * scale
+            K, V = pad(kh[b, :, h]), pad(vh[b, :, h])
+            la, be, dO = pad(log_alpha[b, :, h]), pad(beta[b, :, h]), pad(do[b, :, h])
+
+            def block(c, S0):
+                sl = slice(c * C, (c + 1) * C)
+                G = np.cumsum(la[sl])
+                Dm = np.minimum(G[:, None] - G[None, :], 0.0)
+                f = dict(sl=sl, G=G, E=np.exp(G), bc=be[sl], Kc=K[sl], Vc=V[sl], Qc=Q[sl], dOc=dO[sl])
+                f["Gam"], f["Gs"] = incl * np.exp(Dm), strict * np.exp(Dm)
+                f["A"] = f["Kc"] @ f["Kc"].T
+                f["L"] = f["Gs"] * f["bc"][:, None] * f["A"]
+                f["Tm"] = np.linalg.inv(I + f["L"])
+                f["Kb"] = (f["bc"] * f["E"])[:, None] * f["Kc"]
+                f["Vb"] = f["bc"][:, None] * f["Vc"]
+                f["W"], f["U"] = f["Tm"] @ f["Kb"], f["Tm"] @ f["Vb"]
+                f["Delta"] = f["U"] - f["W"] @ S0.T
+                f["P"] = f["Gam"] * (f["Qc"] @ f["Kc"].T)
+                f["Kd"] = np.exp(G[-1] - G)[:, None] * f["Kc"]
+                return f
+
+            S = np.zeros((dv, dk))
+            starts = []
+            for c in range(nc):
+                starts.append(S)
+                f = block(c, S)
+                S = np.exp(f["G"][-1]) * S + f["Delta"].T @ f["Kd"]
+            dS = np.zeros((dv, dk))
+            for c in range(nc - 1, -1, -1):
+                S0 = starts[c]
+                f = block(c, S0)
+                G, E, bc, Kc, Vc, Qc, dOc = f["G"], f["E"], f["bc"], f["Kc"], f["Vc"], f["Qc"], f["dOc"]
+                Tm, W, Delta, P, Kd, L, A, Gs, Gam = (f[n] for n in ("Tm", "W", "Delta", "P", "Kd", "L", "A", "Gs", "Gam"))
+                gC = G[-1]
+                dG, dE, dgC = np.zeros(C), np.zeros(C), 0.0
+                dbeta = np.zeros(C)
+                # O = diag(E) Q S0^T + P Delta
+                dS0 = dOc.T @ (E[:, None] * Qc)
+                dQ = E[:, None] * (dOc @ S0)
+                dE += (dOc * (Qc @ S0.T)).sum(1)
+                dP = (dOc @ Delta.T) * incl
+                dDelta = P.T @ dOc
+                dQK = dP * Gam
+                dQ += dQK @ Kc
+                dK = dQK.T @ Qc
+                dPP = dP * P
+                dG += dPP.sum(1) - dPP.sum(0)
+                # S_C = e^gC S0 + Delta^T Kd
+                dS0 += np.exp(gC) * dS
+                dgC += np.exp(gC) * float((dS * S0).sum())
+                dDelta += Kd @ dS.T
+                dKd = Delta @ dS
+                dK += np.exp(gC - G)[:, None] * dKd
+                t = (dKd * Kd).sum(1)
+                dgC += float(t.sum())
+                dG -= t
+                # Delta = U - W S0^T
+                dU, dW = dDelta, -dDelta @ S0
+                dS0 -= dDelta.T @ W
+                # W = T Kb, U = T Vb
+                dT = dW @ f["Kb"].T + dU @ f["Vb"].T
+                dKb, dVb = Tm.T @ dW, Tm.T @ dU
+                dK += (bc * E)[:, None] * dKb
+                tk = (dKb * Kc).sum(1)
+                dbeta += E * tk
+                dE += bc * tk
+                dV = bc[:, None] * dVb
+                dbeta += (dVb * Vc).sum(1)
+                # T = (I + L)^-1;  L = Gs beta_r A
+                dL = -(Tm.T @ dT @ Tm.T) * strict
+                dA = dL * Gs * bc[:, None]
+                dK += (dA + dA.T) @ Kc
+                dbeta += (dL * Gs * A).sum(1)
+                dLL = dL * L
+                dG += dLL.sum(1) - dLL.sum(0)
+                # E = e^G, gC = G_{C-1}, G = cumsum(log alpha)
+                dG += E * dE
+                dG[-1] += dgC
+                dla = np.cumsum(dG[::-1])[::-1]
+                rows = min(C, T - c * C)
+                r0 = c * C
+                out["dq"][b, r0:r0 + rows, h] = dQ[:rows] * scale
+                out["dk"][b, r0:r0 + rows, h] = dK[:rows]
+                out["dv"][b, r0:r0 + rows, h] = dV[:rows]
+                out["dla"][b, r0:r0 + rows, h] = dla[:rows]
+                out["dbeta"][b, r0:r0 + rows, h] = dbeta[:rows]
+                dS = dS0
+    return out

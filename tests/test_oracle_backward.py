@@ -83,3 +83,16 @@ def test_planted_mistake_fails_a_check(name):
     exec(compile(src.replace(old, new), mod.__name__, "exec"), mod.__dict__)
     inp, dy = _case(87, T=20, g_mean=-1.0)
     assert _fd_check(mod, inp, dy) != []
+
+
+@pytest.mark.parametrize("T,C", [(1, 64), (63, 64), (64, 64), (65, 64), (200, 64), (50, 16)])
+def test_blocked_backward_algebra_equals_the_oracle_backward(T, C):
+    # the design of a blocked (UT-form) backward, checked against the sequential backward in fp64
+    from chunk_model import chunk_core_backward
+    inp, dy = _case(90 + T, T=T, H=2, d=16, g_mean=-1.0)
+    _, tp = ob._tape(inp, ob.DEFAULT_L2_EPS, ob.DEFAULT_NORM_EPS)
+    ref = ob.vjp(inp, dy)
+    got = chunk_core_backward(tp["h_q"], tp["h_k"], tp["s_v"], tp["la"], tp["beta"], ref["do"], C=C)
+    for n, m in (("dq", "dqh"), ("dk", "dkh"), ("dv", "dvh"), ("dbeta", "dbeta")):
+        np.testing.assert_allclose(got[n], ref[m], rtol=1e-9, atol=1e-11, err_msg=n)
+    np.testing.assert_allclose(got["dla"], ref["dalpha"] * tp["alpha"], rtol=1e-9, atol=1e-11, err_msg="dla")
