@@ -374,6 +374,7 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
         sp.s0 = s0;
         sp.s_end = s_end;
         sp.rev = rev;
+        sp.debug = (c.flags & GDN_FLAG_DEBUG_CHECKS) ? 1 : 0;
         if (plan->NS > 1) {
             if (!mark() || launch_transfer(sp, tmW, tmKt, tmU, s, pdl) != cudaSuccess) return GDN_ERR_CUDA;
             if (!mark() || launch_combine(sp, s, pdl) != cudaSuccess) return GDN_ERR_CUDA;
@@ -398,6 +399,8 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
     OutParams op;
     op.o = o; op.z = in->z; op.tok_stride = plan->tok_stride; op.norm_w = in->norm_w; op.y = y;
     op.B = c.B; op.T = c.T; op.H = c.H; op.dv = c.d_v; op.eps = c.norm_eps;
+    op.debug = (c.flags & GDN_FLAG_DEBUG_CHECKS) ? 1 : 0;
+    op.status = status;
     if (!mark() || launch_output(op, in_type(c.in_dtype), in_type(c.out_dtype), s) != cudaSuccess)
         return GDN_ERR_CUDA;
     if (!mark()) return GDN_ERR_CUDA;

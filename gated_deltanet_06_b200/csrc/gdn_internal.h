@@ -111,6 +111,7 @@ struct ScanParams {
     const float *s0;         // [BH][128 (d_v)][128 (d_k)] state before token 0, or null (zero)
     float *s_end;            // [BH][128][128] state after token T-1, or null (not wanted)
     int rev;                 // reverse scan: block row t is z / y token T-1-t
+    int debug;               // check that every output value is finite (status word)
 };
 // pdl: launch with programmatic stream serialization (see launch_k).
 cudaError_t launch_transfer(const ScanParams &p, const CUtensorMap &tmW, const CUtensorMap &tmKt,
@@ -141,6 +142,8 @@ struct OutParams {
     void *y;  // [B][T][H][dv]
     int B, T, H, dv;
     float eps;
+    int debug;    // check that every output value is finite
+    int *status;
 };
 cudaError_t launch_output(const OutParams &p, InType zt, InType yt, cudaStream_t s);
 

@@ -561,6 +561,14 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
                         yf[1][j][0] = __uint_as_float(v[4 * gl + 2]) * rnB * w0 * silu_tc(fb.x);
                         yf[1][j][1] = __uint_as_float(v[4 * gl + 3]) * rnB * w1 * silu_tc(fb.y);
                     }
+                    if (p.debug) {  // every output of a live row must be finite
+                        bool bad = false;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            bad |= (liveA && !(isfinite(yf[0][j][0]) && isfinite(yf[0][j][1]))) ||
+                                   (liveB && !(isfinite(yf[1][j][0]) && isfinite(yf[1][j][1])));
+                        if (bad) atomicCAS(p.status, kStatusOk, kStatusCheck);
+                    }
                     if (p.out_kind == 1) {  // fp32: each lane stores its 8-byte pairs (a quad covers 32 bytes)
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {

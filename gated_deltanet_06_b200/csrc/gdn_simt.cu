@@ -110,7 +110,11 @@ __global__ void __launch_bounds__(256) gdn_output_kernel(const OutParams p) {
         const ZT *zr = z + tok * p.tok_stride + hh * DV + lane * PER;
         YT *yr = y + row * DV + lane * PER;
 #pragma unroll
-        for (int e = 0; e < PER; ++e) yr[e] = from_f<YT>(ov[e] * rn * w[e] * silu_f(to_f<ZT>(zr[e])));
+        for (int e = 0; e < PER; ++e) {
+            const float v = ov[e] * rn * w[e] * silu_f(to_f<ZT>(zr[e]));
+            if (p.debug && !isfinite(v)) atomicCAS(p.status, kStatusOk, kStatusCheck);
+            yr[e] = from_f<YT>(v);
+        }
     }
 }
 

@@ -75,7 +75,9 @@ typedef enum {
 } gdn_dtype;
 
 /* Plan flags. */
-#define GDN_FLAG_DEBUG_CHECKS 0x1u       /* device-side index/alignment checks into the status word */
+#define GDN_FLAG_DEBUG_CHECKS 0x1u       /* device-side check that every output value of the forward is
+                                            finite (a NaN or Inf in the inputs or the arithmetic):
+                                            GDN_ERR_DEVICE_CHECK in the status word otherwise */
 #define GDN_FLAG_FORCE_SIMT 0x2u         /* use the fp32 CUDA-core path even where the tensor path applies */
 #define GDN_FLAG_REVERSE 0x4u            /* reverse (anti-causal) scan: the operation above on the
                                             time-reversed sequence, outputs in the original order.

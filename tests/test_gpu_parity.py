@@ -217,3 +217,31 @@ def test_bounded_wait_timeout_reports_status_and_context_survives():
     assert plan.device_status(ws.data_ptr(), s) == gdn.ERR_TIMEOUT
     assert plan.device_status(ws.data_ptr(), s) == gdn.OK  # reading clears it
     check_parity(run_gdn(inp), _oracle(inp), "bf16", "bf16", "after timeout")
+
+
+@pytest.mark.parametrize("simt", [False, True])
+def test_debug_checks_report_non_finite_outputs(simt):
+    # GDN_FLAG_DEBUG_CHECKS: a NaN in z reaches one output value, which the device check reports
+    # through the status word; without the flag the status stays OK; a clean input passes the
+    # checks with the same output bit for bit
+    import torch
+    import gated_deltanet_06_b200 as gdn
+    dt = "f32" if simt else "bf16"
+    inp = gdn_inputs.make_inputs(1, 300, 2, 128, dt, 0.0, seed=27)
+    clean = torch_inputs(inp)
+    bad = dict(clean, z=clean["z"].clone())
+    bad["z"][0, 100, 1, 5] = float("nan")
+    code = gdn._torch_dtype_code(clean["q"].dtype)
+    s = torch.cuda.current_stream().cuda_stream
+    base = gdn.FLAG_FORCE_SIMT if simt else 0
+    outs = {}
+    for name, t in (("bad", bad), ("clean", clean)):
+        for flags in (gdn.FLAG_DEBUG_CHECKS, 0):
+            plan = gdn.Plan(1, 300, 2, 128, code, flags=base | flags)
+            ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device="cuda")
+            outs[(name, flags)] = gdn.forward(**t, plan=plan, workspace=ws)
+            st = plan.device_status(ws.data_ptr(), s)
+            expect = gdn.ERR_DEVICE_CHECK if (name == "bad" and flags) else gdn.OK
+            assert st == expect, (name, flags, gdn.status_string(st))
+    assert torch.isnan(outs[("bad", 0)].float()).sum().item() == 1
+    assert torch.equal(outs[("clean", gdn.FLAG_DEBUG_CHECKS)], outs[("clean", 0)])
