@@ -38,12 +38,11 @@ import gdn_inputs  # noqa: E402
 METRIC = "GDN fwd Mtokens/s at T=32760,H=12,d=128 bf16; % of tensor/HBM roofline"
 UNIT = "Mtokens/s"
 FLUSH_BYTES = 256 << 20
-KERNELS_TENSOR_SEG = ("prep", "chunk", "transfer", "combine", "scan")
-KERNELS_TENSOR_ONE = ("prep", "chunk", "scan")
+KERNELS_TENSOR_SEG = ("transfer", "combine", "out")
+KERNELS_TENSOR_ONE = ("out",)
 KERNELS_SIMT = ("prep", "recurrence", "output")
-KERNEL_SOURCES = {"prep": "gdn_prep.cu", "chunk": "gdn_chunk.cu", "transfer": "gdn_scan.cu",
-                  "combine": "gdn_scan.cu", "scan": "gdn_scan.cu", "recurrence": "gdn_simt.cu",
-                  "output": "gdn_simt.cu"}
+KERNEL_SOURCES = {"transfer": "gdn_fused.cu", "combine": "gdn_fused.cu", "out": "gdn_fused.cu",
+                  "prep": "gdn_prep.cu", "recurrence": "gdn_simt.cu", "output": "gdn_simt.cu"}
 
 
 def path_bytes_per_token_head(d, s_in, s_out):
@@ -57,19 +56,23 @@ def path_flops_per_token_head(d, C=64):
 
 
 def kernel_work_per_token_head(name, d, s_in, s_out):
-    """Algorithmic bytes and flops each kernel must move / do per (token, head)
-    on the tensor path (fp16 intermediates, fp32 o)."""
-    if name == "prep":      # q k v in; q^ k^ v^ fp16 out
-        return 3 * d * s_in + 3 * d * 2, 0
-    if name == "chunk":     # q^ k^ v^ + g b in; W U Qt Kt, 3/4 of Aqk, G beta log-alpha out; K K^T, Q K^T, W, U
-        return 3 * d * 2 + 8 + 4 * 128 * 2 + 96 * 2 + 12, 4 * 2 * 128 * d
-    if name == "transfer":  # W U Kt in; W [S|P]^T and Kt^T Delta with N = 2d
-        return 3 * 128 * 2, 2 * 2 * 128 * 2 * d
-    if name == "combine":   # per-segment states only (negligible per token)
+    """HBM bytes each kernel itself must move, and the tensor-core flops it issues, per (token,
+    head) of the token-heads it covers.  Tensor path (d = 128, 64-token blocks): the transfer pass
+    reads raw k, v and the gates and runs the state S and the transfer P side by side; the output
+    pass reads raw q, k, v, z and the gates and writes y; the combine moves only per-segment
+    states (negligible per token).  CUDA-core path: prep, recurrence and output kernels."""
+    C = 64
+    gram, wu = 2 * 128 * C * 128 // C, 2 * 2 * 128 * C * C // C          # [K;Q]K^T or KK^T; W^T and U^T
+    step = 2 * 128 * C * d // C + 2 * 128 * 128 * C // C                # Delta^T, state update
+    if name == "transfer":
+        return 2 * d * s_in + 8, gram + wu + 2 * step
+    if name == "out":          # Delta^T, O^T = N Qt^T, state, O^T += E Aqk^T
+        return 4 * d * s_in + 8 + d * s_out, gram + wu + step + 2 * 128 * C * d // C + 2 * 128 * C * C // C
+    if name == "combine":
         return 0, 0
-    if name == "scan":      # W U Qt Kt, 3/4 of Aqk, z in; y out; W S^T, Qt S^T, Kt^T Delta, Aqk Delta
-        return 4 * 128 * 2 + 96 * 2 + d * s_in + d * s_out, 4 * 2 * 128 * d
-    if name == "output":    # o fp32 + z in; y out
+    if name == "prep":         # q k v in; q^ k^ v^ fp32 out; gates
+        return 3 * d * s_in + 3 * d * 4 + 8 + 12, 0
+    if name == "output":       # o fp32 + z in; y out
         return d * 4 + d * s_in + d * s_out, 0
     if name == "recurrence":
         return 3 * d * 4 + 8 + d * 4, 6 * d * d
@@ -227,7 +230,7 @@ def reference_arm(args, w):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "d": w.d, "sample_T": T_s},
+            "config": dict(workload_config(w, args.out_dtype, 1), sample_T=T_s),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -249,6 +252,106 @@ def job_throughput(world, tokens_per_rank, ms_per_step):
     return world * tokens_per_rank / (ms_per_step / 1e3) / 1e6
 
 
+def out_name_of(w, out_dtype=None):
+    return out_dtype or ("bf16" if w.dtype == "bf16" else "f32")
+
+
+def workload_config(w, out_dtype, world):
+    """The JSON line's config object: the workload's name, shape, types and input recipe."""
+    return {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "d": w.d, "in_dtype": w.dtype,
+            "out_dtype": out_name_of(w, out_dtype), "g_mean": w.g_mean, "seed": w.seed,
+            "l2": "flushed before every step (256 MiB write, outside the timed interval)",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
+def path_roofline(w, s_in, s_out, ms_per_step, peaks):
+    """The method's whole-path roofline: 1288 B and 180,224 chunk flops per (token, head) at d = 128
+    bf16, t_roof = max(bytes / HBM bandwidth, flops / bf16 tensor peak)."""
+    units = w.B * w.T * w.H
+    pb = path_bytes_per_token_head(w.d, s_in, s_out)
+    pf = path_flops_per_token_head(w.d)
+    t_roof = max(pb * units / (peaks["hbm_gbs"] * 1e9), pf * units / (peaks["bf16_tflops"] * 1e12))
+    return {"bytes_per_token_head": pb, "flops_per_token_head": pf, "roofline_ms": t_roof * 1e3,
+            "roofline_Mtokens_s": w.B * w.T / t_roof / 1e6, "frac": (t_roof * 1e3) / ms_per_step,
+            "bound": "hbm" if pb * units / peaks["hbm_gbs"] >= pf * units / (peaks["bf16_tflops"] * 1e3) else "tensor"}
+
+
+def launch_units(name, w, plan):
+    """Token-heads one launch of a kernel covers: the transfer pass runs every segment but the last."""
+    if name == "transfer":
+        ns = plan.segments
+        nb = -(-w.T // 64)
+        ls = -(-nb // ns)
+        return w.B * w.H * min((ns - 1) * ls * 64, w.T)
+    return w.B * w.H * w.T
+
+
+def device_tensors(inp, w, dev):
+    import torch
+    tens = {}
+    for n in ("q", "k", "v", "z"):
+        if w.dtype == "bf16":
+            tens[n] = torch.from_numpy(inp[n + "_bits"].view(np.int16)).view(torch.bfloat16).to(dev)
+        else:
+            tens[n] = torch.from_numpy(inp[n]).to(dev)
+    for n in ("g", "b", "conv_q", "conv_k", "conv_v", "A_log", "dt_bias", "norm_w"):
+        tens[n] = torch.from_numpy(np.ascontiguousarray(inp[n], dtype=np.float32)).to(dev)
+    return tens
+
+
+def time_steps(run, flush, stream, steps):
+    """CUDA-event times (ms) of `steps` calls of run(), the L2 flushed before each, outside the interval."""
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for k in range(steps):
+        flush.zero_()
+        ev[k][0].record(stream)
+        run()
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def bench_other_config(w, dev, flush, stream, steps, cpu_budget_s):
+    """One of the other seeded workloads: the same step, flush and event timing as the headline, the
+    path roofline, and the oracle on a bounded sample as its baseline."""
+    import torch
+
+    import gated_deltanet_06_b200 as gdn
+    inp = gdn_inputs.workload_inputs(w)
+    tens = device_tensors(inp, w, dev)
+    del inp
+    in_code = gdn.DTYPE_BF16 if w.dtype == "bf16" else gdn.DTYPE_F32
+    out_name = out_name_of(w)
+    out_t = {"bf16": torch.bfloat16, "f32": torch.float32}[out_name]
+    plan = gdn.Plan(w.B, w.T, w.H, w.d, in_code, gdn.DTYPE_BF16 if out_name == "bf16" else gdn.DTYPE_F32)
+    ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=dev)
+    y = torch.empty((w.B, w.T, w.H, w.d), dtype=out_t, device=dev)
+    ptrs = gdn.tensor_ptrs(tens)
+    s = stream.cuda_stream
+    run = lambda: plan.forward_raw(ptrs, y.data_ptr(), ws.data_ptr(), s)  # noqa: E731
+    for _ in range(3):
+        run()
+    ms = time_steps(run, flush, stream, steps)
+    st = plan.device_status(ws.data_ptr(), s)
+    if st != gdn.OK:
+        raise SystemExit(f"device status, {w.name}: {gdn.status_string(st)}")
+    ms_step = statistics.mean(ms)
+    s_in = 2 if w.dtype == "bf16" else 4
+    s_out = 2 if out_name == "bf16" else 4
+    out = {"value": w.B * w.T / (ms_step / 1e3) / 1e6, "unit": UNIT, "ms_per_step": ms_step, "steps": steps,
+           "config": workload_config(w, None, 1), "tensor_path": plan.uses_tensor_path,
+           "segments": plan.segments, "launches_per_step": plan.launches,
+           "path_roofline": path_roofline(w, s_in, s_out, ms_step, load_peaks()),
+           "step_ms": {"min": min(ms), "median": statistics.median(ms), "max": max(ms)}}
+    del tens, ws, y
+    torch.cuda.empty_cache()
+    if cpu_budget_s > 0:
+        out["cpu_baseline"] = run_cpu_baseline(w, cpu_budget_s)
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -263,6 +366,7 @@ def main():
     ap.add_argument("--no-state", action="store_true", help="skip the carried-state timing")
     ap.add_argument("--no-reverse", action="store_true", help="skip the reverse-scan timing")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward timing")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other four seeded workloads")
     ap.add_argument("--load-seconds", type=float, default=1.5)
     args = ap.parse_args()
     w = gdn_inputs.by_name(args.workload)
@@ -287,14 +391,8 @@ def main():
     dev = torch.device("cuda", local)
 
     inp = gdn_inputs.workload_inputs(w, T=args.T)
-    tens = {}
-    for n in ("q", "k", "v", "z"):
-        if w.dtype == "bf16":
-            tens[n] = torch.from_numpy(inp[n + "_bits"].view(np.int16)).view(torch.bfloat16).to(dev)
-        else:
-            tens[n] = torch.from_numpy(inp[n]).to(dev)
-    for n in ("g", "b", "conv_q", "conv_k", "conv_v", "A_log", "dt_bias", "norm_w"):
-        tens[n] = torch.from_numpy(np.ascontiguousarray(inp[n], dtype=np.float32)).to(dev)
+    tens = device_tensors(inp, w, dev)
+    del inp
     in_code = gdn.DTYPE_BF16 if w.dtype == "bf16" else gdn.DTYPE_F32
     out_name = args.out_dtype or ("bf16" if w.dtype == "bf16" else "f32")
     out_code = {"bf16": gdn.DTYPE_BF16, "f16": gdn.DTYPE_F16, "f32": gdn.DTYPE_F32}[out_name]
@@ -514,6 +612,17 @@ def main():
                "one_stream": {"value": job_throughput(world, tokens, serial_ms), "ms_per_step": serial_ms}}
         del wss[1], stagings
 
+    # the other four seeded workloads (rank 0 alone, 1 GPU): same step, flush and event timing
+    configs = None
+    if world == 1 and not args.no_configs and not args.T:
+        configs = {}
+        del ws, y
+        torch.cuda.empty_cache()
+        for wo in gdn_inputs.WORKLOADS:
+            if wo.name != w.name:
+                configs[wo.name] = bench_other_config(wo, dev, flush, stream, max(5, min(args.steps, 20)),
+                                                      0.0 if args.no_cpu_baseline else 5.0)
+
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
@@ -522,48 +631,37 @@ def main():
     peaks = load_peaks()
     s_in = 2 if w.dtype == "bf16" else 4
     s_out = {"bf16": 2, "f16": 2, "f32": 4}[out_name]
-    units = w.B * w.T * w.H
+    tokens = w.B * w.T
+    path_roof = path_roofline(w, s_in, s_out, ms_per_step, peaks)
+    # the dominant kernel against the method's roofline (the per-unit figures of the whole path,
+    # 1288 B and 180,224 flops per token-head, times the token-heads the launch covers); the
+    # kernel's own HBM bytes beside them
     top = max(kern_ms, key=kern_ms.get)
-    kb, kf = kernel_work_per_token_head(top, w.d, s_in, s_out)
-    if top == "transfer":  # pass A covers every segment but the last
-        ns = plan.segments
-        ls = -(-(-(-w.T // 128)) // ns)
-        units = w.B * w.H * min((ns - 1) * ls * 128, w.T)
+    units = launch_units(top, w, plan)
+    pb, pf = path_roof["bytes_per_token_head"], path_roof["flops_per_token_head"]
     t_top = kern_ms[top] / 1e3
-    ach_gbs = kb * units / t_top / 1e9
-    ach_tfs = kf * units / t_top / 1e12
-    # a kernel is reported against the roof it is closer to
-    if kf and ach_tfs / peaks["bf16_tflops"] > ach_gbs / peaks["hbm_gbs"]:
-        roof = {"bound": "tensor", "achieved": ach_tfs, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": ach_tfs / peaks["bf16_tflops"]}
-    else:
-        roof = {"bound": "hbm", "achieved": ach_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": ach_gbs / peaks["hbm_gbs"]}
+    ach_gbs = pb * units / t_top / 1e9
+    ach_tfs = pf * units / t_top / 1e12
+    kb, kf = kernel_work_per_token_head(top, w.d, s_in, s_out)
     traffic = ncu_traffic(top, w.name)
-    roof.update(kernel=top, traffic=traffic, peak_source=peaks["source"] + " (MEASURED_PEAKS.json)"
-                if peaks["source"] == "measured" else "fallback",
-                algorithmic_bytes_per_launch=kb * units, algorithmic_flops_per_launch=kf * units,
-                avg_launch_ms=kern_ms[top], units_per_launch=units)
-    units = w.B * w.T * w.H
-    pb = path_bytes_per_token_head(w.d, s_in, s_out)
-    pf = path_flops_per_token_head(w.d)
-    t_roof = max(pb * units / (peaks["hbm_gbs"] * 1e9), pf * units / (peaks["bf16_tflops"] * 1e12))
-    path_roof = {"bytes_per_token_head": pb, "flops_per_token_head": pf, "roofline_ms": t_roof * 1e3,
-                 "roofline_Mtokens_s": tokens / t_roof / 1e6, "frac": (t_roof * 1e3) / ms_per_step}
+    roof = {"bound": "hbm", "achieved": ach_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": ach_gbs / peaks["hbm_gbs"], "traffic": traffic,
+            "peak_source": ("measured (MEASURED_PEAKS.json)" if peaks["source"] == "measured" else "fallback"),
+            "kernel": top, "avg_launch_ms": kern_ms[top], "units_per_launch": units,
+            "algorithmic_bytes_per_launch": pb * units, "algorithmic_flops_per_launch": pf * units,
+            "tensor_frac": ach_tfs / peaks["bf16_tflops"], "kernel_bytes_per_launch": kb * units,
+            "kernel_mma_flops_per_launch": kf * units, "path_frac": path_roof["frac"]}
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         cpu = run_cpu_baseline(w)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f16-mma/f32", "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "d": w.d, "in_dtype": w.dtype,
-                       "out_dtype": out_name, "g_mean": w.g_mean, "seed": w.seed,
-                       "l2": "flushed before every step (256 MiB write, outside the timed interval)",
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "vs_baseline": None, "dtype": "f16-mma/f32" if plan.uses_tensor_path else "f32", "data": "synthetic",
+            "config": workload_config(w, args.out_dtype, world),
             "roofline": roof, "path_roofline": path_roof, "kernels_ms": kern_ms,
             "segments": plan.segments, "cpu_baseline": cpu, "e2e": e2e, "state_io": state_io,
-            "reverse": reverse, "backward": bwd,
+            "reverse": reverse, "backward": bwd, "configs": configs,
             "clocks": clocks, "gpu_launches": L * args.steps,
             "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms), "max": max(step_ms)},
             "other_gpu_processes": None if others_before is None or others_after is None

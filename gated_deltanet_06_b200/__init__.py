@@ -202,8 +202,7 @@ class Plan:
         _check(_lib.gdn_forward_host(self._h, ctypes.byref(ins), y_host, staging, workspace, stream),
                "gdn_forward_host")
 
-    WS_FIELDS = ("status", "qh", "kh", "vh", "G", "beta", "log_alpha", "W", "U", "Qt", "Kt", "Aqk", "o", "Zloc",
-                 "Sstart")
+    WS_FIELDS = ("status", "qh", "kh", "vh", "G", "beta", "log_alpha", "o", "seg_states", "seg_start")
 
     def workspace_offsets(self) -> dict:
         arr = (ctypes.c_size_t * len(self.WS_FIELDS))()

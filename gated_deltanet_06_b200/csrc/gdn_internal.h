@@ -68,58 +68,31 @@ struct PrepParams {
     int rev;                       // reverse scan: internal token t is input token T-1-t
 };
 cudaError_t launch_prep(const PrepParams &p, InType in, bool out_f16, cudaStream_t s);
-// Tensor path (16-bit inputs, d = 128): raw tiles staged by TMA through the
-// 3-D maps tmq/tmk/tmv over [B][T][H*d] (box {64, 131, 1}).
-cudaError_t launch_prep_tma(const PrepParams &p, InType in, const CUtensorMap &tmq, const CUtensorMap &tmk,
-                            const CUtensorMap &tmv, cudaStream_t s);
-
-// Intra-block UT transform on tensor cores (d = 128, fp16 operands).  It
-// also evaluates the gates of its block from g, b (and writes G, beta, log
-// alpha for the scan and the stage tests).
-struct ChunkParams {
-    const float *g, *bg;            // [B][T][H]
-    const float *A_log, *dt_bias;   // [H]
-    float *G, *beta, *log_alpha;    // [BH][Tp]
-    int T, H;
-    __half *W, *U, *Qt, *Kt, *Aqk;  // [BH][Tp][128]
-    int BH, Tp, NB;
+// Tensor path (16-bit inputs, d = 128): the fused transfer and output passes over
+// segments of Ls blocks of 64 tokens, and the combine of the segment states.
+struct FusedParams {
+    const float *g, *bg;                      // [B][T][H]
+    const float *conv_q, *conv_k, *conv_v;    // [H*128][4]
+    const float *A_log, *dt_bias, *norm_w;    // [H], [H], [128]
+    void *y;                                  // [B][T][H][128], out_kind
+    float *SP;                                // [B*H][NS][2][128][128]: S_loc, P of each segment (transfer pass)
+    float *SS;                                // [B*H][NS][128][128]: S at each segment start, rows d_v (combine)
+    const float *s0;                          // [B*H][128 (d_v)][128 (d_k)] state before token 0, or null (zero)
+    float *s_end;                             // [B*H][128][128] state after token T-1, or null
+    int B, T, H, NB, NS, Ls;                  // NB = ceil(T / 64) blocks, NS segments of Ls blocks
+    float l2_eps, q_scale, eps;
+    int rev;                                  // reverse scan: internal token t is input token T-1-t
+    int out_kind;                             // y: 0 bf16, 1 f32, 2 f16
+    int debug;                                // device-side checks (status word)
+    int test_timeout;                         // test hook: one wait that runs out mid-pipeline
     int *status;
     unsigned long long wait_limit_ns;
-    int rev;                        // reverse scan: block row t holds the gates of input token T-1-t
 };
-cudaError_t launch_chunk(const ChunkParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
-                         const CUtensorMap &tmQ, const CUtensorMap &tmW, const CUtensorMap &tmU,
-                         const CUtensorMap &tmQt, const CUtensorMap &tmAqk, const CUtensorMap &tmAqkH,
-                         cudaStream_t s, bool pdl);  // Kt is written with plain coalesced stores
-
-// Inter-block state scan on tensor cores (d = 128), parallel over segments of
-// Ls blocks: pass A (transfer), combine, pass C (outputs + fused output step).
-struct ScanParams {
-    const float *G;          // [BH][Tp]
-    float *Zloc;             // [BH][NS][128][256]: S_loc^T | P^T per segment (pass A)
-    float *Sstart;           // [BH][NS][128][128]: S^T at each segment start (combine)
-    const void *z;           // [B][T][H][128], token stride tok_stride
-    long long tok_stride;
-    const float *norm_w;     // [128]
-    void *y;                 // [B][T][H][128]
-    int out_kind;            // 0 bf16, 1 f32, 2 f16
-    float eps;
-    int B, T, H, Tp, NB, NS, Ls;
-    int *status;
-    unsigned long long wait_limit_ns;
-    int test_wait_timeout;
-    const float *s0;         // [BH][128 (d_v)][128 (d_k)] state before token 0, or null (zero)
-    float *s_end;            // [BH][128][128] state after token T-1, or null (not wanted)
-    int rev;                 // reverse scan: block row t is z / y token T-1-t
-    int debug;               // check that every output value is finite (status word)
-};
-// pdl: launch with programmatic stream serialization (see launch_k).
-cudaError_t launch_transfer(const ScanParams &p, const CUtensorMap &tmW, const CUtensorMap &tmKt,
-                            const CUtensorMap &tmU, cudaStream_t s, bool pdl);
-cudaError_t launch_combine(const ScanParams &p, cudaStream_t s, bool pdl);
-cudaError_t launch_scan_out(const ScanParams &p, InType zt, const CUtensorMap &tmW, const CUtensorMap &tmQt,
-                            const CUtensorMap &tmKt, const CUtensorMap &tmAqk, const CUtensorMap &tmAqkH,
-                            const CUtensorMap &tmU, const CUtensorMap &tmZ, cudaStream_t s, bool pdl);
+// maps: raw q, k, v [B][T][H*128] boxes {128, 67, 1}; z {128, 64, 1}; y {128, 64, 1} (16-bit
+// outputs); y tail {128, T - 64 (NB - 1), 1} (the reverse scan's ragged block).
+cudaError_t launch_fused_transfer(const FusedParams &p, InType in, const CUtensorMap *maps, cudaStream_t s, bool pdl);
+cudaError_t launch_fused_combine(const FusedParams &p, cudaStream_t s, bool pdl);
+cudaError_t launch_fused_output(const FusedParams &p, InType in, const CUtensorMap *maps, cudaStream_t s, bool pdl);
 
 // Sequential fp32 recurrence on CUDA cores (fp32 inputs or d = 64).
 struct RecurParams {

@@ -39,26 +39,50 @@ def test_headline_roofline_time():
 
 
 @pytest.mark.parametrize("name,expected_bytes", [
-    ("prep", 3 * 128 * 2 + 3 * 128 * 2),                      # q k v bf16 in, q^ k^ v^ fp16 out
-    ("chunk", 3 * 256 + 8 + 4 * 256 + 192 + 12),              # q^ k^ v^, g b; W U Qt Kt, 3/4 Aqk, G beta log-alpha
-    ("transfer", 3 * 256),                                    # W U Kt
-    ("scan", 4 * 256 + 192 + 256 + 256),                      # W U Qt Kt, 3/4 Aqk, z; y
+    ("transfer", 2 * 128 * 2 + 8),          # raw k, v bf16 in; g, b fp32 in
+    ("out", 4 * 128 * 2 + 8 + 128 * 2),     # raw q, k, v, z bf16 in; g, b fp32 in; y bf16 out
+    ("combine", 0),                         # per-segment states only
 ])
 def test_kernel_bytes(name, expected_bytes):
     assert bench.kernel_work_per_token_head(name, 128, 2, 2)[0] == expected_bytes
 
 
-def test_chunk_launch_bytes_at_the_headline():
+def test_kernel_flops_per_64_token_block():
+    C, d = 64, 128
+    gram = 2 * 128 * C * d          # [K; Q] K^T: M = 128 stacked rows, N = C, K = d
+    wu = 2 * (2 * 128 * C * C)      # W^T = K^T T_w^T and U^T = V^T T_u^T: M = d, N = K = C
+    delta = 2 * 128 * C * d         # Delta^T = U^T + N W^T: M = d_v, N = C, K = d_k
+    state = 2 * 128 * 128 * C       # N += E Kt: M = d_v, N = d_k, K = C
+    o1, o2 = 2 * 128 * C * d, 2 * 128 * C * C
+    assert bench.kernel_work_per_token_head("out", d, 2, 2)[1] * C == gram + wu + delta + state + o1 + o2
+    assert bench.kernel_work_per_token_head("transfer", d, 2, 2)[1] * C == gram + wu + 2 * (delta + state)
+    # the output pass's products are exactly the method's chunk count per token-head
+    assert bench.kernel_work_per_token_head("out", d, 2, 2)[1] == bench.path_flops_per_token_head(d)
+
+
+def test_dominant_launch_units():
+    class P:
+        segments = 12
     w = gdn_inputs.HEADLINE
-    kb, kf = bench.kernel_work_per_token_head("chunk", w.d, 2, 2)
-    assert kb * w.B * w.T * w.H == 787812480
-    assert kf == 4 * 2 * 128 * 128  # K K^T, Q K^T, T V~, T K~ as 128-row tiles
+    assert bench.launch_units("out", w, P) == w.B * w.H * w.T
+    nb = -(-w.T // 64)
+    ls = -(-nb // 12)
+    assert bench.launch_units("transfer", w, P) == w.H * 11 * ls * 64
 
 
-def test_traffic_is_dropped_when_the_kernel_source_changed(monkeypatch):
-    real = bench.kernel_source_sha("chunk")
-    monkeypatch.setattr(bench, "kernel_source_sha", lambda name: "0" * 16 if name == "chunk" else real)
-    assert bench.ncu_traffic("chunk", "wan21_480x832_81f") is None
+def test_path_roofline_fraction():
+    w = gdn_inputs.HEADLINE
+    p = bench.load_peaks()
+    r = bench.path_roofline(w, 2, 2, 0.5, p)
+    assert r["bound"] == "hbm"
+    assert r["frac"] == pytest.approx(r["roofline_ms"] / 0.5)
+    assert r["roofline_Mtokens_s"] == pytest.approx(w.B * w.T / (r["roofline_ms"] / 1e3) / 1e6)
+
+
+def test_traffic_is_dropped_when_the_kernel_source_changed(monkeypatch, tmp_path):
+    real = bench.kernel_source_sha("out")
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda name: "0" * 16 if name == "out" else real)
+    assert bench.ncu_traffic("out", "wan21_480x832_81f") is None
 
 
 def test_sample_text():
