@@ -50,6 +50,9 @@
 namespace gdn {
 namespace {
 
+// timeline stamp k of block i (compiled in only for tuning builds, see GDN_TRACE)
+#define FTRACE(i, k) GDN_TRACE_AT((kOut ? 0 : 4096) + (i) * 32 + (k))
+
 constexpr int kC = 64;                      // tokens per block
 constexpr int kRawRows = kC + 3;            // conv window: 3 tokens of history
 constexpr uint32_t kRawBytes = kRawRows * 256;  // one raw box: 67 tokens x 128 channels x 16 bit
@@ -57,80 +60,90 @@ constexpr int kThreads = 544;               // 17 warps
 enum { W_MMA = 0, W_PREP = 1, W_UT = 5, W_CH = 9, W_X = 13 };  // first warp of each role
 enum { NB_PREP = 1, NB_UT = 2, NB_X = 3 };                      // named barriers (128 threads)
 
-// Shared-memory map (offsets from a 1024-byte aligned base).
+// Shared-memory map (offsets from a 1024-byte aligned base).  The KQ, W^T, Aqk, T and TW
+// tiles come in two slots (block i uses slot i & 1), so that the next block's UT transform
+// runs while the current block's state step reads its operands.
 template <bool kOut>
 struct Lay;
 template <>
 struct Lay<true> {  // output pass
-    static constexpr uint32_t KQ = 0;        // 2 slots x [128 rows: K^ (0-63) -> Kt, Q^ (64-127) -> Qt][128] fp16
-    static constexpr uint32_t WT = 65536;    // 2 slots x W^T [128 d_k][64 tokens] fp16
-    static constexpr uint32_t AQK = 98304;   // 2 slots x Aqk [64][64] fp16
-    static constexpr uint32_t V = 114688;    // V^ [64][128] fp16
-    static constexpr uint32_t T = 131072;    // L -> T -> T diag(beta) [64][64] fp16
-    static constexpr uint32_t TW = 139264;   // T diag(beta e^G) [64][64] fp16
-    static constexpr uint32_t RAW = 147456;  // raw q, k, v boxes
-    static constexpr uint32_t Z = 198912;    // z box [64][128] 16-bit, y written over it
-    static constexpr uint32_t MISC = 215296;
-    static constexpr int NRAW = 3;
+    static constexpr uint32_t KQ = 0;        // 2 x [128 rows: K' (0-63) -> Kt, Q' (64-127) -> Qt][128] fp16
+    static constexpr uint32_t WT = 65536;    // 2 x W^T [128 d_k][64 tokens] fp16
+    static constexpr uint32_t AQK = 98304;   // 2 x Aqk [64][64] fp16
+    static constexpr uint32_t V = 114688;    // V' [64][128] fp16
+    static constexpr uint32_t T = 131072;    // 2 x (L -> T -> T diag(beta)) [64][64] fp16
+    static constexpr uint32_t TW = 147456;   // 2 x T diag(beta e^G / |k'|) [64][64] fp16
+    static constexpr uint32_t RAW = 163840;  // 2 raw-box slots; the block's k, q, v boxes rotate through them
+    static constexpr uint32_t Z = 198144;    // z box [64][128] 16-bit, y written over it
+    static constexpr uint32_t MISC = 214528;
+    static constexpr int NRAWSLOT = 2, NTENS = 3;
 };
 template <>
 struct Lay<false> {  // transfer pass
-    static constexpr uint32_t KQ = 0;        // 2 slots x [128 rows: K^ (0-63) -> Kt, V^ (64-127)][128] fp16
+    static constexpr uint32_t KQ = 0;        // 2 x [128 rows: K' (0-63) -> Kt, V' (64-127)][128] fp16
     static constexpr uint32_t WT = 65536;
     static constexpr uint32_t N16S = 98304;  // fp16 copy of -S, A operand [128][128] K-major
     static constexpr uint32_t N16P = 131072; // fp16 copy of -P
     static constexpr uint32_t T = 163840;
-    static constexpr uint32_t TW = 172032;
-    static constexpr uint32_t RAW = 180224;  // raw k, v boxes
-    static constexpr uint32_t MISC = 214528;
-    static constexpr int NRAW = 2;
+    static constexpr uint32_t TW = 180224;
+    static constexpr uint32_t RAW = 196608;  // one raw-box slot: the block's k, then v
+    static constexpr uint32_t MISC = 213760;
+    static constexpr int NRAWSLOT = 1, NTENS = 2;
 };
 // MISC sub-layout
-constexpr uint32_t M_GATE = 0;      // 2 slots x {G, beta, ec, beta e^G} x 64 fp32
-constexpr uint32_t M_LDIAG = 2048;  // the diagonal 16x16 blocks of L, fp32 [4][16][16]
-constexpr uint32_t M_RED = 6144;    // output step: per-token partial sums of squares [64][4]
-constexpr uint32_t M_RN = 7168;     // per-token 1/rms [64]
-constexpr uint32_t M_NW = 7424;     // norm weight [128]
-constexpr uint32_t M_WTOT = 7936;   // gate scan: warp totals
-constexpr uint32_t M_BAR = 7968;
-constexpr int NBAR = 26;
+constexpr uint32_t M_GATE = 0;      // 2 slots x {G, beta, ec, beta e^G / |k'|} x 64 fp32
+constexpr uint32_t M_INVN = 2048;   // 2 slots x {1/|k'|, 1/(sqrt(d) |q'|)} x 64 fp32 (prep)
+constexpr uint32_t M_LDIAG = 3072;  // the diagonal 16x16 blocks of L, fp32 [4][16][16]
+constexpr uint32_t M_RED = 7168;    // output step: per-token partial sums of squares [64][4]
+constexpr uint32_t M_RN = 8192;     // per-token 1/rms [64]
+constexpr uint32_t M_NW = 8448;     // norm weight [128]
+constexpr uint32_t M_WTOT = 8960;   // gate scan: warp totals
+constexpr uint32_t M_CONV = 8992;   // conv taps of the CTA's head: [tensor][j][cg] float4, channel 8 cg + j
+constexpr uint32_t M_BAR = M_CONV + 3 * 128 * 16;
+constexpr int NBAR = 28;
 constexpr uint32_t M_SLOT = M_BAR + NBAR * 8;  // TMEM base address, abort flag
 constexpr uint32_t M_SIZE = M_SLOT + 16;
 template <bool kOut>
 constexpr uint32_t smem_bytes() { return Lay<kOut>::MISC + M_SIZE + 1024; }
 static_assert(smem_bytes<true>() <= 227 * 1024 && smem_bytes<false>() <= 227 * 1024, "shared memory");
+static_assert(Lay<true>::RAW + 2 * kRawBytes <= Lay<true>::Z && Lay<true>::Z + 16384 <= Lay<true>::MISC, "layout");
+static_assert(Lay<false>::RAW + kRawBytes <= Lay<false>::MISC, "layout");
 
+// mbarriers; "2:" = one per slot (block i uses slot i & 1), so that a waiter that runs a block
+// ahead or behind never mistakes one block's phase for another's
 enum {
-    B_RAW = 0,         // 3: raw box of tensor w landed
-    B_PREP = 3,        // 2: prepared tiles of slot s complete (4 prep warps)
-    B_FREE = 5,        // 2: every MMA that reads slot s is complete (commit)
-    B_VFREE = 7,       // U^T read the V tile (commit)
+    B_RAW = 0,         // 2: raw-box slot landed (TMA)
+    B_PREP = 2,        // 2: K', Q' tiles (transfer pass: K', V') and their inverse norms complete (4 prep warps)
+    B_PREPV = 4,       // output pass: the V' tile is complete (4 prep warps)
+    B_FREE = 5,        // 2: every MMA that reads the slot's tiles is complete (commit)
+    B_VFREE = 7,       // U^T read the V' tile (commit)
     B_GRAM = 8,        // Gram complete (commit)
-    B_GATE = 9,        // 2: gates of slot s in shared memory (4 UT warps)
-    B_TREADY = 11,     // T diag(beta), T diag(beta e^G) tiles complete (4 UT warps)
-    B_WT = 12,         // W^T and U^T complete (commit)
-    B_UTD = 13,        // 2: W^T tile, Kt, Qt, Aqk of slot s complete (4 UT warps)
-    B_DELTA = 15,      // Delta^T (and the first half of O^T) complete (commit)
-    B_E16 = 16,        // fp16 Delta in TMEM, state decayed (state warps)
-    B_STATE = 17,      // state update complete (commit)
-    B_N16 = 18,        // fp16 state copy ready (state warps)
-    B_OFULL = 19,      // 2: O^T buffer complete (commit)
-    B_OFREE = 21,      // 2: O^T buffer read (4 output warps)
-    B_Z = 23,          // z box landed
-    B_TEST = 24,       // never completes (test hook)
-    B_DRAIN = 25       // teardown: every MMA issued so far is complete (commit)
+    B_GATE = 9,        // 2: gates of the slot in shared memory (4 UT warps)
+    B_TREADY = 11,     // 2: T tiles, Qt and Aqk of the slot complete (4 UT warps)
+    B_WT = 13,         // 2: W^T and U^T of the slot complete (commit)
+    B_UTD = 15,        // 2: W^T tile and Kt of the slot complete (4 state warps)
+    B_DELTA = 17,      // Delta^T (and the first half of O^T) complete (commit)
+    B_E16 = 18,        // fp16 Delta in TMEM (state warps)
+    B_STATE = 19,      // state update complete (commit)
+    B_N16 = 20,        // fp16 state copy ready, state decayed by the next block's decay (state warps)
+    B_OFULL = 21,      // 2: O^T buffer complete (commit)
+    B_OFREE = 23,      // 2: O^T buffer read (4 output warps)
+    B_Z = 25,          // z box landed
+    B_TEST = 26,       // never completes (test hook)
+    B_DRAIN = 27       // teardown: every MMA issued so far is complete (commit)
 };
 
-// TMEM columns (512 allocated)
+// TMEM columns (512 allocated).  The fp16 Delta (E16) is written over the first 32 columns of
+// the fp32 Delta^T it comes from.
 template <bool kOut>
 struct Tm;
 template <>
 struct Tm<true> {
-    static constexpr uint32_t N = 0, N16 = 128, UD = 192, E16 = 256, GW = 288, O = 352;  // O: 2 x 64
+    static constexpr uint32_t N = 0, N16 = 128, UD = 192, E16 = 192, GA = 256, GB = 320, O = 384;  // O: 2 x 64
 };
 template <>
 struct Tm<false> {
-    static constexpr uint32_t N = 0, NP = 128, UD = 256, UDP = 320, E16 = 384, E16P = 416, GW = 448;
+    static constexpr uint32_t N = 0, NP = 128, UD = 256, UDP = 320, E16 = 256, E16P = 320, GA = 384, GB = 448;
 };
 
 // 8 consecutive 16-bit inputs -> fp32
@@ -166,7 +179,7 @@ __device__ __forceinline__ void put8h(uint8_t *tile, int rows, int r, int chunk,
 }
 // Row r of a panel tile scaled in place by f, chunks [ch0, ch0 + nch).
 __device__ __forceinline__ void scale_row_chunks(uint8_t *tile, int rows, int r, int ch0, int nch, float f) {
-#pragma unroll 4
+#pragma unroll 2
     for (int c = ch0; c < ch0 + nch; ++c) {
         uint4 *pu = reinterpret_cast<uint4 *>(tile + tile_off(rows, r, c));
         const uint4 u = *pu;
@@ -306,6 +319,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *misc = sm + Ly::MISC;
     float *gate = reinterpret_cast<float *>(misc + M_GATE);
     float *ldiag = reinterpret_cast<float *>(misc + M_LDIAG);
+    float *invn = reinterpret_cast<float *>(misc + M_INVN);
+    float4 *convs = reinterpret_cast<float4 *>(misc + M_CONV);
     float *red = reinterpret_cast<float *>(misc + M_RED);
     float *rns = reinterpret_cast<float *>(misc + M_RN);
     float *nw = reinterpret_cast<float *>(misc + M_NW);
@@ -321,13 +336,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t lim = p.wait_limit_ns;
 
     if (tid == 0) {
-        const int pre = kOut ? 4 : 8;  // state-warp arrivals on E16 / N16
         for (int i = 0; i < NBAR; ++i) {
-            int cnt = 1;
-            if (i == B_PREP || i == B_PREP + 1 || i == B_GATE || i == B_GATE + 1 || i == B_TREADY || i == B_UTD ||
-                i == B_UTD + 1 || i == B_OFREE || i == B_OFREE + 1)
-                cnt = 4;
-            if (i == B_E16 || i == B_N16) cnt = pre;
+            int cnt = 1;  // TMA and tensor-core commits
+            if ((i >= B_PREP && i < B_FREE) || (i >= B_GATE && i < B_WT) || i == B_UTD || i == B_UTD + 1 ||
+                i == B_OFREE || i == B_OFREE + 1)
+                cnt = 4;  // one arrival per warp of a 4-warp group
+            if (i == B_E16 || i == B_N16) cnt = kOut ? 4 : 8;  // the state warps (and the transfer warps)
             mbar_init(&bars[i], cnt);
         }
         ab->flag = 0;
@@ -351,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ab->flag) goto teardown;
 
     if (warp == W_MMA) {
-        // ================================================================ MMA issue
+        // ================================================================ MMA issue (one thread)
         if (lane == 0) {
             bool issued = false;
             auto kq = [&](int s) { return sb + Ly::KQ + static_cast<uint32_t>(s) * 32768u; };
@@ -360,86 +374,110 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t id_mk64 = idesc_f16_f32(128, 64, true, false);    // W^T, U^T
             const uint32_t id_km64 = idesc_f16_f32(128, 64, false, true);    // Delta^T (B = W^T)
             const uint32_t id_km128 = idesc_f16_f32(128, 128, false, true);  // state (B = Kt)
-            auto gram = [&](int s) {
-#pragma unroll
+            // byte offset of K-step kk (16 elements) in a K-major tile whose 64-element panels are
+            // `panel` bytes apart
+            auto kmaj = [](int kk, uint32_t panel) { return static_cast<uint32_t>(kk >> 2) * panel + (kk & 3) * 32u; };
+            // the stacked Gram [K'; Q'] K'^T (transfer pass: [K'; V'] K'^T, lanes 64-127 unused) of block j
+            auto gram = [&](int j) {
+                const int s = j & 1;
+#pragma unroll 1
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t d = sdesc_sw128(kq(s) + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                    umma_f16(tmem + TM::GW, d, d, id_kk64, kk > 0);
+                    const uint64_t d = sdesc_sw128(kq(s) + kmaj(kk, 16384), 16, 1024);
+                    umma_f16(tmem + TM::GA, d, d, id_kk64, kk > 0);
                 }
                 umma_commit(&bars[B_GRAM]);
             };
-            auto wt_ut = [&](int s) {
-#pragma unroll
+            // W^T = K'^T (T diag(beta e^G / |k'|))^T and U^T = V'^T (T diag(beta))^T of block j
+            // (output pass: U^T once the V' tile is complete)
+            auto wt_ut = [&](int j) -> bool {
+                const int s = j & 1;
+                const uint32_t tt = sb + Ly::T + s * 8192u, tw = sb + Ly::TW + s * 8192u;
+#pragma unroll 1
                 for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(tmem + TM::GW, sdesc_sw128(kq(s) + kk * 2048, 16384, 1024),
-                             sdesc_sw128(sb + Ly::TW + kk * 32, 16, 1024), id_mk64, kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    uint64_t ad;
-                    if constexpr (kOut) ad = sdesc_sw128(sb + Lay<true>::V + kk * 2048, 8192, 1024);
-                    else ad = sdesc_sw128(kq(s) + 8192 + kk * 2048, 16384, 1024);
-                    umma_f16(tmem + TM::UD, ad, sdesc_sw128(sb + Ly::T + kk * 32, 16, 1024), id_mk64, kk > 0);
+                    umma_f16(tmem + TM::GB, sdesc_sw128(kq(s) + kk * 2048, 16384, 1024),
+                             sdesc_sw128(tw + kk * 32, 16, 1024), id_mk64, kk > 0);
+                if (kOut) {
+                    if (!mbar_wait(&bars[B_PREPV], j & 1, ab, p.status, lim)) return false;
+                    tc_fence_after();
                 }
-                umma_commit(&bars[B_WT]);
+#pragma unroll 1
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t ad = kOut ? sdesc_sw128(sb + Lay<true>::V + kk * 2048, 8192, 1024)
+                                             : sdesc_sw128(kq(s) + 8192 + kk * 2048, 16384, 1024);
+                    umma_f16(tmem + TM::UD, ad, sdesc_sw128(tt + kk * 32, 16, 1024), id_mk64, kk > 0);
+                }
+                umma_commit(&bars[B_WT + s]);
                 if (kOut) umma_commit(&bars[B_VFREE]);
+                return true;
             };
-            bool ok = mbar_wait(&bars[B_PREP], 0, ab, p.status, lim);
+            // The Gram of block j needs its prepared tiles and the Gram columns free: block j - 1's
+            // L and Aqk are out once its T tiles are (TREADY).  `gram_next` is the next block whose
+            // Gram is to be issued, `tready_seen` the last block whose TREADY this thread has waited for.
+            int gram_next = 0, tready_seen = -1;
+            auto try_gram = [&](bool block) -> bool {
+                while (gram_next < n && tready_seen >= gram_next - 1) {
+                    const int j = gram_next, s = j & 1;
+                    if (block) {
+                        if (!mbar_wait(&bars[B_PREP + s], (j >> 1) & 1, ab, p.status, lim)) return false;
+                    } else if (!mbar_try_wait(&bars[B_PREP + s], (j >> 1) & 1)) {
+                        return true;
+                    }
+                    tc_fence_after();
+                    gram(j);
+                    issued = true;
+                    if (j == 0) FTRACE(0, 5);
+                    ++gram_next;
+                    if (!block) break;
+                    block = false;
+                }
+                return true;
+            };
+            bool ok = try_gram(true);
+            ok = ok && mbar_wait(&bars[B_TREADY], 0, ab, p.status, lim);
             if (ok) {
+                tready_seen = 0;
                 tc_fence_after();
-                gram(0);
-                issued = true;
-                ok = mbar_wait(&bars[B_TREADY], 0, ab, p.status, lim);
-            }
-            if (ok) {
-                tc_fence_after();
-                wt_ut(0);
+                ok = wt_ut(0);
             }
             if (ok && p.test_timeout) {
                 // test hook: a wait on a barrier nothing arrives on, with tensor-core work in flight
                 mbar_wait(&bars[B_TEST], 0, ab, p.status, lim);
                 ok = false;
             }
+            ok = ok && try_gram(false);
             for (int i = 0; ok && i < n; ++i) {
                 const int s = i & 1;
+                FTRACE(i, 0);
                 ok = mbar_wait(&bars[B_UTD + s], (i >> 1) & 1, ab, p.status, lim) &&
                      mbar_wait(&bars[B_N16], i & 1, ab, p.status, lim) &&
                      (!kOut || i < 2 || mbar_wait(&bars[B_OFREE + s], ((i >> 1) - 1) & 1, ab, p.status, lim));
                 if (!ok) break;
+                FTRACE(i, 1);
                 tc_fence_after();
                 // Delta^T = U^T + N W^T (and the first half of O^T = -(S Qt^T))
-                if constexpr (kOut) {
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_f16_ts(tmem + TM::UD, tmem + Tm<true>::N16 + kk * 8,
-                                    sdesc_sw128(wtile(s) + kk * 2048, 8192, 1024), id_km64, 1);
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
+#pragma unroll 1
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t bd = sdesc_sw128(wtile(s) + kk * 2048, 8192, 1024);
+                    if constexpr (kOut) {
+                        umma_f16_ts(tmem + TM::UD, tmem + Tm<true>::N16 + kk * 8, bd, id_km64, 1);
                         umma_f16_ts(tmem + Tm<true>::O + s * 64, tmem + Tm<true>::N16 + kk * 8,
-                                    sdesc_sw128(kq(s) + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32, 16, 1024),
-                                    id_kk64, kk > 0);
-                } else {
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t ao = (kk >> 2) * 16384 + (kk & 3) * 32;
-                        const uint64_t bd = sdesc_sw128(wtile(s) + kk * 2048, 8192, 1024);
+                                    sdesc_sw128(kq(s) + 8192 + kmaj(kk, 16384), 16, 1024), id_kk64, kk > 0);
+                    } else {
+                        const uint32_t ao = kmaj(kk, 16384);
                         umma_f16(tmem + TM::UD, sdesc_sw128(sb + Lay<false>::N16S + ao, 16, 1024), bd, id_km64, 1);
                         umma_f16(tmem + Tm<false>::UDP, sdesc_sw128(sb + Lay<false>::N16P + ao, 16, 1024), bd, id_km64,
                                  kk > 0);
                     }
                 }
                 umma_commit(&bars[B_DELTA]);
-                // the next block's Gram, if its operands are ready already
-                bool gram_next = false;
-                if (i + 1 < n && mbar_try_wait(&bars[B_PREP + (s ^ 1)], ((i + 1) >> 1) & 1)) {
-                    tc_fence_after();
-                    gram(s ^ 1);
-                    gram_next = true;
-                }
-                ok = mbar_wait(&bars[B_E16], i & 1, ab, p.status, lim);
+                FTRACE(i, 2);
+                ok = try_gram(false);
+                ok = ok && mbar_wait(&bars[B_E16], i & 1, ab, p.status, lim);
                 if (!ok) break;
+                FTRACE(i, 3);
                 tc_fence_after();
                 // N += E16 Kt  (E16 = -Delta^T, fp16 in TMEM; Kt MN-major, N = d_k)
-#pragma unroll
+#pragma unroll 1
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint64_t bd = sdesc_sw128(kq(s) + kk * 2048, 16384, 1024);
                     umma_f16_ts(tmem + TM::N, tmem + TM::E16 + kk * 8, bd, id_km128, 1);
@@ -449,24 +487,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if constexpr (kOut) {
                     // O^T += E16 Aqk^T
                     const uint32_t aq = sb + Lay<true>::AQK + static_cast<uint32_t>(s) * 8192u;
-#pragma unroll
+#pragma unroll 1
                     for (int kk = 0; kk < 4; ++kk)
                         umma_f16_ts(tmem + Tm<true>::O + s * 64, tmem + TM::E16 + kk * 8,
                                     sdesc_sw128(aq + kk * 32, 16, 1024), id_kk64, 1);
                     umma_commit(&bars[B_OFULL + s]);
                 }
                 umma_commit(&bars[B_FREE + s]);
+                FTRACE(i, 4);
                 if (i + 1 < n) {
-                    if (!gram_next) {
-                        ok = mbar_wait(&bars[B_PREP + (s ^ 1)], ((i + 1) >> 1) & 1, ab, p.status, lim);
-                        if (!ok) break;
-                        tc_fence_after();
-                        gram(s ^ 1);
-                    }
-                    ok = mbar_wait(&bars[B_TREADY], (i + 1) & 1, ab, p.status, lim);
+                    // the next block's W^T and U^T (its Gram first, if it is still to be issued); U^T goes
+                    // to the Delta^T columns, whose fp16 Delta the state update above has read
+                    ok = (gram_next > i + 1 || try_gram(true)) &&
+                         mbar_wait(&bars[B_TREADY + (s ^ 1)], ((i + 1) >> 1) & 1, ab, p.status, lim);
                     if (!ok) break;
+                    tready_seen = i + 1;
+                    FTRACE(i, 6);
                     tc_fence_after();
-                    wt_ut(s ^ 1);
+                    ok = wt_ut(i + 1) && try_gram(false);
                 }
             }
             if (issued) {  // every tensor-core operation issued so far has completed
@@ -476,257 +514,292 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp < W_UT) {
         // ================================================================ prep
+        // conv4 + SiLU of the block's raw boxes into fp16 operand tiles.  q' and k' are stored as
+        // they are; the inverse norms 1/|k'| and 1/(sqrt(d_k) |q'|) of every token go to shared
+        // memory and are applied where the tiles are scaled or read next (L, Aqk, Qt, Kt, and the
+        // columns of T diag(beta e^G)), so that no per-token reduction sits between a token's
+        // conv and its store.  Thread (cg, rg) owns channels 8 cg .. 8 cg + 7 of tokens
+        // 8 rg .. 8 rg + 7.  The raw boxes are loads number l = NTENS i + w (tensor w of block i),
+        // through slot l % NRAWSLOT; load l + NRAWSLOT is issued once load l has been read.
         const int pt = tid - 32 * W_PREP;
         const int cg = pt & 15, rg = pt >> 4, rbeg = rg * 8;
-        const CUtensorMap *maps[3];
-        const float *convw[3];
-        if constexpr (kOut) {
-            maps[0] = &tmq; maps[1] = &tmk; maps[2] = &tmv;
-            convw[0] = p.conv_q; convw[1] = p.conv_k; convw[2] = p.conv_v;
-        } else {
-            maps[0] = &tmk; maps[1] = &tmv; maps[2] = &tmv;
-            convw[0] = p.conv_k; convw[1] = p.conv_v; convw[2] = p.conv_v;
-        }
+        constexpr int NT = Ly::NTENS, NSL = Ly::NRAWSLOT;
+        // output pass: k, q (-> Gram), then v; transfer pass: k, v
+        auto map_of = [&](int w) -> const CUtensorMap * {
+            if constexpr (kOut) return w == 0 ? &tmk : (w == 1 ? &tmq : &tmv);
+            else return w == 0 ? &tmk : &tmv;
+        };
+        auto conv_of = [&](int w) -> const float * {
+            if constexpr (kOut) return w == 0 ? p.conv_k : (w == 1 ? p.conv_q : p.conv_v);
+            else return w == 0 ? p.conv_k : p.conv_v;
+        };
         auto row0 = [&](int c) { return p.rev ? p.T - kC - c * kC : c * kC - 3; };
-        // thread 0 issues every raw box; per tensor, the last block whose box it issued and the last
-        // one whose box the loop has consumed (what is left in flight when the loop ends early)
-        int issued[3] = {-1, -1, -1}, consumed[3] = {-1, -1, -1};
+        const int nload = n * NT;
+        auto issue = [&](int l) {  // thread 0
+            const int sl = l % NSL, i = l / NT, w = l % NT;
+            mbar_arrive_expect_tx(&bars[B_RAW + sl], kRawBytes);
+            tma_load_3d(sm + Ly::RAW + sl * kRawBytes, map_of(w), &bars[B_RAW + sl], h * kD, row0(c0 + i), b);
+            if (i + 1 < n) tma_prefetch_3d(map_of(w), h * kD, max(row0(c0 + i + 1), 0), b);
+        };
+        int issued_hi = -1, consumed_hi = -1;  // thread 0: last load issued / read
         if (pt == 0) {
-            for (int w = 0; w < Ly::NRAW; ++w) {
-                mbar_arrive_expect_tx(&bars[B_RAW + w], kRawBytes);
-                tma_load_3d(sm + Ly::RAW + w * kRawBytes, maps[w], &bars[B_RAW + w], h * kD, row0(c0), b);
-                if (n > 1) tma_prefetch_3d(maps[w], h * kD, max(row0(c0 + 1), 0), b);
-                issued[w] = 0;
-            }
+            for (int l = 0; l < NSL && l < nload; ++l) issue(l);
+            issued_hi = min(NSL, nload) - 1;
         }
+        // the head's conv taps, once: [tensor][j][cg] so that a token row's 16 threads read 16
+        // consecutive float4
+        for (int e = pt; e < NT * 128; e += 128) {
+            const int w = e >> 7, ch = e & 127;
+            convs[w * 128 + (ch & 7) * 16 + (ch >> 3)] =
+                __ldg(reinterpret_cast<const float4 *>(conv_of(w)) + static_cast<size_t>(h) * kD + ch);
+        }
+        named_sync(NB_PREP, 128);
         bool ok = true;
         for (int i = 0; ok && i < n; ++i) {
             const int c = c0 + i, s = i & 1;
             uint8_t *kq = sm + Ly::KQ + s * 32768;
+            const bool ragged = (c + 1) * kC > p.T;
+            if (pt == 0) FTRACE(i, 8);
             if (i >= 2) ok = mbar_wait(&bars[B_FREE + s], ((i >> 1) - 1) & 1, ab, p.status, lim);
 #pragma unroll 1
-            for (int w = 0; w < Ly::NRAW; ++w) {
-                // destination: output pass q -> KQ rows 64+, k -> KQ rows 0-63, v -> V tile;
+            for (int w = 0; w < NT; ++w) {
+                // destination: output pass k -> KQ rows 0-63, q -> KQ rows 64+, v -> V tile;
                 // transfer pass k -> KQ rows 0-63, v -> KQ rows 64+
-                const bool is_v = kOut ? (w == 2) : (w == 1);
-                const float scale = (kOut && w == 0) ? p.q_scale : 1.0f;
+                const bool is_v = w == NT - 1;
                 uint8_t *dst = kq;
-                int drows = 128, doff = ((kOut && w == 0) || (!kOut && w == 1)) ? 64 : 0;
+                int drows = 128, doff = (w == 1) ? 64 : 0;
                 if (kOut && is_v) {
                     dst = sm + Lay<true>::V;
                     drows = 64;
                     doff = 0;
                     if (i >= 1) ok = ok && mbar_wait(&bars[B_VFREE], (i - 1) & 1, ab, p.status, lim);
                 }
-                ok = ok && mbar_wait(&bars[B_RAW + w], i & 1, ab, p.status, lim);
+                const int l = i * NT + w, sl = l % NSL;
+                ok = ok && mbar_wait(&bars[B_RAW + sl], (l / NSL) & 1, ab, p.status, lim);
                 ok = group_all(NB_PREP, 128, ok);
                 if (!ok) break;
-                consumed[w] = i;
-                const uint8_t *tile = sm + Ly::RAW + w * kRawBytes + cg * 16;
+                if (pt == 0) FTRACE(i, 9 + 2 * w);
+                consumed_hi = l;
+                const uint8_t *tile = sm + Ly::RAW + sl * kRawBytes + cg * 16;
                 float4 wt[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    wt[j] = __ldg(reinterpret_cast<const float4 *>(convw[w]) + static_cast<size_t>(h) * kD + cg * 8 + j);
-                auto rowp = [&](int k) { return tile + (p.rev ? (kRawRows - 1 - k) : k) * 256; };
-                float win[4][8];
+                for (int j = 0; j < 8; ++j) wt[j] = convs[w * 128 + j * 16 + cg];
+                // box row of window row k (k = 0 .. 66; the reverse scan reads its box bottom-up)
+                const uint8_t *rp = tile + (p.rev ? (kRawRows - 1 - rbeg) * 256 : rbeg * 256);
+                const int rstep = p.rev ? -256 : 256;
+                // u_t = w0 x_(t-3) + w1 x_(t-2) + w2 x_(t-1) + w3 x_t: each raw row x_t completes u_t
+                // and feeds the partial sums p0, p1, p2 of u_(t+1), u_(t+2), u_(t+3)
+                float p0[8], p1[8], p2[8], ss[8], x[8];
+                load8<InT>(rp, x);
 #pragma unroll
-                for (int k = 0; k < 3; ++k) load8<InT>(rowp(rbeg + k), win[k]);
+                for (int j = 0; j < 8; ++j) p0[j] = wt[j].x * x[j];
+                load8<InT>(rp + rstep, x);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    p0[j] = fmaf(wt[j].y, x[j], p0[j]);
+                    p1[j] = wt[j].x * x[j];
+                }
+                load8<InT>(rp + 2 * rstep, x);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    p0[j] = fmaf(wt[j].z, x[j], p0[j]);
+                    p1[j] = fmaf(wt[j].y, x[j], p1[j]);
+                    p2[j] = wt[j].x * x[j];
+                }
 #pragma unroll
                 for (int r = 0; r < 8; ++r) {
-                    load8<InT>(rowp(rbeg + r + 3), win[(r + 3) & 3]);
-                    float u[8], ss = 0.0f;
+                    load8<InT>(rp + (r + 3) * rstep, x);
+                    float u[8];
+                    ss[r] = 0.0f;
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        float a = wt[j].x * win[r & 3][j];
-                        a = fmaf(wt[j].y, win[(r + 1) & 3][j], a);
-                        a = fmaf(wt[j].z, win[(r + 2) & 3][j], a);
-                        a = fmaf(wt[j].w, win[(r + 3) & 3][j], a);
-                        u[j] = silu_tc(a);
-                        ss = fmaf(u[j], u[j], ss);
+                        u[j] = silu_tc(fmaf(wt[j].w, x[j], p0[j]));
+                        p0[j] = fmaf(wt[j].z, x[j], p1[j]);
+                        p1[j] = fmaf(wt[j].y, x[j], p2[j]);
+                        p2[j] = wt[j].x * x[j];
+                        ss[r] = fmaf(u[j], u[j], ss[r]);
                     }
-                    if (!is_v) {
-#pragma unroll
-                        for (int off = 8; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-                        const float sc = rsqrtf(ss + p.l2_eps) * scale;
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) u[j] *= sc;
-                    }
-                    if (c * kC + rbeg + r >= p.T) {
+                    if (ragged && c * kC + rbeg + r >= p.T) {
 #pragma unroll
                         for (int j = 0; j < 8; ++j) u[j] = 0.0f;
                     }
                     put8h(dst, drows, doff + rbeg + r, cg, u);
                 }
+                if (!is_v) {
+                    // |x'|^2 of the run's eight tokens over the 16 threads of each token row, as eight
+                    // independent chains; then 1/|k'| or 1/(sqrt(d_k) |q'|) (padding tokens: their
+                    // zero rows make the factor irrelevant)
+#pragma unroll
+                    for (int off = 8; off > 0; off >>= 1)
+#pragma unroll
+                        for (int r = 0; r < 8; ++r) ss[r] += __shfl_xor_sync(0xffffffffu, ss[r], off);
+                    if (cg == 0) {
+                        const float sc = (kOut && w == 1) ? p.q_scale : 1.0f;
+                        float *dn = invn + s * 128 + (w == 1 ? 64 : 0) + rbeg;
+#pragma unroll
+                        for (int r = 0; r < 8; ++r) dn[r] = rsqrtf(ss[r] + p.l2_eps) * sc;
+                    }
+                }
                 named_sync(NB_PREP, 128);  // every read of this raw box is done
-                if (pt == 0 && i + 1 < n) {
-                    mbar_arrive_expect_tx(&bars[B_RAW + w], kRawBytes);
-                    tma_load_3d(sm + Ly::RAW + w * kRawBytes, maps[w], &bars[B_RAW + w], h * kD, row0(c + 1), b);
-                    if (i + 2 < n) tma_prefetch_3d(maps[w], h * kD, max(row0(c + 2), 0), b);
-                    issued[w] = i + 1;
+                if (pt == 0) FTRACE(i, 10 + 2 * w);
+                if (pt == 0 && l + NSL < nload) {
+                    issue(l + NSL);
+                    issued_hi = l + NSL;
+                }
+                if (w == 1 || (kOut && is_v)) {
+                    fence_proxy_async();  // the tiles are read by the tensor cores next
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars[is_v && kOut ? B_PREPV : B_PREP + s]);
                 }
             }
             if (!ok) break;
-            fence_proxy_async();  // the tiles are read by the tensor cores next
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[B_PREP + s]);
+            if (pt == 0) FTRACE(i, 15);
         }
         if (pt == 0) {  // raw boxes still in flight land before shared memory goes away
-            for (int w = 0; w < Ly::NRAW; ++w)
-                if (issued[w] > consumed[w]) mbar_wait_drain(&bars[B_RAW + w], issued[w] & 1, lim);
+            for (int l = consumed_hi + 1; l <= issued_hi; ++l)
+                mbar_wait_drain(&bars[B_RAW + l % NSL], (l / NSL) & 1, lim);
         }
     } else if (warp < W_CH) {
-        // ================================================================ gates, UT transform
+        // ================================================================ gates, L, Aqk, Qt, T
+        // Per block j: the gates (into the slot of block j - 2, free once the state warps have
+        // finished that block's W^T tile and Kt), then from the block's Gram the rows of L (lanes
+        // 0-63: K'K'^T) and of Aqk (lanes 64-127: Q'K'^T) and Qt, then T = (I + L)^-1 and the two
+        // scaled T tiles of the slot (free once block j - 2's W^T and U^T are done).
         const int ut = tid - 32 * W_UT;
         const int q4 = warp & 3;
         const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
-        const int bb = b;
         const float eA = __expf(p.A_log[h]), dtb = p.dt_bias[h];
-        uint8_t *Tt = sm + Ly::T;
-        uint8_t *TWt = sm + Ly::TW;
         bool ok = true;
-        for (int i = 0; ok && i < n; ++i) {
-            const int c = c0 + i, s = i & 1;
+        for (int j = 0; ok && j < n; ++j) {
+            const int c = c0 + j, s = j & 1;
             float *Gs = gate + s * 256, *Bs = Gs + 64, *Ec = Gs + 128, *Bw = Gs + 192;
+            const float *ik = invn + s * 128, *iq = ik + 64;  // 1/|k'|, 1/(sqrt(d_k) |q'|) of the tokens
             uint8_t *kq = sm + Ly::KQ + s * 32768;
-            // ---- gates of the block: log alpha = -exp(A_log) softplus(g + dt_bias), beta = sigmoid(b),
-            //      G = inclusive cumulative sum of log alpha over the block (padding rows: 0, 0)
-            float cs = 0.0f, be = 0.0f;
-            if (ut < 64) {
-                const int t = c * kC + ut;
-                float la = 0.0f;
-                if (t < p.T) {
-                    const size_t gi = (static_cast<size_t>(bb) * p.T + (p.rev ? p.T - 1 - t : t)) * p.H + h;
-                    if (p.debug && gi >= static_cast<size_t>(p.B) * p.T * p.H) {
-                        atomicCAS(p.status, kStatusOk, kStatusCheck);
-                    } else {
-                        const float xg = p.g[gi] + dtb;
-                        const float sp = xg > 20.0f ? xg : __logf(1.0f + __expf(xg));
-                        la = -eA * sp;
-                        be = __fdividef(1.0f, 1.0f + __expf(-p.bg[gi]));
-                    }
-                }
-                cs = la;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float v = __shfl_up_sync(0xffffffffu, cs, off);
-                    if (lane >= off) cs += v;
-                }
-                if (lane == 31) wtot[ut >> 5] = cs;
-            }
-            named_sync(NB_UT, 128);
-            if (ut < 64) {
-                const float G = cs + (ut >= 32 ? wtot[0] : 0.0f);
-                Gs[ut] = G;
-                Bs[ut] = be;
-                Bw[ut] = be * __expf(G);
-            }
-            named_sync(NB_UT, 128);
-            if (ut < 64) Ec[ut] = __expf(fminf(Gs[ut | 15] - Gs[ut], 0.0f));
-            named_sync(NB_UT, 128);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[B_GATE + s]);
-
-            // ---- L (lanes 0-63 of the Gram: K K^T) and Aqk (lanes 64-127: Q K^T) rows
-            ok = group_all(NB_UT, 128, mbar_wait(&bars[B_GRAM], i & 1, ab, p.status, lim));
+            uint8_t *Tt = sm + Ly::T + s * 8192, *TWt = sm + Ly::TW + s * 8192;
+            if (ut == 0) FTRACE(j, 16);
+            // ---- gates: log alpha = -exp(A_log) softplus(g + dt_bias), beta = sigmoid(b), G = inclusive
+            //      cumulative sum of log alpha over the block (padding rows: 0, 0), and the column factors
+            //      e^(G_m - G_j) of the split decay (m the last row of j's 16-row group)
+            ok = group_all(NB_UT, 128, j < 2 || mbar_wait(&bars[B_UTD + s], ((j >> 1) - 1) & 1, ab, p.status, lim));
             if (!ok) break;
+            {
+                float cs = 0.0f, be = 0.0f;
+                if (ut < 64) {
+                    const int t = c * kC + ut;
+                    float la = 0.0f;
+                    if (t < p.T) {
+                        const size_t gi = (static_cast<size_t>(b) * p.T + (p.rev ? p.T - 1 - t : t)) * p.H + h;
+                        if (p.debug && gi >= static_cast<size_t>(p.B) * p.T * p.H) {
+                            atomicCAS(p.status, kStatusOk, kStatusCheck);
+                        } else {
+                            const float xg = p.g[gi] + dtb;
+                            const float sp = xg > 20.0f ? xg : __logf(1.0f + __expf(xg));
+                            la = -eA * sp;
+                            be = __fdividef(1.0f, 1.0f + __expf(-p.bg[gi]));
+                        }
+                    }
+                    cs = la;
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const float v = __shfl_up_sync(0xffffffffu, cs, off);
+                        if (lane >= off) cs += v;
+                    }
+                    if (lane == 31) wtot[ut >> 5] = cs;
+                }
+                named_sync(NB_UT, 128);
+                if (ut < 64) {
+                    Gs[ut] = cs + (ut >= 32 ? wtot[0] : 0.0f);
+                    Bs[ut] = be;
+                }
+                named_sync(NB_UT, 128);
+                if (ut < 64) Ec[ut] = __expf(fminf(Gs[ut | 15] - Gs[ut], 0.0f));
+                named_sync(NB_UT, 128);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[B_GATE + s]);
+            }
+            if (ut == 0) FTRACE(j, 17);
+            // ---- L and Aqk rows; Qt
+            ok = group_all(NB_UT, 128,
+                           mbar_wait(&bars[B_PREP + s], (j >> 1) & 1, ab, p.status, lim) &&
+                               mbar_wait(&bars[B_GRAM], j & 1, ab, p.status, lim) &&
+                               (j < 2 || mbar_wait(&bars[B_WT + s], ((j >> 1) - 1) & 1, ab, p.status, lim)));
+            if (!ok) break;
+            if (ut == 0) FTRACE(j, 18);
             tc_fence_after();
             {
                 const int r = (q4 & 1) * 32 + lane;  // row within the block
-                const float Gr = Gs[r];
                 const bool lrow = q4 < 2;
                 if (lrow || kOut) {
-                    const float br = lrow ? Bs[r] : 1.0f;
+                    // L_rj = beta_r e^(G_r - G_j) k_r.k_j (j < r);  Aqk_rj = e^(G_r - G_j) q_r.k_j / sqrt(d_k)
+                    // (j <= r); below r's 16-row group the decay splits as e^(G_r - G_m) e^(G_m - G_j)
+                    const float Gr = Gs[r];
+                    const float br = lrow ? Bs[r] * ik[r] : iq[r];
                     uint8_t *dstt = lrow ? Tt : (sm + (kOut ? Lay<true>::AQK : 0) + s * 8192);
                     const int rg16 = r >> 4;
+                    const int lim_j = lrow ? r : r + 1;  // columns j < lim_j are kept
+#pragma unroll 1
+                    for (int g = 0; g < 4; ++g) {
+                        float a[16], l[16];
+                        tmem_ld16(tmem + lane_base + TM::GA + g * 16, a);
+                        if (g < rg16) {
+                            const float fr = br * __expf(fminf(Gr - Gs[16 * g + 15], 0.0f));
 #pragma unroll
-                    for (int hf = 0; hf < 2; ++hf) {
-                        float a[32];
-                        tmem_ld32(tmem + lane_base + TM::GW + hf * 32, a);
+                            for (int e = 0; e < 16; ++e) l[e] = fr * Ec[16 * g + e] * ik[16 * g + e] * a[e];
+                        } else {
 #pragma unroll
-                        for (int gq = 0; gq < 2; ++gq) {  // 16-column group g = 2 hf + gq
-                            const int g = 2 * hf + gq;
-                            float l[16];
-                            if (g < rg16) {
-                                const float fr = br * __expf(fminf(Gr - Gs[16 * g + 15], 0.0f));
-#pragma unroll
-                                for (int e = 0; e < 16; ++e) l[e] = fr * Ec[16 * g + e] * a[16 * gq + e];
-                            } else if (g == rg16) {
-#pragma unroll
-                                for (int e = 0; e < 16; ++e) {
-                                    const int j = 16 * g + e;
-                                    const bool in = lrow ? (j < r) : (j <= r);
-                                    l[e] = in ? br * __expf(fminf(Gr - Gs[j], 0.0f)) * a[16 * gq + e] : 0.0f;
-                                }
-                                if (lrow) {
-                                    float *dd = ldiag + rg16 * 256 + (r & 15) * 16;
-#pragma unroll
-                                    for (int e = 0; e < 16; e += 4)
-                                        *reinterpret_cast<float4 *>(dd + e) = make_float4(l[e], l[e + 1], l[e + 2], l[e + 3]);
-                                }
-                            } else {
-#pragma unroll
-                                for (int e = 0; e < 16; ++e) l[e] = 0.0f;
+                            for (int e = 0; e < 16; ++e) {
+                                const int jj = 16 * g + e;
+                                l[e] = (jj < lim_j) ? br * __expf(fminf(Gr - Gs[jj], 0.0f)) * ik[jj] * a[e] : 0.0f;
                             }
-                            put8h(dstt, 64, r, 2 * g, l);
-                            put8h(dstt, 64, r, 2 * g + 1, l + 8);
+                            if (lrow && g == rg16) {
+                                float *dd = ldiag + rg16 * 256 + (r & 15) * 16;
+#pragma unroll
+                                for (int e = 0; e < 16; e += 4)
+                                    *reinterpret_cast<float4 *>(dd + e) = make_float4(l[e], l[e + 1], l[e + 2], l[e + 3]);
+                            }
                         }
+                        put8h(dstt, 64, r, 2 * g, l);
+                        put8h(dstt, 64, r, 2 * g + 1, l + 8);
                     }
-                    if (kOut && !lrow) scale_row_chunks(kq, 128, 64 + r, 0, 16, __expf(fminf(Gr, 0.0f)));  // Qt
+                    if (kOut && !lrow) scale_row_chunks(kq, 128, 64 + r, 0, 16, __expf(fminf(Gr, 0.0f)) * iq[r]);  // Qt
                 }
+                if (ut < 64) Bw[ut] = Bs[ut] * __expf(Gs[ut]) * ik[ut];
             }
+            tc_fence_before();
             named_sync(NB_UT, 128);
-            // ---- T = (I + L)^-1, then T diag(beta e^G) (TW tile) and T diag(beta) (in place)
+            if (ut == 0) FTRACE(j, 19);
+            // ---- T = (I + L)^-1, then T diag(beta e^G / |k'|) (TW tile) and T diag(beta) (in place)
             invert_unit_lower64(Tt, ldiag, ut);
+            if (ut == 0) FTRACE(j, 20);
             {
-                const int r = ut >> 1, ch0 = (ut & 1) * 4;
+                const int rr = ut >> 1, ch0 = (ut & 1) * 4;
 #pragma unroll
                 for (int ch = ch0; ch < ch0 + 4; ++ch) {
-                    uint4 *pu = reinterpret_cast<uint4 *>(Tt + tile_off(64, r, ch));
+                    uint4 *pu = reinterpret_cast<uint4 *>(Tt + tile_off(64, rr, ch));
                     const uint4 u = *pu;
                     const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
                     uint32_t ow[4], ou[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float2 x = unpack_half2(w4[e]);
-                        const int j = ch * 8 + 2 * e;
-                        ow[e] = pack_half2(x.x * Bw[j], x.y * Bw[j + 1]);
-                        ou[e] = pack_half2(x.x * Bs[j], x.y * Bs[j + 1]);
+                        const float2 xx = unpack_half2(w4[e]);
+                        const int jj = ch * 8 + 2 * e;
+                        ow[e] = pack_half2(xx.x * Bw[jj], xx.y * Bw[jj + 1]);
+                        ou[e] = pack_half2(xx.x * Bs[jj], xx.y * Bs[jj + 1]);
                     }
-                    *reinterpret_cast<uint4 *>(TWt + tile_off(64, r, ch)) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    *reinterpret_cast<uint4 *>(TWt + tile_off(64, rr, ch)) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                     *pu = make_uint4(ou[0], ou[1], ou[2], ou[3]);
                 }
             }
             fence_proxy_async();
             named_sync(NB_UT, 128);
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[B_TREADY]);
-
-            // ---- W^T out of TMEM into the slot's W^T tile (row = d_k); Kt = diag(e^(G_C - G)) K^
-            ok = group_all(NB_UT, 128, mbar_wait(&bars[B_WT], i & 1, ab, p.status, lim));
-            if (!ok) break;
-            tc_fence_after();
-            {
-                const int row = q4 * 32 + lane;
-                uint8_t *wt = sm + Ly::WT + s * 16384;
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    float a[32];
-                    tmem_ld32(tmem + lane_base + TM::GW + hf * 32, a);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) put8h(wt, 128, row, hf * 4 + q, a + 8 * q);
-                }
-                const int r = ut >> 1;
-                scale_row_chunks(kq, 128, r, (ut & 1) * 8, 8, __expf(fminf(Gs[kC - 1] - Gs[r], 0.0f)));
-            }
-            fence_proxy_async();
-            tc_fence_before();
-            named_sync(NB_UT, 128);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[B_UTD + s]);
+            if (lane == 0) mbar_arrive(&bars[B_TREADY + s]);
+            if (ut == 0) FTRACE(j, 21);
         }
     } else if (warp < W_X || !kOut) {
         // ================================================================ state step
-        // warps 9-12: the state S (lanes = d_v); transfer pass warps 13-16: the transfer P (lanes = d_k)
+        // warps 9-12: the state S (lanes = d_v), and each block's W^T tile and Kt (lanes = d_k);
+        // transfer pass warps 13-16: the transfer P (lanes = d_k)
         const bool isP = !kOut && warp >= W_X;
         const int q4 = warp & 3;
         const int row = q4 * 32 + lane;
@@ -748,7 +821,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int q = 0; q < 4; ++q) put8h(n16s, 128, row, ch * 4 + q, v + 8 * q);
             }
         };
-        // initial (negated) state: row `row` of S_start, or -I for the transfer matrix
+        // initial (negated) state: row `row` of S_start, or -I for the transfer matrix; its fp16 copy,
+        // then the state decayed by the first block's decay
+        bool ok = true;
         {
             const float *src = nullptr;
             if (!isP) {
@@ -759,85 +834,122 @@ __global__ void __launch_bounds__(kThreads, 1)
                     src = p.SS + ((static_cast<size_t>(bh) * p.NS + seg) * kD + row) * kD;
                 }
             }
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_GATE], 0, ab, p.status, lim));
+            const float gC = ok ? __expf(fminf(gate[kC - 1], 0.0f)) : 0.0f;
 #pragma unroll 1
             for (int ch = 0; ch < 4; ++ch) {
                 float v[32];
 #pragma unroll
                 for (int e = 0; e < 32; e += 4) {
-                    float4 x = src ? *reinterpret_cast<const float4 *>(src + ch * 32 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    float4 xv = src ? *reinterpret_cast<const float4 *>(src + ch * 32 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
                     if (isP) {
-                        x.x = (ch * 32 + e == row) ? 1.0f : 0.0f;
-                        x.y = (ch * 32 + e + 1 == row) ? 1.0f : 0.0f;
-                        x.z = (ch * 32 + e + 2 == row) ? 1.0f : 0.0f;
-                        x.w = (ch * 32 + e + 3 == row) ? 1.0f : 0.0f;
+                        xv.x = (ch * 32 + e == row) ? 1.0f : 0.0f;
+                        xv.y = (ch * 32 + e + 1 == row) ? 1.0f : 0.0f;
+                        xv.z = (ch * 32 + e + 2 == row) ? 1.0f : 0.0f;
+                        xv.w = (ch * 32 + e + 3 == row) ? 1.0f : 0.0f;
                     }
-                    v[e] = -x.x; v[e + 1] = -x.y; v[e + 2] = -x.z; v[e + 3] = -x.w;
+                    v[e] = -xv.x; v[e + 1] = -xv.y; v[e + 2] = -xv.z; v[e + 3] = -xv.w;
                 }
-                tmem_st32(tN + ch * 32, v);
                 put_n16(v, ch);
-            }
-        }
-        tmem_st_wait();
-        if (!kOut) fence_proxy_async();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[B_N16]);
-        bool ok = true;
-        for (int i = 0; ok && i < n; ++i) {
-            const int s = i & 1;
-            // decay the fp32 state by the block's total decay while Delta^T is formed
-            ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_GATE + s], (i >> 1) & 1, ab, p.status, lim));
-            if (!ok) break;
-            const float gC = __expf(fminf(gate[s * 256 + kC - 1], 0.0f));
-            tc_fence_after();
-#pragma unroll 1
-            for (int ch = 0; ch < 4; ++ch) {
-                float v[32];
-                tmem_ld32(tN + ch * 32, v);
 #pragma unroll
                 for (int e = 0; e < 32; ++e) v[e] *= gC;
                 tmem_st32(tN + ch * 32, v);
             }
+            tmem_st_wait();
+            if (!kOut) fence_proxy_async();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[B_N16]);
+        }
+        for (int i = 0; ok && i < n; ++i) {
+            const int s = i & 1;
+            if (!isP) {
+                // ---- block i's W^T (lanes = d_k) into its slot's tile, and Kt = diag(e^(G_C - G) / |k'|) K'
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_WT + s], (i >> 1) & 1, ab, p.status, lim) &&
+                                                 mbar_wait(&bars[B_PREP + s], (i >> 1) & 1, ab, p.status, lim) &&
+                                                 mbar_wait(&bars[B_GATE + s], (i >> 1) & 1, ab, p.status, lim));
+                if (!ok) break;
+                if (tid == 32 * W_CH) FTRACE(i, 24);
+                tc_fence_after();
+                {
+                    float a[32], a2[32];
+                    tmem_ld32x2(tmem + lb + TM::GB, tmem + lb + TM::GB + 32, a, a2);
+                    uint8_t *wt = sm + Ly::WT + s * 16384;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) put8h(wt, 128, row, q, a + 8 * q);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) put8h(wt, 128, row, 4 + q, a2 + 8 * q);
+                }
+                {
+                    const float *Gs = gate + s * 256, *ik = invn + s * 128;
+                    const int r = row >> 1;
+                    scale_row_chunks(sm + Ly::KQ + s * 32768, 128, r, (row & 1) * 8, 8,
+                                     __expf(fminf(Gs[kC - 1] - Gs[r], 0.0f)) * ik[r]);
+                }
+                fence_proxy_async();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[B_UTD + s]);
+            }
+            // ---- Delta^T -> E16 = fp16(-Delta^T), written over the first half of its columns
             ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_DELTA], i & 1, ab, p.status, lim));
             if (!ok) break;
+            if (tid == 32 * W_CH) FTRACE(i, 25);
             tc_fence_after();
             {
-                float d[32];
+                float d0[32], d1[32];
                 uint32_t pk[16];
-                tmem_ld32(tU, d);
+                tmem_ld32x2(tU, tU + 32, d0, d1);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) pk[e] = pack_half2(-d[2 * e], -d[2 * e + 1]);
+                for (int e = 0; e < 16; ++e) pk[e] = pack_half2(-d0[2 * e], -d0[2 * e + 1]);
                 tmem_st16(tE, pk);
-                tmem_ld32(tU + 32, d);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) pk[e] = pack_half2(-d[2 * e], -d[2 * e + 1]);
+                for (int e = 0; e < 16; ++e) pk[e] = pack_half2(-d1[2 * e], -d1[2 * e + 1]);
                 tmem_st16(tE + 16, pk);
             }
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[B_E16]);
+            if (tid == 32 * W_CH) FTRACE(i, 26);
             ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_STATE], i & 1, ab, p.status, lim));
             if (!ok) break;
-            tc_fence_after();
+            if (tid == 32 * W_CH) FTRACE(i, 27);
             if (i + 1 < n) {
+                // one read of the state: its fp16 copy for block i + 1's products, and the state
+                // decayed by block i + 1's total decay for its update
+                const int s1 = (i + 1) & 1;
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_GATE + s1], ((i + 1) >> 1) & 1, ab, p.status, lim));
+                if (!ok) break;
+                const float gC = __expf(fminf(gate[s1 * 256 + kC - 1], 0.0f));
+                tc_fence_after();
 #pragma unroll 1
-                for (int ch = 0; ch < 4; ++ch) {
-                    float v[32];
-                    tmem_ld32(tN + ch * 32, v);
-                    put_n16(v, ch);
+                for (int hf = 0; hf < 2; ++hf) {
+                    float a[32], a2[32];
+                    tmem_ld32x2(tN + hf * 64, tN + hf * 64 + 32, a, a2);
+                    put_n16(a, 2 * hf);
+                    put_n16(a2, 2 * hf + 1);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        a[e] *= gC;
+                        a2[e] *= gC;
+                    }
+                    tmem_st32(tN + hf * 64, a);
+                    tmem_st32(tN + hf * 64 + 32, a2);
                 }
                 tmem_st_wait();
                 if (!kOut) fence_proxy_async();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[B_N16]);
+                if (tid == 32 * W_CH) FTRACE(i, 28);
             } else {
                 // end of the segment: S_loc / P (transfer pass), or the final state
                 float *dst = nullptr;
                 if (!kOut) dst = p.SP + ((static_cast<size_t>(bh) * p.NS + seg) * 2 + (isP ? 1 : 0)) * kD * kD;
                 else if (p.s_end && seg == p.NS - 1) dst = p.s_end + static_cast<size_t>(bh) * kD * kD;
                 if (dst) {
+                    tc_fence_after();
                     float *d = dst + static_cast<size_t>(row) * kD;
 #pragma unroll 1
                     for (int ch = 0; ch < 4; ++ch) {
@@ -852,6 +964,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ================================================================ output step (output pass)
+        // y = o / sqrt(mean(o^2) + eps) * w * SiLU(z), o = -(the O^T accumulator), lanes = d_v
         const int et = tid - 32 * W_X;
         const int q4 = warp & 3;
         const int row = q4 * 32 + lane;  // d_v channel (TMEM lane)
@@ -866,45 +979,40 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (n > 1) tma_prefetch_3d(&tmz, h * kD, max(zrow0(c0 + 1), 0), b);
             zpend = 0;
         }
-        const float wv = nw[row];
+        const float nwv = -nw[row];  // the O^T accumulator holds -o
+        // row t of the z / y box (the reverse scan's box runs backwards)
+        uint8_t *zrow = zt + (p.rev ? (kC - 1) * 256 : 0) + row * 2;
+        const int zstep = p.rev ? -256 : 256;
         bool ok = true;
         for (int i = 0; ok && i < n; ++i) {
             const int c = c0 + i, s = i & 1;
             const uint32_t tO = tmem + lb + Tm<true>::O + s * 64;
             ok = group_all(NB_X, 128, mbar_wait(&bars[B_OFULL + s], (i >> 1) & 1, ab, p.status, lim));
             if (!ok) break;
+            if (et == 0) FTRACE(i, 29);
             tc_fence_after();
-            // sum over the 128 channels of o^2 per token: reduce-scatter across the warp's lanes
-            // (lane l ends with tokens 2l, 2l+1), then across the four warps through shared memory
-            {
-                float x[64];
-                {
-                    float a[32];
-                    tmem_ld32(tO, a);
+            // sum over the 128 channels of o^2 per token: reduce-scatter across the warp's lanes, 32
+            // tokens at a time (lane l ends with token 32 hf + l), then across the four warps
+#pragma unroll 1
+            for (int hf = 0; hf < 2; ++hf) {
+                float x[32];
+                tmem_ld32(tO + hf * 32, x);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) x[e] = a[e];
-                    tmem_ld32(tO + 32, a);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) x[32 + e] = a[e];
-                }
-#pragma unroll
-                for (int e = 0; e < 64; ++e) x[e] *= x[e];
+                for (int e = 0; e < 32; ++e) x[e] *= x[e];
 #pragma unroll
                 for (int lvl = 0; lvl < 5; ++lvl) {
-                    const int half = 32 >> lvl;
-                    const int m = 16 >> lvl;
-                    const bool up = (lane & m) != 0;
+                    const int half = 16 >> lvl;  // current length 2 * half
+                    const bool up = (lane & half) != 0;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        if (j < half) {
-                            const float send = up ? x[j] : x[j + half];
-                            const float keep = up ? x[j + half] : x[j];
-                            x[j] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                    for (int jj = 0; jj < 16; ++jj) {
+                        if (jj < half) {
+                            const float send = up ? x[jj] : x[jj + half];
+                            const float keep = up ? x[jj + half] : x[jj];
+                            x[jj] = keep + __shfl_xor_sync(0xffffffffu, send, half);
                         }
                     }
                 }
-                red[(2 * lane) * 4 + q4] = x[0];
-                red[(2 * lane + 1) * 4 + q4] = x[1];
+                red[(hf * 32 + lane) * 4 + q4] = x[0];
             }
             named_sync(NB_X, 128);
             if (et < 64) {
@@ -913,25 +1021,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ok = group_all(NB_X, 128, mbar_wait(&bars[B_Z], i & 1, ab, p.status, lim));  // (also publishes rns)
             if (!ok) break;
-            if (et == 0) zpend = -1;
+            if (et == 0) {
+                FTRACE(i, 30);
+                zpend = -1;
+            }
             bool bad = false;
+            // padding rows have o = 0 and z = 0, so y = 0 there; only fp32 outputs, stored directly,
+            // need the live-row test
 #pragma unroll 1
-            for (int hf = 0; hf < 2; ++hf) {
-                float o[32];
-                tmem_ld32(tO + hf * 32, o);
-#pragma unroll 4
-                for (int e = 0; e < 32; ++e) {
-                    const int t = hf * 32 + e;
-                    const int tt = c * kC + t;
-                    const bool live = tt < p.T;
-                    const int j = p.rev ? kC - 1 - t : t;  // row of the z / y box
-                    uint8_t *zp = zt + j * 256 + row * 2;
-                    const float yv = -o[e] * rns[t] * wv * silu_tc(load1(zp, zhalf));
-                    if (p.debug) bad |= live && !isfinite(yv);
+            for (int ch = 0; ch < 4; ++ch) {  // 16 tokens at a time
+                float o[16];
+                tmem_ld16(tO + ch * 16, o);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int t = ch * 16 + e;
+                    uint8_t *zp = zrow + t * zstep;
+                    const float yv = o[e] * (rns[t] * nwv) * silu_tc(load1(zp, zhalf));
+                    bad |= !isfinite(yv);
                     if (p.out_kind == 1) {
-                        if (live) {
-                            const int x = p.rev ? p.T - 1 - tt : tt;
-                            static_cast<float *>(p.y)[((static_cast<size_t>(b) * p.T + x) * p.H + h) * kD + row] = yv;
+                        const int tt = c * kC + t;
+                        if (tt < p.T) {
+                            const int xr = p.rev ? p.T - 1 - tt : tt;
+                            static_cast<float *>(p.y)[((static_cast<size_t>(b) * p.T + xr) * p.H + h) * kD + row] = yv;
                         }
                     } else if (p.out_kind == 0) {
                         *reinterpret_cast<__nv_bfloat16 *>(zp) = __float2bfloat16_rn(yv);
@@ -943,7 +1054,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[B_OFREE + s]);
-            if (bad) atomicCAS(p.status, kStatusOk, kStatusCheck);
+            if (p.debug && bad) atomicCAS(p.status, kStatusOk, kStatusCheck);
             if (p.out_kind != 1) fence_proxy_async();
             named_sync(NB_X, 128);  // every read of the z box (and write of the y box) is done
             if (et == 0) {
@@ -957,6 +1068,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     bulk_commit();
                     bulk_wait_read_all();
                 }
+                FTRACE(i, 31);
                 if (i + 1 < n) {
                     mbar_arrive_expect_tx(&bars[B_Z], kC * 256);
                     tma_load_3d(zt, &tmz, &bars[B_Z], h * kD, zrow0(c + 1), b);
@@ -1071,3 +1183,5 @@ cudaError_t launch_fused_output(const FusedParams &p, InType in, const CUtensorM
 }
 
 }  // namespace gdn
+
+GDN_TRACE_EXPORT(fused)
