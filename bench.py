@@ -38,11 +38,23 @@ import gdn_inputs  # noqa: E402
 METRIC = "GDN fwd Mtokens/s at T=32760,H=12,d=128 bf16; % of tensor/HBM roofline"
 UNIT = "Mtokens/s"
 FLUSH_BYTES = 256 << 20
-KERNELS_TENSOR_SEG = ("transfer", "combine", "out")
-KERNELS_TENSOR_ONE = ("out",)
+KERNELS_TENSOR_SEG = ("prep", "chunk", "transfer", "combine", "scan")
+KERNELS_TENSOR_ONE = ("prep", "chunk", "scan")
+KERNELS_FUSED_SEG = ("fused_transfer", "fused_combine", "fused_out")
+KERNELS_FUSED_ONE = ("fused_out",)
 KERNELS_SIMT = ("prep", "recurrence", "output")
-KERNEL_SOURCES = {"transfer": "gdn_fused.cu", "combine": "gdn_fused.cu", "out": "gdn_fused.cu",
-                  "prep": "gdn_prep.cu", "recurrence": "gdn_simt.cu", "output": "gdn_simt.cu"}
+KERNEL_SOURCES = {"prep": "gdn_prep.cu", "chunk": "gdn_chunk.cu", "transfer": "gdn_scan.cu",
+                  "combine": "gdn_scan.cu", "scan": "gdn_scan.cu", "fused_transfer": "gdn_fused.cu",
+                  "fused_combine": "gdn_fused.cu", "fused_out": "gdn_fused.cu", "recurrence": "gdn_simt.cu",
+                  "output": "gdn_simt.cu"}
+
+
+def kernel_names(plan, fused=False):
+    if not plan.uses_tensor_path:
+        return KERNELS_SIMT
+    if fused:
+        return KERNELS_FUSED_SEG if plan.segments > 1 else KERNELS_FUSED_ONE
+    return KERNELS_TENSOR_SEG if plan.segments > 1 else KERNELS_TENSOR_ONE
 
 
 def path_bytes_per_token_head(d, s_in, s_out):
@@ -57,22 +69,32 @@ def path_flops_per_token_head(d, C=64):
 
 def kernel_work_per_token_head(name, d, s_in, s_out):
     """HBM bytes each kernel itself must move, and the tensor-core flops it issues, per (token,
-    head) of the token-heads it covers.  Tensor path (d = 128, 64-token blocks): the transfer pass
-    reads raw k, v and the gates and runs the state S and the transfer P side by side; the output
-    pass reads raw q, k, v, z and the gates and writes y; the combine moves only per-segment
-    states (negligible per token).  CUDA-core path: prep, recurrence and output kernels."""
+    head) of the token-heads it covers.
+
+    Tensor path (d = 128, 128-token blocks, fp16 intermediates): prep writes q^, k^, v^; chunk
+    builds W, U, Qt, Kt and the live 3/4 of Aqk; transfer runs each segment's [S | P] from W, U,
+    Kt; combine moves per-segment states only; scan rebuilds Delta and writes y.
+    Fused tensor path (64-token blocks, no intermediates in HBM): the transfer pass reads raw k, v
+    and the gates and runs S and P side by side; the output pass reads raw q, k, v, z and the
+    gates and writes y.  CUDA-core path: prep, recurrence and output kernels."""
+    if name == "prep":      # q k v in; q^ k^ v^ fp16 out
+        return 3 * d * s_in + 3 * d * 2, 0
+    if name == "chunk":     # q^ k^ v^ + g b in; W U Qt Kt, 3/4 of Aqk, G beta log-alpha out; K K^T, Q K^T, W, U
+        return 3 * d * 2 + 8 + 4 * 128 * 2 + 96 * 2 + 12, 4 * 2 * 128 * d
+    if name == "transfer":  # W U Kt in; W [S|P]^T and Kt^T Delta with N = 2d
+        return 3 * 128 * 2, 2 * 2 * 128 * 2 * d
+    if name in ("combine", "fused_combine"):  # per-segment states only (negligible per token)
+        return 0, 0
+    if name == "scan":      # W U Qt Kt, 3/4 of Aqk, z in; y out; W S^T, Qt S^T, Kt^T Delta, Aqk Delta
+        return 4 * 128 * 2 + 96 * 2 + d * s_in + d * s_out, 4 * 2 * 128 * d
     C = 64
     gram, wu = 2 * 128 * C * 128 // C, 2 * 2 * 128 * C * C // C          # [K;Q]K^T or KK^T; W^T and U^T
     step = 2 * 128 * C * d // C + 2 * 128 * 128 * C // C                # Delta^T, state update
-    if name == "transfer":
+    if name == "fused_transfer":
         return 2 * d * s_in + 8, gram + wu + 2 * step
-    if name == "out":          # Delta^T, O^T = N Qt^T, state, O^T += E Aqk^T
+    if name == "fused_out":    # Delta^T, O^T = N Qt^T, state, O^T += E Aqk^T
         return 4 * d * s_in + 8 + d * s_out, gram + wu + step + 2 * 128 * C * d // C + 2 * 128 * C * C // C
-    if name == "combine":
-        return 0, 0
-    if name == "prep":         # q k v in; q^ k^ v^ fp32 out; gates
-        return 3 * d * s_in + 3 * d * 4 + 8 + 12, 0
-    if name == "output":       # o fp32 + z in; y out
+    if name == "output":    # o fp32 + z in; y out
         return d * 4 + d * s_in + d * s_out, 0
     if name == "recurrence":
         return 3 * d * 4 + 8 + d * 4, 6 * d * d
@@ -277,12 +299,14 @@ def path_roofline(w, s_in, s_out, ms_per_step, peaks):
 
 
 def launch_units(name, w, plan):
-    """Token-heads one launch of a kernel covers: the transfer pass runs every segment but the last."""
-    if name == "transfer":
+    """Token-heads one launch of a kernel covers: a transfer pass runs every segment but the last
+    (segments of Ls blocks of 128 tokens on the tensor path, of 64 on the fused path)."""
+    if name in ("transfer", "fused_transfer"):
+        C = 64 if name == "fused_transfer" else 128
         ns = plan.segments
-        nb = -(-w.T // 64)
+        nb = -(-w.T // C)
         ls = -(-nb // ns)
-        return w.B * w.H * min((ns - 1) * ls * 64, w.T)
+        return w.B * w.H * min((ns - 1) * ls * C, w.T)
     return w.B * w.H * w.T
 
 
@@ -367,6 +391,8 @@ def main():
     ap.add_argument("--no-reverse", action="store_true", help="skip the reverse-scan timing")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward timing")
     ap.add_argument("--no-configs", action="store_true", help="skip the other four seeded workloads")
+    ap.add_argument("--fused", action="store_true", help="time the fused forward (FLAG_FUSED) as the main path")
+    ap.add_argument("--no-fused", action="store_true", help="skip the fused-forward timing beside the main path")
     ap.add_argument("--load-seconds", type=float, default=1.5)
     args = ap.parse_args()
     w = gdn_inputs.by_name(args.workload)
@@ -397,7 +423,8 @@ def main():
     out_name = args.out_dtype or ("bf16" if w.dtype == "bf16" else "f32")
     out_code = {"bf16": gdn.DTYPE_BF16, "f16": gdn.DTYPE_F16, "f32": gdn.DTYPE_F32}[out_name]
     out_t = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[out_name]
-    plan = gdn.Plan(w.B, w.T, w.H, w.d, in_code, out_code)
+    base_flags = gdn.FLAG_FUSED if args.fused else 0
+    plan = gdn.Plan(w.B, w.T, w.H, w.d, in_code, out_code, flags=base_flags)
     ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=dev)
     y = torch.empty((w.B, w.T, w.H, w.d), dtype=out_t, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -405,10 +432,7 @@ def main():
     s = stream.cuda_stream
     ptrs = gdn.tensor_ptrs(tens)
     L = plan.launches
-    if plan.uses_tensor_path:
-        names = KERNELS_TENSOR_SEG if plan.segments > 1 else KERNELS_TENSOR_ONE
-    else:
-        names = KERNELS_SIMT
+    names = kernel_names(plan, args.fused)
     assert len(names) == L
 
     for _ in range(args.warmup):
@@ -497,7 +521,7 @@ def main():
     # the reverse (anti-causal) scan of the same workload, its own plan and workspace
     reverse = None
     if not args.no_reverse:
-        plan_r = gdn.Plan(w.B, w.T, w.H, w.d, in_code, out_code, flags=gdn.FLAG_REVERSE)
+        plan_r = gdn.Plan(w.B, w.T, w.H, w.d, in_code, out_code, flags=gdn.FLAG_REVERSE | base_flags)
         ws_r = torch.empty(plan_r.workspace_bytes, dtype=torch.uint8, device=dev)
         n_r = max(3, min(args.steps, 10))
         for _ in range(2):
@@ -612,6 +636,40 @@ def main():
                "one_stream": {"value": job_throughput(world, tokens, serial_ms), "ms_per_step": serial_ms}}
         del wss[1], stagings
 
+    # the fused forward (FLAG_FUSED) of the same workload beside the main path: step time, its
+    # per-kernel breakdown and its roofline figures
+    fused = None
+    if not args.fused and not args.no_fused and plan.uses_tensor_path:
+        plan_f = gdn.Plan(w.B, w.T, w.H, w.d, in_code, out_code, flags=gdn.FLAG_FUSED)
+        ws_f = torch.empty(plan_f.workspace_bytes, dtype=torch.uint8, device=dev)
+        run_f = lambda: plan_f.forward_raw(ptrs, y.data_ptr(), ws_f.data_ptr(), s)  # noqa: E731
+        for _ in range(3):
+            run_f()
+        n_f = max(5, min(args.steps, 20))
+        f_ms = ranks_max(sum(time_steps(run_f, flush, stream, n_f)), world, dist, dev) / n_f
+        st = plan_f.device_status(ws_f.data_ptr(), s)
+        if st != gdn.OK:
+            raise SystemExit(f"device status after the fused forward: {gdn.status_string(st)}")
+        fnames = kernel_names(plan_f, True)
+        evf = [[torch.cuda.Event(enable_timing=True) for _ in range(len(fnames) + 1)] for _ in range(3)]
+        for row in evf:
+            for e in row:
+                e.record(stream)
+        torch.cuda.synchronize()
+        for k in range(3):
+            flush.zero_()
+            plan_f.forward_timed_raw(ptrs, y.data_ptr(), ws_f.data_ptr(), s, [e.cuda_event for e in evf[k]])
+        torch.cuda.synchronize()
+        fk = {fnames[i]: statistics.mean(evf[k][i].elapsed_time(evf[k][i + 1]) for k in range(3))
+              for i in range(len(fnames))}
+        s_in_f = 2 if w.dtype == "bf16" else 4
+        s_out_f = {"bf16": 2, "f16": 2, "f32": 4}[out_name]
+        fused = {"ms_per_step": f_ms, "value": job_throughput(world, w.B * w.T, f_ms), "unit": UNIT,
+                 "steps": n_f, "launches_per_step": plan_f.launches, "kernels_ms": fk,
+                 "workspace_bytes": plan_f.workspace_bytes,
+                 "path_frac": path_roofline(w, s_in_f, s_out_f, f_ms, load_peaks())["frac"]}
+        del ws_f
+
     # the other four seeded workloads (rank 0 alone, 1 GPU): same step, flush and event timing
     configs = None
     if world == 1 and not args.no_configs and not args.T:
@@ -658,10 +716,12 @@ def main():
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f16-mma/f32" if plan.uses_tensor_path else "f32", "data": "synthetic",
-            "config": workload_config(w, args.out_dtype, world),
+            "config": dict(workload_config(w, args.out_dtype, world),
+                           path="fused tensor (FLAG_FUSED)" if args.fused else
+                           ("tensor" if plan.uses_tensor_path else "CUDA-core fp32")),
             "roofline": roof, "path_roofline": path_roof, "kernels_ms": kern_ms,
             "segments": plan.segments, "cpu_baseline": cpu, "e2e": e2e, "state_io": state_io,
-            "reverse": reverse, "backward": bwd, "configs": configs,
+            "reverse": reverse, "backward": bwd, "fused": fused, "configs": configs,
             "clocks": clocks, "gpu_launches": L * args.steps,
             "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms), "max": max(step_ms)},
             "other_gpu_processes": None if others_before is None or others_after is None

@@ -30,6 +30,7 @@ DTYPE_BF16, DTYPE_F32, DTYPE_F16 = 0, 1, 2
 FLAG_DEBUG_CHECKS = 0x1
 FLAG_FORCE_SIMT = 0x2
 FLAG_REVERSE = 0x4
+FLAG_FUSED = 0x8
 FLAG_TEST_WAIT_TIMEOUT = 0x100
 
 
@@ -202,7 +203,8 @@ class Plan:
         _check(_lib.gdn_forward_host(self._h, ctypes.byref(ins), y_host, staging, workspace, stream),
                "gdn_forward_host")
 
-    WS_FIELDS = ("status", "qh", "kh", "vh", "G", "beta", "log_alpha", "o", "seg_states", "seg_start")
+    WS_FIELDS = ("status", "qh", "kh", "vh", "G", "beta", "log_alpha", "W", "U", "Qt", "Kt", "Aqk", "o", "Zloc",
+                 "Sstart", "seg_states", "seg_start")
 
     def workspace_offsets(self) -> dict:
         arr = (ctypes.c_size_t * len(self.WS_FIELDS))()

@@ -18,12 +18,13 @@ struct gdn_plan_s {
     gdn_config cfg;
     int device;
     bool tensor;
-    int Tp, NB, NS, Ls;
+    bool fused;              // GDN_FLAG_FUSED: the two-pass fused forward (64-token blocks)
+    int Tp, NB, NS, Ls;      // tensor path: 128-token blocks; fused: 64-token blocks
     long long tok_stride;
-    size_t in_esize, out_esize;
-    // workspace layout: the status word; the tensor path's per-segment S_loc / P and segment
-    // start states; the CUDA-core path's prepared q, k, v, gates and pre-norm output
-    size_t off_status, off_qh, off_kh, off_vh, off_G, off_beta, off_la, off_o, off_SP, off_SS, ws_bytes;
+    size_t in_esize, out_esize, inter_esize;
+    // workspace layout
+    size_t off_status, off_qh, off_kh, off_vh, off_G, off_beta, off_la;
+    size_t off_W, off_U, off_Qt, off_Kt, off_Aqk, off_Zloc, off_Sstart, off_o, off_SP, off_SS, ws_bytes;
     // backward workspace layout (gdn_backward)
     size_t b_status, b_qh, b_kh, b_vh, b_G, b_beta, b_la, b_o, b_ckpt, b_dO, b_dvh, b_dqp, b_dkp, b_dap, b_dbp,
         b_dnw, b_dconv, b_dA, b_ddt, bws_bytes;
@@ -33,9 +34,8 @@ struct gdn_plan_s {
 
 namespace {
 
-constexpr unsigned long long kWaitLimitNs = 2000ull * 1000 * 1000;      // 2 s per device-side wait
-constexpr unsigned long long kTestWaitLimitNs = 50ull * 1000 * 1000;   // the test hook's waits: 50 ms
-constexpr int kChunk = 64;  // tokens per block of the tensor path
+constexpr unsigned long long kWaitLimitNs = 2000ull * 1000 * 1000;  // 2 s per device-side wait
+constexpr int kChunk = 64;  // tokens per block of the fused path
 
 size_t esize(gdn_dtype t) { return t == GDN_DTYPE_F32 ? 4 : 2; }
 
@@ -64,6 +64,19 @@ EncodeTiledFn encode_fn() {
         return nullptr;
     }();
     return fn;
+}
+
+// [rows][128] fp16 row-major, loaded as {64, 128} boxes with the 128-byte swizzle.
+bool make_tile_map(CUtensorMap *m, void *base, unsigned long long rows, unsigned box_rows = 128) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {128, rows};
+    const cuuint64_t strides[1] = {128 * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Raw activations [B][T][H*d] (token stride tok_stride elements), 16-bit,
@@ -122,7 +135,7 @@ gdn_status gdn_plan(const gdn_config *cfg, gdn_plan_t *out, size_t *workspace_by
     if ((ts * static_cast<long long>(esize(c.in_dtype))) % 16 != 0) return GDN_ERR_INVALID_ARG;
     const long long Tp = (static_cast<long long>(c.T) + kBlk - 1) / kBlk * kBlk;
     const long long BH = static_cast<long long>(c.B) * c.H;
-    if (BH * Tp >= (1ll << 31)) return GDN_ERR_UNSUPPORTED;  // 32-bit row indices
+    if (BH * Tp >= (1ll << 31)) return GDN_ERR_UNSUPPORTED;  // TMA row coordinates are int32
 
     int dev = -1, major = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return GDN_ERR_NO_DEVICE; }
@@ -138,10 +151,10 @@ gdn_status gdn_plan(const gdn_config *cfg, gdn_plan_t *out, size_t *workspace_by
     p->cfg = c;
     p->device = dev;
     p->tensor = (c.in_dtype != GDN_DTYPE_F32) && d == 128 && !(c.flags & GDN_FLAG_FORCE_SIMT);
+    p->fused = p->tensor && (c.flags & GDN_FLAG_FUSED);
     p->Tp = static_cast<int>(Tp);
-    // tensor path: blocks of 64 tokens, cut into segments so that about one CTA per SM runs over
-    // all (b, h); the CUDA-core path keeps one chain per (b, h)
-    p->NB = static_cast<int>((static_cast<long long>(c.T) + kChunk - 1) / kChunk);
+    p->NB = static_cast<int>(p->fused ? (static_cast<long long>(c.T) + kChunk - 1) / kChunk : Tp / kBlk);
+    // segments: about one scan CTA per SM over all (b, h)
     {
         long long ns = sms / BH;
         if (ns < 1) ns = 1;
@@ -152,24 +165,35 @@ gdn_status gdn_plan(const gdn_config *cfg, gdn_plan_t *out, size_t *workspace_by
     p->tok_stride = ts;
     p->in_esize = esize(c.in_dtype);
     p->out_esize = esize(c.out_dtype);
+    p->inter_esize = p->tensor ? 2 : 4;
 
     const size_t A = 1024;
     const size_t nTok = static_cast<size_t>(BH) * Tp;
     const size_t act = nTok * d;
     size_t off = 0;
     p->off_status = off; off = align_up(off + 256, A);
-    if (p->tensor) {
+    if (p->fused) {
         const size_t mat = 128 * 128 * 4;
         p->off_SP = off; off = align_up(off + static_cast<size_t>(BH) * p->NS * 2 * mat, A);
         p->off_SS = off; off = align_up(off + static_cast<size_t>(BH) * p->NS * mat, A);
     } else {
-        p->off_qh = off; off = align_up(off + act * 4, A);
-        p->off_kh = off; off = align_up(off + act * 4, A);
-        p->off_vh = off; off = align_up(off + act * 4, A);
+        p->off_qh = off; off = align_up(off + act * p->inter_esize, A);
+        p->off_kh = off; off = align_up(off + act * p->inter_esize, A);
+        p->off_vh = off; off = align_up(off + act * p->inter_esize, A);
         p->off_G = off; off = align_up(off + nTok * 4, A);
         p->off_beta = off; off = align_up(off + nTok * 4, A);
         p->off_la = off; off = align_up(off + nTok * 4, A);
-        p->off_o = off; off = align_up(off + static_cast<size_t>(c.B) * c.T * c.H * d * 4, A);
+        if (p->tensor) {
+            p->off_W = off; off = align_up(off + act * 2, A);
+            p->off_U = off; off = align_up(off + act * 2, A);
+            p->off_Qt = off; off = align_up(off + act * 2, A);
+            p->off_Kt = off; off = align_up(off + act * 2, A);
+            p->off_Aqk = off; off = align_up(off + act * 2, A);
+            p->off_Zloc = off; off = align_up(off + static_cast<size_t>(BH) * p->NS * 128 * 256 * 4, A);
+            p->off_Sstart = off; off = align_up(off + static_cast<size_t>(BH) * p->NS * 128 * 128 * 4, A);
+        } else {
+            p->off_o = off; off = align_up(off + static_cast<size_t>(c.B) * c.T * c.H * d * 4, A);
+        }
     }
     p->ws_bytes = off;
 
@@ -233,7 +257,8 @@ gdn_status gdn_destroy(gdn_plan_t plan) {
 int gdn_launches_per_forward(gdn_plan_t plan) {
     if (!plan) return 0;
     if (!plan->tensor) return 3;          // prep, recurrence, output
-    return plan->NS > 1 ? 3 : 1;          // [transfer pass, combine,] output pass
+    if (plan->fused) return plan->NS > 1 ? 3 : 1;  // [transfer pass, combine,] output pass
+    return plan->NS > 1 ? 5 : 3;          // prep, chunk, [transfer, combine,] scan+output
 }
 
 int gdn_plan_uses_tensor_path(gdn_plan_t plan) { return plan && plan->tensor ? 1 : 0; }
@@ -244,9 +269,11 @@ size_t gdn_staging_bytes(gdn_plan_t plan) { return plan ? plan->staging_bytes : 
 
 int gdn_workspace_offsets(gdn_plan_t plan, size_t *offsets, int n) {
     if (!plan || !offsets || n <= 0) return 0;
-    const size_t all[10] = {plan->off_status, plan->off_qh, plan->off_kh, plan->off_vh, plan->off_G,
-                            plan->off_beta, plan->off_la, plan->off_o, plan->off_SP, plan->off_SS};
-    const int m = n < 10 ? n : 10;
+    const size_t all[17] = {plan->off_status, plan->off_qh, plan->off_kh, plan->off_vh, plan->off_G,
+                            plan->off_beta, plan->off_la, plan->off_W, plan->off_U, plan->off_Qt,
+                            plan->off_Kt, plan->off_Aqk, plan->off_o, plan->off_Zloc, plan->off_Sstart,
+                            plan->off_SP, plan->off_SS};
+    const int m = n < 17 ? n : 17;
     for (int i = 0; i < m; ++i) offsets[i] = all[i];
     return m;
 }
@@ -292,7 +319,7 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
     };
 
     const int rev = (c.flags & GDN_FLAG_REVERSE) ? 1 : 0;
-    if (plan->tensor) {
+    if (plan->fused) {
         // raw q, k, v boxes of 64 tokens + 3 of conv history; z and y boxes of 64 tokens; the
         // reverse scan's ragged last block stores only its T - 64 (NB - 1) live rows
         CUtensorMap maps[6];
@@ -329,7 +356,7 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
         fp.debug = (c.flags & GDN_FLAG_DEBUG_CHECKS) ? 1 : 0;
         fp.test_timeout = (c.flags & GDN_FLAG_TEST_WAIT_TIMEOUT) ? 1 : 0;
         fp.status = status;
-        fp.wait_limit_ns = fp.test_timeout ? kTestWaitLimitNs : kWaitLimitNs;
+        fp.wait_limit_ns = kWaitLimitNs;
         // The kernels after the first start with programmatic dependent launch (prologue overlapped
         // with the previous kernel), except when per-kernel events are recorded between them.
         const bool pdl = events == nullptr;
@@ -357,8 +384,70 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
     pp.status = status;
     pp.wait_limit_ns = kWaitLimitNs;
     pp.rev = rev;
-    if (!mark() || launch_prep(pp, in_type(c.in_dtype), false, s) != cudaSuccess) return GDN_ERR_CUDA;
-    {
+    if (plan->tensor) {
+        CUtensorMap rq, rk, rv;
+        if (!make_raw_map(&rq, in->q, c.B, c.T, c.H * d, plan->tok_stride, 64 + 3, 128) ||
+            !make_raw_map(&rk, in->k, c.B, c.T, c.H * d, plan->tok_stride, 64 + 3, 128) ||
+            !make_raw_map(&rv, in->v, c.B, c.T, c.H * d, plan->tok_stride, 64 + 3, 128))
+            return GDN_ERR_CUDA;
+        if (!mark() || launch_prep_tma(pp, in_type(c.in_dtype), rq, rk, rv, s) != cudaSuccess) return GDN_ERR_CUDA;
+    } else if (!mark() || launch_prep(pp, in_type(c.in_dtype), false, s) != cudaSuccess) {
+        return GDN_ERR_CUDA;
+    }
+
+    if (plan->tensor) {
+        const unsigned long long rows = static_cast<unsigned long long>(c.B) * c.H * plan->Tp;
+        CUtensorMap tmQ, tmK, tmV, tmW, tmU, tmQt, tmKt, tmAqk, tmAqkH;
+        if (!make_tile_map(&tmQ, ws + plan->off_qh, rows) || !make_tile_map(&tmK, ws + plan->off_kh, rows) ||
+            !make_tile_map(&tmV, ws + plan->off_vh, rows) || !make_tile_map(&tmW, ws + plan->off_W, rows) ||
+            !make_tile_map(&tmU, ws + plan->off_U, rows) || !make_tile_map(&tmQt, ws + plan->off_Qt, rows) ||
+            !make_tile_map(&tmKt, ws + plan->off_Kt, rows) || !make_tile_map(&tmAqk, ws + plan->off_Aqk, rows) ||
+            !make_tile_map(&tmAqkH, ws + plan->off_Aqk, rows, 64))  // Aqk's lower-right quadrant
+            return GDN_ERR_CUDA;
+        ChunkParams cp;
+        cp.g = in->g; cp.bg = in->b; cp.A_log = in->A_log; cp.dt_bias = in->dt_bias;
+        cp.G = G; cp.beta = beta; cp.log_alpha = la;
+        cp.T = c.T; cp.H = c.H;
+        cp.W = reinterpret_cast<__half *>(ws + plan->off_W);
+        cp.U = reinterpret_cast<__half *>(ws + plan->off_U);
+        cp.Qt = reinterpret_cast<__half *>(ws + plan->off_Qt);
+        cp.Kt = reinterpret_cast<__half *>(ws + plan->off_Kt);
+        cp.Aqk = reinterpret_cast<__half *>(ws + plan->off_Aqk);
+        cp.BH = c.B * c.H; cp.Tp = plan->Tp; cp.NB = plan->NB;
+        cp.status = status;
+        cp.wait_limit_ns = kWaitLimitNs;
+        cp.rev = rev;
+        // Kernels after the first start with programmatic dependent launch (prologue overlapped with
+        // the previous kernel's tail), except when per-kernel events are recorded between them.
+        const bool pdl = events == nullptr;
+        if (!mark() || launch_chunk(cp, tmK, tmV, tmQ, tmW, tmU, tmQt, tmAqk, tmAqkH, s, pdl) != cudaSuccess)
+            return GDN_ERR_CUDA;
+        ScanParams sp;
+        sp.G = G;
+        sp.Zloc = reinterpret_cast<float *>(ws + plan->off_Zloc);
+        sp.Sstart = reinterpret_cast<float *>(ws + plan->off_Sstart);
+        sp.z = in->z; sp.tok_stride = plan->tok_stride; sp.norm_w = in->norm_w; sp.y = y;
+        sp.out_kind = c.out_dtype == GDN_DTYPE_BF16 ? 0 : (c.out_dtype == GDN_DTYPE_F32 ? 1 : 2);
+        sp.eps = c.norm_eps;
+        sp.B = c.B; sp.T = c.T; sp.H = c.H; sp.Tp = plan->Tp; sp.NB = plan->NB; sp.NS = plan->NS; sp.Ls = plan->Ls;
+        sp.status = status;
+        sp.wait_limit_ns = kWaitLimitNs;
+        sp.test_wait_timeout = (c.flags & GDN_FLAG_TEST_WAIT_TIMEOUT) ? 1 : 0;
+        sp.s0 = s0;
+        sp.s_end = s_end;
+        sp.rev = rev;
+        sp.debug = (c.flags & GDN_FLAG_DEBUG_CHECKS) ? 1 : 0;
+        if (plan->NS > 1) {
+            if (!mark() || launch_transfer(sp, tmW, tmKt, tmU, s, pdl) != cudaSuccess) return GDN_ERR_CUDA;
+            if (!mark() || launch_combine(sp, s, pdl) != cudaSuccess) return GDN_ERR_CUDA;
+        }
+        CUtensorMap tmZ;
+        if (!make_raw_map(&tmZ, in->z, c.B, c.T, c.H * d, plan->tok_stride, kBlk, 128)) return GDN_ERR_CUDA;
+        if (!mark() || launch_scan_out(sp, in_type(c.in_dtype), tmW, tmQt, tmKt, tmAqk, tmAqkH, tmU, tmZ, s, pdl) != cudaSuccess)
+            return GDN_ERR_CUDA;
+        if (!mark()) return GDN_ERR_CUDA;
+        return GDN_OK;
+    } else {
         RecurParams rp;
         rp.qh = reinterpret_cast<const float *>(ws + plan->off_qh);
         rp.kh = reinterpret_cast<const float *>(ws + plan->off_kh);

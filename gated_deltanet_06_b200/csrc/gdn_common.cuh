@@ -120,11 +120,10 @@ struct AbortState {
 // most limit_ns of wall time.  Returns false when the limit ran out or another
 // thread of the CTA already aborted; the first thread to run out records
 // kStatusTimeout in *status.
-static __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile AbortState *ab,
-                                              int *status, uint64_t limit_ns) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile AbortState *ab,
+                                          int *status, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    uint32_t nap = 32;
     while (true) {
         if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
 #ifdef GDN_TRACE
@@ -136,10 +135,14 @@ static __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, vo
             atomicCAS(status, kStatusOk, kStatusTimeout);
             return false;
         }
-        // back off, so that a waiting warp takes few issue slots from the warps doing the work
-        __nanosleep(nap);
-        nap = nap < 256 ? 2 * nap : 256;
     }
+}
+
+// mbar_wait as one out-of-line copy, for kernels whose many call sites would otherwise grow the
+// code past what the instruction caches hold.
+static __device__ __noinline__ bool mbar_wait_ol(uint64_t *bar, uint32_t parity, volatile AbortState *ab,
+                                                 int *status, uint64_t limit_ns) {
+    return mbar_wait(bar, parity, ab, status, limit_ns);
 }
 
 // Like mbar_wait but blind to the CTA's abort flag: used on the way out, to let

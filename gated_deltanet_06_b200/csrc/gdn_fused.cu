@@ -397,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     umma_f16(tmem + TM::GB, sdesc_sw128(kq(s) + kk * 2048, 16384, 1024),
                              sdesc_sw128(tw + kk * 32, 16, 1024), id_mk64, kk > 0);
                 if (kOut) {
-                    if (!mbar_wait(&bars[B_PREPV], j & 1, ab, p.status, lim)) return false;
+                    if (!mbar_wait_ol(&bars[B_PREPV], j & 1, ab, p.status, lim)) return false;
                     tc_fence_after();
                 }
 #pragma unroll 1
@@ -418,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 while (gram_next < n && tready_seen >= gram_next - 1) {
                     const int j = gram_next, s = j & 1;
                     if (block) {
-                        if (!mbar_wait(&bars[B_PREP + s], (j >> 1) & 1, ab, p.status, lim)) return false;
+                        if (!mbar_wait_ol(&bars[B_PREP + s], (j >> 1) & 1, ab, p.status, lim)) return false;
                     } else if (!mbar_try_wait(&bars[B_PREP + s], (j >> 1) & 1)) {
                         return true;
                     }
@@ -433,24 +433,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return true;
             };
             bool ok = try_gram(true);
-            ok = ok && mbar_wait(&bars[B_TREADY], 0, ab, p.status, lim);
+            ok = ok && mbar_wait_ol(&bars[B_TREADY], 0, ab, p.status, lim);
             if (ok) {
                 tready_seen = 0;
                 tc_fence_after();
                 ok = wt_ut(0);
             }
             if (ok && p.test_timeout) {
-                // test hook: a wait on a barrier nothing arrives on, with tensor-core work in flight
-                mbar_wait(&bars[B_TEST], 0, ab, p.status, lim);
+                // test hook: a wait on a barrier nothing arrives on (bounded, ~50 ms), with tensor-core
+                // work and raw loads in flight; the drains at the end let them finish
+                mbar_wait_ol(&bars[B_TEST], 0, ab, p.status, 50ull * 1000 * 1000);
                 ok = false;
             }
             ok = ok && try_gram(false);
             for (int i = 0; ok && i < n; ++i) {
                 const int s = i & 1;
                 FTRACE(i, 0);
-                ok = mbar_wait(&bars[B_UTD + s], (i >> 1) & 1, ab, p.status, lim) &&
-                     mbar_wait(&bars[B_N16], i & 1, ab, p.status, lim) &&
-                     (!kOut || i < 2 || mbar_wait(&bars[B_OFREE + s], ((i >> 1) - 1) & 1, ab, p.status, lim));
+                ok = mbar_wait_ol(&bars[B_UTD + s], (i >> 1) & 1, ab, p.status, lim) &&
+                     mbar_wait_ol(&bars[B_N16], i & 1, ab, p.status, lim) &&
+                     (!kOut || i < 2 || mbar_wait_ol(&bars[B_OFREE + s], ((i >> 1) - 1) & 1, ab, p.status, lim));
                 if (!ok) break;
                 FTRACE(i, 1);
                 tc_fence_after();
@@ -472,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma_commit(&bars[B_DELTA]);
                 FTRACE(i, 2);
                 ok = try_gram(false);
-                ok = ok && mbar_wait(&bars[B_E16], i & 1, ab, p.status, lim);
+                ok = ok && mbar_wait_ol(&bars[B_E16], i & 1, ab, p.status, lim);
                 if (!ok) break;
                 FTRACE(i, 3);
                 tc_fence_after();
@@ -499,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // the next block's W^T and U^T (its Gram first, if it is still to be issued); U^T goes
                     // to the Delta^T columns, whose fp16 Delta the state update above has read
                     ok = (gram_next > i + 1 || try_gram(true)) &&
-                         mbar_wait(&bars[B_TREADY + (s ^ 1)], ((i + 1) >> 1) & 1, ab, p.status, lim);
+                         mbar_wait_ol(&bars[B_TREADY + (s ^ 1)], ((i + 1) >> 1) & 1, ab, p.status, lim);
                     if (!ok) break;
                     tready_seen = i + 1;
                     FTRACE(i, 6);
@@ -560,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint8_t *kq = sm + Ly::KQ + s * 32768;
             const bool ragged = (c + 1) * kC > p.T;
             if (pt == 0) FTRACE(i, 8);
-            if (i >= 2) ok = mbar_wait(&bars[B_FREE + s], ((i >> 1) - 1) & 1, ab, p.status, lim);
+            if (i >= 2) ok = mbar_wait_ol(&bars[B_FREE + s], ((i >> 1) - 1) & 1, ab, p.status, lim);
 #pragma unroll 1
             for (int w = 0; w < NT; ++w) {
                 // destination: output pass k -> KQ rows 0-63, q -> KQ rows 64+, v -> V tile;
@@ -572,10 +573,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     dst = sm + Lay<true>::V;
                     drows = 64;
                     doff = 0;
-                    if (i >= 1) ok = ok && mbar_wait(&bars[B_VFREE], (i - 1) & 1, ab, p.status, lim);
+                    if (i >= 1) ok = ok && mbar_wait_ol(&bars[B_VFREE], (i - 1) & 1, ab, p.status, lim);
                 }
                 const int l = i * NT + w, sl = l % NSL;
-                ok = ok && mbar_wait(&bars[B_RAW + sl], (l / NSL) & 1, ab, p.status, lim);
+                ok = ok && mbar_wait_ol(&bars[B_RAW + sl], (l / NSL) & 1, ab, p.status, lim);
                 ok = group_all(NB_PREP, 128, ok);
                 if (!ok) break;
                 if (pt == 0) FTRACE(i, 9 + 2 * w);
@@ -680,7 +681,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // ---- gates: log alpha = -exp(A_log) softplus(g + dt_bias), beta = sigmoid(b), G = inclusive
             //      cumulative sum of log alpha over the block (padding rows: 0, 0), and the column factors
             //      e^(G_m - G_j) of the split decay (m the last row of j's 16-row group)
-            ok = group_all(NB_UT, 128, j < 2 || mbar_wait(&bars[B_UTD + s], ((j >> 1) - 1) & 1, ab, p.status, lim));
+            ok = group_all(NB_UT, 128, j < 2 || mbar_wait_ol(&bars[B_UTD + s], ((j >> 1) - 1) & 1, ab, p.status, lim));
             if (!ok) break;
             {
                 float cs = 0.0f, be = 0.0f;
@@ -720,9 +721,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ut == 0) FTRACE(j, 17);
             // ---- L and Aqk rows; Qt
             ok = group_all(NB_UT, 128,
-                           mbar_wait(&bars[B_PREP + s], (j >> 1) & 1, ab, p.status, lim) &&
-                               mbar_wait(&bars[B_GRAM], j & 1, ab, p.status, lim) &&
-                               (j < 2 || mbar_wait(&bars[B_WT + s], ((j >> 1) - 1) & 1, ab, p.status, lim)));
+                           mbar_wait_ol(&bars[B_PREP + s], (j >> 1) & 1, ab, p.status, lim) &&
+                               mbar_wait_ol(&bars[B_GRAM], j & 1, ab, p.status, lim) &&
+                               (j < 2 || mbar_wait_ol(&bars[B_WT + s], ((j >> 1) - 1) & 1, ab, p.status, lim)));
             if (!ok) break;
             if (ut == 0) FTRACE(j, 18);
             tc_fence_after();
@@ -834,7 +835,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     src = p.SS + ((static_cast<size_t>(bh) * p.NS + seg) * kD + row) * kD;
                 }
             }
-            ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_GATE], 0, ab, p.status, lim));
+            ok = __all_sync(0xffffffffu, mbar_wait_ol(&bars[B_GATE], 0, ab, p.status, lim));
             const float gC = ok ? __expf(fminf(gate[kC - 1], 0.0f)) : 0.0f;
 #pragma unroll 1
             for (int ch = 0; ch < 4; ++ch) {
@@ -865,9 +866,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int s = i & 1;
             if (!isP) {
                 // ---- block i's W^T (lanes = d_k) into its slot's tile, and Kt = diag(e^(G_C - G) / |k'|) K'
-                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_WT + s], (i >> 1) & 1, ab, p.status, lim) &&
-                                                 mbar_wait(&bars[B_PREP + s], (i >> 1) & 1, ab, p.status, lim) &&
-                                                 mbar_wait(&bars[B_GATE + s], (i >> 1) & 1, ab, p.status, lim));
+                ok = __all_sync(0xffffffffu, mbar_wait_ol(&bars[B_WT + s], (i >> 1) & 1, ab, p.status, lim) &&
+                                                 mbar_wait_ol(&bars[B_PREP + s], (i >> 1) & 1, ab, p.status, lim) &&
+                                                 mbar_wait_ol(&bars[B_GATE + s], (i >> 1) & 1, ab, p.status, lim));
                 if (!ok) break;
                 if (tid == 32 * W_CH) FTRACE(i, 24);
                 tc_fence_after();
@@ -892,7 +893,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) mbar_arrive(&bars[B_UTD + s]);
             }
             // ---- Delta^T -> E16 = fp16(-Delta^T), written over the first half of its columns
-            ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_DELTA], i & 1, ab, p.status, lim));
+            ok = __all_sync(0xffffffffu, mbar_wait_ol(&bars[B_DELTA], i & 1, ab, p.status, lim));
             if (!ok) break;
             if (tid == 32 * W_CH) FTRACE(i, 25);
             tc_fence_after();
@@ -912,14 +913,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[B_E16]);
             if (tid == 32 * W_CH) FTRACE(i, 26);
-            ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_STATE], i & 1, ab, p.status, lim));
+            ok = __all_sync(0xffffffffu, mbar_wait_ol(&bars[B_STATE], i & 1, ab, p.status, lim));
             if (!ok) break;
             if (tid == 32 * W_CH) FTRACE(i, 27);
             if (i + 1 < n) {
                 // one read of the state: its fp16 copy for block i + 1's products, and the state
                 // decayed by block i + 1's total decay for its update
                 const int s1 = (i + 1) & 1;
-                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_GATE + s1], ((i + 1) >> 1) & 1, ab, p.status, lim));
+                ok = __all_sync(0xffffffffu, mbar_wait_ol(&bars[B_GATE + s1], ((i + 1) >> 1) & 1, ab, p.status, lim));
                 if (!ok) break;
                 const float gC = __expf(fminf(gate[s1 * 256 + kC - 1], 0.0f));
                 tc_fence_after();
@@ -987,7 +988,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; ok && i < n; ++i) {
             const int c = c0 + i, s = i & 1;
             const uint32_t tO = tmem + lb + Tm<true>::O + s * 64;
-            ok = group_all(NB_X, 128, mbar_wait(&bars[B_OFULL + s], (i >> 1) & 1, ab, p.status, lim));
+            ok = group_all(NB_X, 128, mbar_wait_ol(&bars[B_OFULL + s], (i >> 1) & 1, ab, p.status, lim));
             if (!ok) break;
             if (et == 0) FTRACE(i, 29);
             tc_fence_after();
@@ -1019,7 +1020,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float4 r4 = *reinterpret_cast<const float4 *>(red + et * 4);
                 rns[et] = rsqrtf((r4.x + r4.y + r4.z + r4.w) * (1.0f / 128.0f) + p.eps);
             }
-            ok = group_all(NB_X, 128, mbar_wait(&bars[B_Z], i & 1, ab, p.status, lim));  // (also publishes rns)
+            ok = group_all(NB_X, 128, mbar_wait_ol(&bars[B_Z], i & 1, ab, p.status, lim));  // (also publishes rns)
             if (!ok) break;
             if (et == 0) {
                 FTRACE(i, 30);

@@ -11,20 +11,48 @@
 
 namespace gdn {
 
-// Raise a kernel's dynamic shared-memory limit once per device.  Safe to call from
-// several host threads (a repeated call only repeats the same attribute set).
+// Unique id (cuCtxGetId) of the calling thread's current CUDA context; ids are never reused
+// within a process, so a context created by a cudaDeviceReset and a later call gets a new one.
+// False when no context is current or the driver cannot say.
+inline bool current_context_id(unsigned long long *id) {
+    typedef CUresult (*GetCurrentFn)(CUcontext *);
+    typedef CUresult (*GetIdFn)(CUcontext, unsigned long long *);
+    static const auto lookup = [](const char *name) -> void * {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        return p;
+    };
+    static const GetCurrentFn get_current = reinterpret_cast<GetCurrentFn>(lookup("cuCtxGetCurrent"));
+    static const GetIdFn get_id = reinterpret_cast<GetIdFn>(lookup("cuCtxGetId"));
+    if (!get_current || !get_id) return false;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per CUDA context (the attribute belongs to
+// the context's copy of the kernel, so a context re-created by cudaDeviceReset needs it again).
+// Safe to call from several host threads (a repeated call only repeats the same attribute set).
 constexpr int kMaxDevices = 64;
 struct SmemOnce {
-    std::atomic<int> done[kMaxDevices];  // zero-initialised: objects of this type are static
-};
+    std::atomic<unsigned long long> ctx[kMaxDevices];  // context id it was set in; zero-initialised
+};                                                      // (objects of this type are static)
 template <typename K>
 inline cudaError_t raise_smem_once(SmemOnce &once, K kernel, int bytes) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < kMaxDevices && once.done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    unsigned long long id = 0;
+    const bool have_id = current_context_id(&id) && id != 0;
+    const bool tracked = have_id && dev >= 0 && dev < kMaxDevices;
+    if (tracked && once.ctx[dev].load(std::memory_order_acquire) == id) return cudaSuccess;
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) once.done[dev].store(1, std::memory_order_release);
+    if (e == cudaSuccess && tracked) once.ctx[dev].store(id, std::memory_order_release);
     return e;
 }
 
@@ -68,8 +96,62 @@ struct PrepParams {
     int rev;                       // reverse scan: internal token t is input token T-1-t
 };
 cudaError_t launch_prep(const PrepParams &p, InType in, bool out_f16, cudaStream_t s);
-// Tensor path (16-bit inputs, d = 128): the fused transfer and output passes over
-// segments of Ls blocks of 64 tokens, and the combine of the segment states.
+// Tensor path (16-bit inputs, d = 128): raw tiles staged by TMA through the
+// 3-D maps tmq/tmk/tmv over [B][T][H*d] (box {64, 131, 1}).
+cudaError_t launch_prep_tma(const PrepParams &p, InType in, const CUtensorMap &tmq, const CUtensorMap &tmk,
+                            const CUtensorMap &tmv, cudaStream_t s);
+
+// Intra-block UT transform on tensor cores (d = 128, fp16 operands).  It
+// also evaluates the gates of its block from g, b (and writes G, beta, log
+// alpha for the scan and the stage tests).
+struct ChunkParams {
+    const float *g, *bg;            // [B][T][H]
+    const float *A_log, *dt_bias;   // [H]
+    float *G, *beta, *log_alpha;    // [BH][Tp]
+    int T, H;
+    __half *W, *U, *Qt, *Kt, *Aqk;  // [BH][Tp][128]
+    int BH, Tp, NB;
+    int *status;
+    unsigned long long wait_limit_ns;
+    int rev;                        // reverse scan: block row t holds the gates of input token T-1-t
+};
+cudaError_t launch_chunk(const ChunkParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                         const CUtensorMap &tmQ, const CUtensorMap &tmW, const CUtensorMap &tmU,
+                         const CUtensorMap &tmQt, const CUtensorMap &tmAqk, const CUtensorMap &tmAqkH,
+                         cudaStream_t s, bool pdl);  // Kt is written with plain coalesced stores
+
+// Inter-block state scan on tensor cores (d = 128), parallel over segments of
+// Ls blocks: pass A (transfer), combine, pass C (outputs + fused output step).
+struct ScanParams {
+    const float *G;          // [BH][Tp]
+    float *Zloc;             // [BH][NS][128][256]: S_loc^T | P^T per segment (pass A)
+    float *Sstart;           // [BH][NS][128][128]: S^T at each segment start (combine)
+    const void *z;           // [B][T][H][128], token stride tok_stride
+    long long tok_stride;
+    const float *norm_w;     // [128]
+    void *y;                 // [B][T][H][128]
+    int out_kind;            // 0 bf16, 1 f32, 2 f16
+    float eps;
+    int B, T, H, Tp, NB, NS, Ls;
+    int *status;
+    unsigned long long wait_limit_ns;
+    int test_wait_timeout;
+    const float *s0;         // [BH][128 (d_v)][128 (d_k)] state before token 0, or null (zero)
+    float *s_end;            // [BH][128][128] state after token T-1, or null (not wanted)
+    int rev;                 // reverse scan: block row t is z / y token T-1-t
+    int debug;               // check that every output value is finite (status word)
+};
+// pdl: launch with programmatic stream serialization (see launch_k).
+cudaError_t launch_transfer(const ScanParams &p, const CUtensorMap &tmW, const CUtensorMap &tmKt,
+                            const CUtensorMap &tmU, cudaStream_t s, bool pdl);
+cudaError_t launch_combine(const ScanParams &p, cudaStream_t s, bool pdl);
+cudaError_t launch_scan_out(const ScanParams &p, InType zt, const CUtensorMap &tmW, const CUtensorMap &tmQt,
+                            const CUtensorMap &tmKt, const CUtensorMap &tmAqk, const CUtensorMap &tmAqkH,
+                            const CUtensorMap &tmU, const CUtensorMap &tmZ, cudaStream_t s, bool pdl);
+
+// Fused tensor path (GDN_FLAG_FUSED; 16-bit inputs, d = 128): the transfer and output passes
+// over segments of Ls blocks of 64 tokens, each recomputing the preparation and the UT transform
+// from the raw inputs, and the combine of the segment states.
 struct FusedParams {
     const float *g, *bg;                      // [B][T][H]
     const float *conv_q, *conv_k, *conv_v;    // [H*128][4]

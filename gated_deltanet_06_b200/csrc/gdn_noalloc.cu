@@ -21,9 +21,13 @@
 // device status word) at the start of each call.
 //
 // In host code the array's name is only a host-side stand-in, so its device
-// address is looked up with cudaGetSymbolAddress -- once per device, with that
-// device current, on the first call made on that device -- and cached.  That
-// first call should therefore come before any stream capture.
+// address is looked up with cudaGetSymbolAddress and cached per device together
+// with the unique id of the CUDA context it belongs to.  A later call in another
+// context (after cudaDeviceReset, or from a thread with another context current)
+// sees a different id and looks the address up again, since the array's address
+// in a new context need not be the old one.  The first call on a device, and the
+// first after a reset, should come before any stream capture.
+#include <cuda.h>
 #include <cuda_fp16.h>
 
 #include <mutex>
@@ -36,23 +40,34 @@ namespace {
 static __device__ __align__(256) unsigned char g_gdn_noalloc_scratch[GDN_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
-void *g_scratch_ptr[kMaxDevices] = {};
+struct ScratchEntry {
+    unsigned long long ctx_id;  // cuCtxGetId of the context `ptr` belongs to
+    void *ptr;                  // nullptr: not looked up in any context yet
+};
+ScratchEntry g_scratch[kMaxDevices] = {};
 std::mutex g_scratch_mu;
 
-// Device address of the scratch array on the current device (looked up once per device).
+// Device address of the scratch array in the current device's current context.
 gdn_status scratch_address(void **out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GDN_ERR_CUDA;
+    unsigned long long id = 0;
+    bool have_id = gdn::current_context_id(&id);
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_gdn_noalloc_scratch) != cudaSuccess || !p) {
-            cudaGetLastError();
-            return GDN_ERR_CUDA;
-        }
-        g_scratch_ptr[dev] = p;
+    ScratchEntry &e = g_scratch[dev];
+    if (have_id && e.ptr && e.ctx_id == id) {
+        *out = e.ptr;
+        return GDN_OK;
     }
-    *out = g_scratch_ptr[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_gdn_noalloc_scratch) != cudaSuccess || !p) {
+        cudaGetLastError();
+        return GDN_ERR_CUDA;
+    }
+    if (!have_id) have_id = gdn::current_context_id(&id);  // the lookup made the device's context current
+    e.ctx_id = have_id ? id : 0;
+    e.ptr = have_id ? p : nullptr;                      // without an id nothing is cached
+    *out = p;
     return GDN_OK;
 }
 

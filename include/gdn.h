@@ -89,9 +89,19 @@ typedef enum {
                                             is a bidirectional Mamba2 block); a bidirectional layer is
                                             a forward and a reverse call on the same or separate
                                             parameters, combined by the caller. */
-#define GDN_FLAG_TEST_WAIT_TIMEOUT 0x100u /* test hook: the scan kernel waits on a barrier nothing
-                                            arrives on, gives up after ~50 ms and reports
-                                            GDN_ERR_TIMEOUT in the status word */
+#define GDN_FLAG_FUSED 0x8u              /* tensor path only (ignored elsewhere): the fused forward,
+                                            which recomputes the prep and the 64-token UT transform
+                                            on chip in two persistent passes (segment transfer,
+                                            then scan with the output step) instead of writing the
+                                            q^, k^, v^, W, U, Qt, Kt, Aqk intermediates to HBM.
+                                            Same results within the tensor path's tolerance; fewer
+                                            HBM bytes, but slower on B200 at the documented sizes
+                                            (the fused passes are issue-bound), so not the default */
+#define GDN_FLAG_TEST_WAIT_TIMEOUT 0x100u /* test hook (tensor path): mid-pipeline, with TMA loads
+                                            and tensor-core work in flight, the last kernel waits
+                                            on a barrier nothing arrives on, gives up after ~50 ms,
+                                            reports GDN_ERR_TIMEOUT in the status word, lets the
+                                            work in flight finish and exits; y is then undefined */
 
 typedef struct {
     int B, T, H, d_k, d_v;   /* d_k == d_v, 64 or 128; B, H >= 1; T >= 1 */
@@ -180,9 +190,11 @@ gdn_status gdn_forward_host(gdn_plan_t plan, const gdn_inputs *in_host, void *y_
  * gdn_forward.  Errors: INVALID_ARG (null plan, inputs or y, or the checks of
  * gdn_forward), UNSUPPORTED when the plan's workspace is larger than
  * GDN_NOALLOC_SCRATCH_BYTES (nothing is enqueued), CUDA if the array's device
- * address cannot be looked up.  The first call on a device looks that address
- * up (cudaGetSymbolAddress, with the device current) and caches it, so make
- * that first call before any stream capture.  All calls on a device share the
+ * address cannot be looked up.  The first call in a CUDA context looks that
+ * address up (cudaGetSymbolAddress) and caches it with the context's unique
+ * id; a call in another context (after cudaDeviceReset, say) looks it up
+ * again.  Make the first call on a device, and the first after a reset,
+ * before any stream capture.  All calls on a device share the
  * array: calls that may overlap on the GPU (unordered streams, several host
  * threads) race on it; calls on one stream are safe.  The array keeps the last
  * call's contents; the only value that must start at zero, the device status
@@ -238,7 +250,9 @@ gdn_status gdn_get_device_status(gdn_plan_t plan, void *workspace, gdn_stream_t 
 
 /* Number of kernel launches one gdn_forward enqueues for this plan: 3 or 5 on
  * the tensor path (prep, UT transform, [segment transfer, combine,] scan with
- * the output step), 3 on the CUDA-core path (prep, recurrence, output). */
+ * the output step), 1 or 3 on the fused tensor path ([transfer pass,
+ * combine,] output pass), 3 on the CUDA-core path (prep, recurrence,
+ * output). */
 int gdn_launches_per_forward(gdn_plan_t plan);
 
 /* 1 if the plan runs the tensor-core (tcgen05) path, 0 for the fp32 CUDA-core path. */
@@ -260,8 +274,13 @@ int gdn_plan_segments(gdn_plan_t plan);
  *     quadrant in each 128-row block is never written), 12 o ([B][T][H][d_v] fp32 before the output norm; CUDA-core
  *     path only, else 0), 13 per-segment [S_loc^T | P^T] ([B][H][NS][128][256]
  *     fp32) and 14 segment start states S^T ([B][H][NS][128][128] fp32)
- *     (tensor path only, else 0).
- * Returns the number of offsets written (15 at most). */
+ *     (tensor path without GDN_FLAG_FUSED only, else 0),
+ *   15 per-segment [S_loc | P] ([B][H][NS][2][128][128] fp32, S_end =
+ *     S_start P + S_loc with the state's d_k index first) and 16 segment
+ *     start states ([B][H][NS][128][128] fp32, the same orientation)
+ *     (GDN_FLAG_FUSED plans only, else 0; on those plans 1-14 are 0: the
+ *     fused forward keeps its other intermediates on chip).
+ * Returns the number of offsets written (17 at most). */
 int gdn_workspace_offsets(gdn_plan_t plan, size_t *offsets, int n);
 
 /* Free a plan (host memory only).  NULL is accepted. */

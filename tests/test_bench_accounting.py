@@ -39,35 +39,68 @@ def test_headline_roofline_time():
 
 
 @pytest.mark.parametrize("name,expected_bytes", [
-    ("transfer", 2 * 128 * 2 + 8),          # raw k, v bf16 in; g, b fp32 in
-    ("out", 4 * 128 * 2 + 8 + 128 * 2),     # raw q, k, v, z bf16 in; g, b fp32 in; y bf16 out
+    ("prep", 3 * 128 * 2 + 3 * 128 * 2),    # raw q, k, v bf16 in; q^, k^, v^ fp16 out
+    # q^ k^ v^ fp16 + g b in; W U Qt Kt fp16 out, the 96 live Aqk columns per row, G beta log-alpha
+    ("chunk", 3 * 128 * 2 + 8 + 4 * 128 * 2 + 96 * 2 + 12),
+    ("transfer", 3 * 128 * 2),              # W, U, Kt fp16 in
+    ("scan", 4 * 128 * 2 + 96 * 2 + 128 * 2 + 128 * 2),  # W U Qt Kt, Aqk, z in; y out
     ("combine", 0),                         # per-segment states only
+    ("fused_transfer", 2 * 128 * 2 + 8),    # raw k, v bf16 in; g, b fp32 in
+    ("fused_out", 4 * 128 * 2 + 8 + 128 * 2),  # raw q, k, v, z bf16 in; g, b fp32 in; y bf16 out
+    ("fused_combine", 0),
 ])
 def test_kernel_bytes(name, expected_bytes):
     assert bench.kernel_work_per_token_head(name, 128, 2, 2)[0] == expected_bytes
 
 
-def test_kernel_flops_per_64_token_block():
+def test_fused_kernel_flops_per_64_token_block():
     C, d = 64, 128
     gram = 2 * 128 * C * d          # [K; Q] K^T: M = 128 stacked rows, N = C, K = d
     wu = 2 * (2 * 128 * C * C)      # W^T = K^T T_w^T and U^T = V^T T_u^T: M = d, N = K = C
     delta = 2 * 128 * C * d         # Delta^T = U^T + N W^T: M = d_v, N = C, K = d_k
     state = 2 * 128 * 128 * C       # N += E Kt: M = d_v, N = d_k, K = C
     o1, o2 = 2 * 128 * C * d, 2 * 128 * C * C
-    assert bench.kernel_work_per_token_head("out", d, 2, 2)[1] * C == gram + wu + delta + state + o1 + o2
-    assert bench.kernel_work_per_token_head("transfer", d, 2, 2)[1] * C == gram + wu + 2 * (delta + state)
+    assert bench.kernel_work_per_token_head("fused_out", d, 2, 2)[1] * C == gram + wu + delta + state + o1 + o2
+    assert bench.kernel_work_per_token_head("fused_transfer", d, 2, 2)[1] * C == gram + wu + 2 * (delta + state)
     # the output pass's products are exactly the method's chunk count per token-head
-    assert bench.kernel_work_per_token_head("out", d, 2, 2)[1] == bench.path_flops_per_token_head(d)
+    assert bench.kernel_work_per_token_head("fused_out", d, 2, 2)[1] == bench.path_flops_per_token_head(d)
+
+
+def test_tensor_path_kernel_flops_per_128_token_block():
+    C, d = 128, 128
+    # chunk: K K^T and Q K^T (C x C x d each), W = T (beta K) and U = T (beta V) (C x C x d each)
+    assert bench.kernel_work_per_token_head("chunk", d, 2, 2)[1] * C == 4 * 2 * C * C * d
+    # scan: W S^T and Qt S^T (C x d x d), Kt^T Delta (d x d x C), Aqk Delta (C x C x d)
+    assert bench.kernel_work_per_token_head("scan", d, 2, 2)[1] * C == 4 * 2 * C * d * d
+    # transfer: W [S | P]^T (C x 2d x d) and Kt^T Delta with N = 2d
+    assert bench.kernel_work_per_token_head("transfer", d, 2, 2)[1] * C == 2 * 2 * C * 2 * d * d
 
 
 def test_dominant_launch_units():
     class P:
         segments = 12
     w = gdn_inputs.HEADLINE
-    assert bench.launch_units("out", w, P) == w.B * w.H * w.T
+    assert bench.launch_units("scan", w, P) == w.B * w.H * w.T
+    assert bench.launch_units("fused_out", w, P) == w.B * w.H * w.T
+    nb = -(-w.T // 128)
+    ls = -(-nb // 12)
+    assert bench.launch_units("transfer", w, P) == w.H * 11 * ls * 128
     nb = -(-w.T // 64)
     ls = -(-nb // 12)
-    assert bench.launch_units("transfer", w, P) == w.H * 11 * ls * 64
+    assert bench.launch_units("fused_transfer", w, P) == w.H * 11 * ls * 64
+
+
+def test_kernel_names_per_path():
+    class P:
+        uses_tensor_path = True
+        segments = 3
+    assert bench.kernel_names(P) == ("prep", "chunk", "transfer", "combine", "scan")
+    assert bench.kernel_names(P, fused=True) == ("fused_transfer", "fused_combine", "fused_out")
+    P.segments = 1
+    assert bench.kernel_names(P) == ("prep", "chunk", "scan")
+    assert bench.kernel_names(P, fused=True) == ("fused_out",)
+    P.uses_tensor_path = False
+    assert bench.kernel_names(P) == ("prep", "recurrence", "output")
 
 
 def test_path_roofline_fraction():
@@ -80,9 +113,9 @@ def test_path_roofline_fraction():
 
 
 def test_traffic_is_dropped_when_the_kernel_source_changed(monkeypatch, tmp_path):
-    real = bench.kernel_source_sha("out")
-    monkeypatch.setattr(bench, "kernel_source_sha", lambda name: "0" * 16 if name == "out" else real)
-    assert bench.ncu_traffic("out", "wan21_480x832_81f") is None
+    real = bench.kernel_source_sha("scan")
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda name: "0" * 16 if name == "scan" else real)
+    assert bench.ncu_traffic("scan", "wan21_480x832_81f") is None
 
 
 def test_sample_text():

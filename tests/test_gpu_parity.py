@@ -202,21 +202,38 @@ def test_invalid_arguments_are_rejected_before_launch():
             gdn.Plan(args["B"], args["T"], args["H"], args["d"], gdn.DTYPE_BF16, tok_stride=kw.get("tok_stride", 0))
 
 
-def test_bounded_wait_timeout_reports_status_and_context_survives():
-    # the scan kernel's producer waits on a barrier nothing arrives on; the
-    # wait gives up after ~50 ms, the kernel exits cleanly and the status
-    # word reports the timeout; the next forward on the same context is exact
+@pytest.mark.parametrize("fused", [False, True])
+def test_bounded_wait_timeout_mid_pipeline(fused):
+    # the last kernel's producer, mid-pipeline with TMA loads and tensor-core work in flight, waits
+    # on a barrier nothing arrives on; the wait gives up after ~50 ms, every thread leaves its loop,
+    # the work in flight is drained, the status word reports the timeout, and the next forward on
+    # the same context is exact.  Each drain waits only for the last phase started on its barrier:
+    # a drain that picked the wrong phase would sit out its whole 2 s limit, so the forward must
+    # come back well inside that.  B = 2, H = 12, T = 1000 gives segments of 2 blocks on the tensor
+    # path, so the next block's loads are in flight when the wait starts.
     import torch
     import gated_deltanet_06_b200 as gdn
-    inp = gdn_inputs.make_inputs(1, 300, 2, 128, "bf16", 0.0, seed=27)
+    B, T, H = 2, 1000, 12
+    inp = gdn_inputs.make_inputs(B, T, H, 128, "bf16", 0.0, seed=27)
     t = torch_inputs(inp)
-    plan = gdn.Plan(1, 300, 2, 128, gdn.DTYPE_BF16, flags=gdn.FLAG_TEST_WAIT_TIMEOUT)
+    base = gdn.FLAG_FUSED if fused else 0
+    plan = gdn.Plan(B, T, H, 128, gdn.DTYPE_BF16, flags=base | gdn.FLAG_TEST_WAIT_TIMEOUT)
+    if not fused:
+        assert plan.segments > 1 and -(-T // 128) >= 2 * (plan.segments - 1)
     ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device="cuda")
+    gdn.forward(**t, plan=plan, workspace=ws)  # warm-up: module load, attribute set-up
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
     gdn.forward(**t, plan=plan, workspace=ws)
-    s = torch.cuda.current_stream().cuda_stream
-    assert plan.device_status(ws.data_ptr(), s) == gdn.ERR_TIMEOUT
-    assert plan.device_status(ws.data_ptr(), s) == gdn.OK  # reading clears it
-    check_parity(run_gdn(inp), _oracle(inp), "bf16", "bf16", "after timeout")
+    e1.record(s)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    assert 45.0 <= ms < 1000.0, ms
+    assert plan.device_status(ws.data_ptr(), s.cuda_stream) == gdn.ERR_TIMEOUT
+    assert plan.device_status(ws.data_ptr(), s.cuda_stream) == gdn.OK  # reading clears it
+    check_parity(run_gdn(inp, flags=base), _oracle(inp), "bf16", "bf16", "after timeout")
 
 
 @pytest.mark.parametrize("simt", [False, True])
