@@ -384,6 +384,7 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
     pp.status = status;
     pp.wait_limit_ns = kWaitLimitNs;
     pp.rev = rev;
+    pp.debug = (c.flags & GDN_FLAG_DEBUG_CHECKS) ? 1 : 0;
     if (plan->tensor) {
         CUtensorMap rq, rk, rv;
         if (!make_raw_map(&rq, in->q, c.B, c.T, c.H * d, plan->tok_stride, 64 + 3, 128) ||
@@ -417,6 +418,7 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
         cp.status = status;
         cp.wait_limit_ns = kWaitLimitNs;
         cp.rev = rev;
+        cp.debug = (c.flags & GDN_FLAG_DEBUG_CHECKS) ? 1 : 0;
         // Kernels after the first start with programmatic dependent launch (prologue overlapped with
         // the previous kernel's tail), except when per-kernel events are recorded between them.
         const bool pdl = events == nullptr;

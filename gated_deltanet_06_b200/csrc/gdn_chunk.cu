@@ -139,6 +139,11 @@ __global__ void __launch_bounds__(256, 2)
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const size_t row0 = static_cast<size_t>(bh) * p.Tp + static_cast<size_t>(blk) * kBlk;
     const int y0 = static_cast<int>(row0);
+    // debug: the block's rows inside the [BH][Tp] gate and tile arrays, and its tokens inside T
+    // rounded up to whole blocks (the gates of token t < T are read at [B][T][H])
+    if (!debug_in_bounds(p.debug, row0, kBlk, static_cast<size_t>(p.BH) * p.Tp, p.status) ||
+        !debug_in_bounds(p.debug, static_cast<size_t>(blk) * kBlk, kBlk, static_cast<size_t>(p.NB) * kBlk, p.status))
+        return;
 
     if (tid == 0) {
         mbar_init(bar_load, 1);
@@ -172,8 +177,8 @@ __global__ void __launch_bounds__(256, 2)
         const int bb = bh / p.H, hh = bh - bb * p.H;
         const int t = blk * kBlk + r;
         float la = 0.0f, be = 0.0f;
-        if (t < p.T) {
-            const size_t gi = (static_cast<size_t>(bb) * p.T + (p.rev ? p.T - 1 - t : t)) * p.H + hh;
+        const size_t gi = t < p.T ? (static_cast<size_t>(bb) * p.T + (p.rev ? p.T - 1 - t : t)) * p.H + hh : 0;
+        if (t < p.T && debug_in_bounds(p.debug, gi, 1, static_cast<size_t>(p.BH) * p.T, p.status)) {
             const float xg = p.g[gi] + p.dt_bias[hh];
             const float sp = xg > 20.0f ? xg : __logf(1.0f + __expf(xg));
             la = -__expf(p.A_log[hh]) * sp;

@@ -16,6 +16,15 @@ namespace gdn {
 // Device status word values (first int of the workspace); match gdn_status.
 enum : int { kStatusOk = 0, kStatusTimeout = 4, kStatusCheck = 5 };
 
+// Debug index-bounds check (plans with GDN_FLAG_DEBUG_CHECKS): true when the access of `n`
+// elements at `idx` lies inside a buffer of `size` elements, or when checks are off.  Otherwise
+// it records kStatusCheck in the status word and returns false, and the caller skips the access.
+__device__ __forceinline__ bool debug_in_bounds(int debug, size_t idx, size_t n, size_t size, int *status) {
+    if (!debug || (idx <= size && n <= size - idx)) return true;
+    atomicCAS(status, kStatusOk, kStatusCheck);
+    return false;
+}
+
 // Block size of the tensor path: the inter-block scan advances 128 tokens per
 // step, and every tcgen05 tile below is 128 rows (M = 128, cta_group::1).
 constexpr int kBlk = 128;

@@ -94,6 +94,7 @@ struct PrepParams {
     int *status;
     unsigned long long wait_limit_ns;
     int rev;                       // reverse scan: internal token t is input token T-1-t
+    int debug;                     // GDN_FLAG_DEBUG_CHECKS: index-bounds checks on the stores
 };
 cudaError_t launch_prep(const PrepParams &p, InType in, bool out_f16, cudaStream_t s);
 // Tensor path (16-bit inputs, d = 128): raw tiles staged by TMA through the
@@ -114,6 +115,7 @@ struct ChunkParams {
     int *status;
     unsigned long long wait_limit_ns;
     int rev;                        // reverse scan: block row t holds the gates of input token T-1-t
+    int debug;                      // GDN_FLAG_DEBUG_CHECKS: index-bounds checks on the gate accesses
 };
 cudaError_t launch_chunk(const ChunkParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
                          const CUtensorMap &tmQ, const CUtensorMap &tmW, const CUtensorMap &tmU,

@@ -211,6 +211,17 @@ __global__ void __launch_bounds__(256, 2)
     const int per = (ntiles + gridDim.x - 1) / gridDim.x;
     const int first = blockIdx.x * per, last = min(first + per, ntiles);
     const int tid = threadIdx.x;
+    // debug: the CTA's output rows (tiles first..last-1 of kPrepTok rows) inside q^, k^, v^
+    if (p.debug) {
+        const bool ok = p.Tp % kPrepTok == 0 &&
+                        debug_in_bounds(1, static_cast<size_t>(first) * kPrepTok,
+                                        static_cast<size_t>(max(last - first, 0)) * kPrepTok,
+                                        static_cast<size_t>(p.B) * p.H * p.Tp, p.status);
+        if (!ok) {
+            atomicCAS(p.status, kStatusOk, kStatusCheck);
+            return;
+        }
+    }
     if (tid == 0) {
         mbar_init(&bar[0], 1);
         mbar_init(&bar[1], 1);

@@ -85,6 +85,13 @@ __global__ void __launch_bounds__(288, 1)
     const int c0 = seg * p.Ls, c1 = min(c0 + p.Ls, p.NB);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint64_t lim = p.wait_limit_ns;
+    // debug: the segment's blocks inside the [BH][Tp] tiles and gates, and its [S_loc^T | P^T]
+    // inside Zloc
+    if (!debug_in_bounds(p.debug, static_cast<size_t>(bh) * p.Tp + static_cast<size_t>(c0) * kBlk,
+                         static_cast<size_t>(max(c1 - c0, 0)) * kBlk, static_cast<size_t>(p.B) * p.H * p.Tp, p.status) ||
+        !debug_in_bounds(p.debug, (static_cast<size_t>(bh) * p.NS + seg) * 128 * 256, 128 * 256,
+                         static_cast<size_t>(p.B) * p.H * p.NS * 128 * 256, p.status))
+        return;
 
     if (tid == 0) {
         for (int i = 0; i < NBAR; ++i) mbar_init(&bars[i], i >= CONS_D ? 4 : 1);
@@ -321,6 +328,10 @@ __global__ void __launch_bounds__(256, 1) gdn_combine_kernel(const ScanParams p)
     constexpr size_t kZ = 128 * 256;  // floats per (bh, segment) of Zloc
     const float *Z = p.Zloc + static_cast<size_t>(bh) * p.NS * kZ;
     float *Sst = p.Sstart + static_cast<size_t>(bh) * p.NS * 128 * 128;
+    // debug: this head's segments inside Zloc and Sstart
+    if (!debug_in_bounds(p.debug, static_cast<size_t>(bh) * p.NS * kZ, static_cast<size_t>(p.NS) * kZ,
+                         static_cast<size_t>(p.B) * p.H * p.NS * kZ, p.status))
+        return;
     pdl_launch_dependents();
     pdl_wait();  // the transfer pass's [S_loc^T | P^T] are complete
     if (p.NS < 2) return;
@@ -465,6 +476,12 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint64_t lim = p.wait_limit_ns;
 
+    // debug: the segment's blocks inside the [BH][Tp] tiles and gates, its start state inside Sstart
+    if (!debug_in_bounds(p.debug, static_cast<size_t>(bh) * p.Tp + static_cast<size_t>(c0) * kBlk,
+                         static_cast<size_t>(max(c1 - c0, 0)) * kBlk, static_cast<size_t>(p.B) * p.H * p.Tp, p.status) ||
+        !debug_in_bounds(p.debug, (static_cast<size_t>(bh) * p.NS + seg) * 128 * 128, 128 * 128,
+                         static_cast<size_t>(p.B) * p.H * p.NS * 128 * 128, p.status))
+        return;
     float *sNW = reinterpret_cast<float *>(sm + OFF_NW);
     if (tid == 0) {
         for (int i = 0; i < NBAR; ++i)
@@ -502,13 +519,19 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
         for (int c = c0; c < c1; ++c) {
             const int i = c - c0;
             const int tA = c * kBlk + rA, tB = c * kBlk + rB;
-            const bool liveA = tA < p.T, liveB = tB < p.T;
+            bool liveA = tA < p.T, liveB = tB < p.T;
             // input / output token of each row (the reverse scan's rows run backwards)
             const int xA = liveA ? (p.rev ? p.T - 1 - tA : tA) : 0, xB = liveB ? (p.rev ? p.T - 1 - tB : tB) : 0;
             const size_t zA = (static_cast<size_t>(b) * p.T + xA) * p.tok_stride + static_cast<size_t>(h) * kD;
             const size_t zB = (static_cast<size_t>(b) * p.T + xB) * p.tok_stride + static_cast<size_t>(h) * kD;
             const size_t yA = ((static_cast<size_t>(b) * p.T + xA) * p.H + h) * kD;
             const size_t yB = ((static_cast<size_t>(b) * p.T + xB) * p.H + h) * kD;
+            if (p.debug) {  // z rows inside [B][T] x tok_stride, y rows inside [B][T][H][128]
+                const size_t zsize = (static_cast<size_t>(p.B) * p.T - 1) * p.tok_stride + static_cast<size_t>(p.H) * kD;
+                const size_t ysize = static_cast<size_t>(p.B) * p.T * p.H * kD;
+                liveA = liveA && debug_in_bounds(1, zA, kD, zsize, p.status) && debug_in_bounds(1, yA, kD, ysize, p.status);
+                liveB = liveB && debug_in_bounds(1, zB, kD, zsize, p.status) && debug_in_bounds(1, yB, kD, ysize, p.status);
+            }
             const bool tre = (warp == 5 && lane == 0);
             if (tre) GDN_TRACE_AT(4096 + 64 * i + 32);
             // z: lane t0 of the quad fetches columns 8(4k + t0) .. +7 of its two rows

@@ -22,6 +22,20 @@
  * S is d_v x d_k per (b, h) and is carried in fp32.  The result y is the
  * layer output before the output projection.
  *
+ * Precision and range.  With bf16 or f16 inputs and d = 128 the forward runs
+ * on the tensor cores: the tensor-core operands (q^, k^, v^, the UT-transform
+ * products W, U and the decayed q/k tiles, the fp16 copy of the state and of
+ * Delta = U - W S^T) are fp16 with fp32 accumulation; the state itself and
+ * every sum stay fp32.  fp16 is chosen over bf16 for its 3 extra mantissa
+ * bits; its range ends at 65504.  q^ and k^ are unit vectors and the UT
+ * entries are bounded by the gates, so the range that binds is that of
+ * v^ = SiLU(conv4(v)), U and the state: inputs whose |conv4(v)| or state
+ * entries reach about 6e4 overflow to Inf and give non-finite outputs, which
+ * GDN_FLAG_DEBUG_CHECKS reports (activations of 128x unit scale with conv
+ * taps of 0.1 are well inside).  For such inputs use the fp32
+ * CUDA-core path (GDN_FLAG_FORCE_SIMT).  fp32 inputs, and d = 64, always
+ * take that path.
+ *
  * Layouts (row-major, element strides):
  *   q, k   [B][T][H][d_k]   token stride tok_stride (elements; 0 = H*d_k)
  *   v, z   [B][T][H][d_v]   token stride tok_stride (0 = H*d_v)

@@ -262,3 +262,29 @@ def test_debug_checks_report_non_finite_outputs(simt):
             assert st == expect, (name, flags, gdn.status_string(st))
     assert torch.isnan(outs[("bad", 0)].float()).sum().item() == 1
     assert torch.equal(outs[("clean", gdn.FLAG_DEBUG_CHECKS)], outs[("clean", 0)])
+
+
+@pytest.mark.parametrize("B,T,H,flags", [(1, 1, 2, 0), (2, 129, 3, 0), (1, 3000, 12, 0), (2, 1000, 12, "rev"),
+                                         (1, 2000, 4, "state"), (2, 1000, 12, "fused"), (1, 777, 2, "simt")])
+def test_debug_bounds_checks_pass_clean_runs_bit_for_bit(B, T, H, flags):
+    # GDN_FLAG_DEBUG_CHECKS adds index-bounds checks on every kernel's global accesses (a failed one
+    # skips the access and reports GDN_ERR_DEVICE_CHECK); on valid inputs none may fire, and the
+    # checked run must give the unchecked run's output bit for bit, over ragged, multi-segment,
+    # reverse, carried-state, fused and CUDA-core plans
+    import torch
+    import gated_deltanet_06_b200 as gdn
+    from state_util import random_state
+    inp = gdn_inputs.make_inputs(B, T, H, 128, "bf16", -1.0, seed=T)
+    t = torch_inputs(inp)
+    base = {0: 0, "rev": gdn.FLAG_REVERSE, "state": 0, "fused": gdn.FLAG_FUSED, "simt": gdn.FLAG_FORCE_SIMT}[flags]
+    s = torch.cuda.current_stream().cuda_stream
+    s0 = torch.from_numpy(random_state(B, H, 128, seed=T)).cuda() if flags == "state" else None
+    outs = []
+    for dbg in (0, gdn.FLAG_DEBUG_CHECKS):
+        plan = gdn.Plan(B, T, H, 128, gdn.DTYPE_BF16, gdn.DTYPE_F32, flags=base | dbg)
+        ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device="cuda")
+        y = gdn.forward(**t, plan=plan, workspace=ws, out_dtype=torch.float32, s0=s0,
+                        reverse=bool(base & gdn.FLAG_REVERSE))
+        assert plan.device_status(ws.data_ptr(), s) == gdn.OK, (flags, dbg)
+        outs.append(y)
+    assert torch.equal(outs[0], outs[1])
