@@ -391,6 +391,7 @@ def main():
     ap.add_argument("--no-reverse", action="store_true", help="skip the reverse-scan timing")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward timing")
     ap.add_argument("--no-configs", action="store_true", help="skip the other four seeded workloads")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
     ap.add_argument("--fused", action="store_true", help="time the fused forward (FLAG_FUSED) as the main path")
     ap.add_argument("--no-fused", action="store_true", help="skip the fused-forward timing beside the main path")
     ap.add_argument("--load-seconds", type=float, default=1.5)
@@ -477,6 +478,29 @@ def main():
         st = plan.device_status(ws.data_ptr(), s)
         if st != gdn.OK:
             raise SystemExit(f"device status in the per-step check: {gdn.status_string(st)}")
+
+    # the same forward captured once in a CUDA graph and replayed (launch overhead out of the step);
+    # the flush stays outside the graph and outside the timed interval
+    graph = None
+    if not args.no_graph:
+        try:
+            g = torch.cuda.CUDAGraph()
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g):
+                plan.forward_raw(ptrs, y.data_ptr(), ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
+            for _ in range(3):
+                g.replay()
+            g_ms = time_steps(g.replay, flush, stream, args.steps)
+            st = plan.device_status(ws.data_ptr(), s)
+            if st != gdn.OK:
+                raise SystemExit(f"device status after the graph replays: {gdn.status_string(st)}")
+            gm = ranks_max(sum(g_ms), world, dist, dev) / args.steps
+            graph = {"ms_per_step": gm, "value": job_throughput(world, w.B * w.T, gm), "unit": UNIT,
+                     "steps": args.steps, "step_ms": {"min": min(g_ms), "median": statistics.median(g_ms),
+                                                      "max": max(g_ms)}}
+            del g
+        except RuntimeError as e:  # capture refused by the runtime: reported, not fatal
+            graph = {"unavailable": str(e).splitlines()[0][:200]}
 
     # per-kernel breakdown (not part of the timed steps): the library records an event before each
     # launch and after the last one (gdn_forward_timed), which also serialises the launches
@@ -719,9 +743,10 @@ def main():
             "config": dict(workload_config(w, args.out_dtype, world),
                            path="fused tensor (FLAG_FUSED)" if args.fused else
                            ("tensor" if plan.uses_tensor_path else "CUDA-core fp32")),
-            "roofline": roof, "path_roofline": path_roof, "kernels_ms": kern_ms,
+            "roofline": roof, "path_roofline": path_roof, "path_roofline_frac": path_roof["frac"],
+            "kernels_ms": kern_ms,
             "segments": plan.segments, "cpu_baseline": cpu, "e2e": e2e, "state_io": state_io,
-            "reverse": reverse, "backward": bwd, "fused": fused, "configs": configs,
+            "reverse": reverse, "backward": bwd, "fused": fused, "graph": graph, "configs": configs,
             "clocks": clocks, "gpu_launches": L * args.steps,
             "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms), "max": max(step_ms)},
             "other_gpu_processes": None if others_before is None or others_after is None
