@@ -376,6 +376,65 @@ def bench_other_config(w, dev, flush, stream, steps, cpu_budget_s):
     return out
 
 
+def block_flops(w, D):
+    """Tensor-core flops of the two projections per layer: 2 M N K each."""
+    M, Hd = w.B * w.T, w.H * w.d
+    return 2 * M * (4 * Hd + 2 * w.H) * D, 2 * M * D * Hd
+
+
+def bench_block(w, dev, flush, stream, steps, world, dist):
+    """gdn_block_forward on this workload's shape with D = H * d: step time, per-kernel times and the
+    projections' tensor-core throughput against the measured bf16 peak."""
+    import torch
+
+    import gated_deltanet_06_b200 as gdn
+    D = w.H * w.d
+    inp = gdn_inputs.make_block_inputs(w.B, w.T, w.H, w.d, D, seed=w.seed)
+    t = {}
+    for n in ("x", "w_in", "w_out"):
+        t[n] = torch.from_numpy(inp[n + "_bits"].view(np.int16)).view(torch.bfloat16).to(dev)
+    for n in ("conv_q", "conv_k", "conv_v", "A_log", "dt_bias", "norm_w"):
+        t[n] = torch.from_numpy(np.ascontiguousarray(inp[n], dtype=np.float32)).to(dev)
+    del inp
+    bp = gdn.BlockPlan(w.B, w.T, w.H, w.d, D, gdn.DTYPE_BF16)
+    ws = torch.empty(bp.workspace_bytes, dtype=torch.uint8, device=dev)
+    out = torch.empty((w.B, w.T, D), dtype=torch.bfloat16, device=dev)
+    ptrs = {n: v.data_ptr() for n, v in t.items()}
+    s = stream.cuda_stream
+    run = lambda: bp.forward_raw(ptrs, out.data_ptr(), ws.data_ptr(), s)  # noqa: E731
+    for _ in range(3):
+        run()
+    ms = time_steps(run, flush, stream, steps)
+    st = bp.device_status(ws.data_ptr(), s)
+    if st != gdn.OK:
+        raise SystemExit(f"device status after the block forward: {gdn.status_string(st)}")
+    m = ranks_max(sum(ms), world, dist, dev) / steps
+    L = bp.launches
+    names = ["bf16_to_f16", "proj_in", "chunk"] + (["transfer", "combine"] if L == 7 else []) + ["scan", "proj_out"]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(L + 1)] for _ in range(3)]
+    for row in evs:
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+    for k in range(3):
+        flush.zero_()
+        bp.forward_timed_raw(ptrs, out.data_ptr(), ws.data_ptr(), s, [e.cuda_event for e in evs[k]])
+    torch.cuda.synchronize()
+    km = {names[i]: statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(3)) for i in range(L)}
+    f_in, f_out = block_flops(w, D)
+    peak = load_peaks()["bf16_tflops"]
+    res = {"ms_per_step": m, "value": job_throughput(world, w.B * w.T, m), "unit": UNIT, "steps": steps, "D": D,
+           "launches_per_step": L, "kernels_ms": km,
+           "proj_in": {"flops": f_in, "tflops": f_in / (km["proj_in"] / 1e3) / 1e12,
+                       "frac_of_bf16_peak": f_in / (km["proj_in"] / 1e3) / 1e12 / peak},
+           "proj_out": {"flops": f_out, "tflops": f_out / (km["proj_out"] / 1e3) / 1e12,
+                        "frac_of_bf16_peak": f_out / (km["proj_out"] / 1e3) / 1e12 / peak},
+           "step_ms": {"min": min(ms), "median": statistics.median(ms), "max": max(ms)}}
+    del ws, out, t
+    torch.cuda.empty_cache()
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -392,6 +451,7 @@ def main():
     ap.add_argument("--no-backward", action="store_true", help="skip the backward timing")
     ap.add_argument("--no-configs", action="store_true", help="skip the other four seeded workloads")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
+    ap.add_argument("--no-block", action="store_true", help="skip the layer-with-projections timing")
     ap.add_argument("--fused", action="store_true", help="time the fused forward (FLAG_FUSED) as the main path")
     ap.add_argument("--no-fused", action="store_true", help="skip the fused-forward timing beside the main path")
     ap.add_argument("--load-seconds", type=float, default=1.5)
@@ -694,6 +754,13 @@ def main():
                  "path_frac": path_roofline(w, s_in_f, s_out_f, f_ms, load_peaks())["frac"]}
         del ws_f
 
+    # the layer with its projections (gdn_block_forward) at this workload's shape, model width
+    # D = H * d (the Wan2.1-1.3B / Wan2.2-5B widths): input projection with the fused conv / SiLU /
+    # L2 epilogue, the tensor path, output projection
+    block = None
+    if not args.no_block and plan.uses_tensor_path and w.H % 2 == 0:
+        block = bench_block(w, dev, flush, stream, max(5, min(args.steps, 20)), world, dist)
+
     # the other four seeded workloads (rank 0 alone, 1 GPU): same step, flush and event timing
     configs = None
     if world == 1 and not args.no_configs and not args.T:
@@ -746,7 +813,8 @@ def main():
             "roofline": roof, "path_roofline": path_roof, "path_roofline_frac": path_roof["frac"],
             "kernels_ms": kern_ms,
             "segments": plan.segments, "cpu_baseline": cpu, "e2e": e2e, "state_io": state_io,
-            "reverse": reverse, "backward": bwd, "fused": fused, "graph": graph, "configs": configs,
+            "reverse": reverse, "backward": bwd, "fused": fused, "graph": graph, "block": block,
+            "configs": configs,
             "clocks": clocks, "gpu_launches": L * args.steps,
             "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms), "max": max(step_ms)},
             "other_gpu_processes": None if others_before is None or others_after is None

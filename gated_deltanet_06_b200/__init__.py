@@ -94,6 +94,34 @@ _lib.gdn_status_string.argtypes = [ctypes.c_int]
 _lib.gdn_status_string.restype = ctypes.c_char_p
 
 
+class BlockConfig(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int),
+                ("D", ctypes.c_int), ("out_dtype", ctypes.c_int), ("l2_eps", ctypes.c_float),
+                ("norm_eps", ctypes.c_float), ("flags", ctypes.c_uint)]
+
+
+BLOCK_NAMES = ("x", "w_in", "w_out", "conv_q", "conv_k", "conv_v", "A_log", "dt_bias", "norm_w")
+
+
+class BlockInputs(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in BLOCK_NAMES]
+
+
+_lib.gdn_block_plan.argtypes = [ctypes.POINTER(BlockConfig), ctypes.POINTER(_vp), ctypes.POINTER(ctypes.c_size_t)]
+_lib.gdn_block_plan.restype = ctypes.c_int
+_lib.gdn_block_forward.argtypes = [_vp, ctypes.POINTER(BlockInputs), _vp, _vp, _vp]
+_lib.gdn_block_forward.restype = ctypes.c_int
+_lib.gdn_block_forward_timed.argtypes = [_vp, ctypes.POINTER(BlockInputs), _vp, _vp, _vp, ctypes.POINTER(_vp),
+                                         ctypes.c_int]
+_lib.gdn_block_forward_timed.restype = ctypes.c_int
+_lib.gdn_block_launches.argtypes = [_vp]
+_lib.gdn_block_launches.restype = ctypes.c_int
+_lib.gdn_block_device_status.argtypes = [_vp, _vp, _vp]
+_lib.gdn_block_device_status.restype = ctypes.c_int
+_lib.gdn_block_destroy.argtypes = [_vp]
+_lib.gdn_block_destroy.restype = ctypes.c_int
+
+
 class GDNError(RuntimeError):
     def __init__(self, status: int, where: str):
         super().__init__(f"{where}: {status_string(status)} (status {status})")
@@ -298,4 +326,71 @@ def backward(q, k, v, z, g, b, conv_q, conv_k, conv_v, A_log, dt_bias, norm_w, d
              dt_bias=dt_bias, norm_w=norm_w)
     plan.backward_raw(tensor_ptrs(t), dy.contiguous().data_ptr(), {n: out[n].data_ptr() for n in GRAD_NAMES},
                       workspace.data_ptr(), s)
+    return out
+
+
+# ------------------------------------------------------------------ the layer
+class BlockPlan:
+    """A gdn_block_plan_t: the GDN layer with its input and output projections (host state only)."""
+
+    def __init__(self, B, T, H, d, D, out_dtype=DTYPE_BF16, l2_eps=1e-6, norm_eps=1e-6, flags=0):
+        self.cfg = BlockConfig(B, T, H, d, D, out_dtype, l2_eps, norm_eps, flags)
+        self._h = _vp()
+        ws = ctypes.c_size_t()
+        _check(_lib.gdn_block_plan(ctypes.byref(self.cfg), ctypes.byref(self._h), ctypes.byref(ws)),
+               "gdn_block_plan")
+        self.workspace_bytes = ws.value
+
+    @property
+    def launches(self) -> int:
+        return _lib.gdn_block_launches(self._h)
+
+    def forward_raw(self, ptrs: dict, out: int, workspace: int, stream: int) -> None:
+        ins = BlockInputs(*[ptrs[n] for n in BLOCK_NAMES])
+        _check(_lib.gdn_block_forward(self._h, ctypes.byref(ins), out, workspace, stream), "gdn_block_forward")
+
+    def forward_timed_raw(self, ptrs: dict, out: int, workspace: int, stream: int, events: list) -> None:
+        ins = BlockInputs(*[ptrs[n] for n in BLOCK_NAMES])
+        arr = (_vp * len(events))(*events)
+        _check(_lib.gdn_block_forward_timed(self._h, ctypes.byref(ins), out, workspace, stream, arr, len(events)),
+               "gdn_block_forward_timed")
+
+    def device_status(self, workspace: int, stream: int) -> int:
+        return _lib.gdn_block_device_status(self._h, workspace, stream)
+
+    def close(self):
+        if self._h:
+            _lib.gdn_block_destroy(self._h)
+            self._h = _vp()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def block_forward(x, w_in, w_out, conv_q, conv_k, conv_v, A_log, dt_bias, norm_w, out_dtype=None, l2_eps=1e-6,
+                  norm_eps=1e-6, plan: BlockPlan | None = None, workspace=None, out=None, stream=None):
+    """The GDN layer on CUDA tensors: x [B,T,D] bf16, w_in [4*H*d + 2*H, D] bf16 (rows q, k, v, z, g, b),
+    w_out [D, H*d] bf16, conv_* [H*d, 4], A_log, dt_bias [H], norm_w [d] fp32.  Returns out [B,T,D]
+    (bf16, or out_dtype=torch.float32): (x W_in^T -> GDN forward -> y W_out^T)."""
+    import torch
+    B, T, D = x.shape
+    H = A_log.shape[0]
+    d = norm_w.shape[0]
+    odt = torch.bfloat16 if out_dtype is None else out_dtype
+    if plan is None:
+        plan = BlockPlan(B, T, H, d, D, _torch_dtype_code(odt), l2_eps, norm_eps)
+    if workspace is None:
+        workspace = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=x.device)
+    if out is None:
+        out = torch.empty((B, T, D), dtype=odt, device=x.device)
+    s = torch.cuda.current_stream(x.device).cuda_stream if stream is None else stream
+    t = dict(x=x, w_in=w_in, w_out=w_out, conv_q=conv_q, conv_k=conv_k, conv_v=conv_v, A_log=A_log,
+             dt_bias=dt_bias, norm_w=norm_w)
+    for n, v in t.items():
+        if not v.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    plan.forward_raw({n: v.data_ptr() for n, v in t.items()}, out.data_ptr(), workspace.data_ptr(), s)
     return out

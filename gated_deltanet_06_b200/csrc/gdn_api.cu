@@ -32,6 +32,20 @@ struct gdn_plan_s {
     size_t st_q, st_k, st_v, st_z, st_g, st_b, st_cq, st_ck, st_cv, st_A, st_dt, st_nw, st_y, staging_bytes;
 };
 
+EncodeTiledFn gdn::encode_fn() {
+    // looked up once (function-local statics initialise thread-safely)
+    static const EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            return reinterpret_cast<EncodeTiledFn>(ptr);
+        cudaGetLastError();
+        return nullptr;
+    }();
+    return fn;
+}
+
 namespace {
 
 constexpr unsigned long long kWaitLimitNs = 2000ull * 1000 * 1000;  // 2 s per device-side wait
@@ -46,25 +60,6 @@ InType in_type(gdn_dtype t) {
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
-                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                  CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    // looked up once (function-local statics initialise thread-safely)
-    static const EncodeTiledFn fn = []() -> EncodeTiledFn {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            return reinterpret_cast<EncodeTiledFn>(ptr);
-        cudaGetLastError();
-        return nullptr;
-    }();
-    return fn;
-}
 
 // [rows][128] fp16 row-major, loaded as {64, 128} boxes with the 128-byte swizzle.
 bool make_tile_map(CUtensorMap *m, void *base, unsigned long long rows, unsigned box_rows = 128) {
@@ -99,6 +94,88 @@ bool make_raw_map(CUtensorMap *m, const void *base, int B, int T, int Hd, long l
 
 
 size_t gdn::plan_workspace_bytes(const gdn_plan_s *plan) { return plan ? plan->ws_bytes : 0; }
+
+int gdn::run_tensor_core(const gdn_plan_s *plan, const float *g, const float *b, const float *A_log,
+                         const float *dt_bias, const float *norm_w, const void *z, InType z_type, long long z_stride,
+                         void *y, void *workspace, cudaStream_t s, bool pdl_first, void *const *events, int *ev,
+                         const float *s0, float *s_end) {
+    const gdn_config &c = plan->cfg;
+    const int d = c.d_k;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    int *status = reinterpret_cast<int *>(ws + plan->off_status);
+    float *G = reinterpret_cast<float *>(ws + plan->off_G);
+    float *beta = reinterpret_cast<float *>(ws + plan->off_beta);
+    float *la = reinterpret_cast<float *>(ws + plan->off_la);
+    const int rev = (c.flags & GDN_FLAG_REVERSE) ? 1 : 0;
+    auto mark = [&]() -> bool {
+        if (!events) return true;
+        return cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[(*ev)++]), s) == cudaSuccess;
+    };
+    {
+        const unsigned long long rows = static_cast<unsigned long long>(c.B) * c.H * plan->Tp;
+        CUtensorMap tmQ, tmK, tmV, tmW, tmU, tmQt, tmKt, tmAqk, tmAqkH;
+        if (!make_tile_map(&tmQ, ws + plan->off_qh, rows) || !make_tile_map(&tmK, ws + plan->off_kh, rows) ||
+            !make_tile_map(&tmV, ws + plan->off_vh, rows) || !make_tile_map(&tmW, ws + plan->off_W, rows) ||
+            !make_tile_map(&tmU, ws + plan->off_U, rows) || !make_tile_map(&tmQt, ws + plan->off_Qt, rows) ||
+            !make_tile_map(&tmKt, ws + plan->off_Kt, rows) || !make_tile_map(&tmAqk, ws + plan->off_Aqk, rows) ||
+            !make_tile_map(&tmAqkH, ws + plan->off_Aqk, rows, 64))  // Aqk's lower-right quadrant
+            return GDN_ERR_CUDA;
+        ChunkParams cp;
+        cp.g = g; cp.bg = b; cp.A_log = A_log; cp.dt_bias = dt_bias;
+        cp.G = G; cp.beta = beta; cp.log_alpha = la;
+        cp.T = c.T; cp.H = c.H;
+        cp.W = reinterpret_cast<__half *>(ws + plan->off_W);
+        cp.U = reinterpret_cast<__half *>(ws + plan->off_U);
+        cp.Qt = reinterpret_cast<__half *>(ws + plan->off_Qt);
+        cp.Kt = reinterpret_cast<__half *>(ws + plan->off_Kt);
+        cp.Aqk = reinterpret_cast<__half *>(ws + plan->off_Aqk);
+        cp.BH = c.B * c.H; cp.Tp = plan->Tp; cp.NB = plan->NB;
+        cp.status = status;
+        cp.wait_limit_ns = kWaitLimitNs;
+        cp.rev = rev;
+        cp.debug = (c.flags & GDN_FLAG_DEBUG_CHECKS) ? 1 : 0;
+        // The kernels start with programmatic dependent launch (prologue overlapped with the previous
+        // kernel's tail), except when per-kernel events are recorded between them.
+        const bool pdl = events == nullptr;
+        if (!mark() || launch_chunk(cp, tmK, tmV, tmQ, tmW, tmU, tmQt, tmAqk, tmAqkH, s, pdl && pdl_first) != cudaSuccess)
+            return GDN_ERR_CUDA;
+        ScanParams sp;
+        sp.G = G;
+        sp.Zloc = reinterpret_cast<float *>(ws + plan->off_Zloc);
+        sp.Sstart = reinterpret_cast<float *>(ws + plan->off_Sstart);
+        sp.z = z; sp.tok_stride = z_stride; sp.norm_w = norm_w; sp.y = y;
+        sp.out_kind = c.out_dtype == GDN_DTYPE_BF16 ? 0 : (c.out_dtype == GDN_DTYPE_F32 ? 1 : 2);
+        sp.eps = c.norm_eps;
+        sp.B = c.B; sp.T = c.T; sp.H = c.H; sp.Tp = plan->Tp; sp.NB = plan->NB; sp.NS = plan->NS; sp.Ls = plan->Ls;
+        sp.status = status;
+        sp.wait_limit_ns = kWaitLimitNs;
+        sp.test_wait_timeout = (c.flags & GDN_FLAG_TEST_WAIT_TIMEOUT) ? 1 : 0;
+        sp.s0 = s0;
+        sp.s_end = s_end;
+        sp.rev = rev;
+        sp.debug = (c.flags & GDN_FLAG_DEBUG_CHECKS) ? 1 : 0;
+        if (plan->NS > 1) {
+            if (!mark() || launch_transfer(sp, tmW, tmKt, tmU, s, pdl) != cudaSuccess) return GDN_ERR_CUDA;
+            if (!mark() || launch_combine(sp, s, pdl) != cudaSuccess) return GDN_ERR_CUDA;
+        }
+        CUtensorMap tmZ;
+        if (!make_raw_map(&tmZ, z, c.B, c.T, c.H * d, z_stride, kBlk, 128)) return GDN_ERR_CUDA;
+        if (!mark() || launch_scan_out(sp, z_type, tmW, tmQt, tmKt, tmAqk, tmAqkH, tmU, tmZ, s, pdl) != cudaSuccess)
+            return GDN_ERR_CUDA;
+        return GDN_OK;
+    }
+}
+
+int gdn::tensor_core_launches(const gdn_plan_s *plan) { return plan->NS > 1 ? 4 : 2; }
+
+bool gdn::plan_layout(const gdn_plan_s *plan, PlanLayout *out) {
+    if (!plan || !out || !plan->tensor || plan->fused) return false;
+    out->B = plan->cfg.B; out->T = plan->cfg.T; out->H = plan->cfg.H; out->Tp = plan->Tp;
+    out->off_status = plan->off_status; out->off_qh = plan->off_qh; out->off_kh = plan->off_kh;
+    out->off_vh = plan->off_vh; out->ws_bytes = plan->ws_bytes;
+    return true;
+}
+
 
 extern "C" {
 
@@ -397,56 +474,10 @@ static gdn_status forward_impl(gdn_plan_t plan, const gdn_inputs *in, void *y, v
     }
 
     if (plan->tensor) {
-        const unsigned long long rows = static_cast<unsigned long long>(c.B) * c.H * plan->Tp;
-        CUtensorMap tmQ, tmK, tmV, tmW, tmU, tmQt, tmKt, tmAqk, tmAqkH;
-        if (!make_tile_map(&tmQ, ws + plan->off_qh, rows) || !make_tile_map(&tmK, ws + plan->off_kh, rows) ||
-            !make_tile_map(&tmV, ws + plan->off_vh, rows) || !make_tile_map(&tmW, ws + plan->off_W, rows) ||
-            !make_tile_map(&tmU, ws + plan->off_U, rows) || !make_tile_map(&tmQt, ws + plan->off_Qt, rows) ||
-            !make_tile_map(&tmKt, ws + plan->off_Kt, rows) || !make_tile_map(&tmAqk, ws + plan->off_Aqk, rows) ||
-            !make_tile_map(&tmAqkH, ws + plan->off_Aqk, rows, 64))  // Aqk's lower-right quadrant
-            return GDN_ERR_CUDA;
-        ChunkParams cp;
-        cp.g = in->g; cp.bg = in->b; cp.A_log = in->A_log; cp.dt_bias = in->dt_bias;
-        cp.G = G; cp.beta = beta; cp.log_alpha = la;
-        cp.T = c.T; cp.H = c.H;
-        cp.W = reinterpret_cast<__half *>(ws + plan->off_W);
-        cp.U = reinterpret_cast<__half *>(ws + plan->off_U);
-        cp.Qt = reinterpret_cast<__half *>(ws + plan->off_Qt);
-        cp.Kt = reinterpret_cast<__half *>(ws + plan->off_Kt);
-        cp.Aqk = reinterpret_cast<__half *>(ws + plan->off_Aqk);
-        cp.BH = c.B * c.H; cp.Tp = plan->Tp; cp.NB = plan->NB;
-        cp.status = status;
-        cp.wait_limit_ns = kWaitLimitNs;
-        cp.rev = rev;
-        cp.debug = (c.flags & GDN_FLAG_DEBUG_CHECKS) ? 1 : 0;
-        // Kernels after the first start with programmatic dependent launch (prologue overlapped with
-        // the previous kernel's tail), except when per-kernel events are recorded between them.
-        const bool pdl = events == nullptr;
-        if (!mark() || launch_chunk(cp, tmK, tmV, tmQ, tmW, tmU, tmQt, tmAqk, tmAqkH, s, pdl) != cudaSuccess)
-            return GDN_ERR_CUDA;
-        ScanParams sp;
-        sp.G = G;
-        sp.Zloc = reinterpret_cast<float *>(ws + plan->off_Zloc);
-        sp.Sstart = reinterpret_cast<float *>(ws + plan->off_Sstart);
-        sp.z = in->z; sp.tok_stride = plan->tok_stride; sp.norm_w = in->norm_w; sp.y = y;
-        sp.out_kind = c.out_dtype == GDN_DTYPE_BF16 ? 0 : (c.out_dtype == GDN_DTYPE_F32 ? 1 : 2);
-        sp.eps = c.norm_eps;
-        sp.B = c.B; sp.T = c.T; sp.H = c.H; sp.Tp = plan->Tp; sp.NB = plan->NB; sp.NS = plan->NS; sp.Ls = plan->Ls;
-        sp.status = status;
-        sp.wait_limit_ns = kWaitLimitNs;
-        sp.test_wait_timeout = (c.flags & GDN_FLAG_TEST_WAIT_TIMEOUT) ? 1 : 0;
-        sp.s0 = s0;
-        sp.s_end = s_end;
-        sp.rev = rev;
-        sp.debug = (c.flags & GDN_FLAG_DEBUG_CHECKS) ? 1 : 0;
-        if (plan->NS > 1) {
-            if (!mark() || launch_transfer(sp, tmW, tmKt, tmU, s, pdl) != cudaSuccess) return GDN_ERR_CUDA;
-            if (!mark() || launch_combine(sp, s, pdl) != cudaSuccess) return GDN_ERR_CUDA;
-        }
-        CUtensorMap tmZ;
-        if (!make_raw_map(&tmZ, in->z, c.B, c.T, c.H * d, plan->tok_stride, kBlk, 128)) return GDN_ERR_CUDA;
-        if (!mark() || launch_scan_out(sp, in_type(c.in_dtype), tmW, tmQt, tmKt, tmAqk, tmAqkH, tmU, tmZ, s, pdl) != cudaSuccess)
-            return GDN_ERR_CUDA;
+        const int st = run_tensor_core(plan, in->g, in->b, in->A_log, in->dt_bias, in->norm_w, in->z,
+                                       in_type(c.in_dtype), plan->tok_stride, y, workspace, s, events == nullptr,
+                                       events, &ev, s0, s_end);
+        if (st != GDN_OK) return static_cast<gdn_status>(st);
         if (!mark()) return GDN_ERR_CUDA;
         return GDN_OK;
     } else {

@@ -17,10 +17,11 @@ namespace gdn {
 enum : int { kStatusOk = 0, kStatusTimeout = 4, kStatusCheck = 5 };
 
 // Debug index-bounds check (plans with GDN_FLAG_DEBUG_CHECKS): true when the access of `n`
-// elements at `idx` lies inside a buffer of `size` elements, or when checks are off.  Otherwise
-// it records kStatusCheck in the status word and returns false, and the caller skips the access.
+// elements at `idx` lies inside a buffer of `size` elements (an empty access always does), or
+// when checks are off.  Otherwise it records kStatusCheck in the status word and returns false,
+// and the caller skips the access.
 __device__ __forceinline__ bool debug_in_bounds(int debug, size_t idx, size_t n, size_t size, int *status) {
-    if (!debug || (idx <= size && n <= size - idx)) return true;
+    if (!debug || n == 0 || (idx <= size && n <= size - idx)) return true;
     atomicCAS(status, kStatusOk, kStatusCheck);
     return false;
 }
@@ -447,6 +448,14 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn_maj
            | (0u << 7) | (0u << 10)                   // A, B format: F16
            | ((a_mn_major ? 1u : 0u) << 15)           // A major
            | ((b_mn_major ? 1u : 0u) << 16)           // B major
+           | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
+           | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
+}
+
+// Instruction descriptor for kind::f16 with bf16 A and B (both K-major) and fp32 D.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+    return (1u << 4)                                  // D format: F32
+           | (1u << 7) | (1u << 10)                   // A, B format: BF16
            | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
            | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
 }

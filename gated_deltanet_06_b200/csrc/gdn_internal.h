@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -242,4 +243,59 @@ struct gdn_plan_s;
 namespace gdn {
 // Workspace bytes a plan's forward needs (the value gdn_plan reported).
 size_t plan_workspace_bytes(const gdn_plan_s *plan);
+}  // namespace gdn
+
+namespace gdn {
+// The projections around the core (tcgen05 GEMM, C = A B^T, bf16 operands both K-major, fp32
+// accumulation).  mode 0: the input projection x W_in^T, N = 4 H 128 + 2 H columns in the order
+// q | k | v | z | g | b, with conv4 + SiLU (+ L2 norm for q, k) in the epilogue; mode 1: the
+// output projection y W_out^T.
+struct ProjParams {
+    int M, N, K;                 // rows (B*T), output columns, reduction (multiple of 64)
+    int m_step;                  // rows an M tile advances by (125 in mode 0: 3 history rows)
+    int m_tiles, n_tiles;
+    int B, T, H, Tp;             // mode 0: batch, tokens, heads, T rounded up to 128
+    const float *conv_q, *conv_k, *conv_v;  // [H*128][4], tap 3 on the current token
+    __half *qh, *kh, *vh;        // [B][H][Tp][128] fp16 (mode 0)
+    __half *z;                   // [B][T][H*128] fp16 (mode 0)
+    float *g, *b;                // [B][T][H] fp32 (mode 0)
+    float l2_eps, q_scale;
+    void *out;                   // [M][N] (mode 1)
+    int out_kind;                // 0 bf16, 1 fp32 (mode 1)
+    int f16;                     // operands fp16 instead of bf16
+    int debug;
+    int *status;
+    unsigned long long wait_limit_ns;
+};
+cudaError_t launch_proj(const ProjParams &p, int mode, const CUtensorMap &tmA, const CUtensorMap &tmB,
+                        cudaStream_t s, bool pdl);
+int proj_m_step(int mode);
+// dst[i] = fp16(src[i]) for n bf16 elements (n a multiple of 8; 16-byte aligned pointers).
+cudaError_t launch_bf16_to_f16(const void *src, void *dst, size_t n, cudaStream_t s);
+int proj_n_tile();
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (nullptr if unavailable).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn();
+
+// Layout facts of a tensor-path plan that the block forward needs.
+struct PlanLayout {
+    int B, T, H, Tp;
+    size_t off_status, off_qh, off_kh, off_vh, ws_bytes;
+};
+bool plan_layout(const gdn_plan_s *plan, PlanLayout *out);
+
+// The tensor path after its prep step: q^, k^, v^ are in the plan's workspace (fp16
+// [B][H][Tp][128], zero rows past T); g, b raw gates [B][T][H]; z [B][T][H*128] of type z_type
+// with token stride z_stride; y bf16/f16/f32 per the plan.  The status word is not cleared here.
+// Returns a gdn_status value.
+// events (optional): one cudaEvent_t recorded before each launch, *ev counts them.
+int run_tensor_core(const gdn_plan_s *plan, const float *g, const float *b, const float *A_log,
+                    const float *dt_bias, const float *norm_w, const void *z, InType z_type,
+                    long long z_stride, void *y, void *workspace, cudaStream_t s, bool pdl_first,
+                    void *const *events, int *ev, const float *s0, float *s_end);
+int tensor_core_launches(const gdn_plan_s *plan);
 }  // namespace gdn

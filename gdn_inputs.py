@@ -121,3 +121,31 @@ def workload_inputs(w: Workload, T: int | None = None, B: int | None = None,
     (same seed and distributions, smaller shape)."""
     return make_inputs(B if B is not None else w.B, T if T is not None else w.T,
                        H if H is not None else w.H, w.d, w.dtype, w.g_mean, w.seed)
+
+
+def make_block_inputs(B: int, T: int, H: int, d: int, D: int, seed: int = 0) -> dict:
+    """Draw one seeded input set for the GDN layer with its projections.
+
+    x [B, T, D] ~ N(0, 1) and the weights W_in [4*H*d + 2*H, D] ~ N(0, 1/D) and
+    W_out [D, H*d] ~ N(0, 1/(H*d)) are rounded to bf16 (bits in x_bits,
+    w_in_bits, w_out_bits; the exact fp32 widenings in x, w_in, w_out), so that
+    the projections of q, k, v, z, g, b come out near N(0, 1) like the core's
+    inputs.  The conv weights, A_log, dt_bias and norm_w follow make_inputs.
+    """
+    rng = np.random.Generator(np.random.PCG64(seed))
+    out = {}
+    N = 4 * H * d + 2 * H
+    for name, shape, std in (("x", (B, T, D), 1.0), ("w_in", (N, D), 1.0 / math.sqrt(D)),
+                             ("w_out", (D, H * d), 1.0 / math.sqrt(H * d))):
+        x = rng.standard_normal(shape, dtype=np.float32) * np.float32(std)
+        bits = f32_to_bf16_bits(x)
+        out[name + "_bits"] = bits
+        out[name] = bf16_bits_to_f32(bits)
+    out["conv_q"] = (np.float32(0.1) * rng.standard_normal((H * d, 4), dtype=np.float32))
+    out["conv_k"] = (np.float32(0.1) * rng.standard_normal((H * d, 4), dtype=np.float32))
+    out["conv_v"] = (np.float32(0.1) * rng.standard_normal((H * d, 4), dtype=np.float32))
+    out["A_log"] = rng.uniform(0.0, math.log(16.0), H).astype(np.float32)
+    out["dt_bias"] = (np.float32(0.1) * rng.standard_normal(H, dtype=np.float32))
+    out["norm_w"] = np.ones(d, dtype=np.float32)
+    out["meta"] = dict(B=B, T=T, H=H, d=d, D=D, seed=seed)
+    return out

@@ -303,6 +303,76 @@ gdn_status gdn_destroy(gdn_plan_t plan);
 /* Static description of a status code. */
 const char *gdn_status_string(gdn_status s);
 
+/* ------------------------------------------------------------------------
+ * The GDN layer with its projections (gdn_block_*): hidden states in,
+ * projected layer output out.  The LinMorph page ("Why learn the
+ * initialization?") builds the GDN module's q/k/v/o-side parameters from the
+ * attention block's projections; the T3-Video page (Table 1) counts those
+ * projections at 7.0T (QKV) and 2.3T (O) MACs for Wan2.1-1.3B at 480x832.
+ * For every token row m = b*T + t:
+ *   [q | k | v | z | g | b]_m = x_m W_in^T      (W_in: [4*H*d + 2*H][D])
+ *   y = the GDN forward above on q, k, v, z, g, b (causal scan)
+ *   out_m = y_m W_out^T                          (W_out: [D][H*d])
+ * with q, k, v, z [H*d] head-major (head h at columns h*d .. h*d+d-1) and
+ * g, b [H].  Operands bf16, fp32 accumulation on the tensor cores.  The
+ * input projection runs conv4, SiLU and the q/k L2 norm in its epilogue and
+ * hands the prepared operands to the tensor path in fp16 (the projections of
+ * q, k, v, z are not rounded to bf16 first); y is stored in bf16 between the
+ * scan and the output projection, as the layer's activation type.
+ * Requirements: d = 128, H even, D a multiple of 64, B*T < 2^31.
+ * Layouts: x [B][T][D] bf16 and out [B][T][D] (bf16 or fp32), dense; the
+ * conv, gate and norm parameters as in gdn_inputs.  All pointers device,
+ * 16-byte aligned, caller-owned. */
+typedef struct {
+    int B, T, H, d;          /* d must be 128; H even */
+    int D;                   /* model width, a multiple of 64 */
+    gdn_dtype out_dtype;     /* out: GDN_DTYPE_BF16 or GDN_DTYPE_F32 */
+    float l2_eps, norm_eps;  /* as in gdn_config */
+    unsigned flags;          /* GDN_FLAG_DEBUG_CHECKS only */
+} gdn_block_config;
+
+typedef struct {
+    const void *x;                          /* [B][T][D] bf16 */
+    const void *w_in;                       /* [4*H*d + 2*H][D] bf16 (rows: q, k, v, z, g, b) */
+    const void *w_out;                      /* [D][H*d] bf16 */
+    const float *conv_q, *conv_k, *conv_v;  /* [H*d][4] fp32 */
+    const float *A_log, *dt_bias;           /* [H] fp32 */
+    const float *norm_w;                    /* [d] fp32 */
+} gdn_block_inputs;
+
+typedef struct gdn_block_plan_s *gdn_block_plan_t;
+
+/* Validate cfg and build a block plan for the current device; *workspace_bytes
+ * receives the device workspace gdn_block_forward needs (256-byte aligned).
+ * Host only.  Errors: INVALID_ARG, UNSUPPORTED (d != 128, odd H, D not a
+ * multiple of 64, out_dtype not bf16/f32, flags other than DEBUG_CHECKS),
+ * NO_DEVICE. */
+gdn_status gdn_block_plan(const gdn_block_config *cfg, gdn_block_plan_t *out, size_t *workspace_bytes);
+
+/* Enqueue the layer on `stream`: out <- (x W_in^T -> GDN -> W_out).  Host
+ * argument errors return before any launch; device-side errors go to the
+ * status word read by gdn_block_device_status. */
+gdn_status gdn_block_forward(gdn_block_plan_t plan, const gdn_block_inputs *in, void *out, void *workspace,
+                             gdn_stream_t stream);
+
+/* gdn_block_forward with events[i] recorded before the i-th of its
+ * gdn_block_launches(plan) launches and events[L] after the last (n_events
+ * must be L + 1); the launches are then not overlapped. */
+gdn_status gdn_block_forward_timed(gdn_block_plan_t plan, const gdn_block_inputs *in, void *out, void *workspace,
+                                   gdn_stream_t stream, void *const *events, int n_events);
+
+/* Kernel launches of one gdn_block_forward: the input projection, the tensor
+ * path's UT transform, [segment transfer, combine,] scan with the output
+ * step, and the output projection (4 or 6). */
+int gdn_block_launches(gdn_block_plan_t plan);
+
+/* Synchronise `stream`, then read and clear the block workspace's status word
+ * (as gdn_get_device_status). */
+gdn_status gdn_block_device_status(gdn_block_plan_t plan, void *workspace, gdn_stream_t stream);
+
+/* Free a block plan (host memory only).  NULL is accepted. */
+gdn_status gdn_block_destroy(gdn_block_plan_t plan);
+
 #ifdef __cplusplus
 }
 #endif
