@@ -13,8 +13,8 @@
 //                K = 16 per instruction) into one of two 256-column fp32
 //                accumulators, so that a tile's epilogue overlaps the next
 //                tile's products;
-//   warps 2-9    epilogue: warp w reads TMEM lane quarter w % 4 (rows) of
-//                column half (w - 2) / 4 (128 columns = one head).
+//   warps 2-17   epilogue: warp w reads TMEM lane quarter w % 4 (rows) of
+//                the 64-column quarter (w - 2) / 4 of the tile (half a head).
 // Tiles are handed out round-robin, N fastest, so that the CTAs working at one
 // time share A rows and the whole weight through L2.
 //
@@ -24,7 +24,9 @@
 // M tile covers 128 consecutive rows but advances by 125: its first 3 rows are
 // the previous tokens (history only), rows 3..127 are its outputs.  Inside a
 // warp the history comes by shuffles; the first 3 lanes of a quarter get the
-// last 3 rows of the quarter above through shared memory.  Taps reaching
+// last 3 rows of the quarter above through shared memory.  The taps of the
+// tile's channels are staged in shared memory once per tile, and the two warps
+// holding the halves of a head's row add their sums of squares there.  Taps reaching
 // before the start of a batch item read zero, as in the definition.  q and k
 // are then L2-normalised over their head (q also scaled by 1/sqrt(d)), and
 // q^, k^, v^ are written as fp16 in the tensor path's [B][H][Tp][128]
@@ -43,14 +45,20 @@ constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr uint32_t A_BYTES = BM * BK * 2;              // 16 KB
 constexpr uint32_t B_BYTES = BN * BK * 2;              // 32 KB
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr uint32_t OFF_HALO = STAGES * STAGE_BYTES;    // conv history rows: [2 parity][2 half][4 quarter][3][33] fp32
-constexpr int HALO_SLOT = 100;                         // floats per (parity, half, quarter) slot (3 rows of 33)
-constexpr uint32_t HALO_BYTES = 2 * 2 * 4 * HALO_SLOT * 4;
-constexpr uint32_t OFF_BAR = OFF_HALO + HALO_BYTES;
+// conv history rows, per (chunk parity, sub, quarter): the last 3 rows of the quarter, 32 values
+// each, rows 36 floats apart (16-byte aligned)
+constexpr int HALO_SLOT = 112;
+constexpr uint32_t OFF_HALO = STAGES * STAGE_BYTES;
+constexpr uint32_t HALO_BYTES = 2 * 4 * 4 * HALO_SLOT * 4;
+constexpr uint32_t OFF_TAPS = OFF_HALO + HALO_BYTES;   // conv taps of the tile, per sub [4 taps][64 channels]
+constexpr uint32_t TAPS_BYTES = 4 * 4 * 64 * 4;
+constexpr uint32_t OFF_SS = OFF_TAPS + TAPS_BYTES;     // q/k sums of squares, [tile parity][2 heads][4 quarters][2 parts][32]
+constexpr uint32_t SS_BYTES = 2 * 2 * 4 * 2 * 32 * 4;
+constexpr uint32_t OFF_BAR = OFF_SS + SS_BYTES;
 enum { FULL = 0, EMPTY = STAGES, ACC_FULL = 2 * STAGES, ACC_EMPTY = ACC_FULL + 2, NBAR = ACC_EMPTY + 2 };
 constexpr uint32_t SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
-constexpr int kThreads = 320;
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;
+constexpr int kThreads = 32 * (2 + kEpiWarps);
 constexpr int kHist = 3;  // conv history rows at the top of an input-projection M tile
 }  // namespace pj
 
@@ -79,11 +87,18 @@ __device__ __forceinline__ void store32_bf16(__nv_bfloat16 *dst, const float (&v
     }
 }
 
-// The input projection's epilogue for one 128 x 128 half tile held in TMEM at `tacc` (this
-// thread's lane, column 0 of the half).  Row r = 32 q + lane is token row m = m0 - 3 + r.
-__device__ __forceinline__ void epilogue_in(const ProjParams &p, uint32_t tacc, int mi, int ni, int half, int q,
-                                            int lane, int c_base, float *halo) {
+struct EpiSmem {
+    float *halo, *taps, *ss;
+};
+
+// The input projection's epilogue for one 128-row x 64-column quarter of a tile (this warp's
+// lane quarter q; TMEM address tacc = this thread's lane, the quarter's first column).  Row
+// r = 32 q + lane is token row m = m0 - 3 + r; sub = 64-column quarter of the 256-column tile
+// (head = sub / 2 of the tile's two heads, part = sub % 2 of its 128 columns).
+__device__ __forceinline__ void epilogue_in(const ProjParams &p, uint32_t tacc, int mi, int ni, int sub, int q,
+                                            int lane, int c_base, int tpar, const EpiSmem &es) {
     using namespace pj;
+    const int half = sub >> 1, part = sub & 1;
     const int r = q * 32 + lane;
     const int m = mi * p.m_step - kHist + r;
     const bool out_row = r >= kHist && m < p.M;
@@ -91,16 +106,16 @@ __device__ __forceinline__ void epilogue_in(const ProjParams &p, uint32_t tacc, 
     const int tt = m - bb * p.T;  // token within its batch item (valid for m >= 0)
     const int per_tensor = p.H / 2;
     if (ni >= 4 * per_tensor) {
-        // g | b tile: columns 0 .. H-1 are g, H .. 2H-1 are b (half 0 holds them all for H <= 64)
-        if (half != 0) return;
+        // g | b tile: columns 0 .. H-1 are g, H .. 2H-1 are b
         const size_t gi = static_cast<size_t>(m) * p.H;
-        for (int c = 0; c * 32 < 2 * p.H; ++c) {
+        const bool ok = out_row && debug_in_bounds(p.debug, gi, p.H, static_cast<size_t>(p.M) * p.H, p.status);
+        for (int cc = 0; cc < 2 && sub * 64 + 32 * cc < 2 * p.H; ++cc) {
             float x[32];
-            tmem_ld32(tacc + 32 * c, x);
-            if (out_row && debug_in_bounds(p.debug, gi, p.H, static_cast<size_t>(p.M) * p.H, p.status)) {
+            tmem_ld32(tacc + 32 * cc, x);
+            if (ok) {
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    const int col = 32 * c + e;
+                    const int col = sub * 64 + 32 * cc + e;
                     if (col < p.H) p.g[gi + col] = x[e];
                     else if (col < 2 * p.H) p.b[gi + col - p.H] = x[e];
                 }
@@ -110,84 +125,119 @@ __device__ __forceinline__ void epilogue_in(const ProjParams &p, uint32_t tacc, 
     }
     const int tensor = ni / per_tensor;               // 0 q, 1 k, 2 v, 3 z
     const int head = 2 * (ni - tensor * per_tensor) + half;
+    const int col0 = part * 64;                       // first column of this quarter within the head
     if (tensor == 3) {                                // z: no conv, fp16 out
-        __half *dst = p.z + static_cast<size_t>(m) * p.H * kD + static_cast<size_t>(head) * kD;
-        const bool ok = out_row && debug_in_bounds(p.debug, static_cast<size_t>(m) * p.H * kD + head * kD, kD,
-                                                   static_cast<size_t>(p.M) * p.H * kD, p.status);
+        const size_t o = static_cast<size_t>(m) * p.H * kD + static_cast<size_t>(head) * kD + col0;
+        const bool ok = out_row && debug_in_bounds(p.debug, o, 64, static_cast<size_t>(p.M) * p.H * kD, p.status);
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int cc = 0; cc < 2; ++cc) {
             float x[32];
-            tmem_ld32(tacc + 32 * c, x);
-            if (ok) store32_f16(dst + 32 * c, x, 1.0f);
+            tmem_ld32(tacc + 32 * cc, x);
+            if (ok) store32_f16(p.z + o + 32 * cc, x, 1.0f);
         }
         return;
     }
     const float *conv = tensor == 0 ? p.conv_q : (tensor == 1 ? p.conv_k : p.conv_v);
     __half *outp = tensor == 0 ? p.qh : (tensor == 1 ? p.kh : p.vh);
     const size_t orow = (static_cast<size_t>(bb) * p.H + head) * p.Tp + tt;
-    const bool ok = out_row && debug_in_bounds(p.debug, orow * kD, kD, static_cast<size_t>(p.B) * p.H * p.Tp * kD,
-                                               p.status);
-    __half *dst = outp + orow * kD;
+    const bool ok = out_row && debug_in_bounds(p.debug, orow * kD + col0, 64,
+                                               static_cast<size_t>(p.B) * p.H * p.Tp * kD, p.status);
+    __half *dst = outp + orow * kD + col0;
+    // the taps of this quarter's 64 channels, [tap][channel]; published by the first history barrier
+    float *taps = es.taps + sub * 256;
+    {
+        const int i = q * 32 + lane;  // 0 .. 127 over the sub's four warps
+        const float *src = conv + static_cast<size_t>(head * kD + col0) * 4;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int idx = i + 128 * k;  // channel idx / 4, tap idx % 4
+            taps[(idx & 3) * 64 + (idx >> 2)] = __ldg(src + idx);
+        }
+    }
+    // taps that reach before the batch item's first token read zero
+    const float m1 = tt >= 1 ? 1.0f : 0.0f, m2 = tt >= 2 ? 1.0f : 0.0f, m3 = tt >= 3 ? 1.0f : 0.0f;
     float ss = 0.0f;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int cc = 0; cc < 2; ++cc) {
         float x[32];
-        tmem_ld32(tacc + 32 * c, x);
+        tmem_ld32(tacc + 32 * cc, x);
         // publish this quarter's last 3 rows for the quarter below; slots alternate by chunk parity
-        const int par = (c_base + c) & 1;
-        float *mine = halo + ((par * 2 + half) * 4 + q) * HALO_SLOT;
-        const float *prev = halo + ((par * 2 + half) * 4 + ((q + 3) & 3)) * HALO_SLOT;
+        const int par = (c_base + cc) & 1;
+        float *mine = es.halo + ((par * 4 + sub) * 4 + q) * HALO_SLOT;
+        const float *prev = es.halo + ((par * 4 + sub) * 4 + ((q + 3) & 3)) * HALO_SLOT;
         if (lane >= 29) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) mine[(lane - 29) * 33 + e] = x[e];
+            for (int e4 = 0; e4 < 8; ++e4)
+                *reinterpret_cast<float4 *>(mine + (lane - 29) * 36 + 4 * e4) =
+                    make_float4(x[4 * e4], x[4 * e4 + 1], x[4 * e4 + 2], x[4 * e4 + 3]);
         }
-        named_sync(1 + half, 128);
-        const int ch0 = head * kD + 32 * c;
+        named_sync(2 + sub, 128);
+        // lane l < j takes row r - j from slot row 3 + l - j of the quarter above (other lanes
+        // read a clamped row and discard it)
+        const float *h1 = prev + min(2 + lane, 2) * 36, *h2 = prev + min(1 + lane, 2) * 36, *h3 = prev + min(lane, 2) * 36;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-            float x1 = __shfl_up_sync(0xffffffffu, x[e], 1);
-            float x2 = __shfl_up_sync(0xffffffffu, x[e], 2);
-            float x3 = __shfl_up_sync(0xffffffffu, x[e], 3);
-            // lane l < j takes row r - j from lane 32 + l - j of the quarter above (slot row 3 + l - j)
-            if (lane < 1) x1 = prev[(2 + lane) * 33 + e];
-            if (lane < 2) x2 = prev[(1 + lane) * 33 + e];
-            if (lane < 3) x3 = prev[lane * 33 + e];
-            const float4 w = __ldg(reinterpret_cast<const float4 *>(conv) + ch0 + e);  // tap 3: current token
-            float u = w.w * x[e];
-            if (tt >= 1) u = fmaf(w.z, x1, u);
-            if (tt >= 2) u = fmaf(w.y, x2, u);
-            if (tt >= 3) u = fmaf(w.x, x3, u);
-            u = silu_f(u);
-            ss = fmaf(u, u, ss);
-            x[e] = u;
+        for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 w0 = *reinterpret_cast<const float4 *>(taps + 0 * 64 + 32 * cc + 4 * e4);
+            const float4 w1 = *reinterpret_cast<const float4 *>(taps + 1 * 64 + 32 * cc + 4 * e4);
+            const float4 w2 = *reinterpret_cast<const float4 *>(taps + 2 * 64 + 32 * cc + 4 * e4);
+            const float4 w3 = *reinterpret_cast<const float4 *>(taps + 3 * 64 + 32 * cc + 4 * e4);
+            const float4 p1 = *reinterpret_cast<const float4 *>(h1 + 4 * e4);
+            const float4 p2 = *reinterpret_cast<const float4 *>(h2 + 4 * e4);
+            const float4 p3 = *reinterpret_cast<const float4 *>(h3 + 4 * e4);
+            const float w0a[4] = {w0.x, w0.y, w0.z, w0.w}, w1a[4] = {w1.x, w1.y, w1.z, w1.w};
+            const float w2a[4] = {w2.x, w2.y, w2.z, w2.w}, w3a[4] = {w3.x, w3.y, w3.z, w3.w};
+            const float p1a[4] = {p1.x, p1.y, p1.z, p1.w}, p2a[4] = {p2.x, p2.y, p2.z, p2.w};
+            const float p3a[4] = {p3.x, p3.y, p3.z, p3.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int e = 4 * e4 + i;
+                const float s1 = __shfl_up_sync(0xffffffffu, x[e], 1);
+                const float s2 = __shfl_up_sync(0xffffffffu, x[e], 2);
+                const float s3 = __shfl_up_sync(0xffffffffu, x[e], 3);
+                const float x1 = (lane < 1 ? p1a[i] : s1) * m1;
+                const float x2 = (lane < 2 ? p2a[i] : s2) * m2;
+                const float x3 = (lane < 3 ? p3a[i] : s3) * m3;
+                float u = w3a[i] * x[e];  // tap 3: the current token
+                u = fmaf(w2a[i], x1, u);
+                u = fmaf(w1a[i], x2, u);
+                u = fmaf(w0a[i], x3, u);
+                u = silu_f(u);
+                ss = fmaf(u, u, ss);
+                x[e] = u;
+            }
         }
         if (tensor == 2) {
-            if (ok) store32_f16(dst + 32 * c, x, 1.0f);
+            if (ok) store32_f16(dst + 32 * cc, x, 1.0f);
         } else {
-            tmem_st32(tacc + 32 * c, x);  // the activated value waits in TMEM for the head's norm
+            tmem_st32(tacc + 32 * cc, x);  // the activated value waits in TMEM for the head's norm
         }
     }
     if (tensor == 2) return;
+    // the head's sum of squares: this quarter's 64 columns plus the partner warp's other 64
+    float *ssl = es.ss + ((tpar * 2 + half) * 4 + q) * 64;
+    ssl[part * 32 + lane] = ss;
+    named_sync(6 + half, 256);
+    ss += ssl[(part ^ 1) * 32 + lane];
     tmem_st_wait();
     const float sc = rsqrtf(ss + p.l2_eps) * (tensor == 0 ? p.q_scale : 1.0f);
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int cc = 0; cc < 2; ++cc) {
         float x[32];
-        tmem_ld32(tacc + 32 * c, x);
-        if (ok) store32_f16(dst + 32 * c, x, sc);
+        tmem_ld32(tacc + 32 * cc, x);
+        if (ok) store32_f16(dst + 32 * cc, x, sc);
     }
 }
 
-// The output projection's epilogue: row m = m0 + r, columns n0 + 128 half + 32 c + e.
-__device__ __forceinline__ void epilogue_out(const ProjParams &p, uint32_t tacc, int mi, int ni, int half, int q,
+// The output projection's epilogue: row m = m0 + r, columns n0 + 64 sub + 32 cc + e.
+__device__ __forceinline__ void epilogue_out(const ProjParams &p, uint32_t tacc, int mi, int ni, int sub, int q,
                                              int lane) {
     const int m = mi * p.m_step + q * 32 + lane;
-    const int n0 = ni * pj::BN + half * 128;
+    const int n0 = ni * pj::BN + sub * 64;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int cc = 0; cc < 2; ++cc) {
         float x[32];
-        tmem_ld32(tacc + 32 * c, x);
-        const int n = n0 + 32 * c;
+        tmem_ld32(tacc + 32 * cc, x);
+        const int n = n0 + 32 * cc;
         if (m >= p.M || n >= p.N) continue;
         const size_t o = static_cast<size_t>(m) * p.N + n;
         if (!debug_in_bounds(p.debug, o, 32, static_cast<size_t>(p.M) * p.N, p.status)) continue;
@@ -212,7 +262,8 @@ __global__ void __launch_bounds__(pj::kThreads, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NBAR);
     AbortState *ab = reinterpret_cast<AbortState *>(tmem_slot + 1);
-    float *halo = reinterpret_cast<float *>(sm + OFF_HALO);
+    const EpiSmem es = {reinterpret_cast<float *>(sm + OFF_HALO), reinterpret_cast<float *>(sm + OFF_TAPS),
+                        reinterpret_cast<float *>(sm + OFF_SS)};
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ntiles = p.m_tiles * p.n_tiles;
     const int nkb = p.K / BK;
@@ -304,21 +355,22 @@ __global__ void __launch_bounds__(pj::kThreads, 1)
                     mbar_wait_drain(&bars[ACC_FULL + b2], (committed[STAGES + b2] - 1) & 1, lim);
         }
     } else {
-        const int q = warp & 3, half = (warp - 2) >> 2;
+        const int q = warp & 3, sub = (warp - 2) >> 2;
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         int local = 0, chunks = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
             const int buf = local & 1;
             const bool w = mbar_wait(&bars[ACC_FULL + buf], (local >> 1) & 1, ab, p.status, lim);
-            if (!group_all(1 + half, 128, w)) break;  // the half's four warps go on, or stop, together
+            // all epilogue warps go on, or stop, together: the head-level barrier below joins two subs
+            if (!group_all(1, 32 * kEpiWarps, w)) break;
             tc_fence_after();
             const int mi = t / p.n_tiles, ni = t - mi * p.n_tiles;
-            const uint32_t tacc = tmem + lane_base + buf * BN + half * 128;
+            const uint32_t tacc = tmem + lane_base + buf * BN + sub * 64;
             if (kMode == 0) {
-                epilogue_in(p, tacc, mi, ni, half, q, lane, chunks, halo);
-                chunks += 4;
+                epilogue_in(p, tacc, mi, ni, sub, q, lane, chunks, local & 1, es);
+                chunks += 2;
             } else {
-                epilogue_out(p, tacc, mi, ni, half, q, lane);
+                epilogue_out(p, tacc, mi, ni, sub, q, lane);
             }
             tc_fence_before();
             __syncwarp();
