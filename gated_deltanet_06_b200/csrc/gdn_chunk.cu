@@ -13,17 +13,18 @@
 // stores.  Only exponentials of non-positive differences of the cumulative
 // log decay G are taken.
 //
-// T = (I + L)^-1 by block forward substitution over the 8 x 8 grid of 16x16
-// blocks: the diagonal blocks D_i = (I + L_ii)^-1 by fp32 column solves (one
-// thread per column, 16 rows); then, all at once, M_ik = D_i L_ik for k < i;
-// then block row by block row
-//     T_ij = -D_i sum_{k=j}^{i-1} L_ik T_kj = -sum_{k=j}^{i-1} M_ik T_kj,  j < i,
-// all as warp-level tensor-core products (mma.sync m16n8k16, fp16 operands
-// fetched with ldmatrix from the swizzled tile, fp32 accumulation).  L, then
-// M, then T live in one tile, each block overwritten in place once its last
-// reader is done: T comes out directly in the K-major operand layout of
-// W = T K~ and U = T V~.  Seven short dependent levels replace a 128-step
-// serial solve.
+// T = (I + L)^-1 over the 8 x 8 grid of 16x16 blocks: the diagonal blocks
+// D_i = (I + L_ii)^-1 by fp32 column solves (one thread per column, 16 rows);
+// then three doubling levels, each joining pairs of inverted diagonal blocks
+// of size n into inverses of size 2n by
+//     [[A11, 0], [L21, A22]]^-1 = [[T11, 0], [-T22 L21 T11, T22]],
+// as warp-level tensor-core products (mma.sync m16n8k16, fp16 operands
+// fetched with ldmatrix from the swizzled tile, fp32 accumulation; the
+// intermediate T22 L21 passes from accumulator to operand fragments in
+// registers).  L and T live in one tile, each block overwritten in place
+// once its last reader is done: T comes out directly in the K-major operand
+// layout of W = T K~ and U = T V~.  Three dependent levels of two products
+// each replace a 128-step serial solve.
 //
 // Two warp groups work side by side.  Warps 0-3 evaluate the gates, build L
 // and invert I + L.  Warps 4-7 write Kt straight from the K tile to global
@@ -298,73 +299,138 @@ __global__ void __launch_bounds__(256, 2)
         group_sync(1);
         if (tid == 0) GDN_TRACE_AT(3);
 
-        // ---- M_ik = D_i L_ik (k < i), over L_ik: the 28 blocks spread over the four warps, both
-        //      16x8 halves of a block read before either is written
+        // ---- T by recursive doubling over the diagonal blocks: with the 16x16 inverses D_b on the
+        //      diagonal and L below it, level s (s = 1, 2, 3) joins pairs of 2^(s-1) blocks into
+        //      inverses of 2^s blocks: for [[A11, 0], [L21, A22]], T21 = -T22 L21 T11.  Z = T22 L21
+        //      accumulates in registers (fp32), becomes the A operand of Z T11 in fp16, and -Z T11 is
+        //      written over L21.  Warp w computes block row(s) of its own output; a barrier separates
+        //      the last read of a level's L21 from the first write over it.
         const uint32_t tT = sbase + OFF_LT;
         uint8_t *Tt = sm + OFF_LT;
         const int g = lane >> 2, t4 = lane & 3;
         const int lm = lane >> 3, lr = lane & 7;
         const int arow = (lm & 1) * 8 + lr, achk = lm >> 1;  // ldmatrix row / 16-byte chunk of this lane
-#pragma unroll 1
-        for (int q = warp; q < 28; q += 4) {
-            int i = 1;
-            while (q >= i * (i + 1) / 2) ++i;  // q = i(i-1)/2 + k
-            const int k = q - i * (i - 1) / 2;
-            uint32_t a[4], b0[2], b1[2];
-            ldsm_x4(tT + tile_off(128, 16 * i + arow, 2 * i + achk), a);
-            ldsm_x2_trans(tT + tile_off(128, 16 * i + arow, 2 * k), b0);
-            ldsm_x2_trans(tT + tile_off(128, 16 * i + arow, 2 * k + 1), b1);
-            float o0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, o1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-            mma16816(o0, a, b0);
-            mma16816(o1, a, b1);
+        // A fragment of block (R, K); B fragments (two 8-column halves) of block (K, J)
+        auto lda = [&](int R, int K, uint32_t (&a)[4]) { ldsm_x4(tT + tile_off(128, 16 * R + arow, 2 * K + achk), a); };
+        auto ldb = [&](int K, int J, int hf, uint32_t (&b)[2]) {
+            ldsm_x2_trans(tT + tile_off(128, 16 * K + arow, 2 * J + hf), b);
+        };
+        // C fragments (two 8-column halves of a 16x16 block) -> the A fragment of that block, fp16
+        auto c2a = [&](const float (&c0)[4], const float (&c1)[4], uint32_t (&a)[4]) {
+            a[0] = pack_half2(c0[0], c0[1]);
+            a[1] = pack_half2(c0[2], c0[3]);
+            a[2] = pack_half2(c1[0], c1[1]);
+            a[3] = pack_half2(c1[2], c1[3]);
+        };
+        auto put_neg = [&](int R, int J, const float (&c0)[4], const float (&c1)[4]) {
+            const int col = 16 * J + 2 * t4;
+            *reinterpret_cast<uint32_t *>(Tt + tile_elem_off(128, 16 * R + g, col)) = pack_half2(-c0[0], -c0[1]);
+            *reinterpret_cast<uint32_t *>(Tt + tile_elem_off(128, 16 * R + g + 8, col)) = pack_half2(-c0[2], -c0[3]);
+            *reinterpret_cast<uint32_t *>(Tt + tile_elem_off(128, 16 * R + g, col + 8)) = pack_half2(-c1[0], -c1[1]);
+            *reinterpret_cast<uint32_t *>(Tt + tile_elem_off(128, 16 * R + g + 8, col + 8)) = pack_half2(-c1[2], -c1[3]);
+        };
+        // level 1: pairs (2w, 2w+1), one per warp: T_{2w+1,2w} = -D_{2w+1} L_{2w+1,2w} D_{2w}
+        {
+            const int R = 2 * warp + 1, J = 2 * warp;
+            uint32_t a[4], b[2];
+            float z0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, z1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            lda(R, R, a);
+            ldb(R, J, 0, b);
+            mma16816(z0, a, b);
+            ldb(R, J, 1, b);
+            mma16816(z1, a, b);
+            c2a(z0, z1, a);
+            float y0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, y1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            ldb(J, J, 0, b);
+            mma16816(y0, a, b);
+            ldb(J, J, 1, b);
+            mma16816(y1, a, b);
             __syncwarp();
-            const int col = 16 * k + 2 * t4;
-            *reinterpret_cast<uint32_t *>(Tt + tile_elem_off(128, 16 * i + g, col)) = pack_half2(o0[0], o0[1]);
-            *reinterpret_cast<uint32_t *>(Tt + tile_elem_off(128, 16 * i + g + 8, col)) = pack_half2(o0[2], o0[3]);
-            *reinterpret_cast<uint32_t *>(Tt + tile_elem_off(128, 16 * i + g, col + 8)) = pack_half2(o1[0], o1[1]);
-            *reinterpret_cast<uint32_t *>(Tt + tile_elem_off(128, 16 * i + g + 8, col + 8)) = pack_half2(o1[2], o1[3]);
+            put_neg(R, J, y0, y1);
         }
         group_sync(1);
         if (tid == 0) GDN_TRACE_AT(20);
-        // ---- block rows i = 1..7: T_ij = -sum_{k=j}^{i-1} M_ik T_kj, as two 16x8 halves each; the
-        //      2i halves of a level are spread over the four warps, computed, then (after a barrier,
-        //      since M_ij is still read by the level's other halves) written over M_ij
-        //      A warp's halves q = warp + 4 sl (j = q / 2, column half q % 2) advance together over k,
-        //      sharing the A fragment M_ik: up to four independent accumulation chains.
-#pragma unroll 1
-        for (int i = 1; i < 8; ++i) {
-            float acc[4][4];
+        // level 2: 64-blocks q = 0, 1 (blocks 4q .. 4q+3); warp w takes output block row R = 4q+2+i
+        {
+            const int q = warp >> 1, i = warp & 1;
+            const int R = 4 * q + 2 + i, J0 = 4 * q;
+            float z[2][2][4];
 #pragma unroll
-            for (int sl = 0; sl < 4; ++sl) acc[sl][0] = acc[sl][1] = acc[sl][2] = acc[sl][3] = 0.0f;
-#pragma unroll 1
-            for (int k = 0; k < i; ++k) {
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) z[j][h][0] = z[j][h][1] = z[j][h][2] = z[j][h][3] = 0.0f;
+            for (int K = 4 * q + 2; K <= R; ++K) {  // Z = T22 L21, row R
                 uint32_t a[4];
-                ldsm_x4(tT + tile_off(128, 16 * i + arow, 2 * k + achk), a);
+                lda(R, K, a);
 #pragma unroll
-                for (int sl = 0; sl < 4; ++sl) {
-                    const int q = warp + 4 * sl;
-                    if (q < 2 * i && (q >> 1) <= k) {
-                        uint32_t bq[2];
-                        ldsm_x2_trans(tT + tile_off(128, 16 * k + arow, q), bq);  // chunk 2j + hf = q
-                        mma16816(acc[sl], a, bq);
+                for (int j = 0; j < 2; ++j)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t b[2];
+                        ldb(K, J0 + j, h, b);
+                        mma16816(z[j][h], a, b);
                     }
-                }
             }
-            group_sync(1);
+            group_sync(1);  // every read of this level's L21 is done
+            uint32_t za[2][4];
 #pragma unroll
-            for (int sl = 0; sl < 4; ++sl) {
-                const int q = warp + 4 * sl;
-                if (q < 2 * i) {
-                    const int col = 16 * (q >> 1) + 8 * (q & 1) + 2 * t4;
-                    *reinterpret_cast<uint32_t *>(Tt + tile_elem_off(128, 16 * i + g, col)) =
-                        pack_half2(-acc[sl][0], -acc[sl][1]);
-                    *reinterpret_cast<uint32_t *>(Tt + tile_elem_off(128, 16 * i + g + 8, col)) =
-                        pack_half2(-acc[sl][2], -acc[sl][3]);
+            for (int j = 0; j < 2; ++j) c2a(z[j][0], z[j][1], za[j]);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {  // Y = Z T11, row R: Y_j = sum_{k >= j} Z_k T11_kj
+                float y0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, y1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+                for (int k = j; k < 2; ++k) {
+                    uint32_t b[2];
+                    ldb(J0 + k, J0 + j, 0, b);
+                    mma16816(y0, za[k], b);
+                    ldb(J0 + k, J0 + j, 1, b);
+                    mma16816(y1, za[k], b);
                 }
+                put_neg(R, J0 + j, y0, y1);
             }
-            group_sync(1);
-            if (tid == 0) GDN_TRACE_AT(20 + i);
         }
+        group_sync(1);
+        if (tid == 0) GDN_TRACE_AT(21);
+        // level 3: the 128-block; warp w takes output block row R = 4 + w
+        {
+            const int R = 4 + warp;
+            float z[4][2][4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) z[j][h][0] = z[j][h][1] = z[j][h][2] = z[j][h][3] = 0.0f;
+            for (int K = 4; K <= R; ++K) {  // Z = T22 L21, row R
+                uint32_t a[4];
+                lda(R, K, a);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t b[2];
+                        ldb(K, j, h, b);
+                        mma16816(z[j][h], a, b);
+                    }
+            }
+            group_sync(1);  // every read of L21 is done
+            uint32_t za[4][4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) c2a(z[j][0], z[j][1], za[j]);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {  // Y = Z T11, row R
+                float y0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, y1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+                for (int k = j; k < 4; ++k) {
+                    uint32_t b[2];
+                    ldb(k, j, 0, b);
+                    mma16816(y0, za[k], b);
+                    ldb(k, j, 1, b);
+                    mma16816(y1, za[k], b);
+                }
+                put_neg(R, j, y0, y1);
+            }
+        }
+        group_sync(1);
+        if (tid == 0) GDN_TRACE_AT(22);
         fence_proxy_async();  // T is read by the tensor cores next
         if (tid == 0) GDN_TRACE_AT(4);
     } else {
