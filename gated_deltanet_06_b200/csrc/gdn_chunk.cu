@@ -9,8 +9,8 @@
 //   Kt   = diag(e^(G_last - G)) K,  Qt = diag(e^G) Q,
 //   Aqk  = [i <= r] e^(G_r - G_i) QK_ri
 //
-// and stores W, U, Kt, Qt, Aqk (fp16) for the inter-block scan with TMA bulk
-// stores.  Only exponentials of non-positive differences of the cumulative
+// and stores W, U, Kt, Qt, Aqk (fp16) for the inter-block scan (TMA bulk
+// stores for W, U, Qt; plain 16-byte stores for Kt and Aqk).  Only exponentials of non-positive differences of the cumulative
 // log decay G are taken.
 //
 // T = (I + L)^-1 over the 8 x 8 grid of 16x16 blocks: the diagonal blocks
@@ -26,20 +26,20 @@
 // layout of W = T K~ and U = T V~.  Three dependent levels of two products
 // each replace a 128-step serial solve.
 //
-// Two warp groups work side by side.  Warps 0-3 evaluate the gates, build L
-// and invert I + L.  Warps 4-7 write Kt straight from the K tile to global
-// memory while scaling the tile in place into K~ = diag(beta e^G) K, build Qt
-// and Aqk and store them, load the V tile and scale it into V~ = diag(beta) V,
-// so that T enters both products unscaled.  The decay factors of L and Aqk
+// Two warp groups work side by side.  Warps 0-3 evaluate the gates, build L,
+// invert I + L, then build Aqk and store it straight to global memory.  Warps
+// 4-7 write Kt straight from the K tile to global memory while scaling the
+// tile in place into K~ = diag(beta e^G) K, build Qt and store it, load the V
+// tile and scale it into V~ = diag(beta) V, so that T enters both products
+// unscaled.  The decay factors of L and Aqk
 // below the diagonal 32x32 blocks are split as e^(G_r - G_m) e^(G_m - G_j) (m
 // the last row of j's 32-row group, both exponents <= 0): one exponential per
 // row and per column instead of one per entry.
 //
 // Footprint: about 108 KB of shared memory and 256 TMEM columns, so that two
 // CTAs share an SM.  Shared memory is reused through the block's life: the K
-// tile becomes K~; the Q tile becomes Qt, then the staging area of Aqk, then
-// V~, then the staging area of U; the L tile becomes M and T, then the staging
-// area of W.
+// tile becomes K~; the Q tile becomes Qt, then V~, then the staging area of U;
+// the L tile becomes T, then the staging area of W.
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 
@@ -48,8 +48,8 @@ namespace {
 
 // Shared-memory map (offsets from a 1024-byte aligned base).
 constexpr uint32_t OFF_K = 0;           // 128x128 fp16 panel tile: K -> K~
-constexpr uint32_t OFF_QV = 32768;      // 128x128 fp16: Q -> Qt -> Aqk staging -> V~ -> U staging
-constexpr uint32_t OFF_LT = 65536;      // 128x128 fp16: L -> M -> T (K-major A operand) -> W staging
+constexpr uint32_t OFF_QV = 32768;      // 128x128 fp16: Q -> Qt -> V~ -> U staging
+constexpr uint32_t OFF_LT = 65536;      // 128x128 fp16: L -> T (K-major A operand) -> W staging
 constexpr uint32_t OFF_LDIAG = 98304;   // fp32 [8][16][16]: the diagonal 16x16 blocks of L
 constexpr uint32_t OFF_G = OFF_LDIAG + 8192;    // fp32 [128]
 constexpr uint32_t OFF_BETA = OFF_G + 512;      // fp32 [128]
@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(256, 2)
 
     const int blk = blockIdx.x, bh = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const bool groupL = tid < 128;  // warps 0-3: gates, L, T;  warps 4-7: Kt, K~, Qt, Aqk, V~
+    const bool groupL = tid < 128;  // warps 0-3: gates, L, T, Aqk;  warps 4-7: Kt, K~, Qt, V~
     const int r = tid & 127;        // TMEM lane / row (or column of T) owned by this thread
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const size_t row0 = static_cast<size_t>(bh) * p.Tp + static_cast<size_t>(blk) * kBlk;
@@ -433,6 +433,43 @@ __global__ void __launch_bounds__(256, 2)
         if (tid == 0) GDN_TRACE_AT(22);
         fence_proxy_async();  // T is read by the tensor cores next
         if (tid == 0) GDN_TRACE_AT(4);
+        // ---- Aqk rows (the decay split as for the L rows), stored straight to global memory: a
+        //      block's 128 rows are 32 contiguous KB.  Aqk is block lower triangular; its upper-right
+        //      64x64 quadrant (zero) is never stored, the rest is, zeros above the diagonal included.
+        {
+            __half *arow_g = p.Aqk + (row0 + r) * 128;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                if (r < 64 && c >= 2) break;
+                float a[32];
+                if (c > warp) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) a[i] = 0.0f;
+                } else {
+                    tmem_ld32(tmem + lane_base + TM_QK + c * 32, a);
+                    if (c < warp) {
+                        const float fr = __expf(fminf(Gr - sG[c * 32 + 31], 0.0f));
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) a[i] *= fr * sEc[c * 32 + i];
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const int j = c * 32 + i;
+                            a[i] = (j <= r) ? __expf(fminf(Gr - sG[j], 0.0f)) * a[i] : 0.0f;
+                        }
+                    }
+                }
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint4 u;
+                    u.x = pack_half2(a[8 * q4], a[8 * q4 + 1]);
+                    u.y = pack_half2(a[8 * q4 + 2], a[8 * q4 + 3]);
+                    u.z = pack_half2(a[8 * q4 + 4], a[8 * q4 + 5]);
+                    u.w = pack_half2(a[8 * q4 + 6], a[8 * q4 + 7]);
+                    *reinterpret_cast<uint4 *>(arow_g + c * 32 + q4 * 8) = u;
+                }
+            }
+        }
     } else {
         // ---- Kt = e^(G_last - G) K straight to global memory, and the K tile scaled in place into
         //      K~ = diag(beta e^G) K (the A_kk product, K's last reader, is complete).  Each warp
@@ -475,40 +512,7 @@ __global__ void __launch_bounds__(256, 2)
         }
         group_sync(2);
         if (tid == 128) GDN_TRACE_AT(11);
-        // ---- Aqk rows (same split of the decay as the L rows) staged in the same area -> bulk
-        //      store; then the V tile is loaded into it
-        const int w = warp & 3;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-            float a[32];
-            if (c > w) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) a[i] = 0.0f;
-            } else {
-                tmem_ld32(tmem + lane_base + TM_QK + c * 32, a);
-                if (c < w) {
-                    const float fr = __expf(fminf(Gr - sG[c * 32 + 31], 0.0f));
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) a[i] *= fr * sEc[c * 32 + i];
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int j = c * 32 + i;
-                        a[i] = (j <= r) ? __expf(fminf(Gr - sG[j], 0.0f)) * a[i] : 0.0f;
-                    }
-                }
-            }
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) put8(sm + OFF_QV, 128, r, c * 4 + q4, &a[q4 * 8]);
-        }
-        fence_proxy_async();
-        group_sync(2);
-        if (tid == 128) {
-            // Aqk is block lower triangular: its upper-right 64x64 quadrant (zero) is not stored
-            tma_store_2d(&tmAqk, sm + OFF_QV, 0, y0);
-            tma_store_2d(&tmAqkH, sm + OFF_QV + 16384 + 64 * 128, 64, y0 + 64);
-            bulk_commit();
-            bulk_wait_read_all();
+        if (tid == 128) {  // the Q area is free again: V goes into it
             mbar_arrive_expect_tx(bar_v, 32768u);
             tma_load_2d(sm + OFF_QV, &tmV, bar_v, 0, y0);
             tma_load_2d(sm + OFF_QV + 16384, &tmV, bar_v, 64, y0);
