@@ -793,6 +793,13 @@ def main():
     ach_tfs = pf * units / t_top / 1e12
     kb, kf = kernel_work_per_token_head(top, w.d, s_in, s_out)
     traffic = ncu_traffic(top, w.name)
+    # the whole forward's DRAM bytes (every kernel's capture, while all their sources are unchanged)
+    path_traffic = None
+    kt = [ncu_traffic(n, w.name) for n in names]
+    if all(x is not None for x in kt):
+        path_traffic = {"bytes_per_step": int(sum(kt)), "per_kernel": {n: int(x) for n, x in zip(names, kt)},
+                        "algorithmic_bytes_per_step": int(path_bytes_per_token_head(w.d, s_in, s_out) * w.B * w.T * w.H),
+                        "ratio": sum(kt) / (path_bytes_per_token_head(w.d, s_in, s_out) * w.B * w.T * w.H)}
     roof = {"bound": "hbm", "achieved": ach_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": ach_gbs / peaks["hbm_gbs"], "traffic": traffic,
             "peak_source": ("measured (MEASURED_PEAKS.json)" if peaks["source"] == "measured" else "fallback"),
@@ -811,6 +818,7 @@ def main():
                            path="fused tensor (FLAG_FUSED)" if args.fused else
                            ("tensor" if plan.uses_tensor_path else "CUDA-core fp32")),
             "roofline": roof, "path_roofline": path_roof, "path_roofline_frac": path_roof["frac"],
+            "path_traffic": path_traffic,
             "kernels_ms": kern_ms,
             "segments": plan.segments, "cpu_baseline": cpu, "e2e": e2e, "state_io": state_io,
             "reverse": reverse, "backward": bwd, "fused": fused, "graph": graph, "block": block,
