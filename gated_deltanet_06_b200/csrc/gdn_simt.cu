@@ -10,57 +10,99 @@
 namespace gdn {
 namespace {
 
-// Thread i owns row i of S (d_k values in registers).  Per token:
+// Four threads own row i of S, a quarter of its d_k values each, in registers.  Per token:
 //   u = S_i . k;  S_i <- alpha (S_i - beta u k) + beta v_i k;  o_i = S_i . q^
-// (q^ already carries 1/sqrt(d_k)).  Rows of S evolve independently, so no
-// cross-thread reduction is needed; k, q, v tiles of 16 tokens are staged in
-// shared memory.
+// (q^ already carries 1/sqrt(d_k)).  Rows of S evolve independently; the two dot products of a
+// row are split over its four threads in four short partial sums each and added with two
+// shuffles, so that a token costs a few dependent steps rather than a d_k-long chain.  k, q, v
+// tiles of 16 tokens (8 at d_k = 128) are double-buffered in shared memory, the next tile's global loads in
+// flight in registers while the current one is processed.
 template <int D>
-__global__ void __launch_bounds__(D) gdn_recurrence_kernel(const RecurParams p) {
-    constexpr int TT = 16;
-    __shared__ float sk[TT][D], sq[TT][D], sv[TT][D], sa[TT], sb[TT];
-    const int h = blockIdx.x, b = blockIdx.y, i = threadIdx.x;
+__global__ void __launch_bounds__(4 * D) gdn_recurrence_kernel(const RecurParams p) {
+    constexpr int TT = D == 128 ? 8 : 16, Q = D / 4;  // tokens per staged tile (48 KB of static smem); columns per thread
+    __shared__ __align__(16) float sk[2][TT][D];
+    __shared__ __align__(16) float sq[2][TT][D];
+    __shared__ float sv[2][TT][D], sa[2][TT], sb[2][TT];
+    const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+    const int i = tid >> 2, part = tid & 3, j0 = part * Q;  // row of S; this thread's columns j0 .. j0+Q-1
     const size_t bh = static_cast<size_t>(b) * p.H + h;
-    float S[D];  // row i of the state (d_v index i, d_k index j)
-    const float *s0 = p.s0 ? p.s0 + (bh * D + i) * D : nullptr;
+    float S[Q];
+    const float *s0 = p.s0 ? p.s0 + (bh * D + i) * D + j0 : nullptr;
 #pragma unroll
-    for (int j = 0; j < D; ++j) S[j] = s0 ? s0[j] : 0.0f;
-    for (int t0 = 0; t0 < p.T; t0 += TT) {
-        __syncthreads();
-#pragma unroll 4
-        for (int tok = 0; tok < TT; ++tok) {
-            const size_t rrow = (bh * p.Tp + t0 + tok) * D + i;
-            sk[tok][i] = p.kh[rrow];
-            sq[tok][i] = p.qh[rrow];
-            sv[tok][i] = p.vh[rrow];
+    for (int j = 0; j < Q; ++j) S[j] = s0 ? s0[j] : 0.0f;
+    // this thread's share of a tile: TT / 4 elements of each of k, q, v (and one gate pair)
+    constexpr int PER = TT * D / (4 * D);
+    float rk[PER], rq[PER], rv[PER], ra = 0.0f, rb = 0.0f;
+    auto fetch = [&](int t0) {  // global -> registers
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+            const int idx = tid + e * 4 * D, tok = idx / D, c = idx - tok * D;
+            const size_t rrow = (bh * p.Tp + t0 + tok) * D + c;
+            rk[e] = p.kh[rrow];
+            rq[e] = p.qh[rrow];
+            rv[e] = p.vh[rrow];
         }
-        if (i < TT) {
-            sa[i] = expf(p.log_alpha[bh * p.Tp + t0 + i]);
-            sb[i] = p.beta[bh * p.Tp + t0 + i];
+        if (tid < TT) {
+            ra = expf(p.log_alpha[bh * p.Tp + t0 + tid]);
+            rb = p.beta[bh * p.Tp + t0 + tid];
         }
-        __syncthreads();
+    };
+    auto stage = [&](int buf) {  // registers -> shared memory
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+            const int idx = tid + e * 4 * D, tok = idx / D, c = idx - tok * D;
+            sk[buf][tok][c] = rk[e];
+            sq[buf][tok][c] = rq[e];
+            sv[buf][tok][c] = rv[e];
+        }
+        if (tid < TT) {
+            sa[buf][tid] = ra;
+            sb[buf][tid] = rb;
+        }
+    };
+    fetch(0);
+    stage(0);
+    __syncthreads();
+    for (int t0 = 0, buf = 0; t0 < p.T; t0 += TT, buf ^= 1) {
+        const bool more = t0 + TT < p.T;
+        if (more) fetch(t0 + TT);  // the next tile's loads are in flight while this one is processed
         const int n = min(TT, p.T - t0);
         for (int tok = 0; tok < n; ++tok) {
-            float u = 0.0f;
+            float k[Q], q[Q];
 #pragma unroll
-            for (int j = 0; j < D; ++j) u = fmaf(S[j], sk[tok][j], u);
-            const float a = sa[tok], be = sb[tok];
-            const float c1 = be * u, c2 = be * sv[tok][i];
-            float o = 0.0f;
-#pragma unroll
-            for (int j = 0; j < D; ++j) {
-                const float kj = sk[tok][j];
-                S[j] = fmaf(a, fmaf(-c1, kj, S[j]), c2 * kj);
-                o = fmaf(S[j], sq[tok][j], o);
+            for (int j = 0; j < Q; j += 4) {
+                const float4 k4 = *reinterpret_cast<const float4 *>(&sk[buf][tok][j0 + j]);
+                const float4 q4 = *reinterpret_cast<const float4 *>(&sq[buf][tok][j0 + j]);
+                k[j] = k4.x; k[j + 1] = k4.y; k[j + 2] = k4.z; k[j + 3] = k4.w;
+                q[j] = q4.x; q[j + 1] = q4.y; q[j + 2] = q4.z; q[j + 3] = q4.w;
             }
+            float u4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+            for (int j = 0; j < Q; ++j) u4[j & 3] = fmaf(S[j], k[j], u4[j & 3]);
+            float u = (u4[0] + u4[1]) + (u4[2] + u4[3]);
+            u += __shfl_xor_sync(0xffffffffu, u, 1);
+            u += __shfl_xor_sync(0xffffffffu, u, 2);
+            const float a = sa[buf][tok], be = sb[buf][tok];
+            const float c1 = be * u, c2 = be * sv[buf][tok][i];
+            float o4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+            for (int j = 0; j < Q; ++j) {
+                S[j] = fmaf(a, fmaf(-c1, k[j], S[j]), c2 * k[j]);
+                o4[j & 3] = fmaf(S[j], q[j], o4[j & 3]);
+            }
+            float o = (o4[0] + o4[1]) + (o4[2] + o4[3]);
+            o += __shfl_xor_sync(0xffffffffu, o, 1);
+            o += __shfl_xor_sync(0xffffffffu, o, 2);
             const int to = p.rev ? p.T - 1 - (t0 + tok) : t0 + tok;  // input token order
-            p.o[((static_cast<size_t>(b) * p.T + to) * p.H + h) * D + i] = o;
+            if (part == 0) p.o[((static_cast<size_t>(b) * p.T + to) * p.H + h) * D + i] = o;
         }
+        if (more) stage(buf ^ 1);  // the other buffer's last readers finished before the previous barrier
+        __syncthreads();
     }
     if (p.s_end) {
-        float *se = p.s_end + (bh * D + i) * D;
+        float *se = p.s_end + (bh * D + i) * D + j0;
 #pragma unroll
-        for (int j = 0; j < D; ++j) se[j] = S[j];
+        for (int j = 0; j < Q; ++j) se[j] = S[j];
     }
 }
 
@@ -142,9 +184,9 @@ cudaError_t launch_out_z(const OutParams &p, InType yt, cudaStream_t s) {
 cudaError_t launch_recurrence(const RecurParams &p, cudaStream_t s) {
     dim3 grid(p.H, p.B);
     if (p.d == 128)
-        gdn_recurrence_kernel<128><<<grid, 128, 0, s>>>(p);
+        gdn_recurrence_kernel<128><<<grid, 512, 0, s>>>(p);
     else
-        gdn_recurrence_kernel<64><<<grid, 64, 0, s>>>(p);
+        gdn_recurrence_kernel<64><<<grid, 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 
