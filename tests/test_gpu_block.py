@@ -43,7 +43,8 @@ def _run(inp, out_dtype, flags=0):
 
 
 @pytest.mark.parametrize("B,T,H,D", [(1, 300, 2, 256), (1, 129, 2, 128), (2, 1001, 4, 512), (3, 250, 2, 192),
-                                     (1, 4000, 12, 1536)])
+                                     (1, 4000, 12, 1536), (1, 1, 2, 128), (2, 3, 2, 128), (1, 125, 2, 64),
+                                     (3, 126, 4, 320)])
 def test_block_matches_oracle_fp32_out(B, T, H, D):
     import torch
     inp = gdn_inputs.make_block_inputs(B, T, H, 128, D, seed=T + D)
