@@ -252,7 +252,7 @@ def reference_arm(args, w):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": dict(workload_config(w, args.out_dtype, 1), sample_T=T_s),
+            "config": workload_config(w, args.out_dtype, max(1, args.gpus)), "sample_T": T_s,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -814,9 +814,8 @@ def main():
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f16-mma/f32" if plan.uses_tensor_path else "f32", "data": "synthetic",
-            "config": dict(workload_config(w, args.out_dtype, world),
-                           path="fused tensor (FLAG_FUSED)" if args.fused else
-                           ("tensor" if plan.uses_tensor_path else "CUDA-core fp32")),
+            "config": workload_config(w, args.out_dtype, world),
+            "path": "fused tensor (FLAG_FUSED)" if args.fused else ("tensor" if plan.uses_tensor_path else "CUDA-core fp32"),
             "roofline": roof, "path_roofline": path_roof, "path_roofline_frac": path_roof["frac"],
             "path_traffic": path_traffic,
             "kernels_ms": kern_ms,
