@@ -122,3 +122,29 @@ def test_sample_text():
     w = gdn_inputs.HEADLINE
     assert bench.sample_text(w, w.T).startswith("the whole")
     assert "T=1000 instead of" in bench.sample_text(w, 1000)
+
+
+def test_block_flops_per_layer():
+    # x W_in^T: M = B*T rows, N = 4*H*d + 2*H, K = D; y W_out^T: M, N = D, K = H*d
+    w = gdn_inputs.HEADLINE
+    f_in, f_out = bench.block_flops(w, 1536)
+    M = w.B * w.T
+    assert f_in == 2 * M * (4 * 1536 + 2 * 12) * 1536
+    assert f_out == 2 * M * 1536 * 1536
+    # the T3-Video page's Table 1 counts 7.0T QKV and 2.3T O MACs over the 30 layers of Wan2.1-1.3B at
+    # 480x832x81f; one layer's q, k, v and o projections here are 3 and 1 of those D x D products
+    qkv_macs_per_layer = 3 * M * 1536 * 1536
+    assert 30 * qkv_macs_per_layer == pytest.approx(7.0e12, rel=0.01)
+    assert 30 * M * 1536 * 1536 == pytest.approx(2.3e12, rel=0.02)
+
+
+def test_recorded_traffic_covers_every_forward_kernel():
+    # profiles/dram_traffic.json holds one full-size capture per kernel of the tensor path; the sum is
+    # the path's DRAM bytes, reported beside the method's 1288 B per token-head
+    w = gdn_inputs.HEADLINE
+    names = bench.KERNELS_TENSOR_SEG
+    kt = [bench.ncu_traffic(n, w.name) for n in names]
+    if any(x is None for x in kt):
+        pytest.skip("a kernel changed since its capture")
+    assert sum(kt) > bench.path_bytes_per_token_head(128, 2, 2) * w.B * w.T * w.H
+    assert kt[names.index("chunk")] <= bench.kernel_work_per_token_head("chunk", 128, 2, 2)[0] * w.B * w.T * w.H
