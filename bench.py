@@ -435,6 +435,24 @@ def bench_block(w, dev, flush, stream, steps, world, dist):
     return res
 
 
+def backward_kernel_names(launches: int):
+    """Names of gdn_backward's launches in order: the tensor-core backward (12 launches, or 8 with
+    one segment per sequence) or the fp32 CUDA-core backward (6)."""
+    if launches == 6:
+        return ("prep_f32", "fwd_rows", "out_bwd", "core_bwd", "tokens_bwd", "params")
+    if launches == 12:
+        return ("prep", "ut_keep", "transfer", "combine", "scan_out_o", "out_bwd", "bwd_transfer", "bwd_combine",
+                "bwd_scan", "bwd_grad", "tokens_bwd", "params")
+    if launches == 8:
+        return ("prep", "ut_keep", "scan_out_o", "out_bwd", "bwd_scan", "bwd_grad", "tokens_bwd", "params")
+    raise ValueError(launches)
+
+
+def backward_grad_flops(bh: int, blocks: int) -> float:
+    """FLOPs of the block-gradient kernel: 16 products of 128 x 128 x 128 per 128-token block."""
+    return 16 * 2.0 * 128 ** 3 * bh * blocks
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -661,10 +679,15 @@ def main():
         flush.zero_()
         plan.backward_timed_raw(ptrs, dy.data_ptr(), gp, ws_b.data_ptr(), s, [e.cuda_event for e in evk])
         torch.cuda.synchronize()
-        bnames = ("prep_f32", "fwd_rows", "out_bwd", "core_bwd", "tokens_bwd", "params")
+        bnames = backward_kernel_names(LB)
+        kms = {bnames[i]: evk[i].elapsed_time(evk[i + 1]) for i in range(LB)}
         bwd = {"ms_per_step": b_ms, "value": job_throughput(world, w.B * w.T, b_ms), "unit": UNIT,
-               "steps": n_b, "launches_per_step": LB, "precision": "fp32 CUDA cores",
-               "kernels_ms": {bnames[i]: evk[i].elapsed_time(evk[i + 1]) for i in range(LB)}}
+               "steps": n_b, "launches_per_step": LB,
+               "precision": ("fp16 tensor-core operands, fp32 accumulation" if LB != 6 else "fp32 CUDA cores"),
+               "vs_forward": b_ms / ms_per_step, "kernels_ms": kms}
+        if "bwd_grad" in kms:  # the block-gradient kernel: 16 products of 128 x 128 x 128 per block
+            fl = backward_grad_flops(w.B * w.H, -(-w.T // 128))
+            bwd["bwd_grad_tflops"] = fl / (kms["bwd_grad"] / 1e3) / 1e12
         del ws_b, gr, dy
 
     # end to end through the public host-buffer entry point (gdn_forward_host: every input copied from

@@ -67,6 +67,8 @@ _lib.gdn_backward_timed.argtypes = [_vp, ctypes.POINTER(Inputs), _vp, ctypes.POI
 _lib.gdn_backward_timed.restype = ctypes.c_int
 _lib.gdn_backward_workspace_bytes.argtypes = [_vp]
 _lib.gdn_backward_workspace_bytes.restype = ctypes.c_size_t
+_lib.gdn_backward_workspace_offsets.argtypes = [_vp, ctypes.POINTER(ctypes.c_size_t), ctypes.c_int]
+_lib.gdn_backward_workspace_offsets.restype = ctypes.c_int
 _lib.gdn_backward_launches.argtypes = [_vp]
 _lib.gdn_backward_launches.restype = ctypes.c_int
 _lib.gdn_forward_timed.argtypes = [_vp, ctypes.POINTER(Inputs), _vp, _vp, _vp, ctypes.POINTER(_vp), ctypes.c_int]
@@ -239,6 +241,16 @@ class Plan:
         n = _lib.gdn_workspace_offsets(self._h, arr, len(self.WS_FIELDS))
         return {self.WS_FIELDS[i]: arr[i] for i in range(n)}
 
+    BWD_WS_FIELDS = ("T", "S0", "o", "dO", "dSloc", "dSend", "dSb", "dqh", "dkh", "dvh", "dla", "dbeta",
+                     "dnw_part", "dconv_part", "dA_part")
+
+    def backward_workspace_offsets(self) -> dict:
+        """Offsets of the tensor-core backward's buffers in the gdn_backward workspace (empty for
+        plans without that backward)."""
+        arr = (ctypes.c_size_t * len(self.BWD_WS_FIELDS))()
+        n = _lib.gdn_backward_workspace_offsets(self._h, arr, len(self.BWD_WS_FIELDS))
+        return {self.BWD_WS_FIELDS[i]: arr[i] for i in range(n)}
+
     def device_status(self, workspace: int, stream: int) -> int:
         return _lib.gdn_get_device_status(self._h, workspace, stream)
 
@@ -354,6 +366,16 @@ class BlockPlan:
         arr = (_vp * len(events))(*events)
         _check(_lib.gdn_block_forward_timed(self._h, ctypes.byref(ins), out, workspace, stream, arr, len(events)),
                "gdn_block_forward_timed")
+
+    BWD_WS_FIELDS = ("T", "S0", "o", "dO", "dSloc", "dSend", "dSb", "dqh", "dkh", "dvh", "dla", "dbeta",
+                     "dnw_part", "dconv_part", "dA_part")
+
+    def backward_workspace_offsets(self) -> dict:
+        """Offsets of the tensor-core backward's buffers in the gdn_backward workspace (empty for
+        plans without that backward)."""
+        arr = (ctypes.c_size_t * len(self.BWD_WS_FIELDS))()
+        n = _lib.gdn_backward_workspace_offsets(self._h, arr, len(self.BWD_WS_FIELDS))
+        return {self.BWD_WS_FIELDS[i]: arr[i] for i in range(n)}
 
     def device_status(self, workspace: int, stream: int) -> int:
         return _lib.gdn_block_device_status(self._h, workspace, stream)

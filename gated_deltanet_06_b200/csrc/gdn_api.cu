@@ -28,6 +28,12 @@ struct gdn_plan_s {
     // backward workspace layout (gdn_backward)
     size_t b_status, b_qh, b_kh, b_vh, b_G, b_beta, b_la, b_o, b_ckpt, b_dO, b_dvh, b_dqp, b_dkp, b_dap, b_dbp,
         b_dnw, b_dconv, b_dA, b_ddt, bws_bytes;
+    // the tensor-core backward (tensor plans but fused ones): the forward's layout first, then the
+    // kept T and block start states, dO (fp16), the segment-end gradients and dS^T at block ends;
+    // b_o, b_dqp / b_dkp / b_dvh (whole dq^ dk^ dv^), b_dap / b_dbp (d log alpha, dbeta) and the
+    // partial sums reuse the names above
+    bool tc_bwd;
+    size_t t_T, t_S0, t_dO16, t_dSloc, t_dSend, t_dSb;
     // staging layout (gdn_forward_host)
     size_t st_q, st_k, st_v, st_z, st_g, st_b, st_cq, st_ck, st_cv, st_A, st_dt, st_nw, st_y, staging_bytes;
 };
@@ -98,7 +104,7 @@ size_t gdn::plan_workspace_bytes(const gdn_plan_s *plan) { return plan ? plan->w
 int gdn::run_tensor_core(const gdn_plan_s *plan, const float *g, const float *b, const float *A_log,
                          const float *dt_bias, const float *norm_w, const void *z, InType z_type, long long z_stride,
                          void *y, void *workspace, cudaStream_t s, bool pdl_first, void *const *events, int *ev,
-                         const float *s0, float *s_end) {
+                         const float *s0, float *s_end, const FwdSave *save) {
     const gdn_config &c = plan->cfg;
     const int d = c.d_k;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -120,6 +126,8 @@ int gdn::run_tensor_core(const gdn_plan_s *plan, const float *g, const float *b,
             !make_tile_map(&tmKt, ws + plan->off_Kt, rows) || !make_tile_map(&tmAqk, ws + plan->off_Aqk, rows) ||
             !make_tile_map(&tmAqkH, ws + plan->off_Aqk, rows, 64))  // Aqk's lower-right quadrant
             return GDN_ERR_CUDA;
+        CUtensorMap tmT = tmQt;  // read only when T is kept
+        if (save && !make_tile_map(&tmT, save->T, rows)) return GDN_ERR_CUDA;
         ChunkParams cp;
         cp.g = g; cp.bg = b; cp.A_log = A_log; cp.dt_bias = dt_bias;
         cp.G = G; cp.beta = beta; cp.log_alpha = la;
@@ -134,10 +142,12 @@ int gdn::run_tensor_core(const gdn_plan_s *plan, const float *g, const float *b,
         cp.wait_limit_ns = kWaitLimitNs;
         cp.rev = rev;
         cp.debug = (c.flags & GDN_FLAG_DEBUG_CHECKS) ? 1 : 0;
+        cp.save = save ? 1 : 0;
         // The kernels start with programmatic dependent launch (prologue overlapped with the previous
         // kernel's tail), except when per-kernel events are recorded between them.
         const bool pdl = events == nullptr;
-        if (!mark() || launch_chunk(cp, tmK, tmV, tmQ, tmW, tmU, tmQt, tmAqk, tmAqkH, s, pdl && pdl_first) != cudaSuccess)
+        if (!mark() ||
+            launch_chunk(cp, tmK, tmV, tmQ, tmW, tmU, tmQt, tmAqk, tmAqkH, tmT, s, pdl && pdl_first) != cudaSuccess)
             return GDN_ERR_CUDA;
         ScanParams sp;
         sp.G = G;
@@ -154,6 +164,16 @@ int gdn::run_tensor_core(const gdn_plan_s *plan, const float *g, const float *b,
         sp.s_end = s_end;
         sp.rev = rev;
         sp.debug = (c.flags & GDN_FLAG_DEBUG_CHECKS) ? 1 : 0;
+        sp.raw_o = 0;
+        sp.S0b = nullptr;
+        sp.Lb = nullptr;
+        sp.Sb = nullptr;
+        if (save) {  // o itself (fp32) and the block start states, for the backward
+            sp.raw_o = 1;
+            sp.y = save->o;
+            sp.out_kind = 1;
+            sp.S0b = save->S0b;
+        }
         if (plan->NS > 1) {
             if (!mark() || launch_transfer(sp, tmW, tmKt, tmU, s, pdl) != cudaSuccess) return GDN_ERR_CUDA;
             if (!mark() || launch_combine(sp, s, pdl) != cudaSuccess) return GDN_ERR_CUDA;
@@ -302,6 +322,32 @@ gdn_status gdn_plan(const gdn_config *cfg, gdn_plan_t *out, size_t *workspace_by
         p->b_ddt = o2; o2 = align_up(o2 + static_cast<size_t>(BH) * ntile * 4, A);
         p->bws_bytes = o2;
     }
+    p->tc_bwd = p->tensor && !p->fused;
+    if (p->tc_bwd) {  // the tensor-core backward's layout (replaces the one above)
+        const size_t act2 = nTok * 128 * 2, act4 = nTok * 128 * 4, tok4 = nTok * 4;
+        const size_t seg4 = static_cast<size_t>(BH) * p->NS * 128 * 128 * 4;
+        const size_t ntile = static_cast<size_t>(Tp) / 64;
+        const size_t nout = static_cast<size_t>(bwd_out_blocks(static_cast<long long>(c.B) * c.T * c.H));
+        size_t o2 = p->ws_bytes;  // the forward's buffers at their usual offsets (status at 0)
+        p->b_status = p->off_status;
+        p->t_T = o2; o2 = align_up(o2 + act2, A);
+        p->t_S0 = o2; o2 = align_up(o2 + act2, A);
+        p->b_o = o2; o2 = align_up(o2 + static_cast<size_t>(c.B) * c.T * c.H * 128 * 4, A);
+        p->t_dO16 = o2; o2 = align_up(o2 + act2, A);
+        p->t_dSloc = o2; o2 = align_up(o2 + seg4, A);
+        p->t_dSend = o2; o2 = align_up(o2 + seg4, A);
+        p->t_dSb = o2; o2 = align_up(o2 + act2, A);
+        p->b_dqp = o2; o2 = align_up(o2 + act4, A);
+        p->b_dkp = o2; o2 = align_up(o2 + act4, A);
+        p->b_dvh = o2; o2 = align_up(o2 + act4, A);
+        p->b_dap = o2; o2 = align_up(o2 + tok4, A);
+        p->b_dbp = o2; o2 = align_up(o2 + tok4, A);
+        p->b_dnw = o2; o2 = align_up(o2 + nout * 128 * 4, A);
+        p->b_dconv = o2; o2 = align_up(o2 + static_cast<size_t>(c.B) * ntile * 3 * c.H * 128 * 4 * 4, A);
+        p->b_dA = o2; o2 = align_up(o2 + static_cast<size_t>(BH) * ntile * 4, A);
+        p->b_ddt = o2; o2 = align_up(o2 + static_cast<size_t>(BH) * ntile * 4, A);
+        p->bws_bytes = o2;
+    }
 
     const size_t ntok_in = static_cast<size_t>(c.B) * c.T;
     const size_t a_in = ntok_in * c.H * d * p->in_esize;
@@ -351,6 +397,16 @@ int gdn_workspace_offsets(gdn_plan_t plan, size_t *offsets, int n) {
                             plan->off_Kt, plan->off_Aqk, plan->off_o, plan->off_Zloc, plan->off_Sstart,
                             plan->off_SP, plan->off_SS};
     const int m = n < 17 ? n : 17;
+    for (int i = 0; i < m; ++i) offsets[i] = all[i];
+    return m;
+}
+
+int gdn_backward_workspace_offsets(gdn_plan_t plan, size_t *offsets, int n) {
+    if (!plan || !offsets || n <= 0 || !plan->tc_bwd) return 0;
+    const size_t all[15] = {plan->t_T,    plan->t_S0,   plan->b_o,   plan->t_dO16, plan->t_dSloc,
+                            plan->t_dSend, plan->t_dSb, plan->b_dqp, plan->b_dkp,  plan->b_dvh,
+                            plan->b_dap,  plan->b_dbp,  plan->b_dnw, plan->b_dconv, plan->b_dA};
+    const int m = n < 15 ? n : 15;
     for (int i = 0; i < m; ++i) offsets[i] = all[i];
     return m;
 }
@@ -564,7 +620,147 @@ gdn_status gdn_forward_host(gdn_plan_t plan, const gdn_inputs *in_host, void *y_
 
 size_t gdn_backward_workspace_bytes(gdn_plan_t plan) { return plan ? plan->bws_bytes : 0; }
 
-int gdn_backward_launches(gdn_plan_t plan) { return plan ? 6 : 0; }  // prep + the five backward kernels
+int gdn_backward_launches(gdn_plan_t plan) {
+    if (!plan) return 0;
+    // tensor-core backward: prep, the forward with its intermediates kept (UT, [transfer, combine,]
+    // output pass), the output step backwards, [the backward transfer and combine,] the final
+    // backward pass, the block gradients, the per-token and parameter steps
+    if (plan->tc_bwd) return plan->NS > 1 ? 12 : 8;
+    return 6;  // prep + the five fp32 backward kernels
+}
+
+// The tensor-core backward: the forward with its intermediates kept, the output step backwards,
+// the reverse scan of the state gradient over segments, every block's local gradients, then the
+// per-token (L2 norm, SiLU, conv, gates) and parameter steps.
+static gdn_status backward_tc(gdn_plan_t plan, const gdn_inputs *in, const void *dy, const gdn_grads *gr, uint8_t *ws,
+                              cudaStream_t s, void *const *events) {
+    const gdn_config &c = plan->cfg;
+    const int d = c.d_k;
+    int *status = reinterpret_cast<int *>(ws + plan->off_status);
+    auto F = [&](size_t off) { return reinterpret_cast<float *>(ws + off); };
+    auto H16 = [&](size_t off) { return reinterpret_cast<__half *>(ws + off); };
+    int ev = 0;
+    auto mark = [&]() -> bool {
+        if (!events) return true;
+        return cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[ev++]), s) == cudaSuccess;
+    };
+    const float q_scale = 1.0f / sqrtf(static_cast<float>(d));
+    const unsigned long long rows = static_cast<unsigned long long>(c.B) * c.H * plan->Tp;
+    const int BH = c.B * c.H;
+
+    // ---- forward (prep, UT transform, segment scan), keeping T, the block start states and o
+    PrepParams pp;
+    memset(&pp, 0, sizeof(pp));
+    pp.q = in->q; pp.k = in->k; pp.v = in->v;
+    pp.tok_stride = plan->tok_stride;
+    pp.g = in->g; pp.b = in->b;
+    pp.conv_q = in->conv_q; pp.conv_k = in->conv_k; pp.conv_v = in->conv_v;
+    pp.A_log = in->A_log; pp.dt_bias = in->dt_bias;
+    pp.qh = ws + plan->off_qh; pp.kh = ws + plan->off_kh; pp.vh = ws + plan->off_vh;
+    pp.G = F(plan->off_G); pp.beta = F(plan->off_beta); pp.log_alpha = F(plan->off_la);
+    pp.B = c.B; pp.T = c.T; pp.H = c.H; pp.d = d; pp.Tp = plan->Tp;
+    pp.l2_eps = c.l2_eps;
+    pp.q_scale = q_scale;
+    pp.status = status;
+    pp.wait_limit_ns = kWaitLimitNs;
+    {
+        CUtensorMap rq, rk, rv;
+        if (!make_raw_map(&rq, in->q, c.B, c.T, c.H * d, plan->tok_stride, 64 + 3, 128) ||
+            !make_raw_map(&rk, in->k, c.B, c.T, c.H * d, plan->tok_stride, 64 + 3, 128) ||
+            !make_raw_map(&rv, in->v, c.B, c.T, c.H * d, plan->tok_stride, 64 + 3, 128))
+            return GDN_ERR_CUDA;
+        if (!mark() || launch_prep_tma(pp, in_type(c.in_dtype), rq, rk, rv, s) != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    FwdSave save;
+    save.T = H16(plan->t_T);
+    save.S0b = H16(plan->t_S0);
+    save.o = F(plan->b_o);
+    const int st = run_tensor_core(plan, in->g, in->b, in->A_log, in->dt_bias, in->norm_w, in->z, in_type(c.in_dtype),
+                                   plan->tok_stride, nullptr, ws, s, true, events, &ev, nullptr, nullptr, &save);
+    if (st != GDN_OK) return static_cast<gdn_status>(st);
+
+    // ---- the output step backwards: dO (fp16, zero on padding rows), dz, norm-weight partials
+    BwdParams bp;
+    memset(&bp, 0, sizeof(bp));
+    bp.q = in->q; bp.k = in->k; bp.v = in->v; bp.z = in->z; bp.dy = dy;
+    bp.tok_stride = plan->tok_stride;
+    bp.g = in->g; bp.bg = in->b; bp.conv_q = in->conv_q; bp.conv_k = in->conv_k; bp.conv_v = in->conv_v;
+    bp.A_log = in->A_log; bp.dt_bias = in->dt_bias; bp.norm_w = in->norm_w;
+    bp.log_alpha = F(plan->off_la);
+    bp.o = F(plan->b_o);
+    bp.dO16 = H16(plan->t_dO16);
+    bp.dvh = F(plan->b_dvh);
+    bp.dq_part = F(plan->b_dqp); bp.dk_part = F(plan->b_dkp); bp.da_part = F(plan->b_dap); bp.db_part = F(plan->b_dbp);
+    bp.dnw_part = F(plan->b_dnw); bp.dconv_part = F(plan->b_dconv); bp.dA_part = F(plan->b_dA);
+    bp.ddt_part = F(plan->b_ddt);
+    bp.dq = gr->dq; bp.dk = gr->dk; bp.dv = gr->dv; bp.dz = gr->dz; bp.dg = gr->dg; bp.db = gr->db;
+    bp.dconv_q = gr->dconv_q; bp.dconv_k = gr->dconv_k; bp.dconv_v = gr->dconv_v;
+    bp.dA_log = gr->dA_log; bp.ddt_bias = gr->ddt_bias; bp.dnorm_w = gr->dnorm_w;
+    bp.B = c.B; bp.T = c.T; bp.H = c.H; bp.d = d; bp.Tp = plan->Tp;
+    bp.l2_eps = c.l2_eps; bp.norm_eps = c.norm_eps; bp.q_scale = q_scale;
+    bp.groups = 1;
+    bp.tc = 1;
+    if (plan->Tp > c.T &&
+        cudaMemset2DAsync(bp.dO16 + static_cast<size_t>(c.T) * 128, static_cast<size_t>(plan->Tp) * 256, 0,
+                          static_cast<size_t>(plan->Tp - c.T) * 256, BH, s) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (!mark() || launch_bwd_out(bp, in_type(c.in_dtype), in_type(c.out_dtype), s) != cudaSuccess) return GDN_ERR_CUDA;
+
+    // ---- reverse scan of dS: transfer pass, combine, final pass (dS^T at every block end)
+    CUtensorMap tmAqk, tmDO, tmKt, tmQt, tmW;
+    if (!make_tile_map(&tmAqk, ws + plan->off_Aqk, rows) || !make_tile_map(&tmDO, bp.dO16, rows) ||
+        !make_tile_map(&tmKt, ws + plan->off_Kt, rows) || !make_tile_map(&tmQt, ws + plan->off_Qt, rows) ||
+        !make_tile_map(&tmW, ws + plan->off_W, rows))
+        return GDN_ERR_CUDA;
+    BwdTcParams tp;
+    memset(&tp, 0, sizeof(tp));
+    tp.G = F(plan->off_G); tp.beta = F(plan->off_beta);
+    tp.Q = H16(plan->off_qh); tp.K = H16(plan->off_kh); tp.V = H16(plan->off_vh);
+    tp.W = H16(plan->off_W); tp.U = H16(plan->off_U); tp.Kt = H16(plan->off_Kt); tp.Aqk = H16(plan->off_Aqk);
+    tp.S0b = save.S0b;
+    tp.dSb = H16(plan->t_dSb);
+    tp.dSloc = F(plan->t_dSloc);
+    tp.dSend = F(plan->t_dSend);
+    tp.dqh = bp.dq_part; tp.dkh = bp.dk_part; tp.dvh = bp.dvh;
+    tp.dla = bp.da_part; tp.dbeta = bp.db_part;
+    tp.BH = BH; tp.Tp = plan->Tp; tp.NB = plan->NB; tp.NS = plan->NS; tp.Ls = plan->Ls;
+    tp.q_scale = q_scale;
+    tp.status = status;
+    tp.wait_limit_ns = kWaitLimitNs;
+    const bool pdl = events == nullptr;
+    if (plan->NS > 1) {
+        if (!mark() || launch_bwd_scan(tp, false, tmAqk, tmDO, tmKt, tmQt, tmW, s, pdl) != cudaSuccess)
+            return GDN_ERR_CUDA;
+        ScanParams sp;
+        memset(&sp, 0, sizeof(sp));
+        sp.Zloc = F(plan->off_Zloc);
+        sp.Lb = tp.dSloc;
+        sp.Sb = F(plan->t_dSend);
+        sp.B = c.B; sp.T = c.T; sp.H = c.H; sp.Tp = plan->Tp; sp.NB = plan->NB; sp.NS = plan->NS; sp.Ls = plan->Ls;
+        sp.status = status;
+        sp.wait_limit_ns = kWaitLimitNs;
+        if (!mark() || launch_combine_bwd(sp, s, pdl) != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    if (!mark() || launch_bwd_scan(tp, true, tmAqk, tmDO, tmKt, tmQt, tmW, s, pdl && plan->NS > 1) != cudaSuccess)
+        return GDN_ERR_CUDA;
+
+    // ---- every block's local gradients
+    BwdTcMaps mp;
+    if (!make_tile_map(&mp.S0, save.S0b, rows) || !make_tile_map(&mp.W, ws + plan->off_W, rows) ||
+        !make_tile_map(&mp.dO, bp.dO16, rows) || !make_tile_map(&mp.Aqk, ws + plan->off_Aqk, rows) ||
+        !make_tile_map(&mp.Kt, ws + plan->off_Kt, rows) || !make_tile_map(&mp.dS, tp.dSb, rows) ||
+        !make_tile_map(&mp.K, ws + plan->off_kh, rows) || !make_tile_map(&mp.Q, ws + plan->off_qh, rows) ||
+        !make_tile_map(&mp.T, save.T, rows) || !make_tile_map(&mp.U, ws + plan->off_U, rows) ||
+        !make_tile_map(&mp.V, ws + plan->off_vh, rows))
+        return GDN_ERR_CUDA;
+    if (!mark() || launch_bwd_grad(tp, mp, s, pdl) != cudaSuccess) return GDN_ERR_CUDA;
+
+    // ---- per token (L2 norm, SiLU and conv backwards, gates) and the parameter sums
+    if (!mark() || launch_bwd_tokens(bp, in_type(c.in_dtype), s) != cudaSuccess) return GDN_ERR_CUDA;
+    if (!mark() || launch_bwd_params(bp, s) != cudaSuccess) return GDN_ERR_CUDA;
+    if (!mark()) return GDN_ERR_CUDA;
+    return GDN_OK;
+}
 
 static gdn_status backward_impl(gdn_plan_t plan, const gdn_inputs *in, const void *dy, const gdn_grads *gr,
                                 void *workspace, gdn_stream_t stream, void *const *events) {
@@ -591,6 +787,7 @@ static gdn_status backward_impl(gdn_plan_t plan, const gdn_inputs *in, const voi
     int *status = reinterpret_cast<int *>(ws + plan->b_status);
     if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return GDN_ERR_CUDA;
     auto F = [&](size_t off) { return reinterpret_cast<float *>(ws + off); };
+    if (plan->tc_bwd) return backward_tc(plan, in, dy, gr, ws, s, events);
 
     PrepParams pp;
     memset(&pp, 0, sizeof(pp));
@@ -611,6 +808,8 @@ static gdn_status backward_impl(gdn_plan_t plan, const gdn_inputs *in, const voi
     if (launch_prep(pp, in_type(c.in_dtype), false, s) != cudaSuccess) return GDN_ERR_CUDA;
 
     BwdParams bp;
+    memset(&bp, 0, sizeof(bp));
+    bp.groups = d / 8;
     bp.q = in->q; bp.k = in->k; bp.v = in->v; bp.z = in->z; bp.dy = dy;
     bp.tok_stride = plan->tok_stride;
     bp.g = in->g; bp.bg = in->b; bp.conv_q = in->conv_q; bp.conv_k = in->conv_k; bp.conv_v = in->conv_v;

@@ -21,7 +21,11 @@
 //   of C tokens, last to first: states recomputed from the checkpoint into
 //   shared memory, the gradient run backwards, the row sums taken from shared
 //   memory) -> gdn_bwd_tokens (group sums, L2-norm, SiLU and conv backwards,
-//   gates) -> gdn_bwd_params (sums over tokens of the parameter gradients).
+//   gates) -> gdn_bwd_params_split (sums over tokens of the parameter gradients).
+// The output-step, per-token and parameter kernels also serve the tensor-core
+// backward (gdn_bwd_tc.cu), which hands them dO in fp16, whole per-token
+// gradients of q^ k^ v^ and d log alpha; its per-token step is
+// gdn_bwd_tokens_rows (one warp per token row).
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 
@@ -141,7 +145,7 @@ __global__ void __launch_bounds__(kBT) gdn_bwd_fwd_rows(const BwdParams p) {
 // One warp per (b, t, h) row.  y = o rn w SiLU(z), rn = 1/sqrt(mean(o^2) + eps):
 //   gz = dy w SiLU(z);  do = rn gz - o rn^3 (o . gz) / D;  dz = dy o rn w SiLU'(z);
 //   dw += dy o rn SiLU(z)  (per-CTA partial sums, in a fixed order).
-template <typename ZT, typename YT, int D>
+template <typename ZT, typename YT, int D, bool kF16>
 __global__ void __launch_bounds__(256) gdn_bwd_out(const BwdParams p) {
     constexpr int PER = D / 32;
     __shared__ float sw[8][D];
@@ -186,7 +190,8 @@ __global__ void __launch_bounds__(256) gdn_bwd_out(const BwdParams p) {
         for (int e = 0; e < PER; ++e) {
             const int c = lane * PER + e;
             const float gz = gv[e] * w[e] * sz[e];
-            p.dO[(bhr * p.Tp + t) * D + c] = rn * gz - ov[e] * k3;
+            if constexpr (kF16) p.dO16[(bhr * p.Tp + t) * D + c] = __float2half_rn(rn * gz - ov[e] * k3);
+            else p.dO[(bhr * p.Tp + t) * D + c] = rn * gz - ov[e] * k3;
             p.dz[row * D + c] = gv[e] * ov[e] * rn * w[e] * dsilu(zv[e]);
             dw[e] = fmaf(gv[e] * ov[e] * rn, sz[e], dw[e]);
         }
@@ -357,7 +362,7 @@ __global__ void __launch_bounds__(256) gdn_bwd_tokens(const BwdParams p) {
     const size_t BH = static_cast<size_t>(p.B) * p.H;
     const int t0 = tile * kTile;
     const int tid = threadIdx.x, cg = tid % CPR, rg = tid / CPR, c0 = cg * 8;
-    const int G = D / kR;
+    const int G = p.groups;
     const int ntile = p.Tp / kTile;
 
     for (int which = 0; which < 3; ++which) {
@@ -485,7 +490,7 @@ __global__ void __launch_bounds__(256) gdn_bwd_tokens(const BwdParams p) {
             const float xg = p.g[gi] + p.dt_bias[h];
             const float eA = expf(p.A_log[h]);
             const float la = -eA * softplus_f(xg);
-            const float dla = da * expf(la);
+            const float dla = p.tc ? da : da * expf(la);  // d log alpha (given, or from d alpha)
             dgv = dla * (-eA * sigm(xg));
             dla_la = dla * la;
             const float be = sigm(p.bg[gi]);
@@ -510,38 +515,260 @@ __global__ void __launch_bounds__(256) gdn_bwd_tokens(const BwdParams p) {
     }
 }
 
+// ------------------------------------------------------------ per-token backwards, one warp per row
+// The tensor-core backward's per-token step (d = 128, whole dq^ / dk^ / dv^ and d log alpha).  One
+// CTA per (64-token tile, h, b), 8 warps, lane l on channels 4l .. 4l+3 of a token row.  For q, k, v
+// in turn: pass 1 takes the tile's tokens and the 3 after it, one token per warp at a time (the rows
+// are independent): the conv of the 4 input rows, SiLU, the L2-norm sums as warp reductions, and
+// da = dL/d(conv output) into shared memory; pass 2 takes the tile's tokens again for
+// dx[t] = sum_k w_k da[t+3-k] and the conv-weight sums (input rows re-read, from L1), reduced over
+// the warps in a fixed order into the tile's partial slot.  Then the gates of the tile's tokens.
+template <typename InT>
+__device__ __forceinline__ void ld4_in(const InT *src, float (&v)[4]);
+template <>
+__device__ __forceinline__ void ld4_in<float>(const float *src, float (&v)[4]) {
+    const float4 x = *reinterpret_cast<const float4 *>(src);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+}
+template <>
+__device__ __forceinline__ void ld4_in<__nv_bfloat16>(const __nv_bfloat16 *src, float (&v)[4]) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(src);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+}
+template <>
+__device__ __forceinline__ void ld4_in<__half>(const __half *src, float (&v)[4]) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(src);
+    const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&u.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&u.y));
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+}
+
+template <typename InT>
+__global__ void __launch_bounds__(256) gdn_bwd_tokens_rows(const BwdParams p) {
+    constexpr int D = 128, NR = kTile + 3;
+    __shared__ float4 sda[NR][32];    // da of token t0 + tt, channels 4 lane .. 4 lane + 3
+    __shared__ float4 swt[4][32];     // conv taps of channel 4 lane + j
+    __shared__ float sg[8][2];
+    // per-warp conv-weight sums of channel 4 lane + j, over sda once pass 2 has read it
+    float4 (*sdw)[4][32] = reinterpret_cast<float4 (*)[4][32]>(&sda[0][0]);
+    static_assert(sizeof(sda) >= 8 * 4 * 32 * sizeof(float4), "the warp sums fit in sda");
+    const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const size_t bh = static_cast<size_t>(b) * p.H + h;
+    const int t0 = tile * kTile;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, c0 = lane * 4;
+    const int ntile = p.Tp / kTile;
+    for (int which = 0; which < 3; ++which) {
+        const InT *x = static_cast<const InT *>(which == 0 ? p.q : (which == 1 ? p.k : p.v));
+        const float *wc = which == 0 ? p.conv_q : (which == 1 ? p.conv_k : p.conv_v);
+        const float *dh_src = which == 0 ? p.dq_part : (which == 1 ? p.dk_part : p.dvh);
+        float *dx = which == 0 ? p.dq : (which == 1 ? p.dk : p.dv);
+        const float sc = which == 0 ? p.q_scale : 1.0f;
+        auto xrow = [&](int t, float (&v)[4]) {
+            if (t >= 0 && t < p.T) {
+                ld4_in<InT>(x + (static_cast<size_t>(b) * p.T + t) * p.tok_stride + static_cast<size_t>(h) * D + c0, v);
+            } else {
+                v[0] = v[1] = v[2] = v[3] = 0.0f;
+            }
+        };
+        __syncthreads();  // the previous tensor's reads of swt and of sda (and the warp sums over it) are done
+        if (warp < 4) swt[warp][lane] = reinterpret_cast<const float4 *>(wc)[static_cast<size_t>(h) * D + c0 + warp];
+        __syncthreads();
+        float w[4][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float4 t4 = swt[j][lane];
+            w[j][0] = t4.x; w[j][1] = t4.y; w[j][2] = t4.z; w[j][3] = t4.w;
+        }
+        // pass 1: da of tokens t0 .. t0 + 66 (zero past T).  Warp w takes tokens 8w .. 8w+7 (warp 7 also
+        // the 3 after the tile) in runs of 4: the 7 input rows and 4 gradient rows of a run are all
+        // fetched before any is used, and the 4 tokens' reductions are independent.
+        for (int rb = 8 * warp; rb < (warp == 7 ? NR : 8 * warp + 8); rb += 4) {
+            float xr[7][4], dh[4][4];
+#pragma unroll
+            for (int k = 0; k < 7; ++k) xrow(t0 + rb - 3 + k, xr[k]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int t = t0 + rb + i;
+                if (t < p.T && rb + i < NR) {
+                    ld4_in<float>(dh_src + (bh * p.Tp + t) * D + c0, dh[i]);
+                } else {
+                    dh[i][0] = dh[i][1] = dh[i][2] = dh[i][3] = 0.0f;
+                }
+            }
+            // sigma(a) once per element (fast exponential and division); SiLU' = sigma (1 + a (1 - sigma))
+            float a[4][4], sg[4][4], sv[4][4], ss[4], pr[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                ss[i] = 0.0f;
+                pr[i] = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    a[i][j] = w[j][0] * xr[i][j] + w[j][1] * xr[i + 1][j] + w[j][2] * xr[i + 2][j] + w[j][3] * xr[i + 3][j];
+                    sg[i][j] = __fdividef(1.0f, 1.0f + __expf(-a[i][j]));
+                    sv[i][j] = a[i][j] * sg[i][j];
+                    ss[i] = fmaf(sv[i][j], sv[i][j], ss[i]);
+                    pr[i] = fmaf(sv[i][j], dh[i][j], pr[i]);
+                }
+            }
+            if (which < 2) {
+                // with u = s / n, n = sqrt(|s|^2 + eps): d s = sc (dh - u (u . dh)) / n
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        ss[i] += __shfl_xor_sync(0xffffffffu, ss[i], off);
+                        pr[i] += __shfl_xor_sync(0xffffffffu, pr[i], off);
+                    }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float inv = rsqrtf(ss[i] + p.l2_eps);
+                    const float k2 = inv * inv * pr[i];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) dh[i][j] = sc * inv * (dh[i][j] - sv[i][j] * k2);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int t = t0 + rb + i;
+                if (rb + i < NR) {
+                    float da[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        da[j] = t < p.T ? dh[i][j] * sg[i][j] * (1.0f + a[i][j] * (1.0f - sg[i][j])) : 0.0f;
+                    sda[rb + i][lane] = make_float4(da[0], da[1], da[2], da[3]);
+                }
+            }
+        }
+        __syncthreads();
+        // pass 2: dx[t] = sum_k w_k da[t + 3 - k] and the conv-weight sums (tap k multiplies x[t - 3 + k])
+        float dw[4][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) dw[j][k] = 0.0f;
+        for (int tt = warp; tt < kTile; tt += 8) {
+            const int t = t0 + tt;
+            if (t >= p.T) break;
+            float dr[4][4], xr[4][4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float4 v = sda[tt + k][lane];
+                dr[k][0] = v.x; dr[k][1] = v.y; dr[k][2] = v.z; dr[k][3] = v.w;
+                xrow(t - 3 + k, xr[k]);
+            }
+            float o[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                o[j] = w[j][0] * dr[3][j] + w[j][1] * dr[2][j] + w[j][2] * dr[1][j] + w[j][3] * dr[0][j];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) dw[j][k] = fmaf(dr[0][j], xr[k][j], dw[j][k]);
+            }
+            *reinterpret_cast<float4 *>(dx + (static_cast<size_t>(b) * p.T + t) * p.H * D + static_cast<size_t>(h) * D + c0) =
+                make_float4(o[0], o[1], o[2], o[3]);
+        }
+        __syncthreads();  // every read of sda is done
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sdw[warp][j][lane] = make_float4(dw[j][0], dw[j][1], dw[j][2], dw[j][3]);
+        __syncthreads();
+        if (warp < 4) {  // warp j: channel 4 lane + j, the 8 warps' sums in order
+            float4 acc = sdw[0][warp][lane];
+#pragma unroll
+            for (int k = 1; k < 8; ++k) {
+                const float4 v = sdw[k][warp][lane];
+                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+            }
+            float *out = p.dconv_part + ((static_cast<size_t>(b) * ntile + tile) * 3 + which) * static_cast<size_t>(p.H) * D * 4 +
+                         (static_cast<size_t>(h) * D + c0 + warp) * 4;
+            *reinterpret_cast<float4 *>(out) = acc;
+        }
+    }
+
+    // gates: log alpha = -exp(A_log) softplus(g + dt_bias), beta = sigmoid(b); d log alpha is given
+    float dla_la = 0.0f, dgv = 0.0f;
+    if (threadIdx.x < kTile) {
+        const int t = t0 + threadIdx.x;
+        if (t < p.T) {
+            const float eA = expf(p.A_log[h]);
+            const float dla = p.da_part[bh * p.Tp + t];
+            const float db = p.db_part[bh * p.Tp + t];
+            const size_t gi = (static_cast<size_t>(b) * p.T + t) * p.H + h;
+            const float xg = p.g[gi] + p.dt_bias[h];
+            const float la = -eA * softplus_f(xg);
+            const float dg = dla * (-eA * sigm(xg));
+            dgv = dg;
+            dla_la = dla * la;
+            const float be = sigm(p.bg[gi]);
+            p.dg[gi] = dg;
+            p.db[gi] = db * be * (1.0f - be);
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        dla_la += __shfl_xor_sync(0xffffffffu, dla_la, off);
+        dgv += __shfl_xor_sync(0xffffffffu, dgv, off);
+    }
+    if (lane == 0) {
+        sg[warp][0] = dla_la;
+        sg[warp][1] = dgv;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const size_t k = bh * ntile + tile;
+        p.dA_part[k] = sg[0][0] + sg[1][0];
+        p.ddt_part[k] = sg[0][1] + sg[1][1];
+    }
+}
+
 // ------------------------------------------------------------ parameter sums
-// One thread per parameter gradient element, summing its partials in a fixed order.
-__global__ void __launch_bounds__(256) gdn_bwd_params(const BwdParams p, int D, int nout_part) {
+// 32 parameter gradient elements per CTA, 8 warps: warp g sums partials g, g + 8, ... of lane l's
+// element, then the 8 warp sums are added in order (a fixed order throughout).
+__global__ void __launch_bounds__(256) gdn_bwd_params_split(const BwdParams p, int D, int nout_part) {
+    __shared__ float red[8][32];
     const int HD4 = p.H * D * 4;
     const int ntile = p.Tp / kTile;
     const int total = 3 * HD4 + 2 * p.H + D;
-    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
+    const int lane = threadIdx.x & 31, g = threadIdx.x >> 5;
+    const int e = blockIdx.x * 32 + lane;
+    float sum = 0.0f;
+    if (e < 3 * HD4) {
+        const int which = e / HD4, k = e % HD4;
+        for (int bt = g; bt < p.B * ntile; bt += 8) sum += p.dconv_part[(static_cast<size_t>(bt) * 3 + which) * HD4 + k];
+    } else if (e < 3 * HD4 + 2 * p.H) {
+        const int k = e - 3 * HD4, h = k % p.H;
+        const float *part = k < p.H ? p.dA_part : p.ddt_part;
+        for (int i = g; i < p.B * ntile; i += 8) {
+            const int b = i / ntile, t = i % ntile;
+            sum += part[(static_cast<size_t>(b) * p.H + h) * ntile + t];
+        }
+    } else if (e < total) {
+        const int c = e - 3 * HD4 - 2 * p.H;
+        for (int q = g; q < nout_part; q += 8) sum += p.dnw_part[static_cast<size_t>(q) * D + c];
+    }
+    red[g][lane] = sum;
+    __syncthreads();
+    if (g == 0 && e < total) {
+        float s = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) s += red[k][lane];
         if (e < 3 * HD4) {
             const int which = e / HD4, k = e % HD4;
-            float s = 0.0f;
-            for (int bt = 0; bt < p.B * ntile; ++bt) s += p.dconv_part[(static_cast<size_t>(bt) * 3 + which) * HD4 + k];
             (which == 0 ? p.dconv_q : (which == 1 ? p.dconv_k : p.dconv_v))[k] = s;
         } else if (e < 3 * HD4 + 2 * p.H) {
-            const int k = e - 3 * HD4, h = k % p.H;
-            const float *part = k < p.H ? p.dA_part : p.ddt_part;
-            float s = 0.0f;
-            for (int b = 0; b < p.B; ++b)
-                for (int t = 0; t < ntile; ++t) s += part[(static_cast<size_t>(b) * p.H + h) * ntile + t];
-            (k < p.H ? p.dA_log : p.ddt_bias)[h] = s;
+            const int k = e - 3 * HD4;
+            (k < p.H ? p.dA_log : p.ddt_bias)[k % p.H] = s;
         } else {
-            const int c = e - 3 * HD4 - 2 * p.H;
-            float s = 0.0f;
-            for (int q = 0; q < nout_part; ++q) s += p.dnw_part[static_cast<size_t>(q) * D + c];
-            p.dnorm_w[c] = s;
+            p.dnorm_w[e - 3 * HD4 - 2 * p.H] = s;
         }
     }
 }
 
 template <typename ZT, typename YT>
 cudaError_t launch_out_bwd(const BwdParams &p, int blocks, cudaStream_t s) {
-    if (p.d == 128) gdn_bwd_out<ZT, YT, 128><<<blocks, 256, 0, s>>>(p);
-    else gdn_bwd_out<ZT, YT, 64><<<blocks, 256, 0, s>>>(p);
+    if (p.dO16) gdn_bwd_out<ZT, YT, 128, true><<<blocks, 256, 0, s>>>(p);
+    else if (p.d == 128) gdn_bwd_out<ZT, YT, 128, false><<<blocks, 256, 0, s>>>(p);
+    else gdn_bwd_out<ZT, YT, 64, false><<<blocks, 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 template <typename ZT>
@@ -570,6 +797,32 @@ cudaError_t launch_tokens_bwd(const BwdParams &p, cudaStream_t s) {
 }
 
 }  // namespace
+
+cudaError_t launch_bwd_out(const BwdParams &p, InType in, InType out, cudaStream_t s) {
+    const int nb = bwd_out_blocks(static_cast<long long>(p.B) * p.T * p.H);
+    if (in == InType::BF16) return launch_out_bwd_z<__nv_bfloat16>(p, out, nb, s);
+    if (in == InType::F16) return launch_out_bwd_z<__half>(p, out, nb, s);
+    return launch_out_bwd_z<float>(p, out, nb, s);
+}
+
+cudaError_t launch_bwd_tokens(const BwdParams &p, InType in, cudaStream_t s) {
+    if (p.tc && p.d == 128) {  // whole per-token gradients: one warp per row
+        const dim3 grid(p.Tp / kTile, p.H, p.B);
+        if (in == InType::BF16) gdn_bwd_tokens_rows<__nv_bfloat16><<<grid, 256, 0, s>>>(p);
+        else if (in == InType::F16) gdn_bwd_tokens_rows<__half><<<grid, 256, 0, s>>>(p);
+        else gdn_bwd_tokens_rows<float><<<grid, 256, 0, s>>>(p);
+        return cudaGetLastError();
+    }
+    if (in == InType::BF16) return launch_tokens_bwd<__nv_bfloat16>(p, s);
+    if (in == InType::F16) return launch_tokens_bwd<__half>(p, s);
+    return launch_tokens_bwd<float>(p, s);
+}
+
+cudaError_t launch_bwd_params(const BwdParams &p, cudaStream_t s) {
+    const int total = 3 * p.H * p.d * 4 + 2 * p.H + p.d;
+    gdn_bwd_params_split<<<(total + 31) / 32, 256, 0, s>>>(p, p.d, bwd_out_blocks(static_cast<long long>(p.B) * p.T * p.H));
+    return cudaGetLastError();
+}
 
 int bwd_out_blocks(long long rows) {
     long long blocks = (rows + 7) / 8;
@@ -608,8 +861,7 @@ cudaError_t launch_backward(const BwdParams &p, InType in, InType out, cudaStrea
     if (e != cudaSuccess) return e;
     ++n;
     if ((e = mark(4)) != cudaSuccess) return e;
-    gdn_bwd_params<<<64, 256, 0, s>>>(p, p.d, nb);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_bwd_params(p, s)) != cudaSuccess) return e;
     ++n;
     if ((e = mark(5)) != cudaSuccess) return e;
     if (launches) *launches = n;

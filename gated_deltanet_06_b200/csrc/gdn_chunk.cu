@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(256, 2)
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmU,
                      const __grid_constant__ CUtensorMap tmQt, const __grid_constant__ CUtensorMap tmAqk,
-                     const __grid_constant__ CUtensorMap tmAqkH) {
+                     const __grid_constant__ CUtensorMap tmAqkH, const __grid_constant__ CUtensorMap tmT) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
@@ -432,6 +432,14 @@ __global__ void __launch_bounds__(256, 2)
         group_sync(1);
         if (tid == 0) GDN_TRACE_AT(22);
         fence_proxy_async();  // T is read by the tensor cores next
+        if (p.save) {  // T kept for the backward: one bulk store of the finished tile
+            group_sync(1);
+            if (tid == 0) {
+                tma_store_2d(&tmT, sm + OFF_LT, 0, y0);
+                tma_store_2d(&tmT, sm + OFF_LT + 16384, 64, y0);
+                bulk_commit();
+            }
+        }
         if (tid == 0) GDN_TRACE_AT(4);
         // ---- Aqk rows (the decay split as for the L rows), stored straight to global memory: a
         //      block's 128 rows are 32 contiguous KB.  Aqk is block lower triangular; its upper-right
@@ -440,7 +448,7 @@ __global__ void __launch_bounds__(256, 2)
             __half *arow_g = p.Aqk + (row0 + r) * 128;
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
-                if (r < 64 && c >= 2) break;
+                if (r < 64 && c >= 2 && !p.save) break;
                 float a[32];
                 if (c > warp) {
 #pragma unroll
@@ -543,6 +551,7 @@ __global__ void __launch_bounds__(256, 2)
         ++mma_commits;
     }
     mbar_wait(bar_mma, 1, ab, p.status, p.wait_limit_ns);
+    if (tid == 0 && p.save) bulk_wait_read_all();  // the T store has read the tile W is staged in
     __syncthreads();
     if (ab->flag) goto teardown;
     tc_fence_after();
@@ -594,13 +603,13 @@ teardown:
 cudaError_t launch_chunk(const ChunkParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
                          const CUtensorMap &tmQ, const CUtensorMap &tmW, const CUtensorMap &tmU,
                          const CUtensorMap &tmQt, const CUtensorMap &tmAqk, const CUtensorMap &tmAqkH,
-                         cudaStream_t s, bool pdl) {
+                         const CUtensorMap &tmT, cudaStream_t s, bool pdl) {
     static SmemOnce once;
     cudaError_t e = raise_smem_once(once, gdn_chunk_kernel, static_cast<int>(SMEM_BYTES));
     if (e != cudaSuccess) return e;
     dim3 grid(p.NB, p.BH);
     return launch_k(gdn_chunk_kernel, grid, dim3(256), SMEM_BYTES, s, pdl, p, tmK, tmV, tmQ, tmW, tmU, tmQt, tmAqk,
-                    tmAqkH);
+                    tmAqkH, tmT);
 }
 
 }  // namespace gdn

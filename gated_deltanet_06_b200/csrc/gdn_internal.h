@@ -117,11 +117,14 @@ struct ChunkParams {
     unsigned long long wait_limit_ns;
     int rev;                        // reverse scan: block row t holds the gates of input token T-1-t
     int debug;                      // GDN_FLAG_DEBUG_CHECKS: index-bounds checks on the gate accesses
+    int save;                       // for the backward: also store T = (I + L)^-1 (through tmT) and
+                                    // Aqk's zero upper-right quadrant, so that every Aqk tile is whole
 };
 cudaError_t launch_chunk(const ChunkParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
                          const CUtensorMap &tmQ, const CUtensorMap &tmW, const CUtensorMap &tmU,
                          const CUtensorMap &tmQt, const CUtensorMap &tmAqk, const CUtensorMap &tmAqkH,
-                         cudaStream_t s, bool pdl);  // Kt is written with plain coalesced stores
+                         const CUtensorMap &tmT, cudaStream_t s,
+                         bool pdl);  // Kt is written with plain coalesced stores; tmT is read only with save
 
 // Inter-block state scan on tensor cores (d = 128), parallel over segments of
 // Ls blocks: pass A (transfer), combine, pass C (outputs + fused output step).
@@ -143,11 +146,21 @@ struct ScanParams {
     float *s_end;            // [BH][128][128] state after token T-1, or null (not wanted)
     int rev;                 // reverse scan: block row t is z / y token T-1-t
     int debug;               // check that every output value is finite (status word)
+    // for the backward (pass C): o itself instead of the normalised, gated output (fp32 into y,
+    // out_kind 1), and S^T at the start of every block, fp16 [BH][Tp][128] (block c: rows c*128 ..)
+    int raw_o;
+    __half *S0b;
+    // backward combine: dS^T at every segment end from the backward transfer's local gradients
+    const float *Lb;         // [BH][NS][128][128]: local dS^T of each segment (zero at its end)
+    float *Sb;               // [BH][NS][128][128]: dS^T at each segment end
 };
 // pdl: launch with programmatic stream serialization (see launch_k).
 cudaError_t launch_transfer(const ScanParams &p, const CUtensorMap &tmW, const CUtensorMap &tmKt,
                             const CUtensorMap &tmU, cudaStream_t s, bool pdl);
 cudaError_t launch_combine(const ScanParams &p, cudaStream_t s, bool pdl);
+// The combine for the backward: dS^T at each segment end (Sb) from the local gradients (Lb) and the
+// forward's transfers (Zloc), last segment first.
+cudaError_t launch_combine_bwd(const ScanParams &p, cudaStream_t s, bool pdl);
 cudaError_t launch_scan_out(const ScanParams &p, InType zt, const CUtensorMap &tmW, const CUtensorMap &tmQt,
                             const CUtensorMap &tmKt, const CUtensorMap &tmAqk, const CUtensorMap &tmAqkH,
                             const CUtensorMap &tmU, const CUtensorMap &tmZ, cudaStream_t s, bool pdl);
@@ -230,8 +243,48 @@ struct BwdParams {
     float *dnorm_w;                 // [d]
     int B, T, H, d, Tp;
     float l2_eps, norm_eps, q_scale;
+    // the tensor-core backward: one whole gradient per token in dq_part / dk_part (groups = 1) and
+    // d log alpha itself in da_part (tc = 1); dO written as fp16 into dO16 instead of dO
+    int groups;
+    int tc;
+    __half *dO16;
 };
 int bwd_out_blocks(long long rows);
+// The output step backwards (do, dz, norm-weight partials) and the per-token / parameter steps,
+// shared by both backward paths.
+cudaError_t launch_bwd_out(const BwdParams &p, InType in, InType out, cudaStream_t s);
+cudaError_t launch_bwd_tokens(const BwdParams &p, InType in, cudaStream_t s);
+cudaError_t launch_bwd_params(const BwdParams &p, cudaStream_t s);
+
+// The backward on tensor cores (16-bit inputs, d = 128), in the block (UT) form, over the forward's
+// kept intermediates: a reverse scan of the state gradient dS over segments (transfer pass, combine,
+// final pass writing dS^T at every block end), then every block's local gradients.
+struct BwdTcParams {
+    const float *G, *beta;                 // [BH][Tp]: in-block cumulative log decay, update gate
+    const __half *Q, *K, *V;               // q^ (with 1/sqrt(d_k)), k^, v^: [BH][Tp][128]
+    const __half *W, *U, *Kt, *Aqk;        // the UT kernel's tiles (Aqk whole)
+    const __half *S0b;                     // S^T at every block start (pass C with S0b)
+    __half *dSb;                           // dS^T at every block end (the backward's final pass)
+    float *dSloc;                          // [BH][NS][128][128]: each segment's dS^T from zero at its end
+    const float *dSend;                    // [BH][NS][128][128]: dS^T at each segment end (segments < NS-1)
+    float *dqh, *dkh, *dvh;                // [BH][Tp][128]: gradients of Q (q^ with its scale), k^, v^
+    float *dla, *dbeta;                    // [BH][Tp]: gradients of log alpha and beta
+    int BH, Tp, NB, NS, Ls;
+    float q_scale;                         // 1/sqrt(d_k), folded into Q (the per-token step applies it)
+    int *status;
+    unsigned long long wait_limit_ns;
+};
+// Reverse pass over the segments (grid: segments x BH).  final = false: segments 1 .. NS-1 from a zero
+// gradient at their end, writing dSloc; final = true: every segment from dSend (zero for the last),
+// writing dSb.  Tiles: Aqk, dO, Kt, Qt, W ([BH*Tp][128] fp16 maps, {64, 128} boxes, 128-byte swizzle).
+cudaError_t launch_bwd_scan(const BwdTcParams &p, bool final_pass, const CUtensorMap &tmAqk,
+                            const CUtensorMap &tmDO, const CUtensorMap &tmKt, const CUtensorMap &tmQt,
+                            const CUtensorMap &tmW, cudaStream_t s, bool pdl);
+// Local gradients of every block (persistent grid); maps as above.
+struct BwdTcMaps {
+    CUtensorMap S0, W, dO, Aqk, Kt, dS, K, Q, T, U, V;  // V: L2 prefetch only
+};
+cudaError_t launch_bwd_grad(const BwdTcParams &p, const BwdTcMaps &m, cudaStream_t s, bool pdl);
 // Enqueues the five backward kernels after the prep; *launches receives their count.  events
 // (optional, 6 cudaEvent_t) are recorded before each launch and after the last.
 cudaError_t launch_backward(const BwdParams &p, InType in, InType out, cudaStream_t s, int *launches,
@@ -293,9 +346,17 @@ bool plan_layout(const gdn_plan_s *plan, PlanLayout *out);
 // with token stride z_stride; y bf16/f16/f32 per the plan.  The status word is not cleared here.
 // Returns a gdn_status value.
 // events (optional): one cudaEvent_t recorded before each launch, *ev counts them.
+// save (optional, for the backward): keep T = (I + L)^-1 and the whole Aqk tiles, write o itself
+// (fp32 [B][T][H][128]) instead of y, and S^T at every block start (fp16 [BH][Tp][128]).
+struct FwdSave {
+    __half *T;
+    __half *S0b;
+    float *o;
+};
 int run_tensor_core(const gdn_plan_s *plan, const float *g, const float *b, const float *A_log,
                     const float *dt_bias, const float *norm_w, const void *z, InType z_type,
                     long long z_stride, void *y, void *workspace, cudaStream_t s, bool pdl_first,
-                    void *const *events, int *ev, const float *s0, float *s_end);
+                    void *const *events, int *ev, const float *s0, float *s_end,
+                    const FwdSave *save = nullptr);
 int tensor_core_launches(const gdn_plan_s *plan);
 }  // namespace gdn

@@ -45,6 +45,17 @@ __device__ __forceinline__ void store_f16_chunk(uint8_t *tile, int rows, int r, 
     u.w = pack_half2(v[6], v[7]);
     *reinterpret_cast<uint4 *>(tile + tile_off(rows, r, chunk16)) = u;
 }
+// as store_f16_chunk, and the same 16 bytes to global row `grow` (columns 8 chunk16 ..) when grow is set
+__device__ __forceinline__ void store_f16_chunk2(uint8_t *tile, int rows, int r, int chunk16, const float *v,
+                                                 __half *grow) {
+    uint4 u;
+    u.x = pack_half2(v[0], v[1]);
+    u.y = pack_half2(v[2], v[3]);
+    u.z = pack_half2(v[4], v[5]);
+    u.w = pack_half2(v[6], v[7]);
+    *reinterpret_cast<uint4 *>(tile + tile_off(rows, r, chunk16)) = u;
+    if (grow) *reinterpret_cast<uint4 *>(grow + chunk16 * 8) = u;
+}
 
 // Warp-uniform bounded wait (every lane waits; the warp proceeds only if all did).
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t ph, volatile AbortState *ab, int *status,
@@ -315,6 +326,7 @@ __device__ __forceinline__ void mma1688_tf32(float (&d)[4], const uint32_t (&a)[
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
+template <bool kBwd>
 __global__ void __launch_bounds__(256, 1) gdn_combine_kernel(const ScanParams p) {
     using cb::RS;
     extern __shared__ __align__(16) float csm[];
@@ -327,7 +339,16 @@ __global__ void __launch_bounds__(256, 1) gdn_combine_kernel(const ScanParams p)
     const int r0 = warp * 16;  // this warp's rows r0 + g and r0 + g + 8
     constexpr size_t kZ = 128 * 256;  // floats per (bh, segment) of Zloc
     const float *Z = p.Zloc + static_cast<size_t>(bh) * p.NS * kZ;
-    float *Sst = p.Sstart + static_cast<size_t>(bh) * p.NS * 128 * 128;
+    // Backward (gradient of the state, last segment first): with X = dS^T at a segment end,
+    //   X(j) = P_(j+1) X(j+1) + L(j+1),  L = the segment's local dS^T (from zero at its end),
+    // the same recurrence with P_j^T read transposed, the segments taken in reverse order, L from
+    // its own [NS][128][128] array and the results written for segment ends NS-2 .. 0.  Step j of
+    // the loop below uses segment seg_of(j) and writes the start of step j + 1 to out_of(j + 1).
+    auto seg_of = [&](int j) { return kBwd ? p.NS - 1 - j : j; };
+    auto out_of = [&](int j) { return kBwd ? p.NS - 1 - j : j; };
+    const float *Lsrc = kBwd ? p.Lb + static_cast<size_t>(bh) * p.NS * 128 * 128 : Z;
+    constexpr int kLs = kBwd ? 128 : 256;  // row stride of L
+    float *Sst = (kBwd ? p.Sb : p.Sstart) + static_cast<size_t>(bh) * p.NS * 128 * 128;
     // debug: this head's segments inside Zloc and Sstart
     if (!debug_in_bounds(p.debug, static_cast<size_t>(bh) * p.NS * kZ, static_cast<size_t>(p.NS) * kZ,
                          static_cast<size_t>(p.B) * p.H * p.NS * kZ, p.status))
@@ -337,7 +358,7 @@ __global__ void __launch_bounds__(256, 1) gdn_combine_kernel(const ScanParams p)
     if (p.NS < 2) return;
 
     auto load_pt = [&](int j) {  // rows of P_j^T: 32 16-byte pieces each, a warp per row at a time
-        const float *src = Z + j * kZ + 128;
+        const float *src = Z + seg_of(j) * kZ + 128;
         float *dst = PT + (j & 1) * 128 * RS;
 #pragma unroll 4
         for (int e = tid; e < 128 * 32; e += 256) {
@@ -352,8 +373,9 @@ __global__ void __launch_bounds__(256, 1) gdn_combine_kernel(const ScanParams p)
         for (int n = 0; n < 2; ++n)
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh)
-                v[n][hh] = *reinterpret_cast<const float2 *>(Z + j * kZ + static_cast<size_t>(r0 + g + 8 * hh) * 256 +
-                                                            slice * 16 + 8 * n + 2 * t4);
+                v[n][hh] = *reinterpret_cast<const float2 *>(Lsrc + static_cast<size_t>(seg_of(j)) * 128 * kLs +
+                                                            static_cast<size_t>(r0 + g + 8 * hh) * kLs + slice * 16 +
+                                                            8 * n + 2 * t4);
     };
     if (tid == 0) GDN_TRACE_AT(2048);
     if (p.NS > 2) load_pt(1);
@@ -361,9 +383,9 @@ __global__ void __launch_bounds__(256, 1) gdn_combine_kernel(const ScanParams p)
     // S_start(1) = S_loc(0)
     for (int e = tid; e < 128 * 16; e += 256) {
         const int t = e >> 4, c = e & 15;
-        const float v = Z[static_cast<size_t>(t) * 256 + slice * 16 + c];
+        const float v = Lsrc[static_cast<size_t>(seg_of(0)) * 128 * kLs + static_cast<size_t>(t) * kLs + slice * 16 + c];
         curT[c * RS + t] = v;
-        Sst[(static_cast<size_t>(1) * 128 + t) * 128 + slice * 16 + c] = v;
+        Sst[(static_cast<size_t>(out_of(1)) * 128 + t) * 128 + slice * 16 + c] = v;
     }
     float2 sl[2][2];
     if (p.NS > 2) load_sl(1, sl);
@@ -394,10 +416,12 @@ __global__ void __launch_bounds__(256, 1) gdn_combine_kernel(const ScanParams p)
 #pragma unroll 4
         for (int k0 = 0; k0 < 128; k0 += 8) {
             uint32_t ah[4], al[4];
-            split_tf32(P[(r0 + g) * RS + k0 + t4], ah[0], al[0]);
-            split_tf32(P[(r0 + g + 8) * RS + k0 + t4], ah[1], al[1]);
-            split_tf32(P[(r0 + g) * RS + k0 + t4 + 4], ah[2], al[2]);
-            split_tf32(P[(r0 + g + 8) * RS + k0 + t4 + 4], ah[3], al[3]);
+            // A fragment: element (row, k) of P_j^T, or of P_(j+1) (the stored tile transposed)
+            auto pa = [&](int row, int k) { return kBwd ? P[k * RS + row] : P[row * RS + k]; };
+            split_tf32(pa(r0 + g, k0 + t4), ah[0], al[0]);
+            split_tf32(pa(r0 + g + 8, k0 + t4), ah[1], al[1]);
+            split_tf32(pa(r0 + g, k0 + t4 + 4), ah[2], al[2]);
+            split_tf32(pa(r0 + g + 8, k0 + t4 + 4), ah[3], al[3]);
 #pragma unroll
             for (int n = 0; n < 2; ++n) {
                 uint32_t bh2[2], bl2[2];
@@ -423,7 +447,7 @@ __global__ void __launch_bounds__(256, 1) gdn_combine_kernel(const ScanParams p)
                 const float v0 = acc[n][2 * hh], v1 = acc[n][2 * hh + 1];
                 curT[c * RS + t] = v0;
                 curT[(c + 1) * RS + t] = v1;
-                *reinterpret_cast<float2 *>(Sst + (static_cast<size_t>(j + 1) * 128 + t) * 128 + slice * 16 + c) =
+                *reinterpret_cast<float2 *>(Sst + (static_cast<size_t>(out_of(j + 1)) * 128 + t) * 128 + slice * 16 + c) =
                     make_float2(v0, v1);
             }
         }
@@ -562,8 +586,8 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
             ssA += __shfl_xor_sync(0xffffffffu, ssA, 2);
             ssB += __shfl_xor_sync(0xffffffffu, ssB, 1);
             ssB += __shfl_xor_sync(0xffffffffu, ssB, 2);
-            const float rnA = 1.0f / sqrtf(ssA * (1.0f / 128.0f) + p.eps);
-            const float rnB = 1.0f / sqrtf(ssB * (1.0f / 128.0f) + p.eps);
+            const float rnA = p.raw_o ? 1.0f : 1.0f / sqrtf(ssA * (1.0f / 128.0f) + p.eps);
+            const float rnB = p.raw_o ? 1.0f : 1.0f / sqrtf(ssB * (1.0f / 128.0f) + p.eps);
             if (tre) GDN_TRACE_AT(4096 + 64 * i + 34);
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
@@ -589,6 +613,13 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
                         } else {
                             fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wa[j]));
                             fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wb[j]));
+                        }
+                        if (p.raw_o) {  // o itself, for the backward
+                            yf[0][j][0] = __uint_as_float(v[4 * gl]);
+                            yf[0][j][1] = __uint_as_float(v[4 * gl + 1]);
+                            yf[1][j][0] = __uint_as_float(v[4 * gl + 2]);
+                            yf[1][j][1] = __uint_as_float(v[4 * gl + 3]);
+                            continue;
                         }
                         yf[0][j][0] = __uint_as_float(v[4 * gl]) * rnA * w0 * silu_tc(fa.x);
                         yf[0][j][1] = __uint_as_float(v[4 * gl + 1]) * rnA * w1 * silu_tc(fa.y);
@@ -786,8 +817,9 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
                 }
             }
             tmem_st32(tmem + lane_base + TM_S + ch * 32, v);
+            __half *g0 = p.S0b ? p.S0b + (static_cast<size_t>(bh) * p.Tp + static_cast<size_t>(c0) * kBlk + r) * 128 : nullptr;
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq) store_f16_chunk(sm + OFF_S, 128, r, ch * 4 + qq, &v[qq * 8]);
+            for (int qq = 0; qq < 4; ++qq) store_f16_chunk2(sm + OFF_S, 128, r, ch * 4 + qq, &v[qq * 8], g0);
         }
         tmem_st_wait();
         fence_proxy_async();
@@ -838,6 +870,10 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
             if (!warp_wait(&bars[MMA_P], ph, ab, p.status, lim)) break;
             if (tr) GDN_TRACE_AT(4096 + 64 * i + 20);
             tc_fence_after();
+            // the state at the start of block c + 1, kept for the backward
+            __half *gs = (p.S0b && c + 1 < c1)
+                             ? p.S0b + (static_cast<size_t>(bh) * p.Tp + static_cast<size_t>(c + 1) * kBlk + r) * 128
+                             : nullptr;
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
                 float pv[32], sv[32];
@@ -847,7 +883,7 @@ __global__ void __launch_bounds__(tc::kScanThreads, 1)
                 for (int e = 0; e < 32; ++e) sv[e] = fmaf(gC, sv[e], pv[e]);
                 tmem_st32(tmem + lane_base + TM_S + ch * 32, sv);
 #pragma unroll
-                for (int qq = 0; qq < 4; ++qq) store_f16_chunk(sm + OFF_S, 128, r, ch * 4 + qq, &sv[qq * 8]);
+                for (int qq = 0; qq < 4; ++qq) store_f16_chunk2(sm + OFF_S, 128, r, ch * 4 + qq, &sv[qq * 8], gs);
             }
             tmem_st_wait();
             fence_proxy_async();
@@ -891,10 +927,18 @@ cudaError_t launch_transfer(const ScanParams &p, const CUtensorMap &tmW, const C
 
 cudaError_t launch_combine(const ScanParams &p, cudaStream_t s, bool pdl) {
     static SmemOnce once;
-    cudaError_t e = raise_smem_once(once, gdn_combine_kernel, static_cast<int>(cb::SMEM_BYTES));
+    cudaError_t e = raise_smem_once(once, gdn_combine_kernel<false>, static_cast<int>(cb::SMEM_BYTES));
     if (e != cudaSuccess) return e;
     dim3 grid(8, p.H, p.B);
-    return launch_k(gdn_combine_kernel, grid, dim3(256), cb::SMEM_BYTES, s, pdl, p);
+    return launch_k(gdn_combine_kernel<false>, grid, dim3(256), cb::SMEM_BYTES, s, pdl, p);
+}
+
+cudaError_t launch_combine_bwd(const ScanParams &p, cudaStream_t s, bool pdl) {
+    static SmemOnce once;
+    cudaError_t e = raise_smem_once(once, gdn_combine_kernel<true>, static_cast<int>(cb::SMEM_BYTES));
+    if (e != cudaSuccess) return e;
+    dim3 grid(8, p.H, p.B);
+    return launch_k(gdn_combine_kernel<true>, grid, dim3(256), cb::SMEM_BYTES, s, pdl, p);
 }
 
 cudaError_t launch_scan_out(const ScanParams &p, InType zt, const CUtensorMap &tmW, const CUtensorMap &tmQt,

@@ -229,11 +229,15 @@ typedef struct {
 } gdn_grads;
 
 /* Bytes of device workspace gdn_backward needs for this plan (256-byte
- * aligned; a separate size from gdn_forward's): the forward recomputed in
+ * aligned; a separate size from gdn_forward's).  Tensor-path plans without
+ * GDN_FLAG_FUSED: the forward's workspace, then the kept block tiles and
+ * states, the state gradients and the per-token gradients
+ * (gdn_backward_workspace_offsets).  Other plans: the forward recomputed in
  * fp32, the state every 8 tokens, and per-group partial sums. */
 size_t gdn_backward_workspace_bytes(gdn_plan_t plan);
 
-/* Kernel launches one gdn_backward enqueues (6). */
+/* Kernel launches one gdn_backward enqueues: 12 (8 with one segment) on the
+ * tensor-core backward, 6 otherwise. */
 int gdn_backward_launches(gdn_plan_t plan);
 
 /* No counterpart written out in the pages, which train the GDN modules
@@ -241,10 +245,22 @@ int gdn_backward_launches(gdn_plan_t plan);
  * mapping) without giving the gradient: the gradient of the forward of
  * gdn_forward with respect to every input and parameter, for the loss
  * L = sum(y * dy).  dy is [B][T][H][d_v] of the plan's out_dtype, dense.
- * Computed in fp32 on CUDA cores for every plan (bf16/f16 inputs are widened
- * exactly): the forward is recomputed from the inputs, the recurrence's state
- * is checkpointed every 8 tokens and rebuilt chunk by chunk while its
- * gradient runs backwards.  Deterministic: every sum has a fixed order.
+ * Plans on the tensor path without GDN_FLAG_FUSED (16-bit inputs, d = 128):
+ * on tensor cores, in the block (UT) form of the recurrence.  The forward
+ * runs once more keeping its 128-token block tiles (and T = (I + L)^-1, the
+ * state at every block start, o); the state gradient dS runs backwards over
+ * segments of blocks in parallel (a transfer pass, a combine through the
+ * forward's segment transfers, a final pass that writes dS at every block
+ * end), then every block's gradients follow from its tiles, S and dS by 16
+ * tcgen05 products (fp16 operands, fp32 accumulation), and the per-token
+ * steps (L2 norm, SiLU, conv, gates) run in fp32.  Precision: relative L2
+ * errors of a few 1e-4 against the exact gradient on N(0,1) inputs (fp16
+ * operand rounding, as in the forward); the fp16 range limits of the
+ * forward apply to the kept tiles, the states and dL/do.  Other plans (fp32
+ * inputs, d = 64, GDN_FLAG_FUSED): fp32 on CUDA cores, the forward
+ * recomputed from the inputs, the recurrence's state checkpointed every 8
+ * tokens and rebuilt chunk by chunk while its gradient runs backwards.
+ * Deterministic on both paths: every sum has a fixed order.
  * Errors: INVALID_ARG (null or misaligned pointers, the workspace checks of
  * gdn_forward), UNSUPPORTED for GDN_FLAG_REVERSE plans; asynchronous on
  * `stream` like gdn_forward. */
@@ -296,6 +312,26 @@ int gdn_plan_segments(gdn_plan_t plan);
  *     fused forward keeps its other intermediates on chip).
  * Returns the number of offsets written (17 at most). */
 int gdn_workspace_offsets(gdn_plan_t plan, size_t *offsets, int n);
+
+/* Byte offsets of the tensor-core backward's own buffers inside the
+ * gdn_backward workspace (plans on the tensor path without GDN_FLAG_FUSED;
+ * their gdn_backward workspace starts with the forward's layout, at the
+ * offsets gdn_workspace_offsets reports), in this order:
+ *   0 T = (I + L)^-1 per 128-token block, 1 S^T at every block start
+ *     (both [B][H][Tp][128] fp16, block c at rows 128c ..),
+ *   2 o before the output norm ([B][T][H][d_v] fp32), 3 dL/do
+ *     ([B][H][Tp][128] fp16, zero past T),
+ *   4 each segment's local dS^T from zero at its end and 5 dS^T at every
+ *     segment end ([B][H][NS][128][128] fp32; 5 unused for the last segment),
+ *   6 dS^T at every block end ([B][H][Tp][128] fp16),
+ *   7 dL/dQ for Q = q^/sqrt(d_k), 8 dL/dk^, 9 dL/dv^
+ *     ([B][H][Tp][128] fp32), 10 dL/d log alpha and 11 dL/d beta
+ *     ([B][H][Tp] fp32),
+ *   12 norm-weight partial sums, 13 conv-weight partial sums, 14 A_log
+ *     partial sums.
+ * Returns the number of offsets written (15 at most), 0 for other plans.
+ * For tests and profiling: the contents are valid after gdn_backward. */
+int gdn_backward_workspace_offsets(gdn_plan_t plan, size_t *offsets, int n);
 
 /* Free a plan (host memory only).  NULL is accepted. */
 gdn_status gdn_destroy(gdn_plan_t plan);

@@ -250,3 +250,109 @@ def chunk_core_backward(qh, kh, vh, log_alpha, beta, do, C=64):
                 out["dbeta"][b, r0:r0 + rows, h] = dbeta[:rows]
                 dS = dS0
     return out
+
+
+def ut_backward(qh, kh, vh, log_alpha, beta, do, C=128):
+    """The block backward as the tensor-core kernels take it (fp64, no rounding):
+    the forward's block tiles (T, W, U, P = Aqk, Qt, Kt) and S0 at every block
+    start, the state gradient dS at every block end by the reverse recurrence
+      dDelta = P^T dO + Kt dS^T,  dS_start = e^(G_last) dS + dO^T Qt - dDelta^T W,
+    then every block's local gradients from its tiles, S0 and dS alone:
+      dQ  = diag(E) dO S0 + dQK K,  dQK = (dO Delta^T) o Gam
+      dK  = dQK^T Q + diag(e^(G_last - G)) Delta dS + diag(beta E) T^T dW + (dA + dA^T) K
+      dV  = diag(beta) T^T dDelta,  dW = -dDelta S0
+      dL  = -(dKb W^T + dVb U^T) o strict,  dA = diag(beta) dL o Gam
+    with dG collected from every e^G factor (row sums minus column sums of the
+    decay-masked products) and d log alpha its reverse cumulative sum over the
+    block, plus e^(G_last) <dS, S0> + sum(dKd o Kt) on every token.
+    Returns the gradients (as chunk_core_backward) and the per-(b, h) lists of
+    S0^T and dS^T per block (d_k x d_v)."""
+    B, T, H, dk = qh.shape
+    dv = vh.shape[-1]
+    nc = -(-T // C)
+    Tp = nc * C
+    scale = 1.0 / np.sqrt(dk)
+    out = {n: np.zeros(s) for n, s in (("dq", qh.shape), ("dk", kh.shape), ("dv", vh.shape),
+                                       ("dla", log_alpha.shape), ("dbeta", beta.shape))}
+    out["S0T"] = np.zeros((B, H, nc, dk, dv))
+    out["dST"] = np.zeros((B, H, nc, dk, dv))
+    strict = np.tril(np.ones((C, C)), -1)
+    incl = np.tril(np.ones((C, C)))
+    for b in range(B):
+        for h in range(H):
+            def pad(x):
+                o_ = np.zeros((Tp,) + x.shape[1:])
+                o_[:T] = x
+                return o_
+            Q = pad(qh[b, :, h]) * scale
+            K, V = pad(kh[b, :, h]), pad(vh[b, :, h])
+            la, be, dO = pad(log_alpha[b, :, h]), pad(beta[b, :, h]), pad(do[b, :, h])
+            blocks = []
+            S = np.zeros((dv, dk))
+            for c in range(nc):
+                sl = slice(c * C, (c + 1) * C)
+                G = np.cumsum(la[sl])
+                E, bc = np.exp(G), be[sl]
+                Dm = np.minimum(G[:, None] - G[None, :], 0.0)
+                Gs, Gam = strict * np.exp(Dm), incl * np.exp(Dm)
+                Kc, Vc, Qc = K[sl], V[sl], Q[sl]
+                A = Kc @ Kc.T
+                Tm = np.linalg.inv(np.eye(C) + Gs * bc[:, None] * A)
+                W, U = Tm @ ((bc * E)[:, None] * Kc), Tm @ (bc[:, None] * Vc)
+                P = Gam * (Qc @ Kc.T)
+                Qt, Kt = E[:, None] * Qc, np.exp(G[-1] - G)[:, None] * Kc
+                blocks.append(dict(G=G, E=E, bc=bc, Kc=Kc, Vc=Vc, Qc=Qc, Tm=Tm, W=W, U=U, P=P, Qt=Qt, Kt=Kt,
+                                   S0=S.copy(), Gs=Gs, Gam=Gam, A=A, dO=dO[sl]))
+                out["S0T"][b, h, c] = S.T
+                S = np.exp(G[-1]) * S + (U - W @ S.T).T @ Kt
+            dS = np.zeros((dv, dk))
+            dS_end = [None] * nc
+            for c in range(nc - 1, -1, -1):
+                f = blocks[c]
+                dS_end[c] = dS
+                out["dST"][b, h, c] = dS.T
+                dDelta = f["P"].T @ f["dO"] + f["Kt"] @ dS.T
+                dS = np.exp(f["G"][-1]) * dS + f["dO"].T @ f["Qt"] - dDelta.T @ f["W"]
+            for c in range(nc):
+                f = blocks[c]
+                G, E, bc, Kc, Vc, Qc = f["G"], f["E"], f["bc"], f["Kc"], f["Vc"], f["Qc"]
+                Tm, W, U, P, Kt, S0, Gs, Gam, A, dOc = (f[n] for n in ("Tm", "W", "U", "P", "Kt", "S0", "Gs", "Gam",
+                                                                        "A", "dO"))
+                dSc, gL = dS_end[c], G[-1]
+                Delta = U - W @ S0.T
+                dDelta = P.T @ dOc + Kt @ dSc.T
+                dOS = dOc @ S0
+                dE = (dOS * Qc).sum(1)
+                dPr = dOc @ Delta.T
+                dQK = dPr * Gam
+                dPP = dPr * P
+                dG = dPP.sum(1) - dPP.sum(0)
+                dQ = E[:, None] * dOS + dQK @ Kc
+                dKd = Delta @ dSc
+                t = (dKd * Kt).sum(1)
+                dG -= t
+                dgC = np.exp(gL) * float((dSc * S0).sum()) + float(t.sum())
+                dK = dQK.T @ Qc + np.exp(gL - G)[:, None] * dKd
+                dW = -dDelta @ S0
+                dKb, dVb = Tm.T @ dW, Tm.T @ dDelta
+                tk = (dKb * Kc).sum(1)
+                dK += (bc * E)[:, None] * dKb
+                dbeta = E * tk + (dVb * Vc).sum(1)
+                dE += bc * tk
+                dL = -(dKb @ W.T + dVb @ U.T) * strict
+                dLGA = dL * Gs * A
+                dbeta += dLGA.sum(1)
+                dLL = bc[:, None] * dLGA
+                dG += dLL.sum(1) - dLL.sum(0)
+                dA = bc[:, None] * dL * Gs
+                dK += (dA + dA.T) @ Kc
+                dG += E * dE
+                dla = np.cumsum(dG[::-1])[::-1] + dgC
+                rows = min(C, T - c * C)
+                r0 = c * C
+                out["dq"][b, r0:r0 + rows, h] = dQ[:rows] * scale
+                out["dk"][b, r0:r0 + rows, h] = dK[:rows]
+                out["dv"][b, r0:r0 + rows, h] = bc[:rows, None] * dVb[:rows]
+                out["dla"][b, r0:r0 + rows, h] = dla[:rows]
+                out["dbeta"][b, r0:r0 + rows, h] = dbeta[:rows]
+    return out

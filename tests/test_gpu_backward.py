@@ -1,11 +1,13 @@
-"""gdn_backward on a B200 against the oracle's backward (fp64, written out
-per step and pinned by finite differences).
+"""gdn_backward's fp32 CUDA-core path on a B200 against the oracle's backward
+(fp64, written out per step and pinned by finite differences): fp32 plans,
+d = 64 plans, and 16-bit plans with GDN_FLAG_FORCE_SIMT (16-bit plans with
+d = 128 otherwise take the tensor-core backward, tested in
+test_gpu_backward_tc.py).
 
-The bar: the backward runs in fp32 on CUDA cores for every plan, so each
-gradient tensor takes the fp32 forward's bar, rel-L2 <= 1e-5 against the
-oracle on the same inputs and dy.  Measured: about 2e-7 for the per-token
-gradients and up to 1.2e-6 for dA_log and ddt_bias, whose H entries are each
-a sum over every token with cancellation.
+The bar: each gradient tensor takes the fp32 forward's bar, rel-L2 <= 1e-5
+against the oracle on the same inputs and dy.  Measured: about 2e-7 for the
+per-token gradients and up to 1.2e-6 for dA_log and ddt_bias, whose H entries
+are each a sum over every token with cancellation.
 """
 import numpy as np
 import pytest
@@ -56,11 +58,12 @@ def _check_all(got, ref, what):
                                                   ("bf16", 128, 1, 130, 3, 0.0),
                                                   ("bf16", 64, 1, 77, 2, 1.0)])
 def test_backward_matches_the_oracle(dtype, d, B, T, H, g_mean):
+    import gated_deltanet_06_b200 as gdn
     inp = gdn_inputs.make_inputs(B, T, H, d, dtype, g_mean, seed=500 + T)
     rng = np.random.default_rng(T)
     inp["norm_w"] = (1.0 + 0.3 * rng.standard_normal(d)).astype(np.float32)
     dy = _dy((B, T, H, d), 600 + T, dtype)
-    got = _run(inp, dy)
+    got = _run(inp, dy, flags=gdn.FLAG_FORCE_SIMT)
     ref = ob.vjp(inp, dy)
     _check_all(got, ref, f"{dtype} d={d} T={T}")
 
@@ -77,17 +80,19 @@ def test_backward_is_linear_in_dy_and_deterministic_at_the_headline_size():
     # at any size: bitwise repeatability, and linearity in dy (the backward of dy1 + dy2 equals the
     # sum of the two backwards), with an fp32 dy
     import torch
+    import gated_deltanet_06_b200 as gdn
     w = gdn_inputs.HEADLINE
     inp = gdn_inputs.workload_inputs(w)
     dy1 = _dy((w.B, w.T, w.H, w.d), 620, "f32")
     dy2 = _dy((w.B, w.T, w.H, w.d), 621, "f32")
-    g1 = _run(inp, dy1, out_dtype=torch.float32)
-    g1b = _run(inp, dy1, out_dtype=torch.float32)
+    f = gdn.FLAG_FORCE_SIMT
+    g1 = _run(inp, dy1, flags=f, out_dtype=torch.float32)
+    g1b = _run(inp, dy1, flags=f, out_dtype=torch.float32)
     for n in KEY:
         assert np.array_equal(g1[n], g1b[n]), n
         assert np.all(np.isfinite(g1[n])), n
-    g2 = _run(inp, dy2, out_dtype=torch.float32)
-    gs = _run(inp, dy1 + dy2, out_dtype=torch.float32)
+    g2 = _run(inp, dy2, flags=f, out_dtype=torch.float32)
+    gs = _run(inp, dy1 + dy2, flags=f, out_dtype=torch.float32)
     for n in KEY:
         assert rel_l2(gs[n], g1[n] + g2[n]) <= REL_L2_GRAD, n
 

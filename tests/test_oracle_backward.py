@@ -96,3 +96,17 @@ def test_blocked_backward_algebra_equals_the_oracle_backward(T, C):
     for n, m in (("dq", "dqh"), ("dk", "dkh"), ("dv", "dvh"), ("dbeta", "dbeta")):
         np.testing.assert_allclose(got[n], ref[m], rtol=1e-9, atol=1e-11, err_msg=n)
     np.testing.assert_allclose(got["dla"], ref["dalpha"] * tp["alpha"], rtol=1e-9, atol=1e-11, err_msg="dla")
+
+
+@pytest.mark.parametrize("T,C", [(1, 128), (127, 128), (128, 128), (300, 128), (130, 64)])
+def test_kernel_form_backward_equals_the_oracle_backward(T, C):
+    # the block backward as the tensor-core kernels take it (reverse recurrence of dS at block ends,
+    # then each block's gradients from its tiles, S0 and dS alone), against the sequential backward
+    from chunk_model import ut_backward
+    inp, dy = _case(120 + T, T=T, H=2, d=16, g_mean=-0.5)
+    _, tp = ob._tape(inp, ob.DEFAULT_L2_EPS, ob.DEFAULT_NORM_EPS)
+    ref = ob.vjp(inp, dy)
+    got = ut_backward(tp["h_q"], tp["h_k"], tp["s_v"], tp["la"], tp["beta"], ref["do"], C=C)
+    for n, m in (("dq", "dqh"), ("dk", "dkh"), ("dv", "dvh"), ("dbeta", "dbeta")):
+        np.testing.assert_allclose(got[n], ref[m], rtol=1e-9, atol=1e-11, err_msg=n)
+    np.testing.assert_allclose(got["dla"], ref["dalpha"] * tp["alpha"], rtol=1e-9, atol=1e-11, err_msg="dla")
