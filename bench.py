@@ -688,6 +688,9 @@ def main():
         if "bwd_grad" in kms:  # the block-gradient kernel: 16 products of 128 x 128 x 128 per block
             fl = backward_grad_flops(w.B * w.H, -(-w.T // 128))
             bwd["bwd_grad_tflops"] = fl / (kms["bwd_grad"] / 1e3) / 1e12
+            pk = load_peaks()
+            if pk and pk.get("bf16_tflops"):  # fp16 and bf16 run at the same dense rate
+                bwd["bwd_grad_frac_of_tensor_peak"] = bwd["bwd_grad_tflops"] / pk["bf16_tflops"]
         del ws_b, gr, dy
 
     # end to end through the public host-buffer entry point (gdn_forward_host: every input copied from

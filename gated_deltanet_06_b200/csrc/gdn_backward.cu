@@ -141,11 +141,34 @@ __global__ void __launch_bounds__(kBT) gdn_bwd_fwd_rows(const BwdParams p) {
     }
 }
 
+// four consecutive 16-bit or fp32 values as fp32 (8- or 16-byte aligned)
+template <typename InT>
+__device__ __forceinline__ void ld4_in(const InT *src, float (&v)[4]);
+template <>
+__device__ __forceinline__ void ld4_in<float>(const float *src, float (&v)[4]) {
+    const float4 x = *reinterpret_cast<const float4 *>(src);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+}
+template <>
+__device__ __forceinline__ void ld4_in<__nv_bfloat16>(const __nv_bfloat16 *src, float (&v)[4]) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(src);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+}
+template <>
+__device__ __forceinline__ void ld4_in<__half>(const __half *src, float (&v)[4]) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(src);
+    const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&u.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&u.y));
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+}
+
 // ------------------------------------------------------------ output step backwards
 // One warp per (b, t, h) row.  y = o rn w SiLU(z), rn = 1/sqrt(mean(o^2) + eps):
 //   gz = dy w SiLU(z);  do = rn gz - o rn^3 (o . gz) / D;  dz = dy o rn w SiLU'(z);
 //   dw += dy o rn SiLU(z)  (per-CTA partial sums, in a fixed order).
-template <typename ZT, typename YT, int D, bool kF16>
+template <typename ZT, typename YT, int D>
 __global__ void __launch_bounds__(256) gdn_bwd_out(const BwdParams p) {
     constexpr int PER = D / 32;
     __shared__ float sw[8][D];
@@ -190,14 +213,96 @@ __global__ void __launch_bounds__(256) gdn_bwd_out(const BwdParams p) {
         for (int e = 0; e < PER; ++e) {
             const int c = lane * PER + e;
             const float gz = gv[e] * w[e] * sz[e];
-            if constexpr (kF16) p.dO16[(bhr * p.Tp + t) * D + c] = __float2half_rn(rn * gz - ov[e] * k3);
-            else p.dO[(bhr * p.Tp + t) * D + c] = rn * gz - ov[e] * k3;
+            p.dO[(bhr * p.Tp + t) * D + c] = rn * gz - ov[e] * k3;
             p.dz[row * D + c] = gv[e] * ov[e] * rn * w[e] * dsilu(zv[e]);
             dw[e] = fmaf(gv[e] * ov[e] * rn, sz[e], dw[e]);
         }
     }
 #pragma unroll
     for (int e = 0; e < PER; ++e) sw[warp][lane * PER + e] = dw[e];
+    __syncthreads();
+    for (int c = threadIdx.x; c < D; c += 256) {
+        float s = 0.0f;
+        for (int k = 0; k < 8; ++k) s += sw[k][c];
+        p.dnw_part[static_cast<size_t>(blockIdx.x) * D + c] = s;
+    }
+}
+
+// The output step backwards for the tensor-core backward (d = 128, dO in fp16): one warp per
+// (b, t, h) row, lane l on columns 4l .. 4l+3 with 8- and 16-byte loads and stores, two rows per
+// warp step (both rows' loads in flight before either is used), SiLU's sigmoid once per element.
+template <typename ZT, typename YT>
+__global__ void __launch_bounds__(256) gdn_bwd_out_rows(const BwdParams p) {
+    constexpr int D = 128;
+    __shared__ float sw[8][D];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, c0 = lane * 4;
+    const int nrows = p.B * p.T * p.H;  // < 2^31: the plan bounds B * H * Tp
+    float w[4], dw[4];
+    ld4_in<float>(p.norm_w + c0, w);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dw[e] = 0.0f;
+    const ZT *z = static_cast<const ZT *>(p.z);
+    const YT *dy = static_cast<const YT *>(p.dy);
+    const int stride = gridDim.x * 16;
+    for (int r0 = blockIdx.x * 16 + warp * 2; r0 < nrows; r0 += stride) {
+        float ov[2][4], zv[2][4], gv[2][4];
+        int tokv[2], hv[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int row = r0 + i;
+            tokv[i] = row / p.H;
+            hv[i] = row - tokv[i] * p.H;
+            if (row < nrows) {
+                ld4_in<float>(p.o + static_cast<size_t>(row) * D + c0, ov[i]);
+                ld4_in<ZT>(z + static_cast<size_t>(tokv[i]) * p.tok_stride + hv[i] * D + c0, zv[i]);
+                ld4_in<YT>(dy + static_cast<size_t>(row) * D + c0, gv[i]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) ov[i][e] = zv[i][e] = gv[i][e] = 0.0f;
+            }
+        }
+        float ss[2], og[2], sg[2][4], sz[2][4];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            ss[i] = 0.0f;
+            og[i] = 0.0f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                sg[i][e] = __fdividef(1.0f, 1.0f + __expf(-zv[i][e]));
+                sz[i][e] = zv[i][e] * sg[i][e];
+                ss[i] = fmaf(ov[i][e], ov[i][e], ss[i]);
+                og[i] = fmaf(ov[i][e], gv[i][e] * w[e] * sz[i][e], og[i]);
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                ss[i] += __shfl_xor_sync(0xffffffffu, ss[i], off);
+                og[i] += __shfl_xor_sync(0xffffffffu, og[i], off);
+            }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int row = r0 + i;
+            if (row >= nrows) break;
+            const int bb = tokv[i] / p.T, t = tokv[i] - bb * p.T;
+            const float rn = rsqrtf(ss[i] * (1.0f / D) + p.norm_eps);
+            const float k3 = rn * rn * rn * og[i] * (1.0f / D);
+            float d[4], dzv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                d[e] = rn * gv[i][e] * w[e] * sz[i][e] - ov[i][e] * k3;
+                dzv[e] = gv[i][e] * ov[i][e] * rn * w[e] * sg[i][e] * (1.0f + zv[i][e] * (1.0f - sg[i][e]));
+                dw[e] = fmaf(gv[i][e] * ov[i][e] * rn, sz[i][e], dw[e]);
+            }
+            const size_t bhr = static_cast<size_t>(bb) * p.H + hv[i];
+            *reinterpret_cast<uint2 *>(p.dO16 + (bhr * p.Tp + t) * D + c0) =
+                make_uint2(pack_half2(d[0], d[1]), pack_half2(d[2], d[3]));
+            *reinterpret_cast<float4 *>(p.dz + static_cast<size_t>(row) * D + c0) = make_float4(dzv[0], dzv[1], dzv[2], dzv[3]);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sw[warp][c0 + e] = dw[e];
     __syncthreads();
     for (int c = threadIdx.x; c < D; c += 256) {
         float s = 0.0f;
@@ -524,28 +629,6 @@ __global__ void __launch_bounds__(256) gdn_bwd_tokens(const BwdParams p) {
 // dx[t] = sum_k w_k da[t+3-k] and the conv-weight sums (input rows re-read, from L1), reduced over
 // the warps in a fixed order into the tile's partial slot.  Then the gates of the tile's tokens.
 template <typename InT>
-__device__ __forceinline__ void ld4_in(const InT *src, float (&v)[4]);
-template <>
-__device__ __forceinline__ void ld4_in<float>(const float *src, float (&v)[4]) {
-    const float4 x = *reinterpret_cast<const float4 *>(src);
-    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
-}
-template <>
-__device__ __forceinline__ void ld4_in<__nv_bfloat16>(const __nv_bfloat16 *src, float (&v)[4]) {
-    const uint2 u = *reinterpret_cast<const uint2 *>(src);
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
-    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
-}
-template <>
-__device__ __forceinline__ void ld4_in<__half>(const __half *src, float (&v)[4]) {
-    const uint2 u = *reinterpret_cast<const uint2 *>(src);
-    const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&u.x));
-    const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&u.y));
-    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
-}
-
-template <typename InT>
 __global__ void __launch_bounds__(256) gdn_bwd_tokens_rows(const BwdParams p) {
     constexpr int D = 128, NR = kTile + 3;
     __shared__ float4 sda[NR][32];    // da of token t0 + tt, channels 4 lane .. 4 lane + 3
@@ -554,12 +637,12 @@ __global__ void __launch_bounds__(256) gdn_bwd_tokens_rows(const BwdParams p) {
     // per-warp conv-weight sums of channel 4 lane + j, over sda once pass 2 has read it
     float4 (*sdw)[4][32] = reinterpret_cast<float4 (*)[4][32]>(&sda[0][0]);
     static_assert(sizeof(sda) >= 8 * 4 * 32 * sizeof(float4), "the warp sums fit in sda");
-    const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z / 3, which = blockIdx.z % 3;
     const size_t bh = static_cast<size_t>(b) * p.H + h;
     const int t0 = tile * kTile;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, c0 = lane * 4;
     const int ntile = p.Tp / kTile;
-    for (int which = 0; which < 3; ++which) {
+    {
         const InT *x = static_cast<const InT *>(which == 0 ? p.q : (which == 1 ? p.k : p.v));
         const float *wc = which == 0 ? p.conv_q : (which == 1 ? p.conv_k : p.conv_v);
         const float *dh_src = which == 0 ? p.dq_part : (which == 1 ? p.dk_part : p.dvh);
@@ -572,7 +655,6 @@ __global__ void __launch_bounds__(256) gdn_bwd_tokens_rows(const BwdParams p) {
                 v[0] = v[1] = v[2] = v[3] = 0.0f;
             }
         };
-        __syncthreads();  // the previous tensor's reads of swt and of sda (and the warp sums over it) are done
         if (warp < 4) swt[warp][lane] = reinterpret_cast<const float4 *>(wc)[static_cast<size_t>(h) * D + c0 + warp];
         __syncthreads();
         float w[4][4];
@@ -581,15 +663,15 @@ __global__ void __launch_bounds__(256) gdn_bwd_tokens_rows(const BwdParams p) {
             const float4 t4 = swt[j][lane];
             w[j][0] = t4.x; w[j][1] = t4.y; w[j][2] = t4.z; w[j][3] = t4.w;
         }
-        // pass 1: da of tokens t0 .. t0 + 66 (zero past T).  Warp w takes tokens 8w .. 8w+7 (warp 7 also
-        // the 3 after the tile) in runs of 4: the 7 input rows and 4 gradient rows of a run are all
-        // fetched before any is used, and the 4 tokens' reductions are independent.
-        for (int rb = 8 * warp; rb < (warp == 7 ? NR : 8 * warp + 8); rb += 4) {
-            float xr[7][4], dh[4][4];
+        // pass 1: da of tokens t0 .. t0 + 66 (zero past T), in runs of two consecutive tokens taken by the
+        // warps in turn: a run's 5 input rows and 2 gradient rows are fetched before any is used, and
+        // the two tokens' reductions are independent
+        for (int rb = 2 * warp; rb < NR; rb += 16) {
+            float xr[5][4], dh[2][4];
 #pragma unroll
-            for (int k = 0; k < 7; ++k) xrow(t0 + rb - 3 + k, xr[k]);
+            for (int k = 0; k < 5; ++k) xrow(t0 + rb - 3 + k, xr[k]);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < 2; ++i) {
                 const int t = t0 + rb + i;
                 if (t < p.T && rb + i < NR) {
                     ld4_in<float>(dh_src + (bh * p.Tp + t) * D + c0, dh[i]);
@@ -598,9 +680,9 @@ __global__ void __launch_bounds__(256) gdn_bwd_tokens_rows(const BwdParams p) {
                 }
             }
             // sigma(a) once per element (fast exponential and division); SiLU' = sigma (1 + a (1 - sigma))
-            float a[4][4], sg[4][4], sv[4][4], ss[4], pr[4];
+            float a[2][4], sg[2][4], sv[2][4], ss[2], pr[2];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < 2; ++i) {
                 ss[i] = 0.0f;
                 pr[i] = 0.0f;
 #pragma unroll
@@ -617,12 +699,12 @@ __global__ void __launch_bounds__(256) gdn_bwd_tokens_rows(const BwdParams p) {
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
+                    for (int i = 0; i < 2; ++i) {
                         ss[i] += __shfl_xor_sync(0xffffffffu, ss[i], off);
                         pr[i] += __shfl_xor_sync(0xffffffffu, pr[i], off);
                     }
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
+                for (int i = 0; i < 2; ++i) {
                     const float inv = rsqrtf(ss[i] + p.l2_eps);
                     const float k2 = inv * inv * pr[i];
 #pragma unroll
@@ -630,7 +712,7 @@ __global__ void __launch_bounds__(256) gdn_bwd_tokens_rows(const BwdParams p) {
                 }
             }
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < 2; ++i) {
                 const int t = t0 + rb + i;
                 if (rb + i < NR) {
                     float da[4];
@@ -685,7 +767,9 @@ __global__ void __launch_bounds__(256) gdn_bwd_tokens_rows(const BwdParams p) {
         }
     }
 
-    // gates: log alpha = -exp(A_log) softplus(g + dt_bias), beta = sigmoid(b); d log alpha is given
+    // gates (the q CTA of the tile): log alpha = -exp(A_log) softplus(g + dt_bias), beta = sigmoid(b);
+    // d log alpha is given
+    if (which != 0) return;
     float dla_la = 0.0f, dgv = 0.0f;
     if (threadIdx.x < kTile) {
         const int t = t0 + threadIdx.x;
@@ -766,9 +850,9 @@ __global__ void __launch_bounds__(256) gdn_bwd_params_split(const BwdParams p, i
 
 template <typename ZT, typename YT>
 cudaError_t launch_out_bwd(const BwdParams &p, int blocks, cudaStream_t s) {
-    if (p.dO16) gdn_bwd_out<ZT, YT, 128, true><<<blocks, 256, 0, s>>>(p);
-    else if (p.d == 128) gdn_bwd_out<ZT, YT, 128, false><<<blocks, 256, 0, s>>>(p);
-    else gdn_bwd_out<ZT, YT, 64, false><<<blocks, 256, 0, s>>>(p);
+    if (p.dO16) gdn_bwd_out_rows<ZT, YT><<<blocks, 256, 0, s>>>(p);
+    else if (p.d == 128) gdn_bwd_out<ZT, YT, 128><<<blocks, 256, 0, s>>>(p);
+    else gdn_bwd_out<ZT, YT, 64><<<blocks, 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 template <typename ZT>
@@ -807,7 +891,7 @@ cudaError_t launch_bwd_out(const BwdParams &p, InType in, InType out, cudaStream
 
 cudaError_t launch_bwd_tokens(const BwdParams &p, InType in, cudaStream_t s) {
     if (p.tc && p.d == 128) {  // whole per-token gradients: one warp per row
-        const dim3 grid(p.Tp / kTile, p.H, p.B);
+        const dim3 grid(p.Tp / kTile, p.H, p.B * 3);  // one CTA per (tile, head, sequence, tensor)
         if (in == InType::BF16) gdn_bwd_tokens_rows<__nv_bfloat16><<<grid, 256, 0, s>>>(p);
         else if (in == InType::F16) gdn_bwd_tokens_rows<__half><<<grid, 256, 0, s>>>(p);
         else gdn_bwd_tokens_rows<float><<<grid, 256, 0, s>>>(p);
@@ -826,7 +910,7 @@ cudaError_t launch_bwd_params(const BwdParams &p, cudaStream_t s) {
 
 int bwd_out_blocks(long long rows) {
     long long blocks = (rows + 7) / 8;
-    return static_cast<int>(blocks < 1024 ? blocks : 1024);
+    return static_cast<int>(blocks < 4096 ? blocks : 4096);
 }
 
 cudaError_t launch_backward(const BwdParams &p, InType in, InType out, cudaStream_t s, int *launches,

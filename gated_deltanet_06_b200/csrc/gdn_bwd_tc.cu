@@ -56,20 +56,6 @@ __device__ __forceinline__ void put_h32(uint8_t *tile, int r, int col, const flo
     }
 }
 
-// 64 fp16 values (128 contiguous bytes of global memory) kept packed, for use after a wait
-__device__ __forceinline__ void pf_h64(const __half *src, uint4 (&u)[8]) {
-    const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) u[k] = s4[k];
-}
-// element e (0..31, a compile-time index) of the 32-column chunk ch of a packed row
-__device__ __forceinline__ float hsel(const uint4 (&u)[8], int ch, int e) {
-    const uint4 v = ch ? u[4 + (e >> 3)] : u[e >> 3];
-    const int wi = (e & 7) >> 1;
-    const uint32_t w = wi == 0 ? v.x : (wi == 1 ? v.y : (wi == 2 ? v.z : v.w));
-    const float2 f = unpack_half2(w);
-    return (e & 1) ? f.y : f.x;
-}
 // 8 fp16 values (16-byte chunk c16 of row r of a 128-row panel tile) as fp32
 __device__ __forceinline__ void tile_h8(const uint8_t *tile, int r, int c16, float (&f)[8]) {
     const uint4 v = *reinterpret_cast<const uint4 *>(tile + tile_off(128, r, c16));
@@ -117,13 +103,18 @@ __device__ __forceinline__ uint64_t kdesc(uint32_t base, int kk) {
 }
 __device__ __forceinline__ uint64_t mdesc(uint32_t base, int kk) { return sdesc_sw128(base + kk * 2048, 16384, 1024); }
 
-// D (+)= A B over K = 128: eight 16-wide steps; accumulate = false overwrites D on the first step
+// D (+)= A B over K = 128: eight 16-wide steps; accumulate = false overwrites D on the first step.
+// A step's descriptor is the first one with the step's byte offset / 16 added to its address field
+// (no carry out of it: shared-memory addresses stay below 256 KB).
 __device__ __forceinline__ void gemm128(uint32_t d, uint32_t a, bool a_mn, uint32_t b, bool b_mn, bool accumulate) {
     const uint32_t id = idesc_f16_f32(128, 128, a_mn, b_mn);
-#pragma unroll 1  // (descriptors formed per step: unrolled, the producer's many products would hoist them all)
-    for (int kk = 0; kk < 8; ++kk)
-        umma_f16(d, a_mn ? mdesc(a, kk) : kdesc(a, kk), b_mn ? mdesc(b, kk) : kdesc(b, kk), id,
-                 (accumulate || kk > 0) ? 1u : 0u);
+    const uint64_t da = a_mn ? mdesc(a, 0) : kdesc(a, 0), db = b_mn ? mdesc(b, 0) : kdesc(b, 0);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t ka = a_mn ? kk * 2048 : (kk >> 2) * 16384 + (kk & 3) * 32;
+        const uint32_t kb = b_mn ? kk * 2048 : (kk >> 2) * 16384 + (kk & 3) * 32;
+        umma_f16(d, da + (ka >> 4), db + (kb >> 4), id, (accumulate || kk > 0) ? 1u : 0u);
+    }
 }
 
 // ============================================================ reverse scan of dS
@@ -353,22 +344,41 @@ __global__ void __launch_bounds__(bs::kThreads, 1)
 
 // ============================================================ local gradients of every block
 namespace bg {
-constexpr int kThreads = 288;  // warps 0-7: epilogues (TMEM lane quarter w & 3, column half w >> 2); warp 8: loads, MMAs
-constexpr uint32_t SLOT = 32768;  // six 128 x 128 fp16 tile slots
+// 16 warps: TMEM lane quarter w & 3, 32-column quarter w >> 2 of every accumulator.  Thread 0 also
+// issues the TMA loads and the tensor-core products, each phase's after the barrier that ends the
+// previous epilogue (so there is no separate producer warp, and 128 registers per thread).
+constexpr int kThreads = 512;
+constexpr uint32_t SLOT = 32768;                 // six 128 x 128 fp16 tile slots
 constexpr uint32_t OFF_G = 6 * SLOT;             // fp32 [128]: G of the block
 constexpr uint32_t OFF_COL = OFF_G + 512;        // fp32 [4][128]: column sums over each lane quarter's rows
-constexpr uint32_t OFF_X = OFF_COL + 2048;       // fp32 [3][128]: row partials of column half 1
-constexpr uint32_t OFF_WS = OFF_X + 1536;        // fp32 [8][2]: per-warp sums; [4] suffix-scan totals
-constexpr uint32_t OFF_BAR = OFF_WS + 128;
-enum { FULL0 = 0, MMA_A = 6, MMA_B, MMA_C, MMA_D, MMA_E, CONS_A, CONS_B, CONS_C, CONS_D, CONS_E, NBAR };
+constexpr uint32_t OFF_X = OFF_COL + 2048;       // fp32 [3][4][128]: row partials of column quarters 1-3
+constexpr uint32_t OFF_WS = OFF_X + 6144;        // fp32 [16][2] per-warp sums, [4] suffix-scan totals
+constexpr uint32_t OFF_CNT = OFF_WS + 256;       // int [6] loads per slot, [11] phases per barrier (thread 0)
+constexpr uint32_t OFF_BAR = OFF_CNT + 128;
+enum { FULL0 = 0, MMA_A = 6, MMA_B, MMA_C, MMA_D, MMA_E, NBAR };
 constexpr uint32_t SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
 constexpr uint32_t TM0 = 0, TM1 = 128, TM2 = 256, TM3 = 384;
 }  // namespace bg
 
+// 32 fp16 values (64 contiguous bytes of global memory) kept packed, for use after a wait
+__device__ __forceinline__ void pf_h32(const __half *src, uint4 (&u)[4]) {
+    const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) u[k] = s4[k];
+}
+// element e (a compile-time index) of a packed 32-value row
+__device__ __forceinline__ float hget(const uint4 (&u)[4], int e) {
+    const uint4 v = u[e >> 3];
+    const int wi = (e & 7) >> 1;
+    const uint32_t w = wi == 0 ? v.x : (wi == 1 ? v.y : (wi == 2 ? v.z : v.w));
+    const float2 f = unpack_half2(w);
+    return (e & 1) ? f.y : f.x;
+}
+
 // Slot use per block (s0 .. s5), tile loaded by TMA or written by the epilogue (E*):
 //   phase A: S0^T s0, W s1, dO s2, P s3, Kt s4, dS^T s5   -> A3 dO S0 (TM2), A1 W S0^T (TM0),
 //                                                           A2 P^T dO + Kt dS^T (TM1)
-//   EA: Delta -> s3, dDelta -> s4, TM2 *= E;  K -> s1
+//   EA: Delta -> s3, dDelta -> s4, TM2 *= E;  then K -> s1
 //   phase B: B1 dO Delta^T (TM0), B2 Delta dS (TM3), B3 dDelta S0 (TM1)
 //   EB: dQK -> s3, dW -> s5, TM3 = e^(G_last - G) o TM3;  Q -> s0, T -> s2
 //   phase C: C1 TM2 += dQK K, C2 TM3 += dQK^T Q, C3 T^T dW (TM0), C4 T^T dDelta (TM1)
@@ -391,7 +401,7 @@ __global__ void __launch_bounds__(bg::kThreads, 1)
     const int total = p.BH * p.NB;
 
     if (tid == 0) {
-        for (int i = 0; i < NBAR; ++i) mbar_init(&bars[i], i >= CONS_A ? 8 : 1);
+        for (int i = 0; i < NBAR; ++i) mbar_init(&bars[i], 1);
         ab->flag = 0;
         fence_mbar_init();
     }
@@ -406,368 +416,342 @@ __global__ void __launch_bounds__(bg::kThreads, 1)
     const uint32_t tmem = *tmem_slot;
     pdl_wait();  // dS^T at every block end is complete
 
-    if (warp == 8) {
+    // thread 0's loads and products; its counters live in shared memory, not in every thread's registers
+    int *nld = reinterpret_cast<int *>(sm + OFF_CNT);  // loads issued into each slot
+    int *started = nld + 6;                            // phases started on every barrier (for the drain)
+    if (tid == 0)
+        for (int k = 0; k < 6 + NBAR; ++k) nld[k] = 0;
+    auto load = [&](int slot, const CUtensorMap *map, int w) {
+        const int y = (w / p.NB) * p.Tp + (w % p.NB) * kBlk;
+        uint64_t *bar = &bars[FULL0 + slot];
+        mbar_arrive_expect_tx(bar, SLOT);
+        tma_load_2d(sm + slot * SLOT, map, bar, 0, y);
+        tma_load_2d(sm + slot * SLOT + 16384, map, bar, 64, y);
+        ++nld[slot];
+        ++started[FULL0 + slot];
+    };
+    auto ready = [&](int slot) { return mbar_wait(&bars[FULL0 + slot], (nld[slot] - 1) & 1, ab, p.status, lim); };
+    auto commit = [&](int b) {
+        umma_commit(&bars[b]);
+        ++started[b];
+    };
+    // the slots' addresses, re-formed wherever products are issued (an opaque copy of the base) so that
+    // the descriptors of the block's 16 products are not all kept live across the loop
+    uint32_t s0, s1, s2, s3, s4, s5;
+    auto slots = [&]() {
+        uint32_t b;
+        asm volatile("mov.b32 %0, %1;" : "=r"(b) : "r"(sbase));
+        s0 = b; s1 = b + SLOT; s2 = b + 2 * SLOT; s3 = b + 3 * SLOT; s4 = b + 4 * SLOT; s5 = b + 5 * SLOT;
+    };
+
+    const int q = warp & 3, cq = warp >> 2;
+    const int r = q * 32 + lane;  // the block row (token) this thread owns, columns cb .. cb + 31
+    const int cb = cq * 32;
+    const uint32_t lb = tmem + (static_cast<uint32_t>(q * 32) << 16) + cb;
+    float *sG = reinterpret_cast<float *>(sm + OFF_G);
+    float *colpart = reinterpret_cast<float *>(sm + OFF_COL);
+    float *xch = reinterpret_cast<float *>(sm + OFF_X);
+    float *wsum = reinterpret_cast<float *>(sm + OFF_WS);
+    uint8_t *t3 = sm + 3 * SLOT, *t4 = sm + 4 * SLOT, *t5 = sm + 5 * SLOT;
+    const bool issuer = tid == 0;
+    // after an epilogue: its shared-memory tiles visible to the tensor cores and its TMEM accesses
+    // ordered before the next products, for the issuing thread
+    auto end_phase = [&]() {
+        tmem_st_wait();
+        fence_proxy_async();
+        tc_fence_before();
+        named_sync(2, kThreads);
+        if (issuer) tc_fence_after();
+    };
+
+    if (issuer && blockIdx.x < total) {
+        const int w = blockIdx.x;
+        load(0, &m.S0, w);
+        load(1, &m.W, w);
+        load(2, &m.dO, w);
+        load(3, &m.Aqk, w);
+        load(4, &m.Kt, w);
+        load(5, &m.dS, w);
+    }
+    for (int w = blockIdx.x, i = 0; w < total; w += gridDim.x, ++i) {
+        const uint32_t ph = i & 1;
+        const int wn = w + gridDim.x;
+        const int bh = w / p.NB, c = w % p.NB;
+        const size_t row0 = static_cast<size_t>(bh) * p.Tp + static_cast<size_t>(c) * kBlk;
+        const size_t grow = row0 + r;
+        const size_t gel = grow * 128 + cb;  // element offset of this thread's columns in [BH][Tp][128]
+        const float Gr = p.G[grow], be = p.beta[grow], gL = p.G[row0 + kBlk - 1];
+        const float Er = __expf(Gr), fr = __expf(fminf(gL - Gr, 0.0f)), eC = __expf(gL);
+        if (cq == 0) sG[r] = Gr;
+        float dG = 0.0f, dbeta = 0.0f, dE = 0.0f, sdot = 0.0f, sdgc = 0.0f;
+        uint4 pa[4], pb[4];
+        pf_h32(p.U + gel, pa);
+        pf_h32(p.Q + gel, pb);
+
+        // ---- phase A (the previous block's epilogues have read TM0-TM2)
+        if (issuer && ready(0) && ready(1) && ready(2) && ready(3) && ready(4) && ready(5)) {
+            tc_fence_after();
+            slots();
+            gemm128(tmem + TM2, s2, false, s0, false, false);  // A3: dO S0 (B = S0^T read K-major)
+            gemm128(tmem + TM0, s1, false, s0, true, false);   // A1: W S0^T (B = S0^T MN-major)
+            gemm128(tmem + TM1, s3, true, s2, true, false);    // A2: P^T dO
+            gemm128(tmem + TM1, s4, false, s5, true, true);    //     + Kt dS^T
+            commit(MMA_A);
+        }
+        // ---- EA: Delta = U - W S0^T -> s3;  dDelta -> s4;  TM2 = E o dO S0, rowsum(dO S0 o Q);  <dS, S0>
+        //      (U and Q rows fetched before the wait; S0^T and dS^T rows from their tiles)
+        bool ok = warp_wait_all(&bars[MMA_A], ph, ab, p.status, lim) &&
+                  warp_wait_all(&bars[FULL0 + 0], ph, ab, p.status, lim) &&  // S0^T: load 3i of slot 0
+                  warp_wait_all(&bars[FULL0 + 5], ph, ab, p.status, lim);    // dS^T: load i of slot 5
+        if (!group_all(1, kThreads, ok)) break;
+        tc_fence_after();
+        {
+            float x[32];
+            tmem_ld32(lb + TM0, x);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] = hget(pa, e) - x[e];
+            put_h32(t3, r, cb, x);
+            tmem_ld32(lb + TM1, x);
+            put_h32(t4, r, cb, x);
+            tmem_ld32(lb + TM2, x);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                dE = fmaf(x[e], hget(pb, e), dE);
+                x[e] *= Er;
+            }
+            tmem_st32(lb + TM2, x);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float d8[8], s8[8];
+                tile_h8(sm + 5 * SLOT, r, cb / 8 + k, d8);
+                tile_h8(sm, r, cb / 8 + k, s8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) sdot = fmaf(d8[e], s8[e], sdot);
+            }
+        }
+        pf_h32(p.Aqk + gel, pa);  // the P row EB reads, fetched while the products of phase B run
+        end_phase();
+        if (issuer) {  // ---- phase B (TM3 was read in the previous block's EE)
+            slots();
+            load(1, &m.K, w);
+            gemm128(tmem + TM0, s2, false, s3, false, false);  // B1: dO Delta^T
+            gemm128(tmem + TM3, s3, false, s5, false, false);  // B2: Delta dS (B = dS^T read K-major)
+            gemm128(tmem + TM1, s4, false, s0, false, false);  // B3: dDelta S0
+            commit(MMA_B);
+        }
+
+        // ---- EB: TM3 = e^(G_last - G) o dKd, rowsum(dKd o Kt) (= e^(G_last - G_r) rowsum(dKd o K), K from
+        //      its tile: load 2i + 1 of slot 1);  dW = -dDelta S0 -> s5;  dQK = dP o Gam -> s3, rowsum /
+        //      colsum of dP o P
+        ok = warp_wait_all(&bars[MMA_B], ph, ab, p.status, lim) && warp_wait_all(&bars[FULL0 + 1], 1, ab, p.status, lim);
+        if (!group_all(1, kThreads, ok)) break;
+        tc_fence_after();
+        if (issuer) {  // S0^T and dO have their last readers behind them
+            load(0, &m.Q, w);
+            load(2, &m.T, w);
+        }
+        {
+            float x[32], v[32];
+            float t = 0.0f;
+            tmem_ld32(lb + TM3, x);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float k8[8];
+                tile_h8(sm + SLOT, r, cb / 8 + k, k8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    t = fmaf(x[8 * k + e], k8[e], t);
+                    x[8 * k + e] *= fr;
+                }
+            }
+            tmem_st32(lb + TM3, x);
+            tmem_ld32(lb + TM1, x);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] = -x[e];
+            put_h32(t5, r, cb, x);
+            float rs = 0.0f;
+            tmem_ld32(lb + TM0, x);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int j = cb + e;
+                const float dpp = x[e] * hget(pa, e);
+                v[e] = dpp;
+                rs += dpp;
+                x[e] = (j <= r) ? x[e] * __expf(Gr - sG[j]) : 0.0f;
+            }
+            put_h32(t3, r, cb, x);
+            colpart[q * 128 + cb + lane] = colsum32(v, lane);
+            t *= fr;
+            dG += rs - t;
+            sdgc += t;
+        }
+        pf_h32(p.V + gel, pa);  // the V row EC reads
+        end_phase();
+        if (issuer && ready(0) && ready(1) && ready(2)) {  // ---- phase C
+            slots();
+            gemm128(tmem + TM2, s3, false, s1, true, true);    // C1: dQ += dQK K
+            gemm128(tmem + TM3, s3, true, s0, true, true);     // C2: dK += dQK^T Q
+            gemm128(tmem + TM0, s2, true, s5, true, false);    // C3: dKb = T^T dW
+            gemm128(tmem + TM1, s2, true, s4, true, false);    // C4: dVb = T^T dDelta
+            commit(MMA_C);
+        }
+
+        // ---- EC: dQ out;  dKb -> s3, TM3 += diag(beta E) dKb, rowsum(dKb o K);  dVb -> s4,
+        //      dv^ = beta dVb out, rowsum(dVb o V)
+        if (!group_all(1, kThreads, warp_wait_all(&bars[MMA_C], ph, ab, p.status, lim))) break;
+        tc_fence_after();
+        if (issuer) {  // Q and T have their last readers behind them
+            load(0, &m.W, w);
+            load(2, &m.U, w);
+        }
+        {
+            float x[32], u[32];
+            float tk = 0.0f, tv = 0.0f;
+            tmem_ld32(lb + TM2, x);
+            st_f32(p.dqh + gel, x, 1.0f);
+            tmem_ld32(lb + TM0, x);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float k8[8];
+                tile_h8(sm + SLOT, r, cb / 8 + k, k8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) tk = fmaf(x[8 * k + e], k8[e], tk);
+            }
+            tmem_ld32(lb + TM3, u);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) u[e] = fmaf(be * Er, x[e], u[e]);
+            tmem_st32(lb + TM3, u);
+            put_h32(t3, r, cb, x);
+            tmem_ld32(lb + TM1, x);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) tv = fmaf(x[e], hget(pa, e), tv);
+            st_f32(p.dvh + gel, x, be);
+            put_h32(t4, r, cb, x);
+            dbeta = fmaf(Er, tk, dbeta) + tv;
+            dE = fmaf(be, tk, dE);
+        }
+        end_phase();
+        if (issuer && ready(0) && ready(2)) {  // ---- phase D
+            slots();
+            gemm128(tmem + TM0, s3, false, s0, false, false);  // D1: dKb W^T
+            gemm128(tmem + TM0, s4, false, s2, false, true);   //     + dVb U^T
+            gemm128(tmem + TM1, s1, false, s1, false, false);  // D2: K K^T
+            commit(MMA_D);
+        }
+
+        // ---- ED: dL = -(dKb W^T + dVb U^T) below the diagonal, A = K K^T: dA = beta dL o Gam -> s5,
+        //      rowsum(dL o Gam o A) into dbeta, rowsum / colsum of dLL = beta dL o Gam o A
+        if (!group_all(1, kThreads, warp_wait_all(&bars[MMA_D], ph, ab, p.status, lim))) break;
+        tc_fence_after();
+        if (issuer && wn < total) {  // the next block's tiles into the slots phase D has freed
+            const int yn = (wn / p.NB) * p.Tp + (wn % p.NB) * kBlk;
+            for (int hf = 0; hf < 2; ++hf) {  // and, into L2, the rows its epilogues read from global memory
+                tma_prefetch_2d(&m.U, hf * 64, yn);  // and the two tiles loaded after this block's last products
+                tma_prefetch_2d(&m.Q, hf * 64, yn);
+                tma_prefetch_2d(&m.V, hf * 64, yn);
+                tma_prefetch_2d(&m.W, hf * 64, yn);
+                tma_prefetch_2d(&m.dS, hf * 64, yn);
+            }
+            load(0, &m.S0, wn);
+            load(2, &m.dO, wn);
+            load(3, &m.Aqk, wn);
+            load(4, &m.Kt, wn);
+        }
+        {
+            float mv[32], a[32];
+            float rs = 0.0f, db = 0.0f;
+            tmem_ld32(lb + TM0, mv);
+            tmem_ld32(lb + TM1, a);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int j = cb + e;
+                if (j < r) {
+                    const float gs = __expf(Gr - sG[j]);
+                    const float dl = -mv[e];
+                    const float dlga = dl * gs * a[e];
+                    db += dlga;
+                    a[e] = be * dlga;  // dLL
+                    rs += a[e];
+                    mv[e] = be * dl * gs;  // dA
+                } else {
+                    a[e] = 0.0f;
+                    mv[e] = 0.0f;
+                }
+            }
+            put_h32(t5, r, cb, mv);
+            colpart[q * 128 + cb + lane] += colsum32(a, lane);
+            dbeta += db;
+            dG += rs;
+        }
+        end_phase();
+        if (issuer) {  // ---- phase E
+            slots();
+            gemm128(tmem + TM3, s5, false, s1, true, true);    // E1: dK += dA K
+            gemm128(tmem + TM3, s5, true, s1, true, true);     //     + dA^T K
+            commit(MMA_E);
+        }
+
+        // ---- EE: dk^ out; the row sums of the four column quarters, the column sums, d log alpha
+        if (!group_all(1, kThreads, warp_wait_all(&bars[MMA_E], ph, ab, p.status, lim))) break;
+        tc_fence_after();
+        if (issuer && wn < total) {  // K and dA have their last readers behind them
+            load(1, &m.W, wn);
+            load(5, &m.dS, wn);
+        }
+        {
+            float x[32];
+            tmem_ld32(lb + TM3, x);
+            st_f32(p.dkh + gel, x, 1.0f);
+        }
+        if (cq > 0) {
+            xch[(0 * 4 + cq) * 128 + r] = dG;
+            xch[(1 * 4 + cq) * 128 + r] = dbeta;
+            xch[(2 * 4 + cq) * 128 + r] = dE;
+        }
+        sdot = warp_sum(sdot);
+        sdgc = warp_sum(sdgc);
         if (lane == 0) {
-            int nld[6] = {};             // loads issued into each slot
-            int started[CONS_A] = {};    // phases started on FULL0..5 and MMA_A..E (for the drain)
-            auto load = [&](int slot, const CUtensorMap *map, int w) {
-                const int y = (w / p.NB) * p.Tp + (w % p.NB) * kBlk;
-                uint64_t *bar = &bars[FULL0 + slot];
-                mbar_arrive_expect_tx(bar, SLOT);
-                tma_load_2d(sm + slot * SLOT, map, bar, 0, y);
-                tma_load_2d(sm + slot * SLOT + 16384, map, bar, 64, y);
-                ++nld[slot];
-                ++started[FULL0 + slot];
-            };
-            auto ready = [&](int slot) { return mbar_wait(&bars[FULL0 + slot], (nld[slot] - 1) & 1, ab, p.status, lim); };
-            auto commit = [&](int b) {
-                umma_commit(&bars[b]);
-                ++started[b];
-            };
-            const uint32_t s0 = sbase, s1 = sbase + SLOT, s2 = sbase + 2 * SLOT, s3 = sbase + 3 * SLOT,
-                           s4 = sbase + 4 * SLOT, s5 = sbase + 5 * SLOT;
-            int w = blockIdx.x;
-            if (w < total) {
-                load(0, &m.S0, w);
-                load(1, &m.W, w);
-                load(2, &m.dO, w);
-                load(3, &m.Aqk, w);
-                load(4, &m.Kt, w);
-                load(5, &m.dS, w);
-            }
-            bool ok = true;
-            for (int i = 0; ok && w < total; w += gridDim.x, ++i) {
-                const uint32_t ph = i & 1;
-                const int wn = w + gridDim.x;
-                // ---- phase A (TM0, TM1 were read out in the previous block's ED, TM2 in its EC)
-                ok = ready(0) && ready(1) && ready(2) && ready(3) && ready(4) && ready(5);
-                if (!ok) break;
-                tc_fence_after();
-                gemm128(tmem + TM2, s2, false, s0, false, false);  // A3: dO S0 (B = S0^T read K-major)
-                gemm128(tmem + TM0, s1, false, s0, true, false);   // A1: W S0^T (B = S0^T MN-major)
-                gemm128(tmem + TM1, s3, true, s2, true, false);    // A2: P^T dO
-                gemm128(tmem + TM1, s4, false, s5, true, true);    //     + Kt dS^T
-                commit(MMA_A);
-                ok = mbar_wait(&bars[MMA_A], ph, ab, p.status, lim);
-                if (!ok) break;
-                load(1, &m.K, w);
-                // ---- phase B (TM3 was read out in the previous block's EE)
-                ok = mbar_wait(&bars[CONS_A], ph, ab, p.status, lim) &&
-                     (i == 0 || mbar_wait(&bars[CONS_E], ph ^ 1, ab, p.status, lim));
-                if (!ok) break;
-                tc_fence_after();
-                gemm128(tmem + TM0, s2, false, s3, false, false);  // B1: dO Delta^T
-                gemm128(tmem + TM3, s3, false, s5, false, false);  // B2: Delta dS (B = dS^T read K-major)
-                gemm128(tmem + TM1, s4, false, s0, false, false);  // B3: dDelta S0
-                commit(MMA_B);
-                ok = mbar_wait(&bars[MMA_B], ph, ab, p.status, lim);
-                if (!ok) break;
-                load(0, &m.Q, w);
-                load(2, &m.T, w);
-                // ---- phase C
-                ok = mbar_wait(&bars[CONS_B], ph, ab, p.status, lim) && ready(0) && ready(1) && ready(2);
-                if (!ok) break;
-                tc_fence_after();
-                gemm128(tmem + TM2, s3, false, s1, true, true);    // C1: dQ += dQK K
-                gemm128(tmem + TM3, s3, true, s0, true, true);     // C2: dK += dQK^T Q
-                gemm128(tmem + TM0, s2, true, s5, true, false);    // C3: dKb = T^T dW
-                gemm128(tmem + TM1, s2, true, s4, true, false);    // C4: dVb = T^T dDelta
-                commit(MMA_C);
-                ok = mbar_wait(&bars[MMA_C], ph, ab, p.status, lim);
-                if (!ok) break;
-                load(0, &m.W, w);
-                load(2, &m.U, w);
-                // ---- phase D
-                ok = mbar_wait(&bars[CONS_C], ph, ab, p.status, lim) && ready(0) && ready(2);
-                if (!ok) break;
-                tc_fence_after();
-                gemm128(tmem + TM0, s3, false, s0, false, false);  // D1: dKb W^T
-                gemm128(tmem + TM0, s4, false, s2, false, true);   //     + dVb U^T
-                gemm128(tmem + TM1, s1, false, s1, false, false);  // D2: K K^T
-                commit(MMA_D);
-                ok = mbar_wait(&bars[MMA_D], ph, ab, p.status, lim);
-                if (!ok) break;
-                if (wn < total) {
-                    const int yn = (wn / p.NB) * p.Tp + (wn % p.NB) * kBlk;
-                    for (int hf = 0; hf < 2; ++hf) {  // rows the next block's epilogues read from global memory
-                        tma_prefetch_2d(&m.U, hf * 64, yn);
-                        tma_prefetch_2d(&m.Q, hf * 64, yn);
-                        tma_prefetch_2d(&m.V, hf * 64, yn);
-                    }
-                    load(0, &m.S0, wn);
-                    load(2, &m.dO, wn);
-                    load(3, &m.Aqk, wn);
-                    load(4, &m.Kt, wn);
-                }
-                // ---- phase E
-                ok = mbar_wait(&bars[CONS_D], ph, ab, p.status, lim);
-                if (!ok) break;
-                tc_fence_after();
-                gemm128(tmem + TM3, s5, false, s1, true, true);    // E1: dK += dA K
-                gemm128(tmem + TM3, s5, true, s1, true, true);     //     + dA^T K
-                commit(MMA_E);
-                ok = mbar_wait(&bars[MMA_E], ph, ab, p.status, lim);
-                if (!ok) break;
-                if (wn < total) {
-                    load(1, &m.W, wn);
-                    load(5, &m.dS, wn);
-                }
-            }
-#pragma unroll
-            for (int kb = 0; kb < CONS_A; ++kb)
-                if (started[kb] > 0) mbar_wait_drain(&bars[kb], (started[kb] - 1) & 1, lim);
+            wsum[2 * warp] = sdot;
+            wsum[2 * warp + 1] = sdgc;
         }
-    } else {
-        // ------------------------------------------------------------ epilogues
-        const int q = warp & 3, hf = warp >> 2;
-        const int r = q * 32 + lane;  // the block row (token) this thread owns, columns cb .. cb + 63
-        const int cb = hf * 64;
-        const uint32_t lb = tmem + (static_cast<uint32_t>(q * 32) << 16) + cb;
-        float *sG = reinterpret_cast<float *>(sm + OFF_G);
-        float *colpart = reinterpret_cast<float *>(sm + OFF_COL);
-        float *xch = reinterpret_cast<float *>(sm + OFF_X);
-        float *wsum = reinterpret_cast<float *>(sm + OFF_WS);
-        uint8_t *t3 = sm + 3 * SLOT, *t4 = sm + 4 * SLOT, *t5 = sm + 5 * SLOT;
-        auto arrive = [&](int b) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[b]);
-        };
-        for (int w = blockIdx.x, i = 0; w < total; w += gridDim.x, ++i) {
-            const uint32_t ph = i & 1;
-            const int bh = w / p.NB, c = w % p.NB;
-            const size_t row0 = static_cast<size_t>(bh) * p.Tp + static_cast<size_t>(c) * kBlk;
-            const size_t grow = row0 + r;
-            const size_t gel = grow * 128 + cb;  // element offset of this thread's columns in [BH][Tp][128]
-            const float Gr = p.G[grow], be = p.beta[grow], gL = p.G[row0 + kBlk - 1];
-            const float Er = __expf(Gr), fr = __expf(fminf(gL - Gr, 0.0f)), eC = __expf(gL);
-            if (hf == 0) sG[r] = Gr;
-            float dG = 0.0f, dbeta = 0.0f, dE = 0.0f, sdot = 0.0f, sdgc = 0.0f;
-
-            // ---- EA: Delta = U - W S0^T -> s3;  dDelta -> s4;  TM2 = E o dO S0, rowsum(dO S0 o Q);  <dS, S0>
-            //      (U and Q rows fetched before the wait; S0^T and dS^T rows from their tiles)
-            uint4 pa[8], pb[8];
-            pf_h64(p.U + gel, pa);
-            pf_h64(p.Q + gel, pb);
-            bool ok = warp_wait_all(&bars[MMA_A], ph, ab, p.status, lim) &&
-                      warp_wait_all(&bars[FULL0 + 0], ph, ab, p.status, lim) &&  // S0^T: load 3i of slot 0
-                      warp_wait_all(&bars[FULL0 + 5], ph, ab, p.status, lim);    // dS^T: load i of slot 5
-            if (!group_all(1, 256, ok)) break;
-            tc_fence_after();
-#pragma unroll 1
-            for (int ch = 0; ch < 2; ++ch) {
-                const int col = cb + ch * 32;
-                float x[32];
-                tmem_ld32(lb + TM0 + ch * 32, x);
+        tc_fence_before();
+        named_sync(2, kThreads);
+        if (cq == 0) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) x[e] = hsel(pa, ch, e) - x[e];
-                put_h32(t3, r, col, x);
-                tmem_ld32(lb + TM1 + ch * 32, x);
-                put_h32(t4, r, col, x);
-                tmem_ld32(lb + TM2 + ch * 32, x);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    dE = fmaf(x[e], hsel(pb, ch, e), dE);
-                    x[e] *= Er;
-                }
-                tmem_st32(lb + TM2 + ch * 32, x);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    float d8[8], s8[8];
-                    tile_h8(sm + 5 * SLOT, r, col / 8 + k, d8);
-                    tile_h8(sm, r, col / 8 + k, s8);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) sdot = fmaf(d8[e], s8[e], sdot);
-                }
+            for (int k = 1; k < 4; ++k) {
+                dG += xch[(0 * 4 + k) * 128 + r];
+                dbeta += xch[(1 * 4 + k) * 128 + r];
+                dE += xch[(2 * 4 + k) * 128 + r];
             }
-            // the P row EB reads, fetched while the products of phase B run
-            pf_h64(p.Aqk + gel, pa);
-            tmem_st_wait();
-            fence_proxy_async();
-            named_sync(2, 256);  // sG complete
-            arrive(CONS_A);
-
-            // ---- EB: dQK = dP o Gam -> s3, rowsum / colsum of dP o P;  TM3 = e^(G_last - G) o dKd,
-            //      rowsum(dKd o Kt);  dW = -dDelta S0 -> s5
-            //      (sum(dKd o Kt) = e^(G_last - G_r) sum(dKd o K), K from its tile: load 2i + 1 of slot 1)
-            ok = warp_wait_all(&bars[MMA_B], ph, ab, p.status, lim) &&
-                 warp_wait_all(&bars[FULL0 + 1], 1, ab, p.status, lim);
-            if (!group_all(1, 256, ok)) break;
-            tc_fence_after();
-            {
-                float t = 0.0f;
-#pragma unroll 1
-                for (int ch = 0; ch < 2; ++ch) {
-                    float x[32];
-                    tmem_ld32(lb + TM3 + ch * 32, x);
+            dG -= colpart[r] + colpart[128 + r] + colpart[256 + r] + colpart[384 + r];
+            dG = fmaf(Er, dE, dG);
+            float sd = 0.0f, sgc = 0.0f;
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        float k8[8];
-                        tile_h8(sm + SLOT, r, (cb + ch * 32) / 8 + k, k8);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            t = fmaf(x[8 * k + e], k8[e], t);
-                            x[8 * k + e] *= fr;
-                        }
-                    }
-                    tmem_st32(lb + TM3 + ch * 32, x);
-                    tmem_ld32(lb + TM1 + ch * 32, x);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) x[e] = -x[e];
-                    put_h32(t5, r, cb + ch * 32, x);
-                }
-                float rs = 0.0f;
-#pragma unroll 1
-                for (int ch = 0; ch < 2; ++ch) {
-                    const int col = cb + ch * 32;
-                    float x[32], v[32];
-                    tmem_ld32(lb + TM0 + ch * 32, x);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int j = col + e;
-                        const float dpp = x[e] * hsel(pa, ch, e);
-                        v[e] = dpp;
-                        rs += dpp;
-                        x[e] = (j <= r) ? x[e] * __expf(Gr - sG[j]) : 0.0f;
-                    }
-                    put_h32(t3, r, col, x);
-                    const float cs = colsum32(v, lane);
-                    colpart[q * 128 + col + lane] = cs;
-                }
-                t *= fr;
-                dG += rs - t;
-                sdgc += t;
+            for (int k = 0; k < 16; ++k) {
+                sd += wsum[2 * k];
+                sgc += wsum[2 * k + 1];
             }
-            pf_h64(p.V + gel, pa);  // the V row EC reads
-            tmem_st_wait();
-            fence_proxy_async();
-            arrive(CONS_B);
-
-            // ---- EC: dQ out;  dKb -> s3, TM3 += diag(beta E) dKb, rowsum(dKb o K);  dVb -> s4,
-            //      dv^ = beta dVb out, rowsum(dVb o V)
-            if (!group_all(1, 256, warp_wait_all(&bars[MMA_C], ph, ab, p.status, lim))) break;
-            tc_fence_after();
-            {
-                float tk = 0.0f, tv = 0.0f;
-#pragma unroll 1
-                for (int ch = 0; ch < 2; ++ch) {
-                    const int col = cb + ch * 32;
-                    float x[32], u[32];
-                    tmem_ld32(lb + TM2 + ch * 32, x);
-                    st_f32(p.dqh + gel + ch * 32, x, 1.0f);
-                    tmem_ld32(lb + TM0 + ch * 32, x);
+            const float dgC = fmaf(eC, sd, sgc);
+            // d log alpha_r = sum_{s >= r} dG_s (+ dG_last's share on every token)
+            float sc = dG;
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        float k8[8];
-                        tile_h8(sm + SLOT, r, col / 8 + k, k8);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) tk = fmaf(x[8 * k + e], k8[e], tk);
-                    }
-                    tmem_ld32(lb + TM3 + ch * 32, u);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) u[e] = fmaf(be * Er, x[e], u[e]);
-                    tmem_st32(lb + TM3 + ch * 32, u);
-                    put_h32(t3, r, col, x);
-                    tmem_ld32(lb + TM1 + ch * 32, x);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) tv = fmaf(x[e], hsel(pa, ch, e), tv);
-                    st_f32(p.dvh + gel + ch * 32, x, be);
-                    put_h32(t4, r, col, x);
-                }
-                dbeta = fmaf(Er, tk, dbeta) + tv;
-                dE = fmaf(be, tk, dE);
+            for (int off = 1; off < 32; off <<= 1) {
+                const float nb = __shfl_down_sync(0xffffffffu, sc, off);
+                if (lane + off < 32) sc += nb;
             }
-            tmem_st_wait();
-            fence_proxy_async();
-            arrive(CONS_C);
-
-            // ---- ED: dL = -(dKb W^T + dVb U^T) below the diagonal, A = K K^T: dA = beta dL o Gam -> s5,
-            //      rowsum(dL o Gam o A) into dbeta, rowsum / colsum of dLL = beta dL o Gam o A
-            if (!group_all(1, 256, warp_wait_all(&bars[MMA_D], ph, ab, p.status, lim))) break;
-            tc_fence_after();
-            {
-                float rs = 0.0f, db = 0.0f;
-#pragma unroll 1
-                for (int ch = 0; ch < 2; ++ch) {
-                    const int col = cb + ch * 32;
-                    float mv[32], a[32], v[32];
-                    tmem_ld32(lb + TM0 + ch * 32, mv);
-                    tmem_ld32(lb + TM1 + ch * 32, a);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int j = col + e;
-                        if (j < r) {
-                            const float gs = __expf(Gr - sG[j]);
-                            const float dl = -mv[e];
-                            const float dlga = dl * gs * a[e];
-                            db += dlga;
-                            v[e] = be * dlga;
-                            rs += v[e];
-                            mv[e] = be * dl * gs;
-                        } else {
-                            v[e] = 0.0f;
-                            mv[e] = 0.0f;
-                        }
-                    }
-                    put_h32(t5, r, col, mv);
-                    const float cs = colsum32(v, lane);
-                    colpart[q * 128 + col + lane] += cs;
-                }
-                dbeta += db;
-                dG += rs;
-            }
-            fence_proxy_async();
-            arrive(CONS_D);
-
-            // ---- EE: dk^ out; the row sums of both column halves, the column sums, d log alpha
-            if (!group_all(1, 256, warp_wait_all(&bars[MMA_E], ph, ab, p.status, lim))) break;
-            tc_fence_after();
-#pragma unroll 1
-            for (int ch = 0; ch < 2; ++ch) {
-                float x[32];
-                tmem_ld32(lb + TM3 + ch * 32, x);
-                st_f32(p.dkh + gel + ch * 32, x, 1.0f);
-            }
-            arrive(CONS_E);
-            if (hf == 1) {
-                xch[r] = dG;
-                xch[128 + r] = dbeta;
-                xch[256 + r] = dE;
-            }
-            sdot = warp_sum(sdot);
-            sdgc = warp_sum(sdgc);
-            if (lane == 0) {
-                wsum[2 * warp] = sdot;
-                wsum[2 * warp + 1] = sdgc;
-            }
-            named_sync(2, 256);
-            if (hf == 0) {
-                dG += xch[r];
-                dbeta += xch[128 + r];
-                dE += xch[256 + r];
-                dG -= colpart[r] + colpart[128 + r] + colpart[256 + r] + colpart[384 + r];
-                dG = fmaf(Er, dE, dG);
-                float sd = 0.0f, sg = 0.0f;
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    sd += wsum[2 * k];
-                    sg += wsum[2 * k + 1];
-                }
-                const float dgC = fmaf(eC, sd, sg);
-                // d log alpha_r = sum_{s >= r} dG_s (+ dG_last's share on every token)
-                float s = dG;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float nb = __shfl_down_sync(0xffffffffu, s, off);
-                    if (lane + off < 32) s += nb;
-                }
-                if (lane == 0) wsum[16 + q] = s;
-                named_sync(3, 128);
-                for (int q2 = q + 1; q2 < 4; ++q2) s += wsum[16 + q2];
-                p.dla[grow] = s + dgC;
-                p.dbeta[grow] = dbeta;
-            }
+            if (lane == 0) wsum[32 + q] = sc;
+            named_sync(3, 128);
+            for (int q2 = q + 1; q2 < 4; ++q2) sc += wsum[32 + q2];
+            p.dla[grow] = sc + dgC;
+            p.dbeta[grow] = dbeta;
         }
+    }
+    if (issuer) {
+        // loads and products still in flight (after an abort) complete before shared memory and TMEM go
+        // away; immediate when everything has completed
+#pragma unroll
+        for (int kb = 0; kb < NBAR; ++kb)
+            if (started[kb] > 0) mbar_wait_drain(&bars[kb], (started[kb] - 1) & 1, lim);
     }
     tc_fence_before();
     __syncthreads();
