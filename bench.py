@@ -657,7 +657,9 @@ def main():
             gr[n] = torch.empty((w.H * w.d, 4), **f32)
         gp = {n: gr[n].data_ptr() for n in gdn.GRAD_NAMES}
         n_b = 3
+        torch.cuda.nvtx.range_push("gdn_backward")  # the first call, for a profiler's launch list (--nvtx)
         plan.backward_raw(ptrs, dy.data_ptr(), gp, ws_b.data_ptr(), s)
+        torch.cuda.nvtx.range_pop()
         ev_b = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_b)]
         torch.cuda.synchronize()
         for k in range(n_b):

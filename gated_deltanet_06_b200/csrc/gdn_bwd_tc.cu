@@ -67,6 +67,32 @@ __device__ __forceinline__ void tile_h8(const uint8_t *tile, int r, int c16, flo
         f[2 * e + 1] = x.y;
     }
 }
+// A warp's 32 x 32 block (lane = row, v = its 32 columns) transposed in registers: afterwards lane l
+// holds column l (v[k] = row k).  Five exchange stages; at stage m a lane trades the elements whose
+// index differs from its own lane index in bit m with lane ^ m.
+__device__ __forceinline__ void transpose32(float (&v)[32], int lane) {
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) {
+        const bool b = (lane & m) != 0;
+#pragma unroll
+        for (int j0 = 0; j0 < 32; ++j0) {
+            if (j0 & m) continue;
+            const int j1 = j0 | m;
+            const float send = b ? v[j0] : v[j1];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, m);
+            if (b) v[j0] = recv;
+            else v[j1] = recv;
+        }
+    }
+}
+// A warp's 32 rows x 32 columns of fp32 output (lane = row) to rows row0 .. row0+31 of a [.][128]
+// array, columns c0 .. c0+31: transposed first, so that each store writes one row's 128 bytes.
+__device__ __forceinline__ void store_rows32(float *dst, size_t row0, int c0, float (&v)[32], int lane) {
+    transpose32(v, lane);
+#pragma unroll
+    for (int k = 0; k < 32; ++k) dst[(row0 + k) * 128 + c0 + lane] = v[k];
+}
+
 // 32 fp32 values to global memory (16-byte aligned)
 __device__ __forceinline__ void st_f32(float *dst, const float (&v)[32], float s) {
 #pragma unroll
@@ -608,7 +634,7 @@ __global__ void __launch_bounds__(bg::kThreads, 1)
             float x[32], u[32];
             float tk = 0.0f, tv = 0.0f;
             tmem_ld32(lb + TM2, x);
-            st_f32(p.dqh + gel, x, 1.0f);
+            store_rows32(p.dqh, row0 + q * 32, cb, x, lane);
             tmem_ld32(lb + TM0, x);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -625,8 +651,10 @@ __global__ void __launch_bounds__(bg::kThreads, 1)
             tmem_ld32(lb + TM1, x);
 #pragma unroll
             for (int e = 0; e < 32; ++e) tv = fmaf(x[e], hget(pa, e), tv);
-            st_f32(p.dvh + gel, x, be);
             put_h32(t4, r, cb, x);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] *= be;
+            store_rows32(p.dvh, row0 + q * 32, cb, x, lane);
             dbeta = fmaf(Er, tk, dbeta) + tv;
             dE = fmaf(be, tk, dE);
         }
@@ -701,7 +729,7 @@ __global__ void __launch_bounds__(bg::kThreads, 1)
         {
             float x[32];
             tmem_ld32(lb + TM3, x);
-            st_f32(p.dkh + gel, x, 1.0f);
+            store_rows32(p.dkh, row0 + q * 32, cb, x, lane);
         }
         if (cq > 0) {
             xch[(0 * 4 + cq) * 128 + r] = dG;
