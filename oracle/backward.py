@@ -184,3 +184,17 @@ def vjp(inp: dict, dy, l2_eps=DEFAULT_L2_EPS, norm_eps=DEFAULT_NORM_EPS) -> dict
         grads[n] = dx
         grads["conv_" + n] = dw.reshape(-1, 4)
     return grads
+
+
+def sum_magnitudes(inp: dict, dy, l2_eps=DEFAULT_L2_EPS, norm_eps=DEFAULT_NORM_EPS) -> dict:
+    """For the parameter gradients that are sums over tokens, the sum of their terms' magnitudes:
+    A_log and dt_bias [H] (terms d log alpha * log alpha and dL/dg, summed over b, t), norm_w [d_v]
+    (terms dy * o * rn * SiLU(z), summed over b, t, h).  A sum whose terms carry a relative error e
+    is off by at most e times this, so it sets the scale of a parity bound on such a gradient."""
+    g = vjp(inp, dy, l2_eps, norm_eps)
+    _, tp = _tape(inp, l2_eps, norm_eps)
+    dy = np.asarray(dy, dtype=np.float64)
+    dla = g["dalpha"] * tp["alpha"]
+    return {"A_log": np.abs(dla * tp["la"]).sum(axis=(0, 1)),
+            "dt_bias": np.abs(g["g"]).sum(axis=(0, 1)),
+            "norm_w": np.abs(dy * tp["o"] * tp["rn"] * tp["sz"]).sum(axis=(0, 1, 2))}

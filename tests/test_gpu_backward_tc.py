@@ -7,8 +7,15 @@ max |g_ref|, the bf16 parity bar of the forward applied to each gradient (its
 elementwise bound scaled by the tensor's largest entry, since the gradients'
 magnitudes differ from tensor to tensor).  The path rounds every tensor-core
 operand to fp16, as the forward does; the CPU model of that rounding (the
-block algebra with every operand rounded to fp16) gives about 7e-4, so the bar
-leaves a factor of about 3.
+block algebra with every operand rounded to fp16) gives about 7e-4 on the
+per-token gradients, so the bar leaves a factor of about 3.
+
+dA_log, ddt_bias and dnorm_w are sums over every token of terms of both
+signs.  A sum whose terms are each within a relative e is within e times the
+sum of the terms' magnitudes, so their bound is 2e-3 * ||sum |terms| ||_2
+(oracle.backward.sum_magnitudes) in place of 2e-3 * ||g_ref||_2, and their
+elementwise bound scales the same way.  With cancellation, ||g_ref|| can be
+much smaller than the magnitudes.
 
 The workspace stage test compares the kernels' intermediates (the state S at
 every block start, the state gradient dS at every block end, dq^, dk^, dv^,
@@ -54,11 +61,15 @@ def _run(inp, dy, out_f32=False, flags=0, keep=False):
     return got
 
 
-def _check_all(got, ref, what):
+def _check_all(got, ref, what, mags=None):
+    # mags: oracle.backward.sum_magnitudes of the case (the scale of the sums over tokens)
     errs = {}
     for n, rn in KEY.items():
-        e = rel_l2(got[n], ref[rn])
-        m = float(np.abs(got[n] - ref[rn]).max() / max(np.abs(ref[rn]).max(), 1e-300))
+        scale = ref[rn]
+        if mags is not None and rn in mags:
+            scale = mags[rn]
+        e = float(np.linalg.norm((got[n] - ref[rn]).ravel()) / max(np.linalg.norm(np.ravel(scale)), 1e-300))
+        m = float(np.abs(got[n] - ref[rn]).max() / max(np.abs(scale).max(), 1e-300))
         errs[n] = (e, m)
     bad = {n: v for n, v in errs.items() if not (v[0] <= REL_L2 and v[1] <= MAX_REL)}
     assert not bad, f"{what}: {bad} (all: {errs})"
@@ -76,7 +87,7 @@ def test_tensor_core_backward_matches_the_oracle(B, T, H, g_mean, out_f32):
     rng = np.random.default_rng(T)
     inp["norm_w"] = (1.0 + 0.3 * rng.standard_normal(128)).astype(np.float32)
     dy = _dy((B, T, H, 128), 800 + T)
-    _check_all(_run(inp, dy, out_f32=out_f32), ob.vjp(inp, dy), f"B={B} T={T} H={H}")
+    _check_all(_run(inp, dy, out_f32=out_f32), ob.vjp(inp, dy), f"B={B} T={T} H={H}", ob.sum_magnitudes(inp, dy))
 
 
 def test_tensor_core_backward_with_segments_of_several_blocks():
@@ -90,7 +101,7 @@ def test_tensor_core_backward_with_segments_of_several_blocks():
     got = _run(inp, dy)
     if plan.segments * 2 > -(-T // 128):
         pytest.skip(f"{plan.segments} segments on this GPU: segments hold one block each")
-    _check_all(got, ob.vjp(inp, dy), "T=1700 H=12")
+    _check_all(got, ob.vjp(inp, dy), "T=1700 H=12", ob.sum_magnitudes(inp, dy))
 
 
 def test_stages_match_the_block_model():

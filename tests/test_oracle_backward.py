@@ -110,3 +110,20 @@ def test_kernel_form_backward_equals_the_oracle_backward(T, C):
     for n, m in (("dq", "dqh"), ("dk", "dkh"), ("dv", "dvh"), ("dbeta", "dbeta")):
         np.testing.assert_allclose(got[n], ref[m], rtol=1e-9, atol=1e-11, err_msg=n)
     np.testing.assert_allclose(got["dla"], ref["dalpha"] * tp["alpha"], rtol=1e-9, atol=1e-11, err_msg="dla")
+
+
+def test_sum_magnitudes_bound_the_parameter_gradients():
+    # the scale used for the parity bound of the sums over tokens: at least the sum's own magnitude
+    # (triangle inequality); and equal to it when every term has one sign, as norm_w's terms do in
+    # the second case (every input and dy positive, z > 1)
+    inp, dy = _case(140, T=30, H=2, d=8)
+    ref = ob.vjp(inp, dy)
+    mags = ob.sum_magnitudes(inp, dy)
+    for k in ("A_log", "dt_bias", "norm_w"):
+        assert np.all(mags[k] >= np.abs(ref[k]) * (1 - 1e-12)), k
+    one_sign = {n: np.abs(v) if isinstance(v, np.ndarray) else v for n, v in inp.items()}
+    dy_pos = np.abs(dy)
+    one_sign["z"] = np.abs(inp["z"]) + 1.0
+    ref1 = ob.vjp(one_sign, dy_pos)
+    mags1 = ob.sum_magnitudes(one_sign, dy_pos)
+    np.testing.assert_allclose(mags1["norm_w"], np.abs(ref1["norm_w"]), rtol=1e-9)
