@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(256) gdn_bwd_out(const BwdParams p) {
 // (b, t, h) row, lane l on columns 4l .. 4l+3 with 8- and 16-byte loads and stores, two rows per
 // warp step (both rows' loads in flight before either is used), SiLU's sigmoid once per element.
 template <typename ZT, typename YT>
-__global__ void __launch_bounds__(256) gdn_bwd_out_rows(const BwdParams p) {
+__global__ void __launch_bounds__(256, 4) gdn_bwd_out_rows(const BwdParams p) {
     constexpr int D = 128;
     __shared__ float sw[8][D];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, c0 = lane * 4;
@@ -657,12 +657,8 @@ __global__ void __launch_bounds__(256) gdn_bwd_tokens_rows(const BwdParams p) {
         };
         if (warp < 4) swt[warp][lane] = reinterpret_cast<const float4 *>(wc)[static_cast<size_t>(h) * D + c0 + warp];
         __syncthreads();
-        float w[4][4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float4 t4 = swt[j][lane];
-            w[j][0] = t4.x; w[j][1] = t4.y; w[j][2] = t4.z; w[j][3] = t4.w;
-        }
+        // conv taps read from shared memory at each use
+        auto wt = [&](int j) { return swt[j][lane]; };
         // pass 1: da of tokens t0 .. t0 + 66 (zero past T), in runs of two consecutive tokens taken by the
         // warps in turn: a run's 5 input rows and 2 gradient rows are fetched before any is used, and
         // the two tokens' reductions are independent
@@ -687,7 +683,8 @@ __global__ void __launch_bounds__(256) gdn_bwd_tokens_rows(const BwdParams p) {
                 pr[i] = 0.0f;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    a[i][j] = w[j][0] * xr[i][j] + w[j][1] * xr[i + 1][j] + w[j][2] * xr[i + 2][j] + w[j][3] * xr[i + 3][j];
+                    const float4 w4 = wt(j);
+                    a[i][j] = w4.x * xr[i][j] + w4.y * xr[i + 1][j] + w4.z * xr[i + 2][j] + w4.w * xr[i + 3][j];
                     sg[i][j] = __fdividef(1.0f, 1.0f + __expf(-a[i][j]));
                     sv[i][j] = a[i][j] * sg[i][j];
                     ss[i] = fmaf(sv[i][j], sv[i][j], ss[i]);
@@ -743,7 +740,8 @@ __global__ void __launch_bounds__(256) gdn_bwd_tokens_rows(const BwdParams p) {
             float o[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                o[j] = w[j][0] * dr[3][j] + w[j][1] * dr[2][j] + w[j][2] * dr[1][j] + w[j][3] * dr[0][j];
+                const float4 w4 = wt(j);
+                o[j] = w4.x * dr[3][j] + w4.y * dr[2][j] + w4.z * dr[1][j] + w4.w * dr[0][j];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) dw[j][k] = fmaf(dr[0][j], xr[k][j], dw[j][k]);
             }
