@@ -162,3 +162,25 @@ def test_tensor_core_backward_at_the_headline_size():
     simt = _run(inp, dy1, out_f32=True, flags=gdn.FLAG_FORCE_SIMT)
     for n in KEY:
         assert rel_l2(g1[n], simt[n]) <= REL_L2, (n, rel_l2(g1[n], simt[n]))
+
+
+def test_tensor_core_backward_with_f16_inputs_and_output():
+    # fp16 activations and an fp16 dy (the draws rounded to fp16, and the oracle given the same
+    # values): the same path with the 16-bit loads of the other type
+    import torch
+    import gated_deltanet_06_b200 as gdn
+    B, T, H = 1, 200, 2
+    inp = gdn_inputs.make_inputs(B, T, H, 128, "bf16", -0.5, seed=761)
+    t = torch_inputs(inp)
+    for n in ("q", "k", "v", "z"):
+        inp[n] = inp[n].astype(np.float16).astype(np.float32)
+        t[n] = torch.from_numpy(inp[n]).to("cuda", torch.float16)
+    dy = _dy((B, T, H, 128), 862).astype(np.float16).astype(np.float32)
+    plan = gdn.Plan(B, T, H, 128, gdn.DTYPE_F16, gdn.DTYPE_F16)
+    assert plan.uses_tensor_path and plan.backward_launches in (8, 12)
+    ws = torch.empty(plan.backward_workspace_bytes, dtype=torch.uint8, device="cuda")
+    out = gdn.backward(**t, dy=torch.from_numpy(dy).to("cuda", torch.float16), plan=plan, workspace=ws)
+    torch.cuda.synchronize()
+    assert plan.device_status(ws.data_ptr(), torch.cuda.current_stream().cuda_stream) == gdn.OK
+    got = {n: v.double().cpu().numpy() for n, v in out.items()}
+    _check_all(got, ob.vjp(inp, dy), "f16 T=200", ob.sum_magnitudes(inp, dy))
