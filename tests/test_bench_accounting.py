@@ -148,3 +148,15 @@ def test_recorded_traffic_covers_every_forward_kernel():
         pytest.skip("a kernel changed since its capture")
     assert sum(kt) > bench.path_bytes_per_token_head(128, 2, 2) * w.B * w.T * w.H
     assert kt[names.index("chunk")] <= bench.kernel_work_per_token_head("chunk", 128, 2, 2)[0] * w.B * w.T * w.H
+
+
+def test_backward_launch_names_and_block_gradient_flops():
+    # the tensor-core backward's launches (with and without the segment passes) and the fp32 one's
+    assert len(bench.backward_kernel_names(12)) == 12 and len(bench.backward_kernel_names(8)) == 8
+    assert bench.backward_kernel_names(12)[9] == "bwd_grad" and bench.backward_kernel_names(8)[5] == "bwd_grad"
+    assert bench.backward_kernel_names(6) == ("prep_f32", "fwd_rows", "out_bwd", "core_bwd", "tokens_bwd", "params")
+    with pytest.raises(ValueError):
+        bench.backward_kernel_names(7)
+    # 16 products of 128 x 128 x 128 per 128-token block: at the headline (12 heads, 256 blocks each)
+    assert bench.backward_grad_flops(1, 1) == 16 * 2 * 128 ** 3
+    assert bench.backward_grad_flops(12, 256) == 12 * 256 * 16 * 2 * 128 ** 3
